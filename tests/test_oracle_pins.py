@@ -1,0 +1,234 @@
+"""The fp64 oracle pinned to things other than itself (CPU only).
+
+Pins: scalar brute force, the library SDPA routine, autograd, central finite
+differences, closed forms and the invariants the pages state.
+"""
+
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+from oracle import MaskDesc
+from tests import oracle_pins as P
+
+SCALE = 0.37
+
+
+@pytest.mark.parametrize("case", list(P.tiny_masks(2, 9, 11).keys()))
+def test_forward_matches_brute_force(case):
+    q, k, v, _ = P.tiny_inputs(1, B=2)
+    mask = P.tiny_masks(2, 9, 11)[case]
+    O, L = oracle.attention_forward(q, k, v, mask, SCALE)
+    allowed = P.dense_allowed(mask, 2, 9, 11)
+    Ob, Lb = P.brute_force_forward(q, k, v, allowed, SCALE)
+    assert np.max(np.abs(O - Ob)) < 1e-12
+    fin = np.isfinite(Lb)
+    assert np.array_equal(fin, np.isfinite(L))
+    assert np.max(np.abs(L[fin] - Lb[fin])) < 1e-12
+
+
+@pytest.mark.parametrize("case", ["none", "causal", "window3", "padding", "segments", "seg+window"])
+def test_forward_matches_library_sdpa(case):
+    q, k, v, _ = P.tiny_inputs(2, B=2, Sq=12, Skv=12, D=6)
+    mask = P.tiny_masks(2, 12, 12, seed=3)[case]
+    allowed = P.dense_allowed(mask, 2, 12, 12)
+    if not all(a.any(axis=1).all() for a in allowed):
+        pytest.skip("SDPA is undefined on rows without keys")
+    O, _ = oracle.attention_forward(q, k, v, mask, SCALE)
+    Os = P.sdpa_forward(q, k, v, allowed, SCALE)
+    assert np.max(np.abs(O - Os)) < 1e-12
+
+
+@pytest.mark.parametrize("case", ["none", "causal", "window3", "padding", "segments"])
+def test_backward_matches_autograd(case):
+    q, k, v, dO = P.tiny_inputs(4, B=2, Sq=10, Skv=10, D=4)
+    v = v[..., :4].copy()
+    dO = dO[..., :4].copy()
+    mask = P.tiny_masks(2, 10, 10, seed=5)[case]
+    allowed = P.dense_allowed(mask, 2, 10, 10)
+    if not all(a.any(axis=1).all() for a in allowed):
+        pytest.skip("SDPA is undefined on rows without keys")
+    dq, dk, dv = oracle.attention_backward(q, k, v, dO, mask, SCALE)
+    aq, ak, av = P.autograd_backward(q, k, v, dO, allowed, SCALE)
+    for x, y in ((dq, aq), (dk, ak), (dv, av)):
+        assert np.max(np.abs(x - y)) < 1e-11
+
+
+def test_backward_matches_finite_differences_with_empty_rows():
+    # A window on Sq > Skv leaves the first rows without keys: gradients through
+    # them are zero and the rest must still match central differences.
+    q, k, v, dO = P.tiny_inputs(6, B=1, Sq=8, Skv=6, D=3)
+    mask = MaskDesc(window=2)
+    fwd = lambda a, b_, c: oracle.attention_forward(a, b_, c, mask, SCALE)[0]
+    dq, dk, dv = oracle.attention_backward(q, k, v, dO, mask, SCALE)
+    rng = np.random.default_rng(0)
+    for which, grad, shp in ((0, dq, q.shape), (1, dk, k.shape), (2, dv, v.shape)):
+        idx = [tuple(int(rng.integers(0, s)) for s in shp) for _ in range(12)]
+        fd = P.finite_difference_grad(fwd, q, k, v, dO, which, idx)
+        an = np.array([grad[i] for i in idx])
+        assert np.max(np.abs(fd - an)) < 1e-7
+    O, L = oracle.attention_forward(q, k, v, mask, SCALE)
+    assert np.all(O[0, :2] == 0) and np.all(np.isneginf(L[0, :, :2]))
+    assert np.all(dq[0, :2] == 0)
+
+
+# ---------------------------------------------------------------- closed forms
+
+def test_closed_form_equal_keys_give_mean_of_values():
+    rng = np.random.default_rng(7)
+    q = rng.standard_normal((1, 5, 1, 4))
+    k = np.repeat(rng.standard_normal((1, 1, 1, 4)), 9, axis=1)
+    v = rng.standard_normal((1, 9, 1, 3))
+    mask = MaskDesc(kv_valid_len=np.array([6]))
+    O, L = oracle.attention_forward(q, k, v, mask, SCALE)
+    assert np.allclose(O[0, :, 0], v[0, :6, 0].mean(axis=0), atol=1e-13)
+    s = SCALE * (q[0, :, 0] @ k[0, 0, 0])
+    assert np.allclose(L[0, 0], s + math.log(6), atol=1e-13)
+
+
+def test_closed_form_single_key():
+    rng = np.random.default_rng(8)
+    q, k, v = (rng.standard_normal((1, 6, 1, 4)) for _ in range(3))
+    # window=1: each row sees exactly its own (diagonal) key
+    O, L = oracle.attention_forward(q, k, v, MaskDesc(window=1), SCALE)
+    assert np.allclose(O[0, :, 0], v[0, :, 0], atol=1e-14)
+    assert np.allclose(L[0, 0], SCALE * (q[0, :, 0] * k[0, :, 0]).sum(1), atol=1e-14)
+
+
+def test_closed_form_zero_query_is_uniform():
+    rng = np.random.default_rng(9)
+    q = np.zeros((1, 4, 1, 4))
+    k, v = (rng.standard_normal((1, 7, 1, 4)) for _ in range(2))
+    O, L = oracle.attention_forward(q, k, v, MaskDesc(), SCALE)
+    assert np.allclose(O[0, :, 0], v[0, :, 0].mean(axis=0), atol=1e-14)
+    assert np.allclose(L, math.log(7), atol=1e-14)
+
+
+def test_wide_window_is_plain_causal():
+    q, k, v, _ = P.tiny_inputs(10, Sq=7, Skv=9, D=3)
+    a, la = oracle.attention_forward(q, k, v, MaskDesc(window=50), SCALE)
+    b, lb = oracle.attention_forward(q, k, v, MaskDesc(window=0), SCALE)
+    assert np.array_equal(a, b) and np.array_equal(la, lb)
+
+
+def test_mask_predicates_count_keys():
+    Sq, Skv, W = 40, 56, 7
+    o = Skv - Sq
+    a = oracle.allowed_rows(MaskDesc(window=W), 0, np.arange(Sq), Sq, Skv)
+    for i in range(Sq):
+        lo, hi = max(0, i + o - W + 1), min(Skv - 1, i + o)
+        assert a[i].sum() == max(0, hi - lo + 1)
+        assert a[i, hi] and (lo == 0 or not a[i, lo - 1])
+    assert a[Sq - 1, Skv - 1]  # bottom-right alignment
+    cu = np.array([0, 10, 25, 31, 40])
+    a = oracle.allowed_rows(MaskDesc(cu_seqlens=cu, n_align_tail=1), 0, np.arange(40), 40, 40)
+    for s in range(3):
+        for i in range(cu[s], cu[s + 1]):
+            assert a[i].sum() == cu[s + 1] - cu[s] and a[i, cu[s]:cu[s + 1]].all()
+    assert not a[31:].any() and not a[:, 31:].any()
+    a = oracle.allowed_rows(MaskDesc(kv_valid_len=np.array([5, 9])), 1, np.arange(4), 4, 12)
+    assert (a.sum(axis=1) == 9).all()
+
+
+# ---------------------------------------------------------------- invariants
+
+def test_constant_segment_ids_equal_no_mask():
+    q, k, v, dO = P.tiny_inputs(11, B=2, Sq=12, Skv=12, D=4)
+    v, dO = v[..., :4].copy(), dO[..., :4].copy()
+    seg = np.full((2, 12), 3)
+    m = MaskDesc(seg_q=seg, seg_kv=seg)
+    a = oracle.attention_forward(q, k, v, m, SCALE)
+    b = oracle.attention_forward(q, k, v, MaskDesc(), SCALE)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+    ga = oracle.attention_backward(q, k, v, dO, m, SCALE)
+    gb = oracle.attention_backward(q, k, v, dO, MaskDesc(), SCALE)
+    for x, y in zip(ga, gb):
+        assert np.array_equal(x, y)
+
+
+def test_alignment_rows_never_reach_real_rows():
+    rng = np.random.default_rng(12)
+    cu = np.array([0, 13, 21, 24])
+    m = MaskDesc(cu_seqlens=cu, n_align_tail=1)
+    q, k, v = (rng.standard_normal((1, 24, 2, 4)) for _ in range(3))
+    O, L = oracle.attention_forward(q, k, v, m, SCALE)
+    q2, k2, v2 = q.copy(), k.copy(), v.copy()
+    for t in (q2, k2, v2):
+        t[:, 21:] = rng.standard_normal(t[:, 21:].shape) * 50
+    O2, L2 = oracle.attention_forward(q2, k2, v2, m, SCALE)
+    assert np.array_equal(O[:, :21], O2[:, :21]) and np.array_equal(L[..., :21], L2[..., :21])
+    assert np.all(O[:, 21:] == 0) and np.all(np.isneginf(L[..., 21:]))
+
+
+def test_padding_contents_do_not_matter():
+    rng = np.random.default_rng(13)
+    m = MaskDesc(kv_valid_len=np.array([10]))
+    q = rng.standard_normal((1, 8, 1, 4))
+    k, v = (rng.standard_normal((1, 16, 1, 4)) for _ in range(2))
+    O, L = oracle.attention_forward(q, k, v, m, SCALE)
+    k2, v2 = k.copy(), v.copy()
+    k2[:, 10:] *= 100
+    v2[:, 10:] = 1e6  # finite: 0 * NaN would be NaN in any product
+    O2, L2 = oracle.attention_forward(q, k2, v2, m, SCALE)
+    assert np.array_equal(O, O2) and np.array_equal(L, L2)
+
+
+def test_fixed_m_equals_online():
+    q, k, v, _ = P.tiny_inputs(14, B=2, Sq=20, Skv=24, D=6)
+    for name, m in P.tiny_masks(2, 20, 24, seed=2).items():
+        a = oracle.attention_forward(q, k, v, m, SCALE)
+        b = oracle.attention_forward_fixed_m(q, k, v, m, SCALE)
+        assert np.max(np.abs(a[0] - b[0])) < 1e-12, name
+        fin = np.isfinite(a[1])
+        assert np.array_equal(fin, np.isfinite(b[1]))
+        assert np.max(np.abs(a[1][fin] - b[1][fin])) < 1e-12, name
+
+
+def test_fixed_m_bound_dominates_every_score_and_gate_separates_sink():
+    rng = np.random.default_rng(15)
+    D, S = 16, 64
+    q = rng.standard_normal((1, S, 2, D)) * math.sqrt(0.5)
+    k = rng.standard_normal((1, S + 8, 2, D)) * math.sqrt(0.5)
+    k[0, :4, 0] *= 20  # sink keys on head 0
+    k[0, S:] *= 100  # padding keys
+    m = MaskDesc(kv_valid_len=np.array([S]))
+    scale = 1 / math.sqrt(D)
+    kmax, qmax, bound, gate = oracle.fixed_m_bound(q, k, m, scale, gate_limit=64.0)
+    for h in range(2):
+        s = scale * q[0, :, h] @ k[0, :S, h].T
+        assert np.abs(s).max() <= bound[0, h] + 1e-12
+        assert kmax[0, h] == np.linalg.norm(k[0, :S, h], axis=1).max()
+    assert not gate[0, 0] and gate[0, 1]
+
+
+def test_gradient_identities():
+    q, k, v, dO = P.tiny_inputs(16, B=1, Sq=9, Skv=9, D=4)
+    v, dO = v[..., :4].copy(), dO[..., :4].copy()
+    m = MaskDesc(window=3)
+    dq, dk, dv = oracle.attention_backward(q, k, v, dO, m, SCALE)
+    # sum over keys of dV equals the sum of dO over rows that see any key
+    assert np.allclose(dv.sum(axis=1), dO.sum(axis=1), atol=1e-12)
+    # rows of dS sum to zero: with every key equal, dQ vanishes
+    k_eq = np.repeat(k[:, :1], 9, axis=1)
+    dq0, _, _ = oracle.attention_backward(q, k_eq, v, dO, m, SCALE)
+    assert np.max(np.abs(dq0)) < 1e-12
+
+
+def test_key_permutation_with_mask_leaves_output():
+    rng = np.random.default_rng(17)
+    q = rng.standard_normal((1, 6, 1, 4))
+    k, v = (rng.standard_normal((1, 10, 1, 4)) for _ in range(2))
+    seg_q = np.array([[0, 0, 1, 1, 2, 2]])
+    seg_kv = np.array([[0, 1, 2, 0, 1, 2, 0, 1, 2, 2]])
+    perm = rng.permutation(10)
+    a = oracle.attention_forward(q, k, v, MaskDesc(seg_q=seg_q, seg_kv=seg_kv), SCALE)
+    b = oracle.attention_forward(q, k[:, perm], v[:, perm],
+                                 MaskDesc(seg_q=seg_q, seg_kv=seg_kv[:, perm]), SCALE)
+    assert np.allclose(a[0], b[0], atol=1e-14) and np.allclose(a[1], b[1], atol=1e-14)
+
+
+def test_useful_flops_per_tile():
+    assert oracle.useful_flops(1, 128) == 4 * 128 * 128 * 128
+    assert oracle.useful_flops(2, 64, backward=True) == 2.5 * 2 * 4 * 128 * 128 * 64
