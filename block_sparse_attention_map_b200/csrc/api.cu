@@ -1,0 +1,400 @@
+// C ABI of libbsa (declared in include/bsa.h): argument validation, workspace
+// layout, TMA tensor maps and the sequence of launches for each call.  Every
+// argument error is returned before anything is launched; the library
+// allocates nothing and synchronises only in bsa_get_device_status.
+#include <atomic>
+#include <cmath>
+#include <cstring>
+#include <vector>
+
+#include "internal.h"
+
+namespace bsa {
+
+namespace {
+std::atomic<uint64_t> g_launches{0};
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+int64_t cdiv64(int64_t a, int64_t b) { return (a + b - 1) / b; }
+}  // namespace
+
+void count_launch(int n) { g_launches.fetch_add(static_cast<uint64_t>(n)); }
+
+WsLayout compute_layout(const bsa_problem &p) {
+  WsLayout L{};
+  const int64_t B = p.B, H = p.H;
+  L.nM = static_cast<int>(cdiv64(p.Sq, kTile));
+  L.nN = static_cast<int>(cdiv64(p.Skv, kTile));
+  const int64_t nM = L.nM, nN = L.nN;
+  L.nnz_cap = B * nM * nN;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + bytes, 256);
+    return o;
+  };
+  L.status = take(kHdrWords * 4);
+  L.tile_class = take(static_cast<size_t>(B * nM * nN));
+  L.rank = take(4 * static_cast<size_t>(B * nM * nN));
+  L.row_cnt = take(4 * static_cast<size_t>(B * nM));
+  L.row_ptr = take(4 * static_cast<size_t>(B * nM + 1));
+  L.row_ent = take(4 * static_cast<size_t>(L.nnz_cap));
+  L.col_cnt = take(4 * static_cast<size_t>(B * nN));
+  L.col_ptr = take(4 * static_cast<size_t>(B * nN + 1));
+  L.col_ent = take(4 * static_cast<size_t>(L.nnz_cap));
+  L.col_rank = take(4 * static_cast<size_t>(L.nnz_cap));
+  L.perm = take(4 * static_cast<size_t>(nN));
+  L.seg_q = take(4 * static_cast<size_t>(p.Sq));
+  L.seg_kv = take(4 * static_cast<size_t>(p.Skv));
+  L.qblk = take(16 * static_cast<size_t>(B * nM));
+  L.kblk = take(16 * static_cast<size_t>(B * nN));
+  L.kmax = take(8 * static_cast<size_t>(B * H));  // kmax then qmax, adjacent
+  L.qmax = L.kmax + 4 * static_cast<size_t>(B * H);
+  L.gate = take(4 * static_cast<size_t>(B * H));
+  L.qnorm = take(4 * static_cast<size_t>(B * H * p.Sq));
+  L.fwd_end = off;
+  L.delta = take(4 * static_cast<size_t>(B * H * nM * kTile));
+  L.dq_accum = take(4 * static_cast<size_t>(B * H * nM * kTile * p.D));
+  L.sem = take(4 * static_cast<size_t>(B * H * nM));
+  L.total = off;
+  return L;
+}
+
+namespace {
+
+// cuTensorMapEncodeTiled, fetched through the runtime so that the library
+// needs no link-time dependency on libcuda.
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// 4-D map over a bf16 [B, S, H, D] tensor: dims (D, S, H, B), 64 x 128 boxes,
+// 128-byte swizzle.  Out-of-range rows read as zero.
+bool make_map(CUtensorMap *map, const void *ptr, int B, int S, int H, int D,
+              const int64_t *stride) {
+  auto enc = get_encode();
+  if (enc == nullptr) return false;
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(S),
+                              static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(B)};
+  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(stride[1]) * 2,
+                                 static_cast<cuuint64_t>(stride[2]) * 2,
+                                 static_cast<cuuint64_t>(stride[0]) * 2};
+  const cuuint32_t box[4] = {64, static_cast<cuuint32_t>(kTile), 1, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(ptr), dims,
+                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Resolve defaults (contiguous strides, scale) into a private copy.
+bsa_status normalise(const bsa_problem *in, bsa_problem *out) {
+  if (in == nullptr) return BSA_ERR_INVALID_ARG;
+  *out = *in;
+  bsa_problem &p = *out;
+  if (p.B < 1 || p.H < 1 || p.Sq < 1 || p.Skv < 1) return BSA_ERR_INVALID_ARG;
+  if (p.D != 64 && p.D != 128) return BSA_ERR_UNSUPPORTED;
+  if (p.Sq > (1 << 21) || p.Skv > (1 << 21)) return BSA_ERR_UNSUPPORTED;
+  const int64_t nM = cdiv64(p.Sq, kTile), nN = cdiv64(p.Skv, kTile);
+  if (static_cast<int64_t>(p.B) * nM * nN >= (int64_t{1} << 30)) return BSA_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(p.B) * p.H * nM >= (int64_t{1} << 31)) return BSA_ERR_UNSUPPORTED;
+  auto fix = [&](int64_t *s, int64_t S) -> bsa_status {
+    if (s[0] == 0 && s[1] == 0 && s[2] == 0) {
+      s[0] = S * p.H * p.D;
+      s[1] = static_cast<int64_t>(p.H) * p.D;
+      s[2] = p.D;
+    }
+    for (int i = 0; i < 3; ++i) {
+      if (s[i] <= 0) return BSA_ERR_INVALID_ARG;
+      if (s[i] % 8 != 0) return BSA_ERR_UNSUPPORTED;  // 16-byte aligned rows for TMA
+    }
+    return BSA_OK;
+  };
+  bsa_status st;
+  if ((st = fix(p.q_stride, p.Sq)) != BSA_OK) return st;
+  if ((st = fix(p.k_stride, p.Skv)) != BSA_OK) return st;
+  if ((st = fix(p.v_stride, p.Skv)) != BSA_OK) return st;
+  if ((st = fix(p.o_stride, p.Sq)) != BSA_OK) return st;
+  if (!(p.scale > 0.f) || !std::isfinite(p.scale)) p.scale = 1.0f / std::sqrt(static_cast<float>(p.D));
+  return BSA_OK;
+}
+
+bsa_status check_mask(const bsa_problem &p, const bsa_mask_spec *m, bsa_mask_spec *out) {
+  std::memset(out, 0, sizeof(*out));
+  if (m == nullptr) return BSA_OK;
+  *out = *m;
+  const uint32_t known = BSA_MASK_SEGMENT_IDS | BSA_MASK_KV_VALID_LEN | BSA_MASK_VARLEN |
+                         BSA_MASK_CAUSAL_WINDOW;
+  if (m->flags & ~known) return BSA_ERR_INVALID_ARG;
+  if ((m->flags & BSA_MASK_SEGMENT_IDS) && (m->seg_q == nullptr || m->seg_kv == nullptr))
+    return BSA_ERR_INVALID_ARG;
+  if ((m->flags & BSA_MASK_KV_VALID_LEN) && m->kv_valid_len == nullptr) return BSA_ERR_INVALID_ARG;
+  if (m->flags & BSA_MASK_VARLEN) {
+    if (m->flags & BSA_MASK_SEGMENT_IDS) return BSA_ERR_INVALID_ARG;
+    if (m->cu_seqlens == nullptr || m->n_seqs < 1 || m->n_align_tail < 0 ||
+        m->n_align_tail > m->n_seqs || p.B != 1 || p.Sq != p.Skv)
+      return BSA_ERR_INVALID_ARG;
+  }
+  if ((m->flags & BSA_MASK_CAUSAL_WINDOW) && m->window < 0) return BSA_ERR_INVALID_ARG;
+  if (!(m->flags & BSA_MASK_CAUSAL_WINDOW)) out->window = 0;
+  if (!(m->flags & BSA_MASK_VARLEN)) {
+    out->n_seqs = 0;
+    out->n_align_tail = 0;
+  }
+  return BSA_OK;
+}
+
+bsa_status check_options(const bsa_options *o, int nN, bsa_options *out) {
+  std::memset(out, 0, sizeof(*out));
+  out->deterministic = 1;
+  if (o == nullptr) return BSA_OK;
+  *out = *o;
+  if (o->softmax_mode != BSA_SOFTMAX_ONLINE && o->softmax_mode != BSA_SOFTMAX_FIXED_M_GATED)
+    return BSA_ERR_INVALID_ARG;
+  if (o->bwd_order < BSA_ORDER_ASC || o->bwd_order > BSA_ORDER_PERM) return BSA_ERR_INVALID_ARG;
+  if (o->bwd_order == BSA_ORDER_PERM) {
+    if (o->perm == nullptr) return BSA_ERR_INVALID_ARG;
+    std::vector<char> seen(static_cast<size_t>(nN), 0);
+    for (int t = 0; t < nN; ++t) {
+      const int n = o->perm[t];
+      if (n < 0 || n >= nN || seen[static_cast<size_t>(n)]) return BSA_ERR_INVALID_ARG;
+      seen[static_cast<size_t>(n)] = 1;
+    }
+  }
+  return BSA_OK;
+}
+
+PlanSignature signature(const bsa_problem &p, const bsa_mask_spec &m, const bsa_options &o) {
+  PlanSignature s{};
+  s.w[0] = p.B;
+  s.w[1] = p.Sq;
+  s.w[2] = p.Skv;
+  s.w[3] = m.flags;
+  s.w[4] = m.window;
+  s.w[5] = o.bwd_order;
+  s.w[6] = m.n_seqs;
+  return s;
+}
+
+MaskParams mask_params(const bsa_problem &p, const bsa_mask_spec &m, const WsLayout &L,
+                       uint8_t *ws) {
+  MaskParams mp{};
+  mp.flags = m.flags;
+  mp.window = m.window;
+  mp.offset = p.Skv - p.Sq;
+  mp.Sq = p.Sq;
+  mp.Skv = p.Skv;
+  mp.kv_valid_len = (m.flags & BSA_MASK_KV_VALID_LEN) ? m.kv_valid_len : nullptr;
+  if (m.flags & BSA_MASK_SEGMENT_IDS) {
+    mp.seg_q = m.seg_q;
+    mp.seg_kv = m.seg_kv;
+  } else if (m.flags & BSA_MASK_VARLEN) {
+    mp.seg_q = reinterpret_cast<const int32_t *>(ws + L.seg_q);
+    mp.seg_kv = reinterpret_cast<const int32_t *>(ws + L.seg_kv);
+  }
+  return mp;
+}
+
+bool have_device() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  int major = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+    return false;
+  return major == 10;
+}
+
+struct Prepared {
+  bsa_problem p;
+  bsa_mask_spec m;
+  bsa_options o;
+  WsLayout L;
+};
+
+bsa_status prepare(const bsa_problem *prob, const bsa_mask_spec *mask, const bsa_options *opt,
+                   void *ws, size_t ws_bytes, bool backward, Prepared *out) {
+  bsa_status st = normalise(prob, &out->p);
+  if (st != BSA_OK) return st;
+  if ((st = check_mask(out->p, mask, &out->m)) != BSA_OK) return st;
+  out->L = compute_layout(out->p);
+  if ((st = check_options(opt, out->L.nN, &out->o)) != BSA_OK) return st;
+  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return BSA_ERR_INVALID_ARG;
+  if (ws_bytes < (backward ? out->L.total : out->L.fwd_end)) return BSA_ERR_WORKSPACE_TOO_SMALL;
+  if (!have_device()) return BSA_ERR_NO_DEVICE;
+  return BSA_OK;
+}
+
+bsa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? BSA_OK : BSA_ERR_CUDA; }
+
+}  // namespace
+}  // namespace bsa
+
+using namespace bsa;
+
+extern "C" {
+
+bsa_status bsa_workspace_size(const bsa_problem *prob, const bsa_mask_spec *mask,
+                              int32_t with_backward, size_t *bytes) {
+  if (bytes == nullptr) return BSA_ERR_INVALID_ARG;
+  bsa_problem p;
+  bsa_status st = normalise(prob, &p);
+  if (st != BSA_OK) return st;
+  bsa_mask_spec m;
+  if ((st = check_mask(p, mask, &m)) != BSA_OK) return st;
+  const WsLayout L = compute_layout(p);
+  *bytes = with_backward ? L.total : L.fwd_end;
+  return BSA_OK;
+}
+
+bsa_status bsa_workspace_layout(const bsa_problem *prob, const bsa_mask_spec *mask,
+                                bsa_workspace_view *view) {
+  if (view == nullptr) return BSA_ERR_INVALID_ARG;
+  bsa_problem p;
+  bsa_status st = normalise(prob, &p);
+  if (st != BSA_OK) return st;
+  bsa_mask_spec m;
+  if ((st = check_mask(p, mask, &m)) != BSA_OK) return st;
+  const WsLayout L = compute_layout(p);
+  view->total_bytes = L.total;
+  view->fwd_bytes = L.fwd_end;
+  view->off_status = L.status;
+  view->off_tile_class = L.tile_class;
+  view->off_rank = L.rank;
+  view->off_row_ptr = L.row_ptr;
+  view->off_row_ent = L.row_ent;
+  view->off_col_ptr = L.col_ptr;
+  view->off_col_ent = L.col_ent;
+  view->off_col_rank = L.col_rank;
+  view->off_perm = L.perm;
+  view->off_kmax = L.kmax;
+  view->off_qmax = L.qmax;
+  view->off_gate = L.gate;
+  view->off_delta = L.delta;
+  view->off_dq_accum = L.dq_accum;
+  view->off_sem = L.sem;
+  view->nM = L.nM;
+  view->nN = L.nN;
+  return BSA_OK;
+}
+
+bsa_status bsa_plan_build(const bsa_problem *prob, const bsa_mask_spec *mask,
+                          const bsa_options *opt, void *ws, size_t ws_bytes, bsa_stream_t stream) {
+  Prepared P;
+  bsa_status st = prepare(prob, mask, opt, ws, ws_bytes, false, &P);
+  if (st != BSA_OK) return st;
+  return cuda_status(launch_plan(P.p, P.m, P.o, P.L, static_cast<uint8_t *>(ws),
+                                 reinterpret_cast<cudaStream_t>(stream)));
+}
+
+bsa_status bsa_attn_fwd(const bsa_problem *prob, const bsa_mask_spec *mask,
+                        const bsa_options *opt, const void *q, const void *k, const void *v,
+                        void *out, float *lse, void *ws, size_t ws_bytes, bsa_stream_t stream) {
+  if (q == nullptr || k == nullptr || v == nullptr || out == nullptr || lse == nullptr)
+    return BSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return BSA_ERR_UNSUPPORTED;
+  Prepared P;
+  bsa_status st = prepare(prob, mask, opt, ws, ws_bytes, false, &P);
+  if (st != BSA_OK) return st;
+  const bsa_problem &p = P.p;
+  CUtensorMap tq, tk, tv;
+  if (!make_map(&tq, q, p.B, p.Sq, p.H, p.D, p.q_stride) ||
+      !make_map(&tk, k, p.B, p.Skv, p.H, p.D, p.k_stride) ||
+      !make_map(&tv, v, p.B, p.Skv, p.H, p.D, p.v_stride))
+    return BSA_ERR_UNSUPPORTED;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t *w = static_cast<uint8_t *>(ws);
+  if (!P.o.plan_ready) {
+    if ((st = cuda_status(launch_plan(p, P.m, P.o, P.L, w, s))) != BSA_OK) return st;
+  }
+  const MaskParams mp = mask_params(p, P.m, P.L, w);
+  if (P.o.softmax_mode == BSA_SOFTMAX_FIXED_M_GATED) {
+    if ((st = cuda_status(launch_fixed_m_bound(p, mp, P.o, q, k, P.L, w, s))) != BSA_OK) return st;
+  }
+  return cuda_status(launch_fwd(p, mp, P.o, signature(p, P.m, P.o), tq, tk, tv, out, lse, P.L, w, s));
+}
+
+bsa_status bsa_attn_bwd(const bsa_problem *prob, const bsa_mask_spec *mask,
+                        const bsa_options *opt, const void *q, const void *k, const void *v,
+                        const void *out, const void *dout, const float *lse, void *dq, void *dk,
+                        void *dv, void *ws, size_t ws_bytes, bsa_stream_t stream) {
+  if (q == nullptr || k == nullptr || v == nullptr || out == nullptr || dout == nullptr ||
+      lse == nullptr || dq == nullptr || dk == nullptr || dv == nullptr)
+    return BSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(dout) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return BSA_ERR_UNSUPPORTED;
+  Prepared P;
+  bsa_status st = prepare(prob, mask, opt, ws, ws_bytes, true, &P);
+  if (st != BSA_OK) return st;
+  const bsa_problem &p = P.p;
+  CUtensorMap tq, tk, tv, tdo;
+  if (!make_map(&tq, q, p.B, p.Sq, p.H, p.D, p.q_stride) ||
+      !make_map(&tk, k, p.B, p.Skv, p.H, p.D, p.k_stride) ||
+      !make_map(&tv, v, p.B, p.Skv, p.H, p.D, p.v_stride) ||
+      !make_map(&tdo, dout, p.B, p.Sq, p.H, p.D, p.o_stride))
+    return BSA_ERR_UNSUPPORTED;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t *w = static_cast<uint8_t *>(ws);
+  if (!P.o.plan_ready) {
+    if ((st = cuda_status(launch_plan(p, P.m, P.o, P.L, w, s))) != BSA_OK) return st;
+  }
+  const MaskParams mp = mask_params(p, P.m, P.L, w);
+  return cuda_status(launch_bwd(p, mp, P.o, signature(p, P.m, P.o), tq, tk, tv, tdo, out, dout,
+                                lse, dq, dk, dv, P.L, w, s));
+}
+
+bsa_status bsa_get_device_status(void *ws, size_t ws_bytes, bsa_stream_t stream, int32_t clear) {
+  if (ws == nullptr || ws_bytes < kHdrWords * 4) return BSA_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint32_t h[2] = {0, 0};
+  if (cudaMemcpyAsync(h, ws, sizeof(h), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return BSA_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return BSA_ERR_CUDA;
+  if (clear) {
+    if (cudaMemsetAsync(ws, 0, sizeof(h), s) != cudaSuccess) return BSA_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return BSA_ERR_CUDA;
+  }
+  if (h[kHdrStatus] != 0) return static_cast<bsa_status>(h[kHdrStatus]);
+  if (h[kHdrGateWarn] != 0) return BSA_WARN_GATE_VIOLATION;
+  return BSA_OK;
+}
+
+const char *bsa_status_string(bsa_status status) {
+  switch (status) {
+    case BSA_OK: return "ok";
+    case BSA_ERR_INVALID_ARG: return "invalid argument";
+    case BSA_ERR_UNSUPPORTED: return "unsupported shape, dtype, stride or alignment";
+    case BSA_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case BSA_ERR_CUDA: return "CUDA runtime error";
+    case BSA_ERR_SEM_TIMEOUT: return "a bounded device wait timed out; results are incomplete";
+    case BSA_ERR_PLAN_MISMATCH: return "workspace plan was built for another problem";
+    case BSA_ERR_BAD_MASK_DATA: return "cu_seqlens is not a non-decreasing [0 .. Sq] sequence";
+    case BSA_WARN_GATE_VIOLATION: return "a gated fixed-m row summed below 2^-100";
+    case BSA_ERR_NO_DEVICE: return "no sm_100 device is current";
+  }
+  return "unknown status";
+}
+
+uint64_t bsa_launch_count(void) { return g_launches.load(); }
+
+}  // extern "C"

@@ -1,0 +1,96 @@
+// Internal declarations shared by the library's translation units: the
+// workspace layout, the mask parameters every kernel evaluates, and the
+// launchers of each step of the hot path.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "../../include/bsa.h"
+
+namespace bsa {
+
+constexpr int kTile = BSA_TILE;
+constexpr uint32_t kFullBit = 1u << 30;
+constexpr uint32_t kIndexMask = (1u << 30) - 1u;
+constexpr uint32_t kPlanMagic = 0xB5A7C0DEu;
+
+// Header words at the start of the workspace.
+enum HeaderWord : int {
+  kHdrStatus = 0,      // sticky bsa_status
+  kHdrGateWarn = 1,    // rows of gated heads whose fixed-m sum fell below 2^-100
+  kHdrFwdTicket = 2,   // forward work-unit ticket counter
+  kHdrBwdTicket = 3,   // backward column ticket counter
+  kHdrMagic = 4,       // plan signature: magic, B, Sq, Skv, flags, window, order, n_seqs
+  kHdrB = 5,
+  kHdrSq = 6,
+  kHdrSkv = 7,
+  kHdrFlags = 8,
+  kHdrWindow = 9,
+  kHdrOrder = 10,
+  kHdrNSeqs = 11,
+  kHdrWords = 64
+};
+
+struct WsLayout {
+  size_t status;                      // header (256 bytes)
+  size_t tile_class, rank;            // dense [B, nM, nN]
+  size_t row_cnt, row_ptr, row_ent;   // row CSR (forward)
+  size_t col_cnt, col_ptr, col_ent, col_rank;  // column CSR (backward)
+  size_t perm;                        // pi [nN]
+  size_t seg_q, seg_kv;               // varlen-derived segment ids [Sq], [Skv]
+  size_t qblk, kblk;                  // per-block segment summaries [B*nM*4], [B*nN*4]
+  size_t kmax, qmax, gate;            // [B, H]
+  size_t qnorm;                       // [B, H, Sq]
+  size_t fwd_end;
+  size_t delta, dq_accum, sem;        // backward scratch
+  size_t total;
+  int nM, nN;
+  int64_t nnz_cap;
+};
+
+WsLayout compute_layout(const bsa_problem &p);
+
+// Plan signature words (B, Sq, Skv, flags, window, order, n_seqs) the planner
+// stores in the header and every kernel that reads the plan checks.
+struct PlanSignature {
+  uint32_t w[7];
+};
+
+// Mask predicates as every kernel sees them.  Varlen masks arrive here as
+// segment ids derived by the planner (alignment rows: -1 on the query side,
+// -2 on the key side, so they never match anything).
+struct MaskParams {
+  uint32_t flags;
+  int32_t window;       // 0 = plain causal (when the flag is set)
+  int32_t offset;       // o = Skv - Sq (bottom-right alignment)
+  int32_t Sq, Skv;
+  const int32_t *seg_q;   // [B, Sq] or null
+  const int32_t *seg_kv;  // [B, Skv] or null
+  const int32_t *kv_valid_len;  // [B] or null
+};
+
+// Launchers (each returns cudaGetLastError() of its launches).
+cudaError_t launch_plan(const bsa_problem &p, const bsa_mask_spec &m, const bsa_options &o,
+                        const WsLayout &L, uint8_t *ws, cudaStream_t s);
+
+cudaError_t launch_fixed_m_bound(const bsa_problem &p, const MaskParams &mp,
+                                 const bsa_options &o, const void *q, const void *k,
+                                 const WsLayout &L, uint8_t *ws, cudaStream_t s);
+
+cudaError_t launch_fwd(const bsa_problem &p, const MaskParams &mp, const bsa_options &o,
+                       const PlanSignature &sig, const CUtensorMap &tq, const CUtensorMap &tk,
+                       const CUtensorMap &tv, void *out, float *lse, const WsLayout &L,
+                       uint8_t *ws, cudaStream_t s);
+
+cudaError_t launch_bwd(const bsa_problem &p, const MaskParams &mp, const bsa_options &o,
+                       const PlanSignature &sig, const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                       const CUtensorMap &tdo, const void *out, const void *dout,
+                       const float *lse, void *dq, void *dk, void *dv, const WsLayout &L,
+                       uint8_t *ws, cudaStream_t s);
+
+void count_launch(int n = 1);
+
+}  // namespace bsa

@@ -1,0 +1,225 @@
+/*
+ * bsa.h -- C ABI of libbsa: block-sparse exact softmax attention for sm_100a.
+ *
+ * What the library computes (all of it in its own CUDA kernels):
+ *
+ *   O = softmax(scale * Q K^T + mask) V  and the per-row LSE,
+ *   dQ, dK, dV of sum(O * dO) with a deterministic dQ accumulation.
+ *
+ * The mask is the AND of up to four predicates (segment ids, global KV padding,
+ * varlen cu_seqlens with trailing alignment rows, causal sliding window).  A
+ * block map classifies every 128 x 128 (q-block, kv-block) tile as EMPTY,
+ * PARTIAL or FULL so that empty tiles are never touched and full tiles skip the
+ * per-element mask.
+ *
+ * Sources (the pages this library restates):
+ *  - "Fixed-m softmax for 2D-ring x Ulysses attention (WAN 2.2)" (maxdiffusion
+ *    PR #452): exact softmax attention whose running max may be replaced by the
+ *    Cauchy-Schwarz bound scale*||q_i||*max_j||k_j||, with a per-head gate that
+ *    keeps online softmax where the bound cannot be proven safe.
+ *  - "Let splash attention exceed 524,288 tokens when packing is off" (maxtext
+ *    PR #4929): segment-id masks; constant ids equal no ids; a block mask.
+ *  - maxdiffusion PR #404 review, padding-mask comment: KV padding only at the
+ *    end of the global sequence, masked by global position.
+ *  - sglang PR #47566, "Modifications": cu_seqlens with trailing alignment rows
+ *    that real rows never see; alignment rows are zero in the output.
+ *  - "Add more optimal dk order optional arg" (flash-attention PR #2512):
+ *    deterministic block-sparse backward with per-m_block dQ semaphores,
+ *    rank(m, n), kv-column orders (asc, desc, arbitrary permutation) and one
+ *    rank-sorted list per kv column.
+ *
+ * Conventions for every call:
+ *  - All tensor pointers are DEVICE pointers unless a field says "host".
+ *  - Q, K, V, O, dO, dQ, dK, dV are bf16 [B, S, H, D] with the head dimension
+ *    contiguous; other strides are given in elements (0 = contiguous BSHD).
+ *    Pointers and strides must be 16-byte aligned.  D is 64 or 128.
+ *  - LSE is fp32 [B, H, Sq], natural log; a row with no allowed key has
+ *    LSE = -inf and O = 0.
+ *  - The caller owns every buffer, including the workspace.  The library never
+ *    allocates device memory, never synchronises (except in
+ *    bsa_get_device_status) and issues all work on the given stream.  Pointers
+ *    are borrowed for the duration of the call's stream work only.
+ *  - Argument errors are returned before anything is launched and nothing is
+ *    written.  Errors detected on the device (inconsistent cu_seqlens, a plan
+ *    that does not match the problem, a semaphore wait that timed out) are
+ *    recorded in the workspace's sticky status word; read it with
+ *    bsa_get_device_status.  There is no CPU fallback and no second backend.
+ */
+#ifndef BSA_H_
+#define BSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define BSA_API __attribute__((visibility("default")))
+#else
+#define BSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t / CUstream; 0 is the legacy default stream. */
+typedef struct CUstream_st *bsa_stream_t;
+
+typedef enum bsa_status {
+  BSA_OK = 0,
+  BSA_ERR_INVALID_ARG = 1,         /* null pointer, bad size, inconsistent fields   */
+  BSA_ERR_UNSUPPORTED = 2,         /* D not in {64,128}, misaligned pointer/stride   */
+  BSA_ERR_WORKSPACE_TOO_SMALL = 3, /* ws_bytes below bsa_workspace_size()            */
+  BSA_ERR_CUDA = 4,                /* a CUDA runtime call or launch failed           */
+  BSA_ERR_SEM_TIMEOUT = 5,         /* device: a bounded wait gave up (work skipped)  */
+  BSA_ERR_PLAN_MISMATCH = 6,       /* device: workspace plan built for another problem */
+  BSA_ERR_BAD_MASK_DATA = 7,       /* device: cu_seqlens not [0 .. Sq] non-decreasing */
+  BSA_WARN_GATE_VIOLATION = 8,     /* device: a gated fixed-m row summed below 2^-100 */
+  BSA_ERR_NO_DEVICE = 9            /* no sm_100 device current                        */
+} bsa_status;
+
+/* Block-map tile edge (rows and keys). */
+#define BSA_TILE 128
+
+/* Tile classes stored in the block map. */
+#define BSA_TILE_EMPTY 0
+#define BSA_TILE_PARTIAL 1
+#define BSA_TILE_FULL 2
+
+/* bsa_mask_spec.flags */
+#define BSA_MASK_SEGMENT_IDS 1u   /* seg_q[b,i] == seg_kv[b,j]                         */
+#define BSA_MASK_KV_VALID_LEN 2u  /* j < kv_valid_len[b]                                */
+#define BSA_MASK_VARLEN 4u        /* same cu_seqlens segment, neither in the alignment tail */
+#define BSA_MASK_CAUSAL_WINDOW 8u /* i+o-W < j <= i+o, o = Skv-Sq (W = 0: j <= i+o)      */
+
+/* bsa_options.softmax_mode */
+#define BSA_SOFTMAX_ONLINE 0
+#define BSA_SOFTMAX_FIXED_M_GATED 1
+
+/* bsa_options.bwd_order: order pi of the kv columns for the dQ semaphores */
+#define BSA_ORDER_ASC 0
+#define BSA_ORDER_DESC 1
+#define BSA_ORDER_PERM 2
+
+typedef struct bsa_problem {
+  int32_t B;       /* batch; 1 for varlen                                        */
+  int32_t H;       /* heads (Q, K and V have the same head count)                */
+  int32_t Sq;      /* query rows per batch (varlen: total tokens T)               */
+  int32_t Skv;     /* keys per batch (varlen: T)                                  */
+  int32_t D;       /* head dim, 64 or 128                                         */
+  int32_t reserved0;
+  /* element strides (batch, seq, head); all zero = contiguous BSHD.  q_stride
+   * is used for Q and dQ, k_stride for K and dK, v_stride for V and dV,
+   * o_stride for O and dO. */
+  int64_t q_stride[3];
+  int64_t k_stride[3];
+  int64_t v_stride[3];
+  int64_t o_stride[3];
+  float scale;     /* <= 0: 1/sqrt(D)                                             */
+  int32_t reserved1;
+} bsa_problem;
+
+typedef struct bsa_mask_spec {
+  uint32_t flags;              /* OR of BSA_MASK_*                                  */
+  int32_t window;              /* BSA_MASK_CAUSAL_WINDOW: keys per row including
+                                  the diagonal; 0 = unlimited causal                */
+  const int32_t *seg_q;        /* device [B, Sq]  (BSA_MASK_SEGMENT_IDS)            */
+  const int32_t *seg_kv;       /* device [B, Skv] (BSA_MASK_SEGMENT_IDS)            */
+  const int32_t *kv_valid_len; /* device [B]      (BSA_MASK_KV_VALID_LEN)           */
+  const int32_t *cu_seqlens;   /* device [n_seqs + 1], cu[0] = 0, cu[n_seqs] = Sq    */
+  int32_t n_seqs;              /* segments in cu_seqlens (BSA_MASK_VARLEN)           */
+  int32_t n_align_tail;        /* trailing segments that are alignment rows         */
+} bsa_mask_spec;
+
+typedef struct bsa_options {
+  int32_t softmax_mode;        /* BSA_SOFTMAX_*                                     */
+  float gate_limit;            /* fixed-m gate G: a head runs fixed-m iff
+                                  2*scale*max_i||q_i||*kmax <= G; <= 0: 64          */
+  const float *kmax_override;  /* device [B, H] or NULL: caller-supplied max_j||k_j||
+                                  bound used as is                                  */
+  int32_t bwd_order;           /* BSA_ORDER_*                                       */
+  int32_t deterministic;       /* 1: semaphore-ordered dQ; 0: atomic dQ             */
+  const int32_t *perm;         /* HOST [ceil(Skv/128)] permutation (BSA_ORDER_PERM)  */
+  int64_t sem_timeout_ns;      /* bound of every dQ semaphore wait; <= 0: 1 s       */
+  int32_t plan_ready;          /* 1: the workspace already holds the plan for this
+                                  problem, mask and order (bsa_plan_build or an
+                                  earlier fwd/bwd call); 0: build it first          */
+  int32_t reserved;
+} bsa_options;
+
+/* Where the plan and the scratch arrays sit inside the workspace (byte offsets),
+ * for inspection and tests.  Filled by bsa_workspace_layout. */
+typedef struct bsa_workspace_view {
+  size_t total_bytes;          /* forward + backward workspace                       */
+  size_t fwd_bytes;            /* enough for bsa_plan_build + bsa_attn_fwd           */
+  size_t off_status;           /* uint32 sticky status word                          */
+  size_t off_tile_class;       /* uint8  [B, nM, nN]  BSA_TILE_*                     */
+  size_t off_rank;             /* int32  [B, nM, nN]  rank(m, n), -1 where EMPTY     */
+  size_t off_row_ptr;          /* int32  [B*nM + 1]   row CSR offsets                */
+  size_t off_row_ent;          /* int32  [nnz]        n | FULL << 30, ascending n    */
+  size_t off_col_ptr;          /* int32  [B*nN + 1]   column CSR offsets             */
+  size_t off_col_ent;          /* int32  [nnz]        m | FULL << 30, (rank, m) order */
+  size_t off_col_rank;         /* int32  [nnz]        rank of each column entry      */
+  size_t off_perm;             /* int32  [nN]         pi                             */
+  size_t off_kmax;             /* fp32   [B, H]       fixed-m key-norm bound          */
+  size_t off_qmax;             /* fp32   [B, H]       max query norm                 */
+  size_t off_gate;             /* int32  [B, H]       1 = fixed-m, 0 = online        */
+  size_t off_delta;            /* fp32   [B, H, nM*128]  backward Delta              */
+  size_t off_dq_accum;         /* fp32   backward dQ accumulator                     */
+  size_t off_sem;              /* int32  [B, H, nM]   dQ semaphores                  */
+  int32_t nM, nN;
+} bsa_workspace_view;
+
+/* Bytes of workspace a problem needs.  with_backward = 0 sizes the forward
+ * only (plan + fixed-m bound); 1 adds Delta, the fp32 dQ accumulator and the
+ * semaphores.  Pure host arithmetic; no CUDA call. */
+BSA_API bsa_status bsa_workspace_size(const bsa_problem *prob, const bsa_mask_spec *mask,
+                              int32_t with_backward, size_t *bytes);
+
+/* Offsets of the plan and scratch arrays inside the workspace (host only). */
+BSA_API bsa_status bsa_workspace_layout(const bsa_problem *prob, const bsa_mask_spec *mask,
+                                bsa_workspace_view *view);
+
+/* Block map and backward schedule (steps a1 and a6 of the hot path): tile
+ * classes from the mask predicates, row lists for the forward, rank(m, n)
+ * under the order pi and the rank-sorted column lists for the backward.
+ * Runs as CUDA kernels on `stream`; resets the sticky status word. */
+BSA_API bsa_status bsa_plan_build(const bsa_problem *prob, const bsa_mask_spec *mask,
+                          const bsa_options *opt, void *ws, size_t ws_bytes,
+                          bsa_stream_t stream);
+
+/* Forward: out (bf16, o_stride layout) and lse (fp32 [B,H,Sq]).  With
+ * BSA_SOFTMAX_FIXED_M_GATED it first computes kmax/qmax/gate per (b, h) and
+ * runs the fixed-m body on heads that pass the gate, online softmax on the
+ * others.  Rows in the varlen alignment tail are written as 0 / -inf. */
+BSA_API bsa_status bsa_attn_fwd(const bsa_problem *prob, const bsa_mask_spec *mask,
+                        const bsa_options *opt, const void *q, const void *k,
+                        const void *v, void *out, float *lse, void *ws,
+                        size_t ws_bytes, bsa_stream_t stream);
+
+/* Backward: dq, dk, dv (bf16) from q, k, v, the forward's out and lse and the
+ * incoming gradient dout.  deterministic = 1 orders every dQ contribution by the
+ * dQ semaphores (bit-identical results run to run); 0 uses atomic adds.
+ * Needs a workspace sized with with_backward = 1. */
+BSA_API bsa_status bsa_attn_bwd(const bsa_problem *prob, const bsa_mask_spec *mask,
+                        const bsa_options *opt, const void *q, const void *k,
+                        const void *v, const void *out, const void *dout,
+                        const float *lse, void *dq, void *dk, void *dv, void *ws,
+                        size_t ws_bytes, bsa_stream_t stream);
+
+/* Synchronises `stream`, then returns the sticky device status of `ws`
+ * (BSA_OK if no device-side error was recorded); clear = 1 resets it. */
+BSA_API bsa_status bsa_get_device_status(void *ws, size_t ws_bytes, bsa_stream_t stream,
+                                 int32_t clear);
+
+/* Static description of a status code. */
+BSA_API const char *bsa_status_string(bsa_status status);
+
+/* Number of this library's kernel launches issued by the calling thread since
+ * load (for the bench's launch count). */
+BSA_API uint64_t bsa_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BSA_H_ */

@@ -1,0 +1,150 @@
+"""The C ABI without a GPU: the library loads, exports every function the header
+declares, the ctypes structs match the C layout, and argument errors come back
+as status codes before anything touches CUDA."""
+
+import ctypes
+import os
+import subprocess
+import tempfile
+
+import pytest
+
+from block_sparse_attention_map_b200 import _binding as bd
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    if not os.path.exists(bd.LIB_PATH):
+        from block_sparse_attention_map_b200 import build
+        build.build()
+    return bd.lib()
+
+
+def test_exports_every_declared_function(L):
+    names = bd.header_functions()
+    assert {"bsa_attn_fwd", "bsa_attn_bwd", "bsa_plan_build", "bsa_workspace_size",
+            "bsa_get_device_status", "bsa_status_string"} <= set(names)
+    for n in names:
+        assert hasattr(L, n), n
+    out = subprocess.run(["nm", "-D", "--defined-only", bd.LIB_PATH], capture_output=True, text=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    assert set(names) <= exported
+    # nothing but the C ABI is exported
+    assert {e for e in exported if e.startswith("bsa_")} == set(names)
+
+
+def _c_layout():
+    src = r"""
+#include <stdio.h>
+#include <stddef.h>
+#include "bsa.h"
+#define P(T, f) printf(#T "." #f " %zu\n", offsetof(T, f));
+int main(void) {
+  printf("bsa_problem %zu\nbsa_mask_spec %zu\nbsa_options %zu\nbsa_workspace_view %zu\n",
+         sizeof(bsa_problem), sizeof(bsa_mask_spec), sizeof(bsa_options), sizeof(bsa_workspace_view));
+  P(bsa_problem, q_stride) P(bsa_problem, o_stride) P(bsa_problem, scale)
+  P(bsa_mask_spec, seg_q) P(bsa_mask_spec, cu_seqlens) P(bsa_mask_spec, n_align_tail)
+  P(bsa_options, kmax_override) P(bsa_options, perm) P(bsa_options, sem_timeout_ns) P(bsa_options, plan_ready)
+  P(bsa_workspace_view, off_sem) P(bsa_workspace_view, nN)
+  return 0;
+}
+"""
+    with tempfile.TemporaryDirectory() as d:
+        c = os.path.join(d, "l.c")
+        exe = os.path.join(d, "l")
+        open(c, "w").write(src)
+        subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), c, "-o", exe], check=True)
+        out = subprocess.run([exe], capture_output=True, text=True, check=True).stdout
+    return dict((k, int(v)) for k, v in (line.split() for line in out.splitlines()))
+
+
+def test_ctypes_structs_match_c_layout():
+    c = _c_layout()
+    assert c["bsa_problem"] == ctypes.sizeof(bd.Problem)
+    assert c["bsa_mask_spec"] == ctypes.sizeof(bd.MaskSpec)
+    assert c["bsa_options"] == ctypes.sizeof(bd.Options)
+    assert c["bsa_workspace_view"] == ctypes.sizeof(bd.WorkspaceView)
+    assert c["bsa_problem.q_stride"] == bd.Problem.q_stride.offset
+    assert c["bsa_problem.o_stride"] == bd.Problem.o_stride.offset
+    assert c["bsa_problem.scale"] == bd.Problem.scale.offset
+    assert c["bsa_mask_spec.seg_q"] == bd.MaskSpec.seg_q.offset
+    assert c["bsa_mask_spec.cu_seqlens"] == bd.MaskSpec.cu_seqlens.offset
+    assert c["bsa_mask_spec.n_align_tail"] == bd.MaskSpec.n_align_tail.offset
+    assert c["bsa_options.kmax_override"] == bd.Options.kmax_override.offset
+    assert c["bsa_options.perm"] == bd.Options.perm.offset
+    assert c["bsa_options.sem_timeout_ns"] == bd.Options.sem_timeout_ns.offset
+    assert c["bsa_options.plan_ready"] == bd.Options.plan_ready.offset
+    assert c["bsa_workspace_view.off_sem"] == bd.WorkspaceView.off_sem.offset
+    assert c["bsa_workspace_view.nN"] == bd.WorkspaceView.nN.offset
+
+
+def _prob(B=1, H=2, Sq=256, Skv=256, D=64):
+    p = bd.Problem()
+    p.B, p.H, p.Sq, p.Skv, p.D = B, H, Sq, Skv, D
+    return p
+
+
+def _size(L, p, m=None, bwd=1):
+    n = ctypes.c_size_t(0)
+    rc = L.bsa_workspace_size(ctypes.byref(p), ctypes.byref(m) if m is not None else None, bwd,
+                              ctypes.byref(n))
+    return rc, n.value
+
+
+def test_workspace_size_and_validation(L):
+    rc, fwd = _size(L, _prob(), bwd=0)
+    assert rc == 0 and fwd > 0
+    rc, tot = _size(L, _prob(), bwd=1)
+    # the backward adds Delta, the fp32 dQ accumulator [B,H,nM*128,D] and semaphores
+    assert rc == 0 and tot >= fwd + 4 * 2 * 256 * 64 + 4 * 2 * 256
+    assert _size(L, _prob(D=96))[0] == 2          # unsupported head dim
+    assert _size(L, _prob(B=0))[0] == 1           # invalid
+    p = _prob()
+    p.q_stride[:] = (256 * 2 * 64, 2 * 64 + 4, 64)  # row stride not a multiple of 16 bytes
+    assert _size(L, p)[0] == 2
+    m = bd.MaskSpec()
+    m.flags = bd.MASK_SEGMENT_IDS                   # ids missing
+    assert _size(L, _prob(), m)[0] == 1
+    m = bd.MaskSpec()
+    m.flags = bd.MASK_VARLEN
+    m.cu_seqlens = 16
+    m.n_seqs = 2
+    assert _size(L, _prob(B=2), m)[0] == 1          # varlen needs B == 1
+    assert _size(L, _prob(Sq=100, Skv=120), m)[0] == 1  # and Sq == Skv
+    m.flags = 1 << 7                                # unknown flag
+    assert _size(L, _prob(), m)[0] == 1
+
+
+def test_calls_reject_bad_arguments_before_cuda(L):
+    p = _prob()
+    o = bd.Options()
+    # null tensor pointers
+    assert L.bsa_attn_fwd(ctypes.byref(p), None, ctypes.byref(o), None, None, None, None, None,
+                          None, 0, None) == 1
+    # misaligned pointers
+    assert L.bsa_attn_fwd(ctypes.byref(p), None, ctypes.byref(o), 8, 256, 512, 1024, 4096,
+                          4096, 1 << 20, None) == 2
+    # bad order and a non-permutation
+    o.bwd_order = 7
+    assert L.bsa_plan_build(ctypes.byref(p), None, ctypes.byref(o), 4096, 1 << 30, None) == 1
+    o.bwd_order = 2
+    bad = (ctypes.c_int32 * 2)(0, 0)
+    o.perm = ctypes.cast(bad, ctypes.c_void_p)
+    assert L.bsa_plan_build(ctypes.byref(p), None, ctypes.byref(o), 4096, 1 << 30, None) == 1
+    # workspace too small
+    o = bd.Options()
+    assert L.bsa_plan_build(ctypes.byref(p), None, ctypes.byref(o), 4096, 16, None) == 3
+    assert L.bsa_status_string(0).decode() == "ok"
+    assert L.bsa_status_string(5).decode().startswith("a bounded device wait")
+
+
+def test_layout_offsets_are_aligned(L):
+    v = bd.WorkspaceView()
+    assert L.bsa_workspace_layout(ctypes.byref(_prob(B=2, H=3, Sq=1000, Skv=777, D=128)), None,
+                                  ctypes.byref(v)) == 0
+    assert v.nM == 8 and v.nN == 7
+    offs = [getattr(v, f) for f, _ in bd.WorkspaceView._fields_ if f.startswith("off_")]
+    assert all(o % 4 == 0 for o in offs)
+    assert v.off_status == 0 and v.fwd_bytes <= v.off_delta < v.total_bytes

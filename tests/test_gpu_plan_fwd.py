@@ -1,0 +1,216 @@
+"""GPU parity: the block-map planner and the forward kernel against the oracle."""
+
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_attention_map_b200 as bsa
+import oracle
+from block_sparse_attention_map_b200.workloads import make_workload
+from tests.gpu_common import LSE_TOL, O_TOL, compare_lse, compare_out, mask_desc, np64, sample_rows
+
+pytestmark = pytest.mark.gpu
+
+SMALL = ["tiny", "packed", "packed_const", "window", "window_rect", "varlen", "video"]
+
+
+@pytest.mark.parametrize("name", SMALL)
+def test_plan_tile_classes_match_oracle(name):
+    wl = make_workload(name, device="cuda", small=True)
+    ws = bsa.plan_build(wl.q, wl.k, wl.v, wl.mask)
+    cls = ws.tile_classes().cpu().numpy()
+    ref = oracle.tile_classes(mask_desc(wl), wl.B, wl.Sq, wl.Skv)
+    assert np.array_equal(cls, ref)
+    assert ws.status() == 0
+
+
+@pytest.mark.parametrize("name,B,Sq,Skv", [("window", 1, 8192, 8192), ("window_rect", 1, 4096, 8192)])
+def test_plan_full_size_window_counts(name, B, Sq, Skv):
+    wl = make_workload(name, device="cuda")
+    ws = bsa.plan_build(wl.q, wl.k, wl.v, wl.mask)
+    cls = ws.tile_classes().cpu().numpy()
+    ref = oracle.tile_classes(mask_desc(wl), B, Sq, Skv)
+    assert np.array_equal(cls, ref)
+
+
+@pytest.mark.parametrize("order", ["asc", "desc", "perm"])
+@pytest.mark.parametrize("name", ["window", "packed", "window_rect"])
+def test_plan_ranks_and_column_lists(name, order):
+    wl = make_workload(name, device="cuda", small=True)
+    nN = -(-wl.Skv // 128)
+    perm = np.random.default_rng(5).permutation(nN) if order == "perm" else None
+    ws = bsa.plan_build(wl.q, wl.k, wl.v, wl.mask, order=order, perm=perm)
+    cls = oracle.tile_classes(mask_desc(wl), wl.B, wl.Sq, wl.Skv)
+    pi = oracle.column_order(nN, order, perm)
+    assert np.array_equal(ws.perm().cpu().numpy(), pi)
+    rank = oracle.kv_ranks(cls, pi)
+    assert np.array_equal(ws.ranks().cpu().numpy(), rank)
+    lists = oracle.column_lists(cls, rank)
+    ptr, ent, rk = ws.col_lists()
+    for b in range(wl.B):
+        for n in range(nN):
+            s, e = ptr[b * nN + n], ptr[b * nN + n + 1]
+            got = [(int(x & (bsa._binding.FULL_BIT - 1)), int(r), bool(x & bsa._binding.FULL_BIT))
+                   for x, r in zip(ent[s:e], rk[s:e])]
+            assert got == lists[(b, n)]
+    rptr, rent = ws.row_lists()
+    for b in range(wl.B):
+        for m in range(cls.shape[1]):
+            s, e = rptr[b * cls.shape[1] + m], rptr[b * cls.shape[1] + m + 1]
+            got = [(int(x & (bsa._binding.FULL_BIT - 1)), bool(x & bsa._binding.FULL_BIT)) for x in rent[s:e]]
+            exp = [(n, cls[b, m, n] == oracle.FULL) for n in range(nN) if cls[b, m, n] != oracle.EMPTY]
+            assert got == exp
+
+
+def _fwd_vs_oracle(wl, mode="online", rows=None):
+    o, lse, ws = bsa.attn_fwd(wl.q, wl.k, wl.v, wl.mask, softmax_mode=mode)
+    torch.cuda.synchronize()
+    assert ws.status() == 0
+    q, k, v = np64(wl.q), np64(wl.k), np64(wl.v)
+    O_ref, L_ref = oracle.attention_forward(q, k, v, mask_desc(wl), wl.scale, rows=rows)
+    eo = compare_out(o, O_ref, rows)
+    el, same = compare_lse(lse, L_ref, rows)
+    return eo, el, same, o, lse, ws
+
+
+@pytest.mark.parametrize("name", SMALL)
+def test_fwd_online_matches_oracle(name):
+    wl = make_workload(name, device="cuda", small=True)
+    eo, el, same, *_ = _fwd_vs_oracle(wl)
+    assert eo <= O_TOL and el <= LSE_TOL and same, (eo, el, same)
+
+
+@pytest.mark.parametrize("name", ["video", "tiny", "window", "varlen"])
+def test_fwd_fixed_m_matches_oracle(name):
+    wl = make_workload(name, device="cuda", small=True)
+    eo, el, same, o, lse, ws = _fwd_vs_oracle(wl, "fixed_m")
+    assert eo <= O_TOL and el <= LSE_TOL and same, (eo, el, same)
+
+
+def test_fixed_m_bound_and_gate_match_oracle():
+    wl = make_workload("video", device="cuda", small=True)
+    _, _, ws = bsa.attn_fwd(wl.q, wl.k, wl.v, wl.mask, softmax_mode="fixed_m")
+    torch.cuda.synchronize()
+    kmax, qmax, bound, gate = oracle.fixed_m_bound(np64(wl.q), np64(wl.k), mask_desc(wl), wl.scale)
+    assert np.allclose(ws.kmax().cpu().numpy(), kmax, rtol=1e-5)
+    assert np.allclose(ws.qmax().cpu().numpy(), qmax, rtol=1e-5)
+    g = ws.gate().cpu().numpy().astype(bool)
+    # the gate decision is taken in fp32 on the device: equal unless the bound
+    # sits within 1e-4 of the limit
+    close = np.abs(2 * bound - 64.0) < 1e-4 * 64
+    assert np.array_equal(g[~close], gate[~close])
+    assert not g[0, 0] and g[0, 1:].all()  # the sink head falls back
+
+
+def test_fixed_m_and_online_agree_bitwise_on_fallback_head():
+    wl = make_workload("video", device="cuda", small=True)
+    o1, l1, _ = bsa.attn_fwd(wl.q, wl.k, wl.v, wl.mask, softmax_mode="online")
+    o2, l2, ws = bsa.attn_fwd(wl.q, wl.k, wl.v, wl.mask, softmax_mode="fixed_m")
+    torch.cuda.synchronize()
+    # head 0 fails the gate and runs the online body: identical bits
+    assert torch.equal(o1[:, :, 0], o2[:, :, 0]) and torch.equal(l1[:, 0], l2[:, 0])
+    assert (o1 - o2).abs().max().item() <= O_TOL
+
+
+def test_constant_segment_ids_bitwise_equal_no_mask():
+    wl = make_workload("packed_const", device="cuda", small=True)
+    o1, l1, _ = bsa.attn_fwd(wl.q, wl.k, wl.v, wl.mask)
+    o2, l2, _ = bsa.attn_fwd(wl.q, wl.k, wl.v, None)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_alignment_rows_zero_and_isolated():
+    wl = make_workload("varlen", device="cuda", small=True)
+    T_real = wl.mask["cu_seqlens"][-1 - wl.mask["n_align_tail"]]
+    o1, l1, _ = bsa.attn_fwd(wl.q, wl.k, wl.v, wl.mask)
+    q2, k2, v2 = wl.q.clone(), wl.k.clone(), wl.v.clone()
+    for t in (q2, k2, v2):
+        t[:, T_real:] = (torch.randn_like(t[:, T_real:].float()) * 30).to(t.dtype)
+    o2, l2, _ = bsa.attn_fwd(q2, k2, v2, wl.mask)
+    torch.cuda.synchronize()
+    assert torch.equal(o1[:, :T_real], o2[:, :T_real]) and torch.equal(l1[..., :T_real], l2[..., :T_real])
+    assert (o1[:, T_real:] == 0).all() and torch.isneginf(l1[..., T_real:]).all()
+
+
+def test_padding_contents_do_not_matter():
+    wl = make_workload("video", device="cuda", small=True)
+    L = int(wl.mask["kv_valid_len"][0])
+    o1, l1, _ = bsa.attn_fwd(wl.q, wl.k, wl.v, wl.mask)
+    k2, v2 = wl.k.clone(), wl.v.clone()
+    k2[:, L:] = 0
+    v2[:, L:] = 1000
+    o2, l2, _ = bsa.attn_fwd(wl.q, k2, v2, wl.mask)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_fwd_deterministic_run_to_run():
+    wl = make_workload("packed", device="cuda", small=True)
+    o1, l1, _ = bsa.attn_fwd(wl.q, wl.k, wl.v, wl.mask)
+    for _ in range(3):
+        o2, l2, _ = bsa.attn_fwd(wl.q, wl.k, wl.v, wl.mask)
+        assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_ragged_shapes_and_d64():
+    g = torch.Generator(device="cuda")
+    g.manual_seed(11)
+    for (Sq, Skv, D, W) in [(1, 1, 64, None), (77, 300, 64, 0), (300, 77, 128, 40), (129, 129, 128, None)]:
+        q = torch.randn(2, Sq, 3, D, device="cuda", generator=g).bfloat16()
+        k = torch.randn(2, Skv, 3, D, device="cuda", generator=g).bfloat16()
+        v = torch.randn(2, Skv, 3, D, device="cuda", generator=g).bfloat16()
+        mask = {"window": W} if W is not None else {}
+        o, lse, ws = bsa.attn_fwd(q, k, v, mask)
+        torch.cuda.synchronize()
+        assert ws.status() == 0
+        O_ref, L_ref = oracle.attention_forward(np64(q), np64(k), np64(v), oracle.MaskDesc(**mask), 1 / D ** 0.5)
+        assert compare_out(o, O_ref) <= O_TOL
+        el, same = compare_lse(lse, L_ref)
+        assert el <= LSE_TOL and same
+
+
+def test_strided_inputs():
+    g = torch.Generator(device="cuda")
+    g.manual_seed(12)
+    base = torch.randn(1, 300, 4, 3 * 128, device="cuda", generator=g).bfloat16()
+    q, k, v = base[..., :128], base[..., 128:256], base[..., 256:]
+    out = torch.empty(1, 300, 4, 256, device="cuda", dtype=torch.bfloat16)[..., 64:192]
+    o, lse, _ = bsa.attn_fwd(q, k, v, {"window": 100}, out=out)
+    torch.cuda.synchronize()
+    O_ref, L_ref = oracle.attention_forward(np64(q), np64(k), np64(v), oracle.MaskDesc(window=100), 128 ** -0.5)
+    assert compare_out(o, O_ref) <= O_TOL
+
+
+@pytest.mark.parametrize("name,extra", [("window", ()), ("window_rect", ()), ("varlen", (33002,)),
+                                        ("packed", ())])
+def test_fwd_full_size_sampled_rows(name, extra):
+    wl = make_workload(name, device="cuda")
+    rows = sample_rows(wl.Sq, seed=1, extra=extra)
+    heads = [0, wl.H - 1]
+    o, lse, ws = bsa.attn_fwd(wl.q, wl.k, wl.v, wl.mask)
+    torch.cuda.synchronize()
+    assert ws.status() == 0
+    q, k, v = np64(wl.q[:, :, heads]), np64(wl.k[:, :, heads]), np64(wl.v[:, :, heads])
+    O_ref, L_ref = oracle.attention_forward(q, k, v, mask_desc(wl), wl.scale, rows=rows)
+    assert compare_out(o[:, :, heads], O_ref, rows) <= O_TOL
+    el, same = compare_lse(lse[:, heads], L_ref, rows)
+    assert el <= LSE_TOL and same
+
+
+@pytest.mark.parametrize("mode", ["online", "fixed_m"])
+def test_fwd_video_full_size_sampled_rows(mode):
+    wl = make_workload("video", device="cuda")
+    rows = sample_rows(wl.Sq, seed=2, extra=(75600,))[::3]
+    heads = [0, 1, 39]
+    o, lse, ws = bsa.attn_fwd(wl.q, wl.k, wl.v, wl.mask, softmax_mode=mode)
+    torch.cuda.synchronize()
+    assert ws.status() == 0
+    if mode == "fixed_m":
+        g = ws.gate().cpu().numpy()
+        assert g[0, 0] == 0 and g[0, 1:].all()
+    q, k, v = np64(wl.q[:, :, heads]), np64(wl.k[:, :, heads]), np64(wl.v[:, :, heads])
+    O_ref, L_ref = oracle.attention_forward(q, k, v, mask_desc(wl), wl.scale, rows=rows)
+    assert compare_out(o[:, :, heads], O_ref, rows) <= O_TOL
+    el, same = compare_lse(lse[:, heads], L_ref, rows)
+    assert el <= LSE_TOL and same
