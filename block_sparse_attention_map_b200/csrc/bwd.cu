@@ -1,12 +1,733 @@
-// Backward pass: placeholder until the deterministic kernel lands.
+// Backward pass (steps a4, a5 and a7 of the hot path).
+//
+// a4  preprocess: Delta_i = sum_d dO_id O_id (fp32) for every query row.
+// a5  main loop per kv column n (CTA = (b, h, n)): K_n and V_n stay in shared
+//     memory; for each q-block m of the column's rank-sorted list the CTA
+//     recomputes S^T = K_n Q_m^T and dP^T = V_n dO_m^T, forms
+//     P^T = exp(S^T - LSE) (masked on PARTIAL tiles) and dS^T = P^T o (dP^T - Delta),
+//     accumulates dV += P^T dO_m and dK += dS^T Q_m in TMEM, computes
+//     dQ_m part = dS K_n and adds it to the fp32 dQ accumulator.  With the
+//     deterministic protocol the add for q-block m waits until the per-m_block
+//     semaphore equals rank(m, n), then increments it, so every dQ row sums its
+//     contributions in the fixed order pi ("Add more optimal dk order optional
+//     arg", flash-attention PR #2512, "Sliding window perf issue" and "A simplish
+//     fix").  Columns are handed out by an atomic ticket in pi order, so a column
+//     only ever waits on columns that some running CTA already holds.
+// a7  convert: dQ = bf16(dQ accumulator).
+//
+// sm_100a roles (384 threads, one CTA per SM, persistent over tickets):
+//   warp 0      ticket + TMA producer (K_n, V_n once per column; Q_m, dO_m per entry)
+//   warp 1      TMEM owner and tcgen05.mma issuer (one lane)
+//   warps 4..7  compute: one key row per thread (TMEM lane), P^T back to TMEM as the
+//               A operand of dV, dS^T to shared memory (128-byte swizzle, K-major
+//               for dK, read MN-major as the A operand of dQ), dK/dV epilogue
+//   warps 8..11 dQ: one query row per thread, semaphore wait, vector reductions
+// TMEM columns: S^T / P^T [0,128)  dP^T / dQ [128,256)  dV [256,256+D)  dK [256+D,256+2D)
+#include <cfloat>
+
 #include "internal.h"
+#include "ptx.cuh"
 
 namespace bsa {
-cudaError_t launch_bwd(const bsa_problem &, const MaskParams &, const bsa_options &,
-                       const PlanSignature &, const CUtensorMap &, const CUtensorMap &,
-                       const CUtensorMap &, const CUtensorMap &, const void *, const void *,
-                       const float *, void *, void *, void *, const WsLayout &, uint8_t *,
-                       cudaStream_t) {
-  return cudaErrorNotSupported;
+namespace {
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+struct BwdParams {
+  MaskParams mask;
+  int B, H, Sq, Skv, nM, nN, n_tickets;
+  float scale, scale_log2;
+  const int32_t *col_ptr;
+  const uint32_t *col_ent;
+  const int32_t *col_rank;
+  const int32_t *perm;
+  const float *lse;    // [B, H, Sq]
+  const float *delta;  // [B, H, nM*128]
+  float *dq_accum;     // [B, H, nM, D/4, 128, 4]
+  uint32_t *sem;       // [B, H, nM]
+  __nv_bfloat16 *dk, *dv;
+  int64_t k_sb, k_ss, k_sh, v_sb, v_ss, v_sh;
+  int deterministic;
+  uint32_t *hdr;
+  uint64_t timeout_ns, sem_timeout_ns;
+  uint32_t sig[7];
+  uint32_t sig_mask;
+};
+
+template <int D, int NQ, int NDO>
+struct BwdSmem {
+  static constexpr int kTB = kTile * D * 2;
+  static constexpr int kK = 0;
+  static constexpr int kV = kK + kTB;
+  static constexpr int kDS = kV + kTB;           // dS^T, 128 x 128 bf16
+  static constexpr int kQ = kDS + 32768;
+  static constexpr int kDO = kQ + NQ * kTB;
+  static constexpr int kVec = kDO + NDO * kTB;   // lse[2][128], delta[2][128], segq[2][128]
+  static constexpr int kTk = kVec + 3 * 2 * kTile * 4;  // ticket ring int[2]
+  static constexpr int kBar = kTk + 16;
+  static constexpr int bTkFull = 0, bTkEmpty = 2, bKVFull = 4, bKVFree = 5, bQFull = 6,
+                       bQEmpty = bQFull + NQ, bDOFull = bQEmpty + NQ, bDOEmpty = bDOFull + NDO,
+                       bSdPFull = bDOEmpty + NDO, bPdSReady = bSdPFull + 1, bDVDone = bPdSReady + 1,
+                       bDSFree = bDVDone + 1, bDQFull = bDSFree + 1, bDQFree = bDQFull + 1,
+                       bDKVFull = bDQFree + 1, bDKVFree = bDKVFull + 1, bVecReady = bDKVFree + 1,
+                       bDQAdded = bVecReady + 2, bFinal = bDQAdded + 2, kNumBars = bFinal + 1;
+  static constexpr int kMisc = kBar + kNumBars * 8;
+  static constexpr int kBytes = kMisc + 16;
+  static constexpr int kAlloc = kBytes + 1024;
+};
+
+constexpr int kConsumersPerTicket = 1 + 4 + 4;  // MMA lane, compute warps, dQ warps
+
+__device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity) {
+  const uint32_t a = smem_u32(bar);
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(a, parity)) {
+    if (globaltimer_ns() - t0 > 200000000ull) return;
+  }
 }
+
+// Bounded acquire-spin on a dQ semaphore; gives up (false) on timeout or when
+// another CTA has already recorded an error.
+__device__ bool sem_wait(const uint32_t *sem, uint32_t target, uint64_t limit_ns,
+                         uint32_t *status) {
+  if (ld_acquire_gpu(sem) == target) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (ld_acquire_gpu(sem) == target) return true;
+    if ((it & 63u) == 0u) {
+      if (*reinterpret_cast<volatile uint32_t *>(status) != 0u) return false;
+      if (globaltimer_ns() - t0 > limit_ns) {
+        record_status(status, BSA_ERR_SEM_TIMEOUT);
+        return false;
+      }
+    }
+    __nanosleep(32);
+  }
+}
+
+struct Ticket {
+  int valid, b, h, n, bh, es, ee;
+};
+
+__device__ __forceinline__ Ticket decode_ticket(const BwdParams &p, int t) {
+  Ticket k{};
+  if (t < 0 || t >= p.n_tickets) return k;
+  const int BH = p.B * p.H;
+  const int pos = t / BH, bh = t % BH;
+  k.valid = 1;
+  k.bh = bh;
+  k.b = bh / p.H;
+  k.h = bh % p.H;
+  k.n = p.perm[pos];
+  k.es = p.col_ptr[k.b * p.nN + k.n];
+  k.ee = p.col_ptr[k.b * p.nN + k.n + 1];
+  return k;
+}
+
+template <int D, int NQ, int NDO>
+__global__ void __launch_bounds__(384, 1)
+k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+           const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo,
+           const BwdParams p) {
+  using L = BwdSmem<D, NQ, NDO>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                            ~static_cast<uintptr_t>(1023));
+  uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::kBar);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::kMisc);
+  int *abort_flag = reinterpret_cast<int *>(sm + L::kMisc + 4);
+  volatile int *tk_ring = reinterpret_cast<volatile int *>(sm + L::kTk);
+  float *vec_lse = reinterpret_cast<float *>(sm + L::kVec);          // [2][128]
+  float *vec_delta = vec_lse + 2 * kTile;                             // [2][128]
+  int32_t *vec_seg = reinterpret_cast<int32_t *>(vec_delta + 2 * kTile);  // [2][128]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int kTB = L::kTB;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < L::kNumBars; ++i) {
+      uint32_t cnt = 1;
+      if (i == L::bTkEmpty || i == L::bTkEmpty + 1) cnt = kConsumersPerTicket;
+      if (i == L::bPdSReady || i == L::bDQFree || i == L::bDKVFree || i == L::bVecReady ||
+          i == L::bVecReady + 1)
+        cnt = 128;
+      if (i == L::bDQAdded || i == L::bDQAdded + 1) cnt = 4;
+      mbar_init(&bars[i], cnt);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tq);
+    tma_prefetch_desc(&tk);
+    tma_prefetch_desc(&tv);
+    tma_prefetch_desc(&tdo);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  Watchdog wd{abort_flag, p.hdr + kHdrStatus, p.timeout_ns};
+  if (threadIdx.x == 0) {
+    const volatile uint32_t *h = p.hdr;
+    bool ok = h[kHdrMagic] == kPlanMagic;
+    for (int i = 0; i < 7; ++i) ok = ok && (!((p.sig_mask >> i) & 1u) || h[kHdrB + i] == p.sig[i]);
+    if (!ok) wd.trip(BSA_ERR_PLAN_MISMATCH);
+  }
+  __syncthreads();
+
+  const uint32_t T_S = tmem, T_DP = tmem + 128, T_DV = tmem + 256, T_DK = tmem + 256 + D;
+  constexpr uint32_t kIdS = idesc_bf16_f32(128, 128, 0, 0);      // S^T, dP^T: both K-major
+  constexpr uint32_t kIdKV = idesc_bf16_f32(128, D, 0, 1);       // dV (TS), dK: B MN-major
+  constexpr uint32_t kIdQ = idesc_bf16_f32(128, D, 1, 1);        // dQ: A and B MN-major
+
+  if (wd.aborted()) {
+  } else if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      uint32_t tc = 0, cc = 0, ec = 0, kv_issued = 0, q_issued = 0, do_issued = 0;
+      for (;; ++tc) {
+        const uint32_t slot = tc & 1;
+        if (tc >= 2 && !wd.wait(&bars[L::bTkEmpty + slot], ((tc >> 1) - 1) & 1)) break;
+        const int t = static_cast<int>(atomicAdd(p.hdr + kHdrBwdTicket, 1u));
+        tk_ring[slot] = t < p.n_tickets ? t : -1;
+        mbar_arrive(&bars[L::bTkFull + slot]);
+        const Ticket k = decode_ticket(p, t);
+        if (!k.valid) break;
+        if (k.ee == k.es) continue;
+        bool stop = false;
+        for (int e = k.es; e < k.ee; ++e, ++ec) {
+          const int m = static_cast<int>(p.col_ent[e] & kIndexMask);
+          const uint32_t qs = ec % NQ, ds = ec % NDO;
+          if (ec >= NQ && !wd.wait(&bars[L::bQEmpty + qs], ((ec / NQ) - 1) & 1)) { stop = true; break; }
+          mbar_arrive_expect_tx(&bars[L::bQFull + qs], kTB);
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_4d(sm + L::kQ + qs * kTB + c * 16384, &tq, &bars[L::bQFull + qs], c * 64,
+                        m * kTile, k.h, k.b);
+          ++q_issued;
+          if (ec >= NDO && !wd.wait(&bars[L::bDOEmpty + ds], ((ec / NDO) - 1) & 1)) { stop = true; break; }
+          mbar_arrive_expect_tx(&bars[L::bDOFull + ds], kTB);
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_4d(sm + L::kDO + ds * kTB + c * 16384, &tdo, &bars[L::bDOFull + ds], c * 64,
+                        m * kTile, k.h, k.b);
+          ++do_issued;
+          if (e == k.es) {
+            // K_n, V_n after the first Q/dO so those loads overlap the previous
+            // column's last MMAs
+            if (cc >= 1 && !wd.wait(&bars[L::bKVFree], (cc - 1) & 1)) { stop = true; break; }
+            mbar_arrive_expect_tx(&bars[L::bKVFull], 2 * kTB);
+            for (int c = 0; c < D / 64; ++c) {
+              tma_load_4d(sm + L::kK + c * 16384, &tk, &bars[L::bKVFull], c * 64, k.n * kTile,
+                          k.h, k.b);
+              tma_load_4d(sm + L::kV + c * 16384, &tv, &bars[L::bKVFull], c * 64, k.n * kTile,
+                          k.h, k.b);
+            }
+            ++kv_issued;
+          }
+        }
+        if (stop) break;
+        ++cc;
+      }
+      if (wd.aborted()) {
+        for (uint32_t t = (q_issued > NQ ? q_issued - NQ : 0); t < q_issued; ++t)
+          drain_wait(&bars[L::bQFull + t % NQ], (t / NQ) & 1);
+        for (uint32_t t = (do_issued > NDO ? do_issued - NDO : 0); t < do_issued; ++t)
+          drain_wait(&bars[L::bDOFull + t % NDO], (t / NDO) & 1);
+        if (kv_issued > 0) drain_wait(&bars[L::bKVFull], (kv_issued - 1) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      uint32_t tc = 0, cc = 0, ec = 0;
+      for (;; ++tc) {
+        const uint32_t slot = tc & 1;
+        if (!wd.wait(&bars[L::bTkFull + slot], (tc >> 1) & 1)) break;
+        const int t = tk_ring[slot];
+        mbar_arrive(&bars[L::bTkEmpty + slot]);
+        const Ticket k = decode_ticket(p, t);
+        if (!k.valid) break;
+        if (k.ee == k.es) continue;
+        if (!wd.wait(&bars[L::bKVFull], cc & 1)) break;
+        tc_fence_after();
+        const uint32_t k_addr = smem_u32(sm + L::kK), v_addr = smem_u32(sm + L::kV);
+        const uint32_t ds_addr = smem_u32(sm + L::kDS);
+        bool stop = false;
+        for (int e = k.es; e < k.ee; ++e, ++ec) {
+          const uint32_t qs = ec % NQ, ds = ec % NDO;
+          const bool first = e == k.es, last = e == k.ee - 1;
+          if (!wd.wait(&bars[L::bQFull + qs], (ec / NQ) & 1)) { stop = true; break; }
+          if (ec >= 1 && !wd.wait(&bars[L::bDVDone], (ec - 1) & 1)) { stop = true; break; }
+          tc_fence_after();
+          const uint32_t q_addr = smem_u32(sm + L::kQ + qs * kTB);
+          const uint32_t do_addr = smem_u32(sm + L::kDO + ds * kTB);
+          // S^T = K_n Q_m^T
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+            mma_ss(T_S, sw128_desc(k_addr + off, 16, 1024), sw128_desc(q_addr + off, 16, 1024),
+                   kIdS, kk > 0);
+          }
+          if (!wd.wait(&bars[L::bDOFull + ds], (ec / NDO) & 1)) { stop = true; break; }
+          if (ec >= 1 && !wd.wait(&bars[L::bDQFree], (ec - 1) & 1)) { stop = true; break; }
+          tc_fence_after();
+          // dP^T = V_n dO_m^T
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+            mma_ss(T_DP, sw128_desc(v_addr + off, 16, 1024), sw128_desc(do_addr + off, 16, 1024),
+                   kIdS, kk > 0);
+          }
+          mma_commit(&bars[L::bSdPFull]);
+          if (!wd.wait(&bars[L::bPdSReady], ec & 1)) { stop = true; break; }
+          if (first && cc >= 1 && !wd.wait(&bars[L::bDKVFree], (cc - 1) & 1)) { stop = true; break; }
+          tc_fence_after();
+          // dV += P^T dO_m   (P^T from TMEM, dO as an MN-major B operand)
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts(T_DV, T_S + kk * 8, sw128_desc(do_addr + kk * 2048, 16384, 1024), kIdKV,
+                   (!first || kk > 0) ? 1u : 0u);
+          mma_commit(&bars[L::bDOEmpty + ds]);
+          mma_commit(&bars[L::bDVDone]);
+          // dK += dS^T Q_m
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+            mma_ss(T_DK, sw128_desc(ds_addr + off, 16, 1024),
+                   sw128_desc(q_addr + kk * 2048, 16384, 1024), kIdKV, (!first || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(&bars[L::bQEmpty + qs]);
+          // dQ_m part = dS K_n   (dS read MN-major from the dS^T tile)
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ss(T_DP, sw128_desc(ds_addr + kk * 2048, 16384, 1024),
+                   sw128_desc(k_addr + kk * 2048, 16384, 1024), kIdQ, kk > 0);
+          mma_commit(&bars[L::bDQFull]);
+          mma_commit(&bars[L::bDSFree]);
+          if (last) {
+            mma_commit(&bars[L::bDKVFull]);
+            mma_commit(&bars[L::bKVFree]);
+          }
+        }
+        if (stop) break;
+        ++cc;
+      }
+      mma_commit(&bars[L::bFinal]);
+      drain_wait(&bars[L::bFinal], 0);
+    }
+  } else if (warp >= 4 && warp < 8) {
+    // ------------------------------------------------------------ compute (key rows)
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const MaskParams &mk = p.mask;
+    const bool use_seg = mk.seg_q != nullptr;
+    auto wwait = [&](uint64_t *bar, uint32_t parity) {
+      return __all_sync(0xffffffffu, wd.wait(bar, parity)) != 0;
+    };
+    uint32_t tc = 0, cc = 0, ec = 0;
+    bool stop = false;
+    for (;; ++tc) {
+      const uint32_t slot = tc & 1;
+      if (!wwait(&bars[L::bTkFull + slot], (tc >> 1) & 1)) break;
+      const int t = tk_ring[slot];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[L::bTkEmpty + slot]);
+      const Ticket k = decode_ticket(p, t);
+      if (!k.valid) break;
+      const int j = k.n * kTile + r;
+      const bool row_ok = j < p.Skv;
+      __nv_bfloat16 *dk_row = p.dk + k.b * p.k_sb + static_cast<int64_t>(j) * p.k_ss + k.h * p.k_sh;
+      __nv_bfloat16 *dv_row = p.dv + k.b * p.v_sb + static_cast<int64_t>(j) * p.v_ss + k.h * p.v_sh;
+      if (k.ee == k.es) {
+        if (row_ok) {
+          const int4 z = make_int4(0, 0, 0, 0);
+#pragma unroll
+          for (int c = 0; c < D / 8; ++c) {
+            reinterpret_cast<int4 *>(dk_row)[c] = z;
+            reinterpret_cast<int4 *>(dv_row)[c] = z;
+          }
+        }
+        continue;
+      }
+      // queries this key may be seen by: [qlo, qhi]
+      int qlo = 0, qhi = p.Sq - 1;
+      if (!row_ok) qhi = -1;
+      if (mk.flags & BSA_MASK_CAUSAL_WINDOW) {
+        qlo = max(qlo, j - mk.offset);
+        if (mk.window > 0) qhi = min(qhi, j - mk.offset + mk.window - 1);
+      }
+      if ((mk.flags & BSA_MASK_KV_VALID_LEN) && j >= mk.kv_valid_len[k.b]) qhi = -1;
+      const int seg_j = (use_seg && row_ok) ? mk.seg_kv[static_cast<int64_t>(k.b) * p.Skv + j] : INT_MIN;
+      uint8_t *ds_tile = sm + L::kDS;
+      for (int e = k.es; e < k.ee; ++e, ++ec) {
+        const uint32_t ent = p.col_ent[e];
+        const int m = static_cast<int>(ent & kIndexMask);
+        const bool full = (ent & kFullBit) != 0;
+        // stage LSE (log2 units; +inf where the row has no key or lies past Sq),
+        // Delta and the query segment ids of this q-block
+        {
+          const int i = m * kTile + r;
+          float* vl = vec_lse + (ec & 1) * kTile;
+          float* vd = vec_delta + (ec & 1) * kTile;
+          int32_t* vs = vec_seg + (ec & 1) * kTile;
+          float l2 = INFINITY;
+          if (i < p.Sq) {
+            const float lv = p.lse[static_cast<int64_t>(k.bh) * p.Sq + i];
+            if (lv != -INFINITY) l2 = lv * kLog2e;
+          }
+          vl[r] = l2;
+          vd[r] = p.delta[static_cast<int64_t>(k.bh) * p.nM * kTile + i];
+          if (use_seg) vs[r] = i < p.Sq ? mk.seg_q[static_cast<int64_t>(k.b) * p.Sq + i] : INT_MIN + 1;
+          mbar_arrive(&bars[L::bVecReady + (ec & 1)]);
+        }
+        if (!wwait(&bars[L::bVecReady + (ec & 1)], (ec >> 1) & 1)) { stop = true; break; }
+        const float *vl = vec_lse + (ec & 1) * kTile;
+        const float *vd = vec_delta + (ec & 1) * kTile;
+        uint32_t seg_ok[4] = {~0u, ~0u, ~0u, ~0u};
+        if (!full && use_seg) {
+          const int4 *seg4 = reinterpret_cast<const int4 *>(vec_seg + (ec & 1) * kTile);
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+            uint32_t bits = 0;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              const int4 v = seg4[w * 8 + q];
+              bits |= (static_cast<uint32_t>(v.x == seg_j) << (4 * q)) |
+                      (static_cast<uint32_t>(v.y == seg_j) << (4 * q + 1)) |
+                      (static_cast<uint32_t>(v.z == seg_j) << (4 * q + 2)) |
+                      (static_cast<uint32_t>(v.w == seg_j) << (4 * q + 3));
+            }
+            seg_ok[w] = bits;
+          }
+        }
+        const int c_lo = qlo - m * kTile, c_hi = qhi - m * kTile;
+        if (!wwait(&bars[L::bSdPFull], ec & 1)) { stop = true; break; }
+        if (ec >= 1 && !wwait(&bars[L::bDSFree], (ec - 1) & 1)) { stop = true; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t s[32], dp[32];
+          tmem_ld32(T_S + lane_off + 32 * c, s);
+          tmem_ld32(T_DP + lane_off + 32 * c, dp);
+          tmem_wait_ld();
+          uint32_t pk[16], dk2[16];
+#pragma unroll
+          for (int q = 0; q < 16; ++q) {
+            float pr[2], dsv[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+              const int col = 32 * c + 2 * q + u;
+              float pv = fast_exp2(fmaf(__uint_as_float(s[2 * q + u]), p.scale_log2, -vl[col]));
+              if (!full) {
+                const bool ok = col >= c_lo && col <= c_hi && ((seg_ok[col >> 5] >> (col & 31)) & 1u);
+                pv = ok ? pv : 0.f;
+              }
+              pr[u] = pv;
+              dsv[u] = pv * (__uint_as_float(dp[2 * q + u]) - vd[col]);
+            }
+            pk[q] = pack_bf16x2(pr[0], pr[1]);
+            dk2[q] = pack_bf16x2(dsv[0], dsv[1]);
+          }
+          // P^T chunk -> TMEM columns [16c, 16c+16) of the S^T region
+          tmem_st16(T_S + lane_off + 16 * c, pk);
+          // dS^T chunk -> shared tile, row r, 16-byte chunks 4c..4c+3 (128-byte swizzle)
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int chunk = 4 * c + u;  // 0..15 over 128 queries
+            const int sub = chunk >> 3, cw = chunk & 7;
+            uint8_t *dst = ds_tile + sub * 16384 + r * 128 + ((cw ^ (r & 7)) << 4);
+            *reinterpret_cast<int4 *>(dst) =
+                make_int4(dk2[4 * u], dk2[4 * u + 1], dk2[4 * u + 2], dk2[4 * u + 3]);
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        fence_proxy_async_smem();
+        mbar_arrive(&bars[L::bPdSReady]);
+      }
+      if (stop) break;
+      // epilogue: dV, dK (scaled) -> bf16
+      if (!wwait(&bars[L::bDKVFull], cc & 1)) break;
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t a[32], g[32];
+        tmem_ld32(T_DV + lane_off + 32 * c, a);
+        tmem_ld32(T_DK + lane_off + 32 * c, g);
+        tmem_wait_ld();
+        if (row_ok) {
+          uint32_t wv[16], wk[16];
+#pragma unroll
+          for (int q = 0; q < 16; ++q) {
+            wv[q] = pack_bf16x2(__uint_as_float(a[2 * q]), __uint_as_float(a[2 * q + 1]));
+            wk[q] = pack_bf16x2(__uint_as_float(g[2 * q]) * p.scale,
+                                __uint_as_float(g[2 * q + 1]) * p.scale);
+          }
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            reinterpret_cast<int4 *>(dv_row + 32 * c)[q] =
+                make_int4(wv[4 * q], wv[4 * q + 1], wv[4 * q + 2], wv[4 * q + 3]);
+            reinterpret_cast<int4 *>(dk_row + 32 * c)[q] =
+                make_int4(wk[4 * q], wk[4 * q + 1], wk[4 * q + 2], wk[4 * q + 3]);
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&bars[L::bDKVFree]);
+      ++cc;
+    }
+  } else if (warp >= 8) {
+    // ------------------------------------------------------------ dQ (query rows)
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    auto wwait = [&](uint64_t *bar, uint32_t parity) {
+      return __all_sync(0xffffffffu, wd.wait(bar, parity)) != 0;
+    };
+    uint32_t tc = 0, ec = 0;
+    for (;; ++tc) {
+      const uint32_t slot = tc & 1;
+      if (!wwait(&bars[L::bTkFull + slot], (tc >> 1) & 1)) break;
+      const int t = tk_ring[slot];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[L::bTkEmpty + slot]);
+      const Ticket k = decode_ticket(p, t);
+      if (!k.valid) break;
+      bool stop = false;
+      for (int e = k.es; e < k.ee; ++e, ++ec) {
+        const int m = static_cast<int>(p.col_ent[e] & kIndexMask);
+        const uint32_t rank = static_cast<uint32_t>(p.col_rank[e]);
+        if (!wwait(&bars[L::bDQFull], ec & 1)) { stop = true; break; }
+        tc_fence_after();
+        float acc[D];
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t a[32];
+          tmem_ld32(T_DP + lane_off + 32 * c, a);
+          tmem_wait_ld();
+#pragma unroll
+          for (int q = 0; q < 32; ++q) acc[32 * c + q] = __uint_as_float(a[q]) * p.scale;
+        }
+        tc_fence_before();
+        mbar_arrive(&bars[L::bDQFree]);
+        uint32_t *sem = p.sem + static_cast<int64_t>(k.bh) * p.nM + m;
+        int ok = 1;
+        if (p.deterministic) {
+          if (lane == 0) ok = sem_wait(sem, rank, p.sem_timeout_ns, p.hdr + kHdrStatus) ? 1 : 0;
+          ok = __shfl_sync(0xffffffffu, ok, 0);
+        }
+        if (ok) {
+          float *base = p.dq_accum + (static_cast<int64_t>(k.bh) * p.nM + m) * (D / 4) * (kTile * 4);
+#pragma unroll
+          for (int c = 0; c < D / 4; ++c)
+            red_add_v4(base + (static_cast<int64_t>(c) * kTile + r) * 4, acc[4 * c], acc[4 * c + 1],
+                       acc[4 * c + 2], acc[4 * c + 3]);
+        }
+        if (p.deterministic) {
+          __threadfence();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars[L::bDQAdded + (ec & 1)]);
+          if (warp == 8 && lane == 0) {
+            // the last of the four warps' adds is visible: pass the turn on
+            if (wd.wait(&bars[L::bDQAdded + (ec & 1)], (ec >> 1) & 1)) {
+              __threadfence();
+              red_release_gpu_add(sem, 1u);
+            }
+          }
+          __syncwarp();
+        }
+      }
+      if (stop) break;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------- a4: Delta
+template <int D>
+__global__ void __launch_bounds__(256) k_bwd_delta(const __nv_bfloat16 *__restrict__ o,
+                                                   const __nv_bfloat16 *__restrict__ dout,
+                                                   int64_t sb, int64_t ss, int64_t sh, int B,
+                                                   int Sq, int H, int rows_pad,
+                                                   float *__restrict__ delta) {
+  constexpr int TPV = D / 8;
+  const int64_t g = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) / TPV;
+  const int t = threadIdx.x % TPV;
+  const int64_t total = static_cast<int64_t>(B) * H * rows_pad;
+  const bool in = g < total;  // no early return: the shuffles below need every lane
+  const int i = static_cast<int>(g % rows_pad);
+  const int bh = static_cast<int>(g / rows_pad);
+  const int b = bh / H, h = bh % H;
+  float acc = 0.f;
+  if (in && i < Sq) {
+    const int64_t off = b * sb + static_cast<int64_t>(i) * ss + h * sh + t * 8;
+    const int4 a = *reinterpret_cast<const int4 *>(o + off);
+    const int4 c = *reinterpret_cast<const int4 *>(dout + off);
+    const __nv_bfloat162 *x = reinterpret_cast<const __nv_bfloat162 *>(&a);
+    const __nv_bfloat162 *y = reinterpret_cast<const __nv_bfloat162 *>(&c);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float2 fx = __bfloat1622float2(x[q]), fy = __bfloat1622float2(y[q]);
+      acc = fmaf(fx.x, fy.x, acc);
+      acc = fmaf(fx.y, fy.y, acc);
+    }
+  }
+#pragma unroll
+  for (int s = TPV / 2; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
+  if (t == 0 && in) delta[g] = acc;
+}
+
+// ---------------------------------------------------------------- a7: dQ convert
+template <int D>
+__global__ void __launch_bounds__(256) k_dq_convert(const float *__restrict__ acc, int B, int H,
+                                                    int Sq, int nM, __nv_bfloat16 *__restrict__ dq,
+                                                    int64_t sb, int64_t ss, int64_t sh) {
+  extern __shared__ float tile[];  // [128][D + 4]
+  constexpr int LD = D + 4;
+  const int bhm = blockIdx.x;
+  const int m = bhm % nM, bh = bhm / nM, b = bh / H, h = bh % H;
+  const float *src = acc + static_cast<int64_t>(bhm) * (D / 4) * kTile * 4;
+  for (int idx = threadIdx.x; idx < (D / 4) * kTile; idx += blockDim.x) {
+    const int c = idx / kTile, r = idx % kTile;
+    const float4 v = reinterpret_cast<const float4 *>(src)[idx];
+    float *d = tile + r * LD + 4 * c;
+    d[0] = v.x;
+    d[1] = v.y;
+    d[2] = v.z;
+    d[3] = v.w;
+  }
+  __syncthreads();
+  constexpr int CPR = D / 8;  // 16-byte chunks per row
+  for (int idx = threadIdx.x; idx < kTile * CPR; idx += blockDim.x) {
+    const int r = idx / CPR, c = idx % CPR;
+    const int i = m * kTile + r;
+    if (i >= Sq) continue;
+    const float *s = tile + r * LD + 8 * c;
+    const int4 w = make_int4(pack_bf16x2(s[0], s[1]), pack_bf16x2(s[2], s[3]),
+                             pack_bf16x2(s[4], s[5]), pack_bf16x2(s[6], s[7]));
+    *reinterpret_cast<int4 *>(dq + b * sb + static_cast<int64_t>(i) * ss + h * sh + 8 * c) = w;
+  }
+}
+
+int sm_count_bwd() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+template <int D, int NQ, int NDO>
+cudaError_t run_bwd_main(const BwdParams &bp, const CUtensorMap &tq, const CUtensorMap &tk,
+                         const CUtensorMap &tv, const CUtensorMap &tdo, cudaStream_t s) {
+  using L = BwdSmem<D, NQ, NDO>;
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(k_attn_bwd<D, NQ, NDO>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  const int grid = std::max(1, std::min(bp.n_tickets, sm_count_bwd()));
+  k_attn_bwd<D, NQ, NDO><<<grid, 384, L::kAlloc, s>>>(tq, tk, tv, tdo, bp);
+  count_launch();
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t run_bwd(const bsa_problem &p, const BwdParams &bp, const void *out, const void *dout,
+                    void *dq, const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                    const CUtensorMap &tdo, cudaStream_t s) {
+  const int rows_pad = bp.nM * kTile;
+  const int64_t groups = static_cast<int64_t>(p.B) * p.H * rows_pad;
+  const int64_t threads = groups * (D / 8);
+  k_bwd_delta<D><<<static_cast<unsigned>((threads + 255) / 256), 256, 0, s>>>(
+      static_cast<const __nv_bfloat16 *>(out), static_cast<const __nv_bfloat16 *>(dout),
+      p.o_stride[0], p.o_stride[1], p.o_stride[2], p.B, p.Sq, p.H, rows_pad,
+      const_cast<float *>(bp.delta));
+  count_launch();
+  cudaError_t e = cudaMemsetAsync(bp.dq_accum, 0,
+                                  sizeof(float) * static_cast<size_t>(groups) * D, s);
+  if (e != cudaSuccess) return e;
+  e = cudaMemsetAsync(bp.sem, 0, sizeof(uint32_t) * static_cast<size_t>(p.B) * p.H * bp.nM, s);
+  if (e != cudaSuccess) return e;
+  e = cudaMemsetAsync(bp.hdr + kHdrBwdTicket, 0, sizeof(uint32_t), s);
+  if (e != cudaSuccess) return e;
+  e = (D == 64) ? run_bwd_main<64, 2, 2>(bp, tq, tk, tv, tdo, s)
+                : run_bwd_main<128, 2, 1>(bp, tq, tk, tv, tdo, s);
+  if (e != cudaSuccess) return e;
+  const size_t smem = sizeof(float) * kTile * (D + 4);
+  static bool attr = false;
+  if (!attr) {
+    e = cudaFuncSetAttribute(k_dq_convert<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  k_dq_convert<D><<<p.B * p.H * bp.nM, 256, smem, s>>>(bp.dq_accum, p.B, p.H, p.Sq, bp.nM,
+                                                       static_cast<__nv_bfloat16 *>(dq),
+                                                       p.q_stride[0], p.q_stride[1], p.q_stride[2]);
+  count_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_bwd(const bsa_problem &p, const MaskParams &mp, const bsa_options &o,
+                       const PlanSignature &sig, const CUtensorMap &tq, const CUtensorMap &tk,
+                       const CUtensorMap &tv, const CUtensorMap &tdo, const void *out,
+                       const void *dout, const float *lse, void *dq, void *dk, void *dv,
+                       const WsLayout &L, uint8_t *ws, cudaStream_t s) {
+  BwdParams bp{};
+  bp.mask = mp;
+  bp.B = p.B;
+  bp.H = p.H;
+  bp.Sq = p.Sq;
+  bp.Skv = p.Skv;
+  bp.nM = L.nM;
+  bp.nN = L.nN;
+  bp.n_tickets = p.B * p.H * L.nN;
+  bp.scale = p.scale;
+  bp.scale_log2 = p.scale * kLog2e;
+  bp.col_ptr = reinterpret_cast<const int32_t *>(ws + L.col_ptr);
+  bp.col_ent = reinterpret_cast<const uint32_t *>(ws + L.col_ent);
+  bp.col_rank = reinterpret_cast<const int32_t *>(ws + L.col_rank);
+  bp.perm = reinterpret_cast<const int32_t *>(ws + L.perm);
+  bp.lse = lse;
+  bp.delta = reinterpret_cast<const float *>(ws + L.delta);
+  bp.dq_accum = reinterpret_cast<float *>(ws + L.dq_accum);
+  bp.sem = reinterpret_cast<uint32_t *>(ws + L.sem);
+  bp.dk = static_cast<__nv_bfloat16 *>(dk);
+  bp.dv = static_cast<__nv_bfloat16 *>(dv);
+  bp.k_sb = p.k_stride[0];
+  bp.k_ss = p.k_stride[1];
+  bp.k_sh = p.k_stride[2];
+  bp.v_sb = p.v_stride[0];
+  bp.v_ss = p.v_stride[1];
+  bp.v_sh = p.v_stride[2];
+  bp.deterministic = o.deterministic ? 1 : 0;
+  bp.hdr = reinterpret_cast<uint32_t *>(ws + L.status);
+  bp.timeout_ns = 2000000000ull;
+  bp.sem_timeout_ns = o.sem_timeout_ns > 0 ? static_cast<uint64_t>(o.sem_timeout_ns) : 1000000000ull;
+  for (int i = 0; i < 7; ++i) bp.sig[i] = sig.w[i];
+  bp.sig_mask = 0x7Fu;
+  if (p.D == 64) return run_bwd<64>(p, bp, out, dout, dq, tq, tk, tv, tdo, s);
+  return run_bwd<128>(p, bp, out, dout, dq, tq, tk, tv, tdo, s);
+}
+
 }  // namespace bsa

@@ -372,8 +372,10 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
           for (int c = 0; c < 32; ++c) {
             const float p0 = fast_exp2(fmaf(f[64 * half + 2 * c], p.scale_log2, -mu));
             const float p1 = fast_exp2(fmaf(f[64 * half + 2 * c + 1], p.scale_log2, -mu));
-            rowsum += p0 + p1;
             pk[c] = pack_bf16x2(p0, p1);
+            // l sums the bf16-rounded weights the PV product actually uses, so
+            // numerator and denominator carry the same rounding
+            rowsum += __uint_as_float(pk[c] << 16) + __uint_as_float(pk[c] & 0xffff0000u);
           }
           // P (bf16 pairs) overwrites the first 64 columns of this S buffer
           tmem_st32(t_s + 32 * half, pk);
@@ -441,10 +443,13 @@ __global__ void __launch_bounds__(256) k_row_norms(const __nv_bfloat16 *__restri
   const int r0 = static_cast<int>(blockIdx.x % blocks_per_b) * kRows;
   const int g = threadIdx.x / TPV, t = threadIdx.x % TPV;
   const int groups = blockDim.x / TPV;
-  for (int pair = g; pair < kRows * H; pair += groups) {
+  // uniform trip count across the warp: the shuffles below need every lane
+  for (int base = 0; base < kRows * H; base += groups) {
+    const int pair = base + g;
     const int row = r0 + pair / H, h = pair % H;
+    const bool in = pair < kRows * H && row < S;
     float acc = 0.f;
-    if (row < S) {
+    if (in) {
       const int4 v = *reinterpret_cast<const int4 *>(x + b * sb + static_cast<int64_t>(row) * ss +
                                                     h * sh + t * 8);
       const __nv_bfloat162 *e = reinterpret_cast<const __nv_bfloat162 *>(&v);
@@ -457,7 +462,7 @@ __global__ void __launch_bounds__(256) k_row_norms(const __nv_bfloat16 *__restri
     }
 #pragma unroll
     for (int o = TPV / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if (t == 0 && row < S) {
+    if (t == 0 && in) {
       const float nrm = sqrtf(acc);
       bool valid = true;
       if (is_key) {

@@ -1,0 +1,149 @@
+"""GPU parity of the backward (Delta, deterministic semaphore-ordered dQ, dK/dV)
+against the oracle's analytic gradient, run-to-run bit identity, the
+non-deterministic variant, and the bounded semaphore wait."""
+
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_attention_map_b200 as bsa
+import oracle
+from block_sparse_attention_map_b200.workloads import make_workload
+from tests.gpu_common import O_TOL, mask_desc, np64
+
+pytestmark = pytest.mark.gpu
+
+
+def _grads(wl, **kw):
+    o, lse, ws = bsa.attn_fwd(wl.q, wl.k, wl.v, wl.mask)
+    dq, dk, dv, wsb = bsa.attn_bwd(wl.q, wl.k, wl.v, o, wl.dO, lse, wl.mask, **kw)
+    torch.cuda.synchronize()
+    return o, lse, dq, dk, dv, wsb
+
+
+def _oracle_grads(wl, heads=None):
+    q, k, v, do = np64(wl.q), np64(wl.k), np64(wl.v), np64(wl.dO)
+    if heads is not None:
+        q, k, v, do = q[:, :, heads], k[:, :, heads], v[:, :, heads], do[:, :, heads]
+    return oracle.attention_backward(q, k, v, do, mask_desc(wl), wl.scale)
+
+
+def _err(x, ref):
+    return float(np.max(np.abs(np64(x) - ref)))
+
+
+SMALL = ["tiny", "packed", "window", "window_rect", "varlen", "video"]
+
+
+@pytest.mark.parametrize("name", SMALL)
+def test_bwd_matches_oracle(name):
+    wl = make_workload(name, device="cuda", small=True)
+    if wl.dO is None:
+        g = torch.Generator(device="cuda")
+        g.manual_seed(99)
+        wl.dO = torch.randn(wl.q.shape, device="cuda", generator=g).bfloat16()
+    _, _, dq, dk, dv, ws = _grads(wl)
+    assert ws.status() == 0
+    gq, gk, gv = _oracle_grads(wl)
+    e = (_err(dq, gq), _err(dk, gk), _err(dv, gv))
+    assert max(e) <= O_TOL, e
+
+
+@pytest.mark.parametrize("order", ["asc", "desc", "perm"])
+def test_bwd_orders_match_oracle_and_repeat_bitwise(order):
+    wl = make_workload("window", device="cuda", small=True)
+    nN = -(-wl.Skv // 128)
+    perm = np.random.default_rng(3).permutation(nN) if order == "perm" else None
+    o, lse, dq, dk, dv, ws = _grads(wl, order=order, perm=perm)
+    assert ws.status() == 0
+    gq, gk, gv = _oracle_grads(wl)
+    assert max(_err(dq, gq), _err(dk, gk), _err(dv, gv)) <= O_TOL
+    for _ in range(9):
+        dq2, dk2, dv2, ws2 = bsa.attn_bwd(wl.q, wl.k, wl.v, o, wl.dO, lse, wl.mask, order=order, perm=perm)
+        torch.cuda.synchronize()
+        assert torch.equal(dq, dq2) and torch.equal(dk, dk2) and torch.equal(dv, dv2)
+
+
+def test_bwd_nondeterministic_matches_oracle():
+    wl = make_workload("packed", device="cuda", small=True)
+    _, _, dq, dk, dv, ws = _grads(wl, deterministic=False)
+    assert ws.status() == 0
+    gq, gk, gv = _oracle_grads(wl)
+    assert max(_err(dq, gq), _err(dk, gk), _err(dv, gv)) <= O_TOL
+
+
+def test_bwd_constant_segment_ids_bitwise_equal_no_mask():
+    wl = make_workload("packed_const", device="cuda", small=True)
+    o, lse, ws = bsa.attn_fwd(wl.q, wl.k, wl.v, wl.mask)
+    a = bsa.attn_bwd(wl.q, wl.k, wl.v, o, wl.dO, lse, wl.mask)
+    b = bsa.attn_bwd(wl.q, wl.k, wl.v, o, wl.dO, lse, None)
+    torch.cuda.synchronize()
+    for x, y in zip(a[:3], b[:3]):
+        assert torch.equal(x, y)
+
+
+def test_bwd_ragged_and_d64():
+    g = torch.Generator(device="cuda")
+    g.manual_seed(21)
+    for (Sq, Skv, D, W) in [(77, 300, 64, 0), (300, 77, 128, 40), (129, 257, 128, None), (1, 1, 64, None)]:
+        q = torch.randn(2, Sq, 3, D, device="cuda", generator=g).bfloat16()
+        k = torch.randn(2, Skv, 3, D, device="cuda", generator=g).bfloat16()
+        v = torch.randn(2, Skv, 3, D, device="cuda", generator=g).bfloat16()
+        do = torch.randn(2, Sq, 3, D, device="cuda", generator=g).bfloat16()
+        mask = {"window": W} if W is not None else {}
+        o, lse, _ = bsa.attn_fwd(q, k, v, mask)
+        dq, dk, dv, ws = bsa.attn_bwd(q, k, v, o, do, lse, mask)
+        torch.cuda.synchronize()
+        assert ws.status() == 0
+        gq, gk, gv = oracle.attention_backward(np64(q), np64(k), np64(v), np64(do),
+                                               oracle.MaskDesc(**mask), 1 / D ** 0.5)
+        assert max(_err(dq, gq), _err(dk, gk), _err(dv, gv)) <= O_TOL, (Sq, Skv, D, W)
+
+
+@pytest.mark.parametrize("name", ["window", "window_rect"])
+def test_bwd_full_size_one_head_and_ten_run_identity(name):
+    wl = make_workload(name, device="cuda")
+    o, lse, ws = bsa.attn_fwd(wl.q, wl.k, wl.v, wl.mask)
+    ref = None
+    for it in range(10):
+        dq, dk, dv, wsb = bsa.attn_bwd(wl.q, wl.k, wl.v, o, wl.dO, lse, wl.mask, order="asc")
+        torch.cuda.synchronize()
+        if ref is None:
+            ref = (dq.clone(), dk.clone(), dv.clone())
+            assert wsb.status() == 0
+        else:
+            assert all(torch.equal(x, y) for x, y in zip(ref, (dq, dk, dv)))
+    gq, gk, gv = _oracle_grads(wl, heads=[0])
+    assert _err(ref[0][:, :, [0]], gq) <= O_TOL
+    assert _err(ref[1][:, :, [0]], gk) <= O_TOL
+    assert _err(ref[2][:, :, [0]], gv) <= O_TOL
+
+
+def test_semaphore_wait_is_bounded_and_reported():
+    # Corrupt one rank in the caller-owned plan so that its dQ wait can never be
+    # satisfied: the wait gives up after the bound, the status word says so and
+    # the context stays usable.
+    wl = make_workload("window", device="cuda", small=True)
+    o, lse, _ = bsa.attn_fwd(wl.q, wl.k, wl.v, wl.mask)
+    ws = bsa.plan_build(wl.q, wl.k, wl.v, wl.mask, backward=True)
+    torch.cuda.synchronize()
+    off = ws.view.off_col_rank
+    ranks = ws.buf[off:off + 4 * 8].view(torch.int32)
+    ranks[3] = 1000
+    dq, dk, dv, _ = bsa.attn_bwd(wl.q, wl.k, wl.v, o, wl.dO, lse, wl.mask, workspace=ws,
+                                 plan_ready=True, sem_timeout_ns=50_000_000)
+    torch.cuda.synchronize()
+    assert ws.status(clear=True) == 5  # BSA_ERR_SEM_TIMEOUT
+    # the device is still healthy: a clean run afterwards succeeds
+    _, _, dq2, dk2, dv2, ws2 = _grads(wl)
+    assert ws2.status() == 0
+    gq, gk, gv = _oracle_grads(wl)
+    assert max(_err(dq2, gq), _err(dk2, gk), _err(dv2, gv)) <= O_TOL
+
+
+def test_plan_mismatch_is_reported():
+    wl = make_workload("window", device="cuda", small=True)
+    ws = bsa.plan_build(wl.q, wl.k, wl.v, {"window": 7})
+    o, lse, _ = bsa.attn_fwd(wl.q, wl.k, wl.v, wl.mask, workspace=ws, plan_ready=True)
+    torch.cuda.synchronize()
+    assert ws.status(clear=True) == 6  # BSA_ERR_PLAN_MISMATCH
