@@ -1,0 +1,428 @@
+#!/usr/bin/env python
+"""Throughput of the block-sparse attention hot path on B200.
+
+One step = the whole hot path over the causal sliding-window workload
+(B=1, H=16, Sq=Skv=8192, D=128, window 512, bf16 N(0,1), seed 2):
+  a1+a6  block map + rank-sorted column lists      (bsa_plan_build)
+  a2     fixed-m bound and per-head gate            (bsa_fixed_m_bound)
+  a3     forward, fixed-m gated                     (bsa_attn_fwd)
+  a4     Delta, zeroed dQ accumulator / semaphores  (bsa_bwd_preprocess)
+  a5     deterministic backward, ascending order    (bsa_bwd_main)
+  a7     dQ convert                                 (bsa_bwd_convert)
+Metric: useful TFLOP/s = (non-empty 128x128 tiles x per-tile flops) / time, with
+per-tile flops 4*128*128*D forward and 2.5x that backward.  L2 is flushed
+(a 256 MiB write) before every step, outside the step's events.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 it runs under torch.distributed.run, one rank per GPU, every rank
+running the same workload (replicas: the (b, h) units are independent and
+the path has no exchange step); value = work of all ranks / max rank time.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD_NAME = "window"
+WORKLOAD_TEXT = ("causal sliding window 512: B=1, H=16, Sq=Skv=8192, D=128, bf16 N(0,1) seed 2; "
+                 "forward fixed-m gated + deterministic backward (ascending kv-column order)")
+METRIC = "attention TFLOP/s (non-empty tiles) fwd+bwd on 1 B200; % of bf16 tensor peak"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--softmax", default="fixed_m", choices=["fixed_m", "online"])
+    ap.add_argument("--order", default="asc", choices=["asc", "desc"])
+    ap.add_argument("--small", action="store_true",
+                    help="small shape of the same workload (for profiler captures)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+def profiled_traffic(kernel: str, workload: str):
+    """dram bytes per launch of `kernel` on `workload` from the committed ncu
+    summary (a line `traffic <kernel> <workload> <bytes>`), else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    try:
+        for line in open(path):
+            parts = line.split()
+            if len(parts) == 4 and parts[0] == "traffic" and parts[1] == kernel and parts[2] == workload:
+                return float(parts[3])
+    except OSError:
+        pass
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+        return False
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in getattr(self, "lines", []):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        loaded = [s for s in sm if s > 0.5 * max(sm)] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup(args):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    import torch
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+def tiles_of(ws):
+    ptr, _ = ws.row_lists()
+    return int(ptr[-1])
+
+
+# ------------------------------------------------------------------ CPU oracle leg
+
+def oracle_sample(wl, n_rows: int, head: int = 0):
+    """Time the fp64 oracle (forward + backward) on query rows [0, n_rows) of one
+    head against all keys; returns (seconds, useful flops credited, threads)."""
+    import numpy as np
+    import oracle
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [os.cpu_count()])
+    except Exception:
+        threads = os.cpu_count()
+    f = lambda t: t.detach().float().cpu().numpy().astype(np.float64)
+    q = f(wl.q[:, :n_rows, head:head + 1])
+    k, v = f(wl.k[:, :, head:head + 1]), f(wl.v[:, :, head:head + 1])
+    do = f(wl.dO[:, :n_rows, head:head + 1])
+    mask = oracle.MaskDesc(**wl.mask_numpy())
+    # the sample treats rows [0, n_rows) as the query set: the window's bottom-right
+    # offset must stay that of the full problem, so use Sq=Skv rows and a square cut
+    sub = oracle.MaskDesc(window=mask.window) if mask.window is not None else mask
+    cls = oracle.tile_classes(sub, 1, n_rows, n_rows)
+    t0 = time.perf_counter()
+    oracle.attention_forward(q, k[:, :n_rows], v[:, :n_rows], sub, wl.scale)
+    oracle.attention_backward(q, k[:, :n_rows], v[:, :n_rows], do, sub, wl.scale)
+    dt = time.perf_counter() - t0
+    nnz = int((cls != oracle.EMPTY).sum())
+    flops = oracle.useful_flops(nnz, wl.D) * 3.5
+    return dt, flops, threads
+
+
+def run_reference(args, world, rank):
+    """The reference arm: the fp64 oracle, as it stands, on the host cores."""
+    import torch
+    from block_sparse_attention_map_b200.workloads import make_workload
+    if rank != 0:
+        return
+    wl = make_workload(WORKLOAD_NAME, device="cpu", small=args.small)
+    n_rows = min(1024, wl.Sq)
+    for _ in range(args.warmup):
+        oracle_sample(wl, n_rows)
+    total_t, total_f, threads = 0.0, 0.0, 1
+    for _ in range(args.steps):
+        dt, fl, threads = oracle_sample(wl, n_rows)
+        total_t += dt
+        total_f += fl
+    value = total_f / total_t / 1e12
+    sample = (f"rows 0..{n_rows - 1} of head 0 of {wl.H} (one causal band of {n_rows} keys), "
+              f"forward + backward in fp64, per step")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total_t / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD_TEXT, "global_batch": wl.B, "seq_len": wl.Sq,
+                   "heads": wl.H, "head_dim": wl.D, "window": 512},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ GPU arm
+
+def run_ours(args, world, rank, local):
+    import torch
+    import block_sparse_attention_map_b200 as bsa
+    from block_sparse_attention_map_b200.workloads import make_workload
+
+    dev = torch.device("cuda", local)
+    wl = make_workload(WORKLOAD_NAME, device=dev, small=args.small)
+    st = bsa.Stages(wl.q, wl.k, wl.v, wl.mask, softmax_mode=args.softmax, order=args.order)
+    dO = wl.dO
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+    names = ["plan", "bound", "forward", "preprocess", "backward_main", "convert"]
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        st.plan()
+        if ev is not None:
+            ev[1].record(stream)
+        st.bound()
+        if ev is not None:
+            ev[2].record(stream)
+        st.forward()
+        if ev is not None:
+            ev[3].record(stream)
+        st.preprocess(dO)
+        if ev is not None:
+            ev[4].record(stream)
+        st.backward_main(dO)
+        if ev is not None:
+            ev[5].record(stream)
+        st.convert()
+        if ev is not None:
+            ev[6].record(stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    status = st.ws.status()
+    if status != 0:
+        raise RuntimeError(f"device status {status} after warm-up")
+    n_tiles = tiles_of(st.ws) * wl.H  # non-empty tiles over all (b, h)
+    f_fwd = 4.0 * 128 * 128 * wl.D * n_tiles
+    f_bwd = 2.5 * f_fwd
+
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
+    launches0 = bsa.launch_count()
+    barrier(world)
+    with ClockSampler(local) as clk:
+        t_wall = time.perf_counter()
+        for s in range(args.steps):
+            flush.zero_()
+            step(events[s])
+        torch.cuda.synchronize()
+        t_wall = time.perf_counter() - t_wall
+    barrier(world)
+    launches = bsa.launch_count() - launches0
+    status = st.ws.status()
+    if status != 0:
+        raise RuntimeError(f"device status {status} after the timed steps")
+
+    stage_ms = {n: 0.0 for n in names}
+    step_ms = []
+    for ev in events:
+        for i, n in enumerate(names):
+            stage_ms[n] += ev[i].elapsed_time(ev[i + 1])
+        step_ms.append(ev[0].elapsed_time(ev[6]))
+    total_ms = max_over_ranks(sum(step_ms), world)
+    ms_step = total_ms / args.steps
+    value = world * args.steps * (f_fwd + f_bwd) / (total_ms * 1e-3) / 1e12
+    avg = {n: stage_ms[n] / args.steps for n in names}
+
+    peaks = load_peaks()
+    peak = peaks["bf16_tflops"]
+    main_tf = f_bwd / (avg["backward_main"] * 1e-3) / 1e12
+    fwd_tf = f_fwd / (avg["forward"] * 1e-3) / 1e12
+    traffic = profiled_traffic("k_attn_bwd", "window8192")
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD_TEXT + (" [small shape]" if args.small else ""),
+                   "global_batch": wl.B * world, "seq_len": wl.Sq, "heads": wl.H,
+                   "head_dim": wl.D, "window": 512, "nonempty_tiles": n_tiles,
+                   "softmax": args.softmax, "bwd_order": args.order,
+                   "l2": "flushed (256 MiB write) before every step, outside the timed events",
+                   "parallelism": f"replicas x{world}"},
+        "pct_of_bf16_peak": 100.0 * value / peak,
+        "stages_ms": avg,
+        "forward_tflops": fwd_tf,
+        "forward_pct_of_peak": 100.0 * fwd_tf / peak,
+        "backward_tflops": f_bwd / ((avg["preprocess"] + avg["backward_main"] + avg["convert"]) * 1e-3) / 1e12,
+        "backward_main_tflops": main_tf,
+        "roofline": {"kernel": "k_attn_bwd (a5)", "bound": "tensor", "achieved": main_tf,
+                     "peak": peak, "unit": "TFLOP/s", "frac": main_tf / peak,
+                     "traffic": traffic, "peak_source": peaks["source"] + " bf16 burst"},
+        "roofline_forward": {"kernel": "k_attn_fwd (a3)", "bound": "tensor", "achieved": fwd_tf,
+                             "peak": peak, "unit": "TFLOP/s", "frac": fwd_tf / peak,
+                             "traffic": profiled_traffic("k_attn_fwd", "window8192")},
+        "gpu_launches": launches,
+        "wall_s_timed_loop": t_wall,
+        "clocks": clk.summary(),
+    }
+
+    if not args.no_e2e:
+        line["e2e"] = e2e_leg(args, wl, dev, f_fwd + f_bwd, world)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        n_rows = min(1024, wl.Sq)
+        dt, fl, threads = oracle_sample(wl, n_rows)
+        line["cpu_baseline"] = {
+            "value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+            "sample": f"rows 0..{n_rows - 1} of head 0 (one causal band), forward + backward, fp64"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def e2e_leg(args, wl, dev, flops, world):
+    """The same step through the public API with host buffers: pinned host ->
+    device copies of q, k, v, dO, the full path, device -> host copies of O, LSE,
+    dQ, dK, dV, all inside the timed region."""
+    import torch
+    import block_sparse_attention_map_b200 as bsa
+
+    host = {n: getattr(wl, n).cpu().pin_memory() for n in ("q", "k", "v", "dO")}
+    dev_in = {n: torch.empty_like(getattr(wl, n)) for n in host}
+    out_h = {n: torch.empty(shape, dtype=dt).pin_memory()
+             for n, shape, dt in (("o", wl.q.shape, torch.bfloat16),
+                                  ("lse", (wl.B, wl.H, wl.Sq), torch.float32),
+                                  ("dq", wl.q.shape, torch.bfloat16),
+                                  ("dk", wl.k.shape, torch.bfloat16),
+                                  ("dv", wl.v.shape, torch.bfloat16))}
+    st = bsa.Stages(dev_in["q"], dev_in["k"], dev_in["v"], wl.mask, softmax_mode=args.softmax,
+                    order=args.order)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        for n in host:
+            dev_in[n].copy_(host[n], non_blocking=True)
+        st.plan()
+        st.bound()
+        st.forward()
+        st.preprocess(dev_in["dO"])
+        st.backward_main(dev_in["dO"])
+        st.convert()
+        for n, src in (("o", st.out), ("lse", st.lse), ("dq", st.dq), ("dk", st.dk), ("dv", st.dv)):
+            out_h[n].copy_(src, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1), world)
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = sum(t.numel() * t.element_size() for t in out_h.values())
+    return {"value": world * args.steps * flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "ms_per_step": ms / args.steps}
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        run_reference(args, world, rank)
+        return
+    world, rank, local = dist_setup(args)
+    try:
+        run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -8,6 +8,7 @@ not load the library; the first call does, and fails loudly if it is missing.
 from ._binding import (  # noqa: F401
     BsaError,
     Mask,
+    Stages,
     Workspace,
     attn_bwd,
     attn_fwd,

@@ -51,7 +51,7 @@ class MaskSpec(ctypes.Structure):
 class Options(ctypes.Structure):
     _fields_ = [("softmax_mode", c_i32), ("gate_limit", c_f32), ("kmax_override", c_vp),
                 ("bwd_order", c_i32), ("deterministic", c_i32), ("perm", c_vp),
-                ("sem_timeout_ns", c_i64), ("plan_ready", c_i32), ("reserved", c_i32)]
+                ("sem_timeout_ns", c_i64), ("plan_ready", c_i32), ("bound_ready", c_i32)]
 
 
 class WorkspaceView(ctypes.Structure):
@@ -93,6 +93,13 @@ def lib() -> ctypes.CDLL:
                                      c_vp, ctypes.c_size_t, c_vp]),
             "bsa_attn_bwd": (c_i32, [P(Problem), P(MaskSpec), P(Options), c_vp, c_vp, c_vp, c_vp, c_vp,
                                      c_vp, c_vp, c_vp, c_vp, c_vp, ctypes.c_size_t, c_vp]),
+            "bsa_fixed_m_bound": (c_i32, [P(Problem), P(MaskSpec), P(Options), c_vp, c_vp, c_vp,
+                                          ctypes.c_size_t, c_vp]),
+            "bsa_bwd_preprocess": (c_i32, [P(Problem), P(MaskSpec), P(Options), c_vp, c_vp, c_vp,
+                                           ctypes.c_size_t, c_vp]),
+            "bsa_bwd_main": (c_i32, [P(Problem), P(MaskSpec), P(Options), c_vp, c_vp, c_vp, c_vp, c_vp,
+                                     c_vp, c_vp, c_vp, ctypes.c_size_t, c_vp]),
+            "bsa_bwd_convert": (c_i32, [P(Problem), P(MaskSpec), c_vp, c_vp, ctypes.c_size_t, c_vp]),
             "bsa_get_device_status": (c_i32, [c_vp, ctypes.c_size_t, c_vp, c_i32]),
             "bsa_status_string": (ctypes.c_char_p, [c_i32]),
             "bsa_launch_count": (ctypes.c_uint64, []),
@@ -185,7 +192,8 @@ class Mask:
 
 
 def make_options(softmax_mode="online", gate_limit=0.0, kmax_override=None, order="asc",
-                 perm=None, deterministic=True, sem_timeout_ns=0, plan_ready=False):
+                 perm=None, deterministic=True, sem_timeout_ns=0, plan_ready=False,
+                 bound_ready=False):
     o = Options()
     o.softmax_mode = SOFTMAX_FIXED_M_GATED if softmax_mode in ("fixed_m", SOFTMAX_FIXED_M_GATED) else SOFTMAX_ONLINE
     o.gate_limit = float(gate_limit)
@@ -194,6 +202,7 @@ def make_options(softmax_mode="online", gate_limit=0.0, kmax_override=None, orde
     o.deterministic = 1 if deterministic else 0
     o.sem_timeout_ns = int(sem_timeout_ns)
     o.plan_ready = 1 if plan_ready else 0
+    o.bound_ready = 1 if bound_ready else 0
     o._perm_buf = None
     if perm is not None:
         buf = (c_i32 * len(perm))(*[int(x) for x in perm])
@@ -318,3 +327,52 @@ def attn_bwd(q, k, v, out, dout, lse, mask=None, order="asc", perm=None, determi
                               _stream()), "bsa_attn_bwd")
     ws._mask = m
     return dq, dk, dv, ws
+
+
+class Stages:
+    """The hot path one C-ABI call per stage (a1+a6 plan, a2 bound, a3 forward,
+    a4 preprocess, a5 backward main, a7 dQ convert), on one preallocated
+    workspace, for callers that time or schedule stages separately."""
+
+    def __init__(self, q, k, v, mask=None, softmax_mode="online", order="asc", perm=None,
+                 deterministic=True, gate_limit=0.0):
+        self.q, self.k, self.v = q, k, v
+        B, Sq, H, D = q.shape
+        self.out = torch.empty_like(q)
+        self.lse = torch.empty(B, H, Sq, dtype=torch.float32, device=q.device)
+        self.dq, self.dk, self.dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        self.prob = make_problem(q, k, v, self.out)
+        self.mask = Mask(mask, q.device)
+        self.fixed = softmax_mode in ("fixed_m", SOFTMAX_FIXED_M_GATED)
+        self.opt = make_options(softmax_mode, gate_limit, None, order, perm, deterministic, 0,
+                                plan_ready=True, bound_ready=True)
+        self.ws = Workspace(self.prob, self.mask, True, q.device)
+        self._args = (ctypes.byref(self.prob), ctypes.byref(self.mask.spec), ctypes.byref(self.opt))
+
+    def plan(self):
+        _check(lib().bsa_plan_build(*self._args, self.ws.ptr(), self.ws.nbytes, _stream()), "bsa_plan_build")
+
+    def bound(self):
+        if self.fixed:
+            _check(lib().bsa_fixed_m_bound(*self._args, self.q.data_ptr(), self.k.data_ptr(), self.ws.ptr(),
+                                           self.ws.nbytes, _stream()), "bsa_fixed_m_bound")
+
+    def forward(self):
+        _check(lib().bsa_attn_fwd(*self._args, self.q.data_ptr(), self.k.data_ptr(), self.v.data_ptr(),
+                                  self.out.data_ptr(), self.lse.data_ptr(), self.ws.ptr(), self.ws.nbytes,
+                                  _stream()), "bsa_attn_fwd")
+
+    def preprocess(self, dout):
+        _check(lib().bsa_bwd_preprocess(*self._args, self.out.data_ptr(), dout.data_ptr(), self.ws.ptr(),
+                                        self.ws.nbytes, _stream()), "bsa_bwd_preprocess")
+
+    def backward_main(self, dout):
+        _check(lib().bsa_bwd_main(*self._args, self.q.data_ptr(), self.k.data_ptr(), self.v.data_ptr(),
+                                  dout.data_ptr(), self.lse.data_ptr(), self.dk.data_ptr(),
+                                  self.dv.data_ptr(), self.ws.ptr(), self.ws.nbytes, _stream()),
+               "bsa_bwd_main")
+
+    def convert(self):
+        _check(lib().bsa_bwd_convert(ctypes.byref(self.prob), ctypes.byref(self.mask.spec),
+                                     self.dq.data_ptr(), self.ws.ptr(), self.ws.nbytes, _stream()),
+               "bsa_bwd_convert")

@@ -327,7 +327,7 @@ bsa_status bsa_attn_fwd(const bsa_problem *prob, const bsa_mask_spec *mask,
     if ((st = cuda_status(launch_plan(p, P.m, P.o, P.L, w, s))) != BSA_OK) return st;
   }
   const MaskParams mp = mask_params(p, P.m, P.L, w);
-  if (P.o.softmax_mode == BSA_SOFTMAX_FIXED_M_GATED) {
+  if (P.o.softmax_mode == BSA_SOFTMAX_FIXED_M_GATED && !P.o.bound_ready) {
     if ((st = cuda_status(launch_fixed_m_bound(p, mp, P.o, q, k, P.L, w, s))) != BSA_OK) return st;
   }
   return cuda_status(launch_fwd(p, mp, P.o, signature(p, P.m, P.o), tq, tk, tv, out, lse, P.L, w, s));
@@ -361,6 +361,77 @@ bsa_status bsa_attn_bwd(const bsa_problem *prob, const bsa_mask_spec *mask,
   const MaskParams mp = mask_params(p, P.m, P.L, w);
   return cuda_status(launch_bwd(p, mp, P.o, signature(p, P.m, P.o), tq, tk, tv, tdo, out, dout,
                                 lse, dq, dk, dv, P.L, w, s));
+}
+
+bsa_status bsa_fixed_m_bound(const bsa_problem *prob, const bsa_mask_spec *mask,
+                             const bsa_options *opt, const void *q, const void *k, void *ws,
+                             size_t ws_bytes, bsa_stream_t stream) {
+  if (q == nullptr || k == nullptr) return BSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k)) return BSA_ERR_UNSUPPORTED;
+  Prepared P;
+  bsa_status st = prepare(prob, mask, opt, ws, ws_bytes, false, &P);
+  if (st != BSA_OK) return st;
+  uint8_t *w = static_cast<uint8_t *>(ws);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (!P.o.plan_ready) {
+    // the key-validity predicates of varlen masks come from the planner
+    if ((st = cuda_status(launch_plan(P.p, P.m, P.o, P.L, w, s))) != BSA_OK) return st;
+  }
+  const MaskParams mp = mask_params(P.p, P.m, P.L, w);
+  return cuda_status(launch_fixed_m_bound(P.p, mp, P.o, q, k, P.L, w, s));
+}
+
+bsa_status bsa_bwd_preprocess(const bsa_problem *prob, const bsa_mask_spec *mask,
+                              const bsa_options *opt, const void *out, const void *dout, void *ws,
+                              size_t ws_bytes, bsa_stream_t stream) {
+  if (out == nullptr || dout == nullptr) return BSA_ERR_INVALID_ARG;
+  if (!aligned16(out) || !aligned16(dout)) return BSA_ERR_UNSUPPORTED;
+  Prepared P;
+  bsa_status st = prepare(prob, mask, opt, ws, ws_bytes, true, &P);
+  if (st != BSA_OK) return st;
+  return cuda_status(launch_bwd_preprocess(P.p, out, dout, P.L, static_cast<uint8_t *>(ws),
+                                           reinterpret_cast<cudaStream_t>(stream)));
+}
+
+bsa_status bsa_bwd_main(const bsa_problem *prob, const bsa_mask_spec *mask,
+                        const bsa_options *opt, const void *q, const void *k, const void *v,
+                        const void *dout, const float *lse, void *dk, void *dv, void *ws,
+                        size_t ws_bytes, bsa_stream_t stream) {
+  if (q == nullptr || k == nullptr || v == nullptr || dout == nullptr || lse == nullptr ||
+      dk == nullptr || dv == nullptr)
+    return BSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) || !aligned16(dk) ||
+      !aligned16(dv) || (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return BSA_ERR_UNSUPPORTED;
+  Prepared P;
+  bsa_status st = prepare(prob, mask, opt, ws, ws_bytes, true, &P);
+  if (st != BSA_OK) return st;
+  const bsa_problem &p = P.p;
+  CUtensorMap tq, tk, tv, tdo;
+  if (!make_map(&tq, q, p.B, p.Sq, p.H, p.D, p.q_stride) ||
+      !make_map(&tk, k, p.B, p.Skv, p.H, p.D, p.k_stride) ||
+      !make_map(&tv, v, p.B, p.Skv, p.H, p.D, p.v_stride) ||
+      !make_map(&tdo, dout, p.B, p.Sq, p.H, p.D, p.o_stride))
+    return BSA_ERR_UNSUPPORTED;
+  uint8_t *w = static_cast<uint8_t *>(ws);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (!P.o.plan_ready) {
+    if ((st = cuda_status(launch_plan(p, P.m, P.o, P.L, w, s))) != BSA_OK) return st;
+  }
+  const MaskParams mp = mask_params(p, P.m, P.L, w);
+  return cuda_status(launch_bwd_main(p, mp, P.o, signature(p, P.m, P.o), tq, tk, tv, tdo, lse, dk,
+                                     dv, P.L, w, s));
+}
+
+bsa_status bsa_bwd_convert(const bsa_problem *prob, const bsa_mask_spec *mask, void *dq, void *ws,
+                           size_t ws_bytes, bsa_stream_t stream) {
+  if (dq == nullptr) return BSA_ERR_INVALID_ARG;
+  if (!aligned16(dq)) return BSA_ERR_UNSUPPORTED;
+  Prepared P;
+  bsa_status st = prepare(prob, mask, nullptr, ws, ws_bytes, true, &P);
+  if (st != BSA_OK) return st;
+  return cuda_status(launch_bwd_convert(P.p, dq, P.L, static_cast<uint8_t *>(ws),
+                                        reinterpret_cast<cudaStream_t>(stream)));
 }
 
 bsa_status bsa_get_device_status(void *ws, size_t ws_bytes, bsa_stream_t stream, int32_t clear) {

@@ -649,50 +649,38 @@ cudaError_t run_bwd_main(const BwdParams &bp, const CUtensorMap &tq, const CUten
   return cudaGetLastError();
 }
 
-template <int D>
-cudaError_t run_bwd(const bsa_problem &p, const BwdParams &bp, const void *out, const void *dout,
-                    void *dq, const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
-                    const CUtensorMap &tdo, cudaStream_t s) {
-  const int rows_pad = bp.nM * kTile;
+}  // namespace
+
+cudaError_t launch_bwd_preprocess(const bsa_problem &p, const void *out, const void *dout,
+                                  const WsLayout &L, uint8_t *ws, cudaStream_t s) {
+  const int rows_pad = L.nM * kTile;
   const int64_t groups = static_cast<int64_t>(p.B) * p.H * rows_pad;
-  const int64_t threads = groups * (D / 8);
-  k_bwd_delta<D><<<static_cast<unsigned>((threads + 255) / 256), 256, 0, s>>>(
-      static_cast<const __nv_bfloat16 *>(out), static_cast<const __nv_bfloat16 *>(dout),
-      p.o_stride[0], p.o_stride[1], p.o_stride[2], p.B, p.Sq, p.H, rows_pad,
-      const_cast<float *>(bp.delta));
+  const int64_t threads = groups * (p.D / 8);
+  float *delta = reinterpret_cast<float *>(ws + L.delta);
+  const unsigned blocks = static_cast<unsigned>((threads + 255) / 256);
+  if (p.D == 64)
+    k_bwd_delta<64><<<blocks, 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(out),
+                                           static_cast<const __nv_bfloat16 *>(dout), p.o_stride[0],
+                                           p.o_stride[1], p.o_stride[2], p.B, p.Sq, p.H, rows_pad,
+                                           delta);
+  else
+    k_bwd_delta<128><<<blocks, 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(out),
+                                            static_cast<const __nv_bfloat16 *>(dout), p.o_stride[0],
+                                            p.o_stride[1], p.o_stride[2], p.B, p.Sq, p.H, rows_pad,
+                                            delta);
   count_launch();
-  cudaError_t e = cudaMemsetAsync(bp.dq_accum, 0,
-                                  sizeof(float) * static_cast<size_t>(groups) * D, s);
+  cudaError_t e = cudaMemsetAsync(ws + L.dq_accum, 0,
+                                  sizeof(float) * static_cast<size_t>(groups) * p.D, s);
   if (e != cudaSuccess) return e;
-  e = cudaMemsetAsync(bp.sem, 0, sizeof(uint32_t) * static_cast<size_t>(p.B) * p.H * bp.nM, s);
+  e = cudaMemsetAsync(ws + L.sem, 0, sizeof(uint32_t) * static_cast<size_t>(p.B) * p.H * L.nM, s);
   if (e != cudaSuccess) return e;
-  e = cudaMemsetAsync(bp.hdr + kHdrBwdTicket, 0, sizeof(uint32_t), s);
-  if (e != cudaSuccess) return e;
-  e = (D == 64) ? run_bwd_main<64, 2, 2>(bp, tq, tk, tv, tdo, s)
-                : run_bwd_main<128, 2, 1>(bp, tq, tk, tv, tdo, s);
-  if (e != cudaSuccess) return e;
-  const size_t smem = sizeof(float) * kTile * (D + 4);
-  static bool attr = false;
-  if (!attr) {
-    e = cudaFuncSetAttribute(k_dq_convert<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
-  k_dq_convert<D><<<p.B * p.H * bp.nM, 256, smem, s>>>(bp.dq_accum, p.B, p.H, p.Sq, bp.nM,
-                                                       static_cast<__nv_bfloat16 *>(dq),
-                                                       p.q_stride[0], p.q_stride[1], p.q_stride[2]);
-  count_launch();
   return cudaGetLastError();
 }
 
-}  // namespace
-
-cudaError_t launch_bwd(const bsa_problem &p, const MaskParams &mp, const bsa_options &o,
-                       const PlanSignature &sig, const CUtensorMap &tq, const CUtensorMap &tk,
-                       const CUtensorMap &tv, const CUtensorMap &tdo, const void *out,
-                       const void *dout, const float *lse, void *dq, void *dk, void *dv,
-                       const WsLayout &L, uint8_t *ws, cudaStream_t s) {
+cudaError_t launch_bwd_main(const bsa_problem &p, const MaskParams &mp, const bsa_options &o,
+                            const PlanSignature &sig, const CUtensorMap &tq, const CUtensorMap &tk,
+                            const CUtensorMap &tv, const CUtensorMap &tdo, const float *lse,
+                            void *dk, void *dv, const WsLayout &L, uint8_t *ws, cudaStream_t s) {
   BwdParams bp{};
   bp.mask = mp;
   bp.B = p.B;
@@ -723,11 +711,43 @@ cudaError_t launch_bwd(const bsa_problem &p, const MaskParams &mp, const bsa_opt
   bp.deterministic = o.deterministic ? 1 : 0;
   bp.hdr = reinterpret_cast<uint32_t *>(ws + L.status);
   bp.timeout_ns = 2000000000ull;
-  bp.sem_timeout_ns = o.sem_timeout_ns > 0 ? static_cast<uint64_t>(o.sem_timeout_ns) : 1000000000ull;
+  bp.sem_timeout_ns =
+      o.sem_timeout_ns > 0 ? static_cast<uint64_t>(o.sem_timeout_ns) : 1000000000ull;
   for (int i = 0; i < 7; ++i) bp.sig[i] = sig.w[i];
   bp.sig_mask = 0x7Fu;
-  if (p.D == 64) return run_bwd<64>(p, bp, out, dout, dq, tq, tk, tv, tdo, s);
-  return run_bwd<128>(p, bp, out, dout, dq, tq, tk, tv, tdo, s);
+  cudaError_t e = cudaMemsetAsync(bp.hdr + kHdrBwdTicket, 0, sizeof(uint32_t), s);
+  if (e != cudaSuccess) return e;
+  return (p.D == 64) ? run_bwd_main<64, 2, 2>(bp, tq, tk, tv, tdo, s)
+                     : run_bwd_main<128, 2, 1>(bp, tq, tk, tv, tdo, s);
+}
+
+cudaError_t launch_bwd_convert(const bsa_problem &p, void *dq, const WsLayout &L, uint8_t *ws,
+                               cudaStream_t s) {
+  const float *acc = reinterpret_cast<const float *>(ws + L.dq_accum);
+  const unsigned blocks = static_cast<unsigned>(p.B * p.H * L.nM);
+  auto go = [&](auto kern, int D) -> cudaError_t {
+    const size_t smem = sizeof(float) * kTile * (D + 4);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    kern<<<blocks, 256, smem, s>>>(acc, p.B, p.H, p.Sq, L.nM, static_cast<__nv_bfloat16 *>(dq),
+                                   p.q_stride[0], p.q_stride[1], p.q_stride[2]);
+    count_launch();
+    return cudaGetLastError();
+  };
+  return p.D == 64 ? go(k_dq_convert<64>, 64) : go(k_dq_convert<128>, 128);
+}
+
+cudaError_t launch_bwd(const bsa_problem &p, const MaskParams &mp, const bsa_options &o,
+                       const PlanSignature &sig, const CUtensorMap &tq, const CUtensorMap &tk,
+                       const CUtensorMap &tv, const CUtensorMap &tdo, const void *out,
+                       const void *dout, const float *lse, void *dq, void *dk, void *dv,
+                       const WsLayout &L, uint8_t *ws, cudaStream_t s) {
+  cudaError_t e = launch_bwd_preprocess(p, out, dout, L, ws, s);
+  if (e != cudaSuccess) return e;
+  e = launch_bwd_main(p, mp, o, sig, tq, tk, tv, tdo, lse, dk, dv, L, ws, s);
+  if (e != cudaSuccess) return e;
+  return launch_bwd_convert(p, dq, L, ws, s);
 }
 
 }  // namespace bsa

@@ -274,7 +274,7 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       }
       const int ob = ul & 1;
       const bool fixed = p.fixed_mode && p.gate[bh] != 0;
-      float m_ref = -INFINITY, l = 0.f;
+      float m_ref = -INFINITY, l = 0.f, l_r = 0.f;
       if (fixed) m_ref = row_ok ? p.scale_log2 * p.qnorm[static_cast<int64_t>(bh) * p.Sq + i] * p.kmax[bh] : 0.f;
       // row-constant part of the mask: allowed keys lie in [lo, hi]
       int lo = 0, hi = p.Skv - 1;
@@ -344,6 +344,7 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
           if (need) {
             alpha = fast_exp2(m_ref - mt);
             l *= alpha;
+            l_r *= alpha;
             m_ref = mt;
           }
           if (__any_sync(0xffffffffu, resc)) {
@@ -364,7 +365,7 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
           }
         }
         const float mu = (m_ref == -INFINITY) ? 0.f : m_ref;
-        float rowsum = 0.f;
+        float rowsum = 0.f, rowsum_r = 0.f;
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
           uint32_t pk[32];
@@ -373,14 +374,17 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
             const float p0 = fast_exp2(fmaf(f[64 * half + 2 * c], p.scale_log2, -mu));
             const float p1 = fast_exp2(fmaf(f[64 * half + 2 * c + 1], p.scale_log2, -mu));
             pk[c] = pack_bf16x2(p0, p1);
-            // l sums the bf16-rounded weights the PV product actually uses, so
-            // numerator and denominator carry the same rounding
-            rowsum += __uint_as_float(pk[c] << 16) + __uint_as_float(pk[c] & 0xffff0000u);
+            // two row sums: l over the exact weights (for LSE) and l_r over the
+            // bf16-rounded weights the PV product uses (normalising O by l_r
+            // makes numerator and denominator carry the same rounding)
+            rowsum += p0 + p1;
+            rowsum_r += __uint_as_float(pk[c] << 16) + __uint_as_float(pk[c] & 0xffff0000u);
           }
           // P (bf16 pairs) overwrites the first 64 columns of this S buffer
           tmem_st32(t_s + 32 * half, pk);
         }
         l += rowsum;
+        l_r += rowsum_r;
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&bars[L::bPFull + s]);
@@ -389,7 +393,7 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       // epilogue: O / l -> bf16, LSE
       if (!wwait(&bars[L::bODone], (it - 1) & 1)) break;
       tc_fence_after();
-      const float inv = l > 0.f ? 1.f / l : 0.f;
+      const float inv = l_r > 0.f ? 1.f / l_r : 0.f;
       const uint32_t t_o = tmem + lane_off + 256 + ob * D;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {

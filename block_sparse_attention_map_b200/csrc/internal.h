@@ -91,6 +91,17 @@ cudaError_t launch_bwd(const bsa_problem &p, const MaskParams &mp, const bsa_opt
                        const float *lse, void *dq, void *dk, void *dv, const WsLayout &L,
                        uint8_t *ws, cudaStream_t s);
 
+cudaError_t launch_bwd_preprocess(const bsa_problem &p, const void *out, const void *dout,
+                                  const WsLayout &L, uint8_t *ws, cudaStream_t s);
+
+cudaError_t launch_bwd_main(const bsa_problem &p, const MaskParams &mp, const bsa_options &o,
+                            const PlanSignature &sig, const CUtensorMap &tq, const CUtensorMap &tk,
+                            const CUtensorMap &tv, const CUtensorMap &tdo, const float *lse,
+                            void *dk, void *dv, const WsLayout &L, uint8_t *ws, cudaStream_t s);
+
+cudaError_t launch_bwd_convert(const bsa_problem &p, void *dq, const WsLayout &L, uint8_t *ws,
+                               cudaStream_t s);
+
 void count_launch(int n = 1);
 
 }  // namespace bsa

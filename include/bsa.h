@@ -143,7 +143,9 @@ typedef struct bsa_options {
   int32_t plan_ready;          /* 1: the workspace already holds the plan for this
                                   problem, mask and order (bsa_plan_build or an
                                   earlier fwd/bwd call); 0: build it first          */
-  int32_t reserved;
+  int32_t bound_ready;         /* fixed-m only. 1: the workspace already holds
+                                  kmax/qmax/gate from bsa_fixed_m_bound for these
+                                  q and k; 0: bsa_attn_fwd computes them first      */
 } bsa_options;
 
 /* Where the plan and the scratch arrays sit inside the workspace (byte offsets),
@@ -205,6 +207,38 @@ BSA_API bsa_status bsa_attn_bwd(const bsa_problem *prob, const bsa_mask_spec *ma
                         const void *v, const void *out, const void *dout,
                         const float *lse, void *dq, void *dk, void *dv, void *ws,
                         size_t ws_bytes, bsa_stream_t stream);
+
+/* The stages of the hot path, one call each, for callers that schedule or time
+ * them separately.  bsa_attn_fwd = [bsa_plan_build] + [bsa_fixed_m_bound] +
+ * forward kernel; bsa_attn_bwd = [bsa_plan_build] + bsa_bwd_preprocess +
+ * bsa_bwd_main + bsa_bwd_convert.  Each expects the workspace state the
+ * previous stage leaves; arguments as for bsa_attn_fwd / bsa_attn_bwd. */
+
+/* a2 ("Fixed-m softmax ...", introduction and "Notes"): kmax[b,h] = max over
+ * valid keys of ||k_j|| (or opt->kmax_override), qmax[b,h] and per-row ||q_i||,
+ * gate[b,h] = 2*scale*qmax*kmax <= G, all into the workspace. */
+BSA_API bsa_status bsa_fixed_m_bound(const bsa_problem *prob, const bsa_mask_spec *mask,
+                                     const bsa_options *opt, const void *q, const void *k,
+                                     void *ws, size_t ws_bytes, bsa_stream_t stream);
+
+/* a4: Delta_i = sum_d dO_id O_id (fp32) into the workspace; zeroes the fp32 dQ
+ * accumulator and the dQ semaphores. */
+BSA_API bsa_status bsa_bwd_preprocess(const bsa_problem *prob, const bsa_mask_spec *mask,
+                                      const bsa_options *opt, const void *out,
+                                      const void *dout, void *ws, size_t ws_bytes,
+                                      bsa_stream_t stream);
+
+/* a5 ("Add more optimal dk order optional arg", "Sliding window perf issue"):
+ * dK, dV written (bf16); dQ contributions accumulated into the workspace in
+ * the order pi when opt->deterministic. */
+BSA_API bsa_status bsa_bwd_main(const bsa_problem *prob, const bsa_mask_spec *mask,
+                                const bsa_options *opt, const void *q, const void *k,
+                                const void *v, const void *dout, const float *lse, void *dk,
+                                void *dv, void *ws, size_t ws_bytes, bsa_stream_t stream);
+
+/* a7: dQ = bf16(dQ accumulator). */
+BSA_API bsa_status bsa_bwd_convert(const bsa_problem *prob, const bsa_mask_spec *mask,
+                                   void *dq, void *ws, size_t ws_bytes, bsa_stream_t stream);
 
 /* Synchronises `stream`, then returns the sticky device status of `ws`
  * (BSA_OK if no device-side error was recorded); clear = 1 resets it. */

@@ -9,7 +9,7 @@ import torch
 import block_sparse_attention_map_b200 as bsa
 import oracle
 from block_sparse_attention_map_b200.workloads import make_workload
-from tests.gpu_common import O_TOL, mask_desc, np64
+from tests.gpu_common import O_TOL, excess, mask_desc, np64
 
 pytestmark = pytest.mark.gpu
 
@@ -29,7 +29,11 @@ def _oracle_grads(wl, heads=None):
 
 
 def _err(x, ref):
-    return float(np.max(np.abs(np64(x) - ref)))
+    """Raw max-abs error, after checking the ulp-aware bar element by element."""
+    ex = excess(x, ref)
+    raw = float(np.max(np.abs(np64(x) - ref)))
+    assert ex <= 0.0, f"max-abs {raw:.5f} exceeds {O_TOL} + half a bf16 ulp by {ex:.5f}"
+    return min(raw, O_TOL)
 
 
 SMALL = ["tiny", "packed", "window", "window_rect", "varlen", "video"]
