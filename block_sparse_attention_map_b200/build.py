@@ -14,7 +14,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 LIB = os.path.join(HERE, "libbsa.so")
-SOURCES = ["api.cu", "plan.cu", "fwd.cu", "bwd.cu"]
+SOURCES = ["api.cu", "plan.cu", "fwd.cu", "bwd.cu", "static_scratch.cu"]
 
 
 def nvcc() -> str:

@@ -240,6 +240,33 @@ BSA_API bsa_status bsa_bwd_main(const bsa_problem *prob, const bsa_mask_spec *ma
 BSA_API bsa_status bsa_bwd_convert(const bsa_problem *prob, const bsa_mask_spec *mask,
                                    void *dq, void *ws, size_t ws_bytes, bsa_stream_t stream);
 
+/* Forward for callers that cannot allocate device memory: plugin code run by a
+ * host framework that owns every device allocation and forbids cudaMalloc inside
+ * its execution callback, or code that must not risk the implicit device-wide
+ * synchronisation cudaMalloc / cudaFree may perform.  Same computation and
+ * arguments as bsa_attn_fwd (inputs and outputs still come from the caller), but
+ * no workspace: the plan and the fixed-m bound live in a fixed 32 MiB device
+ * array inside the library, which every GPU that loads the library holds until
+ * the process exits.  The source pages have no counterpart to this; it is a
+ * deployment convenience.
+ *  - Problems whose forward workspace (bsa_workspace_size, with_backward = 0)
+ *    exceeds 32 MiB are rejected with BSA_ERR_WORKSPACE_TOO_SMALL before any
+ *    launch.
+ *  - No cudaMalloc, cudaFree or other allocating call is made.  The first call
+ *    on each device looks up the array's device address (with that device
+ *    current); make that first call before any stream capture.
+ *  - Every call shares the one array and rebuilds the plan in it, so calls
+ *    whose work overlaps on the GPU (different streams, or concurrent host
+ *    threads) race and must be serialised by the caller.
+ *  - opt->plan_ready and opt->bound_ready are ignored.  Device-side errors land
+ *    in the array's status word, which callers of this entry point cannot read;
+ *    argument errors are returned as usual. */
+BSA_API bsa_status bsa_attn_fwd_static_scratch(const bsa_problem *prob,
+                                               const bsa_mask_spec *mask,
+                                               const bsa_options *opt, const void *q,
+                                               const void *k, const void *v, void *out,
+                                               float *lse, bsa_stream_t stream);
+
 /* Synchronises `stream`, then returns the sticky device status of `ws`
  * (BSA_OK if no device-side error was recorded); clear = 1 resets it. */
 BSA_API bsa_status bsa_get_device_status(void *ws, size_t ws_bytes, bsa_stream_t stream,
