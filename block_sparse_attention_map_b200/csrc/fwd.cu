@@ -9,16 +9,22 @@
 //     (one query row per thread) and rescales lazily; fixed-m pins the max to
 //     scale*||q_i||*kmax before streaming and needs neither max nor rescale.
 //
-// sm_100a design: one CTA per SM, persistent over work units (b, h, q-block).
-//   warp 0      TMA producer: Q tile (double-buffered) and K/V tiles
-//               (NS-stage ring), 128-byte swizzled boxes of 64 x 128.
-//   warp 1      owns TMEM (512 columns) and issues tcgen05.mma from one lane:
-//               S = Q K^T (SS, both K-major) into one of two S buffers, then
-//               O += P V (TS: P read from TMEM, V as an MN-major B operand).
-//   warps 2..5  softmax: tcgen05.ld of one S row per thread, mask on PARTIAL
-//               tiles only, exp2, P packed to bf16 and tcgen05.st back over S,
-//               lazy O rescale, epilogue O / l -> bf16 and LSE.
-// TMEM columns: S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [256+D,256+2D).
+// sm_100a design: one CTA per SM, persistent over work units = pairs of
+// q-blocks (A = 2g, B = 2g+1) of one (b, h).  The CTA walks the union of the
+// two row lists, so each K/V tile is loaded once for both q-blocks.
+//   warp 0      TMA producer: Q_A, Q_B once per unit; K and V tiles through
+//               separate stage rings, 128-byte swizzled 64 x 128 boxes.
+//   warp 1      owns TMEM (512 columns) and issues tcgen05.mma from one lane,
+//               ping-ponging the two groups: PV_A(u), S_A(u+1), PV_B(u),
+//               S_B(u+1), so one group's softmax overlaps the other's MMAs.
+//               S = Q K^T is SS (both K-major); O += P V is TS (P read from
+//               TMEM over the S columns, V an MN-major B operand).
+//   warps 4-7   softmax of q-block A, warps 8-11 of q-block B: one query row
+//               per thread (its TMEM lane).  PARTIAL tiles are masked through a
+//               128-bit allowed-key mask (row range AND segment ids); online
+//               mode takes the tile max in a first pass over TMEM and rescales
+//               O lazily; the epilogue writes O / l_r (bf16) and LSE.
+// TMEM columns: S_A [0,128) S_B [128,256) O_A [256,256+D) O_B [256+D,256+2D).
 #include <cfloat>
 
 #include "internal.h"
@@ -50,22 +56,20 @@ struct FwdParams {
   uint32_t sig_mask;   // which signature words must match
 };
 
-template <int D, int NS>
+template <int D, int NK, int NV>
 struct FwdSmem {
-  static constexpr int kTileBytes = kTile * D * 2;
-  static constexpr int kQ = 0;
-  static constexpr int kK = kQ + 2 * kTileBytes;
-  static constexpr int kV = kK + NS * kTileBytes;
-  static constexpr int kSeg = kV + NS * kTileBytes;     // int32 [2][128]
-  static constexpr int kBar = kSeg + 2 * kTile * 4;     // mbarriers
-  // barrier indices
-  static constexpr int bQFull = 0, bQEmpty = 2, bKFull = 4, bKEmpty = 4 + NS, bVFull = 4 + 2 * NS,
-                       bVEmpty = 4 + 3 * NS, bSFull = 4 + 4 * NS, bPFull = bSFull + 2,
-                       bSFree = bPFull + 2, bODone = bSFree + 2, bOFree = bODone + 1,
-                       bSegReady = bOFree + 2, bFinal = bSegReady + 2, kNumBars = bFinal + 1;
-  static constexpr int kMisc = kBar + kNumBars * 8;      // tmem slot, abort flag
-  static constexpr int kBytes = kMisc + 16;
-  static constexpr int kAlloc = kBytes + 1024;           // slack for 1024-byte alignment
+  static constexpr int kTB = kTile * D * 2;
+  static constexpr int kQ = 0;                         // Q tiles of groups A, B
+  static constexpr int kK = 2 * kTB;                   // K ring
+  static constexpr int kV = kK + NK * kTB;             // V ring
+  static constexpr int kSeg = kV + NV * kTB;           // int32 [group][buffer][128]
+  static constexpr int kBar = kSeg + 4 * kTile * 4;
+  static constexpr int bQFull = 0, bQEmpty = 2, bKFull = 4, bKEmpty = bKFull + NK,
+                       bVFull = bKEmpty + NK, bVEmpty = bVFull + NV, bSFull = bVEmpty + NV,
+                       bPFull = bSFull + 2, bPVDone = bPFull + 2, bSegReady = bPVDone + 2,
+                       bFinal = bSegReady + 4, kNumBars = bFinal + 1;
+  static constexpr int kMisc = kBar + kNumBars * 8;  // tmem slot, abort flag
+  static constexpr int kAlloc = kMisc + 16;
 };
 
 // Bounded wait that ignores the abort flag: used only to drain copies already
@@ -78,14 +82,63 @@ __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity) {
   }
 }
 
-template <int D, int NS>
-__global__ void __launch_bounds__(192, 1)
+// One work unit: a pair of q-blocks (A = 2g, B = 2g+1) of one (b, h).
+struct FwdUnit {
+  int b, h, bh, m[2], rs[2], re[2];
+};
+
+__device__ __forceinline__ FwdUnit decode_unit(const FwdParams &p, int u) {
+  FwdUnit w;
+  const int nP = (p.nM + 1) >> 1;
+  w.bh = u / nP;
+  const int g = u % nP;
+  w.b = w.bh / p.H;
+  w.h = w.bh % p.H;
+#pragma unroll
+  for (int x = 0; x < 2; ++x) {
+    w.m[x] = 2 * g + x;
+    if (w.m[x] < p.nM) {
+      w.rs[x] = p.row_ptr[w.b * p.nM + w.m[x]];
+      w.re[x] = p.row_ptr[w.b * p.nM + w.m[x] + 1];
+    } else {
+      w.rs[x] = w.re[x] = 0;
+    }
+  }
+  return w;
+}
+
+// Walks the union of the two row lists in ascending kv-block order.
+struct UnionWalk {
+  const uint32_t *ent;
+  int i[2], e[2];
+  __device__ __forceinline__ bool next(int &n, bool &in0, bool &in1) {
+    const int n0 = i[0] < e[0] ? static_cast<int>(ent[i[0]] & kIndexMask) : INT_MAX;
+    const int n1 = i[1] < e[1] ? static_cast<int>(ent[i[1]] & kIndexMask) : INT_MAX;
+    if (n0 == INT_MAX && n1 == INT_MAX) return false;
+    n = min(n0, n1);
+    in0 = n0 == n;
+    in1 = n1 == n;
+    i[0] += in0;
+    i[1] += in1;
+    return true;
+  }
+};
+
+// Allowed-key bits of columns 32w .. 32w+31 that fall inside [lo, hi].
+__device__ __forceinline__ uint32_t range_bits(int lo, int hi, int w) {
+  const int a = max(lo - 32 * w, 0), z = min(hi - 32 * w, 31);
+  if (a > z) return 0u;
+  const uint32_t top = (z >= 31) ? 0xffffffffu : ((1u << (z + 1)) - 1u);
+  const uint32_t bot = (a <= 0) ? 0xffffffffu : ~((1u << a) - 1u);
+  return top & bot;
+}
+
+template <int D, int NK, int NV>
+__global__ void __launch_bounds__(384, 1)
 k_attn_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
            const __grid_constant__ CUtensorMap tv, const FwdParams p) {
-  using L = FwdSmem<D, NS>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                            ~static_cast<uintptr_t>(1023));
+  using L = FwdSmem<D, NK, NV>;
+  extern __shared__ __align__(1024) uint8_t sm[];
   uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::kBar);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::kMisc);
   int *abort_flag = reinterpret_cast<int *>(sm + L::kMisc + 4);
@@ -96,8 +149,7 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
   if (threadIdx.x == 0) {
     for (int i = 0; i < L::kNumBars; ++i) {
       uint32_t cnt = 1;
-      if (i == L::bPFull || i == L::bPFull + 1 || i == L::bOFree || i == L::bOFree + 1 ||
-          i == L::bSegReady || i == L::bSegReady + 1)
+      if ((i >= L::bPFull && i < L::bPFull + 2) || (i >= L::bSegReady && i < L::bSegReady + 4))
         cnt = 128;
       mbar_init(&bars[i], cnt);
     }
@@ -124,128 +176,157 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
     bool ok = h[kHdrMagic] == kPlanMagic;
     for (int i = 0; i < 7; ++i) ok = ok && (!((p.sig_mask >> i) & 1u) || h[kHdrB + i] == p.sig[i]);
     if (!ok) wd.trip(BSA_ERR_PLAN_MISMATCH);
+    // the swizzled tiles rely on a 1024-byte aligned dynamic shared window
+    if ((smem_u32(sm) & 1023u) != 0u) wd.trip(BSA_ERR_UNSUPPORTED);
   }
   __syncthreads();
 
-  const int nM = p.nM;
   constexpr uint32_t kIdescS = idesc_bf16_f32(128, 128, 0, 0);
   constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, 0, 1);
-  constexpr int kTB = L::kTileBytes;
+  constexpr int kTB = L::kTB;
 
   if (wd.aborted()) {
-    // plan mismatch: nothing to do
+    // plan mismatch or misaligned shared memory: nothing to do
   } else if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      uint32_t kv_it = 0, ul = 0, k_issued = 0, v_issued = 0, q_issued = 0;
-      for (int u = blockIdx.x; u < p.n_units; u += gridDim.x) {
-        const int bh = u / nM, m = u % nM, b = bh / p.H, h = bh % p.H;
-        const int rs = p.row_ptr[b * nM + m], re = p.row_ptr[b * nM + m + 1];
-        if (re == rs) continue;
-        const int qb = ul & 1;
-        if (ul >= 2 && !wd.wait(&bars[L::bQEmpty + qb], ((ul >> 1) - 1) & 1)) break;
-        mbar_arrive_expect_tx(&bars[L::bQFull + qb], kTB);
-        for (int c = 0; c < D / 64; ++c)
-          tma_load_4d(sm + L::kQ + qb * kTB + c * 16384, &tq, &bars[L::bQFull + qb], c * 64,
-                      m * kTile, h, b);
-        ++q_issued;
-        bool stop = false;
-        for (int e = rs; e < re; ++e) {
-          const int n = static_cast<int>(p.row_ent[e] & kIndexMask);
-          const uint32_t st = kv_it % NS;
-          const uint32_t use = kv_it / NS;
-          if (kv_it >= NS && !wd.wait(&bars[L::bKEmpty + st], (use - 1) & 1)) { stop = true; break; }
-          mbar_arrive_expect_tx(&bars[L::bKFull + st], kTB);
+      uint32_t kv = 0, uq[2] = {0, 0}, k_issued = 0, v_issued = 0, q_issued[2] = {0, 0};
+      bool stop = false;
+      for (int u = blockIdx.x; u < p.n_units && !stop; u += gridDim.x) {
+        const FwdUnit w = decode_unit(p, u);
+        const bool has[2] = {w.re[0] > w.rs[0], w.re[1] > w.rs[1]};
+        if (!has[0] && !has[1]) continue;
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+          if (!has[x]) continue;
+          if (uq[x] >= 1 && !wd.wait(&bars[L::bQEmpty + x], (uq[x] - 1) & 1)) { stop = true; break; }
+          mbar_arrive_expect_tx(&bars[L::bQFull + x], kTB);
           for (int c = 0; c < D / 64; ++c)
-            tma_load_4d(sm + L::kK + st * kTB + c * 16384, &tk, &bars[L::bKFull + st], c * 64,
-                        n * kTile, h, b);
-          ++k_issued;
-          if (kv_it >= NS && !wd.wait(&bars[L::bVEmpty + st], (use - 1) & 1)) { stop = true; break; }
-          mbar_arrive_expect_tx(&bars[L::bVFull + st], kTB);
-          for (int c = 0; c < D / 64; ++c)
-            tma_load_4d(sm + L::kV + st * kTB + c * 16384, &tv, &bars[L::bVFull + st], c * 64,
-                        n * kTile, h, b);
-          ++v_issued;
-          ++kv_it;
+            tma_load_4d(sm + L::kQ + x * kTB + c * 16384, &tq, &bars[L::bQFull + x], c * 64,
+                        w.m[x] * kTile, w.h, w.b);
+          ++uq[x];
+          ++q_issued[x];
         }
-        ++ul;
         if (stop) break;
+        UnionWalk uw{p.row_ent, {w.rs[0], w.rs[1]}, {w.re[0], w.re[1]}};
+        int n;
+        bool i0, i1;
+        while (uw.next(n, i0, i1)) {
+          const uint32_t ks = kv % NK, vs = kv % NV;
+          if (kv >= NK && !wd.wait(&bars[L::bKEmpty + ks], ((kv / NK) - 1) & 1)) { stop = true; break; }
+          mbar_arrive_expect_tx(&bars[L::bKFull + ks], kTB);
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_4d(sm + L::kK + ks * kTB + c * 16384, &tk, &bars[L::bKFull + ks], c * 64,
+                        n * kTile, w.h, w.b);
+          ++k_issued;
+          if (kv >= NV && !wd.wait(&bars[L::bVEmpty + vs], ((kv / NV) - 1) & 1)) { stop = true; break; }
+          mbar_arrive_expect_tx(&bars[L::bVFull + vs], kTB);
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_4d(sm + L::kV + vs * kTB + c * 16384, &tv, &bars[L::bVFull + vs], c * 64,
+                        n * kTile, w.h, w.b);
+          ++v_issued;
+          ++kv;
+        }
       }
       if (wd.aborted()) {
         // let every issued copy land before the CTA's shared memory goes away
-        for (uint32_t t = (k_issued > NS ? k_issued - NS : 0); t < k_issued; ++t)
-          drain_wait(&bars[L::bKFull + t % NS], (t / NS) & 1);
-        for (uint32_t t = (v_issued > NS ? v_issued - NS : 0); t < v_issued; ++t)
-          drain_wait(&bars[L::bVFull + t % NS], (t / NS) & 1);
-        for (uint32_t t = (q_issued > 2 ? q_issued - 2 : 0); t < q_issued; ++t)
-          drain_wait(&bars[L::bQFull + (t & 1)], (t >> 1) & 1);
+        for (uint32_t t = (k_issued > NK ? k_issued - NK : 0); t < k_issued; ++t)
+          drain_wait(&bars[L::bKFull + t % NK], (t / NK) & 1);
+        for (uint32_t t = (v_issued > NV ? v_issued - NV : 0); t < v_issued; ++t)
+          drain_wait(&bars[L::bVFull + t % NV], (t / NV) & 1);
+        for (int x = 0; x < 2; ++x)
+          if (q_issued[x] > 0) drain_wait(&bars[L::bQFull + x], (q_issued[x] - 1) & 1);
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      uint32_t it = 0, ul = 0;
-      for (int u = blockIdx.x; u < p.n_units; u += gridDim.x) {
-        const int bh = u / nM, m = u % nM, b = bh / p.H;
-        const int rs = p.row_ptr[b * nM + m], re = p.row_ptr[b * nM + m + 1];
-        const int nt = re - rs;
-        if (nt == 0) continue;
-        const int qb = ul & 1, ob = ul & 1;
-        if (!wd.wait(&bars[L::bQFull + qb], (ul >> 1) & 1)) break;
+      uint32_t kv = 0, uq[2] = {0, 0}, tcount[2] = {0, 0};
+      bool stop = false;
+      const uint32_t q_addr[2] = {smem_u32(sm + L::kQ), smem_u32(sm + L::kQ + kTB)};
+      // S_x = Q_x K^T into the S columns of group x.  The previous PV_x still
+      // reads P_x from those columns; tcgen05.mma ops issued by one thread
+      // execute in issue order, so no completion wait is needed in between.
+      auto issue_s = [&](int x, uint32_t kvi) -> bool {
+        if (!wd.wait(&bars[L::bKFull + kvi % NK], (kvi / NK) & 1)) return false;
         tc_fence_after();
-        const uint32_t q_addr = smem_u32(sm + L::kQ + qb * kTB);
-        const uint32_t o_tmem = tmem + 256 + ob * D;
-        bool stop = false;
-        for (int j = 0; j <= nt && !stop; ++j) {
-          if (j < nt) {
-            const uint32_t t = it + j, s = t & 1, st = t % NS;
-            if (!wd.wait(&bars[L::bKFull + st], (t / NS) & 1)) { stop = true; break; }
-            if (t >= 2 && !wd.wait(&bars[L::bSFree + s], ((t >> 1) - 1) & 1)) { stop = true; break; }
-            tc_fence_after();
-            const uint32_t k_addr = smem_u32(sm + L::kK + st * kTB);
+        const uint32_t k_addr = smem_u32(sm + L::kK + (kvi % NK) * kTB);
 #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-              const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-              mma_ss(tmem + s * 128, sw128_desc(q_addr + off, 16, 1024),
-                     sw128_desc(k_addr + off, 16, 1024), kIdescS, kk > 0);
-            }
-            mma_commit(&bars[L::bSFull + s]);
-            mma_commit(&bars[L::bKEmpty + st]);
-          }
-          if (j >= 1) {
-            const uint32_t t = it + j - 1, s = t & 1, st = t % NS;
-            if (j == 1 && ul >= 2 && !wd.wait(&bars[L::bOFree + ob], ((ul >> 1) - 1) & 1)) {
-              stop = true;
-              break;
-            }
-            if (!wd.wait(&bars[L::bVFull + st], (t / NS) & 1)) { stop = true; break; }
-            if (!wd.wait(&bars[L::bPFull + s], (t >> 1) & 1)) { stop = true; break; }
-            tc_fence_after();
-            const uint32_t v_addr = smem_u32(sm + L::kV + st * kTB);
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          mma_ss(tmem + x * 128, sw128_desc(q_addr[x] + off, 16, 1024),
+                 sw128_desc(k_addr + off, 16, 1024), kIdescS, kk > 0);
+        }
+        mma_commit(&bars[L::bSFull + x]);
+        return true;
+      };
+      for (int u = blockIdx.x; u < p.n_units && !stop; u += gridDim.x) {
+        const FwdUnit w = decode_unit(p, u);
+        const bool has[2] = {w.re[0] > w.rs[0], w.re[1] > w.rs[1]};
+        if (!has[0] && !has[1]) continue;
+        for (int x = 0; x < 2; ++x)
+          if (has[x] && !wd.wait(&bars[L::bQFull + x], uq[x] & 1)) stop = true;
+        if (stop) break;
+        bool first[2] = {true, true};
+        UnionWalk uw{p.row_ent, {w.rs[0], w.rs[1]}, {w.re[0], w.re[1]}};
+        int n;
+        bool in_cur[2], in_nxt[2];
+        uw.next(n, in_cur[0], in_cur[1]);
+        uint32_t kv_cur = kv;
+        for (int x = 0; x < 2 && !stop; ++x)
+          if (in_cur[x] && !issue_s(x, kv_cur)) stop = true;
+        if (stop) break;
+        mma_commit(&bars[L::bKEmpty + kv_cur % NK]);
+        for (;;) {
+          const bool more = uw.next(n, in_nxt[0], in_nxt[1]);
+          const uint32_t kv_nxt = kv_cur + 1;
+          if (!wd.wait(&bars[L::bVFull + kv_cur % NV], (kv_cur / NV) & 1)) { stop = true; break; }
+          for (int x = 0; x < 2; ++x) {
+            if (in_cur[x]) {
+              // O_x += P_x V  (P from TMEM over the S columns, V as an MN-major B operand)
+              if (!wd.wait(&bars[L::bPFull + x], tcount[x] & 1)) { stop = true; break; }
+              tc_fence_after();
+              const uint32_t v_addr = smem_u32(sm + L::kV + (kv_cur % NV) * kTB);
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-              mma_ts(o_tmem, tmem + s * 128 + kk * 8, sw128_desc(v_addr + kk * 2048, 16384, 1024),
-                     kIdescPV, (j > 1 || kk > 0) ? 1u : 0u);
+              for (int kk = 0; kk < 8; ++kk)
+                mma_ts(tmem + 256 + x * D, tmem + x * 128 + kk * 8,
+                       sw128_desc(v_addr + kk * 2048, 16384, 1024), kIdescPV,
+                       (!first[x] || kk > 0) ? 1u : 0u);
+              mma_commit(&bars[L::bPVDone + x]);
+              first[x] = false;
+              ++tcount[x];
             }
-            mma_commit(&bars[L::bVEmpty + st]);
-            mma_commit(&bars[L::bSFree + s]);
-            mma_commit(&bars[L::bODone]);
+            // the next S of this group as soon as its P has been consumed
+            if (more && in_nxt[x] && !issue_s(x, kv_nxt)) { stop = true; break; }
           }
+          if (stop) break;
+          mma_commit(&bars[L::bVEmpty + kv_cur % NV]);
+          if (!more) break;
+          mma_commit(&bars[L::bKEmpty + kv_nxt % NK]);
+          kv_cur = kv_nxt;
+          in_cur[0] = in_nxt[0];
+          in_cur[1] = in_nxt[1];
         }
         if (stop) break;
-        mma_commit(&bars[L::bQEmpty + qb]);
-        it += nt;
-        ++ul;
+        kv = kv_cur + 1;
+        for (int x = 0; x < 2; ++x)
+          if (has[x]) {
+            mma_commit(&bars[L::bQEmpty + x]);
+            ++uq[x];
+          }
       }
       // every tcgen05 op this thread issued is complete before TMEM is freed
       mma_commit(&bars[L::bFinal]);
       drain_wait(&bars[L::bFinal], 0);
     }
-  } else {
-    // ------------------------------------------------------------ softmax
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ softmax, group x
+    const int x = (warp - 4) >> 2;  // 0: q-block 2g, 1: q-block 2g+1
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t t_s = tmem + lane_off + x * 128;
+    const uint32_t t_o = tmem + lane_off + 256 + x * D;
     const MaskParams &mk = p.mask;
     const bool use_seg = mk.seg_q != nullptr;
     // every lane waits, then the warp agrees, so tcgen05 .sync.aligned ops
@@ -253,18 +334,19 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
     auto wwait = [&](uint64_t *bar, uint32_t parity) {
       return __all_sync(0xffffffffu, wd.wait(bar, parity)) != 0;
     };
-    uint32_t it = 0, ul = 0, ps = 0;
+    uint32_t tcount = 0, ps = 0;
     bool stop = false;
     for (int u = blockIdx.x; u < p.n_units && !stop; u += gridDim.x) {
-      const int bh = u / nM, m = u % nM, b = bh / p.H, h = bh % p.H;
-      const int rs = p.row_ptr[b * nM + m], re = p.row_ptr[b * nM + m + 1];
-      const int nt = re - rs;
-      const int i = m * kTile + r;
+      const FwdUnit w = decode_unit(p, u);
+      if (w.m[x] >= p.nM) continue;
+      const int rs = w.rs[x], re = w.re[x], nt = re - rs;
+      const int b = w.b, h = w.h, bh = w.bh;
+      const int i = w.m[x] * kTile + r;
       const bool row_ok = i < p.Sq;
-      __nv_bfloat16 *orow = p.out + b * p.o_sb + static_cast<int64_t>(i) * p.o_ss + h * p.o_sh;
-      float *lse_p = p.lse + (static_cast<int64_t>(bh)) * p.Sq + i;
       if (nt == 0) {
         if (row_ok) {
+          __nv_bfloat16 *orow = p.out + b * p.o_sb + static_cast<int64_t>(i) * p.o_ss + h * p.o_sh;
+          float *lse_p = p.lse + static_cast<int64_t>(bh) * p.Sq + i;
           const int4 z = make_int4(0, 0, 0, 0);
 #pragma unroll
           for (int c = 0; c < D / 8; ++c) reinterpret_cast<int4 *>(orow)[c] = z;
@@ -272,10 +354,10 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
         }
         continue;
       }
-      const int ob = ul & 1;
       const bool fixed = p.fixed_mode && p.gate[bh] != 0;
       float m_ref = -INFINITY, l = 0.f, l_r = 0.f;
-      if (fixed) m_ref = row_ok ? p.scale_log2 * p.qnorm[static_cast<int64_t>(bh) * p.Sq + i] * p.kmax[bh] : 0.f;
+      if (fixed)
+        m_ref = row_ok ? p.scale_log2 * p.qnorm[static_cast<int64_t>(bh) * p.Sq + i] * p.kmax[bh] : 0.f;
       // row-constant part of the mask: allowed keys lie in [lo, hi]
       int lo = 0, hi = p.Skv - 1;
       if (mk.flags & BSA_MASK_CAUSAL_WINDOW) {
@@ -285,58 +367,55 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       if (mk.flags & BSA_MASK_KV_VALID_LEN) hi = min(hi, mk.kv_valid_len[b] - 1);
       const int seg_i = (use_seg && row_ok) ? mk.seg_q[static_cast<int64_t>(b) * p.Sq + i] : INT_MIN;
 
-      for (int j = 0; j < nt; ++j, ++it) {
-        const uint32_t ent = p.row_ent[rs + j];
+      for (int j = rs; j < re; ++j, ++tcount) {
+        const uint32_t ent = p.row_ent[j];
         const int n = static_cast<int>(ent & kIndexMask);
         const bool full = (ent & kFullBit) != 0;
-        const uint32_t s = it & 1;
-        // segment-id equality of this row against the tile's 128 keys, as a
-        // 128-bit mask built before the S row occupies registers
-        uint32_t seg_ok[4] = {~0u, ~0u, ~0u, ~0u};
-        if (!full && use_seg) {
-          int32_t *segt = seg_sm + (ps & 1) * kTile;
-          const int jj = n * kTile + r;
-          segt[r] = jj < p.Skv ? mk.seg_kv[static_cast<int64_t>(b) * p.Skv + jj] : INT_MIN + 1;
-          mbar_arrive(&bars[L::bSegReady + (ps & 1)]);
-          if (!wwait(&bars[L::bSegReady + (ps & 1)], (ps >> 1) & 1)) { stop = true; break; }
-          ++ps;
-          const int4 *seg4 = reinterpret_cast<const int4 *>(segt);
-#pragma unroll
-          for (int w = 0; w < 4; ++w) {
-            uint32_t bits = 0;
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-              const int4 v = seg4[w * 8 + q];
-              bits |= (static_cast<uint32_t>(v.x == seg_i) << (4 * q)) |
-                      (static_cast<uint32_t>(v.y == seg_i) << (4 * q + 1)) |
-                      (static_cast<uint32_t>(v.z == seg_i) << (4 * q + 2)) |
-                      (static_cast<uint32_t>(v.w == seg_i) << (4 * q + 3));
-            }
-            seg_ok[w] = bits;
-          }
-        }
-        if (!wwait(&bars[L::bSFull + s], (it >> 1) & 1)) { stop = true; break; }
-        tc_fence_after();
-        uint32_t x[128];
-        const uint32_t t_s = tmem + lane_off + s * 128;
-        tmem_ld32(t_s + 0, *reinterpret_cast<uint32_t(*)[32]>(&x[0]));
-        tmem_ld32(t_s + 32, *reinterpret_cast<uint32_t(*)[32]>(&x[32]));
-        tmem_ld32(t_s + 64, *reinterpret_cast<uint32_t(*)[32]>(&x[64]));
-        tmem_ld32(t_s + 96, *reinterpret_cast<uint32_t(*)[32]>(&x[96]));
-        tmem_wait_ld();
-        float *f = reinterpret_cast<float *>(x);
+        // allowed-key bits of this tile for this row (range AND segment ids),
+        // built before the S row occupies registers
+        uint32_t allow[4] = {~0u, ~0u, ~0u, ~0u};
         if (!full) {
-          const int c_lo = lo - n * kTile, c_hi = hi - n * kTile;
 #pragma unroll
-          for (int c = 0; c < 128; ++c) {
-            const bool ok = c >= c_lo && c <= c_hi && ((seg_ok[c >> 5] >> (c & 31)) & 1u);
-            f[c] = ok ? f[c] : -INFINITY;
+          for (int q = 0; q < 4; ++q) allow[q] = range_bits(lo - n * kTile, hi - n * kTile, q);
+          if (use_seg) {
+            int32_t *segt = seg_sm + (x * 2 + (ps & 1)) * kTile;
+            const int jj = n * kTile + r;
+            segt[r] = jj < p.Skv ? mk.seg_kv[static_cast<int64_t>(b) * p.Skv + jj] : INT_MIN + 1;
+            mbar_arrive(&bars[L::bSegReady + x * 2 + (ps & 1)]);
+            if (!wwait(&bars[L::bSegReady + x * 2 + (ps & 1)], (ps >> 1) & 1)) { stop = true; break; }
+            ++ps;
+            const int4 *seg4 = reinterpret_cast<const int4 *>(segt);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              uint32_t bits = 0;
+#pragma unroll
+              for (int t = 0; t < 8; ++t) {
+                const int4 v = seg4[q * 8 + t];
+                bits |= (static_cast<uint32_t>(v.x == seg_i) << (4 * t)) |
+                        (static_cast<uint32_t>(v.y == seg_i) << (4 * t + 1)) |
+                        (static_cast<uint32_t>(v.z == seg_i) << (4 * t + 2)) |
+                        (static_cast<uint32_t>(v.w == seg_i) << (4 * t + 3));
+              }
+              allow[q] &= bits;
+            }
           }
         }
+        if (!wwait(&bars[L::bSFull + x], tcount & 1)) { stop = true; break; }
+        tc_fence_after();
         if (!fixed) {
+          // pass 1: the tile's row max (masked)
           float mx = -INFINITY;
 #pragma unroll
-          for (int c = 0; c < 128; ++c) mx = fmaxf(mx, f[c]);
+          for (int c = 0; c < 4; ++c) {
+            uint32_t sv[32];
+            tmem_ld32(t_s + 32 * c, sv);
+            tmem_wait_ld();
+#pragma unroll
+            for (int q = 0; q < 32; ++q) {
+              const float v = ((allow[c] >> q) & 1u) ? __uint_as_float(sv[q]) : -INFINITY;
+              mx = fmaxf(mx, v);
+            }
+          }
           const float mt = mx * p.scale_log2;
           const bool need = mt > m_ref + kRescaleThreshold;
           const bool resc = need && l > 0.f;
@@ -348,10 +427,9 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
             m_ref = mt;
           }
           if (__any_sync(0xffffffffu, resc)) {
-            if (!wwait(&bars[L::bODone], (it - 1) & 1)) { stop = true; break; }
+            if (!wwait(&bars[L::bPVDone + x], (tcount - 1) & 1)) { stop = true; break; }
             tc_fence_after();
             const float a = resc ? alpha : 1.f;
-            const uint32_t t_o = tmem + lane_off + 256 + ob * D;
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
               uint32_t o[32];
@@ -364,58 +442,65 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
             tmem_wait_st();
           }
         }
+        // pass 2: P = exp2(s * scale * log2e - m) in bf16, packed over the first 64 S columns
         const float mu = (m_ref == -INFINITY) ? 0.f : m_ref;
         float rowsum = 0.f, rowsum_r = 0.f;
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          uint32_t pk[32];
+        for (int c = 0; c < 4; ++c) {
+          uint32_t sv[32];
+          tmem_ld32(t_s + 32 * c, sv);
+          tmem_wait_ld();
+          uint32_t pk[16];
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const float p0 = fast_exp2(fmaf(f[64 * half + 2 * c], p.scale_log2, -mu));
-            const float p1 = fast_exp2(fmaf(f[64 * half + 2 * c + 1], p.scale_log2, -mu));
-            pk[c] = pack_bf16x2(p0, p1);
+          for (int q = 0; q < 16; ++q) {
+            float p0 = fast_exp2(fmaf(__uint_as_float(sv[2 * q]), p.scale_log2, -mu));
+            float p1 = fast_exp2(fmaf(__uint_as_float(sv[2 * q + 1]), p.scale_log2, -mu));
+            if (!full) {
+              p0 = ((allow[c] >> (2 * q)) & 1u) ? p0 : 0.f;
+              p1 = ((allow[c] >> (2 * q + 1)) & 1u) ? p1 : 0.f;
+            }
+            pk[q] = pack_bf16x2(p0, p1);
             // two row sums: l over the exact weights (for LSE) and l_r over the
             // bf16-rounded weights the PV product uses (normalising O by l_r
             // makes numerator and denominator carry the same rounding)
             rowsum += p0 + p1;
-            rowsum_r += __uint_as_float(pk[c] << 16) + __uint_as_float(pk[c] & 0xffff0000u);
+            rowsum_r += __uint_as_float(pk[q] << 16) + __uint_as_float(pk[q] & 0xffff0000u);
           }
-          // P (bf16 pairs) overwrites the first 64 columns of this S buffer
-          tmem_st32(t_s + 32 * half, pk);
+          // P chunk c -> TMEM columns [16c, 16c+16): only S columns already read
+          tmem_st16(t_s + 16 * c, pk);
         }
         l += rowsum;
         l_r += rowsum_r;
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&bars[L::bPFull + s]);
+        mbar_arrive(&bars[L::bPFull + x]);
       }
       if (stop) break;
-      // epilogue: O / l -> bf16, LSE
-      if (!wwait(&bars[L::bODone], (it - 1) & 1)) break;
+      // epilogue: O / l_r -> bf16, LSE
+      if (!wwait(&bars[L::bPVDone + x], (tcount - 1) & 1)) break;
       tc_fence_after();
       const float inv = l_r > 0.f ? 1.f / l_r : 0.f;
-      const uint32_t t_o = tmem + lane_off + 256 + ob * D;
+      __nv_bfloat16 *orow = p.out + b * p.o_sb + static_cast<int64_t>(i) * p.o_ss + h * p.o_sh;
+      float *lse_p = p.lse + static_cast<int64_t>(bh) * p.Sq + i;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t o[32];
-        tmem_ld32(t_o + c * 32, o);
+      for (int c = 0; c < D / 16; ++c) {
+        uint32_t o[16];
+        tmem_ld16(t_o + c * 16, o);
         tmem_wait_ld();
         if (row_ok) {
-          uint32_t w[16];
+          uint32_t wv[8];
 #pragma unroll
-          for (int q = 0; q < 16; ++q)
-            w[q] = pack_bf16x2(__uint_as_float(o[2 * q]) * inv, __uint_as_float(o[2 * q + 1]) * inv);
-          int4 *dst = reinterpret_cast<int4 *>(orow + c * 32);
-#pragma unroll
-          for (int q = 0; q < 4; ++q) dst[q] = make_int4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+          for (int q = 0; q < 8; ++q)
+            wv[q] = pack_bf16x2(__uint_as_float(o[2 * q]) * inv, __uint_as_float(o[2 * q + 1]) * inv);
+          int4 *dst = reinterpret_cast<int4 *>(orow + c * 16);
+          dst[0] = make_int4(wv[0], wv[1], wv[2], wv[3]);
+          dst[1] = make_int4(wv[4], wv[5], wv[6], wv[7]);
         }
       }
       tc_fence_before();
-      mbar_arrive(&bars[L::bOFree + ob]);
       if (row_ok) *lse_p = l > 0.f ? (m_ref + __log2f(l)) * kLn2 : -INFINITY;
       if (fixed && l > 0.f && l < 7.888609052210118e-31f /* 2^-100 */)
         atomicAdd(p.hdr + kHdrGateWarn, 1u);
-      ++ul;
     }
   }
 
@@ -516,19 +601,20 @@ int sm_count() {
   return n;
 }
 
-template <int D, int NS>
+template <int D, int NK, int NV>
 cudaError_t run_fwd(const FwdParams &fp, const CUtensorMap &tq, const CUtensorMap &tk,
                     const CUtensorMap &tv, cudaStream_t s) {
-  using L = FwdSmem<D, NS>;
+  using L = FwdSmem<D, NK, NV>;
+  static_assert(L::kAlloc <= 232448, "shared memory budget");
   static bool attr = false;
   if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(k_attn_fwd<D, NS>,
+    cudaError_t e = cudaFuncSetAttribute(k_attn_fwd<D, NK, NV>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
     if (e != cudaSuccess) return e;
     attr = true;
   }
   const int grid = std::min(fp.n_units, sm_count());
-  k_attn_fwd<D, NS><<<grid, 192, L::kAlloc, s>>>(tq, tk, tv, fp);
+  k_attn_fwd<D, NK, NV><<<grid, 384, L::kAlloc, s>>>(tq, tk, tv, fp);
   count_launch();
   return cudaGetLastError();
 }
@@ -570,7 +656,7 @@ cudaError_t launch_fwd(const bsa_problem &p, const MaskParams &mp, const bsa_opt
   fp.Sq = p.Sq;
   fp.Skv = p.Skv;
   fp.nM = L.nM;
-  fp.n_units = p.B * p.H * L.nM;
+  fp.n_units = p.B * p.H * ((L.nM + 1) / 2);
   fp.scale = p.scale;
   fp.scale_log2 = p.scale * kLog2e;
   fp.row_ptr = reinterpret_cast<const int32_t *>(ws + L.row_ptr);
@@ -588,8 +674,8 @@ cudaError_t launch_fwd(const bsa_problem &p, const MaskParams &mp, const bsa_opt
   fp.timeout_ns = 2000000000ull;
   for (int i = 0; i < 7; ++i) fp.sig[i] = sig.w[i];
   fp.sig_mask = 0x7Fu & ~(1u << 5);  // the forward does not depend on the kv-column order
-  if (p.D == 64) return run_fwd<64, 3>(fp, tq, tk, tv, s);
-  return run_fwd<128, 2>(fp, tq, tk, tv, s);
+  if (p.D == 64) return run_fwd<64, 4, 4>(fp, tq, tk, tv, s);
+  return run_fwd<128, 3, 2>(fp, tq, tk, tv, s);
 }
 
 }  // namespace bsa
