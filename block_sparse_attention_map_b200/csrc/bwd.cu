@@ -262,7 +262,8 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
           const uint32_t qs = ec % NQ, ds = ec % NDO;
           const bool first = e == k.es, last = e == k.ee - 1;
           if (!wd.wait(&bars[L::bQFull + qs], (ec / NQ) & 1)) { stop = true; break; }
-          if (ec >= 1 && !wd.wait(&bars[L::bDVDone], (ec - 1) & 1)) { stop = true; break; }
+          // S^T overwrites the columns dV(e-1) read P^T from: tcgen05.mma ops
+          // issued by one thread execute in issue order, so no wait in between
           tc_fence_after();
           const uint32_t q_addr = smem_u32(sm + L::kQ + qs * kTB);
           const uint32_t do_addr = smem_u32(sm + L::kDO + ds * kTB);
@@ -293,7 +294,6 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
             mma_ts(T_DV, T_S + kk * 8, sw128_desc(do_addr + kk * 2048, 16384, 1024), kIdKV,
                    (!first || kk > 0) ? 1u : 0u);
           mma_commit(&bars[L::bDOEmpty + ds]);
-          mma_commit(&bars[L::bDVDone]);
           // dK += dS^T Q_m
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
@@ -369,44 +369,49 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
         const uint32_t ent = p.col_ent[e];
         const int m = static_cast<int>(ent & kIndexMask);
         const bool full = (ent & kFullBit) != 0;
-        // stage LSE (log2 units; +inf where the row has no key or lies past Sq),
-        // Delta and the query segment ids of this q-block
+        // stage LSE, Delta and the query segment ids of this q-block
         {
           const int i = m * kTile + r;
           float* vl = vec_lse + (ec & 1) * kTile;
           float* vd = vec_delta + (ec & 1) * kTile;
           int32_t* vs = vec_seg + (ec & 1) * kTile;
-          float l2 = INFINITY;
+          // stored negated so that the element loop is one packed FMA / add:
+          // -LSE*log2e (-inf where the row has no key or lies past Sq) and -Delta
+          float nl2 = -INFINITY;
           if (i < p.Sq) {
             const float lv = p.lse[static_cast<int64_t>(k.bh) * p.Sq + i];
-            if (lv != -INFINITY) l2 = lv * kLog2e;
+            if (lv != -INFINITY) nl2 = -lv * kLog2e;
           }
-          vl[r] = l2;
-          vd[r] = p.delta[static_cast<int64_t>(k.bh) * p.nM * kTile + i];
+          vl[r] = nl2;
+          vd[r] = -p.delta[static_cast<int64_t>(k.bh) * p.nM * kTile + i];
           if (use_seg) vs[r] = i < p.Sq ? mk.seg_q[static_cast<int64_t>(k.b) * p.Sq + i] : INT_MIN + 1;
           mbar_arrive(&bars[L::bVecReady + (ec & 1)]);
         }
         if (!wwait(&bars[L::bVecReady + (ec & 1)], (ec >> 1) & 1)) { stop = true; break; }
         const float *vl = vec_lse + (ec & 1) * kTile;
         const float *vd = vec_delta + (ec & 1) * kTile;
-        uint32_t seg_ok[4] = {~0u, ~0u, ~0u, ~0u};
-        if (!full && use_seg) {
-          const int4 *seg4 = reinterpret_cast<const int4 *>(vec_seg + (ec & 1) * kTile);
+        // allowed-query bits of this tile for this key row (range AND segment ids)
+        uint32_t allow[4] = {~0u, ~0u, ~0u, ~0u};
+        if (!full) {
 #pragma unroll
-          for (int w = 0; w < 4; ++w) {
-            uint32_t bits = 0;
+          for (int w = 0; w < 4; ++w) allow[w] = range_bits(qlo - m * kTile, qhi - m * kTile, w);
+          if (use_seg) {
+            const int4 *seg4 = reinterpret_cast<const int4 *>(vec_seg + (ec & 1) * kTile);
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-              const int4 v = seg4[w * 8 + q];
-              bits |= (static_cast<uint32_t>(v.x == seg_j) << (4 * q)) |
-                      (static_cast<uint32_t>(v.y == seg_j) << (4 * q + 1)) |
-                      (static_cast<uint32_t>(v.z == seg_j) << (4 * q + 2)) |
-                      (static_cast<uint32_t>(v.w == seg_j) << (4 * q + 3));
+            for (int w = 0; w < 4; ++w) {
+              uint32_t bits = 0;
+#pragma unroll
+              for (int q = 0; q < 8; ++q) {
+                const int4 v = seg4[w * 8 + q];
+                bits |= (static_cast<uint32_t>(v.x == seg_j) << (4 * q)) |
+                        (static_cast<uint32_t>(v.y == seg_j) << (4 * q + 1)) |
+                        (static_cast<uint32_t>(v.z == seg_j) << (4 * q + 2)) |
+                        (static_cast<uint32_t>(v.w == seg_j) << (4 * q + 3));
+              }
+              allow[w] &= bits;
             }
-            seg_ok[w] = bits;
           }
         }
-        const int c_lo = qlo - m * kTile, c_hi = qhi - m * kTile;
         if (!wwait(&bars[L::bSdPFull], ec & 1)) { stop = true; break; }
         if (ec >= 1 && !wwait(&bars[L::bDSFree], (ec - 1) & 1)) { stop = true; break; }
         tc_fence_after();
@@ -417,22 +422,30 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
           tmem_ld32(T_DP + lane_off + 32 * c, dp);
           tmem_wait_ld();
           uint32_t pk[16], dk2[16];
+          const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
 #pragma unroll
-          for (int q = 0; q < 16; ++q) {
-            float pr[2], dsv[2];
+          for (int q4 = 0; q4 < 8; ++q4) {
+            // four query columns: their -LSE and -Delta as one broadcast load each
+            const float4 nl4 = reinterpret_cast<const float4 *>(vl)[8 * c + q4];
+            const float4 nd4 = reinterpret_cast<const float4 *>(vd)[8 * c + q4];
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
-              const int col = 32 * c + 2 * q + u;
-              float pv = fast_exp2(fmaf(__uint_as_float(s[2 * q + u]), p.scale_log2, -vl[col]));
+            for (int h2 = 0; h2 < 2; ++h2) {
+              const int e0 = 4 * q4 + 2 * h2;  // element index in this 32-column chunk
+              const float2 nl = h2 ? make_float2(nl4.z, nl4.w) : make_float2(nl4.x, nl4.y);
+              const float2 nd = h2 ? make_float2(nd4.z, nd4.w) : make_float2(nd4.x, nd4.y);
+              const float2 t = __ffma2_rn(
+                  make_float2(__uint_as_float(s[e0]), __uint_as_float(s[e0 + 1])), sc2, nl);
+              float p0 = fast_exp2(t.x), p1 = fast_exp2(t.y);
               if (!full) {
-                const bool ok = col >= c_lo && col <= c_hi && ((seg_ok[col >> 5] >> (col & 31)) & 1u);
-                pv = ok ? pv : 0.f;
+                p0 = ((allow[c] >> e0) & 1u) ? p0 : 0.f;
+                p1 = ((allow[c] >> (e0 + 1)) & 1u) ? p1 : 0.f;
               }
-              pr[u] = pv;
-              dsv[u] = pv * (__uint_as_float(dp[2 * q + u]) - vd[col]);
+              const float2 dd = __fadd2_rn(
+                  make_float2(__uint_as_float(dp[e0]), __uint_as_float(dp[e0 + 1])), nd);
+              const float2 ds = __fmul2_rn(make_float2(p0, p1), dd);
+              pk[e0 >> 1] = pack_bf16x2(p0, p1);
+              dk2[e0 >> 1] = pack_bf16x2(ds.x, ds.y);
             }
-            pk[q] = pack_bf16x2(pr[0], pr[1]);
-            dk2[q] = pack_bf16x2(dsv[0], dsv[1]);
           }
           // P^T chunk -> TMEM columns [16c, 16c+16) of the S^T region
           tmem_st16(T_S + lane_off + 16 * c, pk);

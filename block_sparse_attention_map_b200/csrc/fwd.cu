@@ -124,15 +124,6 @@ struct UnionWalk {
   }
 };
 
-// Allowed-key bits of columns 32w .. 32w+31 that fall inside [lo, hi].
-__device__ __forceinline__ uint32_t range_bits(int lo, int hi, int w) {
-  const int a = max(lo - 32 * w, 0), z = min(hi - 32 * w, 31);
-  if (a > z) return 0u;
-  const uint32_t top = (z >= 31) ? 0xffffffffu : ((1u << (z + 1)) - 1u);
-  const uint32_t bot = (a <= 0) ? 0xffffffffu : ~((1u << a) - 1u);
-  return top & bot;
-}
-
 template <int D, int NK, int NV>
 __global__ void __launch_bounds__(384, 1)
 k_attn_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
@@ -444,7 +435,8 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
         }
         // pass 2: P = exp2(s * scale * log2e - m) in bf16, packed over the first 64 S columns
         const float mu = (m_ref == -INFINITY) ? 0.f : m_ref;
-        float rowsum = 0.f, rowsum_r = 0.f;
+        const float2 sc2 = make_float2(p.scale_log2, p.scale_log2), nmu = make_float2(-mu, -mu);
+        float2 rs2 = make_float2(0.f, 0.f), rr2 = make_float2(0.f, 0.f);
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint32_t sv[32];
@@ -453,8 +445,9 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
           uint32_t pk[16];
 #pragma unroll
           for (int q = 0; q < 16; ++q) {
-            float p0 = fast_exp2(fmaf(__uint_as_float(sv[2 * q]), p.scale_log2, -mu));
-            float p1 = fast_exp2(fmaf(__uint_as_float(sv[2 * q + 1]), p.scale_log2, -mu));
+            const float2 t = __ffma2_rn(
+                make_float2(__uint_as_float(sv[2 * q]), __uint_as_float(sv[2 * q + 1])), sc2, nmu);
+            float p0 = fast_exp2(t.x), p1 = fast_exp2(t.y);
             if (!full) {
               p0 = ((allow[c] >> (2 * q)) & 1u) ? p0 : 0.f;
               p1 = ((allow[c] >> (2 * q + 1)) & 1u) ? p1 : 0.f;
@@ -463,12 +456,14 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
             // two row sums: l over the exact weights (for LSE) and l_r over the
             // bf16-rounded weights the PV product uses (normalising O by l_r
             // makes numerator and denominator carry the same rounding)
-            rowsum += p0 + p1;
-            rowsum_r += __uint_as_float(pk[q] << 16) + __uint_as_float(pk[q] & 0xffff0000u);
+            rs2 = __fadd2_rn(rs2, make_float2(p0, p1));
+            rr2 = __fadd2_rn(rr2, make_float2(__uint_as_float(pk[q] << 16),
+                                              __uint_as_float(pk[q] & 0xffff0000u)));
           }
           // P chunk c -> TMEM columns [16c, 16c+16): only S columns already read
           tmem_st16(t_s + 16 * c, pk);
         }
+        const float rowsum = rs2.x + rs2.y, rowsum_r = rr2.x + rr2.y;
         l += rowsum;
         l_r += rowsum_r;
         tmem_wait_st();

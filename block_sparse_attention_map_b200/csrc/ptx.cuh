@@ -263,6 +263,15 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t *>(&v);
 }
 
+// Bits of the 32 columns 32w .. 32w+31 (of a 128-column tile) that fall inside [lo, hi].
+__device__ __forceinline__ uint32_t range_bits(int lo, int hi, int w) {
+  const int a = max(lo - 32 * w, 0), z = min(hi - 32 * w, 31);
+  if (a > z) return 0u;
+  const uint32_t top = (z >= 31) ? 0xffffffffu : ((1u << (z + 1)) - 1u);
+  const uint32_t bot = (a <= 0) ? 0xffffffffu : ~((1u << a) - 1u);
+  return top & bot;
+}
+
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
