@@ -62,18 +62,18 @@ struct BwdSmem {
   static constexpr int kDS = kV + kTB;           // dS^T, 128 x 128 bf16
   static constexpr int kQ = kDS + 32768;
   static constexpr int kDO = kQ + NQ * kTB;
-  static constexpr int kVec = kDO + NDO * kTB;   // lse[2][128], delta[2][128], segq[2][128]
-  static constexpr int kTk = kVec + 3 * 2 * kTile * 4;  // ticket ring int[2]
+  static constexpr int kVec = kDO + NDO * kTB;   // -LSE*log2e [2][128], -Delta [2][128]
+  static constexpr int kTk = kVec + 2 * 2 * kTile * 4;  // ticket ring int[2]
   static constexpr int kBar = kTk + 16;
   static constexpr int bTkFull = 0, bTkEmpty = 2, bKVFull = 4, bKVFree = 5, bQFull = 6,
                        bQEmpty = bQFull + NQ, bDOFull = bQEmpty + NQ, bDOEmpty = bDOFull + NDO,
-                       bSdPFull = bDOEmpty + NDO, bPdSReady = bSdPFull + 1, bDVDone = bPdSReady + 1,
-                       bDSFree = bDVDone + 1, bDQFull = bDSFree + 1, bDQFree = bDQFull + 1,
-                       bDKVFull = bDQFree + 1, bDKVFree = bDKVFull + 1, bVecReady = bDKVFree + 1,
-                       bDQAdded = bVecReady + 2, bFinal = bDQAdded + 2, kNumBars = bFinal + 1;
+                       bSFull = bDOEmpty + NDO, bDPFull = bSFull + 1, bPReady = bDPFull + 1,
+                       bDSReady = bPReady + 1, bDSFree = bDSReady + 1, bDQFull = bDSFree + 1,
+                       bDQFree = bDQFull + 1, bDKVFull = bDQFree + 1, bDKVFree = bDKVFull + 1,
+                       bVecReady = bDKVFree + 1, bDQAdded = bVecReady + 2, bFinal = bDQAdded + 2,
+                       kNumBars = bFinal + 1;
   static constexpr int kMisc = kBar + kNumBars * 8;
-  static constexpr int kBytes = kMisc + 16;
-  static constexpr int kAlloc = kBytes + 1024;
+  static constexpr int kAlloc = kMisc + 16;
 };
 
 constexpr int kConsumersPerTicket = 1 + 4 + 4;  // MMA lane, compute warps, dQ warps
@@ -130,16 +130,13 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
            const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo,
            const BwdParams p) {
   using L = BwdSmem<D, NQ, NDO>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                            ~static_cast<uintptr_t>(1023));
+  extern __shared__ __align__(1024) uint8_t sm[];
   uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::kBar);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::kMisc);
   int *abort_flag = reinterpret_cast<int *>(sm + L::kMisc + 4);
   volatile int *tk_ring = reinterpret_cast<volatile int *>(sm + L::kTk);
-  float *vec_lse = reinterpret_cast<float *>(sm + L::kVec);          // [2][128]
-  float *vec_delta = vec_lse + 2 * kTile;                             // [2][128]
-  int32_t *vec_seg = reinterpret_cast<int32_t *>(vec_delta + 2 * kTile);  // [2][128]
+  float *vec_nl = reinterpret_cast<float *>(sm + L::kVec);  // [2][128] -LSE*log2e
+  float *vec_nd = vec_nl + 2 * kTile;                        // [2][128] -Delta
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr int kTB = L::kTB;
@@ -148,8 +145,8 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
     for (int i = 0; i < L::kNumBars; ++i) {
       uint32_t cnt = 1;
       if (i == L::bTkEmpty || i == L::bTkEmpty + 1) cnt = kConsumersPerTicket;
-      if (i == L::bPdSReady || i == L::bDQFree || i == L::bDKVFree || i == L::bVecReady ||
-          i == L::bVecReady + 1)
+      if (i == L::bPReady || i == L::bDSReady || i == L::bDQFree || i == L::bDKVFree ||
+          i == L::bVecReady || i == L::bVecReady + 1)
         cnt = 128;
       if (i == L::bDQAdded || i == L::bDQAdded + 1) cnt = 4;
       mbar_init(&bars[i], cnt);
@@ -178,6 +175,8 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
     bool ok = h[kHdrMagic] == kPlanMagic;
     for (int i = 0; i < 7; ++i) ok = ok && (!((p.sig_mask >> i) & 1u) || h[kHdrB + i] == p.sig[i]);
     if (!ok) wd.trip(BSA_ERR_PLAN_MISMATCH);
+    // the swizzled tiles rely on a 1024-byte aligned dynamic shared window
+    if ((smem_u32(sm) & 1023u) != 0u) wd.trip(BSA_ERR_UNSUPPORTED);
   }
   __syncthreads();
 
@@ -210,14 +209,8 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
             tma_load_4d(sm + L::kQ + qs * kTB + c * 16384, &tq, &bars[L::bQFull + qs], c * 64,
                         m * kTile, k.h, k.b);
           ++q_issued;
-          if (ec >= NDO && !wd.wait(&bars[L::bDOEmpty + ds], ((ec / NDO) - 1) & 1)) { stop = true; break; }
-          mbar_arrive_expect_tx(&bars[L::bDOFull + ds], kTB);
-          for (int c = 0; c < D / 64; ++c)
-            tma_load_4d(sm + L::kDO + ds * kTB + c * 16384, &tdo, &bars[L::bDOFull + ds], c * 64,
-                        m * kTile, k.h, k.b);
-          ++do_issued;
           if (e == k.es) {
-            // K_n, V_n after the first Q/dO so those loads overlap the previous
+            // K_n, V_n after the first Q so that load overlaps the previous
             // column's last MMAs
             if (cc >= 1 && !wd.wait(&bars[L::bKVFree], (cc - 1) & 1)) { stop = true; break; }
             mbar_arrive_expect_tx(&bars[L::bKVFull], 2 * kTB);
@@ -229,6 +222,12 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
             }
             ++kv_issued;
           }
+          if (ec >= NDO && !wd.wait(&bars[L::bDOEmpty + ds], ((ec / NDO) - 1) & 1)) { stop = true; break; }
+          mbar_arrive_expect_tx(&bars[L::bDOFull + ds], kTB);
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_4d(sm + L::kDO + ds * kTB + c * 16384, &tdo, &bars[L::bDOFull + ds], c * 64,
+                        m * kTile, k.h, k.b);
+          ++do_issued;
         }
         if (stop) break;
         ++cc;
@@ -243,8 +242,44 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
+    // Per entry e: dV(e), S^T(e+1), dK(e), dQ(e), dP^T(e+1).  S^T(e+1) reuses the
+    // columns dV(e) reads P^T from: tcgen05.mma ops issued by one thread run in
+    // issue order, so it follows dV(e) without a wait and the next entry's
+    // exponentials overlap this entry's dK and dQ.
     if (lane == 0) {
       uint32_t tc = 0, cc = 0, ec = 0;
+      const uint32_t k_addr = smem_u32(sm + L::kK), v_addr = smem_u32(sm + L::kV);
+      const uint32_t ds_addr = smem_u32(sm + L::kDS);
+      auto issue_s = [&](uint32_t e_idx) -> bool {  // S^T = K_n Q_m^T
+        const uint32_t qs = e_idx % NQ;
+        if (!wd.wait(&bars[L::bQFull + qs], (e_idx / NQ) & 1)) return false;
+        tc_fence_after();
+        const uint32_t q_addr = smem_u32(sm + L::kQ + qs * kTB);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          mma_ss(T_S, sw128_desc(k_addr + off, 16, 1024), sw128_desc(q_addr + off, 16, 1024),
+                 kIdS, kk > 0);
+        }
+        mma_commit(&bars[L::bSFull]);
+        return true;
+      };
+      auto issue_dp = [&](uint32_t e_idx) -> bool {  // dP^T = V_n dO_m^T
+        const uint32_t ds = e_idx % NDO;
+        if (!wd.wait(&bars[L::bDOFull + ds], (e_idx / NDO) & 1)) return false;
+        // the dQ of the previous entry occupies these columns until read out
+        if (e_idx >= 1 && !wd.wait(&bars[L::bDQFree], (e_idx - 1) & 1)) return false;
+        tc_fence_after();
+        const uint32_t do_addr = smem_u32(sm + L::kDO + ds * kTB);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          mma_ss(T_DP, sw128_desc(v_addr + off, 16, 1024), sw128_desc(do_addr + off, 16, 1024),
+                 kIdS, kk > 0);
+        }
+        mma_commit(&bars[L::bDPFull]);
+        return true;
+      };
       for (;; ++tc) {
         const uint32_t slot = tc & 1;
         if (!wd.wait(&bars[L::bTkFull + slot], (tc >> 1) & 1)) break;
@@ -254,47 +289,25 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
         if (!k.valid) break;
         if (k.ee == k.es) continue;
         if (!wd.wait(&bars[L::bKVFull], cc & 1)) break;
-        tc_fence_after();
-        const uint32_t k_addr = smem_u32(sm + L::kK), v_addr = smem_u32(sm + L::kV);
-        const uint32_t ds_addr = smem_u32(sm + L::kDS);
-        bool stop = false;
-        for (int e = k.es; e < k.ee; ++e, ++ec) {
+        bool stop = !issue_s(ec) || !issue_dp(ec);
+        for (int e = k.es; e < k.ee && !stop; ++e, ++ec) {
           const uint32_t qs = ec % NQ, ds = ec % NDO;
           const bool first = e == k.es, last = e == k.ee - 1;
-          if (!wd.wait(&bars[L::bQFull + qs], (ec / NQ) & 1)) { stop = true; break; }
-          // S^T overwrites the columns dV(e-1) read P^T from: tcgen05.mma ops
-          // issued by one thread execute in issue order, so no wait in between
-          tc_fence_after();
-          const uint32_t q_addr = smem_u32(sm + L::kQ + qs * kTB);
-          const uint32_t do_addr = smem_u32(sm + L::kDO + ds * kTB);
-          // S^T = K_n Q_m^T
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-            mma_ss(T_S, sw128_desc(k_addr + off, 16, 1024), sw128_desc(q_addr + off, 16, 1024),
-                   kIdS, kk > 0);
-          }
-          if (!wd.wait(&bars[L::bDOFull + ds], (ec / NDO) & 1)) { stop = true; break; }
-          if (ec >= 1 && !wd.wait(&bars[L::bDQFree], (ec - 1) & 1)) { stop = true; break; }
-          tc_fence_after();
-          // dP^T = V_n dO_m^T
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-            mma_ss(T_DP, sw128_desc(v_addr + off, 16, 1024), sw128_desc(do_addr + off, 16, 1024),
-                   kIdS, kk > 0);
-          }
-          mma_commit(&bars[L::bSdPFull]);
-          if (!wd.wait(&bars[L::bPdSReady], ec & 1)) { stop = true; break; }
+          if (!wd.wait(&bars[L::bPReady], ec & 1)) { stop = true; break; }
           if (first && cc >= 1 && !wd.wait(&bars[L::bDKVFree], (cc - 1) & 1)) { stop = true; break; }
           tc_fence_after();
           // dV += P^T dO_m   (P^T from TMEM, dO as an MN-major B operand)
+          const uint32_t do_addr = smem_u32(sm + L::kDO + ds * kTB);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
             mma_ts(T_DV, T_S + kk * 8, sw128_desc(do_addr + kk * 2048, 16384, 1024), kIdKV,
                    (!first || kk > 0) ? 1u : 0u);
           mma_commit(&bars[L::bDOEmpty + ds]);
+          if (!last && !issue_s(ec + 1)) { stop = true; break; }
+          if (!wd.wait(&bars[L::bDSReady], ec & 1)) { stop = true; break; }
+          tc_fence_after();
           // dK += dS^T Q_m
+          const uint32_t q_addr = smem_u32(sm + L::kQ + qs * kTB);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
             const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
@@ -312,6 +325,9 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
           if (last) {
             mma_commit(&bars[L::bDKVFull]);
             mma_commit(&bars[L::bKVFree]);
+          } else if (!issue_dp(ec + 1)) {
+            stop = true;
+            break;
           }
         }
         if (stop) break;
@@ -330,6 +346,7 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
     auto wwait = [&](uint64_t *bar, uint32_t parity) {
       return __all_sync(0xffffffffu, wd.wait(bar, parity)) != 0;
     };
+    const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
     uint32_t tc = 0, cc = 0, ec = 0;
     bool stop = false;
     for (;; ++tc) {
@@ -342,10 +359,10 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       if (!k.valid) break;
       const int j = k.n * kTile + r;
       const bool row_ok = j < p.Skv;
-      __nv_bfloat16 *dk_row = p.dk + k.b * p.k_sb + static_cast<int64_t>(j) * p.k_ss + k.h * p.k_sh;
-      __nv_bfloat16 *dv_row = p.dv + k.b * p.v_sb + static_cast<int64_t>(j) * p.v_ss + k.h * p.v_sh;
       if (k.ee == k.es) {
         if (row_ok) {
+          __nv_bfloat16 *dk_row = p.dk + k.b * p.k_sb + static_cast<int64_t>(j) * p.k_ss + k.h * p.k_sh;
+          __nv_bfloat16 *dv_row = p.dv + k.b * p.v_sb + static_cast<int64_t>(j) * p.v_ss + k.h * p.v_sh;
           const int4 z = make_int4(0, 0, 0, 0);
 #pragma unroll
           for (int c = 0; c < D / 8; ++c) {
@@ -369,87 +386,104 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
         const uint32_t ent = p.col_ent[e];
         const int m = static_cast<int>(ent & kIndexMask);
         const bool full = (ent & kFullBit) != 0;
-        // stage LSE, Delta and the query segment ids of this q-block
+        // stage -LSE*log2e (-inf where the row has no key or lies past Sq) and
+        // -Delta of this q-block, negated so the element loop is one packed
+        // FMA / add
         {
           const int i = m * kTile + r;
-          float* vl = vec_lse + (ec & 1) * kTile;
-          float* vd = vec_delta + (ec & 1) * kTile;
-          int32_t* vs = vec_seg + (ec & 1) * kTile;
-          // stored negated so that the element loop is one packed FMA / add:
-          // -LSE*log2e (-inf where the row has no key or lies past Sq) and -Delta
           float nl2 = -INFINITY;
           if (i < p.Sq) {
             const float lv = p.lse[static_cast<int64_t>(k.bh) * p.Sq + i];
             if (lv != -INFINITY) nl2 = -lv * kLog2e;
           }
-          vl[r] = nl2;
-          vd[r] = -p.delta[static_cast<int64_t>(k.bh) * p.nM * kTile + i];
-          if (use_seg) vs[r] = i < p.Sq ? mk.seg_q[static_cast<int64_t>(k.b) * p.Sq + i] : INT_MIN + 1;
+          vec_nl[(ec & 1) * kTile + r] = nl2;
+          vec_nd[(ec & 1) * kTile + r] = -p.delta[static_cast<int64_t>(k.bh) * p.nM * kTile + i];
           mbar_arrive(&bars[L::bVecReady + (ec & 1)]);
         }
-        if (!wwait(&bars[L::bVecReady + (ec & 1)], (ec >> 1) & 1)) { stop = true; break; }
-        const float *vl = vec_lse + (ec & 1) * kTile;
-        const float *vd = vec_delta + (ec & 1) * kTile;
-        // allowed-query bits of this tile for this key row (range AND segment ids)
+        // allowed-query bits of this tile for this key row (range AND segment
+        // ids, the latter read through L1 as broadcasts)
         uint32_t allow[4] = {~0u, ~0u, ~0u, ~0u};
         if (!full) {
 #pragma unroll
           for (int w = 0; w < 4; ++w) allow[w] = range_bits(qlo - m * kTile, qhi - m * kTile, w);
           if (use_seg) {
-            const int4 *seg4 = reinterpret_cast<const int4 *>(vec_seg + (ec & 1) * kTile);
+            const int32_t *sq = mk.seg_q + static_cast<int64_t>(k.b) * p.Sq + m * kTile;
+            const int lim = p.Sq - m * kTile;
 #pragma unroll
             for (int w = 0; w < 4; ++w) {
               uint32_t bits = 0;
-#pragma unroll
-              for (int q = 0; q < 8; ++q) {
-                const int4 v = seg4[w * 8 + q];
-                bits |= (static_cast<uint32_t>(v.x == seg_j) << (4 * q)) |
-                        (static_cast<uint32_t>(v.y == seg_j) << (4 * q + 1)) |
-                        (static_cast<uint32_t>(v.z == seg_j) << (4 * q + 2)) |
-                        (static_cast<uint32_t>(v.w == seg_j) << (4 * q + 3));
+#pragma unroll 8
+              for (int q = 0; q < 32; ++q) {
+                const int ii = 32 * w + q;
+                bits |= static_cast<uint32_t>(ii < lim && __ldg(sq + ii) == seg_j) << q;
               }
               allow[w] &= bits;
             }
           }
         }
-        if (!wwait(&bars[L::bSdPFull], ec & 1)) { stop = true; break; }
-        if (ec >= 1 && !wwait(&bars[L::bDSFree], (ec - 1) & 1)) { stop = true; break; }
+        if (!wwait(&bars[L::bVecReady + (ec & 1)], (ec >> 1) & 1)) { stop = true; break; }
+        const float4 *nl4p = reinterpret_cast<const float4 *>(vec_nl + (ec & 1) * kTile);
+        const float4 *nd4p = reinterpret_cast<const float4 *>(vec_nd + (ec & 1) * kTile);
+        // phase 1: P^T = exp2(S^T * scale * log2e - LSE*log2e) -> bf16 in TMEM
+        // (over the first 64 S^T columns) and kept packed in registers
+        if (!wwait(&bars[L::bSFull], ec & 1)) { stop = true; break; }
         tc_fence_after();
+        uint32_t pk[64];
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          uint32_t s[32], dp[32];
+          uint32_t s[32];
           tmem_ld32(T_S + lane_off + 32 * c, s);
-          tmem_ld32(T_DP + lane_off + 32 * c, dp);
           tmem_wait_ld();
-          uint32_t pk[16], dk2[16];
-          const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
 #pragma unroll
           for (int q4 = 0; q4 < 8; ++q4) {
-            // four query columns: their -LSE and -Delta as one broadcast load each
-            const float4 nl4 = reinterpret_cast<const float4 *>(vl)[8 * c + q4];
-            const float4 nd4 = reinterpret_cast<const float4 *>(vd)[8 * c + q4];
+            const float4 nl4 = nl4p[8 * c + q4];
 #pragma unroll
             for (int h2 = 0; h2 < 2; ++h2) {
-              const int e0 = 4 * q4 + 2 * h2;  // element index in this 32-column chunk
+              const int e0 = 4 * q4 + 2 * h2;
               const float2 nl = h2 ? make_float2(nl4.z, nl4.w) : make_float2(nl4.x, nl4.y);
-              const float2 nd = h2 ? make_float2(nd4.z, nd4.w) : make_float2(nd4.x, nd4.y);
-              const float2 t = __ffma2_rn(
+              const float2 tt = __ffma2_rn(
                   make_float2(__uint_as_float(s[e0]), __uint_as_float(s[e0 + 1])), sc2, nl);
-              float p0 = fast_exp2(t.x), p1 = fast_exp2(t.y);
+              float p0 = fast_exp2(tt.x), p1 = fast_exp2(tt.y);
               if (!full) {
                 p0 = ((allow[c] >> e0) & 1u) ? p0 : 0.f;
                 p1 = ((allow[c] >> (e0 + 1)) & 1u) ? p1 : 0.f;
               }
-              const float2 dd = __fadd2_rn(
-                  make_float2(__uint_as_float(dp[e0]), __uint_as_float(dp[e0 + 1])), nd);
-              const float2 ds = __fmul2_rn(make_float2(p0, p1), dd);
-              pk[e0 >> 1] = pack_bf16x2(p0, p1);
-              dk2[e0 >> 1] = pack_bf16x2(ds.x, ds.y);
+              pk[16 * c + (e0 >> 1)] = pack_bf16x2(p0, p1);
             }
           }
-          // P^T chunk -> TMEM columns [16c, 16c+16) of the S^T region
-          tmem_st16(T_S + lane_off + 16 * c, pk);
-          // dS^T chunk -> shared tile, row r, 16-byte chunks 4c..4c+3 (128-byte swizzle)
+          // P^T chunk -> TMEM columns [16c, 16c+16): only S^T columns already read
+          tmem_st16(T_S + lane_off + 16 * c,
+                    *reinterpret_cast<const uint32_t(*)[16]>(&pk[16 * c]));
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&bars[L::bPReady]);
+        // phase 2: dS^T = P^T o (dP^T - Delta), with the bf16 P^T the dV product
+        // uses, -> bf16 shared tile (128-byte swizzle, K-major)
+        if (ec >= 1 && !wwait(&bars[L::bDSFree], (ec - 1) & 1)) { stop = true; break; }
+        if (!wwait(&bars[L::bDPFull], ec & 1)) { stop = true; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t dp[32];
+          tmem_ld32(T_DP + lane_off + 32 * c, dp);
+          tmem_wait_ld();
+          uint32_t dk2[16];
+#pragma unroll
+          for (int q4 = 0; q4 < 8; ++q4) {
+            const float4 nd4 = nd4p[8 * c + q4];
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+              const int e0 = 4 * q4 + 2 * h2;
+              const float2 nd = h2 ? make_float2(nd4.z, nd4.w) : make_float2(nd4.x, nd4.y);
+              const uint32_t pp = pk[16 * c + (e0 >> 1)];
+              const float2 pv = make_float2(__uint_as_float(pp << 16), __uint_as_float(pp & 0xffff0000u));
+              const float2 dd = __fadd2_rn(
+                  make_float2(__uint_as_float(dp[e0]), __uint_as_float(dp[e0 + 1])), nd);
+              const float2 dsv = __fmul2_rn(pv, dd);
+              dk2[e0 >> 1] = pack_bf16x2(dsv.x, dsv.y);
+            }
+          }
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
             const int chunk = 4 * c + u;  // 0..15 over 128 queries
@@ -459,15 +493,16 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
                 make_int4(dk2[4 * u], dk2[4 * u + 1], dk2[4 * u + 2], dk2[4 * u + 3]);
           }
         }
-        tmem_wait_st();
-        tc_fence_before();
         fence_proxy_async_smem();
-        mbar_arrive(&bars[L::bPdSReady]);
+        tc_fence_before();
+        mbar_arrive(&bars[L::bDSReady]);
       }
       if (stop) break;
       // epilogue: dV, dK (scaled) -> bf16
       if (!wwait(&bars[L::bDKVFull], cc & 1)) break;
       tc_fence_after();
+      __nv_bfloat16 *dk_row = p.dk + k.b * p.k_sb + static_cast<int64_t>(j) * p.k_ss + k.h * p.k_sh;
+      __nv_bfloat16 *dv_row = p.dv + k.b * p.v_sb + static_cast<int64_t>(j) * p.v_ss + k.h * p.v_sh;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t a[32], g[32];
@@ -649,6 +684,7 @@ template <int D, int NQ, int NDO>
 cudaError_t run_bwd_main(const BwdParams &bp, const CUtensorMap &tq, const CUtensorMap &tk,
                          const CUtensorMap &tv, const CUtensorMap &tdo, cudaStream_t s) {
   using L = BwdSmem<D, NQ, NDO>;
+  static_assert(L::kAlloc <= 232448, "shared memory budget");
   static bool attr = false;
   if (!attr) {
     cudaError_t e = cudaFuncSetAttribute(k_attn_bwd<D, NQ, NDO>,
@@ -731,7 +767,7 @@ cudaError_t launch_bwd_main(const bsa_problem &p, const MaskParams &mp, const bs
   cudaError_t e = cudaMemsetAsync(bp.hdr + kHdrBwdTicket, 0, sizeof(uint32_t), s);
   if (e != cudaSuccess) return e;
   return (p.D == 64) ? run_bwd_main<64, 2, 2>(bp, tq, tk, tv, tdo, s)
-                     : run_bwd_main<128, 2, 1>(bp, tq, tk, tv, tdo, s);
+                     : run_bwd_main<128, 2, 2>(bp, tq, tk, tv, tdo, s);
 }
 
 cudaError_t launch_bwd_convert(const bsa_problem &p, void *dq, const WsLayout &L, uint8_t *ws,
