@@ -389,7 +389,7 @@ bsa_status bsa_bwd_preprocess(const bsa_problem *prob, const bsa_mask_spec *mask
   Prepared P;
   bsa_status st = prepare(prob, mask, opt, ws, ws_bytes, true, &P);
   if (st != BSA_OK) return st;
-  return cuda_status(launch_bwd_preprocess(P.p, out, dout, P.L, static_cast<uint8_t *>(ws),
+  return cuda_status(launch_bwd_preprocess(P.p, P.o, out, dout, P.L, static_cast<uint8_t *>(ws),
                                            reinterpret_cast<cudaStream_t>(stream)));
 }
 

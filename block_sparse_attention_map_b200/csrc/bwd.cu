@@ -572,10 +572,19 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
         }
         if (ok) {
           float *base = p.dq_accum + (static_cast<int64_t>(k.bh) * p.nM + m) * (D / 4) * (kTile * 4);
+          if (p.deterministic && rank == 0) {
+            // the first contributor in the order pi initialises the accumulator
+            // rows, so the deterministic path needs no zeroing pass
 #pragma unroll
-          for (int c = 0; c < D / 4; ++c)
-            red_add_v4(base + (static_cast<int64_t>(c) * kTile + r) * 4, acc[4 * c], acc[4 * c + 1],
-                       acc[4 * c + 2], acc[4 * c + 3]);
+            for (int c = 0; c < D / 4; ++c)
+              st_v4(base + (static_cast<int64_t>(c) * kTile + r) * 4, acc[4 * c], acc[4 * c + 1],
+                    acc[4 * c + 2], acc[4 * c + 3]);
+          } else {
+#pragma unroll
+            for (int c = 0; c < D / 4; ++c)
+              red_add_v4(base + (static_cast<int64_t>(c) * kTile + r) * 4, acc[4 * c],
+                         acc[4 * c + 1], acc[4 * c + 2], acc[4 * c + 3]);
+          }
         }
         if (p.deterministic) {
           __threadfence();
@@ -640,13 +649,26 @@ __global__ void __launch_bounds__(256) k_bwd_delta(const __nv_bfloat16 *__restri
 // ---------------------------------------------------------------- a7: dQ convert
 template <int D>
 __global__ void __launch_bounds__(256) k_dq_convert(const float *__restrict__ acc, int B, int H,
-                                                    int Sq, int nM, __nv_bfloat16 *__restrict__ dq,
+                                                    int Sq, int nM, const int32_t *__restrict__ row_ptr,
+                                                    __nv_bfloat16 *__restrict__ dq,
                                                     int64_t sb, int64_t ss, int64_t sh) {
   extern __shared__ float tile[];  // [128][D + 4]
   constexpr int LD = D + 4;
   const int bhm = blockIdx.x;
   const int m = bhm % nM, bh = bhm / nM, b = bh / H, h = bh % H;
   const float *src = acc + static_cast<int64_t>(bhm) * (D / 4) * kTile * 4;
+  if (row_ptr[b * nM + m + 1] == row_ptr[b * nM + m]) {
+    // a q-block without non-empty tiles got no contribution: dQ = 0
+    constexpr int CPR = D / 8;
+    for (int idx = threadIdx.x; idx < kTile * CPR; idx += blockDim.x) {
+      const int r = idx / CPR, c = idx % CPR;
+      const int i = m * kTile + r;
+      if (i < Sq)
+        *reinterpret_cast<int4 *>(dq + b * sb + static_cast<int64_t>(i) * ss + h * sh + 8 * c) =
+            make_int4(0, 0, 0, 0);
+    }
+    return;
+  }
   for (int idx = threadIdx.x; idx < (D / 4) * kTile; idx += blockDim.x) {
     const int c = idx / kTile, r = idx % kTile;
     const float4 v = reinterpret_cast<const float4 *>(src)[idx];
@@ -700,8 +722,9 @@ cudaError_t run_bwd_main(const BwdParams &bp, const CUtensorMap &tq, const CUten
 
 }  // namespace
 
-cudaError_t launch_bwd_preprocess(const bsa_problem &p, const void *out, const void *dout,
-                                  const WsLayout &L, uint8_t *ws, cudaStream_t s) {
+cudaError_t launch_bwd_preprocess(const bsa_problem &p, const bsa_options &o, const void *out,
+                                  const void *dout, const WsLayout &L, uint8_t *ws,
+                                  cudaStream_t s) {
   const int rows_pad = L.nM * kTile;
   const int64_t groups = static_cast<int64_t>(p.B) * p.H * rows_pad;
   const int64_t threads = groups * (p.D / 8);
@@ -718,9 +741,13 @@ cudaError_t launch_bwd_preprocess(const bsa_problem &p, const void *out, const v
                                             p.o_stride[1], p.o_stride[2], p.B, p.Sq, p.H, rows_pad,
                                             delta);
   count_launch();
-  cudaError_t e = cudaMemsetAsync(ws + L.dq_accum, 0,
-                                  sizeof(float) * static_cast<size_t>(groups) * p.D, s);
-  if (e != cudaSuccess) return e;
+  cudaError_t e = cudaSuccess;
+  if (!o.deterministic) {
+    // atomic adds need a zeroed accumulator; the deterministic path initialises
+    // it with the first contributor's stores instead
+    e = cudaMemsetAsync(ws + L.dq_accum, 0, sizeof(float) * static_cast<size_t>(groups) * p.D, s);
+    if (e != cudaSuccess) return e;
+  }
   e = cudaMemsetAsync(ws + L.sem, 0, sizeof(uint32_t) * static_cast<size_t>(p.B) * p.H * L.nM, s);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
@@ -779,8 +806,10 @@ cudaError_t launch_bwd_convert(const bsa_problem &p, void *dq, const WsLayout &L
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    kern<<<blocks, 256, smem, s>>>(acc, p.B, p.H, p.Sq, L.nM, static_cast<__nv_bfloat16 *>(dq),
-                                   p.q_stride[0], p.q_stride[1], p.q_stride[2]);
+    kern<<<blocks, 256, smem, s>>>(acc, p.B, p.H, p.Sq, L.nM,
+                                   reinterpret_cast<const int32_t *>(ws + L.row_ptr),
+                                   static_cast<__nv_bfloat16 *>(dq), p.q_stride[0], p.q_stride[1],
+                                   p.q_stride[2]);
     count_launch();
     return cudaGetLastError();
   };
@@ -792,7 +821,7 @@ cudaError_t launch_bwd(const bsa_problem &p, const MaskParams &mp, const bsa_opt
                        const CUtensorMap &tv, const CUtensorMap &tdo, const void *out,
                        const void *dout, const float *lse, void *dq, void *dk, void *dv,
                        const WsLayout &L, uint8_t *ws, cudaStream_t s) {
-  cudaError_t e = launch_bwd_preprocess(p, out, dout, L, ws, s);
+  cudaError_t e = launch_bwd_preprocess(p, o, out, dout, L, ws, s);
   if (e != cudaSuccess) return e;
   e = launch_bwd_main(p, mp, o, sig, tq, tk, tv, tdo, lse, dk, dv, L, ws, s);
   if (e != cudaSuccess) return e;

@@ -508,54 +508,82 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
 }
 
 // ---------------------------------------------------------------- fixed-m bound
-// Norms of every (row, head) vector of Q or K.  Keys: running max per (b, h)
-// over valid keys (padding and varlen alignment keys excluded).  Queries: the
-// per-row norm is stored and the running max per (b, h) kept.
+// Norms of every (row, head) vector of K (blockIdx.y == 0) and Q (== 1).
+// Keys: running max per (b, h) over valid keys (padding and varlen alignment
+// keys excluded).  Queries: the per-row norm is stored and the running max per
+// (b, h) kept.  Each group of D/8 threads owns one vector at a time and keeps
+// four vectors' loads in flight.
+struct NormArgs {
+  const __nv_bfloat16 *k, *q;
+  int64_t ks[3], qs[3];
+  int B, Skv, Sq, H, only_q;
+  MaskParams mk;
+  float *kmax, *qmax, *qnorm;
+};
+
 template <int D>
-__global__ void __launch_bounds__(256) k_row_norms(const __nv_bfloat16 *__restrict__ x,
-                                                   int64_t sb, int64_t ss, int64_t sh, int B,
-                                                   int S, int H, int is_key, MaskParams mk,
-                                                   float *__restrict__ rowmax,
-                                                   float *__restrict__ qnorm) {
+__global__ void __launch_bounds__(256) k_row_norms(const NormArgs a) {
   constexpr int TPV = D / 8;  // threads per vector, 16 bytes each
-  constexpr int kRows = 16;
+  constexpr int kRows = 32;
+  constexpr int kUnroll = 4;
   extern __shared__ unsigned int smax[];  // [H]
-  for (int h = threadIdx.x; h < H; h += blockDim.x) smax[h] = 0u;
-  __syncthreads();
-  const int64_t blocks_per_b = (S + kRows - 1) / kRows;
+  const int is_key = !a.only_q && blockIdx.y == 0;
+  const __nv_bfloat16 *x = is_key ? a.k : a.q;
+  const int S = is_key ? a.Skv : a.Sq;
+  const int64_t sb = is_key ? a.ks[0] : a.qs[0], ss = is_key ? a.ks[1] : a.qs[1],
+                sh = is_key ? a.ks[2] : a.qs[2];
+  float *rowmax = is_key ? a.kmax : a.qmax;
+  const int H = a.H, Sq = a.Sq, Skv = a.Skv;
+  const MaskParams &mk = a.mk;
+  float *qnorm = a.qnorm;
+  const int64_t blocks_per_b = (max(Sq, Skv) + kRows - 1) / kRows;
   const int b = static_cast<int>(blockIdx.x / blocks_per_b);
   const int r0 = static_cast<int>(blockIdx.x % blocks_per_b) * kRows;
+  if (r0 >= S) return;  // whole block past this tensor's rows (uniform)
+  for (int h = threadIdx.x; h < H; h += blockDim.x) smax[h] = 0u;
+  __syncthreads();
   const int g = threadIdx.x / TPV, t = threadIdx.x % TPV;
   const int groups = blockDim.x / TPV;
+  const int pairs = kRows * H;
   // uniform trip count across the warp: the shuffles below need every lane
-  for (int base = 0; base < kRows * H; base += groups) {
-    const int pair = base + g;
-    const int row = r0 + pair / H, h = pair % H;
-    const bool in = pair < kRows * H && row < S;
-    float acc = 0.f;
-    if (in) {
-      const int4 v = *reinterpret_cast<const int4 *>(x + b * sb + static_cast<int64_t>(row) * ss +
-                                                    h * sh + t * 8);
-      const __nv_bfloat162 *e = reinterpret_cast<const __nv_bfloat162 *>(&v);
+  for (int base = 0; base < pairs; base += groups * kUnroll) {
+    float acc[kUnroll];
+    int row[kUnroll], hh[kUnroll];
+    bool in[kUnroll];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const float2 f = __bfloat1622float2(e[q]);
-        acc = fmaf(f.x, f.x, acc);
-        acc = fmaf(f.y, f.y, acc);
+    for (int u = 0; u < kUnroll; ++u) {
+      const int pair = base + u * groups + g;
+      row[u] = r0 + pair / H;
+      hh[u] = pair % H;
+      in[u] = pair < pairs && row[u] < S;
+      acc[u] = 0.f;
+      if (in[u]) {
+        const int4 v = *reinterpret_cast<const int4 *>(x + b * sb + static_cast<int64_t>(row[u]) * ss +
+                                                      hh[u] * sh + t * 8);
+        const __nv_bfloat162 *e = reinterpret_cast<const __nv_bfloat162 *>(&v);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float2 f = __bfloat1622float2(e[q]);
+          acc[u] = fmaf(f.x, f.x, acc[u]);
+          acc[u] = fmaf(f.y, f.y, acc[u]);
+        }
       }
     }
 #pragma unroll
-    for (int o = TPV / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if (t == 0 && in) {
-      const float nrm = sqrtf(acc);
-      bool valid = true;
-      if (is_key) {
-        if (mk.flags & BSA_MASK_KV_VALID_LEN) valid = row < mk.kv_valid_len[b];
-        if ((mk.flags & BSA_MASK_VARLEN) && mk.seg_kv != nullptr) valid = valid && mk.seg_kv[row] >= 0;
-      } else {
-        qnorm[(static_cast<int64_t>(b) * H + h) * S + row] = nrm;
+    for (int u = 0; u < kUnroll; ++u) {
+#pragma unroll
+      for (int o = TPV / 2; o > 0; o >>= 1) acc[u] += __shfl_xor_sync(0xffffffffu, acc[u], o);
+      if (t == 0 && in[u]) {
+        const float nrm = sqrtf(acc[u]);
+        bool valid = true;
+        if (is_key) {
+          if (mk.flags & BSA_MASK_KV_VALID_LEN) valid = row[u] < mk.kv_valid_len[b];
+          if ((mk.flags & BSA_MASK_VARLEN) && mk.seg_kv != nullptr) valid = valid && mk.seg_kv[row[u]] >= 0;
+        } else {
+          qnorm[(static_cast<int64_t>(b) * H + hh[u]) * S + row[u]] = nrm;
+        }
+        if (valid) atomicMax(&smax[hh[u]], __float_as_uint(nrm));
       }
-      if (valid) atomicMax(&smax[h], __float_as_uint(nrm));
     }
   }
   __syncthreads();
@@ -570,19 +598,6 @@ __global__ void k_gate(int BH, float scale, float limit, const float *kmax_overr
   const float km = kmax_override != nullptr ? kmax_override[t] : kmax[t];
   kmax[t] = km;
   gate[t] = (2.f * scale * qmax[t] * km <= limit) ? 1 : 0;
-}
-
-template <int D>
-cudaError_t run_norms(const bsa_problem &p, const MaskParams &mp, const void *x,
-                      const int64_t *st, int S, int is_key, float *rowmax, float *qnorm,
-                      cudaStream_t s) {
-  const int64_t blocks = static_cast<int64_t>(p.B) * ((S + 15) / 16);
-  const size_t smem = sizeof(unsigned int) * p.H;
-  k_row_norms<D><<<static_cast<unsigned>(blocks), 256, smem, s>>>(
-      static_cast<const __nv_bfloat16 *>(x), st[0], st[1], st[2], p.B, S, p.H, is_key, mp,
-      rowmax, qnorm);
-  count_launch();
-  return cudaGetLastError();
 }
 
 int sm_count() {
@@ -619,22 +634,33 @@ cudaError_t run_fwd(const FwdParams &fp, const CUtensorMap &tq, const CUtensorMa
 cudaError_t launch_fixed_m_bound(const bsa_problem &p, const MaskParams &mp,
                                  const bsa_options &o, const void *q, const void *k,
                                  const WsLayout &L, uint8_t *ws, cudaStream_t s) {
-  float *kmax = reinterpret_cast<float *>(ws + L.kmax);
-  float *qmax = reinterpret_cast<float *>(ws + L.qmax);
-  float *qnorm = reinterpret_cast<float *>(ws + L.qnorm);
-  cudaError_t e = cudaMemsetAsync(kmax, 0, sizeof(float) * p.B * p.H * 2, s);  // kmax, qmax
-  if (e != cudaSuccess) return e;
-  if (o.kmax_override == nullptr) {
-    e = p.D == 64 ? run_norms<64>(p, mp, k, p.k_stride, p.Skv, 1, kmax, nullptr, s)
-                  : run_norms<128>(p, mp, k, p.k_stride, p.Skv, 1, kmax, nullptr, s);
-    if (e != cudaSuccess) return e;
+  NormArgs na{};
+  na.k = static_cast<const __nv_bfloat16 *>(k);
+  na.q = static_cast<const __nv_bfloat16 *>(q);
+  for (int i = 0; i < 3; ++i) {
+    na.ks[i] = p.k_stride[i];
+    na.qs[i] = p.q_stride[i];
   }
-  e = p.D == 64 ? run_norms<64>(p, mp, q, p.q_stride, p.Sq, 0, qmax, qnorm, s)
-                : run_norms<128>(p, mp, q, p.q_stride, p.Sq, 0, qmax, qnorm, s);
+  na.B = p.B;
+  na.Skv = p.Skv;
+  na.Sq = p.Sq;
+  na.H = p.H;
+  na.only_q = o.kmax_override != nullptr;  // a caller-supplied kmax needs no key pass
+  na.mk = mp;
+  na.kmax = reinterpret_cast<float *>(ws + L.kmax);
+  na.qmax = reinterpret_cast<float *>(ws + L.qmax);
+  na.qnorm = reinterpret_cast<float *>(ws + L.qnorm);
+  cudaError_t e = cudaMemsetAsync(na.kmax, 0, sizeof(float) * p.B * p.H * 2, s);  // kmax, qmax
   if (e != cudaSuccess) return e;
+  const int64_t blocks = static_cast<int64_t>(p.B) * ((std::max(p.Sq, p.Skv) + 31) / 32);
+  const dim3 grid(static_cast<unsigned>(blocks), na.only_q ? 1u : 2u);
+  const size_t smem = sizeof(unsigned int) * p.H;
+  if (p.D == 64) k_row_norms<64><<<grid, 256, smem, s>>>(na);
+  else k_row_norms<128><<<grid, 256, smem, s>>>(na);
+  count_launch();
   const float limit = o.gate_limit > 0.f ? o.gate_limit : 64.f;
   const int BH = p.B * p.H;
-  k_gate<<<(BH + 127) / 128, 128, 0, s>>>(BH, p.scale, limit, o.kmax_override, kmax, qmax,
+  k_gate<<<(BH + 127) / 128, 128, 0, s>>>(BH, p.scale, limit, o.kmax_override, na.kmax, na.qmax,
                                           reinterpret_cast<int32_t *>(ws + L.gate));
   count_launch();
   return cudaGetLastError();

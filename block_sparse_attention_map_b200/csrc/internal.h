@@ -91,8 +91,9 @@ cudaError_t launch_bwd(const bsa_problem &p, const MaskParams &mp, const bsa_opt
                        const float *lse, void *dq, void *dk, void *dv, const WsLayout &L,
                        uint8_t *ws, cudaStream_t s);
 
-cudaError_t launch_bwd_preprocess(const bsa_problem &p, const void *out, const void *dout,
-                                  const WsLayout &L, uint8_t *ws, cudaStream_t s);
+cudaError_t launch_bwd_preprocess(const bsa_problem &p, const bsa_options &o, const void *out,
+                                  const void *dout, const WsLayout &L, uint8_t *ws,
+                                  cudaStream_t s);
 
 cudaError_t launch_bwd_main(const bsa_problem &p, const MaskParams &mp, const bsa_options &o,
                             const PlanSignature &sig, const CUtensorMap &tq, const CUtensorMap &tk,

@@ -76,20 +76,15 @@ struct ClassifyArgs {
   const int32_t *kv_valid_len;
   const int4 *qblk, *kblk;  // null unless segment ids / varlen
   uint8_t *cls;
+  int32_t *row_cnt, *col_cnt;
 };
 
-// Tile class per (b, m, n): the AND-combination of one class per enabled
+// Tile class of (b, m, n): the AND-combination of one class per enabled
 // predicate (EMPTY if any predicate is empty, FULL if all are full).  Window,
 // padding and out-of-range columns are classified analytically and exactly;
 // segment ids through per-block [min, max] intervals, exact for
 // non-decreasing ids and conservative (PARTIAL instead of EMPTY) otherwise.
-__global__ void k_classify(ClassifyArgs a) {
-  const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int64_t total = static_cast<int64_t>(a.B) * a.nM * a.nN;
-  if (idx >= total) return;
-  const int n = static_cast<int>(idx % a.nN);
-  const int m = static_cast<int>((idx / a.nN) % a.nM);
-  const int b = static_cast<int>(idx / (static_cast<int64_t>(a.nN) * a.nM));
+__device__ __forceinline__ uint8_t tile_class(const ClassifyArgs &a, int b, int m, int n) {
   const int i0 = m * kTile, i1 = min(a.Sq, i0 + kTile) - 1;
   const int j0 = n * kTile, jv1 = min(a.Skv, j0 + kTile) - 1;
   uint8_t c = BSA_TILE_FULL;
@@ -98,123 +93,179 @@ __global__ void k_classify(ClassifyArgs a) {
     const int o = a.Skv - a.Sq, W = a.window;
     const bool any = (j0 <= i1 + o) && (W == 0 || jv1 >= i0 + o - W + 1);
     const bool all = (jv1 <= i0 + o) && (W == 0 || j0 >= i1 + o - W + 1);
-    if (!any) { a.cls[idx] = BSA_TILE_EMPTY; return; }
+    if (!any) return BSA_TILE_EMPTY;
     if (!all) c = BSA_TILE_PARTIAL;
   }
   if (a.flags & BSA_MASK_KV_VALID_LEN) {
     const int L = a.kv_valid_len[b];
-    if (j0 >= L) { a.cls[idx] = BSA_TILE_EMPTY; return; }
+    if (j0 >= L) return BSA_TILE_EMPTY;
     if (jv1 >= L) c = BSA_TILE_PARTIAL;
   }
   if (a.qblk != nullptr) {
     const int4 q = a.qblk[b * a.nM + m];
     const int4 k = a.kblk[b * a.nN + n];
-    if (q.z == 0 || k.z == 0 || q.y < k.x || k.y < q.x) { a.cls[idx] = BSA_TILE_EMPTY; return; }
+    if (q.z == 0 || k.z == 0 || q.y < k.x || k.y < q.x) return BSA_TILE_EMPTY;
     const bool one = q.x == q.y && k.x == k.y && q.x == k.x && q.w == 0 && k.w == 0;
     if (!one) c = BSA_TILE_PARTIAL;
   }
-  a.cls[idx] = c;
+  return c;
 }
 
-__global__ void k_make_perm(int nN, int order, int32_t *perm) {
-  const int t = blockIdx.x * blockDim.x + threadIdx.x;
-  if (t < nN) perm[t] = (order == BSA_ORDER_DESC) ? (nN - 1 - t) : t;
-}
-
-// rank(m, n): walk row m's columns in the order pi; non-empty ones get 0, 1, 2, ...
-__global__ void k_row_rank(const uint8_t *__restrict__ cls, const int32_t *__restrict__ perm,
-                           int BnM, int nN, int32_t *__restrict__ rank,
-                           int32_t *__restrict__ row_cnt) {
-  const int r = blockIdx.x * blockDim.x + threadIdx.x;
-  if (r >= BnM) return;
-  const uint8_t *row = cls + static_cast<int64_t>(r) * nN;
-  int32_t *rk = rank + static_cast<int64_t>(r) * nN;
+// One warp per (b, m): classify the row of tiles, count its non-empty tiles
+// and add each non-empty tile to its column's count (an order-independent sum).
+__global__ void k_classify_rows(ClassifyArgs a) {
+  const int wid = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (wid >= a.B * a.nM) return;
+  const int b = wid / a.nM, m = wid % a.nM;
+  uint8_t *row = a.cls + static_cast<int64_t>(wid) * a.nN;
   int cnt = 0;
-  for (int t = 0; t < nN; ++t) {
-    const int n = perm[t];
-    rk[n] = row[n] != BSA_TILE_EMPTY ? cnt++ : -1;
+  for (int n0 = 0; n0 < a.nN; n0 += 32) {
+    const int n = n0 + lane;
+    uint8_t c = BSA_TILE_EMPTY;
+    if (n < a.nN) {
+      c = tile_class(a, b, m, n);
+      row[n] = c;
+      if (c != BSA_TILE_EMPTY) atomicAdd(a.col_cnt + b * a.nN + n, 1);
+    }
+    cnt += __popc(__ballot_sync(0xffffffffu, c != BSA_TILE_EMPTY));
   }
-  row_cnt[r] = cnt;
-}
-
-__global__ void k_col_count(const uint8_t *__restrict__ cls, int B, int nM, int nN,
-                            int32_t *__restrict__ col_cnt) {
-  const int t = blockIdx.x * blockDim.x + threadIdx.x;
-  if (t >= B * nN) return;
-  const int b = t / nN, n = t % nN;
-  int cnt = 0;
-  for (int m = 0; m < nM; ++m) cnt += cls[(static_cast<int64_t>(b) * nM + m) * nN + n] != 0;
-  col_cnt[t] = cnt;
+  if (lane == 0) a.row_cnt[wid] = cnt;
 }
 
 // Exclusive scans of row and column counts into CSR offsets (block 0: rows,
-// block 1: columns); ptr[count] receives the total.
+// block 1: columns); ptr[count] receives the total.  Block 0 then writes the
+// plan signature that the forward and backward kernels check.
 __global__ void k_scan2(const int32_t *__restrict__ c0, int32_t *__restrict__ p0, int n0,
-                        const int32_t *__restrict__ c1, int32_t *__restrict__ p1, int n1) {
+                        const int32_t *__restrict__ c1, int32_t *__restrict__ p1, int n1,
+                        uint32_t *hdr, uint32_t B, uint32_t Sq, uint32_t Skv, uint32_t flags,
+                        uint32_t window, uint32_t order, uint32_t n_seqs) {
   const int32_t *c = blockIdx.x == 0 ? c0 : c1;
   int32_t *p = blockIdx.x == 0 ? p0 : p1;
   const int n = blockIdx.x == 0 ? n0 : n1;
-  __shared__ int32_t buf[1024];
+  __shared__ int32_t warp_tot[32];
   __shared__ int32_t carry;
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   if (threadIdx.x == 0) carry = 0;
   __syncthreads();
   for (int base = 0; base < n; base += 1024) {
     const int i = base + threadIdx.x;
     const int32_t v = i < n ? c[i] : 0;
-    buf[threadIdx.x] = v;
-    __syncthreads();
-    for (int o = 1; o < 1024; o <<= 1) {
-      const int32_t add = threadIdx.x >= o ? buf[threadIdx.x - o] : 0;
-      __syncthreads();
-      buf[threadIdx.x] += add;
-      __syncthreads();
+    int32_t x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int32_t y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
     }
-    if (i < n) p[i] = carry + buf[threadIdx.x] - v;
+    if (lane == 31) warp_tot[wid] = x;
     __syncthreads();
-    if (threadIdx.x == 1023) carry += buf[1023];
+    if (wid == 0) {
+      int32_t t = warp_tot[lane];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int32_t y = __shfl_up_sync(0xffffffffu, t, o);
+        if (lane >= o) t += y;
+      }
+      warp_tot[lane] = t;  // inclusive over warps
+    }
+    __syncthreads();
+    const int32_t before = (wid > 0 ? warp_tot[wid - 1] : 0) + carry;
+    if (i < n) p[i] = before + x - v;
+    __syncthreads();
+    if (threadIdx.x == 0) carry += warp_tot[31];
     __syncthreads();
   }
-  if (threadIdx.x == 0) p[n] = carry;
+  if (threadIdx.x == 0) {
+    p[n] = carry;
+    if (blockIdx.x == 0) {
+      hdr[kHdrB] = B;
+      hdr[kHdrSq] = Sq;
+      hdr[kHdrSkv] = Skv;
+      hdr[kHdrFlags] = flags;
+      hdr[kHdrWindow] = window;
+      hdr[kHdrOrder] = order;
+      hdr[kHdrNSeqs] = n_seqs;
+      __threadfence();
+      hdr[kHdrMagic] = kPlanMagic;
+    }
+  }
 }
 
-// Row lists for the forward: ascending n, FULL flag in bit 30.
-__global__ void k_row_fill(const uint8_t *__restrict__ cls, int BnM, int nN,
-                           const int32_t *__restrict__ row_ptr, uint32_t *__restrict__ row_ent) {
-  const int r = blockIdx.x * blockDim.x + threadIdx.x;
-  if (r >= BnM) return;
-  const uint8_t *row = cls + static_cast<int64_t>(r) * nN;
-  int pos = row_ptr[r];
-  for (int n = 0; n < nN; ++n) {
-    const uint8_t c = row[n];
-    if (c != BSA_TILE_EMPTY) row_ent[pos++] = n | (c == BSA_TILE_FULL ? kFullBit : 0u);
+// One warp per (b, m): the forward's row list (ascending n, FULL flag in bit
+// 30) and rank(m, n): row m's non-empty columns numbered 0, 1, 2, ... in the
+// order pi (-1 for empty tiles).  pi is ascending, descending, or the
+// caller's permutation already in the workspace; warp 0 writes it out for
+// the asc / desc orders.
+__global__ void k_row_fill(const uint8_t *__restrict__ cls, int BnM, int nN, int order,
+                           int32_t *__restrict__ perm, const int32_t *__restrict__ row_ptr,
+                           uint32_t *__restrict__ row_ent, int32_t *__restrict__ rank) {
+  const int wid = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (wid >= BnM) return;
+  const uint8_t *row = cls + static_cast<int64_t>(wid) * nN;
+  if (wid == 0 && order != BSA_ORDER_PERM)
+    for (int t = lane; t < nN; t += 32) perm[t] = order == BSA_ORDER_DESC ? nN - 1 - t : t;
+  int pos = row_ptr[wid];
+  for (int n0 = 0; n0 < nN; n0 += 32) {
+    const int n = n0 + lane;
+    const uint8_t c = n < nN ? row[n] : BSA_TILE_EMPTY;
+    const uint32_t bal = __ballot_sync(0xffffffffu, c != BSA_TILE_EMPTY);
+    if (c != BSA_TILE_EMPTY)
+      row_ent[pos + __popc(bal & ((1u << lane) - 1u))] = n | (c == BSA_TILE_FULL ? kFullBit : 0u);
+    pos += __popc(bal);
+  }
+  int32_t *rk = rank + static_cast<int64_t>(wid) * nN;
+  int r = 0;
+  for (int t0 = 0; t0 < nN; t0 += 32) {
+    const int t = t0 + lane;
+    int n = -1;
+    if (t < nN) n = order == BSA_ORDER_PERM ? perm[t] : (order == BSA_ORDER_DESC ? nN - 1 - t : t);
+    const bool ne = n >= 0 && row[n] != BSA_TILE_EMPTY;
+    const uint32_t bal = __ballot_sync(0xffffffffu, ne);
+    if (n >= 0) rk[n] = ne ? r + __popc(bal & ((1u << lane) - 1u)) : -1;
+    r += __popc(bal);
   }
 }
 
 // Column lists for the backward: the unified partial+full list of column n,
-// sorted by (rank(m, n), m).  One block per (b, n); the column's entries are
-// gathered into shared memory and each entry's position is the number of
-// entries with a smaller key.
+// sorted by (rank(m, n), m).  One block per (b, n): the column's entries are
+// gathered in ascending m by a block-wide compaction, then each entry's
+// position is the number of entries with a smaller key.
 __global__ void k_col_fill(const uint8_t *__restrict__ cls, const int32_t *__restrict__ rank,
-                          int nM, int nN, const int32_t *__restrict__ col_ptr,
-                          uint32_t *__restrict__ col_ent, int32_t *__restrict__ col_rank) {
+                           int nM, int nN, const int32_t *__restrict__ col_ptr,
+                           uint32_t *__restrict__ col_ent, int32_t *__restrict__ col_rank) {
   extern __shared__ unsigned long long keys[];
-  __shared__ int cnt;
+  __shared__ int warp_cnt[32];
+  __shared__ int base_cnt;
   const int bn = blockIdx.x;
   const int b = bn / nN, n = bn % nN;
-  if (threadIdx.x == 0) {
-    int c = 0;
-    for (int m = 0; m < nM; ++m) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  if (threadIdx.x == 0) base_cnt = 0;
+  __syncthreads();
+  for (int m0 = 0; m0 < nM; m0 += blockDim.x) {
+    const int m = m0 + threadIdx.x;
+    unsigned long long key = 0;
+    bool ne = false;
+    if (m < nM) {
       const int64_t t = (static_cast<int64_t>(b) * nM + m) * nN + n;
       const uint8_t k = cls[t];
-      if (k != BSA_TILE_EMPTY) {
-        keys[c++] = (static_cast<unsigned long long>(rank[t]) << 32) |
-                    (static_cast<unsigned long long>(m) << 1) | (k == BSA_TILE_FULL ? 1ull : 0ull);
-      }
+      ne = k != BSA_TILE_EMPTY;
+      if (ne)
+        key = (static_cast<unsigned long long>(rank[t]) << 32) |
+              (static_cast<unsigned long long>(m) << 1) | (k == BSA_TILE_FULL ? 1ull : 0ull);
     }
-    cnt = c;
+    const uint32_t bal = __ballot_sync(0xffffffffu, ne);
+    if (lane == 0) warp_cnt[wid] = __popc(bal);
+    __syncthreads();
+    int before = base_cnt;
+    for (int w = 0; w < wid; ++w) before += warp_cnt[w];
+    if (ne) keys[before + __popc(bal & ((1u << lane) - 1u))] = key;
+    __syncthreads();
+    if (threadIdx.x == 0)
+      for (int w = 0; w < nw; ++w) base_cnt += warp_cnt[w];
+    __syncthreads();
   }
-  __syncthreads();
-  const int c = cnt;
+  const int c = base_cnt;
   const int base = col_ptr[bn];
   for (int e = threadIdx.x; e < c; e += blockDim.x) {
     const unsigned long long ke = keys[e];
@@ -224,19 +275,6 @@ __global__ void k_col_fill(const uint8_t *__restrict__ cls, const int32_t *__res
     col_ent[base + pos] = m | ((ke & 1ull) ? kFullBit : 0u);
     col_rank[base + pos] = static_cast<int32_t>(ke >> 32);
   }
-}
-
-__global__ void k_signature(uint32_t *hdr, int B, int Sq, int Skv, uint32_t flags, int window,
-                            int order, int n_seqs) {
-  hdr[kHdrB] = B;
-  hdr[kHdrSq] = Sq;
-  hdr[kHdrSkv] = Skv;
-  hdr[kHdrFlags] = flags;
-  hdr[kHdrWindow] = window;
-  hdr[kHdrOrder] = order;
-  hdr[kHdrNSeqs] = n_seqs;
-  __threadfence();
-  hdr[kHdrMagic] = kPlanMagic;
 }
 
 inline unsigned cdiv(int64_t a, int64_t b) { return static_cast<unsigned>((a + b - 1) / b); }
@@ -276,6 +314,18 @@ cudaError_t launch_plan(const bsa_problem &p, const bsa_mask_spec &m, const bsa_
     kblk = kb;
   }
 
+  int32_t *rank = reinterpret_cast<int32_t *>(ws + L.rank);
+  int32_t *row_cnt = reinterpret_cast<int32_t *>(ws + L.row_cnt);
+  int32_t *row_ptr = reinterpret_cast<int32_t *>(ws + L.row_ptr);
+  int32_t *col_cnt = reinterpret_cast<int32_t *>(ws + L.col_cnt);
+  int32_t *col_ptr = reinterpret_cast<int32_t *>(ws + L.col_ptr);
+  int32_t *perm = reinterpret_cast<int32_t *>(ws + L.perm);
+  e = cudaMemsetAsync(col_cnt, 0, sizeof(int32_t) * B * nN, s);
+  if (e != cudaSuccess) return e;
+  if (o.bwd_order == BSA_ORDER_PERM) {
+    e = cudaMemcpyAsync(perm, o.perm, sizeof(int32_t) * nN, cudaMemcpyHostToDevice, s);
+    if (e != cudaSuccess) return e;
+  }
   ClassifyArgs ca;
   ca.B = B; ca.nM = nM; ca.nN = nN; ca.Sq = p.Sq; ca.Skv = p.Skv;
   ca.flags = m.flags;
@@ -284,28 +334,14 @@ cudaError_t launch_plan(const bsa_problem &p, const bsa_mask_spec &m, const bsa_
   ca.qblk = qblk;
   ca.kblk = kblk;
   ca.cls = ws + L.tile_class;
-  k_classify<<<cdiv(static_cast<int64_t>(B) * nM * nN, 256), 256, 0, s>>>(ca);
-  count_launch();
-
-  int32_t *perm = reinterpret_cast<int32_t *>(ws + L.perm);
-  if (o.bwd_order == BSA_ORDER_PERM) {
-    e = cudaMemcpyAsync(perm, o.perm, sizeof(int32_t) * nN, cudaMemcpyHostToDevice, s);
-    if (e != cudaSuccess) return e;
-  } else {
-    k_make_perm<<<cdiv(nN, 256), 256, 0, s>>>(nN, o.bwd_order, perm);
-    count_launch();
-  }
-
-  int32_t *rank = reinterpret_cast<int32_t *>(ws + L.rank);
-  int32_t *row_cnt = reinterpret_cast<int32_t *>(ws + L.row_cnt);
-  int32_t *row_ptr = reinterpret_cast<int32_t *>(ws + L.row_ptr);
-  int32_t *col_cnt = reinterpret_cast<int32_t *>(ws + L.col_cnt);
-  int32_t *col_ptr = reinterpret_cast<int32_t *>(ws + L.col_ptr);
-  k_row_rank<<<cdiv(B * nM, 128), 128, 0, s>>>(ws + L.tile_class, perm, B * nM, nN, rank, row_cnt);
-  k_col_count<<<cdiv(B * nN, 128), 128, 0, s>>>(ws + L.tile_class, B, nM, nN, col_cnt);
-  k_scan2<<<2, 1024, 0, s>>>(row_cnt, row_ptr, B * nM, col_cnt, col_ptr, B * nN);
-  k_row_fill<<<cdiv(B * nM, 128), 128, 0, s>>>(ws + L.tile_class, B * nM, nN, row_ptr,
-                                               reinterpret_cast<uint32_t *>(ws + L.row_ent));
+  ca.row_cnt = row_cnt;
+  ca.col_cnt = col_cnt;
+  k_classify_rows<<<cdiv(static_cast<int64_t>(B) * nM * 32, 256), 256, 0, s>>>(ca);
+  k_scan2<<<2, 1024, 0, s>>>(row_cnt, row_ptr, B * nM, col_cnt, col_ptr, B * nN, hdr, B, p.Sq,
+                             p.Skv, m.flags, m.window, o.bwd_order, m.n_seqs);
+  k_row_fill<<<cdiv(static_cast<int64_t>(B) * nM * 32, 256), 256, 0, s>>>(
+      ws + L.tile_class, B * nM, nN, o.bwd_order, perm, row_ptr,
+      reinterpret_cast<uint32_t *>(ws + L.row_ent), rank);
   const size_t smem = sizeof(unsigned long long) * static_cast<size_t>(nM);
   if (smem > 48 * 1024) {
     e = cudaFuncSetAttribute(k_col_fill, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -315,8 +351,7 @@ cudaError_t launch_plan(const bsa_problem &p, const bsa_mask_spec &m, const bsa_
   k_col_fill<<<B * nN, 256, smem, s>>>(ws + L.tile_class, rank, nM, nN, col_ptr,
                                        reinterpret_cast<uint32_t *>(ws + L.col_ent),
                                        reinterpret_cast<int32_t *>(ws + L.col_rank));
-  k_signature<<<1, 1, 0, s>>>(hdr, B, p.Sq, p.Skv, m.flags, m.window, o.bwd_order, m.n_seqs);
-  count_launch(6);
+  count_launch(4);
   return cudaGetLastError();
 }
 
