@@ -25,7 +25,7 @@ TILE = 128
 TILE_EMPTY, TILE_PARTIAL, TILE_FULL = 0, 1, 2
 MASK_SEGMENT_IDS, MASK_KV_VALID_LEN, MASK_VARLEN, MASK_CAUSAL_WINDOW = 1, 2, 4, 8
 SOFTMAX_ONLINE, SOFTMAX_FIXED_M_GATED = 0, 1
-ORDER = {"asc": 0, "desc": 1, "perm": 2}
+ORDER = {"asc": 0, "desc": 1, "perm": 2, "outside_in": 3, "greedy": 4}
 FULL_BIT = 1 << 30
 STATUS = {
     0: "BSA_OK", 1: "BSA_ERR_INVALID_ARG", 2: "BSA_ERR_UNSUPPORTED",

@@ -112,7 +112,7 @@ bsa_status normalise(const bsa_problem *in, bsa_problem *out) {
   bsa_problem &p = *out;
   if (p.B < 1 || p.H < 1 || p.Sq < 1 || p.Skv < 1) return BSA_ERR_INVALID_ARG;
   if (p.D != 64 && p.D != 128) return BSA_ERR_UNSUPPORTED;
-  if (p.Sq > (1 << 21) || p.Skv > (1 << 21)) return BSA_ERR_UNSUPPORTED;
+  if (p.Sq > kMaxSeq || p.Skv > kMaxSeq) return BSA_ERR_UNSUPPORTED;
   const int64_t nM = cdiv64(p.Sq, kTile), nN = cdiv64(p.Skv, kTile);
   if (static_cast<int64_t>(p.B) * nM * nN >= (int64_t{1} << 30)) return BSA_ERR_UNSUPPORTED;
   if (static_cast<int64_t>(p.B) * p.H * nM >= (int64_t{1} << 31)) return BSA_ERR_UNSUPPORTED;
@@ -169,7 +169,7 @@ bsa_status check_options(const bsa_options *o, int nN, bsa_options *out) {
   *out = *o;
   if (o->softmax_mode != BSA_SOFTMAX_ONLINE && o->softmax_mode != BSA_SOFTMAX_FIXED_M_GATED)
     return BSA_ERR_INVALID_ARG;
-  if (o->bwd_order < BSA_ORDER_ASC || o->bwd_order > BSA_ORDER_PERM) return BSA_ERR_INVALID_ARG;
+  if (o->bwd_order < BSA_ORDER_ASC || o->bwd_order > BSA_ORDER_GREEDY) return BSA_ERR_INVALID_ARG;
   if (o->bwd_order == BSA_ORDER_PERM) {
     if (o->perm == nullptr) return BSA_ERR_INVALID_ARG;
     std::vector<char> seen(static_cast<size_t>(nN), 0);

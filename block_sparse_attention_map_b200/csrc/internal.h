@@ -16,6 +16,8 @@ constexpr int kTile = BSA_TILE;
 constexpr uint32_t kFullBit = 1u << 30;
 constexpr uint32_t kIndexMask = (1u << 30) - 1u;
 constexpr uint32_t kPlanMagic = 0xB5A7C0DEu;
+// Largest Sq and Skv accepted (bsa_problem).
+constexpr int kMaxSeq = 1 << 21;
 
 // Header words at the start of the workspace.
 enum HeaderWord : int {

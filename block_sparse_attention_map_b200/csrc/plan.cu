@@ -191,11 +191,83 @@ __global__ void k_scan2(const int32_t *__restrict__ c0, int32_t *__restrict__ p0
   }
 }
 
+// pi[t] for the orders with a closed form: ascending, descending, and
+// outside-in (0, nN-1, 1, nN-2, ...).
+__device__ __forceinline__ int closed_form_order(int order, int t, int nN) {
+  if (order == BSA_ORDER_DESC) return nN - 1 - t;
+  if (order == BSA_ORDER_OUTSIDE_IN) return (t & 1) ? nN - 1 - (t >> 1) : (t >> 1);
+  return t;
+}
+
+__device__ __forceinline__ bool order_in_workspace(int order) {
+  return order == BSA_ORDER_PERM || order == BSA_ORDER_GREEDY;
+}
+
+// The greedy order, one block: the columns are placed one at a time; w[n] is
+// the presumed semaphore wait of column n if it came next, the number of
+// (already placed column, row block) pairs that share a non-empty row block
+// with it, summed over all batches.  Each step takes the smallest (w[n], n)
+// among the unplaced columns, then adds one to w[n'] for every unplaced n'
+// per row block the placed column reaches (a warp per row block).
+static_assert(sizeof(int32_t) * (kMaxSeq / kTile) <= 64 * 1024,
+              "the greedy order keeps one presumed wait per kv block in shared memory");
+__global__ void __launch_bounds__(1024) k_greedy_order(const uint8_t *__restrict__ cls, int BnM,
+                                                       int nN, int32_t *__restrict__ perm) {
+  extern __shared__ int32_t w[];
+  __shared__ unsigned long long red[32];
+  __shared__ int chosen;
+  constexpr int32_t kPlaced = 0x7fffffff;
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  for (int n = threadIdx.x; n < nN; n += blockDim.x) w[n] = 0;
+  __syncthreads();
+  for (int step = 0; step < nN; ++step) {
+    unsigned long long best = ~0ull;
+    for (int n = threadIdx.x; n < nN; n += blockDim.x) {
+      const int32_t x = w[n];
+      if (x != kPlaced) {
+        const unsigned long long key = (static_cast<unsigned long long>(x) << 32) |
+                                       static_cast<unsigned>(n);
+        best = key < best ? key : best;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const unsigned long long y = __shfl_xor_sync(0xffffffffu, best, o);
+      best = y < best ? y : best;
+    }
+    if (lane == 0) red[wid] = best;
+    __syncthreads();
+    if (wid == 0) {
+      unsigned long long v = lane < nw ? red[lane] : ~0ull;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const unsigned long long y = __shfl_xor_sync(0xffffffffu, v, o);
+        v = y < v ? y : v;
+      }
+      if (lane == 0) {
+        const int c = static_cast<int>(v & 0xffffffffull);
+        chosen = c;
+        perm[step] = c;
+        w[c] = kPlaced;
+      }
+    }
+    __syncthreads();
+    const int c = chosen;
+    for (int bm = wid; bm < BnM; bm += nw) {
+      const uint8_t *row = cls + static_cast<int64_t>(bm) * nN;
+      if (row[c] == BSA_TILE_EMPTY) continue;
+      for (int n = lane; n < nN; n += 32)
+        if (row[n] != BSA_TILE_EMPTY && w[n] != kPlaced) atomicAdd(w + n, 1);
+    }
+    __syncthreads();
+  }
+}
+
 // One warp per (b, m): the forward's row list (ascending n, FULL flag in bit
 // 30) and rank(m, n): row m's non-empty columns numbered 0, 1, 2, ... in the
-// order pi (-1 for empty tiles).  pi is ascending, descending, or the
-// caller's permutation already in the workspace; warp 0 writes it out for
-// the asc / desc orders.
+// order pi (-1 for empty tiles).  pi has a closed form, or is the caller's
+// permutation or the greedy order already in the workspace; warp 0 writes it
+// out for the closed forms.
 __global__ void k_row_fill(const uint8_t *__restrict__ cls, int BnM, int nN, int order,
                            int32_t *__restrict__ perm, const int32_t *__restrict__ row_ptr,
                            uint32_t *__restrict__ row_ent, int32_t *__restrict__ rank) {
@@ -203,8 +275,9 @@ __global__ void k_row_fill(const uint8_t *__restrict__ cls, int BnM, int nN, int
   const int lane = threadIdx.x & 31;
   if (wid >= BnM) return;
   const uint8_t *row = cls + static_cast<int64_t>(wid) * nN;
-  if (wid == 0 && order != BSA_ORDER_PERM)
-    for (int t = lane; t < nN; t += 32) perm[t] = order == BSA_ORDER_DESC ? nN - 1 - t : t;
+  const bool in_ws = order_in_workspace(order);
+  if (wid == 0 && !in_ws)
+    for (int t = lane; t < nN; t += 32) perm[t] = closed_form_order(order, t, nN);
   int pos = row_ptr[wid];
   for (int n0 = 0; n0 < nN; n0 += 32) {
     const int n = n0 + lane;
@@ -219,7 +292,7 @@ __global__ void k_row_fill(const uint8_t *__restrict__ cls, int BnM, int nN, int
   for (int t0 = 0; t0 < nN; t0 += 32) {
     const int t = t0 + lane;
     int n = -1;
-    if (t < nN) n = order == BSA_ORDER_PERM ? perm[t] : (order == BSA_ORDER_DESC ? nN - 1 - t : t);
+    if (t < nN) n = in_ws ? perm[t] : closed_form_order(order, t, nN);
     const bool ne = n >= 0 && row[n] != BSA_TILE_EMPTY;
     const uint32_t bal = __ballot_sync(0xffffffffu, ne);
     if (n >= 0) rk[n] = ne ? r + __popc(bal & ((1u << lane) - 1u)) : -1;
@@ -339,6 +412,16 @@ cudaError_t launch_plan(const bsa_problem &p, const bsa_mask_spec &m, const bsa_
   k_classify_rows<<<cdiv(static_cast<int64_t>(B) * nM * 32, 256), 256, 0, s>>>(ca);
   k_scan2<<<2, 1024, 0, s>>>(row_cnt, row_ptr, B * nM, col_cnt, col_ptr, B * nN, hdr, B, p.Sq,
                              p.Skv, m.flags, m.window, o.bwd_order, m.n_seqs);
+  if (o.bwd_order == BSA_ORDER_GREEDY) {
+    const size_t gsm = sizeof(int32_t) * static_cast<size_t>(nN);
+    if (gsm > 48 * 1024) {
+      e = cudaFuncSetAttribute(k_greedy_order, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(gsm));
+      if (e != cudaSuccess) return e;
+    }
+    k_greedy_order<<<1, 1024, gsm, s>>>(ws + L.tile_class, B * nM, nN, perm);
+    count_launch();
+  }
   k_row_fill<<<cdiv(static_cast<int64_t>(B) * nM * 32, 256), 256, 0, s>>>(
       ws + L.tile_class, B * nM, nN, o.bwd_order, perm, row_ptr,
       reinterpret_cast<uint32_t *>(ws + L.row_ent), rank);

@@ -99,12 +99,22 @@ typedef enum bsa_status {
 #define BSA_ORDER_ASC 0
 #define BSA_ORDER_DESC 1
 #define BSA_ORDER_PERM 2
+/* The two orders the "dk order" page's benchmark table names without defining
+ * them, under the readings this library takes:
+ *   OUTSIDE_IN  0, nN-1, 1, nN-2, ... (both ends first, then inwards);
+ *   GREEDY      columns placed one at a time; each step takes the unplaced
+ *               column whose non-empty tiles would wait on the most already
+ *               placed tiles of their row blocks the least in total (ties: the
+ *               smaller column), computed on the GPU by bsa_plan_build from
+ *               the tile classes of all batches (one block; nN steps). */
+#define BSA_ORDER_OUTSIDE_IN 3
+#define BSA_ORDER_GREEDY 4
 
 typedef struct bsa_problem {
   int32_t B;       /* batch; 1 for varlen                                        */
   int32_t H;       /* heads (Q, K and V have the same head count)                */
-  int32_t Sq;      /* query rows per batch (varlen: total tokens T)               */
-  int32_t Skv;     /* keys per batch (varlen: T)                                  */
+  int32_t Sq;      /* query rows per batch (varlen: total tokens T); <= 2^21      */
+  int32_t Skv;     /* keys per batch (varlen: T); <= 2^21                         */
   int32_t D;       /* head dim, 64 or 128                                         */
   int32_t reserved0;
   /* element strides (batch, seq, head); all zero = contiguous BSHD.  q_stride

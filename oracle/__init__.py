@@ -32,6 +32,7 @@ from .blockmap import (  # noqa: F401
     FULL,
     tile_classes,
     column_order,
+    greedy_order,
     kv_ranks,
     column_lists,
     partial_then_full_lists,

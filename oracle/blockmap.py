@@ -46,22 +46,68 @@ def tile_classes(mask: MaskDesc, B: int, Sq: int, Skv: int, tile: int = 128) -> 
     return cls
 
 
-def column_order(nN: int, order: str = "asc", perm=None) -> np.ndarray:
-    """pi: the kv-column iteration order (flash-attention PR #2512, "What does this do").
+def column_order(nN: int, order: str = "asc", perm=None, cls=None) -> np.ndarray:
+    """pi: the kv-column iteration order (flash-attention PR #2512, "What does this
+    do" and "The numbers").
 
     "asc" walks columns left to right, "desc" right to left, "perm" takes an
-    arbitrary permutation of range(nN).
+    arbitrary permutation of range(nN).  The page's table also names
+    "outside_in" and "greedy" without defining them; the readings taken here:
+
+    * outside_in: the two ends first, then inwards: 0, nN-1, 1, nN-2, ...
+    * greedy: see :func:`greedy_order` (needs the tile classes ``cls``).
     """
     if order == "asc":
         return np.arange(nN)
     if order == "desc":
         return np.arange(nN)[::-1].copy()
+    if order == "outside_in":
+        out = []
+        lo, hi = 0, nN - 1
+        while lo <= hi:
+            out.append(lo)
+            if hi != lo:
+                out.append(hi)
+            lo, hi = lo + 1, hi - 1
+        return np.asarray(out, dtype=np.int64)
+    if order == "greedy":
+        return greedy_order(cls)
     if order == "perm":
         p = np.asarray(perm, dtype=np.int64)
         if sorted(p.tolist()) != list(range(nN)):
             raise ValueError("perm is not a permutation of the kv blocks")
         return p
     raise ValueError(order)
+
+
+def greedy_order(cls: np.ndarray) -> np.ndarray:
+    """A greedy order on presumed semaphore wait (flash-attention PR #2512, "What
+    does this do": a scheduling heuristic for presumed semaphore wait time).
+
+    Reading taken: the columns are placed one at a time.  Placing column n gives
+    each of its non-empty tiles (b, m, n) the rank cnt[b, m] = number of columns
+    already placed that also reach row block m, and that column must wait for
+    all of them.  At every step the unplaced column with the smallest total
+    presumed wait sum_{b, m non-empty} cnt[b, m] is placed (ties: smaller n),
+    then cnt[b, m] += 1 for its rows.
+    """
+    B, nM, nN = cls.shape
+    ne = cls != EMPTY
+    cnt = np.zeros((B, nM), dtype=np.int64)
+    placed = np.zeros(nN, dtype=bool)
+    out = []
+    for _ in range(nN):
+        best, best_w = -1, None
+        for n in range(nN):
+            if placed[n]:
+                continue
+            w = int((cnt * ne[:, :, n]).sum())
+            if best_w is None or w < best_w:
+                best, best_w = n, w
+        out.append(best)
+        placed[best] = True
+        cnt += ne[:, :, best]
+    return np.asarray(out, dtype=np.int64)
 
 
 def kv_ranks(cls: np.ndarray, pi: np.ndarray) -> np.ndarray:

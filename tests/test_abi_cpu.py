@@ -133,6 +133,10 @@ def test_calls_reject_bad_arguments_before_cuda(L):
     bad = (ctypes.c_int32 * 2)(0, 0)
     o.perm = ctypes.cast(bad, ctypes.c_void_p)
     assert L.bsa_plan_build(ctypes.byref(p), None, ctypes.byref(o), 4096, 1 << 30, None) == 1
+    # an order past the last one
+    o = bd.Options()
+    o.bwd_order = 5
+    assert L.bsa_plan_build(ctypes.byref(p), None, ctypes.byref(o), 4096, 16, None) == 1
     # workspace too small
     o = bd.Options()
     assert L.bsa_plan_build(ctypes.byref(p), None, ctypes.byref(o), 4096, 16, None) == 3

@@ -63,7 +63,7 @@ def test_bwd_matches_oracle(name):
     assert max(e) <= O_TOL, e
 
 
-@pytest.mark.parametrize("order", ["asc", "desc", "perm"])
+@pytest.mark.parametrize("order", ["asc", "desc", "perm", "outside_in", "greedy"])
 def test_bwd_orders_match_oracle_and_repeat_bitwise(order):
     wl = make_workload("window", device="cuda", small=True)
     nN = -(-wl.Skv // 128)

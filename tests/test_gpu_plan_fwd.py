@@ -33,15 +33,15 @@ def test_plan_full_size_window_counts(name, B, Sq, Skv):
     assert np.array_equal(cls, ref)
 
 
-@pytest.mark.parametrize("order", ["asc", "desc", "perm"])
-@pytest.mark.parametrize("name", ["window", "packed", "window_rect"])
+@pytest.mark.parametrize("order", ["asc", "desc", "perm", "outside_in", "greedy"])
+@pytest.mark.parametrize("name", ["window", "packed", "window_rect", "varlen"])
 def test_plan_ranks_and_column_lists(name, order):
     wl = make_workload(name, device="cuda", small=True)
     nN = -(-wl.Skv // 128)
     perm = np.random.default_rng(5).permutation(nN) if order == "perm" else None
     ws = bsa.plan_build(wl.q, wl.k, wl.v, wl.mask, order=order, perm=perm)
     cls = oracle.tile_classes(mask_desc(wl), wl.B, wl.Sq, wl.Skv)
-    pi = oracle.column_order(nN, order, perm)
+    pi = oracle.column_order(nN, order, perm, cls=cls)
     assert np.array_equal(ws.perm().cpu().numpy(), pi)
     rank = oracle.kv_ranks(cls, pi)
     assert np.array_equal(ws.ranks().cpu().numpy(), rank)
@@ -60,6 +60,18 @@ def test_plan_ranks_and_column_lists(name, order):
             got = [(int(x & (bsa._binding.FULL_BIT - 1)), bool(x & bsa._binding.FULL_BIT)) for x in rent[s:e]]
             exp = [(n, cls[b, m, n] == oracle.FULL) for n in range(nN) if cls[b, m, n] != oracle.EMPTY]
             assert got == exp
+
+
+@pytest.mark.parametrize("name", ["window", "video"])
+def test_plan_greedy_order_full_size(name):
+    # the greedy kernel over every column of the full-size block maps
+    wl = make_workload(name, device="cuda")
+    ws = bsa.plan_build(wl.q, wl.k, wl.v, wl.mask, order="greedy")
+    cls = ws.tile_classes().cpu().numpy()
+    if name == "window":
+        assert np.array_equal(cls, oracle.tile_classes(mask_desc(wl), wl.B, wl.Sq, wl.Skv))
+    assert np.array_equal(ws.perm().cpu().numpy(), oracle.greedy_order(cls))
+    assert ws.status() == 0
 
 
 def _fwd_vs_oracle(wl, mode="online", rows=None):

@@ -134,3 +134,46 @@ def test_random_segment_ids_classes_are_consistent_with_dense_mask():
             blk = a[m * 128:(m + 1) * 128, n * 128:(n + 1) * 128]
             full = blk.all() and blk.shape[1] == 128
             assert cls[0, m, n] == (FULL if full else PARTIAL if blk.any() else EMPTY)
+
+
+def test_outside_in_order_closed_form():
+    assert oracle.column_order(6, "outside_in").tolist() == [0, 5, 1, 4, 2, 3]
+    assert oracle.column_order(5, "outside_in").tolist() == [0, 4, 1, 3, 2]
+    assert oracle.column_order(1, "outside_in").tolist() == [0]
+
+
+def test_greedy_order_hand_worked_causal_example():
+    # Causal 3 x 3 block map: column 0 reaches rows {0,1,2}, column 1 {1,2},
+    # column 2 {2}.  Step 1: every wait is 0 -> column 0.  Step 2: column 1
+    # would wait 1 + 1 = 2, column 2 only 1 -> column 2.  Then column 1.
+    cls = np.array([[[PARTIAL, EMPTY, EMPTY],
+                     [FULL, PARTIAL, EMPTY],
+                     [FULL, FULL, PARTIAL]]], dtype=np.uint8)
+    assert oracle.greedy_order(cls).tolist() == [0, 2, 1]
+
+
+def test_greedy_order_is_a_permutation_with_minimal_step_waits():
+    cls = oracle.tile_classes(MaskDesc(window=512), 2, 2048, 3072)
+    pi = oracle.column_order(cls.shape[2], "greedy", cls=cls)
+    assert sorted(pi.tolist()) == list(range(cls.shape[2]))
+    ne = cls != EMPTY
+    cnt = np.zeros(cls.shape[:2], dtype=np.int64)
+    placed = set()
+    for n in pi:
+        waits = {c: int((cnt * ne[:, :, c]).sum()) for c in range(cls.shape[2]) if c not in placed}
+        assert waits[int(n)] == min(waits.values())
+        assert int(n) == min(c for c, w in waits.items() if w == waits[int(n)])
+        placed.add(int(n))
+        cnt += ne[:, :, n]
+
+
+@pytest.mark.parametrize("order", ["outside_in", "greedy"])
+def test_new_orders_deadlock_free_and_ordered(order):
+    cls = oracle.tile_classes(MaskDesc(window=512), 1, 4096, 4096)
+    nN = cls.shape[2]
+    pi = oracle.column_order(nN, order, cls=cls)
+    rank = oracle.kv_ranks(cls, pi)
+    done, _, acc = oracle.simulate_dq_semaphores(oracle.column_lists(cls, rank), pi, 1, cls.shape[1], 24)
+    assert done
+    for (b, m), seq in acc.items():
+        assert seq == [int(n) for n in pi if cls[b, m, n] != EMPTY]
