@@ -20,7 +20,10 @@ Sources (the pages of the subject):
 * sglang PR #47566, "Modifications": varlen ``cu_seqlens`` whose trailing
   alignment segment is never attended by real rows; alignment rows are zeroed.
 * "Add more optimal dk order optional arg" (flash-attention PR #2512): sliding
-  window masks (causal band of W keys) and the backward dQ/dK/dV.
+  window masks (causal band of W keys) and the backward dQ/dK/dV.  Its
+  benchmark ("The numbers") also names prefix_lm, dilated_sliding_window and
+  document masks without defining them; the readings taken are stated in
+  :class:`MaskDesc` and :func:`allowed_rows`.
 """
 
 from __future__ import annotations
@@ -43,6 +46,14 @@ class MaskDesc:
     n_align_tail  : number of trailing cu_seqlens segments that are alignment rows
     window        : None = no window; 0 = plain causal; W > 0 = causal band of W
                     keys including the diagonal, bottom-right aligned.
+    dilation      : (with a window) keep only the keys whose distance back from
+                    the diagonal is a multiple of ``dilation`` (<= 1: all keys);
+                    the reading taken for "dilated_sliding_window".
+    prefix_len    : int array [B] (with a window): keys j < prefix_len[b] are
+                    seen by every row as well; the reading taken for
+                    "prefix_lm" (a bidirectional prefix, causal after it).
+    "document" masks are segment ids (one id per document), optionally with
+    a window (document-causal).
     """
 
     seg_q: Optional[np.ndarray] = None
@@ -51,6 +62,8 @@ class MaskDesc:
     cu_seqlens: Optional[np.ndarray] = None
     n_align_tail: int = 0
     window: Optional[int] = None
+    dilation: int = 1
+    prefix_len: Optional[np.ndarray] = None
 
 
 def _segment_of(cu_seqlens: np.ndarray, pos: np.ndarray) -> np.ndarray:
@@ -67,8 +80,11 @@ def allowed_rows(mask: MaskDesc, b: int, rows: np.ndarray, Sq: int, Skv: int) ->
       cu_seqlens segment and neither lies in one of the trailing ``n_align_tail``
       alignment segments
     * causal window (flash-attention PR #2512 sliding_window masks; causal and
-      bottom-right aligned when Sq != Skv): with o = Skv - Sq,
-      i + o - W < j <= i + o   (W = 0: only j <= i + o)
+      bottom-right aligned when Sq != Skv): with o = Skv - Sq and the distance
+      t = i + o - j of key j back from the diagonal,
+      0 <= t < W   (W = 0: only 0 <= t),
+      with a dilation d > 1 also t mod d == 0 (dilated_sliding_window), and with
+      a prefix OR j < prefix_len[b] (prefix_lm).
     """
     rows = np.asarray(rows, dtype=np.int64)
     i = rows[:, None]
@@ -87,10 +103,17 @@ def allowed_rows(mask: MaskDesc, b: int, rows: np.ndarray, Sq: int, Skv: int) ->
         sj = _segment_of(cu, np.arange(Skv))
         ok &= (si[:, None] == sj[None, :]) & (si[:, None] < n_real) & (sj[None, :] < n_real)
     if mask.window is not None:
-        o = Skv - Sq
-        ok &= j <= i + o
+        t = (i + (Skv - Sq)) - j
+        band = t >= 0
         if mask.window > 0:
-            ok &= j > i + o - int(mask.window)
+            band &= t < int(mask.window)
+        if mask.dilation > 1:
+            band &= np.mod(t, int(mask.dilation)) == 0
+        if mask.prefix_len is not None:
+            band |= j < int(np.asarray(mask.prefix_len)[b])
+        ok &= band
+    elif mask.prefix_len is not None or mask.dilation > 1:
+        raise ValueError("a prefix or a dilation modifies the causal window; set window")
     return ok
 
 

@@ -105,4 +105,7 @@ def tiny_masks(B, Sq, Skv, seed=0):
         "segments": MaskDesc(seg_q=seg_q, seg_kv=seg_kv),
         "seg+window": MaskDesc(seg_q=seg_q, seg_kv=seg_kv, window=4),
         "pad+causal": MaskDesc(kv_valid_len=np.array([Skv - 2] * B), window=0),
+        "prefix_lm": MaskDesc(window=0, prefix_len=np.array([3, 1] * B)[:B]),
+        "dilated": MaskDesc(window=6, dilation=2),
+        "doc_causal": MaskDesc(seg_q=seg_q, seg_kv=seg_kv, window=0),
     }

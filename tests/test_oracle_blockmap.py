@@ -177,3 +177,26 @@ def test_new_orders_deadlock_free_and_ordered(order):
     assert done
     for (b, m), seq in acc.items():
         assert seq == [int(n) for n in pi if cls[b, m, n] != EMPTY]
+
+
+def test_prefix_lm_tile_counts_closed_form():
+    # causal, prefix of 2048 keys = kv blocks 0..15: rows m < 16 reach exactly
+    # those 16 blocks (all full); row m >= 16 adds blocks 16..m-1 (full) and the
+    # diagonal block m (partial): 16*16 + sum_{m=16}^{63} (m + 1) tiles.
+    cls = oracle.tile_classes(MaskDesc(window=0, prefix_len=np.array([2048])), 1, 8192, 8192)
+    assert _counts(cls) == (2200, 2152, 48)
+
+
+def test_dilated_window_tile_counts_closed_form():
+    # span 1024, dilation 2: row block m reaches blocks max(0, m-8) .. m; no
+    # 128-key block can be full when only every other key is kept.
+    cls = oracle.tile_classes(MaskDesc(window=1024, dilation=2), 1, 8192, 8192)
+    assert _counts(cls) == (36 + 56 * 9, 0, 540)
+
+
+def test_document_causal_tile_counts_closed_form():
+    # documents of 128, 256, 128, 512 tokens, causal inside each: the diagonal
+    # blocks are partial, the same-document blocks below them full.
+    ids = np.repeat(np.arange(4), [128, 256, 128, 512])[None, :]
+    cls = oracle.tile_classes(MaskDesc(seg_q=ids, seg_kv=ids, window=0), 1, 1024, 1024)
+    assert _counts(cls) == (15, 7, 8)

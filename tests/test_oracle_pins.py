@@ -29,7 +29,8 @@ def test_forward_matches_brute_force(case):
     assert np.max(np.abs(L[fin] - Lb[fin])) < 1e-12
 
 
-@pytest.mark.parametrize("case", ["none", "causal", "window3", "padding", "segments", "seg+window"])
+@pytest.mark.parametrize("case", ["none", "causal", "window3", "padding", "segments", "seg+window",
+                                  "prefix_lm", "dilated", "doc_causal"])
 def test_forward_matches_library_sdpa(case):
     q, k, v, _ = P.tiny_inputs(2, B=2, Sq=12, Skv=12, D=6)
     mask = P.tiny_masks(2, 12, 12, seed=3)[case]
@@ -41,7 +42,8 @@ def test_forward_matches_library_sdpa(case):
     assert np.max(np.abs(O - Os)) < 1e-12
 
 
-@pytest.mark.parametrize("case", ["none", "causal", "window3", "padding", "segments"])
+@pytest.mark.parametrize("case", ["none", "causal", "window3", "padding", "segments", "prefix_lm",
+                                  "dilated"])
 def test_backward_matches_autograd(case):
     q, k, v, dO = P.tiny_inputs(4, B=2, Sq=10, Skv=10, D=4)
     v = v[..., :4].copy()
@@ -130,6 +132,57 @@ def test_mask_predicates_count_keys():
     assert not a[31:].any() and not a[:, 31:].any()
     a = oracle.allowed_rows(MaskDesc(kv_valid_len=np.array([5, 9])), 1, np.arange(4), 4, 12)
     assert (a.sum(axis=1) == 9).all()
+
+
+def test_prefix_lm_predicate_counts_keys():
+    # causal with a bidirectional prefix of P keys: row i sees keys 0 .. max(P, i+1) - 1
+    Sq = Skv = 40
+    for P_ in (0, 7, 40, 60):
+        a = oracle.allowed_rows(MaskDesc(window=0, prefix_len=np.array([P_])), 0, np.arange(Sq), Sq, Skv)
+        for i in range(Sq):
+            n = min(Skv, max(P_, i + 1))
+            assert a[i].sum() == n and a[i, :n].all()
+    # with a window of 5: the prefix 0..6 and the band i-4 .. i, overlapping or not
+    a = oracle.allowed_rows(MaskDesc(window=5, prefix_len=np.array([7])), 0, np.arange(Sq), Sq, Skv)
+    for i in range(Sq):
+        band_lo = max(0, i - 4)
+        assert a[i].sum() == (max(7, i + 1) if band_lo <= 7 else 7 + 5)
+        assert a[i, :7].all() and a[i, band_lo:i + 1].all()
+
+
+def test_dilated_window_predicate_counts_keys():
+    # span W = 10, dilation 3: keys i, i-3, i-6, i-9 (those >= 0)
+    Sq = Skv = 20
+    a = oracle.allowed_rows(MaskDesc(window=10, dilation=3), 0, np.arange(Sq), Sq, Skv)
+    for i in range(Sq):
+        assert a[i].sum() == min(4, i // 3 + 1)
+        assert a[i, i] and (i < 3 or a[i, i - 3]) and (i < 1 or not a[i, i - 1])
+        assert i < 12 or not a[i, i - 12]
+    # bottom-right alignment with Sq < Skv: the last row's diagonal is the last key
+    a = oracle.allowed_rows(MaskDesc(window=8, dilation=2), 0, np.arange(6), 6, 13)
+    assert a[5].nonzero()[0].tolist() == [6, 8, 10, 12]
+    with pytest.raises(ValueError):
+        oracle.allowed_rows(MaskDesc(dilation=2), 0, np.arange(4), 4, 4)
+
+
+def test_prefix_covering_every_key_is_no_mask():
+    q, k, v, _ = P.tiny_inputs(12, B=1, Sq=9, Skv=11, D=4)
+    O, _ = oracle.attention_forward(q, k, v, MaskDesc(window=2, prefix_len=np.array([11])), SCALE)
+    allowed = [np.ones((9, 11), dtype=bool)]
+    assert np.max(np.abs(O - P.sdpa_forward(q, k, v, allowed, SCALE))) < 1e-12
+
+
+def test_dilated_rows_equal_attention_over_gathered_keys():
+    # each row's output is plain attention over its own keys i+o, i+o-d, ...
+    q, k, v, _ = P.tiny_inputs(13, B=1, Sq=10, Skv=14, D=5)
+    O, L = oracle.attention_forward(q, k, v, MaskDesc(window=9, dilation=4), SCALE)
+    o = 14 - 10
+    for i in range(10):
+        keys = [i + o - 4 * t for t in range(3) if i + o - 4 * t >= 0]
+        s = SCALE * (k[0, keys, 0, :] @ q[0, i, 0, :])
+        w = np.exp(s - s.max())
+        assert np.allclose(O[0, i, 0], (w / w.sum()) @ v[0, keys, 0, :], atol=1e-13)
+        assert abs(L[0, 0, i] - (s.max() + math.log(w.sum()))) < 1e-13
 
 
 # ---------------------------------------------------------------- invariants
