@@ -15,6 +15,10 @@ per-tile flops 4*128*128*D forward and 2.5x that backward.  L2 is flushed
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
+The other mask families and kv-column orders are measured the same way with
+--workload prefix_lm|dilated|document|window_rect, --order desc|outside_in|greedy
+and --nondet (the atomic dQ backward).
+
 With N > 1 it runs under torch.distributed.run, one rank per GPU, every rank
 running the same workload (replicas: the (b, h) units are independent and
 the path has no exchange step); value = work of all ranks / max rank time.
@@ -35,8 +39,22 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 WORKLOAD_NAME = "window"
-WORKLOAD_TEXT = ("causal sliding window 512: B=1, H=16, Sq=Skv=8192, D=128, bf16 N(0,1) seed 2; "
-                 "forward fixed-m gated + deterministic backward (ascending kv-column order)")
+WORKLOADS = {
+    "window": "causal sliding window 512: B=1, H=16, Sq=Skv=8192, D=128, bf16 N(0,1) seed 2",
+    "window_rect": "causal sliding window 512, bottom-right: B=1, H=16, Sq=4096, Skv=8192, D=128, "
+                   "bf16 N(0,1) seed 2",
+    "prefix_lm": "prefix-LM (causal + bidirectional prefix of 2048): B=1, H=16, Sq=Skv=8192, "
+                 "D=128, bf16 N(0,1) seed 2",
+    "dilated": "dilated causal window (span 1024, dilation 2): B=1, H=16, Sq=Skv=8192, D=128, "
+               "bf16 N(0,1) seed 2",
+    "document": "document-causal (runs of 256..2048 tokens): B=1, H=16, Sq=Skv=8192, D=128, "
+                "bf16 N(0,1) seed 2",
+}
+
+
+def workload_text(args):
+    bwd = "atomic (non-deterministic)" if args.nondet else f"deterministic ({args.order} kv-column order)"
+    return f"{WORKLOADS[args.workload]}; forward {args.softmax} + {bwd} backward"
 METRIC = "attention TFLOP/s (non-empty tiles) fwd+bwd on 1 B200; % of bf16 tensor peak"
 
 
@@ -47,7 +65,9 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--softmax", default="fixed_m", choices=["fixed_m", "online"])
-    ap.add_argument("--order", default="asc", choices=["asc", "desc"])
+    ap.add_argument("--order", default="asc", choices=["asc", "desc", "outside_in", "greedy"])
+    ap.add_argument("--nondet", action="store_true", help="atomic (non-deterministic) dQ backward")
+    ap.add_argument("--workload", default=WORKLOAD_NAME, choices=sorted(WORKLOADS))
     ap.add_argument("--small", action="store_true",
                     help="small shape of the same workload (for profiler captures)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -193,10 +213,13 @@ def oracle_sample(wl, n_rows: int, head: int = 0):
     q = f(wl.q[:, :n_rows, head:head + 1])
     k, v = f(wl.k[:, :, head:head + 1]), f(wl.v[:, :, head:head + 1])
     do = f(wl.dO[:, :n_rows, head:head + 1])
-    mask = oracle.MaskDesc(**wl.mask_numpy())
-    # the sample treats rows [0, n_rows) as the query set: the window's bottom-right
-    # offset must stay that of the full problem, so use Sq=Skv rows and a square cut
-    sub = oracle.MaskDesc(window=mask.window) if mask.window is not None else mask
+    # the sample treats rows and keys [0, n_rows) as a square problem with the
+    # same mask predicates (segment ids cut to the sample)
+    desc = wl.mask_numpy()
+    for key in ("seg_q", "seg_kv"):
+        if key in desc:
+            desc[key] = desc[key][:, :n_rows]
+    sub = oracle.MaskDesc(**desc)
     cls = oracle.tile_classes(sub, 1, n_rows, n_rows)
     t0 = time.perf_counter()
     oracle.attention_forward(q, k[:, :n_rows], v[:, :n_rows], sub, wl.scale)
@@ -213,7 +236,7 @@ def run_reference(args, world, rank):
     from block_sparse_attention_map_b200.workloads import make_workload
     if rank != 0:
         return
-    wl = make_workload(WORKLOAD_NAME, device="cpu", small=args.small)
+    wl = make_workload(args.workload, device="cpu", small=args.small)
     n_rows = min(1024, wl.Sq)
     for _ in range(args.warmup):
         oracle_sample(wl, n_rows)
@@ -223,15 +246,15 @@ def run_reference(args, world, rank):
         total_t += dt
         total_f += fl
     value = total_f / total_t / 1e12
-    sample = (f"rows 0..{n_rows - 1} of head 0 of {wl.H} (one causal band of {n_rows} keys), "
+    sample = (f"rows and keys 0..{n_rows - 1} of head 0 of {wl.H} under the same mask, "
               f"forward + backward in fp64, per step")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * total_t / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": WORKLOAD_TEXT, "global_batch": wl.B, "seq_len": wl.Sq,
-                   "heads": wl.H, "head_dim": wl.D, "window": 512},
+        "config": {"workload": workload_text(args), "global_batch": wl.B, "seq_len": wl.Sq,
+                   "heads": wl.H, "head_dim": wl.D, "mask": wl.mask_text()},
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -247,8 +270,9 @@ def run_ours(args, world, rank, local):
     from block_sparse_attention_map_b200.workloads import make_workload
 
     dev = torch.device("cuda", local)
-    wl = make_workload(WORKLOAD_NAME, device=dev, small=args.small)
-    st = bsa.Stages(wl.q, wl.k, wl.v, wl.mask, softmax_mode=args.softmax, order=args.order)
+    wl = make_workload(args.workload, device=dev, small=args.small)
+    st = bsa.Stages(wl.q, wl.k, wl.v, wl.mask, softmax_mode=args.softmax, order=args.order,
+                    deterministic=not args.nondet)
     dO = wl.dO
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
@@ -318,16 +342,18 @@ def run_ours(args, world, rank, local):
     peak = peaks["bf16_tflops"]
     main_tf = f_bwd / (avg["backward_main"] * 1e-3) / 1e12
     fwd_tf = f_fwd / (avg["forward"] * 1e-3) / 1e12
-    traffic = profiled_traffic("k_attn_bwd", "window8192")
+    tag = f"{args.workload}{wl.Sq}" if not args.small else None
+    traffic = profiled_traffic("k_attn_bwd", tag) if not args.nondet else None
 
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": WORKLOAD_TEXT + (" [small shape]" if args.small else ""),
+        "config": {"workload": workload_text(args) + (" [small shape]" if args.small else ""),
                    "global_batch": wl.B * world, "seq_len": wl.Sq, "heads": wl.H,
-                   "head_dim": wl.D, "window": 512, "nonempty_tiles": n_tiles,
-                   "softmax": args.softmax, "bwd_order": args.order,
+                   "head_dim": wl.D, "mask": wl.mask_text(), "nonempty_tiles": n_tiles,
+                   "softmax": args.softmax,
+                   "bwd_order": "nondeterministic" if args.nondet else args.order,
                    "l2": "flushed (256 MiB write) before every step, outside the timed events",
                    "parallelism": f"replicas x{world}"},
         "pct_of_bf16_peak": 100.0 * value / peak,
@@ -341,7 +367,7 @@ def run_ours(args, world, rank, local):
                      "traffic": traffic, "peak_source": peaks["source"] + " bf16 burst"},
         "roofline_forward": {"kernel": "k_attn_fwd (a3)", "bound": "tensor", "achieved": fwd_tf,
                              "peak": peak, "unit": "TFLOP/s", "frac": fwd_tf / peak,
-                             "traffic": profiled_traffic("k_attn_fwd", "window8192")},
+                             "traffic": profiled_traffic("k_attn_fwd", tag)},
         "gpu_launches": launches,
         "wall_s_timed_loop": t_wall,
         "clocks": clk.summary(),
@@ -354,7 +380,8 @@ def run_ours(args, world, rank, local):
         dt, fl, threads = oracle_sample(wl, n_rows)
         line["cpu_baseline"] = {
             "value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-            "sample": f"rows 0..{n_rows - 1} of head 0 (one causal band), forward + backward, fp64"}
+            "sample": f"rows and keys 0..{n_rows - 1} of head 0 under the same mask, forward + "
+                      f"backward, fp64"}
     if rank == 0:
         print(json.dumps(line), flush=True)
 
@@ -375,7 +402,7 @@ def e2e_leg(args, wl, dev, flops, world):
                                   ("dk", wl.k.shape, torch.bfloat16),
                                   ("dv", wl.v.shape, torch.bfloat16))}
     st = bsa.Stages(dev_in["q"], dev_in["k"], dev_in["v"], wl.mask, softmax_mode=args.softmax,
-                    order=args.order)
+                    order=args.order, deterministic=not args.nondet)
     stream = torch.cuda.current_stream()
 
     def step():

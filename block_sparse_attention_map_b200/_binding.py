@@ -23,7 +23,7 @@ c_i32, c_u32, c_i64, c_f32, c_vp = ctypes.c_int32, ctypes.c_uint32, ctypes.c_int
 # --- constants mirrored from include/bsa.h
 TILE = 128
 TILE_EMPTY, TILE_PARTIAL, TILE_FULL = 0, 1, 2
-MASK_SEGMENT_IDS, MASK_KV_VALID_LEN, MASK_VARLEN, MASK_CAUSAL_WINDOW = 1, 2, 4, 8
+MASK_SEGMENT_IDS, MASK_KV_VALID_LEN, MASK_VARLEN, MASK_CAUSAL_WINDOW, MASK_PREFIX_LM = 1, 2, 4, 8, 16
 SOFTMAX_ONLINE, SOFTMAX_FIXED_M_GATED = 0, 1
 ORDER = {"asc": 0, "desc": 1, "perm": 2, "outside_in": 3, "greedy": 4}
 FULL_BIT = 1 << 30
@@ -45,7 +45,8 @@ class Problem(ctypes.Structure):
 class MaskSpec(ctypes.Structure):
     _fields_ = [("flags", c_u32), ("window", c_i32), ("seg_q", c_vp), ("seg_kv", c_vp),
                 ("kv_valid_len", c_vp), ("cu_seqlens", c_vp), ("n_seqs", c_i32),
-                ("n_align_tail", c_i32)]
+                ("n_align_tail", c_i32), ("prefix_len", c_vp), ("dilation", c_i32),
+                ("reserved", c_i32)]
 
 
 class Options(ctypes.Structure):
@@ -160,7 +161,9 @@ class Mask:
 
     Keys of ``desc`` (all optional): ``seg_q``, ``seg_kv`` ([B, S] ints),
     ``kv_valid_len`` ([B]), ``cu_seqlens`` ([n_seqs + 1]) with ``n_align_tail``,
-    ``window`` (None: off, 0: causal, W: causal band of W keys)."""
+    ``window`` (None: off, 0: causal, W: causal band of W keys) with
+    ``dilation`` (keep every d-th key back from the diagonal) and ``prefix_len``
+    ([B]: keys below it are seen by every row)."""
 
     def __init__(self, desc: Optional[dict], device):
         desc = desc or {}
@@ -189,6 +192,11 @@ class Mask:
         if desc.get("window") is not None:
             self.spec.flags |= MASK_CAUSAL_WINDOW
             self.spec.window = int(desc["window"])
+        if desc.get("dilation") is not None:
+            self.spec.dilation = int(desc["dilation"])
+        if desc.get("prefix_len") is not None:
+            self.spec.flags |= MASK_PREFIX_LM
+            self.spec.prefix_len = dev(desc["prefix_len"]).data_ptr()
 
 
 def make_options(softmax_mode="online", gate_limit=0.0, kmax_override=None, order="asc",

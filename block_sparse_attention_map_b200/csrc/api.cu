@@ -139,11 +139,19 @@ bsa_status normalise(const bsa_problem *in, bsa_problem *out) {
 
 bsa_status check_mask(const bsa_problem &p, const bsa_mask_spec *m, bsa_mask_spec *out) {
   std::memset(out, 0, sizeof(*out));
+  out->dilation = 1;
   if (m == nullptr) return BSA_OK;
   *out = *m;
   const uint32_t known = BSA_MASK_SEGMENT_IDS | BSA_MASK_KV_VALID_LEN | BSA_MASK_VARLEN |
-                         BSA_MASK_CAUSAL_WINDOW;
+                         BSA_MASK_CAUSAL_WINDOW | BSA_MASK_PREFIX_LM;
   if (m->flags & ~known) return BSA_ERR_INVALID_ARG;
+  const bool win = (m->flags & BSA_MASK_CAUSAL_WINDOW) != 0;
+  if ((m->flags & BSA_MASK_PREFIX_LM) && (!win || m->prefix_len == nullptr))
+    return BSA_ERR_INVALID_ARG;
+  if (m->dilation < 0 || (m->dilation > 1 && !win)) return BSA_ERR_INVALID_ARG;
+  out->dilation = m->dilation > 1 ? m->dilation : 1;
+  out->reserved = 0;
+  if (!(m->flags & BSA_MASK_PREFIX_LM)) out->prefix_len = nullptr;
   if ((m->flags & BSA_MASK_SEGMENT_IDS) && (m->seg_q == nullptr || m->seg_kv == nullptr))
     return BSA_ERR_INVALID_ARG;
   if ((m->flags & BSA_MASK_KV_VALID_LEN) && m->kv_valid_len == nullptr) return BSA_ERR_INVALID_ARG;
@@ -191,6 +199,7 @@ PlanSignature signature(const bsa_problem &p, const bsa_mask_spec &m, const bsa_
   s.w[4] = m.window;
   s.w[5] = o.bwd_order;
   s.w[6] = m.n_seqs;
+  s.w[7] = m.dilation;
   return s;
 }
 
@@ -203,6 +212,11 @@ MaskParams mask_params(const bsa_problem &p, const bsa_mask_spec &m, const WsLay
   mp.Sq = p.Sq;
   mp.Skv = p.Skv;
   mp.kv_valid_len = (m.flags & BSA_MASK_KV_VALID_LEN) ? m.kv_valid_len : nullptr;
+  mp.prefix_len = (m.flags & BSA_MASK_PREFIX_LM) ? m.prefix_len : nullptr;
+  mp.dilation = m.dilation > 1 ? m.dilation : 1;
+  mp.dil_pattern = 0;
+  for (int k = 0; mp.dilation > 1 && k < 32; k += mp.dilation) mp.dil_pattern |= 1u << k;
+  mp.dil_r32 = 32 % mp.dilation;
   if (m.flags & BSA_MASK_SEGMENT_IDS) {
     mp.seg_q = m.seg_q;
     mp.seg_kv = m.seg_kv;

@@ -18,7 +18,10 @@
 // sm_100a roles (384 threads, one CTA per SM, persistent over tickets):
 //   warp 0      ticket + TMA producer (K_n, V_n once per column; Q_m, dO_m per entry)
 //   warp 1      TMEM owner and tcgen05.mma issuer (one lane)
-//   warps 4..7  compute: one key row per thread (TMEM lane), P^T back to TMEM as the
+//   warps 4..7  compute: one key row per thread (TMEM lane), the 128-bit allowed-query
+//               mask of PARTIAL tiles (a prefix key is seen by every query; other
+//               keys by a query range thinned by the dilation, AND segment ids),
+//               P^T back to TMEM as the
 //               A operand of dV, dS^T to shared memory (128-byte swizzle, K-major
 //               for dK, read MN-major as the A operand of dQ), dK/dV epilogue
 //   warps 8..11 dQ: one query row per thread, semaphore wait, vector reductions
@@ -50,7 +53,7 @@ struct BwdParams {
   int deterministic;
   uint32_t *hdr;
   uint64_t timeout_ns, sem_timeout_ns;
-  uint32_t sig[7];
+  uint32_t sig[kSigWords];
   uint32_t sig_mask;
 };
 
@@ -173,7 +176,7 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
   if (threadIdx.x == 0) {
     const volatile uint32_t *h = p.hdr;
     bool ok = h[kHdrMagic] == kPlanMagic;
-    for (int i = 0; i < 7; ++i) ok = ok && (!((p.sig_mask >> i) & 1u) || h[kHdrB + i] == p.sig[i]);
+    for (int i = 0; i < kSigWords; ++i) ok = ok && (!((p.sig_mask >> i) & 1u) || h[kHdrB + i] == p.sig[i]);
     if (!ok) wd.trip(BSA_ERR_PLAN_MISMATCH);
     // the swizzled tiles rely on a 1024-byte aligned dynamic shared window
     if ((smem_u32(sm) & 1023u) != 0u) wd.trip(BSA_ERR_UNSUPPORTED);
@@ -372,10 +375,13 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
         }
         continue;
       }
-      // queries this key may be seen by: [qlo, qhi]
+      // queries this key may be seen by: [qlo, qhi], thinned by the dilation
+      // unless the key lies in the prefix every query sees
       int qlo = 0, qhi = p.Sq - 1;
       if (!row_ok) qhi = -1;
-      if (mk.flags & BSA_MASK_CAUSAL_WINDOW) {
+      const bool in_prefix = mk.prefix_len != nullptr && j < mk.prefix_len[k.b];
+      const bool dilated = mk.dilation > 1 && !in_prefix;
+      if ((mk.flags & BSA_MASK_CAUSAL_WINDOW) && !in_prefix) {
         qlo = max(qlo, j - mk.offset);
         if (mk.window > 0) qhi = min(qhi, j - mk.offset + mk.window - 1);
       }
@@ -406,6 +412,18 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
         if (!full) {
 #pragma unroll
           for (int w = 0; w < 4; ++w) allow[w] = range_bits(qlo - m * kTile, qhi - m * kTile, w);
+          if (dilated) {
+            // keep query i iff (i + o - j) mod d == 0: bit k of word w is query
+            // 128m + 32w + k, kept iff k == (j - o - 128m - 32w) mod d
+            int ph = (j - mk.offset - m * kTile) % mk.dilation;
+            if (ph < 0) ph += mk.dilation;
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+              allow[w] &= ph < 32 ? (mk.dil_pattern << ph) : 0u;
+              ph -= mk.dil_r32;
+              if (ph < 0) ph += mk.dilation;
+            }
+          }
           if (use_seg) {
             const int32_t *sq = mk.seg_q + static_cast<int64_t>(k.b) * p.Sq + m * kTile;
             const int lim = p.Sq - m * kTile;
@@ -789,8 +807,8 @@ cudaError_t launch_bwd_main(const bsa_problem &p, const MaskParams &mp, const bs
   bp.timeout_ns = 2000000000ull;
   bp.sem_timeout_ns =
       o.sem_timeout_ns > 0 ? static_cast<uint64_t>(o.sem_timeout_ns) : 1000000000ull;
-  for (int i = 0; i < 7; ++i) bp.sig[i] = sig.w[i];
-  bp.sig_mask = 0x7Fu;
+  for (int i = 0; i < kSigWords; ++i) bp.sig[i] = sig.w[i];
+  bp.sig_mask = (1u << kSigWords) - 1u;
   cudaError_t e = cudaMemsetAsync(bp.hdr + kHdrBwdTicket, 0, sizeof(uint32_t), s);
   if (e != cudaSuccess) return e;
   return (p.D == 64) ? run_bwd_main<64, 2, 2>(bp, tq, tk, tv, tdo, s)

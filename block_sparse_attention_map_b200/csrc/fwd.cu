@@ -21,7 +21,8 @@
 //               TMEM over the S columns, V an MN-major B operand).
 //   warps 4-7   softmax of q-block A, warps 8-11 of q-block B: one query row
 //               per thread (its TMEM lane).  PARTIAL tiles are masked through a
-//               128-bit allowed-key mask (row range AND segment ids); online
+//               128-bit allowed-key mask (the window's key range thinned by
+//               its dilation, OR the prefix, AND segment ids); online
 //               mode takes the tile max in a first pass over TMEM and rescales
 //               O lazily; the epilogue writes O / l_r (bf16) and LSE.
 // TMEM columns: S_A [0,128) S_B [128,256) O_A [256,256+D) O_B [256+D,256+2D).
@@ -52,7 +53,7 @@ struct FwdParams {
   const int32_t *gate; // [B, H]
   uint32_t *hdr;
   uint64_t timeout_ns;
-  uint32_t sig[7];     // expected plan signature (B, Sq, Skv, flags, window, order, n_seqs)
+  uint32_t sig[kSigWords];  // expected plan signature (B, Sq, Skv, flags, window, order, n_seqs, dilation)
   uint32_t sig_mask;   // which signature words must match
 };
 
@@ -165,7 +166,7 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
   if (threadIdx.x == 0) {
     const volatile uint32_t *h = p.hdr;
     bool ok = h[kHdrMagic] == kPlanMagic;
-    for (int i = 0; i < 7; ++i) ok = ok && (!((p.sig_mask >> i) & 1u) || h[kHdrB + i] == p.sig[i]);
+    for (int i = 0; i < kSigWords; ++i) ok = ok && (!((p.sig_mask >> i) & 1u) || h[kHdrB + i] == p.sig[i]);
     if (!ok) wd.trip(BSA_ERR_PLAN_MISMATCH);
     // the swizzled tiles rely on a 1024-byte aligned dynamic shared window
     if ((smem_u32(sm) & 1023u) != 0u) wd.trip(BSA_ERR_UNSUPPORTED);
@@ -349,13 +350,15 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       float m_ref = -INFINITY, l = 0.f, l_r = 0.f;
       if (fixed)
         m_ref = row_ok ? p.scale_log2 * p.qnorm[static_cast<int64_t>(bh) * p.Sq + i] * p.kmax[bh] : 0.f;
-      // row-constant part of the mask: allowed keys lie in [lo, hi]
-      int lo = 0, hi = p.Skv - 1;
+      // row-constant part of the mask: allowed keys lie in [lo, hi] (the
+      // window, thinned by the dilation) or in the prefix [0, pre_hi]
+      int lo = 0, hi = p.Skv - 1, pre_hi = -1;
+      if (mk.flags & BSA_MASK_KV_VALID_LEN) hi = min(hi, mk.kv_valid_len[b] - 1);
+      if (mk.prefix_len != nullptr) pre_hi = min(hi, mk.prefix_len[b] - 1);
       if (mk.flags & BSA_MASK_CAUSAL_WINDOW) {
         hi = min(hi, i + mk.offset);
         if (mk.window > 0) lo = max(lo, i + mk.offset - mk.window + 1);
       }
-      if (mk.flags & BSA_MASK_KV_VALID_LEN) hi = min(hi, mk.kv_valid_len[b] - 1);
       const int seg_i = (use_seg && row_ok) ? mk.seg_q[static_cast<int64_t>(b) * p.Sq + i] : INT_MIN;
 
       for (int j = rs; j < re; ++j, ++tcount) {
@@ -368,6 +371,22 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
         if (!full) {
 #pragma unroll
           for (int q = 0; q < 4; ++q) allow[q] = range_bits(lo - n * kTile, hi - n * kTile, q);
+          if (mk.dilation > 1) {
+            // keep key j iff (i + o - j) mod d == 0: bit k of word q is key
+            // 128n + 32q + k, kept iff k == (i + o - 128n - 32q) mod d
+            int ph = (i + mk.offset - n * kTile) % mk.dilation;
+            if (ph < 0) ph += mk.dilation;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              allow[q] &= ph < 32 ? (mk.dil_pattern << ph) : 0u;
+              ph -= mk.dil_r32;
+              if (ph < 0) ph += mk.dilation;
+            }
+          }
+          if (pre_hi >= 0) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) allow[q] |= range_bits(-n * kTile, pre_hi - n * kTile, q);
+          }
           if (use_seg) {
             int32_t *segt = seg_sm + (x * 2 + (ps & 1)) * kTile;
             const int jj = n * kTile + r;
@@ -693,8 +712,9 @@ cudaError_t launch_fwd(const bsa_problem &p, const MaskParams &mp, const bsa_opt
   fp.gate = reinterpret_cast<const int32_t *>(ws + L.gate);
   fp.hdr = reinterpret_cast<uint32_t *>(ws + L.status);
   fp.timeout_ns = 2000000000ull;
-  for (int i = 0; i < 7; ++i) fp.sig[i] = sig.w[i];
-  fp.sig_mask = 0x7Fu & ~(1u << 5);  // the forward does not depend on the kv-column order
+  for (int i = 0; i < kSigWords; ++i) fp.sig[i] = sig.w[i];
+  // the forward does not depend on the kv-column order
+  fp.sig_mask = ((1u << kSigWords) - 1u) & ~(1u << kSigOrderWord);
   if (p.D == 64) return run_fwd<64, 4, 4>(fp, tq, tk, tv, s);
   return run_fwd<128, 3, 2>(fp, tq, tk, tv, s);
 }

@@ -33,6 +33,7 @@ enum HeaderWord : int {
   kHdrWindow = 9,
   kHdrOrder = 10,
   kHdrNSeqs = 11,
+  kHdrDilation = 12,
   kHdrWords = 64
 };
 
@@ -55,10 +56,12 @@ struct WsLayout {
 
 WsLayout compute_layout(const bsa_problem &p);
 
-// Plan signature words (B, Sq, Skv, flags, window, order, n_seqs) the planner
-// stores in the header and every kernel that reads the plan checks.
+// Plan signature words (B, Sq, Skv, flags, window, order, n_seqs, dilation)
+// the planner stores in the header and every kernel that reads the plan checks.
+constexpr int kSigWords = 8;
+constexpr int kSigOrderWord = 5;
 struct PlanSignature {
-  uint32_t w[7];
+  uint32_t w[kSigWords];
 };
 
 // Mask predicates as every kernel sees them.  Varlen masks arrive here as
@@ -72,6 +75,10 @@ struct MaskParams {
   const int32_t *seg_q;   // [B, Sq] or null
   const int32_t *seg_kv;  // [B, Skv] or null
   const int32_t *kv_valid_len;  // [B] or null
+  const int32_t *prefix_len;    // [B] or null (only with the window flag)
+  int32_t dilation;             // > 1: dilated window, else 1
+  uint32_t dil_pattern;         // bits 0, d, 2d, ... below 32 (dilation > 1)
+  int32_t dil_r32;              // 32 mod d
 };
 
 // Launchers (each returns cudaGetLastError() of its launches).

@@ -7,7 +7,9 @@
 // ("Modifications") for varlen alignment rows; "Add more optimal dk order
 // optional arg" (flash-attention PR #2512, "Sliding window perf issue" and "A
 // simplish fix") for rank(m, n), the kv-column orders and the unified column
-// list walked in rank order.
+// list walked in rank order; its benchmark ("The numbers") names the
+// outside_in and greedy orders and the prefix_lm, dilated_sliding_window and
+// document masks, whose readings are stated where they are built.
 //
 // The block map is shared by every head (masks are head independent) and kept
 // as compact CSR lists, so its size is O(non-empty tiles) per batch row plus
@@ -72,47 +74,127 @@ __global__ void k_block_summary(const int32_t *__restrict__ seg, int S, int nblk
 struct ClassifyArgs {
   int B, nM, nN, Sq, Skv;
   uint32_t flags;
-  int window;
+  int window, dilation;
   const int32_t *kv_valid_len;
-  const int4 *qblk, *kblk;  // null unless segment ids / varlen
+  const int32_t *prefix_len;       // null unless BSA_MASK_PREFIX_LM
+  const int4 *qblk, *kblk;         // null unless segment ids / varlen
+  const int32_t *seg_q, *seg_kv;   // the ids the kernels compare (null: none)
+  int64_t seg_q_bstride, seg_kv_bstride;
   uint8_t *cls;
   int32_t *row_cnt, *col_cnt;
 };
 
 // Tile class of (b, m, n): the AND-combination of one class per enabled
-// predicate (EMPTY if any predicate is empty, FULL if all are full).  Window,
-// padding and out-of-range columns are classified analytically and exactly;
-// segment ids through per-block [min, max] intervals, exact for
-// non-decreasing ids and conservative (PARTIAL instead of EMPTY) otherwise.
-__device__ __forceinline__ uint8_t tile_class(const ClassifyArgs &a, int b, int m, int n) {
+// predicate (EMPTY if any predicate is empty, FULL if all are full).  The
+// window (with its prefix), padding and out-of-range columns are classified
+// analytically and exactly over the tile's in-range rows and columns; a
+// dilated window and segment ids only through bounds (the undilated band,
+// per-block [min, max] id intervals).  *exact is cleared when the PARTIAL
+// answer may be wrong: a bound-only predicate, or two predicates that are
+// each partial (their allowed parts may not meet).
+__device__ __forceinline__ uint8_t tile_class(const ClassifyArgs &a, int b, int m, int n,
+                                              bool *exact) {
   const int i0 = m * kTile, i1 = min(a.Sq, i0 + kTile) - 1;
   const int j0 = n * kTile, jv1 = min(a.Skv, j0 + kTile) - 1;
   uint8_t c = BSA_TILE_FULL;
+  int npartial = 0;
+  bool bound_only = false;
   if (j0 + kTile - 1 > jv1) c = BSA_TILE_PARTIAL;  // out-of-range keys must be masked
   if (a.flags & BSA_MASK_CAUSAL_WINDOW) {
     const int o = a.Skv - a.Sq, W = a.window;
-    const bool any = (j0 <= i1 + o) && (W == 0 || jv1 >= i0 + o - W + 1);
-    const bool all = (jv1 <= i0 + o) && (W == 0 || j0 >= i1 + o - W + 1);
+    const int P = a.prefix_len != nullptr ? a.prefix_len[b] : 0;
+    // the band i+o-W < j <= i+o over columns [ja, jv1]
+    auto band_any = [&](int ja) {
+      return ja <= jv1 && ja <= i1 + o && (W == 0 || jv1 >= i0 + o - W + 1);
+    };
+    auto band_all = [&](int ja) {
+      return ja > jv1 || (jv1 <= i0 + o && (W == 0 || ja >= i1 + o - W + 1));
+    };
+    const bool pre_all = jv1 < P, pre_any = j0 < P;
+    const int ja = max(j0, P);  // first column the prefix does not cover
+    const bool any = pre_any || band_any(j0);
+    bool all = pre_all || band_all(ja);
     if (!any) return BSA_TILE_EMPTY;
-    if (!all) c = BSA_TILE_PARTIAL;
+    if (a.dilation > 1 && !pre_all) {
+      all = false;
+      // the band is exact without a dilation; with one its kept keys may miss
+      // the tile, unless the prefix alone already makes it non-empty
+      if (!pre_any) bound_only = true;
+    }
+    if (!all) {
+      c = BSA_TILE_PARTIAL;
+      ++npartial;
+    }
   }
   if (a.flags & BSA_MASK_KV_VALID_LEN) {
     const int L = a.kv_valid_len[b];
     if (j0 >= L) return BSA_TILE_EMPTY;
-    if (jv1 >= L) c = BSA_TILE_PARTIAL;
+    if (jv1 >= L) {
+      c = BSA_TILE_PARTIAL;
+      ++npartial;
+    }
   }
   if (a.qblk != nullptr) {
     const int4 q = a.qblk[b * a.nM + m];
     const int4 k = a.kblk[b * a.nN + n];
     if (q.z == 0 || k.z == 0 || q.y < k.x || k.y < q.x) return BSA_TILE_EMPTY;
     const bool one = q.x == q.y && k.x == k.y && q.x == k.x && q.w == 0 && k.w == 0;
-    if (!one) c = BSA_TILE_PARTIAL;
+    if (!one) {
+      c = BSA_TILE_PARTIAL;
+      bound_only = true;
+    }
   }
+  *exact = !bound_only && npartial <= 1;
   return c;
 }
 
-// One warp per (b, m): classify the row of tiles, count its non-empty tiles
-// and add each non-empty tile to its column's count (an order-independent sum).
+// allowed(i, j) for one in-range element, every enabled predicate: the
+// element-level definition the kernels apply on PARTIAL tiles.
+__device__ __forceinline__ bool allowed_elem(const ClassifyArgs &a, int b, int i, int j,
+                                             int seg_i, int seg_j, int P, int L) {
+  if (j >= L) return false;
+  if (a.seg_q != nullptr && seg_i != seg_j) return false;
+  if (a.flags & BSA_MASK_CAUSAL_WINDOW) {
+    if (j < P) return true;
+    const int t = i + (a.Skv - a.Sq) - j;
+    if (t < 0 || (a.window > 0 && t >= a.window)) return false;
+    if (a.dilation > 1 && t % a.dilation != 0) return false;
+  }
+  return true;
+}
+
+// Exact class of tile (b, m, n) by the whole warp, element by element: lane l
+// takes columns l, l+32, l+64, l+96 of the tile and walks its rows.
+__device__ uint8_t refine_tile(const ClassifyArgs &a, int b, int m, int n, int lane) {
+  const int i0 = m * kTile, i1 = min(a.Sq, i0 + kTile) - 1;
+  const int P = a.prefix_len != nullptr ? a.prefix_len[b] : 0;
+  const int L = (a.flags & BSA_MASK_KV_VALID_LEN) ? a.kv_valid_len[b] : a.Skv;
+  bool any = false, all = true;
+#pragma unroll 1
+  for (int t = lane; t < kTile; t += 32) {
+    const int j = n * kTile + t;
+    if (j >= a.Skv) {
+      all = false;
+      continue;
+    }
+    const int seg_j = a.seg_kv != nullptr ? a.seg_kv[b * a.seg_kv_bstride + j] : 0;
+#pragma unroll 1
+    for (int i = i0; i <= i1; ++i) {
+      const int seg_i = a.seg_q != nullptr ? a.seg_q[b * a.seg_q_bstride + i] : 0;
+      const bool ok = allowed_elem(a, b, i, j, seg_i, seg_j, P, min(L, a.Skv));
+      any |= ok;
+      all &= ok;
+    }
+  }
+  any = __any_sync(0xffffffffu, any);
+  all = __all_sync(0xffffffffu, all);
+  return all ? BSA_TILE_FULL : (any ? BSA_TILE_PARTIAL : BSA_TILE_EMPTY);
+}
+
+// One warp per (b, m): classify the row of tiles (tiles the bounds cannot
+// settle are classified element by element by the whole warp), count its
+// non-empty tiles and add each non-empty tile to its column's count (an
+// order-independent sum).
 __global__ void k_classify_rows(ClassifyArgs a) {
   const int wid = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
@@ -123,8 +205,16 @@ __global__ void k_classify_rows(ClassifyArgs a) {
   for (int n0 = 0; n0 < a.nN; n0 += 32) {
     const int n = n0 + lane;
     uint8_t c = BSA_TILE_EMPTY;
+    bool exact = true;
+    if (n < a.nN) c = tile_class(a, b, m, n, &exact);
+    uint32_t todo = __ballot_sync(0xffffffffu, c == BSA_TILE_PARTIAL && !exact);
+    while (todo != 0u) {
+      const int src = __ffs(todo) - 1;
+      todo &= todo - 1u;
+      const uint8_t rc = refine_tile(a, b, m, n0 + src, lane);
+      if (lane == src) c = rc;
+    }
     if (n < a.nN) {
-      c = tile_class(a, b, m, n);
       row[n] = c;
       if (c != BSA_TILE_EMPTY) atomicAdd(a.col_cnt + b * a.nN + n, 1);
     }
@@ -139,7 +229,7 @@ __global__ void k_classify_rows(ClassifyArgs a) {
 __global__ void k_scan2(const int32_t *__restrict__ c0, int32_t *__restrict__ p0, int n0,
                         const int32_t *__restrict__ c1, int32_t *__restrict__ p1, int n1,
                         uint32_t *hdr, uint32_t B, uint32_t Sq, uint32_t Skv, uint32_t flags,
-                        uint32_t window, uint32_t order, uint32_t n_seqs) {
+                        uint32_t window, uint32_t order, uint32_t n_seqs, uint32_t dilation) {
   const int32_t *c = blockIdx.x == 0 ? c0 : c1;
   int32_t *p = blockIdx.x == 0 ? p0 : p1;
   const int n = blockIdx.x == 0 ? n0 : n1;
@@ -185,6 +275,7 @@ __global__ void k_scan2(const int32_t *__restrict__ c0, int32_t *__restrict__ p0
       hdr[kHdrWindow] = window;
       hdr[kHdrOrder] = order;
       hdr[kHdrNSeqs] = n_seqs;
+      hdr[kHdrDilation] = dilation;
       __threadfence();
       hdr[kHdrMagic] = kPlanMagic;
     }
@@ -362,6 +453,8 @@ cudaError_t launch_plan(const bsa_problem &p, const bsa_mask_spec &m, const bsa_
   if (e != cudaSuccess) return e;
 
   const int4 *qblk = nullptr, *kblk = nullptr;
+  const int32_t *seg_q_ids = nullptr, *seg_kv_ids = nullptr;
+  int64_t seg_q_bs = 0, seg_kv_bs = 0;
   const bool varlen = m.flags & BSA_MASK_VARLEN;
   if (varlen || (m.flags & BSA_MASK_SEGMENT_IDS)) {
     const int32_t *sq = m.seg_q, *sk = m.seg_kv;
@@ -385,6 +478,10 @@ cudaError_t launch_plan(const bsa_problem &p, const bsa_mask_spec &m, const bsa_
     count_launch(2);
     qblk = qb;
     kblk = kb;
+    seg_q_ids = sq;
+    seg_kv_ids = sk;
+    seg_q_bs = bq;
+    seg_kv_bs = bk;
   }
 
   int32_t *rank = reinterpret_cast<int32_t *>(ws + L.rank);
@@ -403,15 +500,22 @@ cudaError_t launch_plan(const bsa_problem &p, const bsa_mask_spec &m, const bsa_
   ca.B = B; ca.nM = nM; ca.nN = nN; ca.Sq = p.Sq; ca.Skv = p.Skv;
   ca.flags = m.flags;
   ca.window = m.window;
+  ca.dilation = m.dilation;
   ca.kv_valid_len = m.kv_valid_len;
+  ca.prefix_len = (m.flags & BSA_MASK_PREFIX_LM) ? m.prefix_len : nullptr;
   ca.qblk = qblk;
   ca.kblk = kblk;
+  ca.seg_q = seg_q_ids;
+  ca.seg_kv = seg_kv_ids;
+  ca.seg_q_bstride = seg_q_bs;
+  ca.seg_kv_bstride = seg_kv_bs;
   ca.cls = ws + L.tile_class;
   ca.row_cnt = row_cnt;
   ca.col_cnt = col_cnt;
   k_classify_rows<<<cdiv(static_cast<int64_t>(B) * nM * 32, 256), 256, 0, s>>>(ca);
   k_scan2<<<2, 1024, 0, s>>>(row_cnt, row_ptr, B * nM, col_cnt, col_ptr, B * nN, hdr, B, p.Sq,
-                             p.Skv, m.flags, m.window, o.bwd_order, m.n_seqs);
+                             p.Skv, m.flags, m.window, o.bwd_order, m.n_seqs,
+                             static_cast<uint32_t>(m.dilation));
   if (o.bwd_order == BSA_ORDER_GREEDY) {
     const size_t gsm = sizeof(int32_t) * static_cast<size_t>(nN);
     if (gsm > 48 * 1024) {

@@ -18,6 +18,16 @@ Workloads (names used by the tests and ``bench.py``):
                3-axis rotary embedding, v ~ N(0, 1); head 0 has 8 "sink" keys
                scaled x20.
 
+The three mask families the dk-order benchmark names besides sliding windows,
+at its 8192x8192 shape and the sliding-window workload's B, H, D and seed
+(the benchmark table states neither their head counts nor their parameters):
+
+``prefix_lm``  causal with a bidirectional prefix of 2048 keys.
+``dilated``    causal band spanning 1024 keys, every second key kept (512 per
+               row, as many as the 512-key sliding window).
+``document``   document-causal: segment ids from runs of uniform{256..2048}
+               tokens, causal inside each document.
+
 ``small=True`` shrinks the sequence lengths (same structure, same recipe) so the
 fp64 oracle finishes in seconds; the parity tests use it for the full-oracle
 comparison and sample rows at full size.
@@ -49,6 +59,17 @@ class Workload:
     scale: float = 0.0
     backward: bool = True
 
+    def mask_text(self) -> str:
+        """The mask parameters in words (arrays by their length)."""
+        parts = []
+        for key, val in self.mask.items():
+            if isinstance(val, (torch.Tensor, np.ndarray)):
+                arr = val.cpu().numpy() if isinstance(val, torch.Tensor) else val
+                parts.append(f"{key}={arr.tolist()}" if arr.size <= 4 else f"{key}[{arr.shape}]")
+            else:
+                parts.append(f"{key}={val}")
+        return ", ".join(parts) or "none"
+
     def mask_numpy(self) -> dict:
         """The mask description with every array on the host (numpy)."""
         out = {}
@@ -57,7 +78,8 @@ class Workload:
         return out
 
 
-WORKLOADS = ("tiny", "packed", "packed_const", "window", "window_rect", "varlen", "video")
+WORKLOADS = ("tiny", "packed", "packed_const", "window", "window_rect", "varlen", "video",
+             "prefix_lm", "dilated", "document")
 
 
 def _normal(shape, gen, device, std=1.0):
@@ -152,6 +174,25 @@ def make_workload(name: str, device="cpu", small: bool = False, seed: Optional[i
         v = _normal((B, Skv, H, D), g, dev).to(bf16)
         dO = _normal((B, Sq, H, D), g, dev).to(bf16)
         return Workload(name, B, H, Sq, Skv, D, q, k, v, dO, {"window": W}, 1.0 / math.sqrt(D))
+
+    if name in ("prefix_lm", "dilated", "document"):
+        sd = 2 if seed is None else seed
+        B, H, D, S = 1, 16, 128, 8192
+        prefix, span, dil, lo, hi = 2048, 1024, 2, 256, 2048
+        if small:
+            H, S = 2, 1000
+            prefix, span, dil, lo, hi = 300, 384, 3, 64, 400
+        g = gen_for(sd)
+        q, k, v, dO = (_normal((B, S, H, D), g, dev).to(bf16) for _ in range(4))
+        if name == "prefix_lm":
+            mask = {"window": 0, "prefix_len": np.full(B, prefix, dtype=np.int32)}
+        elif name == "dilated":
+            mask = {"window": span, "dilation": dil}
+        else:
+            rng = np.random.default_rng(sd)
+            seg = torch.from_numpy(np.stack([_segment_runs(rng, S, lo, hi) for _ in range(B)])).to(dev)
+            mask = {"seg_q": seg, "seg_kv": seg.clone(), "window": 0}
+        return Workload(name, B, H, S, S, D, q, k, v, dO, mask, 1.0 / math.sqrt(D))
 
     if name == "varlen":
         sd = 3 if seed is None else seed

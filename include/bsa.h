@@ -89,7 +89,10 @@ typedef enum bsa_status {
 #define BSA_MASK_SEGMENT_IDS 1u   /* seg_q[b,i] == seg_kv[b,j]                         */
 #define BSA_MASK_KV_VALID_LEN 2u  /* j < kv_valid_len[b]                                */
 #define BSA_MASK_VARLEN 4u        /* same cu_seqlens segment, neither in the alignment tail */
-#define BSA_MASK_CAUSAL_WINDOW 8u /* i+o-W < j <= i+o, o = Skv-Sq (W = 0: j <= i+o)      */
+#define BSA_MASK_CAUSAL_WINDOW 8u /* i+o-W < j <= i+o, o = Skv-Sq (W = 0: j <= i+o);
+                                     with dilation d > 1 also (i+o-j) mod d == 0      */
+#define BSA_MASK_PREFIX_LM 16u    /* with BSA_MASK_CAUSAL_WINDOW: keys j < prefix_len[b]
+                                     are seen by every row as well (OR with the window) */
 
 /* bsa_options.softmax_mode */
 #define BSA_SOFTMAX_ONLINE 0
@@ -138,6 +141,11 @@ typedef struct bsa_mask_spec {
   const int32_t *cu_seqlens;   /* device [n_seqs + 1], cu[0] = 0, cu[n_seqs] = Sq    */
   int32_t n_seqs;              /* segments in cu_seqlens (BSA_MASK_VARLEN)           */
   int32_t n_align_tail;        /* trailing segments that are alignment rows         */
+  const int32_t *prefix_len;   /* device [B]      (BSA_MASK_PREFIX_LM)              */
+  int32_t dilation;            /* BSA_MASK_CAUSAL_WINDOW: keep only the keys whose
+                                  distance back from the diagonal is a multiple of
+                                  it; 0 or 1 = every key.  > 1 needs the window flag */
+  int32_t reserved;
 } bsa_mask_spec;
 
 typedef struct bsa_options {

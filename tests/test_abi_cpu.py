@@ -46,6 +46,7 @@ int main(void) {
          sizeof(bsa_problem), sizeof(bsa_mask_spec), sizeof(bsa_options), sizeof(bsa_workspace_view));
   P(bsa_problem, q_stride) P(bsa_problem, o_stride) P(bsa_problem, scale)
   P(bsa_mask_spec, seg_q) P(bsa_mask_spec, cu_seqlens) P(bsa_mask_spec, n_align_tail)
+  P(bsa_mask_spec, prefix_len) P(bsa_mask_spec, dilation)
   P(bsa_options, kmax_override) P(bsa_options, perm) P(bsa_options, sem_timeout_ns) P(bsa_options, plan_ready)
   P(bsa_workspace_view, off_sem) P(bsa_workspace_view, nN)
   return 0;
@@ -72,6 +73,8 @@ def test_ctypes_structs_match_c_layout():
     assert c["bsa_mask_spec.seg_q"] == bd.MaskSpec.seg_q.offset
     assert c["bsa_mask_spec.cu_seqlens"] == bd.MaskSpec.cu_seqlens.offset
     assert c["bsa_mask_spec.n_align_tail"] == bd.MaskSpec.n_align_tail.offset
+    assert c["bsa_mask_spec.prefix_len"] == bd.MaskSpec.prefix_len.offset
+    assert c["bsa_mask_spec.dilation"] == bd.MaskSpec.dilation.offset
     assert c["bsa_options.kmax_override"] == bd.Options.kmax_override.offset
     assert c["bsa_options.perm"] == bd.Options.perm.offset
     assert c["bsa_options.sem_timeout_ns"] == bd.Options.sem_timeout_ns.offset
@@ -114,6 +117,20 @@ def test_workspace_size_and_validation(L):
     assert _size(L, _prob(B=2), m)[0] == 1          # varlen needs B == 1
     assert _size(L, _prob(Sq=100, Skv=120), m)[0] == 1  # and Sq == Skv
     m.flags = 1 << 7                                # unknown flag
+    assert _size(L, _prob(), m)[0] == 1
+    m = bd.MaskSpec()
+    m.flags = bd.MASK_PREFIX_LM | bd.MASK_CAUSAL_WINDOW  # prefix lengths missing
+    assert _size(L, _prob(), m)[0] == 1
+    m.prefix_len = 16
+    assert _size(L, _prob(), m)[0] == 0
+    m.flags = bd.MASK_PREFIX_LM                     # a prefix needs the window
+    assert _size(L, _prob(), m)[0] == 1
+    m = bd.MaskSpec()
+    m.dilation = 2                                  # a dilation needs the window
+    assert _size(L, _prob(), m)[0] == 1
+    m.flags = bd.MASK_CAUSAL_WINDOW
+    assert _size(L, _prob(), m)[0] == 0
+    m.dilation = -1
     assert _size(L, _prob(), m)[0] == 1
 
 

@@ -36,7 +36,7 @@ def _err(x, ref):
     return min(raw, O_TOL)
 
 
-SMALL = ["tiny", "packed", "window", "window_rect", "varlen", "video"]
+SMALL = ["tiny", "packed", "window", "window_rect", "varlen", "video", "prefix_lm", "dilated", "document"]
 
 
 @pytest.mark.parametrize("name", SMALL)
@@ -114,7 +114,7 @@ def test_bwd_ragged_and_d64():
         assert max(_err(dq, gq), _err(dk, gk), _err(dv, gv)) <= O_TOL, (Sq, Skv, D, W)
 
 
-@pytest.mark.parametrize("name", ["window", "window_rect"])
+@pytest.mark.parametrize("name", ["window", "window_rect", "prefix_lm", "dilated", "document"])
 def test_bwd_full_size_one_head_and_ten_run_identity(name):
     wl = make_workload(name, device="cuda")
     o, lse, ws = bsa.attn_fwd(wl.q, wl.k, wl.v, wl.mask)

@@ -11,7 +11,8 @@ from tests.gpu_common import LSE_TOL, O_TOL, compare_lse, compare_out, mask_desc
 
 pytestmark = pytest.mark.gpu
 
-SMALL = ["tiny", "packed", "packed_const", "window", "window_rect", "varlen", "video"]
+SMALL = ["tiny", "packed", "packed_const", "window", "window_rect", "varlen", "video", "prefix_lm",
+         "dilated", "document"]
 
 
 @pytest.mark.parametrize("name", SMALL)
@@ -24,7 +25,9 @@ def test_plan_tile_classes_match_oracle(name):
     assert ws.status() == 0
 
 
-@pytest.mark.parametrize("name,B,Sq,Skv", [("window", 1, 8192, 8192), ("window_rect", 1, 4096, 8192)])
+@pytest.mark.parametrize("name,B,Sq,Skv", [("window", 1, 8192, 8192), ("window_rect", 1, 4096, 8192),
+                                            ("prefix_lm", 1, 8192, 8192), ("dilated", 1, 8192, 8192),
+                                            ("document", 1, 8192, 8192)])
 def test_plan_full_size_window_counts(name, B, Sq, Skv):
     wl = make_workload(name, device="cuda")
     ws = bsa.plan_build(wl.q, wl.k, wl.v, wl.mask)
@@ -34,7 +37,8 @@ def test_plan_full_size_window_counts(name, B, Sq, Skv):
 
 
 @pytest.mark.parametrize("order", ["asc", "desc", "perm", "outside_in", "greedy"])
-@pytest.mark.parametrize("name", ["window", "packed", "window_rect", "varlen"])
+@pytest.mark.parametrize("name", ["window", "packed", "window_rect", "varlen", "prefix_lm", "dilated",
+                                  "document"])
 def test_plan_ranks_and_column_lists(name, order):
     wl = make_workload(name, device="cuda", small=True)
     nN = -(-wl.Skv // 128)
@@ -195,7 +199,8 @@ def test_strided_inputs():
 
 
 @pytest.mark.parametrize("name,extra", [("window", ()), ("window_rect", ()), ("varlen", (33002,)),
-                                        ("packed", ())])
+                                        ("packed", ()), ("prefix_lm", (2047, 2048)), ("dilated", ()),
+                                        ("document", ())])
 def test_fwd_full_size_sampled_rows(name, extra):
     wl = make_workload(name, device="cuda")
     rows = sample_rows(wl.Sq, seed=1, extra=extra)
