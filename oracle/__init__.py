@@ -7,7 +7,7 @@ legs of ``bench.py`` may call it.  It shares no code with the CUDA path.
 Contents
 --------
 ``attention``  dense masked softmax attention, its analytic gradient, the fixed-m
-               form and the fixed-m bound / per-head gate.
+               form and the fixed-m bound / per-head gate (plain and k-smoothed).
 ``blockmap``   the tile classification (EMPTY / PARTIAL / FULL) of a dense mask,
                the kv-column orders, ``rank(m, n)``, the rank-sorted column lists
                and a discrete simulation of the dQ semaphore protocol.
@@ -24,6 +24,7 @@ from .attention import (  # noqa: F401
     attention_backward,
     attention_forward_fixed_m,
     fixed_m_bound,
+    fixed_m_bound_smoothed,
     useful_flops,
 )
 from .blockmap import (  # noqa: F401

@@ -223,7 +223,8 @@ def attention_backward(q, k, v, dO, mask: MaskDesc, scale: float, chunk: int = 1
 
 
 def attention_forward_fixed_m(q, k, v, mask: MaskDesc, scale: float, kmax=None,
-                              rows=None, heads=None, batches=None, chunk: int = 1024):
+                              rows=None, heads=None, batches=None, chunk: int = 1024,
+                              kbar=None):
     """The fixed-m form ("Fixed-m softmax ...", introduction).
 
     Instead of the row max, each query's reference is pinned before streaming to
@@ -233,6 +234,11 @@ def attention_forward_fixed_m(q, k, v, mask: MaskDesc, scale: float, kmax=None,
       O_i = sum_j exp(s_ij - m_i) v_j / l_i.
     In exact arithmetic this equals :func:`attention_forward`; ``kmax`` may be a
     caller-supplied bound [B, H] (any upper bound keeps the result exact).
+
+    With a key center ``kbar`` [B, H, D] (k-smoothing, see
+    :func:`fixed_m_bound_smoothed`) ``kmax`` is the radius max_j ||k_j - kbar||
+    and the pinned reference is m_i = scale * (q_i . kbar + ||q_i|| * kmax),
+    again an upper bound of every s_ij by Cauchy-Schwarz on k_j - kbar.
     """
     q, k, v = _as64(q), _as64(k), _as64(v)
     B, Sq, H, D = q.shape
@@ -252,6 +258,8 @@ def attention_forward_fixed_m(q, k, v, mask: MaskDesc, scale: float, kmax=None,
             for h in heads:
                 qr = q[b, r, h, :]
                 m = scale * np.sqrt((qr * qr).sum(axis=1)) * kmax[b, h]
+                if kbar is not None:
+                    m = m + scale * (qr @ _as64(kbar)[b, h])
                 s = scale * (qr @ k[b, :, h, :].T)
                 e = np.where(a, np.exp(s - m[:, None]), 0.0)
                 l = e.sum(axis=1)
@@ -289,6 +297,44 @@ def fixed_m_bound(q, k, mask: MaskDesc, scale: float, gate_limit: float = 64.0):
     bound = scale * qmax * kmax
     gate = 2.0 * bound <= gate_limit
     return kmax, qmax, bound, gate
+
+
+def fixed_m_bound_smoothed(q, k, mask: MaskDesc, scale: float, gate_limit: float = 64.0):
+    """The k-smoothed bound ("Fixed-m softmax ...", "Notes": k-smoothing, impossible
+    on a ring because no rank holds the full K, is possible when one device holds
+    all of K).
+
+    Softmax is invariant to a per-row shift, and s_ij = scale * q_i . kbar +
+    scale * q_i . (k_j - kbar) for any vector kbar.  Reading taken: kbar is the
+    mean of the valid keys of the head, R its radius, and
+
+      kbar[b, h]   = mean over valid keys j of k_j
+      radius[b, h] = max over valid keys j of ||k_j - kbar||
+      m_i          = scale * (q_i . kbar + ||q_i|| * radius)     (>= every s_ij)
+      bound[b, h]  = scale * qmax * radius
+      gate[b, h]   = 2 * bound <= gate_limit
+
+    since every s_ij - scale * q_i . kbar lies in [-scale ||q_i|| radius,
+    scale ||q_i|| radius], the pinned m_i sits at most 2 * bound above the row
+    max.  Returns (kbar [B, H, D], radius, qmax, bound, gate).
+    """
+    q, k = _as64(q), _as64(k)
+    B, Sq, H, D = q.shape
+    Skv = k.shape[1]
+    kbar = np.zeros((B, H, D))
+    radius = np.zeros((B, H))
+    qmax = np.zeros((B, H))
+    for b in range(B):
+        vk = valid_keys(mask, b, Skv)
+        for h in range(H):
+            if vk.any():
+                kv = k[b, vk, h, :]
+                kbar[b, h] = kv.mean(axis=0)
+                radius[b, h] = np.sqrt(((kv - kbar[b, h]) ** 2).sum(axis=1)).max()
+            qmax[b, h] = np.sqrt((q[b, :, h, :] ** 2).sum(axis=1)).max()
+    bound = scale * qmax * radius
+    gate = 2.0 * bound <= gate_limit
+    return kbar, radius, qmax, bound, gate
 
 
 def useful_flops(n_tiles: int, D: int, tile: int = 128, backward: bool = False) -> float:

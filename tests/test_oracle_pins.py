@@ -256,6 +256,61 @@ def test_fixed_m_bound_dominates_every_score_and_gate_separates_sink():
     assert not gate[0, 0] and gate[0, 1]
 
 
+def test_smoothed_bound_closed_form_two_keys():
+    # keys u + e and u - e: center u, radius ||e||; with q along e the first
+    # key's score reaches the bound exactly
+    u = np.array([3.0, -1.0, 2.0, 0.5])
+    e = np.array([0.0, 2.0, 0.0, 0.0])
+    k = np.stack([u + e, u - e])[None, :, None, :]
+    q = np.array([[0.0, 1.5, 0.0, 0.0]])[None, :, None, :]
+    kbar, radius, qmax, bound, gate = oracle.fixed_m_bound_smoothed(q, k, MaskDesc(), 0.5)
+    assert np.allclose(kbar[0, 0], u, atol=1e-15) and abs(radius[0, 0] - 2.0) < 1e-15
+    assert abs(bound[0, 0] - 0.5 * 1.5 * 2.0) < 1e-15
+    s = 0.5 * (k[0, :, 0] @ q[0, 0, 0])
+    assert abs(s.max() - 0.5 * (q[0, 0, 0] @ u + 1.5 * 2.0)) < 1e-14
+
+
+def test_smoothed_bound_is_translation_invariant_and_dominates():
+    rng = np.random.default_rng(21)
+    D, S = 16, 50
+    q = rng.standard_normal((1, S, 2, D))
+    k = rng.standard_normal((1, S + 6, 2, D))
+    k[0, S:] *= 100  # padding keys never enter the center or the radius
+    m = MaskDesc(kv_valid_len=np.array([S]))
+    scale = 0.3
+    kbar, radius, qmax, bound, gate = oracle.fixed_m_bound_smoothed(q, k, m, scale)
+    shift = rng.standard_normal(D) * 7
+    k2 = k + shift
+    kbar2, radius2, _, _, _ = oracle.fixed_m_bound_smoothed(q, k2, m, scale)
+    assert np.allclose(kbar2, kbar + shift, atol=1e-12)
+    assert np.allclose(radius2, radius, atol=1e-12)
+    kmax2 = oracle.fixed_m_bound(q, k2, m, scale)[0]
+    assert (kmax2 > radius2 + 5).all()  # the plain bound grows with the offset
+    for h in range(2):
+        s = scale * q[0, :, h] @ k2[0, :S, h].T
+        mi = scale * (q[0, :, h] @ kbar2[0, h] + np.linalg.norm(q[0, :, h], axis=1) * radius2[0, h])
+        assert (s.max(axis=1) <= mi + 1e-12).all()
+        assert (mi - s.max(axis=1) <= 2 * scale * np.linalg.norm(q[0, :, h], axis=1) * radius2[0, h] + 1e-12).all()
+
+
+def test_smoothing_widens_gate_and_stays_exact():
+    # a common key offset of norm 12: the plain gate fails, the smoothed one holds
+    rng = np.random.default_rng(22)
+    D, S = 16, 40
+    q = rng.standard_normal((1, S, 1, D)) * math.sqrt(0.5)
+    k = rng.standard_normal((1, S, 1, D)) * math.sqrt(0.5)
+    k[0, :, 0, 0] += 12.0
+    v = rng.standard_normal((1, S, 1, D))
+    scale = 1 / math.sqrt(D)
+    plain = oracle.fixed_m_bound(q, k, MaskDesc(window=0), scale, gate_limit=16.0)
+    smooth = oracle.fixed_m_bound_smoothed(q, k, MaskDesc(window=0), scale, gate_limit=16.0)
+    assert not plain[3][0, 0] and smooth[4][0, 0]
+    O, L = oracle.attention_forward(q, k, v, MaskDesc(window=0), scale)
+    Os, Ls = oracle.attention_forward_fixed_m(q, k, v, MaskDesc(window=0), scale, kmax=smooth[1],
+                                              kbar=smooth[0])
+    assert np.max(np.abs(O - Os)) < 1e-12 and np.max(np.abs(L - Ls)) < 1e-12
+
+
 def test_gradient_identities():
     q, k, v, dO = P.tiny_inputs(16, B=1, Sq=9, Skv=9, D=4)
     v, dO = v[..., :4].copy(), dO[..., :4].copy()
