@@ -54,7 +54,10 @@ WORKLOADS = {
 
 def workload_text(args):
     bwd = "atomic (non-deterministic)" if args.nondet else f"deterministic ({args.order} kv-column order)"
-    return f"{WORKLOADS[args.workload]}; forward {args.softmax} + {bwd} backward"
+    fwd = args.softmax + (" gated" if args.softmax == "fixed_m" else "")
+    if args.softmax == "fixed_m" and args.bound == "smoothed":
+        fwd += ", k-smoothed bound"
+    return f"{WORKLOADS[args.workload]}; forward {fwd} + {bwd} backward"
 METRIC = "attention TFLOP/s (non-empty tiles) fwd+bwd on 1 B200; % of bf16 tensor peak"
 
 
@@ -65,6 +68,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--softmax", default="fixed_m", choices=["fixed_m", "online"])
+    ap.add_argument("--bound", default="norm", choices=["norm", "smoothed"],
+                    help="fixed-m reference: Cauchy-Schwarz on ||k|| or on the centred keys")
     ap.add_argument("--order", default="asc", choices=["asc", "desc", "outside_in", "greedy"])
     ap.add_argument("--nondet", action="store_true", help="atomic (non-deterministic) dQ backward")
     ap.add_argument("--workload", default=WORKLOAD_NAME, choices=sorted(WORKLOADS))
@@ -272,7 +277,7 @@ def run_ours(args, world, rank, local):
     dev = torch.device("cuda", local)
     wl = make_workload(args.workload, device=dev, small=args.small)
     st = bsa.Stages(wl.q, wl.k, wl.v, wl.mask, softmax_mode=args.softmax, order=args.order,
-                    deterministic=not args.nondet)
+                    deterministic=not args.nondet, bound_mode=args.bound)
     dO = wl.dO
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
@@ -352,7 +357,7 @@ def run_ours(args, world, rank, local):
         "config": {"workload": workload_text(args) + (" [small shape]" if args.small else ""),
                    "global_batch": wl.B * world, "seq_len": wl.Sq, "heads": wl.H,
                    "head_dim": wl.D, "mask": wl.mask_text(), "nonempty_tiles": n_tiles,
-                   "softmax": args.softmax,
+                   "softmax": args.softmax, "bound": args.bound,
                    "bwd_order": "nondeterministic" if args.nondet else args.order,
                    "l2": "flushed (256 MiB write) before every step, outside the timed events",
                    "parallelism": f"replicas x{world}"},
@@ -402,7 +407,7 @@ def e2e_leg(args, wl, dev, flops, world):
                                   ("dk", wl.k.shape, torch.bfloat16),
                                   ("dv", wl.v.shape, torch.bfloat16))}
     st = bsa.Stages(dev_in["q"], dev_in["k"], dev_in["v"], wl.mask, softmax_mode=args.softmax,
-                    order=args.order, deterministic=not args.nondet)
+                    order=args.order, deterministic=not args.nondet, bound_mode=args.bound)
     stream = torch.cuda.current_stream()
 
     def step():

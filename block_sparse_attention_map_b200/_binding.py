@@ -25,6 +25,7 @@ TILE = 128
 TILE_EMPTY, TILE_PARTIAL, TILE_FULL = 0, 1, 2
 MASK_SEGMENT_IDS, MASK_KV_VALID_LEN, MASK_VARLEN, MASK_CAUSAL_WINDOW, MASK_PREFIX_LM = 1, 2, 4, 8, 16
 SOFTMAX_ONLINE, SOFTMAX_FIXED_M_GATED = 0, 1
+BOUND = {"norm": 0, "smoothed": 1}
 ORDER = {"asc": 0, "desc": 1, "perm": 2, "outside_in": 3, "greedy": 4}
 FULL_BIT = 1 << 30
 STATUS = {
@@ -52,14 +53,16 @@ class MaskSpec(ctypes.Structure):
 class Options(ctypes.Structure):
     _fields_ = [("softmax_mode", c_i32), ("gate_limit", c_f32), ("kmax_override", c_vp),
                 ("bwd_order", c_i32), ("deterministic", c_i32), ("perm", c_vp),
-                ("sem_timeout_ns", c_i64), ("plan_ready", c_i32), ("bound_ready", c_i32)]
+                ("sem_timeout_ns", c_i64), ("plan_ready", c_i32), ("bound_ready", c_i32),
+                ("bound_mode", c_i32), ("reserved", c_i32)]
 
 
 class WorkspaceView(ctypes.Structure):
     _fields_ = [(n, ctypes.c_size_t) for n in (
         "total_bytes", "fwd_bytes", "off_status", "off_tile_class", "off_rank", "off_row_ptr",
         "off_row_ent", "off_col_ptr", "off_col_ent", "off_col_rank", "off_perm", "off_kmax",
-        "off_qmax", "off_gate", "off_delta", "off_dq_accum", "off_sem")] + [("nM", c_i32), ("nN", c_i32)]
+        "off_qmax", "off_gate", "off_delta", "off_dq_accum", "off_sem", "off_kbar", "off_qdot")] + \
+        [("nM", c_i32), ("nN", c_i32)]
 
 
 class BsaError(RuntimeError):
@@ -201,7 +204,7 @@ class Mask:
 
 def make_options(softmax_mode="online", gate_limit=0.0, kmax_override=None, order="asc",
                  perm=None, deterministic=True, sem_timeout_ns=0, plan_ready=False,
-                 bound_ready=False):
+                 bound_ready=False, bound_mode="norm"):
     o = Options()
     o.softmax_mode = SOFTMAX_FIXED_M_GATED if softmax_mode in ("fixed_m", SOFTMAX_FIXED_M_GATED) else SOFTMAX_ONLINE
     o.gate_limit = float(gate_limit)
@@ -211,6 +214,7 @@ def make_options(softmax_mode="online", gate_limit=0.0, kmax_override=None, orde
     o.sem_timeout_ns = int(sem_timeout_ns)
     o.plan_ready = 1 if plan_ready else 0
     o.bound_ready = 1 if bound_ready else 0
+    o.bound_mode = BOUND[bound_mode] if isinstance(bound_mode, str) else int(bound_mode)
     o._perm_buf = None
     if perm is not None:
         buf = (c_i32 * len(perm))(*[int(x) for x in perm])
@@ -229,7 +233,7 @@ class Workspace:
         self.view = view
         self.nbytes = view.total_bytes if backward else view.fwd_bytes
         self.buf = torch.empty(self.nbytes, dtype=torch.uint8, device=device)
-        self.B, self.H, self.nM, self.nN = prob.B, prob.H, view.nM, view.nN
+        self.B, self.H, self.D, self.nM, self.nN = prob.B, prob.H, prob.D, view.nM, view.nN
 
     def ptr(self):
         return self.buf.data_ptr()
@@ -271,6 +275,11 @@ class Workspace:
     def gate(self):
         return self._arr(self.view.off_gate, self.B * self.H, torch.int32).view(self.B, self.H)
 
+    def kbar(self):
+        """The k-smoothing centers [B, H, D] (after a smoothed bound)."""
+        return self._arr(self.view.off_kbar, self.B * self.H * self.D, torch.float32).view(
+            self.B, self.H, self.D)
+
     def status(self, clear=False):
         s = torch.cuda.current_stream().cuda_stream
         return int(lib().bsa_get_device_status(self.ptr(), self.nbytes, s, 1 if clear else 0))
@@ -302,14 +311,15 @@ def plan_build(q, k, v, mask=None, workspace: Optional[Workspace] = None, backwa
 
 def attn_fwd(q, k, v, mask=None, softmax_mode="online", gate_limit=0.0, kmax_override=None,
              workspace: Optional[Workspace] = None, out=None, lse=None, plan_ready=False,
-             scale=None, order="asc", perm=None):
+             scale=None, order="asc", perm=None, bound_mode="norm"):
     """O = softmax(scale Q K^T + mask) V and LSE [B, H, Sq] through bsa_attn_fwd."""
     B, Sq, H, D = q.shape
     out = torch.empty_like(q) if out is None else out
     lse = torch.empty(B, H, Sq, dtype=torch.float32, device=q.device) if lse is None else lse
     prob = make_problem(q, k, v, out, scale)
     m = Mask(mask, q.device)
-    o = make_options(softmax_mode, gate_limit, kmax_override, order, perm, True, 0, plan_ready)
+    o = make_options(softmax_mode, gate_limit, kmax_override, order, perm, True, 0, plan_ready,
+                     bound_mode=bound_mode)
     ws = workspace or Workspace(prob, m, False, q.device)
     _check(lib().bsa_attn_fwd(ctypes.byref(prob), ctypes.byref(m.spec), ctypes.byref(o), q.data_ptr(),
                               k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), ws.ptr(),
@@ -343,7 +353,7 @@ class Stages:
     workspace, for callers that time or schedule stages separately."""
 
     def __init__(self, q, k, v, mask=None, softmax_mode="online", order="asc", perm=None,
-                 deterministic=True, gate_limit=0.0):
+                 deterministic=True, gate_limit=0.0, bound_mode="norm"):
         self.q, self.k, self.v = q, k, v
         B, Sq, H, D = q.shape
         self.out = torch.empty_like(q)
@@ -353,7 +363,7 @@ class Stages:
         self.mask = Mask(mask, q.device)
         self.fixed = softmax_mode in ("fixed_m", SOFTMAX_FIXED_M_GATED)
         self.opt = make_options(softmax_mode, gate_limit, None, order, perm, deterministic, 0,
-                                plan_ready=True, bound_ready=True)
+                                plan_ready=True, bound_ready=True, bound_mode=bound_mode)
         self.ws = Workspace(self.prob, self.mask, True, q.device)
         self._args = (ctypes.byref(self.prob), ctypes.byref(self.mask.spec), ctypes.byref(self.opt))
 

@@ -53,6 +53,10 @@ WsLayout compute_layout(const bsa_problem &p) {
   L.qmax = L.kmax + 4 * static_cast<size_t>(B * H);
   L.gate = take(4 * static_cast<size_t>(B * H));
   L.qnorm = take(4 * static_cast<size_t>(B * H * p.Sq));
+  L.kbar = take(4 * static_cast<size_t>(B * H * p.D));
+  L.ksum = take(8 * static_cast<size_t>(B * H * p.D));
+  L.kcount = take(4 * static_cast<size_t>(B));
+  L.qdot = take(4 * static_cast<size_t>(B * H * p.Sq));
   L.fwd_end = off;
   L.delta = take(4 * static_cast<size_t>(B * H * nM * kTile));
   L.dq_accum = take(4 * static_cast<size_t>(B * H * nM * kTile * p.D));
@@ -178,6 +182,8 @@ bsa_status check_options(const bsa_options *o, int nN, bsa_options *out) {
   if (o->softmax_mode != BSA_SOFTMAX_ONLINE && o->softmax_mode != BSA_SOFTMAX_FIXED_M_GATED)
     return BSA_ERR_INVALID_ARG;
   if (o->bwd_order < BSA_ORDER_ASC || o->bwd_order > BSA_ORDER_GREEDY) return BSA_ERR_INVALID_ARG;
+  if (o->bound_mode != BSA_BOUND_NORM && o->bound_mode != BSA_BOUND_SMOOTHED) return BSA_ERR_INVALID_ARG;
+  if (o->bound_mode == BSA_BOUND_SMOOTHED && o->kmax_override != nullptr) return BSA_ERR_INVALID_ARG;
   if (o->bwd_order == BSA_ORDER_PERM) {
     if (o->perm == nullptr) return BSA_ERR_INVALID_ARG;
     std::vector<char> seen(static_cast<size_t>(nN), 0);
@@ -250,6 +256,8 @@ bsa_status prepare(const bsa_problem *prob, const bsa_mask_spec *mask, const bsa
   if ((st = check_mask(out->p, mask, &out->m)) != BSA_OK) return st;
   out->L = compute_layout(out->p);
   if ((st = check_options(opt, out->L.nN, &out->o)) != BSA_OK) return st;
+  if (out->o.bound_mode == BSA_BOUND_SMOOTHED && out->p.H * out->p.D > kMaxSmoothedHD)
+    return BSA_ERR_UNSUPPORTED;
   if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return BSA_ERR_INVALID_ARG;
   if (ws_bytes < (backward ? out->L.total : out->L.fwd_end)) return BSA_ERR_WORKSPACE_TOO_SMALL;
   if (!have_device()) return BSA_ERR_NO_DEVICE;
@@ -304,6 +312,8 @@ bsa_status bsa_workspace_layout(const bsa_problem *prob, const bsa_mask_spec *ma
   view->off_delta = L.delta;
   view->off_dq_accum = L.dq_accum;
   view->off_sem = L.sem;
+  view->off_kbar = L.kbar;
+  view->off_qdot = L.qdot;
   view->nM = L.nM;
   view->nN = L.nN;
   return BSA_OK;

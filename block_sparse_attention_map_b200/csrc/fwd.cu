@@ -4,6 +4,9 @@
 //     per-row ||q_i||, and the per-head gate 2*scale*qmax*kmax <= G ("Fixed-m
 //     softmax for 2D-ring x Ulysses attention (WAN 2.2)", introduction and
 //     "Notes": heads whose bound cannot be proven safe keep online softmax).
+//     With k-smoothing ("Notes": possible when one device holds all of K) the
+//     keys are centred on their mean c first: kmax becomes the radius
+//     max ||k_j - c||, and each row's reference gains the shift scale * q_i . c.
 // a3  the tiled exact softmax attention main loop over each q-block's row list
 //     of non-empty tiles.  Online softmax keeps the running max in registers
 //     (one query row per thread) and rescales lazily; fixed-m pins the max to
@@ -48,8 +51,9 @@ struct FwdParams {
   int64_t o_sb, o_ss, o_sh;
   float *lse;
   int fixed_mode;
-  const float *kmax;   // [B, H]
+  const float *kmax;   // [B, H] (the radius R with k-smoothing)
   const float *qnorm;  // [B, H, Sq]
+  const float *qdot;   // [B, H, Sq] q_i . center with k-smoothing, else null
   const int32_t *gate; // [B, H]
   uint32_t *hdr;
   uint64_t timeout_ns;
@@ -349,7 +353,9 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       const bool fixed = p.fixed_mode && p.gate[bh] != 0;
       float m_ref = -INFINITY, l = 0.f, l_r = 0.f;
       if (fixed)
-        m_ref = row_ok ? p.scale_log2 * p.qnorm[static_cast<int64_t>(bh) * p.Sq + i] * p.kmax[bh] : 0.f;
+        m_ref = row_ok ? p.scale_log2 * fmaf(p.qnorm[static_cast<int64_t>(bh) * p.Sq + i], p.kmax[bh],
+                                             p.qdot != nullptr ? p.qdot[static_cast<int64_t>(bh) * p.Sq + i] : 0.f)
+                       : 0.f;
       // row-constant part of the mask: allowed keys lie in [lo, hi] (the
       // window, thinned by the dilation) or in the prefix [0, pre_hi]
       int lo = 0, hi = p.Skv - 1, pre_hi = -1;
@@ -531,21 +537,81 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
 // Keys: running max per (b, h) over valid keys (padding and varlen alignment
 // keys excluded).  Queries: the per-row norm is stored and the running max per
 // (b, h) kept.  Each group of D/8 threads owns one vector at a time and keeps
-// four vectors' loads in flight.
+// four vectors' loads in flight.  With k-smoothing (center != 0) the keys'
+// norms are taken of k_j - c and the queries also store q_i . c, c being the
+// mean valid key of the head from the fixed-point sums of k_key_sums.
 struct NormArgs {
   const __nv_bfloat16 *k, *q;
   int64_t ks[3], qs[3];
-  int B, Skv, Sq, H, only_q;
+  int B, Skv, Sq, H, only_q, center;
   MaskParams mk;
   float *kmax, *qmax, *qnorm;
+  long long *ksum;        // [B, H, D] fixed-point sums of the valid keys
+  int *kcount;            // [B] valid keys
+  float *kbar, *qdot;     // [B, H, D] center (written once per batch row), [B, H, Sq]
 };
+
+constexpr float kFixScale = 1048576.f;  // fixed-point unit 2^-20 of the key sums
+
+__device__ __forceinline__ bool key_is_valid(const MaskParams &mk, int b, int j) {
+  bool valid = true;
+  if (mk.flags & BSA_MASK_KV_VALID_LEN) valid = j < mk.kv_valid_len[b];
+  if ((mk.flags & BSA_MASK_VARLEN) && mk.seg_kv != nullptr) valid = valid && mk.seg_kv[j] >= 0;
+  return valid;
+}
+
+// k-smoothing, first pass: per (b, h, d) the sum over valid keys of k_jd, each
+// term rounded to a multiple of 2^-20 (|k| clamped to 2^20) and added as an
+// int64, so the total does not depend on the order of the additions; and per
+// b the number of valid keys.  A block takes 64 rows of one batch row; a
+// thread owns 8 dims of one head and walks the rows.
+template <int D>
+__global__ void __launch_bounds__(256) k_key_sums(const NormArgs a) {
+  constexpr int kRows = 64;
+  constexpr int G = D / 8;
+  const int64_t blocks_per_b = (a.Skv + kRows - 1) / kRows;
+  const int b = static_cast<int>(blockIdx.x / blocks_per_b);
+  const int r0 = static_cast<int>(blockIdx.x % blocks_per_b) * kRows;
+  const int r1 = min(a.Skv, r0 + kRows);
+  if (threadIdx.x == 0) {
+    int n = 0;
+    for (int r = r0; r < r1; ++r) n += key_is_valid(a.mk, b, r) ? 1 : 0;
+    if (n != 0) atomicAdd(a.kcount + b, n);
+  }
+  const int cols = a.H * G;
+  for (int c = threadIdx.x; c < cols; c += blockDim.x) {
+    const int h = c / G, g = c % G;
+    long long acc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = 0;
+    const __nv_bfloat16 *base = a.k + b * a.ks[0] + h * a.ks[2] + g * 8;
+#pragma unroll 4
+    for (int r = r0; r < r1; ++r) {
+      if (!key_is_valid(a.mk, b, r)) continue;
+      const int4 v = *reinterpret_cast<const int4 *>(base + static_cast<int64_t>(r) * a.ks[1]);
+      const __nv_bfloat162 *x = reinterpret_cast<const __nv_bfloat162 *>(&v);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __bfloat1622float2(x[e]);
+        acc[2 * e] += __float2ll_rn(fminf(fmaxf(f.x, -kFixScale), kFixScale) * kFixScale);
+        acc[2 * e + 1] += __float2ll_rn(fminf(fmaxf(f.y, -kFixScale), kFixScale) * kFixScale);
+      }
+    }
+    unsigned long long *dst = reinterpret_cast<unsigned long long *>(
+        a.ksum + (static_cast<int64_t>(b) * a.H + h) * D + g * 8);
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      if (acc[e] != 0) atomicAdd(dst + e, static_cast<unsigned long long>(acc[e]));
+  }
+}
 
 template <int D>
 __global__ void __launch_bounds__(256) k_row_norms(const NormArgs a) {
   constexpr int TPV = D / 8;  // threads per vector, 16 bytes each
   constexpr int kRows = 32;
   constexpr int kUnroll = 4;
-  extern __shared__ unsigned int smax[];  // [H]
+  extern __shared__ unsigned int smax[];  // [H], then the centers [H * D] (k-smoothing)
+  float *cen = reinterpret_cast<float *>(smax + a.H);
   const int is_key = !a.only_q && blockIdx.y == 0;
   const __nv_bfloat16 *x = is_key ? a.k : a.q;
   const int S = is_key ? a.Skv : a.Sq;
@@ -560,13 +626,24 @@ __global__ void __launch_bounds__(256) k_row_norms(const NormArgs a) {
   const int r0 = static_cast<int>(blockIdx.x % blocks_per_b) * kRows;
   if (r0 >= S) return;  // whole block past this tensor's rows (uniform)
   for (int h = threadIdx.x; h < H; h += blockDim.x) smax[h] = 0u;
+  if (a.center) {
+    // c = (fixed-point sum) * 2^-20 / (valid keys), the same in every block
+    const double inv = 1.0 / (static_cast<double>(kFixScale) * max(1, a.kcount[b]));
+    const long long *ks = a.ksum + static_cast<int64_t>(b) * H * D;
+    const bool write = is_key && r0 == 0;
+    for (int t = threadIdx.x; t < H * D; t += blockDim.x) {
+      const float c = static_cast<float>(static_cast<double>(ks[t]) * inv);
+      cen[t] = c;
+      if (write) a.kbar[static_cast<int64_t>(b) * H * D + t] = c;
+    }
+  }
   __syncthreads();
   const int g = threadIdx.x / TPV, t = threadIdx.x % TPV;
   const int groups = blockDim.x / TPV;
   const int pairs = kRows * H;
   // uniform trip count across the warp: the shuffles below need every lane
   for (int base = 0; base < pairs; base += groups * kUnroll) {
-    float acc[kUnroll];
+    float acc[kUnroll], dot[kUnroll];
     int row[kUnroll], hh[kUnroll];
     bool in[kUnroll];
 #pragma unroll
@@ -576,13 +653,24 @@ __global__ void __launch_bounds__(256) k_row_norms(const NormArgs a) {
       hh[u] = pair % H;
       in[u] = pair < pairs && row[u] < S;
       acc[u] = 0.f;
+      dot[u] = 0.f;
       if (in[u]) {
         const int4 v = *reinterpret_cast<const int4 *>(x + b * sb + static_cast<int64_t>(row[u]) * ss +
                                                       hh[u] * sh + t * 8);
         const __nv_bfloat162 *e = reinterpret_cast<const __nv_bfloat162 *>(&v);
+        const float *c = cen + hh[u] * D + t * 8;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          const float2 f = __bfloat1622float2(e[q]);
+          float2 f = __bfloat1622float2(e[q]);
+          if (a.center) {
+            if (is_key) {
+              f.x -= c[2 * q];
+              f.y -= c[2 * q + 1];
+            } else {
+              dot[u] = fmaf(f.x, c[2 * q], dot[u]);
+              dot[u] = fmaf(f.y, c[2 * q + 1], dot[u]);
+            }
+          }
           acc[u] = fmaf(f.x, f.x, acc[u]);
           acc[u] = fmaf(f.y, f.y, acc[u]);
         }
@@ -591,15 +679,19 @@ __global__ void __launch_bounds__(256) k_row_norms(const NormArgs a) {
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
 #pragma unroll
-      for (int o = TPV / 2; o > 0; o >>= 1) acc[u] += __shfl_xor_sync(0xffffffffu, acc[u], o);
+      for (int o = TPV / 2; o > 0; o >>= 1) {
+        acc[u] += __shfl_xor_sync(0xffffffffu, acc[u], o);
+        dot[u] += __shfl_xor_sync(0xffffffffu, dot[u], o);
+      }
       if (t == 0 && in[u]) {
         const float nrm = sqrtf(acc[u]);
         bool valid = true;
         if (is_key) {
-          if (mk.flags & BSA_MASK_KV_VALID_LEN) valid = row[u] < mk.kv_valid_len[b];
-          if ((mk.flags & BSA_MASK_VARLEN) && mk.seg_kv != nullptr) valid = valid && mk.seg_kv[row[u]] >= 0;
+          valid = key_is_valid(mk, b, row[u]);
         } else {
-          qnorm[(static_cast<int64_t>(b) * H + hh[u]) * S + row[u]] = nrm;
+          const int64_t idx = (static_cast<int64_t>(b) * H + hh[u]) * S + row[u];
+          qnorm[idx] = nrm;
+          if (a.center) a.qdot[idx] = dot[u];
         }
         if (valid) atomicMax(&smax[hh[u]], __float_as_uint(nrm));
       }
@@ -665,15 +757,37 @@ cudaError_t launch_fixed_m_bound(const bsa_problem &p, const MaskParams &mp,
   na.Sq = p.Sq;
   na.H = p.H;
   na.only_q = o.kmax_override != nullptr;  // a caller-supplied kmax needs no key pass
+  na.center = o.bound_mode == BSA_BOUND_SMOOTHED;
   na.mk = mp;
   na.kmax = reinterpret_cast<float *>(ws + L.kmax);
   na.qmax = reinterpret_cast<float *>(ws + L.qmax);
   na.qnorm = reinterpret_cast<float *>(ws + L.qnorm);
+  na.ksum = reinterpret_cast<long long *>(ws + L.ksum);
+  na.kcount = reinterpret_cast<int *>(ws + L.kcount);
+  na.kbar = reinterpret_cast<float *>(ws + L.kbar);
+  na.qdot = reinterpret_cast<float *>(ws + L.qdot);
   cudaError_t e = cudaMemsetAsync(na.kmax, 0, sizeof(float) * p.B * p.H * 2, s);  // kmax, qmax
   if (e != cudaSuccess) return e;
+  size_t smem = sizeof(unsigned int) * p.H;
+  if (na.center) {
+    // ksum and kcount are adjacent regions: one memset
+    e = cudaMemsetAsync(ws + L.ksum, 0, L.qdot - L.ksum, s);
+    if (e != cudaSuccess) return e;
+    const unsigned sblocks = static_cast<unsigned>(static_cast<int64_t>(p.B) * ((p.Skv + 63) / 64));
+    if (p.D == 64) k_key_sums<64><<<sblocks, 256, 0, s>>>(na);
+    else k_key_sums<128><<<sblocks, 256, 0, s>>>(na);
+    count_launch();
+    smem += sizeof(float) * p.H * p.D;
+  }
   const int64_t blocks = static_cast<int64_t>(p.B) * ((std::max(p.Sq, p.Skv) + 31) / 32);
   const dim3 grid(static_cast<unsigned>(blocks), na.only_q ? 1u : 2u);
-  const size_t smem = sizeof(unsigned int) * p.H;
+  if (smem > 48 * 1024) {
+    e = p.D == 64 ? cudaFuncSetAttribute(k_row_norms<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem))
+                  : cudaFuncSetAttribute(k_row_norms<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+  }
   if (p.D == 64) k_row_norms<64><<<grid, 256, smem, s>>>(na);
   else k_row_norms<128><<<grid, 256, smem, s>>>(na);
   count_launch();
@@ -709,6 +823,7 @@ cudaError_t launch_fwd(const bsa_problem &p, const MaskParams &mp, const bsa_opt
   fp.fixed_mode = o.softmax_mode == BSA_SOFTMAX_FIXED_M_GATED;
   fp.kmax = reinterpret_cast<const float *>(ws + L.kmax);
   fp.qnorm = reinterpret_cast<const float *>(ws + L.qnorm);
+  fp.qdot = o.bound_mode == BSA_BOUND_SMOOTHED ? reinterpret_cast<const float *>(ws + L.qdot) : nullptr;
   fp.gate = reinterpret_cast<const int32_t *>(ws + L.gate);
   fp.hdr = reinterpret_cast<uint32_t *>(ws + L.status);
   fp.timeout_ns = 2000000000ull;

@@ -18,6 +18,9 @@ constexpr uint32_t kIndexMask = (1u << 30) - 1u;
 constexpr uint32_t kPlanMagic = 0xB5A7C0DEu;
 // Largest Sq and Skv accepted (bsa_problem).
 constexpr int kMaxSeq = 1 << 21;
+// Largest H * D of the k-smoothed bound: one block keeps the centers of all
+// heads of a batch row in shared memory (fp32).
+constexpr int kMaxSmoothedHD = 24576;
 
 // Header words at the start of the workspace.
 enum HeaderWord : int {
@@ -47,6 +50,8 @@ struct WsLayout {
   size_t qblk, kblk;                  // per-block segment summaries [B*nM*4], [B*nN*4]
   size_t kmax, qmax, gate;            // [B, H]
   size_t qnorm;                       // [B, H, Sq]
+  size_t kbar, ksum, kcount, qdot;    // k-smoothing: center [B,H,D] fp32, its fixed-point
+                                      // sums [B,H,D] int64, valid keys [B], q.c [B,H,Sq]
   size_t fwd_end;
   size_t delta, dq_accum, sem;        // backward scratch
   size_t total;

@@ -98,6 +98,19 @@ typedef enum bsa_status {
 #define BSA_SOFTMAX_ONLINE 0
 #define BSA_SOFTMAX_FIXED_M_GATED 1
 
+/* bsa_options.bound_mode: the pinned reference of BSA_SOFTMAX_FIXED_M_GATED
+ * ("Fixed-m softmax for 2D-ring x Ulysses attention (WAN 2.2)", introduction and
+ * "Notes": k-smoothing is possible when one device holds all of K).
+ *   NORM      m_i = scale*||q_i||*kmax, kmax = max over valid keys of ||k_j||;
+ *             gate 2*scale*qmax*kmax <= G.
+ *   SMOOTHED  center c = mean of the valid keys, R = max over valid keys of
+ *             ||k_j - c||, m_i = scale*(q_i.c + ||q_i||*R); gate 2*scale*qmax*R <= G.
+ *             The workspace's kmax array then holds R.  c is summed in a fixed-point
+ *             format (terms rounded to 2^-20, |k| clamped to 2^20), so it does not
+ *             depend on the order of the additions; any c keeps m_i a bound. */
+#define BSA_BOUND_NORM 0
+#define BSA_BOUND_SMOOTHED 1
+
 /* bsa_options.bwd_order: order pi of the kv columns for the dQ semaphores */
 #define BSA_ORDER_ASC 0
 #define BSA_ORDER_DESC 1
@@ -164,6 +177,9 @@ typedef struct bsa_options {
   int32_t bound_ready;         /* fixed-m only. 1: the workspace already holds
                                   kmax/qmax/gate from bsa_fixed_m_bound for these
                                   q and k; 0: bsa_attn_fwd computes them first      */
+  int32_t bound_mode;          /* BSA_BOUND_*; SMOOTHED with kmax_override or with
+                                  H*D > 24576 is rejected                           */
+  int32_t reserved;
 } bsa_options;
 
 /* Where the plan and the scratch arrays sit inside the workspace (byte offsets),
@@ -186,6 +202,8 @@ typedef struct bsa_workspace_view {
   size_t off_delta;            /* fp32   [B, H, nM*128]  backward Delta              */
   size_t off_dq_accum;         /* fp32   backward dQ accumulator                     */
   size_t off_sem;              /* int32  [B, H, nM]   dQ semaphores                  */
+  size_t off_kbar;             /* fp32   [B, H, D]    k-smoothing center             */
+  size_t off_qdot;             /* fp32   [B, H, Sq]   q_i . center                   */
   int32_t nM, nN;
 } bsa_workspace_view;
 

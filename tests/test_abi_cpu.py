@@ -48,6 +48,7 @@ int main(void) {
   P(bsa_mask_spec, seg_q) P(bsa_mask_spec, cu_seqlens) P(bsa_mask_spec, n_align_tail)
   P(bsa_mask_spec, prefix_len) P(bsa_mask_spec, dilation)
   P(bsa_options, kmax_override) P(bsa_options, perm) P(bsa_options, sem_timeout_ns) P(bsa_options, plan_ready)
+  P(bsa_options, bound_mode) P(bsa_workspace_view, off_qdot)
   P(bsa_workspace_view, off_sem) P(bsa_workspace_view, nN)
   return 0;
 }
@@ -75,6 +76,8 @@ def test_ctypes_structs_match_c_layout():
     assert c["bsa_mask_spec.n_align_tail"] == bd.MaskSpec.n_align_tail.offset
     assert c["bsa_mask_spec.prefix_len"] == bd.MaskSpec.prefix_len.offset
     assert c["bsa_mask_spec.dilation"] == bd.MaskSpec.dilation.offset
+    assert c["bsa_options.bound_mode"] == bd.Options.bound_mode.offset
+    assert c["bsa_workspace_view.off_qdot"] == bd.WorkspaceView.off_qdot.offset
     assert c["bsa_options.kmax_override"] == bd.Options.kmax_override.offset
     assert c["bsa_options.perm"] == bd.Options.perm.offset
     assert c["bsa_options.sem_timeout_ns"] == bd.Options.sem_timeout_ns.offset
@@ -154,6 +157,16 @@ def test_calls_reject_bad_arguments_before_cuda(L):
     o = bd.Options()
     o.bwd_order = 5
     assert L.bsa_plan_build(ctypes.byref(p), None, ctypes.byref(o), 4096, 16, None) == 1
+    # unknown bound mode; the smoothed bound with a caller-supplied kmax
+    o = bd.Options()
+    o.bound_mode = 2
+    assert L.bsa_plan_build(ctypes.byref(p), None, ctypes.byref(o), 4096, 1 << 30, None) == 1
+    o.bound_mode = 1
+    o.kmax_override = 4096
+    assert L.bsa_plan_build(ctypes.byref(p), None, ctypes.byref(o), 4096, 1 << 30, None) == 1
+    o.kmax_override = None
+    wide = _prob(H=200, D=128)                      # centers of 200 heads exceed shared memory
+    assert L.bsa_plan_build(ctypes.byref(wide), None, ctypes.byref(o), 4096, 1 << 40, None) == 2
     # workspace too small
     o = bd.Options()
     assert L.bsa_plan_build(ctypes.byref(p), None, ctypes.byref(o), 4096, 16, None) == 3

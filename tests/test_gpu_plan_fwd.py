@@ -78,8 +78,8 @@ def test_plan_greedy_order_full_size(name):
     assert ws.status() == 0
 
 
-def _fwd_vs_oracle(wl, mode="online", rows=None):
-    o, lse, ws = bsa.attn_fwd(wl.q, wl.k, wl.v, wl.mask, softmax_mode=mode)
+def _fwd_vs_oracle(wl, mode="online", rows=None, **kw):
+    o, lse, ws = bsa.attn_fwd(wl.q, wl.k, wl.v, wl.mask, softmax_mode=mode, **kw)
     torch.cuda.synchronize()
     assert ws.status() == 0
     q, k, v = np64(wl.q), np64(wl.k), np64(wl.v)
@@ -116,6 +116,51 @@ def test_fixed_m_bound_and_gate_match_oracle():
     close = np.abs(2 * bound - 64.0) < 1e-4 * 64
     assert np.array_equal(g[~close], gate[~close])
     assert not g[0, 0] and g[0, 1:].all()  # the sink head falls back
+
+
+def _with_key_offset(wl, norm=40.0):
+    """The same workload with a common offset of the given norm added to every
+    key (along the first head dim): the case k-smoothing is for."""
+    k = wl.k.float()
+    k[..., 0] += norm
+    wl.k = k.to(torch.bfloat16)
+    return wl
+
+
+@pytest.mark.parametrize("name", ["window", "video", "packed", "varlen"])
+def test_smoothed_bound_matches_oracle(name):
+    wl = make_workload(name, device="cuda", small=True)
+    if name == "window":
+        wl = _with_key_offset(wl)
+    eo, el, same, o, lse, ws = _fwd_vs_oracle(wl, "fixed_m", bound_mode="smoothed")
+    assert eo <= O_TOL and el <= LSE_TOL and same, (eo, el, same)
+    kbar, radius, qmax, bound, gate = oracle.fixed_m_bound_smoothed(np64(wl.q), np64(wl.k), mask_desc(wl),
+                                                                    wl.scale)
+    # the center is summed in 2^-20 fixed point, then divided in fp64 and rounded to fp32
+    assert np.abs(ws.kbar().cpu().numpy() - kbar).max() <= 1e-5 * max(1.0, np.abs(kbar).max())
+    assert np.allclose(ws.kmax().cpu().numpy(), radius, rtol=1e-4, atol=1e-4)
+    assert np.allclose(ws.qmax().cpu().numpy(), qmax, rtol=1e-5)
+    g = ws.gate().cpu().numpy().astype(bool)
+    close = np.abs(2 * bound - 64.0) < 1e-3 * 64
+    assert np.array_equal(g[~close], gate[~close])
+
+
+def test_smoothing_widens_the_gate_and_stays_exact_and_deterministic():
+    wl = _with_key_offset(make_workload("window", device="cuda", small=True))
+    _, _, ws_plain = bsa.attn_fwd(wl.q, wl.k, wl.v, wl.mask, softmax_mode="fixed_m")
+    o, lse, ws = bsa.attn_fwd(wl.q, wl.k, wl.v, wl.mask, softmax_mode="fixed_m", bound_mode="smoothed")
+    torch.cuda.synchronize()
+    plain = oracle.fixed_m_bound(np64(wl.q), np64(wl.k), mask_desc(wl), wl.scale)[3]
+    assert not plain.any() and not ws_plain.gate().cpu().numpy().any()  # the offset breaks the plain gate
+    assert ws.gate().cpu().numpy().all()                               # the centred keys pass it
+    for _ in range(3):
+        o2, l2, _ = bsa.attn_fwd(wl.q, wl.k, wl.v, wl.mask, softmax_mode="fixed_m", bound_mode="smoothed")
+        assert torch.equal(o, o2) and torch.equal(lse, l2)
+    o3, l3, _ = bsa.attn_fwd(wl.q, wl.k, wl.v, wl.mask, softmax_mode="online")
+    torch.cuda.synchronize()
+    assert (o - o3).abs().max().item() <= O_TOL
+    fin = torch.isfinite(l3)
+    assert (lse[fin] - l3[fin]).abs().max().item() <= LSE_TOL
 
 
 def test_fixed_m_and_online_agree_bitwise_on_fallback_head():
