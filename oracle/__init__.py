@@ -18,6 +18,7 @@ live in ``tests/test_oracle_*.py``; no function here is "parity unpinned".
 
 from .attention import (  # noqa: F401
     MaskDesc,
+    kv_head_of,
     allowed_rows,
     valid_keys,
     attention_forward,

@@ -140,6 +140,18 @@ def _as64(x) -> np.ndarray:
     return np.asarray(x, dtype=np.float64)
 
 
+def kv_head_of(H: int, H_kv: int):
+    """Grouped-query attention (GQA / MQA): query head h reads key/value head
+    h // (H / H_kv), so consecutive query heads share one kv head (H_kv == H is
+    plain multi-head attention, H_kv == 1 multi-query).  The pages only name the
+    "kv_mode" column of the dk-order benchmark (all of whose rows are MHA); this
+    contiguous grouping is the reading taken."""
+    if H_kv < 1 or H % H_kv != 0:
+        raise ValueError("H must be a multiple of the kv head count")
+    g = H // H_kv
+    return lambda h: h // g
+
+
 def _row_chunks(rows: np.ndarray, chunk: int):
     for s in range(0, rows.size, chunk):
         yield rows[s:s + chunk]
@@ -149,7 +161,8 @@ def attention_forward(q, k, v, mask: MaskDesc, scale: float, rows=None, heads=No
                       batches=None, chunk: int = 1024):
     """O = softmax(scale * Q K^T + mask) V and LSE, dense, per row.
 
-    q: [B, Sq, H, D], k, v: [B, Skv, H, D] (any float type; computed in fp64).
+    q: [B, Sq, H, D], k, v: [B, Skv, H_kv, D] (any float type; computed in fp64),
+    H a multiple of H_kv (:func:`kv_head_of`).
     Returns (O [B, Sq, H, D] fp64, LSE [B, H, Sq] fp64).  Rows outside ``rows``
     (and heads/batches outside the given subsets) are left as NaN.
 
@@ -162,6 +175,7 @@ def attention_forward(q, k, v, mask: MaskDesc, scale: float, rows=None, heads=No
     rows = np.arange(Sq) if rows is None else np.asarray(rows)
     heads = range(H) if heads is None else heads
     batches = range(B) if batches is None else batches
+    kvh = kv_head_of(H, k.shape[2])
     O = np.full((B, Sq, H, v.shape[3]), np.nan)
     LSE = np.full((B, H, Sq), np.nan)
     for b in batches:
@@ -169,14 +183,15 @@ def attention_forward(q, k, v, mask: MaskDesc, scale: float, rows=None, heads=No
             a = allowed_rows(mask, b, r, Sq, Skv)
             has = a.any(axis=1)
             for h in heads:
-                s = scale * (q[b, r, h, :] @ k[b, :, h, :].T)
+                hk = kvh(h)
+                s = scale * (q[b, r, h, :] @ k[b, :, hk, :].T)
                 s = np.where(a, s, NEG_INF)
                 M = np.where(has, s.max(axis=1), 0.0)
                 e = np.where(a, np.exp(s - M[:, None]), 0.0)
                 l = e.sum(axis=1)
                 safe_l = np.where(has, l, 1.0)
                 P = e / safe_l[:, None]
-                O[b, r, h, :] = P @ v[b, :, h, :]
+                O[b, r, h, :] = P @ v[b, :, hk, :]
                 LSE[b, h, r] = np.where(has, M + np.log(safe_l), NEG_INF)
     return O, LSE
 
@@ -188,7 +203,8 @@ def attention_backward(q, k, v, dO, mask: MaskDesc, scale: float, chunk: int = 1
     With P the softmax weights (0 on masked entries and on empty rows):
       Delta_i = sum_d dO_id O_id   (O from this oracle's own forward)
       dP = dO V^T,  dS = P o (dP - Delta),
-      dQ = scale * dS K,  dK = scale * dS^T Q,  dV = P^T dO.
+      dQ = scale * dS K,  dK = scale * dS^T Q,  dV = P^T dO,
+    with dK and dV of a shared kv head summed over the query heads of its group.
     Returns (dQ, dK, dV) fp64 with the input layouts.
     """
     q, k, v, dO = _as64(q), _as64(k), _as64(v), _as64(dO)
@@ -196,6 +212,7 @@ def attention_backward(q, k, v, dO, mask: MaskDesc, scale: float, chunk: int = 1
     Skv = k.shape[1]
     heads = range(H) if heads is None else heads
     batches = range(B) if batches is None else batches
+    kvh = kv_head_of(H, k.shape[2])
     dQ = np.zeros_like(q)
     dK = np.zeros_like(k)
     dV = np.zeros_like(v)
@@ -205,20 +222,21 @@ def attention_backward(q, k, v, dO, mask: MaskDesc, scale: float, chunk: int = 1
             a = allowed_rows(mask, b, r, Sq, Skv)
             has = a.any(axis=1)
             for h in heads:
-                s = scale * (q[b, r, h, :] @ k[b, :, h, :].T)
+                hk = kvh(h)
+                s = scale * (q[b, r, h, :] @ k[b, :, hk, :].T)
                 s = np.where(a, s, NEG_INF)
                 M = np.where(has, s.max(axis=1), 0.0)
                 e = np.where(a, np.exp(s - M[:, None]), 0.0)
                 l = np.where(has, e.sum(axis=1), 1.0)
                 P = e / l[:, None]
-                O = P @ v[b, :, h, :]
+                O = P @ v[b, :, hk, :]
                 do = dO[b, r, h, :]
                 delta = (do * O).sum(axis=1)
-                dP = do @ v[b, :, h, :].T
+                dP = do @ v[b, :, hk, :].T
                 dS = P * (dP - delta[:, None])
-                dQ[b, r, h, :] = scale * (dS @ k[b, :, h, :])
-                dK[b, :, h, :] += scale * (dS.T @ q[b, r, h, :])
-                dV[b, :, h, :] += P.T @ do
+                dQ[b, r, h, :] = scale * (dS @ k[b, :, hk, :])
+                dK[b, :, hk, :] += scale * (dS.T @ q[b, r, h, :])
+                dV[b, :, hk, :] += P.T @ do
     return dQ, dK, dV
 
 
@@ -246,6 +264,7 @@ def attention_forward_fixed_m(q, k, v, mask: MaskDesc, scale: float, kmax=None,
     if kmax is None:
         kmax = fixed_m_bound(q, k, mask, scale)[0]
     kmax = _as64(kmax)
+    kvh = kv_head_of(H, k.shape[2])
     rows = np.arange(Sq) if rows is None else np.asarray(rows)
     heads = range(H) if heads is None else heads
     batches = range(B) if batches is None else batches
@@ -260,11 +279,11 @@ def attention_forward_fixed_m(q, k, v, mask: MaskDesc, scale: float, kmax=None,
                 m = scale * np.sqrt((qr * qr).sum(axis=1)) * kmax[b, h]
                 if kbar is not None:
                     m = m + scale * (qr @ _as64(kbar)[b, h])
-                s = scale * (qr @ k[b, :, h, :].T)
+                s = scale * (qr @ k[b, :, kvh(h), :].T)
                 e = np.where(a, np.exp(s - m[:, None]), 0.0)
                 l = e.sum(axis=1)
                 safe_l = np.where(has, l, 1.0)
-                O[b, r, h, :] = (e / safe_l[:, None]) @ v[b, :, h, :]
+                O[b, r, h, :] = (e / safe_l[:, None]) @ v[b, :, kvh(h), :]
                 LSE[b, h, r] = np.where(has, m + np.log(safe_l), NEG_INF)
     return O, LSE
 
@@ -286,12 +305,13 @@ def fixed_m_bound(q, k, mask: MaskDesc, scale: float, gate_limit: float = 64.0):
     q, k = _as64(q), _as64(k)
     B, Sq, H, D = q.shape
     Skv = k.shape[1]
+    kvh = kv_head_of(H, k.shape[2])
     kmax = np.zeros((B, H))
     qmax = np.zeros((B, H))
     for b in range(B):
         vk = valid_keys(mask, b, Skv)
         for h in range(H):
-            kn = np.sqrt((k[b, :, h, :] ** 2).sum(axis=1))
+            kn = np.sqrt((k[b, :, kvh(h), :] ** 2).sum(axis=1))
             kmax[b, h] = kn[vk].max() if vk.any() else 0.0
             qmax[b, h] = np.sqrt((q[b, :, h, :] ** 2).sum(axis=1)).max()
     bound = scale * qmax * kmax
@@ -316,11 +336,13 @@ def fixed_m_bound_smoothed(q, k, mask: MaskDesc, scale: float, gate_limit: float
 
     since every s_ij - scale * q_i . kbar lies in [-scale ||q_i|| radius,
     scale ||q_i|| radius], the pinned m_i sits at most 2 * bound above the row
-    max.  Returns (kbar [B, H, D], radius, qmax, bound, gate).
+    max.  Returns (kbar [B, H, D], radius, qmax, bound, gate), indexed by query
+    head (with GQA the query heads of a group share their kv head's values).
     """
     q, k = _as64(q), _as64(k)
     B, Sq, H, D = q.shape
     Skv = k.shape[1]
+    kvh = kv_head_of(H, k.shape[2])
     kbar = np.zeros((B, H, D))
     radius = np.zeros((B, H))
     qmax = np.zeros((B, H))
@@ -328,7 +350,7 @@ def fixed_m_bound_smoothed(q, k, mask: MaskDesc, scale: float, gate_limit: float
         vk = valid_keys(mask, b, Skv)
         for h in range(H):
             if vk.any():
-                kv = k[b, vk, h, :]
+                kv = k[b, vk, kvh(h), :]
                 kbar[b, h] = kv.mean(axis=0)
                 radius[b, h] = np.sqrt(((kv - kbar[b, h]) ** 2).sum(axis=1)).max()
             qmax[b, h] = np.sqrt((q[b, :, h, :] ** 2).sum(axis=1)).max()

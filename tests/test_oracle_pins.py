@@ -311,6 +311,47 @@ def test_smoothing_widens_gate_and_stays_exact():
     assert np.max(np.abs(O - Os)) < 1e-12 and np.max(np.abs(L - Ls)) < 1e-12
 
 
+@pytest.mark.parametrize("H_kv", [1, 2])
+def test_gqa_matches_library_sdpa_and_autograd(H_kv):
+    # torch's SDPA with enable_gqa (a library routine) and autograd through it
+    import torch
+    q, k, v, dO = P.tiny_inputs(23, B=2, Sq=10, Skv=12, D=4, H=4)
+    k, v = k[:, :, :H_kv].copy(), v[:, :, :H_kv].copy()
+    v, dO = v[..., :4].copy(), dO[..., :4].copy()
+    mask = P.tiny_masks(2, 10, 12, seed=4)["window3"]
+    allowed = P.dense_allowed(mask, 2, 10, 12)
+    O, _ = oracle.attention_forward(q, k, v, mask, SCALE)
+    dq, dk, dv = oracle.attention_backward(q, k, v, dO, mask, SCALE)
+    t = lambda x: torch.from_numpy(np.ascontiguousarray(x)).permute(0, 2, 1, 3).clone().requires_grad_(True)
+    qt, kt, vt = t(q), t(k), t(v)
+    m = torch.from_numpy(np.stack(allowed))[:, None, :, :]
+    ot = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, attn_mask=m, scale=SCALE,
+                                                          enable_gqa=True)
+    (ot * torch.from_numpy(dO).permute(0, 2, 1, 3)).sum().backward()
+    back = lambda x: x.detach().permute(0, 2, 1, 3).numpy()
+    assert np.max(np.abs(O - back(ot))) < 1e-12
+    for x, y in ((dq, qt.grad), (dk, kt.grad), (dv, vt.grad)):
+        assert np.max(np.abs(x - back(y))) < 1e-11
+
+
+def test_gqa_equals_mha_with_repeated_kv_heads():
+    q, k, v, dO = P.tiny_inputs(24, B=1, Sq=9, Skv=9, D=4, H=6)
+    k, v = k[:, :, :2].copy(), v[:, :, :2].copy()
+    mask = MaskDesc(window=0)
+    kr, vr = np.repeat(k, 3, axis=2), np.repeat(v, 3, axis=2)
+    assert oracle.kv_head_of(6, 2)(4) == 1
+    a = oracle.attention_forward(q, k, v, mask, SCALE)
+    b = oracle.attention_forward(q, kr, vr, mask, SCALE)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+    gq, gk, gv = oracle.attention_backward(q, k, v, dO, mask, SCALE)
+    rq, rk, rv = oracle.attention_backward(q, kr, vr, dO, mask, SCALE)
+    assert np.array_equal(gq, rq)
+    assert np.max(np.abs(gk - rk.reshape(1, 9, 2, 3, -1).sum(axis=3))) < 1e-13
+    assert np.max(np.abs(gv - rv.reshape(1, 9, 2, 3, -1).sum(axis=3))) < 1e-13
+    with pytest.raises(ValueError):
+        oracle.kv_head_of(6, 4)
+
+
 def test_gradient_identities():
     q, k, v, dO = P.tiny_inputs(16, B=1, Sq=9, Skv=9, D=4)
     v, dO = v[..., :4].copy(), dO[..., :4].copy()
