@@ -49,6 +49,8 @@ WORKLOADS = {
                "bf16 N(0,1) seed 2",
     "document": "document-causal (runs of 256..2048 tokens): B=1, H=16, Sq=Skv=8192, D=128, "
                 "bf16 N(0,1) seed 2",
+    "gqa": "grouped-query causal sliding window 512: B=1, H=16 over H_kv=4, Sq=Skv=8192, D=128, "
+           "bf16 N(0,1) seed 5",
 }
 
 

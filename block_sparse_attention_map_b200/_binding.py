@@ -38,7 +38,7 @@ STATUS = {
 
 class Problem(ctypes.Structure):
     _fields_ = [("B", c_i32), ("H", c_i32), ("Sq", c_i32), ("Skv", c_i32), ("D", c_i32),
-                ("reserved0", c_i32), ("q_stride", c_i64 * 3), ("k_stride", c_i64 * 3),
+                ("H_kv", c_i32), ("q_stride", c_i64 * 3), ("k_stride", c_i64 * 3),
                 ("v_stride", c_i64 * 3), ("o_stride", c_i64 * 3), ("scale", c_f32),
                 ("reserved1", c_i32)]
 
@@ -147,10 +147,11 @@ def make_problem(q, k, v, o=None, scale: Optional[float] = None) -> Problem:
         if t.dtype != torch.bfloat16 or not t.is_cuda:
             raise ValueError("q, k, v must be bf16 CUDA tensors")
     B, Sq, H, D = q.shape
-    if k.shape[0] != B or k.shape[2] != H or k.shape[3] != D or v.shape != k.shape:
-        raise ValueError("k and v must be [B, Skv, H, D] with q's B, H, D")
+    H_kv = k.shape[2]
+    if k.shape[0] != B or H_kv < 1 or H % H_kv != 0 or k.shape[3] != D or v.shape != k.shape:
+        raise ValueError("k and v must be [B, Skv, H_kv, D] with q's B and D and H a multiple of H_kv")
     p = Problem()
-    p.B, p.H, p.Sq, p.Skv, p.D = B, H, Sq, k.shape[1], D
+    p.B, p.H, p.Sq, p.Skv, p.D, p.H_kv = B, H, Sq, k.shape[1], D, H_kv
     p.q_stride[:] = _strides(q)
     p.k_stride[:] = _strides(k)
     p.v_stride[:] = _strides(v)
@@ -234,6 +235,7 @@ class Workspace:
         self.nbytes = view.total_bytes if backward else view.fwd_bytes
         self.buf = torch.empty(self.nbytes, dtype=torch.uint8, device=device)
         self.B, self.H, self.D, self.nM, self.nN = prob.B, prob.H, prob.D, view.nM, view.nN
+        self.H_kv = prob.H_kv or prob.H
 
     def ptr(self):
         return self.buf.data_ptr()
@@ -276,9 +278,9 @@ class Workspace:
         return self._arr(self.view.off_gate, self.B * self.H, torch.int32).view(self.B, self.H)
 
     def kbar(self):
-        """The k-smoothing centers [B, H, D] (after a smoothed bound)."""
-        return self._arr(self.view.off_kbar, self.B * self.H * self.D, torch.float32).view(
-            self.B, self.H, self.D)
+        """The k-smoothing centers [B, H_kv, D] (after a smoothed bound)."""
+        return self._arr(self.view.off_kbar, self.B * self.H_kv * self.D, torch.float32).view(
+            self.B, self.H_kv, self.D)
 
     def status(self, clear=False):
         s = torch.cuda.current_stream().cuda_stream

@@ -115,15 +115,17 @@ bsa_status normalise(const bsa_problem *in, bsa_problem *out) {
   *out = *in;
   bsa_problem &p = *out;
   if (p.B < 1 || p.H < 1 || p.Sq < 1 || p.Skv < 1) return BSA_ERR_INVALID_ARG;
+  if (p.H_kv == 0) p.H_kv = p.H;
+  if (p.H_kv < 1 || p.H % p.H_kv != 0) return BSA_ERR_INVALID_ARG;
   if (p.D != 64 && p.D != 128) return BSA_ERR_UNSUPPORTED;
   if (p.Sq > kMaxSeq || p.Skv > kMaxSeq) return BSA_ERR_UNSUPPORTED;
   const int64_t nM = cdiv64(p.Sq, kTile), nN = cdiv64(p.Skv, kTile);
   if (static_cast<int64_t>(p.B) * nM * nN >= (int64_t{1} << 30)) return BSA_ERR_UNSUPPORTED;
   if (static_cast<int64_t>(p.B) * p.H * nM >= (int64_t{1} << 31)) return BSA_ERR_UNSUPPORTED;
-  auto fix = [&](int64_t *s, int64_t S) -> bsa_status {
+  auto fix = [&](int64_t *s, int64_t S, int64_t heads) -> bsa_status {
     if (s[0] == 0 && s[1] == 0 && s[2] == 0) {
-      s[0] = S * p.H * p.D;
-      s[1] = static_cast<int64_t>(p.H) * p.D;
+      s[0] = S * heads * p.D;
+      s[1] = heads * p.D;
       s[2] = p.D;
     }
     for (int i = 0; i < 3; ++i) {
@@ -133,10 +135,10 @@ bsa_status normalise(const bsa_problem *in, bsa_problem *out) {
     return BSA_OK;
   };
   bsa_status st;
-  if ((st = fix(p.q_stride, p.Sq)) != BSA_OK) return st;
-  if ((st = fix(p.k_stride, p.Skv)) != BSA_OK) return st;
-  if ((st = fix(p.v_stride, p.Skv)) != BSA_OK) return st;
-  if ((st = fix(p.o_stride, p.Sq)) != BSA_OK) return st;
+  if ((st = fix(p.q_stride, p.Sq, p.H)) != BSA_OK) return st;
+  if ((st = fix(p.k_stride, p.Skv, p.H_kv)) != BSA_OK) return st;
+  if ((st = fix(p.v_stride, p.Skv, p.H_kv)) != BSA_OK) return st;
+  if ((st = fix(p.o_stride, p.Sq, p.H)) != BSA_OK) return st;
   if (!(p.scale > 0.f) || !std::isfinite(p.scale)) p.scale = 1.0f / std::sqrt(static_cast<float>(p.D));
   return BSA_OK;
 }
@@ -256,7 +258,7 @@ bsa_status prepare(const bsa_problem *prob, const bsa_mask_spec *mask, const bsa
   if ((st = check_mask(out->p, mask, &out->m)) != BSA_OK) return st;
   out->L = compute_layout(out->p);
   if ((st = check_options(opt, out->L.nN, &out->o)) != BSA_OK) return st;
-  if (out->o.bound_mode == BSA_BOUND_SMOOTHED && out->p.H * out->p.D > kMaxSmoothedHD)
+  if (out->o.bound_mode == BSA_BOUND_SMOOTHED && out->p.H_kv * out->p.D > kMaxSmoothedHD)
     return BSA_ERR_UNSUPPORTED;
   if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return BSA_ERR_INVALID_ARG;
   if (ws_bytes < (backward ? out->L.total : out->L.fwd_end)) return BSA_ERR_WORKSPACE_TOO_SMALL;
@@ -342,8 +344,8 @@ bsa_status bsa_attn_fwd(const bsa_problem *prob, const bsa_mask_spec *mask,
   const bsa_problem &p = P.p;
   CUtensorMap tq, tk, tv;
   if (!make_map(&tq, q, p.B, p.Sq, p.H, p.D, p.q_stride) ||
-      !make_map(&tk, k, p.B, p.Skv, p.H, p.D, p.k_stride) ||
-      !make_map(&tv, v, p.B, p.Skv, p.H, p.D, p.v_stride))
+      !make_map(&tk, k, p.B, p.Skv, p.H_kv, p.D, p.k_stride) ||
+      !make_map(&tv, v, p.B, p.Skv, p.H_kv, p.D, p.v_stride))
     return BSA_ERR_UNSUPPORTED;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   uint8_t *w = static_cast<uint8_t *>(ws);
@@ -373,8 +375,8 @@ bsa_status bsa_attn_bwd(const bsa_problem *prob, const bsa_mask_spec *mask,
   const bsa_problem &p = P.p;
   CUtensorMap tq, tk, tv, tdo;
   if (!make_map(&tq, q, p.B, p.Sq, p.H, p.D, p.q_stride) ||
-      !make_map(&tk, k, p.B, p.Skv, p.H, p.D, p.k_stride) ||
-      !make_map(&tv, v, p.B, p.Skv, p.H, p.D, p.v_stride) ||
+      !make_map(&tk, k, p.B, p.Skv, p.H_kv, p.D, p.k_stride) ||
+      !make_map(&tv, v, p.B, p.Skv, p.H_kv, p.D, p.v_stride) ||
       !make_map(&tdo, dout, p.B, p.Sq, p.H, p.D, p.o_stride))
     return BSA_ERR_UNSUPPORTED;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -433,8 +435,8 @@ bsa_status bsa_bwd_main(const bsa_problem *prob, const bsa_mask_spec *mask,
   const bsa_problem &p = P.p;
   CUtensorMap tq, tk, tv, tdo;
   if (!make_map(&tq, q, p.B, p.Sq, p.H, p.D, p.q_stride) ||
-      !make_map(&tk, k, p.B, p.Skv, p.H, p.D, p.k_stride) ||
-      !make_map(&tv, v, p.B, p.Skv, p.H, p.D, p.v_stride) ||
+      !make_map(&tk, k, p.B, p.Skv, p.H_kv, p.D, p.k_stride) ||
+      !make_map(&tv, v, p.B, p.Skv, p.H_kv, p.D, p.v_stride) ||
       !make_map(&tdo, dout, p.B, p.Sq, p.H, p.D, p.o_stride))
     return BSA_ERR_UNSUPPORTED;
   uint8_t *w = static_cast<uint8_t *>(ws);

@@ -1,7 +1,7 @@
 // Backward pass (steps a4, a5 and a7 of the hot path).
 //
 // a4  preprocess: Delta_i = sum_d dO_id O_id (fp32) for every query row.
-// a5  main loop per kv column n (CTA = (b, h, n)): K_n and V_n stay in shared
+// a5  main loop per kv column n (CTA = (b, kv head, n)): K_n and V_n stay in shared
 //     memory; for each q-block m of the column's rank-sorted list the CTA
 //     recomputes S^T = K_n Q_m^T and dP^T = V_n dO_m^T, forms
 //     P^T = exp(S^T - LSE) (masked on PARTIAL tiles) and dS^T = P^T o (dP^T - Delta),
@@ -15,6 +15,9 @@
 //     only ever waits on columns that some running CTA already holds.
 // a7  convert: dQ = bf16(dQ accumulator).
 //
+// Grouped-query attention: a ticket is a kv column of one kv head; the CTA
+// walks the column's list once per query head of the group, so dK_n and dV_n
+// sum the group's contributions in TMEM and are written once.
 // sm_100a roles (384 threads, one CTA per SM, persistent over tickets):
 //   warp 0      ticket + TMA producer (K_n, V_n once per column; Q_m, dO_m per entry)
 //   warp 1      TMEM owner and tcgen05.mma issuer (one lane)
@@ -39,6 +42,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 struct BwdParams {
   MaskParams mask;
   int B, H, Sq, Skv, nM, nN, n_tickets;
+  int H_kv, kv_group;  // key/value heads; query heads per kv head
   float scale, scale_log2;
   const int32_t *col_ptr;
   const uint32_t *col_ent;
@@ -108,22 +112,30 @@ __device__ bool sem_wait(const uint32_t *sem, uint32_t target, uint64_t limit_ns
   }
 }
 
+// A ticket is one kv column n of one (b, kv head hk).  Its work is the
+// column's entry list once per query head of the group (h0 .. h0+g-1), walked
+// as one flat sequence x = 0 .. tot-1: query head h0 + x / len, entry
+// es + x % len.  dK_n and dV_n accumulate over the whole sequence.
 struct Ticket {
-  int valid, b, h, n, bh, es, ee;
+  int valid, b, hk, h0, n, es, ee, len, tot;
+  __device__ __forceinline__ int entry(int x) const { return es + x % len; }
+  __device__ __forceinline__ int head(int x) const { return h0 + x / len; }
 };
 
 __device__ __forceinline__ Ticket decode_ticket(const BwdParams &p, int t) {
   Ticket k{};
   if (t < 0 || t >= p.n_tickets) return k;
-  const int BH = p.B * p.H;
-  const int pos = t / BH, bh = t % BH;
+  const int BHk = p.B * p.H_kv;
+  const int pos = t / BHk, bhk = t % BHk;
   k.valid = 1;
-  k.bh = bh;
-  k.b = bh / p.H;
-  k.h = bh % p.H;
+  k.b = bhk / p.H_kv;
+  k.hk = bhk % p.H_kv;
+  k.h0 = k.hk * p.kv_group;
   k.n = p.perm[pos];
   k.es = p.col_ptr[k.b * p.nN + k.n];
   k.ee = p.col_ptr[k.b * p.nN + k.n + 1];
+  k.len = k.ee - k.es;
+  k.tot = k.len * p.kv_group;
   return k;
 }
 
@@ -203,25 +215,26 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
         if (!k.valid) break;
         if (k.ee == k.es) continue;
         bool stop = false;
-        for (int e = k.es; e < k.ee; ++e, ++ec) {
+        for (int x = 0; x < k.tot; ++x, ++ec) {
+          const int e = k.entry(x), h = k.head(x);
           const int m = static_cast<int>(p.col_ent[e] & kIndexMask);
           const uint32_t qs = ec % NQ, ds = ec % NDO;
           if (ec >= NQ && !wd.wait(&bars[L::bQEmpty + qs], ((ec / NQ) - 1) & 1)) { stop = true; break; }
           mbar_arrive_expect_tx(&bars[L::bQFull + qs], kTB);
           for (int c = 0; c < D / 64; ++c)
             tma_load_4d(sm + L::kQ + qs * kTB + c * 16384, &tq, &bars[L::bQFull + qs], c * 64,
-                        m * kTile, k.h, k.b);
+                        m * kTile, h, k.b);
           ++q_issued;
-          if (e == k.es) {
+          if (x == 0) {
             // K_n, V_n after the first Q so that load overlaps the previous
             // column's last MMAs
             if (cc >= 1 && !wd.wait(&bars[L::bKVFree], (cc - 1) & 1)) { stop = true; break; }
             mbar_arrive_expect_tx(&bars[L::bKVFull], 2 * kTB);
             for (int c = 0; c < D / 64; ++c) {
               tma_load_4d(sm + L::kK + c * 16384, &tk, &bars[L::bKVFull], c * 64, k.n * kTile,
-                          k.h, k.b);
+                          k.hk, k.b);
               tma_load_4d(sm + L::kV + c * 16384, &tv, &bars[L::bKVFull], c * 64, k.n * kTile,
-                          k.h, k.b);
+                          k.hk, k.b);
             }
             ++kv_issued;
           }
@@ -229,7 +242,7 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
           mbar_arrive_expect_tx(&bars[L::bDOFull + ds], kTB);
           for (int c = 0; c < D / 64; ++c)
             tma_load_4d(sm + L::kDO + ds * kTB + c * 16384, &tdo, &bars[L::bDOFull + ds], c * 64,
-                        m * kTile, k.h, k.b);
+                        m * kTile, h, k.b);
           ++do_issued;
         }
         if (stop) break;
@@ -293,9 +306,9 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
         if (k.ee == k.es) continue;
         if (!wd.wait(&bars[L::bKVFull], cc & 1)) break;
         bool stop = !issue_s(ec) || !issue_dp(ec);
-        for (int e = k.es; e < k.ee && !stop; ++e, ++ec) {
+        for (int x = 0; x < k.tot && !stop; ++x, ++ec) {
           const uint32_t qs = ec % NQ, ds = ec % NDO;
-          const bool first = e == k.es, last = e == k.ee - 1;
+          const bool first = x == 0, last = x == k.tot - 1;
           if (!wd.wait(&bars[L::bPReady], ec & 1)) { stop = true; break; }
           if (first && cc >= 1 && !wd.wait(&bars[L::bDKVFree], (cc - 1) & 1)) { stop = true; break; }
           tc_fence_after();
@@ -364,8 +377,8 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       const bool row_ok = j < p.Skv;
       if (k.ee == k.es) {
         if (row_ok) {
-          __nv_bfloat16 *dk_row = p.dk + k.b * p.k_sb + static_cast<int64_t>(j) * p.k_ss + k.h * p.k_sh;
-          __nv_bfloat16 *dv_row = p.dv + k.b * p.v_sb + static_cast<int64_t>(j) * p.v_ss + k.h * p.v_sh;
+          __nv_bfloat16 *dk_row = p.dk + k.b * p.k_sb + static_cast<int64_t>(j) * p.k_ss + k.hk * p.k_sh;
+          __nv_bfloat16 *dv_row = p.dv + k.b * p.v_sb + static_cast<int64_t>(j) * p.v_ss + k.hk * p.v_sh;
           const int4 z = make_int4(0, 0, 0, 0);
 #pragma unroll
           for (int c = 0; c < D / 8; ++c) {
@@ -388,7 +401,9 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       if ((mk.flags & BSA_MASK_KV_VALID_LEN) && j >= mk.kv_valid_len[k.b]) qhi = -1;
       const int seg_j = (use_seg && row_ok) ? mk.seg_kv[static_cast<int64_t>(k.b) * p.Skv + j] : INT_MIN;
       uint8_t *ds_tile = sm + L::kDS;
-      for (int e = k.es; e < k.ee; ++e, ++ec) {
+      for (int x = 0; x < k.tot; ++x, ++ec) {
+        const int e = k.entry(x);
+        const int64_t bh = static_cast<int64_t>(k.b) * p.H + k.head(x);
         const uint32_t ent = p.col_ent[e];
         const int m = static_cast<int>(ent & kIndexMask);
         const bool full = (ent & kFullBit) != 0;
@@ -399,11 +414,11 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
           const int i = m * kTile + r;
           float nl2 = -INFINITY;
           if (i < p.Sq) {
-            const float lv = p.lse[static_cast<int64_t>(k.bh) * p.Sq + i];
+            const float lv = p.lse[bh * p.Sq + i];
             if (lv != -INFINITY) nl2 = -lv * kLog2e;
           }
           vec_nl[(ec & 1) * kTile + r] = nl2;
-          vec_nd[(ec & 1) * kTile + r] = -p.delta[static_cast<int64_t>(k.bh) * p.nM * kTile + i];
+          vec_nd[(ec & 1) * kTile + r] = -p.delta[bh * p.nM * kTile + i];
           mbar_arrive(&bars[L::bVecReady + (ec & 1)]);
         }
         // allowed-query bits of this tile for this key row (range AND segment
@@ -443,13 +458,15 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
         const float4 *nl4p = reinterpret_cast<const float4 *>(vec_nl + (ec & 1) * kTile);
         const float4 *nd4p = reinterpret_cast<const float4 *>(vec_nd + (ec & 1) * kTile);
         // phase 1: P^T = exp2(S^T * scale * log2e - LSE*log2e) -> bf16 in TMEM
-        // (over the first 64 S^T columns) and kept packed in registers
+        // (over the first 64 S^T columns, the A operand of dV) and kept in
+        // registers as fp16 pairs for dS: P lies in [0, 1], where fp16 keeps 11
+        // significant bits to bf16's 8, so dS carries no extra rounding of P
         if (!wwait(&bars[L::bSFull], ec & 1)) { stop = true; break; }
         tc_fence_after();
         uint32_t pk[64];
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          uint32_t s[32];
+          uint32_t s[32], pb[16];
           tmem_ld32(T_S + lane_off + 32 * c, s);
           tmem_wait_ld();
 #pragma unroll
@@ -466,18 +483,18 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
                 p0 = ((allow[c] >> e0) & 1u) ? p0 : 0.f;
                 p1 = ((allow[c] >> (e0 + 1)) & 1u) ? p1 : 0.f;
               }
-              pk[16 * c + (e0 >> 1)] = pack_bf16x2(p0, p1);
+              pb[e0 >> 1] = pack_bf16x2(p0, p1);
+              pk[16 * c + (e0 >> 1)] = pack_f16x2(p0, p1);
             }
           }
           // P^T chunk -> TMEM columns [16c, 16c+16): only S^T columns already read
-          tmem_st16(T_S + lane_off + 16 * c,
-                    *reinterpret_cast<const uint32_t(*)[16]>(&pk[16 * c]));
+          tmem_st16(T_S + lane_off + 16 * c, pb);
         }
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&bars[L::bPReady]);
-        // phase 2: dS^T = P^T o (dP^T - Delta), with the bf16 P^T the dV product
-        // uses, -> bf16 shared tile (128-byte swizzle, K-major)
+        // phase 2: dS^T = P^T o (dP^T - Delta) in fp32 from the fp16 P^T -> bf16
+        // shared tile (128-byte swizzle, K-major)
         if (ec >= 1 && !wwait(&bars[L::bDSFree], (ec - 1) & 1)) { stop = true; break; }
         if (!wwait(&bars[L::bDPFull], ec & 1)) { stop = true; break; }
         tc_fence_after();
@@ -495,7 +512,7 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
               const int e0 = 4 * q4 + 2 * h2;
               const float2 nd = h2 ? make_float2(nd4.z, nd4.w) : make_float2(nd4.x, nd4.y);
               const uint32_t pp = pk[16 * c + (e0 >> 1)];
-              const float2 pv = make_float2(__uint_as_float(pp << 16), __uint_as_float(pp & 0xffff0000u));
+              const float2 pv = unpack_f16x2(pp);
               const float2 dd = __fadd2_rn(
                   make_float2(__uint_as_float(dp[e0]), __uint_as_float(dp[e0 + 1])), nd);
               const float2 dsv = __fmul2_rn(pv, dd);
@@ -519,8 +536,8 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       // epilogue: dV, dK (scaled) -> bf16
       if (!wwait(&bars[L::bDKVFull], cc & 1)) break;
       tc_fence_after();
-      __nv_bfloat16 *dk_row = p.dk + k.b * p.k_sb + static_cast<int64_t>(j) * p.k_ss + k.h * p.k_sh;
-      __nv_bfloat16 *dv_row = p.dv + k.b * p.v_sb + static_cast<int64_t>(j) * p.v_ss + k.h * p.v_sh;
+      __nv_bfloat16 *dk_row = p.dk + k.b * p.k_sb + static_cast<int64_t>(j) * p.k_ss + k.hk * p.k_sh;
+      __nv_bfloat16 *dv_row = p.dv + k.b * p.v_sb + static_cast<int64_t>(j) * p.v_ss + k.hk * p.v_sh;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t a[32], g[32];
@@ -566,7 +583,9 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       const Ticket k = decode_ticket(p, t);
       if (!k.valid) break;
       bool stop = false;
-      for (int e = k.es; e < k.ee; ++e, ++ec) {
+      for (int x = 0; x < k.tot; ++x, ++ec) {
+        const int e = k.entry(x);
+        const int64_t bh = static_cast<int64_t>(k.b) * p.H + k.head(x);
         const int m = static_cast<int>(p.col_ent[e] & kIndexMask);
         const uint32_t rank = static_cast<uint32_t>(p.col_rank[e]);
         if (!wwait(&bars[L::bDQFull], ec & 1)) { stop = true; break; }
@@ -582,14 +601,14 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
         }
         tc_fence_before();
         mbar_arrive(&bars[L::bDQFree]);
-        uint32_t *sem = p.sem + static_cast<int64_t>(k.bh) * p.nM + m;
+        uint32_t *sem = p.sem + bh * p.nM + m;
         int ok = 1;
         if (p.deterministic) {
           if (lane == 0) ok = sem_wait(sem, rank, p.sem_timeout_ns, p.hdr + kHdrStatus) ? 1 : 0;
           ok = __shfl_sync(0xffffffffu, ok, 0);
         }
         if (ok) {
-          float *base = p.dq_accum + (static_cast<int64_t>(k.bh) * p.nM + m) * (D / 4) * (kTile * 4);
+          float *base = p.dq_accum + (bh * p.nM + m) * (D / 4) * (kTile * 4);
           if (p.deterministic && rank == 0) {
             // the first contributor in the order pi initialises the accumulator
             // rows, so the deterministic path needs no zeroing pass
@@ -783,7 +802,9 @@ cudaError_t launch_bwd_main(const bsa_problem &p, const MaskParams &mp, const bs
   bp.Skv = p.Skv;
   bp.nM = L.nM;
   bp.nN = L.nN;
-  bp.n_tickets = p.B * p.H * L.nN;
+  bp.H_kv = p.H_kv;
+  bp.kv_group = p.H / p.H_kv;
+  bp.n_tickets = p.B * p.H_kv * L.nN;
   bp.scale = p.scale;
   bp.scale_log2 = p.scale * kLog2e;
   bp.col_ptr = reinterpret_cast<const int32_t *>(ws + L.col_ptr);

@@ -14,7 +14,8 @@
 //
 // sm_100a design: one CTA per SM, persistent over work units = pairs of
 // q-blocks (A = 2g, B = 2g+1) of one (b, h).  The CTA walks the union of the
-// two row lists, so each K/V tile is loaded once for both q-blocks.
+// two row lists, so each K/V tile is loaded once for both q-blocks.  With
+// grouped-query attention head h reads the K/V of kv head h / (H / H_kv).
 //   warp 0      TMA producer: Q_A, Q_B once per unit; K and V tiles through
 //               separate stage rings, 128-byte swizzled 64 x 128 boxes.
 //   warp 1      owns TMEM (512 columns) and issues tcgen05.mma from one lane,
@@ -44,6 +45,7 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units: tolerate p up to 2^8
 struct FwdParams {
   MaskParams mask;
   int B, H, Sq, Skv, nM, n_units;
+  int kv_group;  // query heads per key/value head (grouped-query attention)
   float scale, scale_log2;
   const int32_t *row_ptr;
   const uint32_t *row_ent;
@@ -213,13 +215,13 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
           mbar_arrive_expect_tx(&bars[L::bKFull + ks], kTB);
           for (int c = 0; c < D / 64; ++c)
             tma_load_4d(sm + L::kK + ks * kTB + c * 16384, &tk, &bars[L::bKFull + ks], c * 64,
-                        n * kTile, w.h, w.b);
+                        n * kTile, w.h / p.kv_group, w.b);
           ++k_issued;
           if (kv >= NV && !wd.wait(&bars[L::bVEmpty + vs], ((kv / NV) - 1) & 1)) { stop = true; break; }
           mbar_arrive_expect_tx(&bars[L::bVFull + vs], kTB);
           for (int c = 0; c < D / 64; ++c)
             tma_load_4d(sm + L::kV + vs * kTB + c * 16384, &tv, &bars[L::bVFull + vs], c * 64,
-                        n * kTile, w.h, w.b);
+                        n * kTile, w.h / p.kv_group, w.b);
           ++v_issued;
           ++kv;
         }
@@ -543,7 +545,7 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
 struct NormArgs {
   const __nv_bfloat16 *k, *q;
   int64_t ks[3], qs[3];
-  int B, Skv, Sq, H, only_q, center;
+  int B, Skv, Sq, H, Hk, only_q, center;  // Hk: key heads (H / Hk query heads each)
   MaskParams mk;
   float *kmax, *qmax, *qnorm;
   long long *ksum;        // [B, H, D] fixed-point sums of the valid keys
@@ -578,7 +580,7 @@ __global__ void __launch_bounds__(256) k_key_sums(const NormArgs a) {
     for (int r = r0; r < r1; ++r) n += key_is_valid(a.mk, b, r) ? 1 : 0;
     if (n != 0) atomicAdd(a.kcount + b, n);
   }
-  const int cols = a.H * G;
+  const int cols = a.Hk * G;
   for (int c = threadIdx.x; c < cols; c += blockDim.x) {
     const int h = c / G, g = c % G;
     long long acc[8];
@@ -598,7 +600,7 @@ __global__ void __launch_bounds__(256) k_key_sums(const NormArgs a) {
       }
     }
     unsigned long long *dst = reinterpret_cast<unsigned long long *>(
-        a.ksum + (static_cast<int64_t>(b) * a.H + h) * D + g * 8);
+        a.ksum + (static_cast<int64_t>(b) * a.Hk + h) * D + g * 8);
 #pragma unroll
     for (int e = 0; e < 8; ++e)
       if (acc[e] != 0) atomicAdd(dst + e, static_cast<unsigned long long>(acc[e]));
@@ -619,6 +621,8 @@ __global__ void __launch_bounds__(256) k_row_norms(const NormArgs a) {
                 sh = is_key ? a.ks[2] : a.qs[2];
   float *rowmax = is_key ? a.kmax : a.qmax;
   const int H = a.H, Sq = a.Sq, Skv = a.Skv;
+  const int Hx = is_key ? a.Hk : H;  // heads of this tensor
+  const int grp = H / a.Hk;          // query heads per key head
   const MaskParams &mk = a.mk;
   float *qnorm = a.qnorm;
   const int64_t blocks_per_b = (max(Sq, Skv) + kRows - 1) / kRows;
@@ -629,18 +633,18 @@ __global__ void __launch_bounds__(256) k_row_norms(const NormArgs a) {
   if (a.center) {
     // c = (fixed-point sum) * 2^-20 / (valid keys), the same in every block
     const double inv = 1.0 / (static_cast<double>(kFixScale) * max(1, a.kcount[b]));
-    const long long *ks = a.ksum + static_cast<int64_t>(b) * H * D;
+    const long long *ks = a.ksum + static_cast<int64_t>(b) * a.Hk * D;
     const bool write = is_key && r0 == 0;
-    for (int t = threadIdx.x; t < H * D; t += blockDim.x) {
+    for (int t = threadIdx.x; t < a.Hk * D; t += blockDim.x) {
       const float c = static_cast<float>(static_cast<double>(ks[t]) * inv);
       cen[t] = c;
-      if (write) a.kbar[static_cast<int64_t>(b) * H * D + t] = c;
+      if (write) a.kbar[static_cast<int64_t>(b) * a.Hk * D + t] = c;
     }
   }
   __syncthreads();
   const int g = threadIdx.x / TPV, t = threadIdx.x % TPV;
   const int groups = blockDim.x / TPV;
-  const int pairs = kRows * H;
+  const int pairs = kRows * Hx;
   // uniform trip count across the warp: the shuffles below need every lane
   for (int base = 0; base < pairs; base += groups * kUnroll) {
     float acc[kUnroll], dot[kUnroll];
@@ -649,8 +653,8 @@ __global__ void __launch_bounds__(256) k_row_norms(const NormArgs a) {
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
       const int pair = base + u * groups + g;
-      row[u] = r0 + pair / H;
-      hh[u] = pair % H;
+      row[u] = r0 + pair / Hx;
+      hh[u] = pair % Hx;
       in[u] = pair < pairs && row[u] < S;
       acc[u] = 0.f;
       dot[u] = 0.f;
@@ -658,7 +662,7 @@ __global__ void __launch_bounds__(256) k_row_norms(const NormArgs a) {
         const int4 v = *reinterpret_cast<const int4 *>(x + b * sb + static_cast<int64_t>(row[u]) * ss +
                                                       hh[u] * sh + t * 8);
         const __nv_bfloat162 *e = reinterpret_cast<const __nv_bfloat162 *>(&v);
-        const float *c = cen + hh[u] * D + t * 8;
+        const float *c = cen + (is_key ? hh[u] : hh[u] / grp) * D + t * 8;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           float2 f = __bfloat1622float2(e[q]);
@@ -698,8 +702,16 @@ __global__ void __launch_bounds__(256) k_row_norms(const NormArgs a) {
     }
   }
   __syncthreads();
-  for (int h = threadIdx.x; h < H; h += blockDim.x)
-    if (smax[h] != 0u) atomicMax(reinterpret_cast<unsigned int *>(rowmax) + b * H + h, smax[h]);
+  // a key head's maximum goes to every query head of its group
+  for (int h = threadIdx.x; h < Hx; h += blockDim.x)
+    if (smax[h] != 0u) {
+      if (is_key) {
+        for (int i = 0; i < grp; ++i)
+          atomicMax(reinterpret_cast<unsigned int *>(rowmax) + b * H + h * grp + i, smax[h]);
+      } else {
+        atomicMax(reinterpret_cast<unsigned int *>(rowmax) + b * H + h, smax[h]);
+      }
+    }
 }
 
 __global__ void k_gate(int BH, float scale, float limit, const float *kmax_override,
@@ -756,6 +768,7 @@ cudaError_t launch_fixed_m_bound(const bsa_problem &p, const MaskParams &mp,
   na.Skv = p.Skv;
   na.Sq = p.Sq;
   na.H = p.H;
+  na.Hk = p.H_kv;
   na.only_q = o.kmax_override != nullptr;  // a caller-supplied kmax needs no key pass
   na.center = o.bound_mode == BSA_BOUND_SMOOTHED;
   na.mk = mp;
@@ -777,7 +790,7 @@ cudaError_t launch_fixed_m_bound(const bsa_problem &p, const MaskParams &mp,
     if (p.D == 64) k_key_sums<64><<<sblocks, 256, 0, s>>>(na);
     else k_key_sums<128><<<sblocks, 256, 0, s>>>(na);
     count_launch();
-    smem += sizeof(float) * p.H * p.D;
+    smem += sizeof(float) * p.H_kv * p.D;
   }
   const int64_t blocks = static_cast<int64_t>(p.B) * ((std::max(p.Sq, p.Skv) + 31) / 32);
   const dim3 grid(static_cast<unsigned>(blocks), na.only_q ? 1u : 2u);
@@ -810,6 +823,7 @@ cudaError_t launch_fwd(const bsa_problem &p, const MaskParams &mp, const bsa_opt
   fp.Sq = p.Sq;
   fp.Skv = p.Skv;
   fp.nM = L.nM;
+  fp.kv_group = p.H / p.H_kv;
   fp.n_units = p.B * p.H * ((L.nM + 1) / 2);
   fp.scale = p.scale;
   fp.scale_log2 = p.scale * kLog2e;

@@ -28,6 +28,12 @@ at its 8192x8192 shape and the sliding-window workload's B, H, D and seed
 ``document``   document-causal: segment ids from runs of uniform{256..2048}
                tokens, causal inside each document.
 
+And one grouped-query shape (the benchmark's "kv_mode" column is MHA in every
+row; the grouping is this build's reading):
+
+``gqa``        B=1, H=16 query heads over H_kv=4 key/value heads, Sq=Skv=8192,
+               D=128, causal sliding window of 512 keys, N(0,1), seed 5.
+
 ``small=True`` shrinks the sequence lengths (same structure, same recipe) so the
 fp64 oracle finishes in seconds; the parity tests use it for the full-oracle
 comparison and sample rows at full size.
@@ -79,7 +85,7 @@ class Workload:
 
 
 WORKLOADS = ("tiny", "packed", "packed_const", "window", "window_rect", "varlen", "video",
-             "prefix_lm", "dilated", "document")
+             "prefix_lm", "dilated", "document", "gqa")
 
 
 def _normal(shape, gen, device, std=1.0):
@@ -193,6 +199,18 @@ def make_workload(name: str, device="cpu", small: bool = False, seed: Optional[i
             seg = torch.from_numpy(np.stack([_segment_runs(rng, S, lo, hi) for _ in range(B)])).to(dev)
             mask = {"seg_q": seg, "seg_kv": seg.clone(), "window": 0}
         return Workload(name, B, H, S, S, D, q, k, v, dO, mask, 1.0 / math.sqrt(D))
+
+    if name == "gqa":
+        sd = 5 if seed is None else seed
+        B, H, H_kv, D, S, W = 1, 16, 4, 128, 8192, 512
+        if small:
+            H, H_kv, S, W = 4, 2, 1000, 256
+        g = gen_for(sd)
+        q = _normal((B, S, H, D), g, dev).to(bf16)
+        k = _normal((B, S, H_kv, D), g, dev).to(bf16)
+        v = _normal((B, S, H_kv, D), g, dev).to(bf16)
+        dO = _normal((B, S, H, D), g, dev).to(bf16)
+        return Workload(name, B, H, S, S, D, q, k, v, dO, {"window": W}, 1.0 / math.sqrt(D))
 
     if name == "varlen":
         sd = 3 if seed is None else seed

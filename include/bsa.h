@@ -128,11 +128,14 @@ typedef enum bsa_status {
 
 typedef struct bsa_problem {
   int32_t B;       /* batch; 1 for varlen                                        */
-  int32_t H;       /* heads (Q, K and V have the same head count)                */
+  int32_t H;       /* query heads (Q, O, LSE, dQ, dO)                            */
   int32_t Sq;      /* query rows per batch (varlen: total tokens T); <= 2^21      */
   int32_t Skv;     /* keys per batch (varlen: T); <= 2^21                         */
   int32_t D;       /* head dim, 64 or 128                                         */
-  int32_t reserved0;
+  int32_t H_kv;    /* key/value heads (K, V, dK, dV); 0 = H.  H must be a multiple:
+                      query head h reads kv head h / (H / H_kv) (grouped-query
+                      attention; H_kv = 1 is multi-query).  dK and dV of a kv
+                      head are summed over the query heads of its group.        */
   /* element strides (batch, seq, head); all zero = contiguous BSHD.  q_stride
    * is used for Q and dQ, k_stride for K and dK, v_stride for V and dV,
    * o_stride for O and dO. */
@@ -178,7 +181,7 @@ typedef struct bsa_options {
                                   kmax/qmax/gate from bsa_fixed_m_bound for these
                                   q and k; 0: bsa_attn_fwd computes them first      */
   int32_t bound_mode;          /* BSA_BOUND_*; SMOOTHED with kmax_override or with
-                                  H*D > 24576 is rejected                           */
+                                  H_kv*D > 24576 is rejected                        */
   int32_t reserved;
 } bsa_options;
 
@@ -202,7 +205,7 @@ typedef struct bsa_workspace_view {
   size_t off_delta;            /* fp32   [B, H, nM*128]  backward Delta              */
   size_t off_dq_accum;         /* fp32   backward dQ accumulator                     */
   size_t off_sem;              /* int32  [B, H, nM]   dQ semaphores                  */
-  size_t off_kbar;             /* fp32   [B, H, D]    k-smoothing center             */
+  size_t off_kbar;             /* fp32   [B, H_kv, D] k-smoothing center             */
   size_t off_qdot;             /* fp32   [B, H, Sq]   q_i . center                   */
   int32_t nM, nN;
 } bsa_workspace_view;

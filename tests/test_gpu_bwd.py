@@ -22,9 +22,13 @@ def _grads(wl, **kw):
 
 
 def _oracle_grads(wl, heads=None):
+    """Oracle gradients; ``heads`` (query heads) must cover whole kv-head groups."""
     q, k, v, do = np64(wl.q), np64(wl.k), np64(wl.v), np64(wl.dO)
     if heads is not None:
-        q, k, v, do = q[:, :, heads], k[:, :, heads], v[:, :, heads], do[:, :, heads]
+        g = wl.H // wl.k.shape[2]
+        kvh = sorted({h // g for h in heads})
+        q, do = q[:, :, heads], do[:, :, heads]
+        k, v = k[:, :, kvh], v[:, :, kvh]
     return oracle.attention_backward(q, k, v, do, mask_desc(wl), wl.scale)
 
 
@@ -36,7 +40,8 @@ def _err(x, ref):
     return min(raw, O_TOL)
 
 
-SMALL = ["tiny", "packed", "window", "window_rect", "varlen", "video", "prefix_lm", "dilated", "document"]
+SMALL = ["tiny", "packed", "window", "window_rect", "varlen", "video", "prefix_lm", "dilated", "document",
+         "gqa"]
 
 
 @pytest.mark.parametrize("name", SMALL)
@@ -78,6 +83,29 @@ def test_bwd_orders_match_oracle_and_repeat_bitwise(order):
         assert torch.equal(dq, dq2) and torch.equal(dk, dk2) and torch.equal(dv, dv2)
 
 
+def test_gqa_bwd_dq_equals_mha_with_repeated_kv_and_dkv_sum_the_group():
+    # dQ: the same per-head contributions added in the same order pi -> equal
+    # bits.  dK/dV of a kv head: the group's sum, accumulated in fp32 before
+    # one rounding, against the bf16 sum of the per-head MHA gradients.
+    wl = make_workload("gqa", device="cuda", small=True)
+    g = wl.H // wl.k.shape[2]
+    o, lse, dq, dk, dv, ws = _grads(wl)
+    assert ws.status() == 0
+    kr = wl.k.repeat_interleave(g, dim=2).contiguous()
+    vr = wl.v.repeat_interleave(g, dim=2).contiguous()
+    dq2, dk2, dv2, ws2 = bsa.attn_bwd(wl.q, kr, vr, o, wl.dO, lse, wl.mask)
+    torch.cuda.synchronize()
+    assert ws2.status() == 0
+    assert torch.equal(dq, dq2)
+    B, S, Hk, D = wl.k.shape
+    sk = dk2.float().view(B, S, Hk, g, D).sum(3)
+    sv = dv2.float().view(B, S, Hk, g, D).sum(3)
+    assert (dk.float() - sk).abs().max().item() <= 2 * O_TOL
+    assert (dv.float() - sv).abs().max().item() <= 2 * O_TOL
+    gq, gk, gv = _oracle_grads(wl)
+    assert max(_err(dq, gq), _err(dk, gk), _err(dv, gv)) <= O_TOL
+
+
 def test_bwd_nondeterministic_matches_oracle():
     wl = make_workload("packed", device="cuda", small=True)
     _, _, dq, dk, dv, ws = _grads(wl, deterministic=False)
@@ -114,7 +142,7 @@ def test_bwd_ragged_and_d64():
         assert max(_err(dq, gq), _err(dk, gk), _err(dv, gv)) <= O_TOL, (Sq, Skv, D, W)
 
 
-@pytest.mark.parametrize("name", ["window", "window_rect", "prefix_lm", "dilated", "document"])
+@pytest.mark.parametrize("name", ["window", "window_rect", "prefix_lm", "dilated", "document", "gqa"])
 def test_bwd_full_size_one_head_and_ten_run_identity(name):
     wl = make_workload(name, device="cuda")
     o, lse, ws = bsa.attn_fwd(wl.q, wl.k, wl.v, wl.mask)
@@ -127,8 +155,9 @@ def test_bwd_full_size_one_head_and_ten_run_identity(name):
             assert wsb.status() == 0
         else:
             assert all(torch.equal(x, y) for x, y in zip(ref, (dq, dk, dv)))
-    gq, gk, gv = _oracle_grads(wl, heads=[0])
-    assert _err(ref[0][:, :, [0]], gq) <= O_TOL
+    g = wl.H // wl.k.shape[2]
+    gq, gk, gv = _oracle_grads(wl, heads=list(range(g)))  # kv head 0 and its query heads
+    assert _err(ref[0][:, :, :g], gq) <= O_TOL
     assert _err(ref[1][:, :, [0]], gk) <= O_TOL
     assert _err(ref[2][:, :, [0]], gv) <= O_TOL
 

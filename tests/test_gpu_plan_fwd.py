@@ -12,7 +12,7 @@ from tests.gpu_common import LSE_TOL, O_TOL, compare_lse, compare_out, mask_desc
 pytestmark = pytest.mark.gpu
 
 SMALL = ["tiny", "packed", "packed_const", "window", "window_rect", "varlen", "video", "prefix_lm",
-         "dilated", "document"]
+         "dilated", "document", "gqa"]
 
 
 @pytest.mark.parametrize("name", SMALL)
@@ -161,6 +161,34 @@ def test_smoothing_widens_the_gate_and_stays_exact_and_deterministic():
     assert (o - o3).abs().max().item() <= O_TOL
     fin = torch.isfinite(l3)
     assert (lse[fin] - l3[fin]).abs().max().item() <= LSE_TOL
+
+
+@pytest.mark.parametrize("mode", ["online", "fixed_m"])
+def test_gqa_forward_equals_mha_with_repeated_kv_bitwise(mode):
+    wl = make_workload("gqa", device="cuda", small=True)
+    g = wl.H // wl.k.shape[2]
+    o1, l1, _ = bsa.attn_fwd(wl.q, wl.k, wl.v, wl.mask, softmax_mode=mode)
+    kr = wl.k.repeat_interleave(g, dim=2).contiguous()
+    vr = wl.v.repeat_interleave(g, dim=2).contiguous()
+    o2, l2, _ = bsa.attn_fwd(wl.q, kr, vr, wl.mask, softmax_mode=mode)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_gqa_full_size_sampled_rows():
+    wl = make_workload("gqa", device="cuda")
+    g = wl.H // wl.k.shape[2]
+    rows = sample_rows(wl.Sq, seed=3)
+    heads = [0, wl.H - 1]
+    o, lse, ws = bsa.attn_fwd(wl.q, wl.k, wl.v, wl.mask, softmax_mode="fixed_m")
+    torch.cuda.synchronize()
+    assert ws.status() == 0
+    kvh = [h // g for h in heads]
+    q, k, v = np64(wl.q[:, :, heads]), np64(wl.k[:, :, kvh]), np64(wl.v[:, :, kvh])
+    O_ref, L_ref = oracle.attention_forward(q, k, v, mask_desc(wl), wl.scale, rows=rows)
+    assert compare_out(o[:, :, heads], O_ref, rows) <= O_TOL
+    el, same = compare_lse(lse[:, heads], L_ref, rows)
+    assert el <= LSE_TOL and same
 
 
 def test_fixed_m_and_online_agree_bitwise_on_fallback_head():
