@@ -18,16 +18,17 @@
 // Grouped-query attention: a ticket is a kv column of one kv head; the CTA
 // walks the column's list once per query head of the group, so dK_n and dV_n
 // sum the group's contributions in TMEM and are written once.
-// sm_100a roles (384 threads, one CTA per SM, persistent over tickets):
+// sm_100a roles (512 threads, one CTA per SM, persistent over tickets):
 //   warp 0      ticket + TMA producer (K_n, V_n once per column; Q_m, dO_m per entry)
 //   warp 1      TMEM owner and tcgen05.mma issuer (one lane)
-//   warps 4..7  compute: one key row per thread (TMEM lane), the 128-bit allowed-query
-//               mask of PARTIAL tiles (a prefix key is seen by every query; other
-//               keys by a query range thinned by the dilation, AND segment ids),
-//               P^T back to TMEM as the
+//   warps 4..11 compute: one key row per thread (TMEM lane) and half of the 128
+//               query columns per warp (two warps per lane quarter), the allowed-
+//               query mask of PARTIAL tiles (a prefix key is seen by every query;
+//               other keys by a query range thinned by the dilation, AND segment
+//               ids), P^T back to TMEM as the
 //               A operand of dV, dS^T to shared memory (128-byte swizzle, K-major
 //               for dK, read MN-major as the A operand of dQ), dK/dV epilogue
-//   warps 8..11 dQ: one query row per thread, semaphore wait, vector reductions
+//   warps 12..15 dQ: one query row per thread, semaphore wait, vector reductions
 // TMEM columns: S^T / P^T [0,128)  dP^T / dQ [128,256)  dV [256,256+D)  dK [256+D,256+2D)
 #include <cfloat>
 
@@ -83,7 +84,10 @@ struct BwdSmem {
   static constexpr int kAlloc = kMisc + 16;
 };
 
-constexpr int kConsumersPerTicket = 1 + 4 + 4;  // MMA lane, compute warps, dQ warps
+constexpr int kThreads = 512;
+constexpr int kLaunchRegs = 65536 / kThreads;  // 128: the whole register file
+constexpr int kConsumersPerTicket = 1 + 8 + 4;  // MMA lane, compute warps, dQ warps
+constexpr int kComputeThreads = 256;
 
 __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity) {
   const uint32_t a = smem_u32(bar);
@@ -140,7 +144,7 @@ __device__ __forceinline__ Ticket decode_ticket(const BwdParams &p, int t) {
 }
 
 template <int D, int NQ, int NDO>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(kThreads, 1)
 k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
            const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo,
            const BwdParams p) {
@@ -160,9 +164,10 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
     for (int i = 0; i < L::kNumBars; ++i) {
       uint32_t cnt = 1;
       if (i == L::bTkEmpty || i == L::bTkEmpty + 1) cnt = kConsumersPerTicket;
-      if (i == L::bPReady || i == L::bDSReady || i == L::bDQFree || i == L::bDKVFree ||
-          i == L::bVecReady || i == L::bVecReady + 1)
-        cnt = 128;
+      if (i == L::bPReady || i == L::bDSReady || i == L::bDKVFree || i == L::bVecReady ||
+          i == L::bVecReady + 1)
+        cnt = kComputeThreads;
+      if (i == L::bDQFree) cnt = 128;
       if (i == L::bDQAdded || i == L::bDQAdded + 1) cnt = 4;
       mbar_init(&bars[i], cnt);
     }
@@ -200,8 +205,14 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
   constexpr uint32_t kIdKV = idesc_bf16_f32(128, D, 0, 1);       // dV (TS), dK: B MN-major
   constexpr uint32_t kIdQ = idesc_bf16_f32(128, D, 1, 1);        // dQ: A and B MN-major
 
-  if (wd.aborted()) {
-  } else if (warp == 0) {
+  // register budgets, set first thing in each warpgroup's branch: 96 for the
+  // producer / MMA warpgroup, 128 for each compute warpgroup, 160 for the dQ
+  // warpgroup (its rows are 128 fp32 values each): 96 + 128 + 128 + 160 =
+  // 4 x 128, the launch's share
+  const bool run = !wd.aborted();
+  if (warp < 4) {
+    regs_dec<96>();
+    if (run && warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       uint32_t tc = 0, cc = 0, ec = 0, kv_issued = 0, q_issued = 0, do_issued = 0;
@@ -256,7 +267,7 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
         if (kv_issued > 0) drain_wait(&bars[L::bKVFull], (kv_issued - 1) & 1);
       }
     }
-  } else if (warp == 1) {
+    } else if (run && warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     // Per entry e: dV(e), S^T(e+1), dK(e), dQ(e), dP^T(e+1).  S^T(e+1) reuses the
     // columns dV(e) reads P^T from: tcgen05.mma ops issued by one thread run in
@@ -316,7 +327,7 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
           const uint32_t do_addr = smem_u32(sm + L::kDO + ds * kTB);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_ts(T_DV, T_S + kk * 8, sw128_desc(do_addr + kk * 2048, 16384, 1024), kIdKV,
+            mma_ts(T_DV, T_S + kk * 8 + (kk >= 4 ? 32 : 0), sw128_desc(do_addr + kk * 2048, 16384, 1024), kIdKV,
                    (!first || kk > 0) ? 1u : 0u);
           mma_commit(&bars[L::bDOEmpty + ds]);
           if (!last && !issue_s(ec + 1)) { stop = true; break; }
@@ -352,9 +363,13 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       mma_commit(&bars[L::bFinal]);
       drain_wait(&bars[L::bFinal], 0);
     }
-  } else if (warp >= 4 && warp < 8) {
+    }
+  } else if (warp < 12) {
+    if (run) {
     // ------------------------------------------------------------ compute (key rows)
-    const int quarter = warp & 3;
+    // two warps per TMEM lane quarter: `half` 0 takes query columns 0..63,
+    // half 1 columns 64..127 (and the matching halves of the dK/dV rows)
+    const int quarter = warp & 3, half = (warp - 4) >> 2;
     const int r = quarter * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const MaskParams &mk = p.mask;
@@ -363,6 +378,9 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       return __all_sync(0xffffffffu, wd.wait(bar, parity)) != 0;
     };
     const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
+    // this half's P^T columns in TMEM (read as the A operand of dV): inside its
+    // own S^T columns, which only this warp reads
+    const uint32_t t_p = T_S + lane_off + 64 * half;
     uint32_t tc = 0, cc = 0, ec = 0;
     bool stop = false;
     for (;; ++tc) {
@@ -381,7 +399,7 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
           __nv_bfloat16 *dv_row = p.dv + k.b * p.v_sb + static_cast<int64_t>(j) * p.v_ss + k.hk * p.v_sh;
           const int4 z = make_int4(0, 0, 0, 0);
 #pragma unroll
-          for (int c = 0; c < D / 8; ++c) {
+          for (int c = half * (D / 16); c < (half + 1) * (D / 16); ++c) {
             reinterpret_cast<int4 *>(dk_row)[c] = z;
             reinterpret_cast<int4 *>(dv_row)[c] = z;
           }
@@ -407,43 +425,47 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
         const uint32_t ent = p.col_ent[e];
         const int m = static_cast<int>(ent & kIndexMask);
         const bool full = (ent & kFullBit) != 0;
-        // stage -LSE*log2e (-inf where the row has no key or lies past Sq) and
-        // -Delta of this q-block, negated so the element loop is one packed
-        // FMA / add
+        // stage -LSE*log2e (half 0; -inf where the row has no key or lies past
+        // Sq) and -Delta (half 1) of this q-block, negated so the element loops
+        // are one packed FMA / add
         {
           const int i = m * kTile + r;
-          float nl2 = -INFINITY;
-          if (i < p.Sq) {
-            const float lv = p.lse[bh * p.Sq + i];
-            if (lv != -INFINITY) nl2 = -lv * kLog2e;
+          if (half == 0) {
+            float nl2 = -INFINITY;
+            if (i < p.Sq) {
+              const float lv = p.lse[bh * p.Sq + i];
+              if (lv != -INFINITY) nl2 = -lv * kLog2e;
+            }
+            vec_nl[(ec & 1) * kTile + r] = nl2;
+          } else {
+            vec_nd[(ec & 1) * kTile + r] = -p.delta[bh * p.nM * kTile + i];
           }
-          vec_nl[(ec & 1) * kTile + r] = nl2;
-          vec_nd[(ec & 1) * kTile + r] = -p.delta[bh * p.nM * kTile + i];
           mbar_arrive(&bars[L::bVecReady + (ec & 1)]);
         }
-        // allowed-query bits of this tile for this key row (range AND segment
-        // ids, the latter read through L1 as broadcasts)
-        uint32_t allow[4] = {~0u, ~0u, ~0u, ~0u};
+        // allowed-query bits of this half's two 32-query words for this key
+        // row (range AND segment ids, the latter read through L1 as broadcasts)
+        uint32_t allow[2] = {~0u, ~0u};
         if (!full) {
 #pragma unroll
-          for (int w = 0; w < 4; ++w) allow[w] = range_bits(qlo - m * kTile, qhi - m * kTile, w);
+          for (int w = 0; w < 2; ++w)
+            allow[w] = range_bits(qlo - m * kTile, qhi - m * kTile, 2 * half + w);
           if (dilated) {
             // keep query i iff (i + o - j) mod d == 0: bit k of word w is query
             // 128m + 32w + k, kept iff k == (j - o - 128m - 32w) mod d
-            int ph = (j - mk.offset - m * kTile) % mk.dilation;
+            int ph = (j - mk.offset - m * kTile - 64 * half) % mk.dilation;
             if (ph < 0) ph += mk.dilation;
 #pragma unroll
-            for (int w = 0; w < 4; ++w) {
+            for (int w = 0; w < 2; ++w) {
               allow[w] &= ph < 32 ? (mk.dil_pattern << ph) : 0u;
               ph -= mk.dil_r32;
               if (ph < 0) ph += mk.dilation;
             }
           }
           if (use_seg) {
-            const int32_t *sq = mk.seg_q + static_cast<int64_t>(k.b) * p.Sq + m * kTile;
-            const int lim = p.Sq - m * kTile;
+            const int32_t *sq = mk.seg_q + static_cast<int64_t>(k.b) * p.Sq + m * kTile + 64 * half;
+            const int lim = p.Sq - m * kTile - 64 * half;
 #pragma unroll
-            for (int w = 0; w < 4; ++w) {
+            for (int w = 0; w < 2; ++w) {
               uint32_t bits = 0;
 #pragma unroll 8
               for (int q = 0; q < 32; ++q) {
@@ -455,19 +477,19 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
           }
         }
         if (!wwait(&bars[L::bVecReady + (ec & 1)], (ec >> 1) & 1)) { stop = true; break; }
-        const float4 *nl4p = reinterpret_cast<const float4 *>(vec_nl + (ec & 1) * kTile);
-        const float4 *nd4p = reinterpret_cast<const float4 *>(vec_nd + (ec & 1) * kTile);
+        const float4 *nl4p = reinterpret_cast<const float4 *>(vec_nl + (ec & 1) * kTile + 64 * half);
+        const float4 *nd4p = reinterpret_cast<const float4 *>(vec_nd + (ec & 1) * kTile + 64 * half);
         // phase 1: P^T = exp2(S^T * scale * log2e - LSE*log2e) -> bf16 in TMEM
-        // (over the first 64 S^T columns, the A operand of dV) and kept in
-        // registers as fp16 pairs for dS: P lies in [0, 1], where fp16 keeps 11
-        // significant bits to bf16's 8, so dS carries no extra rounding of P
+        // (the A operand of dV) and kept in registers as fp16 pairs for dS: P
+        // lies in [0, 1], where fp16 keeps 11 significant bits to bf16's 8, so
+        // dS carries no extra rounding of P
         if (!wwait(&bars[L::bSFull], ec & 1)) { stop = true; break; }
         tc_fence_after();
-        uint32_t pk[64];
+        uint32_t pk[32];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 2; ++c) {
           uint32_t s[32], pb[16];
-          tmem_ld32(T_S + lane_off + 32 * c, s);
+          tmem_ld32(T_S + lane_off + 64 * half + 32 * c, s);
           tmem_wait_ld();
 #pragma unroll
           for (int q4 = 0; q4 < 8; ++q4) {
@@ -487,8 +509,9 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
               pk[16 * c + (e0 >> 1)] = pack_f16x2(p0, p1);
             }
           }
-          // P^T chunk -> TMEM columns [16c, 16c+16): only S^T columns already read
-          tmem_st16(T_S + lane_off + 16 * c, pb);
+          // P^T chunk -> TMEM columns [16c, 16c+16) of this half's region: S^T
+          // columns this warp has already read
+          tmem_st16(t_p + 16 * c, pb);
         }
         tmem_wait_st();
         tc_fence_before();
@@ -499,9 +522,9 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
         if (!wwait(&bars[L::bDPFull], ec & 1)) { stop = true; break; }
         tc_fence_after();
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 2; ++c) {
           uint32_t dp[32];
-          tmem_ld32(T_DP + lane_off + 32 * c, dp);
+          tmem_ld32(T_DP + lane_off + 64 * half + 32 * c, dp);
           tmem_wait_ld();
           uint32_t dk2[16];
 #pragma unroll
@@ -521,7 +544,7 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
           }
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
-            const int chunk = 4 * c + u;  // 0..15 over 128 queries
+            const int chunk = 8 * half + 4 * c + u;  // 0..15 over 128 queries
             const int sub = chunk >> 3, cw = chunk & 7;
             uint8_t *dst = ds_tile + sub * 16384 + r * 128 + ((cw ^ (r & 7)) << 4);
             *reinterpret_cast<int4 *>(dst) =
@@ -533,13 +556,13 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
         mbar_arrive(&bars[L::bDSReady]);
       }
       if (stop) break;
-      // epilogue: dV, dK (scaled) -> bf16
+      // epilogue: this half's columns of dV, dK (scaled) -> bf16
       if (!wwait(&bars[L::bDKVFull], cc & 1)) break;
       tc_fence_after();
       __nv_bfloat16 *dk_row = p.dk + k.b * p.k_sb + static_cast<int64_t>(j) * p.k_ss + k.hk * p.k_sh;
       __nv_bfloat16 *dv_row = p.dv + k.b * p.v_sb + static_cast<int64_t>(j) * p.v_ss + k.hk * p.v_sh;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = half * (D / 64); c < (half + 1) * (D / 64); ++c) {
         uint32_t a[32], g[32];
         tmem_ld32(T_DV + lane_off + 32 * c, a);
         tmem_ld32(T_DK + lane_off + 32 * c, g);
@@ -565,7 +588,10 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       mbar_arrive(&bars[L::bDKVFree]);
       ++cc;
     }
-  } else if (warp >= 8) {
+    }
+  } else {
+    regs_inc<160>();
+    if (run) {
     // ------------------------------------------------------------ dQ (query rows)
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
@@ -627,7 +653,7 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
           __threadfence();
           __syncwarp();
           if (lane == 0) mbar_arrive(&bars[L::bDQAdded + (ec & 1)]);
-          if (warp == 8 && lane == 0) {
+          if (warp == 12 && lane == 0) {
             // the last of the four warps' adds is visible: pass the turn on
             if (wd.wait(&bars[L::bDQAdded + (ec & 1)], (ec >> 1) & 1)) {
               __threadfence();
@@ -638,6 +664,7 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
         }
       }
       if (stop) break;
+    }
     }
   }
 
@@ -749,10 +776,17 @@ cudaError_t run_bwd_main(const BwdParams &bp, const CUtensorMap &tq, const CUten
     cudaError_t e = cudaFuncSetAttribute(k_attn_bwd<D, NQ, NDO>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
     if (e != cudaSuccess) return e;
+    // the warpgroups' register budgets add up to kThreads x kLaunchRegs: a
+    // kernel built with any other register count must not be launched, since
+    // an increase beyond what the launch holds would never be granted
+    cudaFuncAttributes fa{};
+    e = cudaFuncGetAttributes(&fa, k_attn_bwd<D, NQ, NDO>);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs != kLaunchRegs) return cudaErrorInvalidConfiguration;
     attr = true;
   }
   const int grid = std::max(1, std::min(bp.n_tickets, sm_count_bwd()));
-  k_attn_bwd<D, NQ, NDO><<<grid, 384, L::kAlloc, s>>>(tq, tk, tv, tdo, bp);
+  k_attn_bwd<D, NQ, NDO><<<grid, kThreads, L::kAlloc, s>>>(tq, tk, tv, tdo, bp);
   count_launch();
   return cudaGetLastError();
 }

@@ -45,6 +45,7 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units: tolerate p up to 2^8
 struct FwdParams {
   MaskParams mask;
   int B, H, Sq, Skv, nM, n_units;
+  int n_pairs;   // units [0, n_pairs) are q-block pairs; the rest are single q-blocks
   int kv_group;  // query heads per key/value head (grouped-query attention)
   float scale, scale_log2;
   const int32_t *row_ptr;
@@ -89,7 +90,9 @@ __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity) {
   }
 }
 
-// One work unit: a pair of q-blocks (A = 2g, B = 2g+1) of one (b, h).
+// One work unit: a pair of q-blocks (A = 2g, B = 2g+1) of one (b, h).  The
+// pairs that would make a last, partly filled wave are split into two single
+// q-block units each (slot A only), so that wave takes about half as long.
 struct FwdUnit {
   int b, h, bh, m[2], rs[2], re[2];
 };
@@ -97,13 +100,19 @@ struct FwdUnit {
 __device__ __forceinline__ FwdUnit decode_unit(const FwdParams &p, int u) {
   FwdUnit w;
   const int nP = (p.nM + 1) >> 1;
-  w.bh = u / nP;
-  const int g = u % nP;
+  int pu = u, only = -1;
+  if (u >= p.n_pairs) {
+    const int s = u - p.n_pairs;
+    pu = p.n_pairs + (s >> 1);
+    only = s & 1;
+  }
+  w.bh = pu / nP;
+  const int g = pu % nP;
   w.b = w.bh / p.H;
   w.h = w.bh % p.H;
 #pragma unroll
   for (int x = 0; x < 2; ++x) {
-    w.m[x] = 2 * g + x;
+    w.m[x] = only < 0 ? 2 * g + x : (x == 0 ? 2 * g + only : p.nM);
     if (w.m[x] < p.nM) {
       w.rs[x] = p.row_ptr[w.b * p.nM + w.m[x]];
       w.re[x] = p.row_ptr[w.b * p.nM + w.m[x] + 1];
@@ -267,12 +276,24 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
         if (stop) break;
         bool first[2] = {true, true};
         UnionWalk uw{p.row_ent, {w.rs[0], w.rs[1]}, {w.re[0], w.re[1]}};
+        // Q_x is read by the S MMAs only: once group x's last S of the unit is
+        // issued, its completion frees the buffer for the next unit's Q_x,
+        // which then loads while this unit's last softmax, PV and epilogue run
+        auto release_q = [&](int x) {
+          if (uw.i[x] >= uw.e[x]) {
+            mma_commit(&bars[L::bQEmpty + x]);
+            ++uq[x];
+          }
+        };
         int n;
         bool in_cur[2], in_nxt[2];
         uw.next(n, in_cur[0], in_cur[1]);
         uint32_t kv_cur = kv;
         for (int x = 0; x < 2 && !stop; ++x)
-          if (in_cur[x] && !issue_s(x, kv_cur)) stop = true;
+          if (in_cur[x]) {
+            if (!issue_s(x, kv_cur)) stop = true;
+            else release_q(x);
+          }
         if (stop) break;
         mma_commit(&bars[L::bKEmpty + kv_cur % NK]);
         for (;;) {
@@ -295,7 +316,10 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
               ++tcount[x];
             }
             // the next S of this group as soon as its P has been consumed
-            if (more && in_nxt[x] && !issue_s(x, kv_nxt)) { stop = true; break; }
+            if (more && in_nxt[x]) {
+              if (!issue_s(x, kv_nxt)) { stop = true; break; }
+              release_q(x);
+            }
           }
           if (stop) break;
           mma_commit(&bars[L::bVEmpty + kv_cur % NV]);
@@ -307,11 +331,6 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
         }
         if (stop) break;
         kv = kv_cur + 1;
-        for (int x = 0; x < 2; ++x)
-          if (has[x]) {
-            mma_commit(&bars[L::bQEmpty + x]);
-            ++uq[x];
-          }
       }
       // every tcgen05 op this thread issued is complete before TMEM is freed
       mma_commit(&bars[L::bFinal]);
@@ -824,7 +843,14 @@ cudaError_t launch_fwd(const bsa_problem &p, const MaskParams &mp, const bsa_opt
   fp.Skv = p.Skv;
   fp.nM = L.nM;
   fp.kv_group = p.H / p.H_kv;
-  fp.n_units = p.B * p.H * ((L.nM + 1) / 2);
+  {
+    // split the pairs of a last wave that is at most half full into singles
+    const int pairs = p.B * p.H * ((L.nM + 1) / 2);
+    const int grid0 = std::min(pairs, sm_count());
+    const int r = pairs % grid0;
+    fp.n_pairs = (r != 0 && 2 * r <= grid0) ? pairs - r : pairs;
+    fp.n_units = pairs + (pairs - fp.n_pairs);
+  }
   fp.scale = p.scale;
   fp.scale_log2 = p.scale * kLog2e;
   fp.row_ptr = reinterpret_cast<const int32_t *>(ws + L.row_ptr);

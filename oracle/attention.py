@@ -197,7 +197,7 @@ def attention_forward(q, k, v, mask: MaskDesc, scale: float, rows=None, heads=No
 
 
 def attention_backward(q, k, v, dO, mask: MaskDesc, scale: float, chunk: int = 1024,
-                       heads=None, batches=None):
+                       heads=None, batches=None, ds_out=None):
     """Analytic gradient of sum(O * dO) for the dense definition above.
 
     With P the softmax weights (0 on masked entries and on empty rows):
@@ -205,7 +205,8 @@ def attention_backward(q, k, v, dO, mask: MaskDesc, scale: float, chunk: int = 1
       dP = dO V^T,  dS = P o (dP - Delta),
       dQ = scale * dS K,  dK = scale * dS^T Q,  dV = P^T dO,
     with dK and dV of a shared kv head summed over the query heads of its group.
-    Returns (dQ, dK, dV) fp64 with the input layouts.
+    Returns (dQ, dK, dV) fp64 with the input layouts.  A dict passed as
+    ``ds_out`` also receives dS as ds_out[(b, h)] = [Sq, Skv] (small inputs).
     """
     q, k, v, dO = _as64(q), _as64(k), _as64(v), _as64(dO)
     B, Sq, H, D = q.shape
@@ -234,6 +235,8 @@ def attention_backward(q, k, v, dO, mask: MaskDesc, scale: float, chunk: int = 1
                 delta = (do * O).sum(axis=1)
                 dP = do @ v[b, :, hk, :].T
                 dS = P * (dP - delta[:, None])
+                if ds_out is not None:
+                    ds_out.setdefault((b, h), np.zeros((Sq, Skv)))[r, :] = dS
                 dQ[b, r, h, :] = scale * (dS @ k[b, :, hk, :])
                 dK[b, :, hk, :] += scale * (dS.T @ q[b, r, h, :])
                 dV[b, :, hk, :] += P.T @ do

@@ -9,7 +9,7 @@ import torch
 import block_sparse_attention_map_b200 as bsa
 import oracle
 from block_sparse_attention_map_b200.workloads import make_workload
-from tests.gpu_common import O_TOL, excess, mask_desc, np64
+from tests.gpu_common import O_TOL, ds_rounding_terms, excess, mask_desc, np64
 
 pytestmark = pytest.mark.gpu
 
@@ -21,7 +21,7 @@ def _grads(wl, **kw):
     return o, lse, dq, dk, dv, wsb
 
 
-def _oracle_grads(wl, heads=None):
+def _oracle_grads(wl, heads=None, ds_out=None):
     """Oracle gradients; ``heads`` (query heads) must cover whole kv-head groups."""
     q, k, v, do = np64(wl.q), np64(wl.k), np64(wl.v), np64(wl.dO)
     if heads is not None:
@@ -29,14 +29,16 @@ def _oracle_grads(wl, heads=None):
         kvh = sorted({h // g for h in heads})
         q, do = q[:, :, heads], do[:, :, heads]
         k, v = k[:, :, kvh], v[:, :, kvh]
-    return oracle.attention_backward(q, k, v, do, mask_desc(wl), wl.scale)
+    return oracle.attention_backward(q, k, v, do, mask_desc(wl), wl.scale, ds_out=ds_out)
 
 
-def _err(x, ref):
-    """Raw max-abs error, after checking the ulp-aware bar element by element."""
-    ex = excess(x, ref)
+def _err(x, ref, extra=0.0):
+    """Raw max-abs error, after checking the ulp-aware bar element by element
+    (plus, where given, the per-element term the bf16 dS operand forces)."""
+    ex = excess(x, ref, extra=extra)
     raw = float(np.max(np.abs(np64(x) - ref)))
-    assert ex <= 0.0, f"max-abs {raw:.5f} exceeds {O_TOL} + half a bf16 ulp by {ex:.5f}"
+    what = " + the dS rounding term" if np.any(extra) else ""
+    assert ex <= 0.0, f"max-abs {raw:.5f} exceeds {O_TOL} + half a bf16 ulp{what} by {ex:.5f}"
     return min(raw, O_TOL)
 
 
@@ -53,8 +55,13 @@ def test_bwd_matches_oracle(name):
         wl.dO = torch.randn(wl.q.shape, device="cuda", generator=g).bfloat16()
     _, _, dq, dk, dv, ws = _grads(wl)
     assert ws.status() == 0
-    gq, gk, gv = _oracle_grads(wl)
+    ds = {}
+    gq, gk, gv = _oracle_grads(wl, ds_out=ds)
+    # dQ and dK: the bar plus the rounding of the bf16 dS operand, which rows
+    # with only a few keys (document starts) bring to the order of the bar
+    eq, ek = ds_rounding_terms(wl, ds, wl.scale)
     heads = list(range(wl.H))
+    kv_heads = list(range(wl.k.shape[2]))
     if name == "video":
         # Head 0 of the video shape carries the 8 "sink" keys scaled x20: its
         # scores reach ~110 nats, so the fp32 rounding of S (~1e-3 there) and the
@@ -62,9 +69,10 @@ def test_bwd_matches_oracle(name):
         # dQ = scale dS K multiplies by |k| ~ 40.  The video workload is
         # forward-only; its forward parity covers the sink head.  The backward
         # is compared on the normal heads.
-        heads = heads[1:]
-    e = (_err(dq[:, :, heads], gq[:, :, heads]), _err(dk[:, :, heads], gk[:, :, heads]),
-         _err(dv[:, :, heads], gv[:, :, heads]))
+        heads, kv_heads = heads[1:], kv_heads[1:]
+    e = (_err(dq[:, :, heads], gq[:, :, heads], eq[:, :, heads]),
+         _err(dk[:, :, kv_heads], gk[:, :, kv_heads], ek[:, :, kv_heads]),
+         _err(dv[:, :, kv_heads], gv[:, :, kv_heads]))
     assert max(e) <= O_TOL, e
 
 
