@@ -74,6 +74,8 @@ def parse():
                     help="fixed-m reference: Cauchy-Schwarz on ||k|| or on the centred keys")
     ap.add_argument("--order", default="asc", choices=["asc", "desc", "outside_in", "greedy"])
     ap.add_argument("--nondet", action="store_true", help="atomic (non-deterministic) dQ backward")
+    ap.add_argument("--residual", action="store_true",
+                    help="keep O's bf16 rounding residual for an exact-to-fp32 Delta")
     ap.add_argument("--workload", default=WORKLOAD_NAME, choices=sorted(WORKLOADS))
     ap.add_argument("--small", action="store_true",
                     help="small shape of the same workload (for profiler captures)")
@@ -279,7 +281,7 @@ def run_ours(args, world, rank, local):
     dev = torch.device("cuda", local)
     wl = make_workload(args.workload, device=dev, small=args.small)
     st = bsa.Stages(wl.q, wl.k, wl.v, wl.mask, softmax_mode=args.softmax, order=args.order,
-                    deterministic=not args.nondet, bound_mode=args.bound)
+                    deterministic=not args.nondet, bound_mode=args.bound, keep_o_residual=args.residual)
     dO = wl.dO
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
@@ -359,7 +361,7 @@ def run_ours(args, world, rank, local):
         "config": {"workload": workload_text(args) + (" [small shape]" if args.small else ""),
                    "global_batch": wl.B * world, "seq_len": wl.Sq, "heads": wl.H,
                    "head_dim": wl.D, "mask": wl.mask_text(), "nonempty_tiles": n_tiles,
-                   "softmax": args.softmax, "bound": args.bound,
+                   "softmax": args.softmax, "bound": args.bound, "o_residual": args.residual,
                    "bwd_order": "nondeterministic" if args.nondet else args.order,
                    "l2": "flushed (256 MiB write) before every step, outside the timed events",
                    "parallelism": f"replicas x{world}"},
@@ -409,7 +411,8 @@ def e2e_leg(args, wl, dev, flops, world):
                                   ("dk", wl.k.shape, torch.bfloat16),
                                   ("dv", wl.v.shape, torch.bfloat16))}
     st = bsa.Stages(dev_in["q"], dev_in["k"], dev_in["v"], wl.mask, softmax_mode=args.softmax,
-                    order=args.order, deterministic=not args.nondet, bound_mode=args.bound)
+                    order=args.order, deterministic=not args.nondet, bound_mode=args.bound,
+                    keep_o_residual=args.residual)
     stream = torch.cuda.current_stream()
 
     def step():

@@ -54,14 +54,15 @@ class Options(ctypes.Structure):
     _fields_ = [("softmax_mode", c_i32), ("gate_limit", c_f32), ("kmax_override", c_vp),
                 ("bwd_order", c_i32), ("deterministic", c_i32), ("perm", c_vp),
                 ("sem_timeout_ns", c_i64), ("plan_ready", c_i32), ("bound_ready", c_i32),
-                ("bound_mode", c_i32), ("reserved", c_i32)]
+                ("bound_mode", c_i32), ("keep_o_residual", c_i32)]
 
 
 class WorkspaceView(ctypes.Structure):
     _fields_ = [(n, ctypes.c_size_t) for n in (
         "total_bytes", "fwd_bytes", "off_status", "off_tile_class", "off_rank", "off_row_ptr",
         "off_row_ent", "off_col_ptr", "off_col_ent", "off_col_rank", "off_perm", "off_kmax",
-        "off_qmax", "off_gate", "off_delta", "off_dq_accum", "off_sem", "off_kbar", "off_qdot")] + \
+        "off_qmax", "off_gate", "off_delta", "off_dq_accum", "off_sem", "off_kbar", "off_qdot",
+        "off_o_resid")] + \
         [("nM", c_i32), ("nN", c_i32)]
 
 
@@ -205,7 +206,7 @@ class Mask:
 
 def make_options(softmax_mode="online", gate_limit=0.0, kmax_override=None, order="asc",
                  perm=None, deterministic=True, sem_timeout_ns=0, plan_ready=False,
-                 bound_ready=False, bound_mode="norm"):
+                 bound_ready=False, bound_mode="norm", keep_o_residual=False):
     o = Options()
     o.softmax_mode = SOFTMAX_FIXED_M_GATED if softmax_mode in ("fixed_m", SOFTMAX_FIXED_M_GATED) else SOFTMAX_ONLINE
     o.gate_limit = float(gate_limit)
@@ -216,6 +217,7 @@ def make_options(softmax_mode="online", gate_limit=0.0, kmax_override=None, orde
     o.plan_ready = 1 if plan_ready else 0
     o.bound_ready = 1 if bound_ready else 0
     o.bound_mode = BOUND[bound_mode] if isinstance(bound_mode, str) else int(bound_mode)
+    o.keep_o_residual = 1 if keep_o_residual else 0
     o._perm_buf = None
     if perm is not None:
         buf = (c_i32 * len(perm))(*[int(x) for x in perm])
@@ -313,16 +315,18 @@ def plan_build(q, k, v, mask=None, workspace: Optional[Workspace] = None, backwa
 
 def attn_fwd(q, k, v, mask=None, softmax_mode="online", gate_limit=0.0, kmax_override=None,
              workspace: Optional[Workspace] = None, out=None, lse=None, plan_ready=False,
-             scale=None, order="asc", perm=None, bound_mode="norm"):
-    """O = softmax(scale Q K^T + mask) V and LSE [B, H, Sq] through bsa_attn_fwd."""
+             scale=None, order="asc", perm=None, bound_mode="norm", keep_o_residual=False):
+    """O = softmax(scale Q K^T + mask) V and LSE [B, H, Sq] through bsa_attn_fwd.
+    With keep_o_residual the workspace is sized for the backward and keeps O's
+    bf16 rounding residual for an attn_bwd on the same workspace."""
     B, Sq, H, D = q.shape
     out = torch.empty_like(q) if out is None else out
     lse = torch.empty(B, H, Sq, dtype=torch.float32, device=q.device) if lse is None else lse
     prob = make_problem(q, k, v, out, scale)
     m = Mask(mask, q.device)
     o = make_options(softmax_mode, gate_limit, kmax_override, order, perm, True, 0, plan_ready,
-                     bound_mode=bound_mode)
-    ws = workspace or Workspace(prob, m, False, q.device)
+                     bound_mode=bound_mode, keep_o_residual=keep_o_residual)
+    ws = workspace or Workspace(prob, m, keep_o_residual, q.device)
     _check(lib().bsa_attn_fwd(ctypes.byref(prob), ctypes.byref(m.spec), ctypes.byref(o), q.data_ptr(),
                               k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), ws.ptr(),
                               ws.nbytes, _stream()), "bsa_attn_fwd")
@@ -332,14 +336,16 @@ def attn_fwd(q, k, v, mask=None, softmax_mode="online", gate_limit=0.0, kmax_ove
 
 def attn_bwd(q, k, v, out, dout, lse, mask=None, order="asc", perm=None, deterministic=True,
              workspace: Optional[Workspace] = None, plan_ready=False, scale=None,
-             dq=None, dk=None, dv=None, sem_timeout_ns=0):
-    """dQ, dK, dV of sum(O * dO) through bsa_attn_bwd."""
+             dq=None, dk=None, dv=None, sem_timeout_ns=0, keep_o_residual=False):
+    """dQ, dK, dV of sum(O * dO) through bsa_attn_bwd.  keep_o_residual: Delta
+    uses the O residual an attn_fwd(keep_o_residual=True) left in ``workspace``."""
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
     prob = make_problem(q, k, v, out, scale)
     m = Mask(mask, q.device)
-    o = make_options("online", 0.0, None, order, perm, deterministic, sem_timeout_ns, plan_ready)
+    o = make_options("online", 0.0, None, order, perm, deterministic, sem_timeout_ns, plan_ready,
+                     keep_o_residual=keep_o_residual)
     ws = workspace or Workspace(prob, m, True, q.device)
     _check(lib().bsa_attn_bwd(ctypes.byref(prob), ctypes.byref(m.spec), ctypes.byref(o), q.data_ptr(),
                               k.data_ptr(), v.data_ptr(), out.data_ptr(), dout.data_ptr(), lse.data_ptr(),
@@ -355,7 +361,7 @@ class Stages:
     workspace, for callers that time or schedule stages separately."""
 
     def __init__(self, q, k, v, mask=None, softmax_mode="online", order="asc", perm=None,
-                 deterministic=True, gate_limit=0.0, bound_mode="norm"):
+                 deterministic=True, gate_limit=0.0, bound_mode="norm", keep_o_residual=False):
         self.q, self.k, self.v = q, k, v
         B, Sq, H, D = q.shape
         self.out = torch.empty_like(q)
@@ -365,7 +371,8 @@ class Stages:
         self.mask = Mask(mask, q.device)
         self.fixed = softmax_mode in ("fixed_m", SOFTMAX_FIXED_M_GATED)
         self.opt = make_options(softmax_mode, gate_limit, None, order, perm, deterministic, 0,
-                                plan_ready=True, bound_ready=True, bound_mode=bound_mode)
+                                plan_ready=True, bound_ready=True, bound_mode=bound_mode,
+                                keep_o_residual=keep_o_residual)
         self.ws = Workspace(self.prob, self.mask, True, q.device)
         self._args = (ctypes.byref(self.prob), ctypes.byref(self.mask.spec), ctypes.byref(self.opt))
 

@@ -49,7 +49,8 @@ WsLayout compute_layout(const bsa_problem &p) {
   L.seg_kv = take(4 * static_cast<size_t>(p.Skv));
   L.qblk = take(16 * static_cast<size_t>(B * nM));
   L.kblk = take(16 * static_cast<size_t>(B * nN));
-  L.kmax = take(8 * static_cast<size_t>(B * H));  // kmax then qmax, adjacent
+  // kmax, qmax, then the bound kernel's finished-block counter, adjacent
+  L.kmax = take(8 * static_cast<size_t>(B * H) + 4);
   L.qmax = L.kmax + 4 * static_cast<size_t>(B * H);
   L.gate = take(4 * static_cast<size_t>(B * H));
   L.qnorm = take(4 * static_cast<size_t>(B * H * p.Sq));
@@ -61,6 +62,7 @@ WsLayout compute_layout(const bsa_problem &p) {
   L.delta = take(4 * static_cast<size_t>(B * H * nM * kTile));
   L.dq_accum = take(4 * static_cast<size_t>(B * H * nM * kTile * p.D));
   L.sem = take(4 * static_cast<size_t>(B * H * nM));
+  L.o_resid = take(2 * static_cast<size_t>(B * H * p.Sq * p.D));
   L.total = off;
   return L;
 }
@@ -261,7 +263,9 @@ bsa_status prepare(const bsa_problem *prob, const bsa_mask_spec *mask, const bsa
   if (out->o.bound_mode == BSA_BOUND_SMOOTHED && out->p.H_kv * out->p.D > kMaxSmoothedHD)
     return BSA_ERR_UNSUPPORTED;
   if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return BSA_ERR_INVALID_ARG;
-  if (ws_bytes < (backward ? out->L.total : out->L.fwd_end)) return BSA_ERR_WORKSPACE_TOO_SMALL;
+  // the O residual lives in the backward part of the workspace
+  const bool full = backward || out->o.keep_o_residual != 0;
+  if (ws_bytes < (full ? out->L.total : out->L.fwd_end)) return BSA_ERR_WORKSPACE_TOO_SMALL;
   if (!have_device()) return BSA_ERR_NO_DEVICE;
   return BSA_OK;
 }
@@ -316,6 +320,7 @@ bsa_status bsa_workspace_layout(const bsa_problem *prob, const bsa_mask_spec *ma
   view->off_sem = L.sem;
   view->off_kbar = L.kbar;
   view->off_qdot = L.qdot;
+  view->off_o_resid = L.o_resid;
   view->nM = L.nM;
   view->nN = L.nN;
   return BSA_OK;

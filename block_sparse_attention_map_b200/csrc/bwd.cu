@@ -682,7 +682,10 @@ __global__ void __launch_bounds__(256) k_bwd_delta(const __nv_bfloat16 *__restri
                                                    const __nv_bfloat16 *__restrict__ dout,
                                                    int64_t sb, int64_t ss, int64_t sh, int B,
                                                    int Sq, int H, int rows_pad,
+                                                   const __nv_bfloat16 *__restrict__ resid,
                                                    float *__restrict__ delta) {
+  // D/8 threads per (b, h, i) row vector, 16 bytes of O, dO (and the O
+  // residual) each; rows past Sq (the last q-block's padding) get Delta = 0
   constexpr int TPV = D / 8;
   const int64_t g = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) / TPV;
   const int t = threadIdx.x % TPV;
@@ -694,15 +697,22 @@ __global__ void __launch_bounds__(256) k_bwd_delta(const __nv_bfloat16 *__restri
   float acc = 0.f;
   if (in && i < Sq) {
     const int64_t off = b * sb + static_cast<int64_t>(i) * ss + h * sh + t * 8;
-    const int4 a = *reinterpret_cast<const int4 *>(o + off);
-    const int4 c = *reinterpret_cast<const int4 *>(dout + off);
-    const __nv_bfloat162 *x = reinterpret_cast<const __nv_bfloat162 *>(&a);
-    const __nv_bfloat162 *y = reinterpret_cast<const __nv_bfloat162 *>(&c);
+    const int4 a = __ldg(reinterpret_cast<const int4 *>(o + off));
+    const int4 c = __ldg(reinterpret_cast<const int4 *>(dout + off));
+    int4 r = make_int4(0, 0, 0, 0);
+    if (resid != nullptr)
+      r = __ldg(reinterpret_cast<const int4 *>(resid + ((static_cast<int64_t>(b) * Sq + i) * H + h) * D + t * 8));
+    const uint32_t xa[4] = {static_cast<uint32_t>(a.x), static_cast<uint32_t>(a.y),
+                            static_cast<uint32_t>(a.z), static_cast<uint32_t>(a.w)};
+    const uint32_t xc[4] = {static_cast<uint32_t>(c.x), static_cast<uint32_t>(c.y),
+                            static_cast<uint32_t>(c.z), static_cast<uint32_t>(c.w)};
+    const uint32_t xr[4] = {static_cast<uint32_t>(r.x), static_cast<uint32_t>(r.y),
+                            static_cast<uint32_t>(r.z), static_cast<uint32_t>(r.w)};
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      const float2 fx = __bfloat1622float2(x[q]), fy = __bfloat1622float2(y[q]);
-      acc = fmaf(fx.x, fy.x, acc);
-      acc = fmaf(fx.y, fy.y, acc);
+      const float2 fo = unpack_bf16x2(xa[q]), fd = unpack_bf16x2(xc[q]), fr = unpack_bf16x2(xr[q]);
+      acc = fmaf(fo.x + fr.x, fd.x, acc);
+      acc = fmaf(fo.y + fr.y, fd.y, acc);
     }
   }
 #pragma unroll
@@ -711,47 +721,36 @@ __global__ void __launch_bounds__(256) k_bwd_delta(const __nv_bfloat16 *__restri
 }
 
 // ---------------------------------------------------------------- a7: dQ convert
+// A thread per (row, 4 columns) of a q-block: it reads one float4 of the
+// interleaved accumulator [B, H, nM, D/4, 128, 4] (consecutive threads, rows
+// of one column group: contiguous) and writes 4 bf16 of the row; the row's
+// other pieces come from the neighbouring column groups of the same warp loop,
+// so the L2 merges them into whole sectors.  Q-blocks that no kv column
+// reaches get zeros.
 template <int D>
 __global__ void __launch_bounds__(256) k_dq_convert(const float *__restrict__ acc, int B, int H,
                                                     int Sq, int nM, const int32_t *__restrict__ row_ptr,
                                                     __nv_bfloat16 *__restrict__ dq,
                                                     int64_t sb, int64_t ss, int64_t sh) {
-  extern __shared__ float tile[];  // [128][D + 4]
-  constexpr int LD = D + 4;
-  const int bhm = blockIdx.x;
-  const int m = bhm % nM, bh = bhm / nM, b = bh / H, h = bh % H;
-  const float *src = acc + static_cast<int64_t>(bhm) * (D / 4) * kTile * 4;
-  if (row_ptr[b * nM + m + 1] == row_ptr[b * nM + m]) {
-    // a q-block without non-empty tiles got no contribution: dQ = 0
-    constexpr int CPR = D / 8;
-    for (int idx = threadIdx.x; idx < kTile * CPR; idx += blockDim.x) {
-      const int r = idx / CPR, c = idx % CPR;
-      const int i = m * kTile + r;
-      if (i < Sq)
-        *reinterpret_cast<int4 *>(dq + b * sb + static_cast<int64_t>(i) * ss + h * sh + 8 * c) =
-            make_int4(0, 0, 0, 0);
-    }
-    return;
-  }
-  for (int idx = threadIdx.x; idx < (D / 4) * kTile; idx += blockDim.x) {
-    const int c = idx / kTile, r = idx % kTile;
-    const float4 v = reinterpret_cast<const float4 *>(src)[idx];
-    float *d = tile + r * LD + 4 * c;
-    d[0] = v.x;
-    d[1] = v.y;
-    d[2] = v.z;
-    d[3] = v.w;
-  }
-  __syncthreads();
-  constexpr int CPR = D / 8;  // 16-byte chunks per row
-  for (int idx = threadIdx.x; idx < kTile * CPR; idx += blockDim.x) {
-    const int r = idx / CPR, c = idx % CPR;
+  constexpr int kC = D / 4;  // float4 column groups per row
+  const int64_t total = static_cast<int64_t>(B) * H * nM * kC * kTile;
+  for (int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; t < total;
+       t += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int r = static_cast<int>(t % kTile);
+    const int64_t rest = t / kTile;
+    const int c = static_cast<int>(rest % kC);
+    const int64_t bhm = rest / kC;
+    const int m = static_cast<int>(bhm % nM);
+    const int64_t bh = bhm / nM;
+    const int b = static_cast<int>(bh / H), h = static_cast<int>(bh % H);
     const int i = m * kTile + r;
     if (i >= Sq) continue;
-    const float *s = tile + r * LD + 8 * c;
-    const int4 w = make_int4(pack_bf16x2(s[0], s[1]), pack_bf16x2(s[2], s[3]),
-                             pack_bf16x2(s[4], s[5]), pack_bf16x2(s[6], s[7]));
-    *reinterpret_cast<int4 *>(dq + b * sb + static_cast<int64_t>(i) * ss + h * sh + 8 * c) = w;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (row_ptr[b * nM + m + 1] != row_ptr[b * nM + m]) v = __ldcs(reinterpret_cast<const float4 *>(acc) + t);
+    uint2 w;
+    w.x = pack_bf16x2(v.x, v.y);
+    w.y = pack_bf16x2(v.z, v.w);
+    *reinterpret_cast<uint2 *>(dq + b * sb + static_cast<int64_t>(i) * ss + h * sh + 4 * c) = w;
   }
 }
 
@@ -798,19 +797,20 @@ cudaError_t launch_bwd_preprocess(const bsa_problem &p, const bsa_options &o, co
                                   cudaStream_t s) {
   const int rows_pad = L.nM * kTile;
   const int64_t groups = static_cast<int64_t>(p.B) * p.H * rows_pad;
-  const int64_t threads = groups * (p.D / 8);
   float *delta = reinterpret_cast<float *>(ws + L.delta);
-  const unsigned blocks = static_cast<unsigned>((threads + 255) / 256);
+  const __nv_bfloat16 *resid =
+      o.keep_o_residual ? reinterpret_cast<const __nv_bfloat16 *>(ws + L.o_resid) : nullptr;
+  const unsigned blocks = static_cast<unsigned>((groups * (p.D / 8) + 255) / 256);
   if (p.D == 64)
     k_bwd_delta<64><<<blocks, 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(out),
                                            static_cast<const __nv_bfloat16 *>(dout), p.o_stride[0],
                                            p.o_stride[1], p.o_stride[2], p.B, p.Sq, p.H, rows_pad,
-                                           delta);
+                                           resid, delta);
   else
     k_bwd_delta<128><<<blocks, 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(out),
                                             static_cast<const __nv_bfloat16 *>(dout), p.o_stride[0],
                                             p.o_stride[1], p.o_stride[2], p.B, p.Sq, p.H, rows_pad,
-                                            delta);
+                                            resid, delta);
   count_launch();
   cudaError_t e = cudaSuccess;
   if (!o.deterministic) {
@@ -873,20 +873,19 @@ cudaError_t launch_bwd_main(const bsa_problem &p, const MaskParams &mp, const bs
 cudaError_t launch_bwd_convert(const bsa_problem &p, void *dq, const WsLayout &L, uint8_t *ws,
                                cudaStream_t s) {
   const float *acc = reinterpret_cast<const float *>(ws + L.dq_accum);
-  const unsigned blocks = static_cast<unsigned>(p.B * p.H * L.nM);
-  auto go = [&](auto kern, int D) -> cudaError_t {
-    const size_t smem = sizeof(float) * kTile * (D + 4);
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    kern<<<blocks, 256, smem, s>>>(acc, p.B, p.H, p.Sq, L.nM,
-                                   reinterpret_cast<const int32_t *>(ws + L.row_ptr),
-                                   static_cast<__nv_bfloat16 *>(dq), p.q_stride[0], p.q_stride[1],
-                                   p.q_stride[2]);
-    count_launch();
-    return cudaGetLastError();
-  };
-  return p.D == 64 ? go(k_dq_convert<64>, 64) : go(k_dq_convert<128>, 128);
+  const int64_t total = static_cast<int64_t>(p.B) * p.H * L.nM * (p.D / 4) * kTile;
+  const unsigned blocks = static_cast<unsigned>(
+      std::min<int64_t>((total + 255) / 256, static_cast<int64_t>(sm_count_bwd()) * 8));
+  const int32_t *row_ptr = reinterpret_cast<const int32_t *>(ws + L.row_ptr);
+  __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(dq);
+  if (p.D == 64)
+    k_dq_convert<64><<<blocks, 256, 0, s>>>(acc, p.B, p.H, p.Sq, L.nM, row_ptr, out, p.q_stride[0],
+                                            p.q_stride[1], p.q_stride[2]);
+  else
+    k_dq_convert<128><<<blocks, 256, 0, s>>>(acc, p.B, p.H, p.Sq, L.nM, row_ptr, out, p.q_stride[0],
+                                             p.q_stride[1], p.q_stride[2]);
+  count_launch();
+  return cudaGetLastError();
 }
 
 cudaError_t launch_bwd(const bsa_problem &p, const MaskParams &mp, const bsa_options &o,

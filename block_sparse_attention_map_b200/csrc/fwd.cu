@@ -57,6 +57,7 @@ struct FwdParams {
   const float *kmax;   // [B, H] (the radius R with k-smoothing)
   const float *qnorm;  // [B, H, Sq]
   const float *qdot;   // [B, H, Sq] q_i . center with k-smoothing, else null
+  __nv_bfloat16 *o_resid;  // [B, Sq, H, D] O - bf16(O), or null
   const int32_t *gate; // [B, H]
   uint32_t *hdr;
   uint64_t timeout_ns;
@@ -536,6 +537,19 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
           int4 *dst = reinterpret_cast<int4 *>(orow + c * 16);
           dst[0] = make_int4(wv[0], wv[1], wv[2], wv[3]);
           dst[1] = make_int4(wv[4], wv[5], wv[6], wv[7]);
+          if (p.o_resid != nullptr) {
+            // what the bf16 rounding of O dropped, for an exact-to-fp32 Delta
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              const float2 r = unpack_bf16x2(wv[q]);
+              wv[q] = pack_bf16x2(__uint_as_float(o[2 * q]) * inv - r.x,
+                                  __uint_as_float(o[2 * q + 1]) * inv - r.y);
+            }
+            int4 *rd = reinterpret_cast<int4 *>(p.o_resid + ((static_cast<int64_t>(b) * p.Sq + i) * p.H + h) * D +
+                                                c * 16);
+            rd[0] = make_int4(wv[0], wv[1], wv[2], wv[3]);
+            rd[1] = make_int4(wv[4], wv[5], wv[6], wv[7]);
+          }
         }
       }
       tc_fence_before();
@@ -554,22 +568,28 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
 }
 
 // ---------------------------------------------------------------- fixed-m bound
-// Norms of every (row, head) vector of K (blockIdx.y == 0) and Q (== 1).
-// Keys: running max per (b, h) over valid keys (padding and varlen alignment
-// keys excluded).  Queries: the per-row norm is stored and the running max per
-// (b, h) kept.  Each group of D/8 threads owns one vector at a time and keeps
-// four vectors' loads in flight.  With k-smoothing (center != 0) the keys'
-// norms are taken of k_j - c and the queries also store q_i . c, c being the
-// mean valid key of the head from the fixed-point sums of k_key_sums.
+// Norms of every (row, head) vector of K (blockIdx.y == 0) and Q (== 1): one
+// thread per vector, consecutive threads on consecutive heads of a row, each
+// keeping kU 16-byte chunks in flight.  Keys: the maximum per (b, h) over valid
+// keys (padding and varlen alignment keys excluded), for every query head of
+// the key head's group.  Queries: the per-row norm is stored and the maximum per
+// (b, h) kept.  With k-smoothing (center != 0) the keys' norms are taken of
+// k_j - c and the queries also store q_i . c, c being the mean valid key of
+// the head from the fixed-point sums of k_key_sums.  The block that finishes
+// last computes the per-head gate.
 struct NormArgs {
   const __nv_bfloat16 *k, *q;
   int64_t ks[3], qs[3];
   int B, Skv, Sq, H, Hk, only_q, center;  // Hk: key heads (H / Hk query heads each)
   MaskParams mk;
   float *kmax, *qmax, *qnorm;
-  long long *ksum;        // [B, H, D] fixed-point sums of the valid keys
+  long long *ksum;        // [B, Hk, D] fixed-point sums of the valid keys
   int *kcount;            // [B] valid keys
-  float *kbar, *qdot;     // [B, H, D] center (written once per batch row), [B, H, Sq]
+  float *kbar, *qdot;     // [B, Hk, D] center (written once per batch row), [B, H, Sq]
+  uint32_t *done;         // blocks finished (zero before the launch)
+  const float *kmax_override;
+  float scale, limit;
+  int32_t *gate;
 };
 
 constexpr float kFixScale = 1048576.f;  // fixed-point unit 2^-20 of the key sums
@@ -628,97 +648,78 @@ __global__ void __launch_bounds__(256) k_key_sums(const NormArgs a) {
 
 template <int D>
 __global__ void __launch_bounds__(256) k_row_norms(const NormArgs a) {
-  constexpr int TPV = D / 8;  // threads per vector, 16 bytes each
-  constexpr int kRows = 32;
-  constexpr int kUnroll = 4;
-  extern __shared__ unsigned int smax[];  // [H], then the centers [H * D] (k-smoothing)
+  constexpr int kC = D / 8, kU = 4, kLD = D + 1;  // padded center rows: no bank conflicts
+  extern __shared__ unsigned int smax[];  // [H], then the centers [Hk][D + 1] (k-smoothing)
   float *cen = reinterpret_cast<float *>(smax + a.H);
+  __shared__ bool last_block;
   const int is_key = !a.only_q && blockIdx.y == 0;
   const __nv_bfloat16 *x = is_key ? a.k : a.q;
   const int S = is_key ? a.Skv : a.Sq;
   const int64_t sb = is_key ? a.ks[0] : a.qs[0], ss = is_key ? a.ks[1] : a.qs[1],
                 sh = is_key ? a.ks[2] : a.qs[2];
   float *rowmax = is_key ? a.kmax : a.qmax;
-  const int H = a.H, Sq = a.Sq, Skv = a.Skv;
+  const int H = a.H;
   const int Hx = is_key ? a.Hk : H;  // heads of this tensor
   const int grp = H / a.Hk;          // query heads per key head
-  const MaskParams &mk = a.mk;
-  float *qnorm = a.qnorm;
-  const int64_t blocks_per_b = (max(Sq, Skv) + kRows - 1) / kRows;
-  const int b = static_cast<int>(blockIdx.x / blocks_per_b);
-  const int r0 = static_cast<int>(blockIdx.x % blocks_per_b) * kRows;
-  if (r0 >= S) return;  // whole block past this tensor's rows (uniform)
+  const int bpb = static_cast<int>(gridDim.x / a.B);  // blocks per batch row
+  const int b = static_cast<int>(blockIdx.x) / bpb, blk = static_cast<int>(blockIdx.x) % bpb;
   for (int h = threadIdx.x; h < H; h += blockDim.x) smax[h] = 0u;
   if (a.center) {
     // c = (fixed-point sum) * 2^-20 / (valid keys), the same in every block
     const double inv = 1.0 / (static_cast<double>(kFixScale) * max(1, a.kcount[b]));
-    const long long *ks = a.ksum + static_cast<int64_t>(b) * a.Hk * D;
-    const bool write = is_key && r0 == 0;
+    const long long *ksum = a.ksum + static_cast<int64_t>(b) * a.Hk * D;
+    const bool write = is_key && blk == 0;
     for (int t = threadIdx.x; t < a.Hk * D; t += blockDim.x) {
-      const float c = static_cast<float>(static_cast<double>(ks[t]) * inv);
-      cen[t] = c;
+      const float c = static_cast<float>(static_cast<double>(ksum[t]) * inv);
+      cen[(t / D) * kLD + t % D] = c;
       if (write) a.kbar[static_cast<int64_t>(b) * a.Hk * D + t] = c;
     }
   }
   __syncthreads();
-  const int g = threadIdx.x / TPV, t = threadIdx.x % TPV;
-  const int groups = blockDim.x / TPV;
-  const int pairs = kRows * Hx;
-  // uniform trip count across the warp: the shuffles below need every lane
-  for (int base = 0; base < pairs; base += groups * kUnroll) {
-    float acc[kUnroll], dot[kUnroll];
-    int row[kUnroll], hh[kUnroll];
-    bool in[kUnroll];
+  const int64_t nvec = static_cast<int64_t>(S) * Hx;
+  for (int64_t v = static_cast<int64_t>(blk) * blockDim.x + threadIdx.x; v < nvec;
+       v += static_cast<int64_t>(bpb) * blockDim.x) {
+    const int row = static_cast<int>(v / Hx), hh = static_cast<int>(v % Hx);
+    const int4 *src = reinterpret_cast<const int4 *>(x + b * sb + static_cast<int64_t>(row) * ss + hh * sh);
+    const float *c = cen + (is_key ? hh : hh / grp) * kLD;
+    float acc = 0.f, dot = 0.f;
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const int pair = base + u * groups + g;
-      row[u] = r0 + pair / Hx;
-      hh[u] = pair % Hx;
-      in[u] = pair < pairs && row[u] < S;
-      acc[u] = 0.f;
-      dot[u] = 0.f;
-      if (in[u]) {
-        const int4 v = *reinterpret_cast<const int4 *>(x + b * sb + static_cast<int64_t>(row[u]) * ss +
-                                                      hh[u] * sh + t * 8);
-        const __nv_bfloat162 *e = reinterpret_cast<const __nv_bfloat162 *>(&v);
-        const float *c = cen + (is_key ? hh[u] : hh[u] / grp) * D + t * 8;
+    for (int c0 = 0; c0 < kC; c0 += kU) {
+      int4 w[kU];
+#pragma unroll
+      for (int u = 0; u < kU; ++u) w[u] = __ldg(src + c0 + u);
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const uint32_t xw[4] = {static_cast<uint32_t>(w[u].x), static_cast<uint32_t>(w[u].y),
+                                static_cast<uint32_t>(w[u].z), static_cast<uint32_t>(w[u].w)};
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          float2 f = __bfloat1622float2(e[q]);
+          float2 f = unpack_bf16x2(xw[q]);
+          const int d = 8 * (c0 + u) + 2 * q;
           if (a.center) {
             if (is_key) {
-              f.x -= c[2 * q];
-              f.y -= c[2 * q + 1];
+              f.x -= c[d];
+              f.y -= c[d + 1];
             } else {
-              dot[u] = fmaf(f.x, c[2 * q], dot[u]);
-              dot[u] = fmaf(f.y, c[2 * q + 1], dot[u]);
+              dot = fmaf(f.x, c[d], dot);
+              dot = fmaf(f.y, c[d + 1], dot);
             }
           }
-          acc[u] = fmaf(f.x, f.x, acc[u]);
-          acc[u] = fmaf(f.y, f.y, acc[u]);
+          acc = fmaf(f.x, f.x, acc);
+          acc = fmaf(f.y, f.y, acc);
         }
       }
     }
-#pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-#pragma unroll
-      for (int o = TPV / 2; o > 0; o >>= 1) {
-        acc[u] += __shfl_xor_sync(0xffffffffu, acc[u], o);
-        dot[u] += __shfl_xor_sync(0xffffffffu, dot[u], o);
-      }
-      if (t == 0 && in[u]) {
-        const float nrm = sqrtf(acc[u]);
-        bool valid = true;
-        if (is_key) {
-          valid = key_is_valid(mk, b, row[u]);
-        } else {
-          const int64_t idx = (static_cast<int64_t>(b) * H + hh[u]) * S + row[u];
-          qnorm[idx] = nrm;
-          if (a.center) a.qdot[idx] = dot[u];
-        }
-        if (valid) atomicMax(&smax[hh[u]], __float_as_uint(nrm));
-      }
+    const float nrm = sqrtf(acc);
+    bool valid = true;
+    if (is_key) {
+      valid = key_is_valid(a.mk, b, row);
+    } else {
+      const int64_t idx = (static_cast<int64_t>(b) * H + hh) * S + row;
+      a.qnorm[idx] = nrm;
+      if (a.center) a.qdot[idx] = dot;
     }
+    if (valid) atomicMax(&smax[hh], __float_as_uint(nrm));
   }
   __syncthreads();
   // a key head's maximum goes to every query head of its group
@@ -731,15 +732,23 @@ __global__ void __launch_bounds__(256) k_row_norms(const NormArgs a) {
         atomicMax(reinterpret_cast<unsigned int *>(rowmax) + b * H + h, smax[h]);
       }
     }
-}
-
-__global__ void k_gate(int BH, float scale, float limit, const float *kmax_override,
-                       float *kmax, const float *qmax, int32_t *gate) {
-  const int t = blockIdx.x * blockDim.x + threadIdx.x;
-  if (t >= BH) return;
-  const float km = kmax_override != nullptr ? kmax_override[t] : kmax[t];
-  kmax[t] = km;
-  gate[t] = (2.f * scale * qmax[t] * km <= limit) ? 1 : 0;
+  // the last block to finish takes the gate decision for every (b, h)
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const uint32_t n = gridDim.x * gridDim.y;
+    last_block = atomicAdd(a.done, 1u) == n - 1u;
+  }
+  __syncthreads();
+  if (!last_block) return;
+  __threadfence();
+  const int BH = a.B * H;
+  for (int t = threadIdx.x; t < BH; t += blockDim.x) {
+    const float km = a.kmax_override != nullptr ? a.kmax_override[t] : __ldcg(a.kmax + t);
+    a.kmax[t] = km;
+    a.gate[t] = (2.f * a.scale * __ldcg(a.qmax + t) * km <= a.limit) ? 1 : 0;
+  }
+  if (threadIdx.x == 0) *a.done = 0u;
 }
 
 int sm_count() {
@@ -793,12 +802,18 @@ cudaError_t launch_fixed_m_bound(const bsa_problem &p, const MaskParams &mp,
   na.mk = mp;
   na.kmax = reinterpret_cast<float *>(ws + L.kmax);
   na.qmax = reinterpret_cast<float *>(ws + L.qmax);
+  na.done = reinterpret_cast<uint32_t *>(ws + L.qmax) + p.B * p.H;
   na.qnorm = reinterpret_cast<float *>(ws + L.qnorm);
   na.ksum = reinterpret_cast<long long *>(ws + L.ksum);
   na.kcount = reinterpret_cast<int *>(ws + L.kcount);
   na.kbar = reinterpret_cast<float *>(ws + L.kbar);
   na.qdot = reinterpret_cast<float *>(ws + L.qdot);
-  cudaError_t e = cudaMemsetAsync(na.kmax, 0, sizeof(float) * p.B * p.H * 2, s);  // kmax, qmax
+  na.kmax_override = o.kmax_override;
+  na.scale = p.scale;
+  na.limit = o.gate_limit > 0.f ? o.gate_limit : 64.f;
+  na.gate = reinterpret_cast<int32_t *>(ws + L.gate);
+  // kmax, qmax and the finished-block counter are adjacent: one memset
+  cudaError_t e = cudaMemsetAsync(na.kmax, 0, sizeof(float) * p.B * p.H * 2 + sizeof(uint32_t), s);
   if (e != cudaSuccess) return e;
   size_t smem = sizeof(unsigned int) * p.H;
   if (na.center) {
@@ -809,10 +824,13 @@ cudaError_t launch_fixed_m_bound(const bsa_problem &p, const MaskParams &mp,
     if (p.D == 64) k_key_sums<64><<<sblocks, 256, 0, s>>>(na);
     else k_key_sums<128><<<sblocks, 256, 0, s>>>(na);
     count_launch();
-    smem += sizeof(float) * p.H_kv * p.D;
+    smem += sizeof(float) * p.H_kv * (p.D + 1);
   }
-  const int64_t blocks = static_cast<int64_t>(p.B) * ((std::max(p.Sq, p.Skv) + 31) / 32);
-  const dim3 grid(static_cast<unsigned>(blocks), na.only_q ? 1u : 2u);
+  // blocks per batch row: enough for about eight blocks per SM in all
+  const int64_t vec = static_cast<int64_t>(std::max(p.Sq * p.H, p.Skv * p.H_kv));
+  const int64_t want = std::max<int64_t>(1, (static_cast<int64_t>(sm_count()) * 4) / p.B);
+  const int bpb = static_cast<int>(std::min<int64_t>(want, (vec + 255) / 256));
+  const dim3 grid(static_cast<unsigned>(p.B * bpb), na.only_q ? 1u : 2u);
   if (smem > 48 * 1024) {
     e = p.D == 64 ? cudaFuncSetAttribute(k_row_norms<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem))
@@ -822,11 +840,6 @@ cudaError_t launch_fixed_m_bound(const bsa_problem &p, const MaskParams &mp,
   }
   if (p.D == 64) k_row_norms<64><<<grid, 256, smem, s>>>(na);
   else k_row_norms<128><<<grid, 256, smem, s>>>(na);
-  count_launch();
-  const float limit = o.gate_limit > 0.f ? o.gate_limit : 64.f;
-  const int BH = p.B * p.H;
-  k_gate<<<(BH + 127) / 128, 128, 0, s>>>(BH, p.scale, limit, o.kmax_override, na.kmax, na.qmax,
-                                          reinterpret_cast<int32_t *>(ws + L.gate));
   count_launch();
   return cudaGetLastError();
 }
@@ -864,6 +877,7 @@ cudaError_t launch_fwd(const bsa_problem &p, const MaskParams &mp, const bsa_opt
   fp.kmax = reinterpret_cast<const float *>(ws + L.kmax);
   fp.qnorm = reinterpret_cast<const float *>(ws + L.qnorm);
   fp.qdot = o.bound_mode == BSA_BOUND_SMOOTHED ? reinterpret_cast<const float *>(ws + L.qdot) : nullptr;
+  fp.o_resid = o.keep_o_residual ? reinterpret_cast<__nv_bfloat16 *>(ws + L.o_resid) : nullptr;
   fp.gate = reinterpret_cast<const int32_t *>(ws + L.gate);
   fp.hdr = reinterpret_cast<uint32_t *>(ws + L.status);
   fp.timeout_ns = 2000000000ull;

@@ -54,6 +54,7 @@ struct WsLayout {
                                       // sums [B,H,D] int64, valid keys [B], q.c [B,H,Sq]
   size_t fwd_end;
   size_t delta, dq_accum, sem;        // backward scratch
+  size_t o_resid;                     // [B, Sq, H, D] bf16 O rounding residual
   size_t total;
   int nM, nN;
   int64_t nnz_cap;

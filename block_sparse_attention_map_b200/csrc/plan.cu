@@ -441,6 +441,229 @@ __global__ void k_col_fill(const uint8_t *__restrict__ cls, const int32_t *__res
   }
 }
 
+// Exclusive scan of n counts in shared memory into out[0..n] (out[n] = total),
+// by the whole block: each thread sums a contiguous run, the runs' sums are
+// scanned across the block, then each thread writes its run's offsets.
+__device__ void block_scan_to(const int32_t *cnt, int n, int32_t *out, int32_t *scratch) {
+  const int per = (n + blockDim.x - 1) / blockDim.x;
+  const int lo = min(n, static_cast<int>(threadIdx.x) * per), hi = min(n, lo + per);
+  int32_t run = 0;
+  for (int i = lo; i < hi; ++i) run += cnt[i];
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  int32_t x = run;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int32_t y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) scratch[wid] = x;
+  __syncthreads();
+  if (wid == 0) {
+    int32_t t = lane < static_cast<int>(blockDim.x >> 5) ? scratch[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int32_t y = __shfl_up_sync(0xffffffffu, t, o);
+      if (lane >= o) t += y;
+    }
+    scratch[lane] = t;  // inclusive over warps
+  }
+  __syncthreads();
+  int32_t acc = (wid > 0 ? scratch[wid - 1] : 0) + x - run;
+  for (int i = lo; i < hi; ++i) {
+    out[i] = acc;
+    acc += cnt[i];
+  }
+  if (threadIdx.x == blockDim.x - 1) out[n] = acc;
+  __syncthreads();
+}
+
+struct FusedPlanArgs {
+  ClassifyArgs ca;  // row_cnt / col_cnt unused: the counts live in shared memory
+  int order;
+  int32_t *perm, *rank, *row_ptr, *col_ptr, *col_rank;
+  uint32_t *row_ent, *col_ent, *hdr;
+  uint32_t sig_flags, sig_window, sig_n_seqs, sig_dilation;
+};
+
+// The whole plan in one block, for small block maps without segment or varlen
+// ids: header reset, tile classes with row and column counts, both CSR scans,
+// pi (closed form or greedy), the row lists with rank(m, n), and the column
+// lists sorted by (rank, m) (a warp per column, ranking its entries in shared
+// memory).  Same results as the multi-kernel path.
+__global__ void __launch_bounds__(1024, 1) k_plan_fused(FusedPlanArgs pa) {
+  extern __shared__ int32_t shm[];
+  const ClassifyArgs &a = pa.ca;
+  const int B = a.B, nM = a.nM, nN = a.nN, BnM = B * nM, BnN = B * nN;
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  int32_t *rcnt = shm;                 // [BnM]
+  int32_t *ccnt = rcnt + BnM;          // [BnN]
+  int32_t *scratch = ccnt + BnN;       // [32]
+  int32_t *gw = scratch + 32;          // [nN] greedy presumed waits
+  // [nw][nM] column keys, on an 8-byte boundary after the int32 arrays
+  unsigned long long *keys =
+      reinterpret_cast<unsigned long long *>(shm + ((BnM + BnN + 32 + nN + 1) & ~1));
+  if (threadIdx.x < kHdrWords) pa.hdr[threadIdx.x] = 0u;
+  for (int i = threadIdx.x; i < BnN; i += blockDim.x) ccnt[i] = 0;
+  __syncthreads();
+  // tile classes, a warp per row block
+  for (int row = wid; row < BnM; row += nw) {
+    const int b = row / nM, m = row % nM;
+    uint8_t *crow = a.cls + static_cast<int64_t>(row) * nN;
+    int cnt = 0;
+    for (int n0 = 0; n0 < nN; n0 += 32) {
+      const int n = n0 + lane;
+      uint8_t c = BSA_TILE_EMPTY;
+      bool exact = true;
+      if (n < nN) c = tile_class(a, b, m, n, &exact);
+      uint32_t todo = __ballot_sync(0xffffffffu, c == BSA_TILE_PARTIAL && !exact);
+      while (todo != 0u) {
+        const int src = __ffs(todo) - 1;
+        todo &= todo - 1u;
+        const uint8_t rc = refine_tile(a, b, m, n0 + src, lane);
+        if (lane == src) c = rc;
+      }
+      if (n < nN) {
+        crow[n] = c;
+        if (c != BSA_TILE_EMPTY) atomicAdd(ccnt + b * nN + n, 1);
+      }
+      cnt += __popc(__ballot_sync(0xffffffffu, c != BSA_TILE_EMPTY));
+    }
+    if (lane == 0) rcnt[row] = cnt;
+  }
+  __syncthreads();
+  block_scan_to(rcnt, BnM, pa.row_ptr, scratch);
+  block_scan_to(ccnt, BnN, pa.col_ptr, scratch);
+  // pi
+  const bool in_ws = order_in_workspace(pa.order);
+  if (pa.order == BSA_ORDER_GREEDY) {
+    constexpr int32_t kPlaced = 0x7fffffff;
+    __shared__ unsigned long long red[32];
+    __shared__ int chosen;
+    for (int n = threadIdx.x; n < nN; n += blockDim.x) gw[n] = 0;
+    __syncthreads();
+    for (int step = 0; step < nN; ++step) {
+      unsigned long long best = ~0ull;
+      for (int n = threadIdx.x; n < nN; n += blockDim.x) {
+        const int32_t w = gw[n];
+        if (w != kPlaced) {
+          const unsigned long long key = (static_cast<unsigned long long>(w) << 32) | static_cast<unsigned>(n);
+          best = key < best ? key : best;
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const unsigned long long y = __shfl_xor_sync(0xffffffffu, best, o);
+        best = y < best ? y : best;
+      }
+      if (lane == 0) red[wid] = best;
+      __syncthreads();
+      if (wid == 0) {
+        unsigned long long v = lane < nw ? red[lane] : ~0ull;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          const unsigned long long y = __shfl_xor_sync(0xffffffffu, v, o);
+          v = y < v ? y : v;
+        }
+        if (lane == 0) {
+          const int c = static_cast<int>(v & 0xffffffffull);
+          chosen = c;
+          pa.perm[step] = c;
+          gw[c] = kPlaced;
+        }
+      }
+      __syncthreads();
+      const int c = chosen;
+      for (int bm = wid; bm < BnM; bm += nw) {
+        const uint8_t *crow = a.cls + static_cast<int64_t>(bm) * nN;
+        if (crow[c] == BSA_TILE_EMPTY) continue;
+        for (int n = lane; n < nN; n += 32)
+          if (crow[n] != BSA_TILE_EMPTY && gw[n] != kPlaced) atomicAdd(gw + n, 1);
+      }
+      __syncthreads();
+    }
+  } else if (!in_ws) {
+    for (int t = threadIdx.x; t < nN; t += blockDim.x) pa.perm[t] = closed_form_order(pa.order, t, nN);
+  }
+  __syncthreads();
+  // row lists and rank(m, n), a warp per row block
+  for (int row = wid; row < BnM; row += nw) {
+    const uint8_t *crow = a.cls + static_cast<int64_t>(row) * nN;
+    int pos = pa.row_ptr[row];
+    for (int n0 = 0; n0 < nN; n0 += 32) {
+      const int n = n0 + lane;
+      const uint8_t c = n < nN ? crow[n] : BSA_TILE_EMPTY;
+      const uint32_t bal = __ballot_sync(0xffffffffu, c != BSA_TILE_EMPTY);
+      if (c != BSA_TILE_EMPTY)
+        pa.row_ent[pos + __popc(bal & ((1u << lane) - 1u))] = n | (c == BSA_TILE_FULL ? kFullBit : 0u);
+      pos += __popc(bal);
+    }
+    int32_t *rk = pa.rank + static_cast<int64_t>(row) * nN;
+    int r = 0;
+    for (int t0 = 0; t0 < nN; t0 += 32) {
+      const int t = t0 + lane;
+      int n = -1;
+      if (t < nN) n = in_ws ? pa.perm[t] : closed_form_order(pa.order, t, nN);
+      const bool ne = n >= 0 && crow[n] != BSA_TILE_EMPTY;
+      const uint32_t bal = __ballot_sync(0xffffffffu, ne);
+      if (n >= 0) rk[n] = ne ? r + __popc(bal & ((1u << lane) - 1u)) : -1;
+      r += __popc(bal);
+    }
+  }
+  __syncthreads();
+  // column lists sorted by (rank, m), a warp per column
+  unsigned long long *mykeys = keys + static_cast<int64_t>(wid) * nM;
+  for (int bn = wid; bn < BnN; bn += nw) {
+    const int b = bn / nN, n = bn % nN;
+    int cnt = 0;
+    for (int m0 = 0; m0 < nM; m0 += 32) {
+      const int m = m0 + lane;
+      unsigned long long key = 0;
+      bool ne = false;
+      if (m < nM) {
+        const int64_t t = (static_cast<int64_t>(b) * nM + m) * nN + n;
+        const uint8_t k = a.cls[t];
+        ne = k != BSA_TILE_EMPTY;
+        if (ne)
+          key = (static_cast<unsigned long long>(pa.rank[t]) << 32) |
+                (static_cast<unsigned long long>(m) << 1) | (k == BSA_TILE_FULL ? 1ull : 0ull);
+      }
+      const uint32_t bal = __ballot_sync(0xffffffffu, ne);
+      if (ne) mykeys[cnt + __popc(bal & ((1u << lane) - 1u))] = key;
+      cnt += __popc(bal);
+    }
+    __syncwarp();
+    const int base = pa.col_ptr[bn];
+    for (int e = lane; e < cnt; e += 32) {
+      const unsigned long long ke = mykeys[e];
+      int pos = 0;
+      for (int f = 0; f < cnt; ++f) pos += mykeys[f] < ke;
+      pa.col_ent[base + pos] = static_cast<uint32_t>((ke & 0xffffffffull) >> 1) | ((ke & 1ull) ? kFullBit : 0u);
+      pa.col_rank[base + pos] = static_cast<int32_t>(ke >> 32);
+    }
+    __syncwarp();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    uint32_t *h = pa.hdr;
+    h[kHdrB] = B;
+    h[kHdrSq] = a.Sq;
+    h[kHdrSkv] = a.Skv;
+    h[kHdrFlags] = pa.sig_flags;
+    h[kHdrWindow] = pa.sig_window;
+    h[kHdrOrder] = pa.order;
+    h[kHdrNSeqs] = pa.sig_n_seqs;
+    h[kHdrDilation] = pa.sig_dilation;
+    __threadfence();
+    h[kHdrMagic] = kPlanMagic;
+  }
+}
+
+// Shared memory of k_plan_fused, and whether the fused path applies.
+inline size_t fused_plan_smem(int B, int nM, int nN) {
+  const size_t ints = (static_cast<size_t>(B) * nM + static_cast<size_t>(B) * nN + 32 + nN + 1) & ~size_t{1};
+  return sizeof(int32_t) * ints + sizeof(unsigned long long) * 32 * static_cast<size_t>(nM);
+}
+
 inline unsigned cdiv(int64_t a, int64_t b) { return static_cast<unsigned>((a + b - 1) / b); }
 
 }  // namespace
@@ -449,7 +672,49 @@ cudaError_t launch_plan(const bsa_problem &p, const bsa_mask_spec &m, const bsa_
                         const WsLayout &L, uint8_t *ws, cudaStream_t s) {
   const int B = p.B, nM = L.nM, nN = L.nN;
   uint32_t *hdr = reinterpret_cast<uint32_t *>(ws + L.status);
-  cudaError_t e = cudaMemsetAsync(hdr, 0, kHdrWords * sizeof(uint32_t), s);
+  cudaError_t e;
+  const bool ids = (m.flags & (BSA_MASK_VARLEN | BSA_MASK_SEGMENT_IDS)) != 0;
+  const int64_t tiles = static_cast<int64_t>(B) * nM * nN;
+  const size_t fsm = fused_plan_smem(B, nM, nN);
+  if (!ids && tiles <= 16384 && fsm <= 200 * 1024) {
+    // small map: everything in one block, one launch
+    int32_t *perm = reinterpret_cast<int32_t *>(ws + L.perm);
+    if (o.bwd_order == BSA_ORDER_PERM) {
+      e = cudaMemcpyAsync(perm, o.perm, sizeof(int32_t) * nN, cudaMemcpyHostToDevice, s);
+      if (e != cudaSuccess) return e;
+    }
+    FusedPlanArgs pa{};
+    ClassifyArgs &ca = pa.ca;
+    ca.B = B; ca.nM = nM; ca.nN = nN; ca.Sq = p.Sq; ca.Skv = p.Skv;
+    ca.flags = m.flags;
+    ca.window = m.window;
+    ca.dilation = m.dilation;
+    ca.kv_valid_len = m.kv_valid_len;
+    ca.prefix_len = (m.flags & BSA_MASK_PREFIX_LM) ? m.prefix_len : nullptr;
+    ca.cls = ws + L.tile_class;
+    pa.order = o.bwd_order;
+    pa.perm = perm;
+    pa.rank = reinterpret_cast<int32_t *>(ws + L.rank);
+    pa.row_ptr = reinterpret_cast<int32_t *>(ws + L.row_ptr);
+    pa.col_ptr = reinterpret_cast<int32_t *>(ws + L.col_ptr);
+    pa.col_rank = reinterpret_cast<int32_t *>(ws + L.col_rank);
+    pa.row_ent = reinterpret_cast<uint32_t *>(ws + L.row_ent);
+    pa.col_ent = reinterpret_cast<uint32_t *>(ws + L.col_ent);
+    pa.hdr = hdr;
+    pa.sig_flags = m.flags;
+    pa.sig_window = static_cast<uint32_t>(m.window);
+    pa.sig_n_seqs = static_cast<uint32_t>(m.n_seqs);
+    pa.sig_dilation = static_cast<uint32_t>(m.dilation);
+    if (fsm > 48 * 1024) {
+      e = cudaFuncSetAttribute(k_plan_fused, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(fsm));
+      if (e != cudaSuccess) return e;
+    }
+    k_plan_fused<<<1, 1024, fsm, s>>>(pa);
+    count_launch();
+    return cudaGetLastError();
+  }
+  e = cudaMemsetAsync(hdr, 0, kHdrWords * sizeof(uint32_t), s);
   if (e != cudaSuccess) return e;
 
   const int4 *qblk = nullptr, *kblk = nullptr;

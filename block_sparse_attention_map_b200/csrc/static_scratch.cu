@@ -66,5 +66,6 @@ extern "C" bsa_status bsa_attn_fwd_static_scratch(const bsa_problem *prob,
   if (opt != nullptr) o = *opt;
   o.plan_ready = 0;
   o.bound_ready = 0;
+  o.keep_o_residual = 0;  // no backward shares this scratch
   return bsa_attn_fwd(prob, mask, &o, q, k, v, out, lse, ws, kStaticScratchBytes, stream);
 }

@@ -182,7 +182,13 @@ typedef struct bsa_options {
                                   q and k; 0: bsa_attn_fwd computes them first      */
   int32_t bound_mode;          /* BSA_BOUND_*; SMOOTHED with kmax_override or with
                                   H_kv*D > 24576 is rejected                        */
-  int32_t reserved;
+  int32_t keep_o_residual;     /* 1: bsa_attn_fwd also writes what the bf16 rounding
+                                  of O dropped (fp32 O - bf16 O, as bf16) into the
+                                  backward part of the workspace, which must then be
+                                  sized with_backward, and bsa_bwd_preprocess forms
+                                  Delta = rowsum(dO o (O + that residual)), exact to
+                                  fp32 O; 0: Delta from the bf16 O alone.  Both calls
+                                  must get the same value.                         */
 } bsa_options;
 
 /* Where the plan and the scratch arrays sit inside the workspace (byte offsets),
@@ -207,6 +213,7 @@ typedef struct bsa_workspace_view {
   size_t off_sem;              /* int32  [B, H, nM]   dQ semaphores                  */
   size_t off_kbar;             /* fp32   [B, H_kv, D] k-smoothing center             */
   size_t off_qdot;             /* fp32   [B, H, Sq]   q_i . center                   */
+  size_t off_o_resid;          /* bf16   [B, Sq, H, D] O - bf16(O) (keep_o_residual)  */
   int32_t nM, nN;
 } bsa_workspace_view;
 
@@ -275,7 +282,7 @@ BSA_API bsa_status bsa_bwd_main(const bsa_problem *prob, const bsa_mask_spec *ma
                                 const void *v, const void *dout, const float *lse, void *dk,
                                 void *dv, void *ws, size_t ws_bytes, bsa_stream_t stream);
 
-/* a7: dQ = bf16(dQ accumulator). */
+/* a7: dQ = bf16(dQ accumulator); zero rows for q-blocks no kv column reaches. */
 BSA_API bsa_status bsa_bwd_convert(const bsa_problem *prob, const bsa_mask_spec *mask,
                                    void *dq, void *ws, size_t ws_bytes, bsa_stream_t stream);
 
