@@ -333,6 +333,13 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
           if (!last && !issue_s(ec + 1)) { stop = true; break; }
           if (!wd.wait(&bars[L::bDSReady], ec & 1)) { stop = true; break; }
           tc_fence_after();
+          // dQ_m part = dS K_n   (dS read MN-major from the dS^T tile), first: the
+          // dQ warps' read of it gates the next dP^T, which shares its columns
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ss(T_DP, sw128_desc(ds_addr + kk * 2048, 16384, 1024),
+                   sw128_desc(k_addr + kk * 2048, 16384, 1024), kIdQ, kk > 0);
+          mma_commit(&bars[L::bDQFull]);
           // dK += dS^T Q_m
           const uint32_t q_addr = smem_u32(sm + L::kQ + qs * kTB);
 #pragma unroll
@@ -342,12 +349,6 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
                    sw128_desc(q_addr + kk * 2048, 16384, 1024), kIdKV, (!first || kk > 0) ? 1u : 0u);
           }
           mma_commit(&bars[L::bQEmpty + qs]);
-          // dQ_m part = dS K_n   (dS read MN-major from the dS^T tile)
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ss(T_DP, sw128_desc(ds_addr + kk * 2048, 16384, 1024),
-                   sw128_desc(k_addr + kk * 2048, 16384, 1024), kIdQ, kk > 0);
-          mma_commit(&bars[L::bDQFull]);
           mma_commit(&bars[L::bDSFree]);
           if (last) {
             mma_commit(&bars[L::bDKVFull]);
@@ -521,21 +522,24 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
         if (ec >= 1 && !wwait(&bars[L::bDSFree], (ec - 1) & 1)) { stop = true; break; }
         if (!wwait(&bars[L::bDPFull], ec & 1)) { stop = true; break; }
         tc_fence_after();
+        // four 16-column pieces; the next piece's TMEM load is in flight while
+        // this one is computed (a wait covers every load issued before it)
+        uint32_t dpb[2][16];
+        tmem_ld16(T_DP + lane_off + 64 * half, dpb[0]);
+        tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          uint32_t dp[32];
-          tmem_ld32(T_DP + lane_off + 64 * half + 32 * c, dp);
-          tmem_wait_ld();
-          uint32_t dk2[16];
+        for (int sc = 0; sc < 4; ++sc) {
+          if (sc + 1 < 4) tmem_ld16(T_DP + lane_off + 64 * half + 16 * (sc + 1), dpb[(sc + 1) & 1]);
+          const uint32_t *dp = dpb[sc & 1];
+          uint32_t dk2[8];
 #pragma unroll
-          for (int q4 = 0; q4 < 8; ++q4) {
-            const float4 nd4 = nd4p[8 * c + q4];
+          for (int q4 = 0; q4 < 4; ++q4) {
+            const float4 nd4 = nd4p[4 * sc + q4];
 #pragma unroll
             for (int h2 = 0; h2 < 2; ++h2) {
               const int e0 = 4 * q4 + 2 * h2;
               const float2 nd = h2 ? make_float2(nd4.z, nd4.w) : make_float2(nd4.x, nd4.y);
-              const uint32_t pp = pk[16 * c + (e0 >> 1)];
-              const float2 pv = unpack_f16x2(pp);
+              const float2 pv = unpack_f16x2(pk[8 * sc + (e0 >> 1)]);
               const float2 dd = __fadd2_rn(
                   make_float2(__uint_as_float(dp[e0]), __uint_as_float(dp[e0 + 1])), nd);
               const float2 dsv = __fmul2_rn(pv, dd);
@@ -543,13 +547,14 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
             }
           }
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int chunk = 8 * half + 4 * c + u;  // 0..15 over 128 queries
+          for (int u = 0; u < 2; ++u) {
+            const int chunk = 8 * half + 2 * sc + u;  // 0..15: 8 queries each
             const int sub = chunk >> 3, cw = chunk & 7;
             uint8_t *dst = ds_tile + sub * 16384 + r * 128 + ((cw ^ (r & 7)) << 4);
             *reinterpret_cast<int4 *>(dst) =
                 make_int4(dk2[4 * u], dk2[4 * u + 1], dk2[4 * u + 2], dk2[4 * u + 3]);
           }
+          if (sc + 1 < 4) tmem_wait_ld();
         }
         fence_proxy_async_smem();
         tc_fence_before();
@@ -616,15 +621,16 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
         const uint32_t rank = static_cast<uint32_t>(p.col_rank[e]);
         if (!wwait(&bars[L::bDQFull], ec & 1)) { stop = true; break; }
         tc_fence_after();
+        // every column load in flight at once, one wait: the columns are
+        // handed back to the next dP^T as early as possible
+        uint32_t raw[D];
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c)
+          tmem_ld32(T_DP + lane_off + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&raw[32 * c]));
+        tmem_wait_ld();
         float acc[D];
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t a[32];
-          tmem_ld32(T_DP + lane_off + 32 * c, a);
-          tmem_wait_ld();
-#pragma unroll
-          for (int q = 0; q < 32; ++q) acc[32 * c + q] = __uint_as_float(a[q]) * p.scale;
-        }
+        for (int q = 0; q < D; ++q) acc[q] = __uint_as_float(raw[q]) * p.scale;
         tc_fence_before();
         mbar_arrive(&bars[L::bDQFree]);
         uint32_t *sem = p.sem + bh * p.nM + m;
@@ -721,36 +727,49 @@ __global__ void __launch_bounds__(256) k_bwd_delta(const __nv_bfloat16 *__restri
 }
 
 // ---------------------------------------------------------------- a7: dQ convert
-// A thread per (row, 4 columns) of a q-block: it reads one float4 of the
-// interleaved accumulator [B, H, nM, D/4, 128, 4] (consecutive threads, rows
-// of one column group: contiguous) and writes 4 bf16 of the row; the row's
-// other pieces come from the neighbouring column groups of the same warp loop,
-// so the L2 merges them into whole sectors.  Q-blocks that no kv column
+// A block per 32 rows of one q-block: the rows' slice of the interleaved
+// accumulator [B, H, nM, D/4, 128, 4] (32 consecutive float4 per column group:
+// contiguous) is read with every thread keeping its loads in flight, staged in
+// shared memory, and written as whole bf16 rows.  Q-blocks that no kv column
 // reaches get zeros.
 template <int D>
 __global__ void __launch_bounds__(256) k_dq_convert(const float *__restrict__ acc, int B, int H,
                                                     int Sq, int nM, const int32_t *__restrict__ row_ptr,
                                                     __nv_bfloat16 *__restrict__ dq,
                                                     int64_t sb, int64_t ss, int64_t sh) {
-  constexpr int kC = D / 4;  // float4 column groups per row
-  const int64_t total = static_cast<int64_t>(B) * H * nM * kC * kTile;
-  for (int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; t < total;
-       t += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int r = static_cast<int>(t % kTile);
-    const int64_t rest = t / kTile;
-    const int c = static_cast<int>(rest % kC);
-    const int64_t bhm = rest / kC;
-    const int m = static_cast<int>(bhm % nM);
-    const int64_t bh = bhm / nM;
-    const int b = static_cast<int>(bh / H), h = static_cast<int>(bh % H);
-    const int i = m * kTile + r;
+  constexpr int kC = D / 4, kRows = 32, kLD = D + 4;
+  constexpr int kPer = kC * kRows / 256;  // float4 loads per thread
+  __shared__ __align__(16) float tile[kRows * kLD];
+  const int64_t bhm = blockIdx.x / (kTile / kRows);
+  const int r0 = static_cast<int>(blockIdx.x % (kTile / kRows)) * kRows;
+  const int m = static_cast<int>(bhm % nM);
+  const int64_t bh = bhm / nM;
+  const int b = static_cast<int>(bh / H), h = static_cast<int>(bh % H);
+  const bool empty = row_ptr[b * nM + m + 1] == row_ptr[b * nM + m];
+  const float4 *src = reinterpret_cast<const float4 *>(acc) + bhm * kC * kTile;
+  float4 v[kPer];
+#pragma unroll
+  for (int u = 0; u < kPer; ++u) {
+    const int idx = threadIdx.x + u * 256;  // (column group, row) with rows fastest
+    const int c = idx / kRows, rr = idx % kRows;
+    v[u] = empty ? make_float4(0.f, 0.f, 0.f, 0.f) : __ldcs(src + c * kTile + r0 + rr);
+  }
+#pragma unroll
+  for (int u = 0; u < kPer; ++u) {
+    const int idx = threadIdx.x + u * 256;
+    const int c = idx / kRows, rr = idx % kRows;
+    *reinterpret_cast<float4 *>(tile + rr * kLD + 4 * c) = v[u];
+  }
+  __syncthreads();
+  constexpr int kCPR = D / 8;  // 16-byte output pieces per row
+  for (int idx = threadIdx.x; idx < kRows * kCPR; idx += 256) {
+    const int rr = idx / kCPR, j = idx % kCPR;
+    const int i = m * kTile + r0 + rr;
     if (i >= Sq) continue;
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (row_ptr[b * nM + m + 1] != row_ptr[b * nM + m]) v = __ldcs(reinterpret_cast<const float4 *>(acc) + t);
-    uint2 w;
-    w.x = pack_bf16x2(v.x, v.y);
-    w.y = pack_bf16x2(v.z, v.w);
-    *reinterpret_cast<uint2 *>(dq + b * sb + static_cast<int64_t>(i) * ss + h * sh + 4 * c) = w;
+    const float *t = tile + rr * kLD + 8 * j;
+    const int4 w = make_int4(pack_bf16x2(t[0], t[1]), pack_bf16x2(t[2], t[3]),
+                             pack_bf16x2(t[4], t[5]), pack_bf16x2(t[6], t[7]));
+    *reinterpret_cast<int4 *>(dq + b * sb + static_cast<int64_t>(i) * ss + h * sh + 8 * j) = w;
   }
 }
 
@@ -873,9 +892,7 @@ cudaError_t launch_bwd_main(const bsa_problem &p, const MaskParams &mp, const bs
 cudaError_t launch_bwd_convert(const bsa_problem &p, void *dq, const WsLayout &L, uint8_t *ws,
                                cudaStream_t s) {
   const float *acc = reinterpret_cast<const float *>(ws + L.dq_accum);
-  const int64_t total = static_cast<int64_t>(p.B) * p.H * L.nM * (p.D / 4) * kTile;
-  const unsigned blocks = static_cast<unsigned>(
-      std::min<int64_t>((total + 255) / 256, static_cast<int64_t>(sm_count_bwd()) * 8));
+  const unsigned blocks = static_cast<unsigned>(static_cast<int64_t>(p.B) * p.H * L.nM * (kTile / 32));
   const int32_t *row_ptr = reinterpret_cast<const int32_t *>(ws + L.row_ptr);
   __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(dq);
   if (p.D == 64)

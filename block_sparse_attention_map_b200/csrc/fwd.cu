@@ -683,15 +683,16 @@ __global__ void __launch_bounds__(256) k_row_norms(const NormArgs a) {
     const int4 *src = reinterpret_cast<const int4 *>(x + b * sb + static_cast<int64_t>(row) * ss + hh * sh);
     const float *c = cen + (is_key ? hh : hh / grp) * kLD;
     float acc = 0.f, dot = 0.f;
+    // the whole vector's loads first, then the arithmetic
+    int4 w[kC];
+#pragma unroll
+    for (int u = 0; u < kC; ++u) w[u] = __ldg(src + u);
 #pragma unroll
     for (int c0 = 0; c0 < kC; c0 += kU) {
-      int4 w[kU];
-#pragma unroll
-      for (int u = 0; u < kU; ++u) w[u] = __ldg(src + c0 + u);
 #pragma unroll
       for (int u = 0; u < kU; ++u) {
-        const uint32_t xw[4] = {static_cast<uint32_t>(w[u].x), static_cast<uint32_t>(w[u].y),
-                                static_cast<uint32_t>(w[u].z), static_cast<uint32_t>(w[u].w)};
+        const uint32_t xw[4] = {static_cast<uint32_t>(w[c0 + u].x), static_cast<uint32_t>(w[c0 + u].y),
+                                static_cast<uint32_t>(w[c0 + u].z), static_cast<uint32_t>(w[c0 + u].w)};
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           float2 f = unpack_bf16x2(xw[q]);
