@@ -487,14 +487,20 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
         if (!wwait(&bars[L::bSFull], ec & 1)) { stop = true; break; }
         tc_fence_after();
         uint32_t pk[32];
+        // four 16-column pieces, the next one's TMEM load in flight while this
+        // one is computed
+        uint32_t sb[2][16];
+        tmem_ld16(T_S + lane_off + 64 * half, sb[0]);
+        tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          uint32_t s[32], pb[16];
-          tmem_ld32(T_S + lane_off + 64 * half + 32 * c, s);
-          tmem_wait_ld();
+        for (int sc = 0; sc < 4; ++sc) {
+          if (sc + 1 < 4) tmem_ld16(T_S + lane_off + 64 * half + 16 * (sc + 1), sb[(sc + 1) & 1]);
+          const uint32_t *s = sb[sc & 1];
+          const uint32_t bits = allow[sc >> 1] >> (16 * (sc & 1));
+          uint32_t pb[8];
 #pragma unroll
-          for (int q4 = 0; q4 < 8; ++q4) {
-            const float4 nl4 = nl4p[8 * c + q4];
+          for (int q4 = 0; q4 < 4; ++q4) {
+            const float4 nl4 = nl4p[4 * sc + q4];
 #pragma unroll
             for (int h2 = 0; h2 < 2; ++h2) {
               const int e0 = 4 * q4 + 2 * h2;
@@ -503,16 +509,17 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
                   make_float2(__uint_as_float(s[e0]), __uint_as_float(s[e0 + 1])), sc2, nl);
               float p0 = fast_exp2(tt.x), p1 = fast_exp2(tt.y);
               if (!full) {
-                p0 = ((allow[c] >> e0) & 1u) ? p0 : 0.f;
-                p1 = ((allow[c] >> (e0 + 1)) & 1u) ? p1 : 0.f;
+                p0 = ((bits >> e0) & 1u) ? p0 : 0.f;
+                p1 = ((bits >> (e0 + 1)) & 1u) ? p1 : 0.f;
               }
               pb[e0 >> 1] = pack_bf16x2(p0, p1);
-              pk[16 * c + (e0 >> 1)] = pack_f16x2(p0, p1);
+              pk[8 * sc + (e0 >> 1)] = pack_f16x2(p0, p1);
             }
           }
-          // P^T chunk -> TMEM columns [16c, 16c+16) of this half's region: S^T
+          // P^T piece -> TMEM columns [8sc, 8sc+8) of this half's region: S^T
           // columns this warp has already read
-          tmem_st16(t_p + 16 * c, pb);
+          tmem_st8(t_p + 8 * sc, pb);
+          if (sc + 1 < 4) tmem_wait_ld();
         }
         tmem_wait_st();
         tc_fence_before();

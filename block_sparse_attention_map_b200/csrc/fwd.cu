@@ -277,24 +277,12 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
         if (stop) break;
         bool first[2] = {true, true};
         UnionWalk uw{p.row_ent, {w.rs[0], w.rs[1]}, {w.re[0], w.re[1]}};
-        // Q_x is read by the S MMAs only: once group x's last S of the unit is
-        // issued, its completion frees the buffer for the next unit's Q_x,
-        // which then loads while this unit's last softmax, PV and epilogue run
-        auto release_q = [&](int x) {
-          if (uw.i[x] >= uw.e[x]) {
-            mma_commit(&bars[L::bQEmpty + x]);
-            ++uq[x];
-          }
-        };
         int n;
         bool in_cur[2], in_nxt[2];
         uw.next(n, in_cur[0], in_cur[1]);
         uint32_t kv_cur = kv;
         for (int x = 0; x < 2 && !stop; ++x)
-          if (in_cur[x]) {
-            if (!issue_s(x, kv_cur)) stop = true;
-            else release_q(x);
-          }
+          if (in_cur[x] && !issue_s(x, kv_cur)) stop = true;
         if (stop) break;
         mma_commit(&bars[L::bKEmpty + kv_cur % NK]);
         for (;;) {
@@ -317,10 +305,7 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
               ++tcount[x];
             }
             // the next S of this group as soon as its P has been consumed
-            if (more && in_nxt[x]) {
-              if (!issue_s(x, kv_nxt)) { stop = true; break; }
-              release_q(x);
-            }
+            if (more && in_nxt[x] && !issue_s(x, kv_nxt)) { stop = true; break; }
           }
           if (stop) break;
           mma_commit(&bars[L::bVEmpty + kv_cur % NV]);
@@ -332,6 +317,13 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
         }
         if (stop) break;
         kv = kv_cur + 1;
+        // Q buffers go back to the producer with the unit's last MMAs (releasing
+        // them right after each group's last S measured slower)
+        for (int x = 0; x < 2; ++x)
+          if (has[x]) {
+            mma_commit(&bars[L::bQEmpty + x]);
+            ++uq[x];
+          }
       }
       // every tcgen05 op this thread issued is complete before TMEM is freed
       mma_commit(&bars[L::bFinal]);
@@ -484,31 +476,36 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
         const float mu = (m_ref == -INFINITY) ? 0.f : m_ref;
         const float2 sc2 = make_float2(p.scale_log2, p.scale_log2), nmu = make_float2(-mu, -mu);
         float2 rs2 = make_float2(0.f, 0.f), rr2 = make_float2(0.f, 0.f);
+        // eight 16-column pieces; the next piece's TMEM load is in flight while
+        // this one is computed (a wait covers every load issued before it)
+        uint32_t svb[2][16];
+        tmem_ld16(t_s, svb[0]);
+        tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t sv[32];
-          tmem_ld32(t_s + 32 * c, sv);
-          tmem_wait_ld();
-          uint32_t pk[16];
+        for (int sc = 0; sc < 8; ++sc) {
+          if (sc + 1 < 8) tmem_ld16(t_s + 16 * (sc + 1), svb[(sc + 1) & 1]);
+          const uint32_t *sv = svb[sc & 1];
+          const uint32_t bits = allow[sc >> 1] >> (16 * (sc & 1));
+          uint32_t pk[8];
 #pragma unroll
-          for (int q = 0; q < 16; ++q) {
+          for (int q = 0; q < 8; ++q) {
             const float2 t = __ffma2_rn(
                 make_float2(__uint_as_float(sv[2 * q]), __uint_as_float(sv[2 * q + 1])), sc2, nmu);
             float p0 = fast_exp2(t.x), p1 = fast_exp2(t.y);
             if (!full) {
-              p0 = ((allow[c] >> (2 * q)) & 1u) ? p0 : 0.f;
-              p1 = ((allow[c] >> (2 * q + 1)) & 1u) ? p1 : 0.f;
+              p0 = ((bits >> (2 * q)) & 1u) ? p0 : 0.f;
+              p1 = ((bits >> (2 * q + 1)) & 1u) ? p1 : 0.f;
             }
             pk[q] = pack_bf16x2(p0, p1);
             // two row sums: l over the exact weights (for LSE) and l_r over the
             // bf16-rounded weights the PV product uses (normalising O by l_r
             // makes numerator and denominator carry the same rounding)
             rs2 = __fadd2_rn(rs2, make_float2(p0, p1));
-            rr2 = __fadd2_rn(rr2, make_float2(__uint_as_float(pk[q] << 16),
-                                              __uint_as_float(pk[q] & 0xffff0000u)));
+            rr2 = __fadd2_rn(rr2, unpack_bf16x2(pk[q]));
           }
-          // P chunk c -> TMEM columns [16c, 16c+16): only S columns already read
-          tmem_st16(t_s + 16 * c, pk);
+          // P piece -> TMEM columns [8sc, 8sc+8): only S columns already read
+          tmem_st8(t_s + 8 * sc, pk);
+          if (sc + 1 < 8) tmem_wait_ld();
         }
         const float rowsum = rs2.x + rs2.y, rowsum_r = rr2.x + rr2.y;
         l += rowsum;
@@ -646,11 +643,27 @@ __global__ void __launch_bounds__(256) k_key_sums(const NormArgs a) {
   }
 }
 
+// k-smoothing, second pass: the centers c = sum * 2^-20 / (valid keys).
+template <int D>
+__global__ void __launch_bounds__(256) k_key_centers(const NormArgs a) {
+  const int64_t n = static_cast<int64_t>(a.B) * a.Hk * D;
+  for (int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; t < n;
+       t += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int b = static_cast<int>(t / (static_cast<int64_t>(a.Hk) * D));
+    const double inv = 1.0 / (static_cast<double>(kFixScale) * max(1, a.kcount[b]));
+    a.kbar[t] = static_cast<float>(static_cast<double>(a.ksum[t]) * inv);
+  }
+}
+
+// D/32 threads per (row, head) vector, each with four 16-byte pieces in
+// flight; a block takes kVPB consecutive vectors of one batch row (rows are
+// contiguous over heads).  Per-head maxima are reduced in shared memory first,
+// then one global atomic per head and block.
 template <int D>
 __global__ void __launch_bounds__(256) k_row_norms(const NormArgs a) {
-  constexpr int kC = D / 8, kU = 4, kLD = D + 1;  // padded center rows: no bank conflicts
-  extern __shared__ unsigned int smax[];  // [H], then the centers [Hk][D + 1] (k-smoothing)
-  float *cen = reinterpret_cast<float *>(smax + a.H);
+  constexpr int kT = D / 32;          // threads per vector
+  constexpr int kVPB = 256 / kT;      // vectors per block
+  extern __shared__ unsigned int smax[];  // [H]
   __shared__ bool last_block;
   const int is_key = !a.only_q && blockIdx.y == 0;
   const __nv_bfloat16 *x = is_key ? a.k : a.q;
@@ -664,53 +677,47 @@ __global__ void __launch_bounds__(256) k_row_norms(const NormArgs a) {
   const int bpb = static_cast<int>(gridDim.x / a.B);  // blocks per batch row
   const int b = static_cast<int>(blockIdx.x) / bpb, blk = static_cast<int>(blockIdx.x) % bpb;
   for (int h = threadIdx.x; h < H; h += blockDim.x) smax[h] = 0u;
-  if (a.center) {
-    // c = (fixed-point sum) * 2^-20 / (valid keys), the same in every block
-    const double inv = 1.0 / (static_cast<double>(kFixScale) * max(1, a.kcount[b]));
-    const long long *ksum = a.ksum + static_cast<int64_t>(b) * a.Hk * D;
-    const bool write = is_key && blk == 0;
-    for (int t = threadIdx.x; t < a.Hk * D; t += blockDim.x) {
-      const float c = static_cast<float>(static_cast<double>(ksum[t]) * inv);
-      cen[(t / D) * kLD + t % D] = c;
-      if (write) a.kbar[static_cast<int64_t>(b) * a.Hk * D + t] = c;
-    }
-  }
   __syncthreads();
-  const int64_t nvec = static_cast<int64_t>(S) * Hx;
-  for (int64_t v = static_cast<int64_t>(blk) * blockDim.x + threadIdx.x; v < nvec;
-       v += static_cast<int64_t>(bpb) * blockDim.x) {
-    const int row = static_cast<int>(v / Hx), hh = static_cast<int>(v % Hx);
-    const int4 *src = reinterpret_cast<const int4 *>(x + b * sb + static_cast<int64_t>(row) * ss + hh * sh);
-    const float *c = cen + (is_key ? hh : hh / grp) * kLD;
-    float acc = 0.f, dot = 0.f;
-    // the whole vector's loads first, then the arithmetic
-    int4 w[kC];
+  const int64_t v = static_cast<int64_t>(blk) * kVPB + threadIdx.x / kT;
+  const int t = threadIdx.x % kT;
+  const bool in = v < static_cast<int64_t>(S) * Hx;  // no early return: shuffles below
+  const int row = in ? static_cast<int>(v / Hx) : 0, hh = in ? static_cast<int>(v % Hx) : 0;
+  float acc = 0.f, dot = 0.f;
+  if (in) {
+    const int4 *src = reinterpret_cast<const int4 *>(x + b * sb + static_cast<int64_t>(row) * ss + hh * sh) + 4 * t;
+    int4 w[4];
 #pragma unroll
-    for (int u = 0; u < kC; ++u) w[u] = __ldg(src + u);
+    for (int u = 0; u < 4; ++u) w[u] = __ldg(src + u);
+    const float *c = a.center ? a.kbar + (static_cast<int64_t>(b) * a.Hk + (is_key ? hh : hh / grp)) * D + 32 * t
+                              : nullptr;
 #pragma unroll
-    for (int c0 = 0; c0 < kC; c0 += kU) {
+    for (int u = 0; u < 4; ++u) {
+      const uint32_t xw[4] = {static_cast<uint32_t>(w[u].x), static_cast<uint32_t>(w[u].y),
+                              static_cast<uint32_t>(w[u].z), static_cast<uint32_t>(w[u].w)};
 #pragma unroll
-      for (int u = 0; u < kU; ++u) {
-        const uint32_t xw[4] = {static_cast<uint32_t>(w[c0 + u].x), static_cast<uint32_t>(w[c0 + u].y),
-                                static_cast<uint32_t>(w[c0 + u].z), static_cast<uint32_t>(w[c0 + u].w)};
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          float2 f = unpack_bf16x2(xw[q]);
-          const int d = 8 * (c0 + u) + 2 * q;
-          if (a.center) {
-            if (is_key) {
-              f.x -= c[d];
-              f.y -= c[d + 1];
-            } else {
-              dot = fmaf(f.x, c[d], dot);
-              dot = fmaf(f.y, c[d + 1], dot);
-            }
+      for (int q = 0; q < 4; ++q) {
+        float2 f = unpack_bf16x2(xw[q]);
+        if (c != nullptr) {
+          const float2 cc = *reinterpret_cast<const float2 *>(c + 8 * u + 2 * q);
+          if (is_key) {
+            f.x -= cc.x;
+            f.y -= cc.y;
+          } else {
+            dot = fmaf(f.x, cc.x, dot);
+            dot = fmaf(f.y, cc.y, dot);
           }
-          acc = fmaf(f.x, f.x, acc);
-          acc = fmaf(f.y, f.y, acc);
         }
+        acc = fmaf(f.x, f.x, acc);
+        acc = fmaf(f.y, f.y, acc);
       }
     }
+  }
+#pragma unroll
+  for (int o = kT / 2; o > 0; o >>= 1) {
+    acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    dot += __shfl_xor_sync(0xffffffffu, dot, o);
+  }
+  if (in && t == 0) {
     const float nrm = sqrtf(acc);
     bool valid = true;
     if (is_key) {
@@ -744,10 +751,10 @@ __global__ void __launch_bounds__(256) k_row_norms(const NormArgs a) {
   if (!last_block) return;
   __threadfence();
   const int BH = a.B * H;
-  for (int t = threadIdx.x; t < BH; t += blockDim.x) {
-    const float km = a.kmax_override != nullptr ? a.kmax_override[t] : __ldcg(a.kmax + t);
-    a.kmax[t] = km;
-    a.gate[t] = (2.f * a.scale * __ldcg(a.qmax + t) * km <= a.limit) ? 1 : 0;
+  for (int i = threadIdx.x; i < BH; i += blockDim.x) {
+    const float km = a.kmax_override != nullptr ? a.kmax_override[i] : __ldcg(a.kmax + i);
+    a.kmax[i] = km;
+    a.gate[i] = (2.f * a.scale * __ldcg(a.qmax + i) * km <= a.limit) ? 1 : 0;
   }
   if (threadIdx.x == 0) *a.done = 0u;
 }
@@ -816,29 +823,27 @@ cudaError_t launch_fixed_m_bound(const bsa_problem &p, const MaskParams &mp,
   // kmax, qmax and the finished-block counter are adjacent: one memset
   cudaError_t e = cudaMemsetAsync(na.kmax, 0, sizeof(float) * p.B * p.H * 2 + sizeof(uint32_t), s);
   if (e != cudaSuccess) return e;
-  size_t smem = sizeof(unsigned int) * p.H;
+  const size_t smem = sizeof(unsigned int) * p.H;
   if (na.center) {
     // ksum and kcount are adjacent regions: one memset
     e = cudaMemsetAsync(ws + L.ksum, 0, L.qdot - L.ksum, s);
     if (e != cudaSuccess) return e;
     const unsigned sblocks = static_cast<unsigned>(static_cast<int64_t>(p.B) * ((p.Skv + 63) / 64));
-    if (p.D == 64) k_key_sums<64><<<sblocks, 256, 0, s>>>(na);
-    else k_key_sums<128><<<sblocks, 256, 0, s>>>(na);
-    count_launch();
-    smem += sizeof(float) * p.H_kv * (p.D + 1);
+    const unsigned cblocks = static_cast<unsigned>((static_cast<int64_t>(p.B) * p.H_kv * p.D + 255) / 256);
+    if (p.D == 64) {
+      k_key_sums<64><<<sblocks, 256, 0, s>>>(na);
+      k_key_centers<64><<<cblocks, 256, 0, s>>>(na);
+    } else {
+      k_key_sums<128><<<sblocks, 256, 0, s>>>(na);
+      k_key_centers<128><<<cblocks, 256, 0, s>>>(na);
+    }
+    count_launch(2);
   }
-  // blocks per batch row: enough for about eight blocks per SM in all
+  // blocks per batch row: 256 / (D / 32) vectors each, over the larger tensor
   const int64_t vec = static_cast<int64_t>(std::max(p.Sq * p.H, p.Skv * p.H_kv));
-  const int64_t want = std::max<int64_t>(1, (static_cast<int64_t>(sm_count()) * 4) / p.B);
-  const int bpb = static_cast<int>(std::min<int64_t>(want, (vec + 255) / 256));
+  const int64_t vpb = 256 / (p.D / 32);
+  const int bpb = static_cast<int>((vec + vpb - 1) / vpb);
   const dim3 grid(static_cast<unsigned>(p.B * bpb), na.only_q ? 1u : 2u);
-  if (smem > 48 * 1024) {
-    e = p.D == 64 ? cudaFuncSetAttribute(k_row_norms<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem))
-                  : cudaFuncSetAttribute(k_row_norms<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-  }
   if (p.D == 64) k_row_norms<64><<<grid, 256, smem, s>>>(na);
   else k_row_norms<128><<<grid, 256, smem, s>>>(na);
   count_launch();
