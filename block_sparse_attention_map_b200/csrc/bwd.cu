@@ -73,7 +73,9 @@ struct BwdSmem {
   static constexpr int kVec = kDO + NDO * kTB;   // -LSE*log2e [2][128], -Delta [2][128]
   static constexpr int kTk = kVec + 2 * 2 * kTile * 4;  // ticket ring int[2]
   static constexpr int kBar = kTk + 16;
-  static constexpr int bTkFull = 0, bTkEmpty = 2, bKVFull = 4, bKVFree = 5, bQFull = 6,
+  // kK and kV are two 32 KB buffers X[0], X[1] that swap the K and V roles
+  // from one column to the next (column c: K in X[c & 1], V in the other)
+  static constexpr int bTkFull = 0, bTkEmpty = 2, bKFull = 4, bVFull = 5, bXFree = 6, bQFull = 8,
                        bQEmpty = bQFull + NQ, bDOFull = bQEmpty + NQ, bDOEmpty = bDOFull + NDO,
                        bSFull = bDOEmpty + NDO, bDPFull = bSFull + 1, bPReady = bDPFull + 1,
                        bDSReady = bPReady + 1, bDSFree = bDSReady + 1, bDQFull = bDSFree + 1,
@@ -237,16 +239,21 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
                         m * kTile, h, k.b);
           ++q_issued;
           if (x == 0) {
-            // K_n, V_n after the first Q so that load overlaps the previous
-            // column's last MMAs
-            if (cc >= 1 && !wd.wait(&bars[L::bKVFree], (cc - 1) & 1)) { stop = true; break; }
-            mbar_arrive_expect_tx(&bars[L::bKVFull], 2 * kTB);
-            for (int c = 0; c < D / 64; ++c) {
-              tma_load_4d(sm + L::kK + c * 16384, &tk, &bars[L::bKVFull], c * 64, k.n * kTile,
-                          k.hk, k.b);
-              tma_load_4d(sm + L::kV + c * 16384, &tv, &bars[L::bKVFull], c * 64, k.n * kTile,
-                          k.hk, k.b);
-            }
+            // K_n goes where the previous column kept V, free once that
+            // column's last dP^T is done, so it loads under the previous
+            // column's last entry; V_n then goes where the previous K was,
+            // free after the previous column's last dQ
+            const int kb = cc & 1, vb = kb ^ 1;
+            if (cc >= 1 && !wd.wait(&bars[L::bXFree + kb], (cc - 1) & 1)) { stop = true; break; }
+            mbar_arrive_expect_tx(&bars[L::bKFull], kTB);
+            for (int c = 0; c < D / 64; ++c)
+              tma_load_4d(sm + L::kK + kb * kTB + c * 16384, &tk, &bars[L::bKFull], c * 64,
+                          k.n * kTile, k.hk, k.b);
+            if (cc >= 1 && !wd.wait(&bars[L::bXFree + vb], (cc - 1) & 1)) { stop = true; break; }
+            mbar_arrive_expect_tx(&bars[L::bVFull], kTB);
+            for (int c = 0; c < D / 64; ++c)
+              tma_load_4d(sm + L::kK + vb * kTB + c * 16384, &tv, &bars[L::bVFull], c * 64,
+                          k.n * kTile, k.hk, k.b);
             ++kv_issued;
           }
           if (ec >= NDO && !wd.wait(&bars[L::bDOEmpty + ds], ((ec / NDO) - 1) & 1)) { stop = true; break; }
@@ -264,18 +271,21 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
           drain_wait(&bars[L::bQFull + t % NQ], (t / NQ) & 1);
         for (uint32_t t = (do_issued > NDO ? do_issued - NDO : 0); t < do_issued; ++t)
           drain_wait(&bars[L::bDOFull + t % NDO], (t / NDO) & 1);
-        if (kv_issued > 0) drain_wait(&bars[L::bKVFull], (kv_issued - 1) & 1);
+        if (kv_issued > 0) {
+          drain_wait(&bars[L::bKFull], (kv_issued - 1) & 1);
+          drain_wait(&bars[L::bVFull], (kv_issued - 1) & 1);
+        }
       }
     }
     } else if (run && warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    // Per entry e: dV(e), S^T(e+1), dK(e), dQ(e), dP^T(e+1).  S^T(e+1) reuses the
+    // Per entry e: dV(e), S^T(e+1), dQ(e), dK(e), dP^T(e+1).  S^T(e+1) reuses the
     // columns dV(e) reads P^T from: tcgen05.mma ops issued by one thread run in
     // issue order, so it follows dV(e) without a wait and the next entry's
     // exponentials overlap this entry's dK and dQ.
     if (lane == 0) {
       uint32_t tc = 0, cc = 0, ec = 0;
-      const uint32_t k_addr = smem_u32(sm + L::kK), v_addr = smem_u32(sm + L::kV);
+      uint32_t k_addr = 0, v_addr = 0;  // this column's K and V buffers
       const uint32_t ds_addr = smem_u32(sm + L::kDS);
       auto issue_s = [&](uint32_t e_idx) -> bool {  // S^T = K_n Q_m^T
         const uint32_t qs = e_idx % NQ;
@@ -315,8 +325,15 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
         const Ticket k = decode_ticket(p, t);
         if (!k.valid) break;
         if (k.ee == k.es) continue;
-        if (!wd.wait(&bars[L::bKVFull], cc & 1)) break;
-        bool stop = !issue_s(ec) || !issue_dp(ec);
+        const int kb = cc & 1, vb = kb ^ 1;
+        k_addr = smem_u32(sm + L::kK + kb * kTB);
+        v_addr = smem_u32(sm + L::kK + vb * kTB);
+        if (!wd.wait(&bars[L::bKFull], cc & 1)) break;
+        bool stop = !issue_s(ec);
+        if (!stop && !wd.wait(&bars[L::bVFull], cc & 1)) stop = true;
+        if (!stop && !issue_dp(ec)) stop = true;
+        // V's last use is the column's last dP^T: its buffer takes the next K
+        if (!stop && k.tot == 1) mma_commit(&bars[L::bXFree + vb]);
         for (int x = 0; x < k.tot && !stop; ++x, ++ec) {
           const uint32_t qs = ec % NQ, ds = ec % NDO;
           const bool first = x == 0, last = x == k.tot - 1;
@@ -340,6 +357,8 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
             mma_ss(T_DP, sw128_desc(ds_addr + kk * 2048, 16384, 1024),
                    sw128_desc(k_addr + kk * 2048, 16384, 1024), kIdQ, kk > 0);
           mma_commit(&bars[L::bDQFull]);
+          // K's last use is the column's last dQ: its buffer takes the next V
+          if (last) mma_commit(&bars[L::bXFree + kb]);
           // dK += dS^T Q_m
           const uint32_t q_addr = smem_u32(sm + L::kQ + qs * kTB);
 #pragma unroll
@@ -352,10 +371,12 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
           mma_commit(&bars[L::bDSFree]);
           if (last) {
             mma_commit(&bars[L::bDKVFull]);
-            mma_commit(&bars[L::bKVFree]);
-          } else if (!issue_dp(ec + 1)) {
-            stop = true;
-            break;
+          } else {
+            if (!issue_dp(ec + 1)) {
+              stop = true;
+              break;
+            }
+            if (x + 1 == k.tot - 1) mma_commit(&bars[L::bXFree + vb]);
           }
         }
         if (stop) break;
