@@ -655,16 +655,14 @@ __global__ void __launch_bounds__(256) k_key_centers(const NormArgs a) {
   }
 }
 
-// D/32 threads per (row, head) vector, each with four 16-byte pieces of each
-// of kChunks vectors in flight; a block takes kChunks * kVPB consecutive
-// vectors of one batch row (rows are contiguous over heads).  Per-head maxima
-// are reduced in shared memory first, then one global atomic per head and
-// block, so few blocks pay the finishing fence.
+// D/32 threads per (row, head) vector, each with four 16-byte pieces in
+// flight; a block takes kVPB consecutive vectors of one batch row (rows are
+// contiguous over heads).  Per-head maxima are reduced in shared memory first,
+// then one global atomic per head and block.
 template <int D>
 __global__ void __launch_bounds__(256) k_row_norms(const NormArgs a) {
   constexpr int kT = D / 32;          // threads per vector
-  constexpr int kVPB = 256 / kT;      // vectors per block and chunk
-  constexpr int kChunks = 4;
+  constexpr int kVPB = 256 / kT;      // vectors per block
   extern __shared__ unsigned int smax[];  // [H]
   __shared__ bool last_block;
   const int is_key = !a.only_q && blockIdx.y == 0;
@@ -680,27 +678,16 @@ __global__ void __launch_bounds__(256) k_row_norms(const NormArgs a) {
   const int b = static_cast<int>(blockIdx.x) / bpb, blk = static_cast<int>(blockIdx.x) % bpb;
   for (int h = threadIdx.x; h < H; h += blockDim.x) smax[h] = 0u;
   __syncthreads();
+  const int64_t v = static_cast<int64_t>(blk) * kVPB + threadIdx.x / kT;
   const int t = threadIdx.x % kT;
-  const int64_t nvec = static_cast<int64_t>(S) * Hx;
-  int4 wall[kChunks][4];
-#pragma unroll
-  for (int ch = 0; ch < kChunks; ++ch) {
-    const int64_t v = (static_cast<int64_t>(blk) * kChunks + ch) * kVPB + threadIdx.x / kT;
-    if (v < nvec) {
-      const int row = static_cast<int>(v / Hx), hh = static_cast<int>(v % Hx);
-      const int4 *src = reinterpret_cast<const int4 *>(x + b * sb + static_cast<int64_t>(row) * ss + hh * sh) + 4 * t;
-#pragma unroll
-      for (int u = 0; u < 4; ++u) wall[ch][u] = __ldg(src + u);
-    }
-  }
-#pragma unroll
-  for (int ch = 0; ch < kChunks; ++ch) {
-  const int64_t v = (static_cast<int64_t>(blk) * kChunks + ch) * kVPB + threadIdx.x / kT;
-  const bool in = v < nvec;  // no early exit: shuffles below
+  const bool in = v < static_cast<int64_t>(S) * Hx;  // no early return: shuffles below
   const int row = in ? static_cast<int>(v / Hx) : 0, hh = in ? static_cast<int>(v % Hx) : 0;
   float acc = 0.f, dot = 0.f;
   if (in) {
-    const int4 *w = wall[ch];
+    const int4 *src = reinterpret_cast<const int4 *>(x + b * sb + static_cast<int64_t>(row) * ss + hh * sh) + 4 * t;
+    int4 w[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) w[u] = __ldg(src + u);
     const float *c = a.center ? a.kbar + (static_cast<int64_t>(b) * a.Hk + (is_key ? hh : hh / grp)) * D + 32 * t
                               : nullptr;
 #pragma unroll
@@ -741,7 +728,6 @@ __global__ void __launch_bounds__(256) k_row_norms(const NormArgs a) {
       if (a.center) a.qdot[idx] = dot;
     }
     if (valid) atomicMax(&smax[hh], __float_as_uint(nrm));
-  }
   }
   __syncthreads();
   // a key head's maximum goes to every query head of its group
@@ -855,7 +841,7 @@ cudaError_t launch_fixed_m_bound(const bsa_problem &p, const MaskParams &mp,
   }
   // blocks per batch row: 256 / (D / 32) vectors each, over the larger tensor
   const int64_t vec = static_cast<int64_t>(std::max(p.Sq * p.H, p.Skv * p.H_kv));
-  const int64_t vpb = 4 * (256 / (p.D / 32));  // four chunks of vectors per block
+  const int64_t vpb = 256 / (p.D / 32);
   const int bpb = static_cast<int>((vec + vpb - 1) / vpb);
   const dim3 grid(static_cast<unsigned>(p.B * bpb), na.only_q ? 1u : 2u);
   if (p.D == 64) k_row_norms<64><<<grid, 256, smem, s>>>(na);
