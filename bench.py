@@ -7,7 +7,7 @@ One step = the whole hot path over the causal sliding-window workload
   a2     fixed-m bound and per-head gate            (bsa_fixed_m_bound)
   a3     forward, fixed-m gated                     (bsa_attn_fwd)
   a4     Delta, zeroed dQ accumulator / semaphores  (bsa_bwd_preprocess)
-  a5     deterministic backward, ascending order    (bsa_bwd_main)
+  a5     deterministic backward, descending order   (bsa_bwd_main)
   a7     dQ convert                                 (bsa_bwd_convert)
 Metric: useful TFLOP/s = (non-empty 128x128 tiles x per-tile flops) / time, with
 per-tile flops 4*128*128*D forward and 2.5x that backward.  L2 is flushed
@@ -72,7 +72,7 @@ def parse():
     ap.add_argument("--softmax", default="fixed_m", choices=["fixed_m", "online"])
     ap.add_argument("--bound", default="norm", choices=["norm", "smoothed"],
                     help="fixed-m reference: Cauchy-Schwarz on ||k|| or on the centred keys")
-    ap.add_argument("--order", default="asc", choices=["asc", "desc", "outside_in", "greedy"])
+    ap.add_argument("--order", default="desc", choices=["asc", "desc", "outside_in", "greedy"])
     ap.add_argument("--nondet", action="store_true", help="atomic (non-deterministic) dQ backward")
     ap.add_argument("--residual", action="store_true",
                     help="keep O's bf16 rounding residual for an exact-to-fp32 Delta")

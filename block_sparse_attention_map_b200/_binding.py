@@ -78,7 +78,7 @@ _LIB = None
 def header_functions() -> list[str]:
     """Names of every function include/bsa.h declares."""
     text = open(HEADER).read()
-    return sorted(set(re.findall(r"^\s*BSA_API\s+(?:const\s+)?[a-z_0-9]+\s*\*?\s*(bsa_[a-z_]+)\s*\(", text, re.M)))
+    return sorted(set(re.findall(r"^\s*BSA_API\s+(?:const\s+)?[a-z_0-9]+\s*\*?\s*(bsa_[a-z_0-9]+)\s*\(", text, re.M)))
 
 
 def lib() -> ctypes.CDLL:

@@ -589,36 +589,55 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
         mbar_arrive(&bars[L::bDSReady]);
       }
       if (stop) break;
-      // epilogue: this half's columns of dV, dK (scaled) -> bf16
+      // epilogue: this half's columns of dV, then dK (scaled) -> bf16, staged
+      // through the 4 KB of the dS^T tile that only this warp writes (its 32
+      // rows of sub-tile `half`; the column's MMAs are done with the tile once
+      // DKVFull fires), then stored as whole 128-byte row segments: a warp
+      // store covers 512 / D rows instead of 32 scattered 16-byte pieces
       if (!wwait(&bars[L::bDKVFull], cc & 1)) break;
       tc_fence_after();
-      __nv_bfloat16 *dk_row = p.dk + k.b * p.k_sb + static_cast<int64_t>(j) * p.k_ss + k.hk * p.k_sh;
-      __nv_bfloat16 *dv_row = p.dv + k.b * p.v_sb + static_cast<int64_t>(j) * p.v_ss + k.hk * p.v_sh;
+      {
+        constexpr int kCpr = D / 16;           // 16-byte chunks per half row
+        constexpr int kRowsPerStore = 32 / kCpr;
+        uint8_t *stg = ds_tile + half * 16384 + quarter * 4096;
+        auto slot = [](int s_) { return s_ ^ ((s_ >> 3) & 7); };  // bank-conflict-free
 #pragma unroll
-      for (int c = half * (D / 64); c < (half + 1) * (D / 64); ++c) {
-        uint32_t a[32], g[32];
-        tmem_ld32(T_DV + lane_off + 32 * c, a);
-        tmem_ld32(T_DK + lane_off + 32 * c, g);
-        tmem_wait_ld();
-        if (row_ok) {
-          uint32_t wv[16], wk[16];
+        for (int which = 0; which < 2; ++which) {
+          const uint32_t tsrc = (which ? T_DK : T_DV) + lane_off + 32 * half * (D / 64);
+          const float mul = which ? p.scale : 1.f;
 #pragma unroll
-          for (int q = 0; q < 16; ++q) {
-            wv[q] = pack_bf16x2(__uint_as_float(a[2 * q]), __uint_as_float(a[2 * q + 1]));
-            wk[q] = pack_bf16x2(__uint_as_float(g[2 * q]) * p.scale,
-                                __uint_as_float(g[2 * q + 1]) * p.scale);
+          for (int c = 0; c < D / 64; ++c) {
+            uint32_t a[32];
+            tmem_ld32(tsrc + 32 * c, a);
+            tmem_wait_ld();
+            uint32_t w[16];
+#pragma unroll
+            for (int q = 0; q < 16; ++q)
+              w[q] = pack_bf16x2(__uint_as_float(a[2 * q]) * mul, __uint_as_float(a[2 * q + 1]) * mul);
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              *reinterpret_cast<int4 *>(stg + (slot(lane * kCpr + 4 * c + q) << 4)) =
+                  make_int4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
           }
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            reinterpret_cast<int4 *>(dv_row + 32 * c)[q] =
-                make_int4(wv[4 * q], wv[4 * q + 1], wv[4 * q + 2], wv[4 * q + 3]);
-            reinterpret_cast<int4 *>(dk_row + 32 * c)[q] =
-                make_int4(wk[4 * q], wk[4 * q + 1], wk[4 * q + 2], wk[4 * q + 3]);
+          if (which == 1) {
+            tc_fence_before();
+            mbar_arrive(&bars[L::bDKVFree]);
           }
+          __syncwarp();
+          __nv_bfloat16 *base = which ? p.dk + k.b * p.k_sb + k.hk * p.k_sh
+                                      : p.dv + k.b * p.v_sb + k.hk * p.v_sh;
+          const int64_t rs = which ? p.k_ss : p.v_ss;
+#pragma unroll
+          for (int it = 0; it < D / 16; ++it) {
+            const int rr = it * kRowsPerStore + lane / kCpr, ch = lane % kCpr;
+            const int jj = k.n * kTile + quarter * 32 + rr;
+            const int4 v = *reinterpret_cast<const int4 *>(stg + (slot(rr * kCpr + ch) << 4));
+            if (jj < p.Skv)
+              *reinterpret_cast<int4 *>(base + static_cast<int64_t>(jj) * rs + half * (D / 2) + 8 * ch) = v;
+          }
+          __syncwarp();
         }
       }
-      tc_fence_before();
-      mbar_arrive(&bars[L::bDKVFree]);
       ++cc;
     }
     }
@@ -632,7 +651,23 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
     auto wwait = [&](uint64_t *bar, uint32_t parity) {
       return __all_sync(0xffffffffu, wd.wait(bar, parity)) != 0;
     };
+    // dQ part of entry `ec`: TMEM -> registers (scaled), columns handed back
+    // to the next dP^T.  Every column load is in flight at once, one wait.
+    float acc[D];
+    auto read_dq = [&]() {
+      tc_fence_after();
+      uint32_t raw[D];
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c)
+        tmem_ld32(T_DP + lane_off + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&raw[32 * c]));
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(&bars[L::bDQFree]);
+#pragma unroll
+      for (int q = 0; q < D; ++q) acc[q] = __uint_as_float(raw[q]) * p.scale;
+    };
     uint32_t tc = 0, ec = 0;
+    bool ahead = false;  // acc already holds entry ec's dQ part
     for (;; ++tc) {
       const uint32_t slot = tc & 1;
       if (!wwait(&bars[L::bTkFull + slot], (tc >> 1) & 1)) break;
@@ -647,20 +682,11 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
         const int64_t bh = static_cast<int64_t>(k.b) * p.H + k.head(x);
         const int m = static_cast<int>(p.col_ent[e] & kIndexMask);
         const uint32_t rank = static_cast<uint32_t>(p.col_rank[e]);
-        if (!wwait(&bars[L::bDQFull], ec & 1)) { stop = true; break; }
-        tc_fence_after();
-        // every column load in flight at once, one wait: the columns are
-        // handed back to the next dP^T as early as possible
-        uint32_t raw[D];
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c)
-          tmem_ld32(T_DP + lane_off + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&raw[32 * c]));
-        tmem_wait_ld();
-        float acc[D];
-#pragma unroll
-        for (int q = 0; q < D; ++q) acc[q] = __uint_as_float(raw[q]) * p.scale;
-        tc_fence_before();
-        mbar_arrive(&bars[L::bDQFree]);
+        if (!ahead) {
+          if (!wwait(&bars[L::bDQFull], ec & 1)) { stop = true; break; }
+          read_dq();
+        }
+        ahead = false;
         uint32_t *sem = p.sem + bh * p.nM + m;
         int ok = 1;
         if (p.deterministic) {
@@ -682,6 +708,15 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
               red_add_v4(base + (static_cast<int64_t>(c) * kTile + r) * 4, acc[4 * c],
                          acc[4 * c + 1], acc[4 * c + 2], acc[4 * c + 3]);
           }
+        }
+        // if the column's next dQ part is already complete, take it out of TMEM
+        // before this entry's adds are fenced: the next dP^T then need not wait
+        // for the fence.  A single test, never a wait, so the turn below is
+        // passed on no later than the TMEM read.
+        if (x + 1 < k.tot &&
+            __all_sync(0xffffffffu, mbar_try_wait(smem_u32(&bars[L::bDQFull]), (ec + 1) & 1))) {
+          read_dq();
+          ahead = true;
         }
         if (p.deterministic) {
           __threadfence();

