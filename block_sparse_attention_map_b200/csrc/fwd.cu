@@ -41,6 +41,11 @@ namespace {
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: tolerate p up to 2^8
+// a group's Q slot goes back with its last S of the unit (true) or with the
+// unit's last MMAs (false).  With three slots the next unit's Q_A loads during
+// this unit either way; the late release measured faster (78.8 vs 80.9 us on
+// the 8192 window), as it did with two slots.
+constexpr bool kEarlyQRelease = false;
 
 struct FwdParams {
   MaskParams mask;
@@ -65,15 +70,15 @@ struct FwdParams {
   uint32_t sig_mask;   // which signature words must match
 };
 
-template <int D, int NK, int NV>
+template <int D, int NQ, int NK, int NV>
 struct FwdSmem {
   static constexpr int kTB = kTile * D * 2;
-  static constexpr int kQ = 0;                         // Q tiles of groups A, B
-  static constexpr int kK = 2 * kTB;                   // K ring
+  static constexpr int kQ = 0;                         // Q ring (both groups' tiles, in load order)
+  static constexpr int kK = NQ * kTB;                  // K ring
   static constexpr int kV = kK + NK * kTB;             // V ring
   static constexpr int kSeg = kV + NV * kTB;           // int32 [group][buffer][128]
   static constexpr int kBar = kSeg + 4 * kTile * 4;
-  static constexpr int bQFull = 0, bQEmpty = 2, bKFull = 4, bKEmpty = bKFull + NK,
+  static constexpr int bQFull = 0, bQEmpty = NQ, bKFull = 2 * NQ, bKEmpty = bKFull + NK,
                        bVFull = bKEmpty + NK, bVEmpty = bVFull + NV, bSFull = bVEmpty + NV,
                        bPFull = bSFull + 2, bPVDone = bPFull + 2, bSegReady = bPVDone + 2,
                        bFinal = bSegReady + 4, kNumBars = bFinal + 1;
@@ -141,11 +146,11 @@ struct UnionWalk {
   }
 };
 
-template <int D, int NK, int NV>
+template <int D, int NQ, int NK, int NV>
 __global__ void __launch_bounds__(384, 1)
 k_attn_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
            const __grid_constant__ CUtensorMap tv, const FwdParams p) {
-  using L = FwdSmem<D, NK, NV>;
+  using L = FwdSmem<D, NQ, NK, NV>;
   extern __shared__ __align__(1024) uint8_t sm[];
   uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::kBar);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::kMisc);
@@ -198,7 +203,7 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
   } else if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      uint32_t kv = 0, uq[2] = {0, 0}, k_issued = 0, v_issued = 0, q_issued[2] = {0, 0};
+      uint32_t kv = 0, qi = 0, k_issued = 0, v_issued = 0;
       bool stop = false;
       for (int u = blockIdx.x; u < p.n_units && !stop; u += gridDim.x) {
         const FwdUnit w = decode_unit(p, u);
@@ -207,13 +212,16 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
 #pragma unroll
         for (int x = 0; x < 2; ++x) {
           if (!has[x]) continue;
-          if (uq[x] >= 1 && !wd.wait(&bars[L::bQEmpty + x], (uq[x] - 1) & 1)) { stop = true; break; }
-          mbar_arrive_expect_tx(&bars[L::bQFull + x], kTB);
+          // Q tiles go through a ring of NQ slots in load order (A, B of each
+          // unit): with NQ = 3 the next unit's Q_A loads during this unit, and
+          // its Q_B as soon as this unit's Q_A is released
+          const uint32_t qs = qi % NQ;
+          if (qi >= NQ && !wd.wait(&bars[L::bQEmpty + qs], ((qi / NQ) - 1) & 1)) { stop = true; break; }
+          mbar_arrive_expect_tx(&bars[L::bQFull + qs], kTB);
           for (int c = 0; c < D / 64; ++c)
-            tma_load_4d(sm + L::kQ + x * kTB + c * 16384, &tq, &bars[L::bQFull + x], c * 64,
+            tma_load_4d(sm + L::kQ + qs * kTB + c * 16384, &tq, &bars[L::bQFull + qs], c * 64,
                         w.m[x] * kTile, w.h, w.b);
-          ++uq[x];
-          ++q_issued[x];
+          ++qi;
         }
         if (stop) break;
         UnionWalk uw{p.row_ent, {w.rs[0], w.rs[1]}, {w.re[0], w.re[1]}};
@@ -242,16 +250,17 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
           drain_wait(&bars[L::bKFull + t % NK], (t / NK) & 1);
         for (uint32_t t = (v_issued > NV ? v_issued - NV : 0); t < v_issued; ++t)
           drain_wait(&bars[L::bVFull + t % NV], (t / NV) & 1);
-        for (int x = 0; x < 2; ++x)
-          if (q_issued[x] > 0) drain_wait(&bars[L::bQFull + x], (q_issued[x] - 1) & 1);
+        for (uint32_t t = (qi > NQ ? qi - NQ : 0); t < qi; ++t)
+          drain_wait(&bars[L::bQFull + t % NQ], (t / NQ) & 1);
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      uint32_t kv = 0, uq[2] = {0, 0}, tcount[2] = {0, 0};
+      uint32_t kv = 0, qm = 0, tcount[2] = {0, 0};
       bool stop = false;
-      const uint32_t q_addr[2] = {smem_u32(sm + L::kQ), smem_u32(sm + L::kQ + kTB)};
+      uint32_t q_addr[2] = {0, 0}, q_slot[2] = {0, 0};
+      int s_left[2] = {0, 0};  // S ops of the group still to issue in this unit
       // S_x = Q_x K^T into the S columns of group x.  The previous PV_x still
       // reads P_x from those columns; tcgen05.mma ops issued by one thread
       // execute in issue order, so no completion wait is needed in between.
@@ -266,14 +275,22 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
                  sw128_desc(k_addr + off, 16, 1024), kIdescS, kk > 0);
         }
         mma_commit(&bars[L::bSFull + x]);
+        // the group's last S of the unit: its Q slot can take the next Q tile
+        if (kEarlyQRelease && --s_left[x] == 0) mma_commit(&bars[L::bQEmpty + q_slot[x]]);
         return true;
       };
       for (int u = blockIdx.x; u < p.n_units && !stop; u += gridDim.x) {
         const FwdUnit w = decode_unit(p, u);
         const bool has[2] = {w.re[0] > w.rs[0], w.re[1] > w.rs[1]};
         if (!has[0] && !has[1]) continue;
-        for (int x = 0; x < 2; ++x)
-          if (has[x] && !wd.wait(&bars[L::bQFull + x], uq[x] & 1)) stop = true;
+        for (int x = 0; x < 2; ++x) {
+          if (!has[x]) continue;
+          q_slot[x] = qm % NQ;
+          q_addr[x] = smem_u32(sm + L::kQ + q_slot[x] * kTB);
+          s_left[x] = w.re[x] - w.rs[x];
+          if (!wd.wait(&bars[L::bQFull + q_slot[x]], (qm / NQ) & 1)) stop = true;
+          ++qm;
+        }
         if (stop) break;
         bool first[2] = {true, true};
         UnionWalk uw{p.row_ent, {w.rs[0], w.rs[1]}, {w.re[0], w.re[1]}};
@@ -317,13 +334,9 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
         }
         if (stop) break;
         kv = kv_cur + 1;
-        // Q buffers go back to the producer with the unit's last MMAs (releasing
-        // them right after each group's last S measured slower)
-        for (int x = 0; x < 2; ++x)
-          if (has[x]) {
-            mma_commit(&bars[L::bQEmpty + x]);
-            ++uq[x];
-          }
+        if (!kEarlyQRelease)
+          for (int x = 0; x < 2; ++x)
+            if (has[x]) mma_commit(&bars[L::bQEmpty + q_slot[x]]);
       }
       // every tcgen05 op this thread issued is complete before TMEM is freed
       mma_commit(&bars[L::bFinal]);
@@ -521,11 +534,15 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       const float inv = l_r > 0.f ? 1.f / l_r : 0.f;
       __nv_bfloat16 *orow = p.out + b * p.o_sb + static_cast<int64_t>(i) * p.o_ss + h * p.o_sh;
       float *lse_p = p.lse + static_cast<int64_t>(bh) * p.Sq + i;
+      // 16-column pieces of O, the next piece's TMEM load in flight while this
+      // one is converted and stored (a wait covers every load issued before it)
+      uint32_t ob[2][16];
+      tmem_ld16(t_o, ob[0]);
+      tmem_wait_ld();
 #pragma unroll
       for (int c = 0; c < D / 16; ++c) {
-        uint32_t o[16];
-        tmem_ld16(t_o + c * 16, o);
-        tmem_wait_ld();
+        if (c + 1 < D / 16) tmem_ld16(t_o + (c + 1) * 16, ob[(c + 1) & 1]);
+        const uint32_t *o = ob[c & 1];
         if (row_ok) {
           uint32_t wv[8];
 #pragma unroll
@@ -548,6 +565,7 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
             rd[1] = make_int4(wv[4], wv[5], wv[6], wv[7]);
           }
         }
+        if (c + 1 < D / 16) tmem_wait_ld();
       }
       tc_fence_before();
       if (row_ok) *lse_p = l > 0.f ? (m_ref + __log2f(l)) * kLn2 : -INFINITY;
@@ -770,20 +788,20 @@ int sm_count() {
   return n;
 }
 
-template <int D, int NK, int NV>
+template <int D, int NQ, int NK, int NV>
 cudaError_t run_fwd(const FwdParams &fp, const CUtensorMap &tq, const CUtensorMap &tk,
                     const CUtensorMap &tv, cudaStream_t s) {
-  using L = FwdSmem<D, NK, NV>;
+  using L = FwdSmem<D, NQ, NK, NV>;
   static_assert(L::kAlloc <= 232448, "shared memory budget");
   static bool attr = false;
   if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(k_attn_fwd<D, NK, NV>,
+    cudaError_t e = cudaFuncSetAttribute(k_attn_fwd<D, NQ, NK, NV>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc);
     if (e != cudaSuccess) return e;
     attr = true;
   }
   const int grid = std::min(fp.n_units, sm_count());
-  k_attn_fwd<D, NK, NV><<<grid, 384, L::kAlloc, s>>>(tq, tk, tv, fp);
+  k_attn_fwd<D, NQ, NK, NV><<<grid, 384, L::kAlloc, s>>>(tq, tk, tv, fp);
   count_launch();
   return cudaGetLastError();
 }
@@ -890,8 +908,8 @@ cudaError_t launch_fwd(const bsa_problem &p, const MaskParams &mp, const bsa_opt
   for (int i = 0; i < kSigWords; ++i) fp.sig[i] = sig.w[i];
   // the forward does not depend on the kv-column order
   fp.sig_mask = ((1u << kSigWords) - 1u) & ~(1u << kSigOrderWord);
-  if (p.D == 64) return run_fwd<64, 4, 4>(fp, tq, tk, tv, s);
-  return run_fwd<128, 3, 2>(fp, tq, tk, tv, s);
+  if (p.D == 64) return run_fwd<64, 3, 4, 4>(fp, tq, tk, tv, s);
+  return run_fwd<128, 3, 2, 2>(fp, tq, tk, tv, s);
 }
 
 }  // namespace bsa
