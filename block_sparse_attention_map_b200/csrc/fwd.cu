@@ -679,8 +679,8 @@ __global__ void __launch_bounds__(256) k_key_centers(const NormArgs a) {
 // then one global atomic per head and block.
 template <int D>
 __global__ void __launch_bounds__(256) k_row_norms(const NormArgs a) {
-  constexpr int kT = D / 32;          // threads per vector
-  constexpr int kVPB = 256 / kT;      // vectors per block
+  constexpr int kT = D / 32;          // threads per vector, four 16-byte loads each
+  constexpr int kVPB = 256 / kT;      // vectors per block and pass
   extern __shared__ unsigned int smax[];  // [H]
   __shared__ bool last_block;
   const int is_key = !a.only_q && blockIdx.y == 0;
@@ -696,56 +696,76 @@ __global__ void __launch_bounds__(256) k_row_norms(const NormArgs a) {
   const int b = static_cast<int>(blockIdx.x) / bpb, blk = static_cast<int>(blockIdx.x) % bpb;
   for (int h = threadIdx.x; h < H; h += blockDim.x) smax[h] = 0u;
   __syncthreads();
-  const int64_t v = static_cast<int64_t>(blk) * kVPB + threadIdx.x / kT;
+  // Grid-stride over the batch row's (row, head) vectors, consecutive vectors
+  // on consecutive heads of a row (the tensor's memory order).  Two vectors
+  // per thread and pass keep eight 16-byte loads in flight; the per-head
+  // maxima gather in shared memory over the block's whole range, so the
+  // global atomics and the fence below happen once per block.
+  const int64_t nvec = static_cast<int64_t>(S) * Hx;
+  const int64_t stride = static_cast<int64_t>(bpb) * kVPB;
   const int t = threadIdx.x % kT;
-  const bool in = v < static_cast<int64_t>(S) * Hx;  // no early return: shuffles below
-  const int row = in ? static_cast<int>(v / Hx) : 0, hh = in ? static_cast<int>(v % Hx) : 0;
-  float acc = 0.f, dot = 0.f;
-  if (in) {
-    const int4 *src = reinterpret_cast<const int4 *>(x + b * sb + static_cast<int64_t>(row) * ss + hh * sh) + 4 * t;
-    int4 w[4];
+  for (int64_t base = static_cast<int64_t>(blk) * kVPB; base < nvec; base += 2 * stride) {
+    int64_t vv[2];
+    bool in[2];
+    int4 w[2][4];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) w[u] = __ldg(src + u);
-    const float *c = a.center ? a.kbar + (static_cast<int64_t>(b) * a.Hk + (is_key ? hh : hh / grp)) * D + 32 * t
-                              : nullptr;
+    for (int j = 0; j < 2; ++j) {
+      vv[j] = base + j * stride + threadIdx.x / kT;
+      in[j] = vv[j] < nvec;  // no early exit: the shuffles below need every lane
+      if (in[j]) {
+        const int row = static_cast<int>(vv[j] / Hx), hh = static_cast<int>(vv[j] % Hx);
+        const int4 *src = reinterpret_cast<const int4 *>(x + b * sb + static_cast<int64_t>(row) * ss + hh * sh) + 4 * t;
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const uint32_t xw[4] = {static_cast<uint32_t>(w[u].x), static_cast<uint32_t>(w[u].y),
-                              static_cast<uint32_t>(w[u].z), static_cast<uint32_t>(w[u].w)};
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        float2 f = unpack_bf16x2(xw[q]);
-        if (c != nullptr) {
-          const float2 cc = *reinterpret_cast<const float2 *>(c + 8 * u + 2 * q);
-          if (is_key) {
-            f.x -= cc.x;
-            f.y -= cc.y;
-          } else {
-            dot = fmaf(f.x, cc.x, dot);
-            dot = fmaf(f.y, cc.y, dot);
-          }
-        }
-        acc = fmaf(f.x, f.x, acc);
-        acc = fmaf(f.y, f.y, acc);
+        for (int u = 0; u < 4; ++u) w[j][u] = __ldg(src + u);
       }
     }
-  }
 #pragma unroll
-  for (int o = kT / 2; o > 0; o >>= 1) {
-    acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    dot += __shfl_xor_sync(0xffffffffu, dot, o);
-  }
-  if (in && t == 0) {
-    const float nrm = sqrtf(acc);
-    bool valid = true;
-    if (is_key) {
-      valid = key_is_valid(a.mk, b, row);
-    } else {
-      const int64_t idx = (static_cast<int64_t>(b) * H + hh) * S + row;
-      a.qnorm[idx] = nrm;
-      if (a.center) a.qdot[idx] = dot;
+    for (int j = 0; j < 2; ++j) {
+      const int row = in[j] ? static_cast<int>(vv[j] / Hx) : 0, hh = in[j] ? static_cast<int>(vv[j] % Hx) : 0;
+      float acc = 0.f, dot = 0.f;
+      if (in[j]) {
+        const float *c = a.center ? a.kbar + (static_cast<int64_t>(b) * a.Hk + (is_key ? hh : hh / grp)) * D + 32 * t
+                                  : nullptr;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const uint32_t xw[4] = {static_cast<uint32_t>(w[j][u].x), static_cast<uint32_t>(w[j][u].y),
+                                  static_cast<uint32_t>(w[j][u].z), static_cast<uint32_t>(w[j][u].w)};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            float2 f = unpack_bf16x2(xw[q]);
+            if (c != nullptr) {
+              const float2 cc = *reinterpret_cast<const float2 *>(c + 8 * u + 2 * q);
+              if (is_key) {
+                f.x -= cc.x;
+                f.y -= cc.y;
+              } else {
+                dot = fmaf(f.x, cc.x, dot);
+                dot = fmaf(f.y, cc.y, dot);
+              }
+            }
+            acc = fmaf(f.x, f.x, acc);
+            acc = fmaf(f.y, f.y, acc);
+          }
+        }
+      }
+#pragma unroll
+      for (int o = kT / 2; o > 0; o >>= 1) {
+        acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        dot += __shfl_xor_sync(0xffffffffu, dot, o);
+      }
+      if (in[j] && t == 0) {
+        const float nrm = sqrtf(acc);
+        bool valid = true;
+        if (is_key) {
+          valid = key_is_valid(a.mk, b, row);
+        } else {
+          const int64_t idx = (static_cast<int64_t>(b) * H + hh) * S + row;
+          a.qnorm[idx] = nrm;
+          if (a.center) a.qdot[idx] = dot;
+        }
+        if (valid) atomicMax(&smax[hh], __float_as_uint(nrm));
+      }
     }
-    if (valid) atomicMax(&smax[hh], __float_as_uint(nrm));
   }
   __syncthreads();
   // a key head's maximum goes to every query head of its group
@@ -857,10 +877,12 @@ cudaError_t launch_fixed_m_bound(const bsa_problem &p, const MaskParams &mp,
     }
     count_launch(2);
   }
-  // blocks per batch row: 256 / (D / 32) vectors each, over the larger tensor
+  // blocks per batch row: about four per SM over the whole grid, and no more
+  // than the larger tensor's vectors fill at 256 / (D / 32) per block
   const int64_t vec = static_cast<int64_t>(std::max(p.Sq * p.H, p.Skv * p.H_kv));
   const int64_t vpb = 256 / (p.D / 32);
-  const int bpb = static_cast<int>((vec + vpb - 1) / vpb);
+  const int64_t want = std::max<int64_t>(1, (4 * 148) / (static_cast<int64_t>(p.B) * (na.only_q ? 1 : 2)));
+  const int bpb = static_cast<int>(std::min<int64_t>(want, (vec + vpb - 1) / vpb));
   const dim3 grid(static_cast<unsigned>(p.B * bpb), na.only_q ? 1u : 2u);
   if (p.D == 64) k_row_norms<64><<<grid, 256, smem, s>>>(na);
   else k_row_norms<128><<<grid, 256, smem, s>>>(na);
