@@ -100,6 +100,8 @@ def lib() -> ctypes.CDLL:
                                      c_vp, c_vp, c_vp, c_vp, c_vp, ctypes.c_size_t, c_vp]),
             "bsa_fixed_m_bound": (c_i32, [P(Problem), P(MaskSpec), P(Options), c_vp, c_vp, c_vp,
                                           ctypes.c_size_t, c_vp]),
+            "bsa_plan_and_bound": (c_i32, [P(Problem), P(MaskSpec), P(Options), c_vp, c_vp, c_vp,
+                                           ctypes.c_size_t, c_vp]),
             "bsa_bwd_preprocess": (c_i32, [P(Problem), P(MaskSpec), P(Options), c_vp, c_vp, c_vp,
                                            ctypes.c_size_t, c_vp]),
             "bsa_bwd_main": (c_i32, [P(Problem), P(MaskSpec), P(Options), c_vp, c_vp, c_vp, c_vp, c_vp,
@@ -383,6 +385,15 @@ class Stages:
         if self.fixed:
             _check(lib().bsa_fixed_m_bound(*self._args, self.q.data_ptr(), self.k.data_ptr(), self.ws.ptr(),
                                            self.ws.nbytes, _stream()), "bsa_fixed_m_bound")
+
+    def plan_and_bound(self):
+        """The plan and, in fixed-m mode, the bound in one call (the planner beside
+        the bound's row-norm pass, on the library's side stream)."""
+        if self.fixed:
+            _check(lib().bsa_plan_and_bound(*self._args, self.q.data_ptr(), self.k.data_ptr(), self.ws.ptr(),
+                                            self.ws.nbytes, _stream()), "bsa_plan_and_bound")
+        else:
+            self.plan()
 
     def forward(self):
         _check(lib().bsa_attn_fwd(*self._args, self.q.data_ptr(), self.k.data_ptr(), self.v.data_ptr(),

@@ -1,10 +1,13 @@
 // C ABI of libbsa (declared in include/bsa.h): argument validation, workspace
 // layout, TMA tensor maps and the sequence of launches for each call.  Every
 // argument error is returned before anything is launched; the library
-// allocates nothing and synchronises only in bsa_get_device_status.
+// allocates no device memory and synchronises only in bsa_get_device_status.
+// It owns one non-blocking side stream per device (created on first use), on
+// which the planner runs beside the fixed-m bound.
 #include <atomic>
 #include <cmath>
 #include <cstring>
+#include <mutex>
 #include <vector>
 
 #include "internal.h"
@@ -272,7 +275,104 @@ bsa_status prepare(const bsa_problem *prob, const bsa_mask_spec *mask, const bsa
 
 bsa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? BSA_OK : BSA_ERR_CUDA; }
 
+
+// ---------------------------------------------------------------- plan || bound
+constexpr int kMaxSideDevices = 64;
+std::mutex g_side_mu;
+cudaStream_t g_side[kMaxSideDevices] = {};
+
+// The library's side stream on the current device (non-blocking: it never
+// orders itself against the legacy default stream; every use is joined by
+// events).
+cudaError_t side_stream(cudaStream_t *out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxSideDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_side_mu);
+  if (g_side[dev] == nullptr) {
+    e = cudaStreamCreateWithFlags(&g_side[dev], cudaStreamNonBlocking);
+    if (e != cudaSuccess) return e;
+  }
+  *out = g_side[dev];
+  return cudaSuccess;
+}
+
+// The block-map plan and the fixed-m bound of one call.  The bound reads the
+// planner's output only for varlen masks (the alignment rows' ids); otherwise
+// the two are independent, and the planner (one CTA) runs on the side stream
+// while the bound's row-norm pass (the rest of the GPU) runs on `s`: forked
+// from and joined back into `s` by events, so work after the call on `s` sees
+// both, and stream capture records the same fork and join.
+cudaError_t plan_and_bound(const bsa_problem &p, const bsa_mask_spec &m, const bsa_options &o,
+                           const void *q, const void *k, const WsLayout &L, uint8_t *ws,
+                           cudaStream_t s) {
+  const MaskParams mp = mask_params(p, m, L, ws);
+  if (m.flags & BSA_MASK_VARLEN) {
+    cudaError_t e = launch_plan(p, m, o, L, ws, s);
+    if (e != cudaSuccess) return e;
+    return launch_fixed_m_bound(p, mp, o, q, k, L, ws, s);
+  }
+  cudaStream_t side = nullptr;
+  cudaError_t e = side_stream(&side);
+  if (e != cudaSuccess) return e;
+  cudaEvent_t fork = nullptr, join = nullptr;
+  if ((e = cudaEventCreateWithFlags(&fork, cudaEventDisableTiming)) != cudaSuccess) return e;
+  if ((e = cudaEventCreateWithFlags(&join, cudaEventDisableTiming)) != cudaSuccess) {
+    cudaEventDestroy(fork);
+    return e;
+  }
+  e = cudaEventRecord(fork, s);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(side, fork, 0);
+  if (e == cudaSuccess) e = launch_plan(p, m, o, L, ws, side);
+  if (e == cudaSuccess) e = cudaEventRecord(join, side);
+  cudaError_t eb = cudaSuccess;
+  if (e == cudaSuccess) eb = launch_fixed_m_bound(p, mp, o, q, k, L, ws, s);
+  // join even when the bound failed to launch, so `s` never runs ahead of the plan
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(s, join, 0);
+  cudaEventDestroy(fork);  // released once the recorded work completes
+  cudaEventDestroy(join);
+  return e != cudaSuccess ? e : eb;
+}
+
 }  // namespace
+
+// The forward call.  side_stream_ok = false keeps the plan and the bound on
+// `stream` one after the other (the static-scratch entry makes no call that
+// creates a stream or an event).
+bsa_status attn_fwd_impl(const bsa_problem *prob, const bsa_mask_spec *mask,
+                         const bsa_options *opt, const void *q, const void *k, const void *v,
+                         void *out, float *lse, void *ws, size_t ws_bytes, bsa_stream_t stream,
+                         bool side_stream_ok) {
+  if (q == nullptr || k == nullptr || v == nullptr || out == nullptr || lse == nullptr)
+    return BSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return BSA_ERR_UNSUPPORTED;
+  Prepared P;
+  bsa_status st = prepare(prob, mask, opt, ws, ws_bytes, false, &P);
+  if (st != BSA_OK) return st;
+  const bsa_problem &p = P.p;
+  CUtensorMap tq, tk, tv;
+  if (!make_map(&tq, q, p.B, p.Sq, p.H, p.D, p.q_stride) ||
+      !make_map(&tk, k, p.B, p.Skv, p.H_kv, p.D, p.k_stride) ||
+      !make_map(&tv, v, p.B, p.Skv, p.H_kv, p.D, p.v_stride))
+    return BSA_ERR_UNSUPPORTED;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t *w = static_cast<uint8_t *>(ws);
+  const bool need_bound = P.o.softmax_mode == BSA_SOFTMAX_FIXED_M_GATED && !P.o.bound_ready;
+  if (!P.o.plan_ready && need_bound && side_stream_ok) {
+    if ((st = cuda_status(plan_and_bound(p, P.m, P.o, q, k, P.L, w, s))) != BSA_OK) return st;
+  } else {
+    if (!P.o.plan_ready && (st = cuda_status(launch_plan(p, P.m, P.o, P.L, w, s))) != BSA_OK) return st;
+    if (need_bound &&
+        (st = cuda_status(launch_fixed_m_bound(p, mask_params(p, P.m, P.L, w), P.o, q, k, P.L, w, s))) != BSA_OK)
+      return st;
+  }
+  const MaskParams mp = mask_params(p, P.m, P.L, w);
+  return cuda_status(launch_fwd(p, mp, P.o, signature(p, P.m, P.o), tq, tk, tv, out, lse, P.L, w, s));
+}
+
 }  // namespace bsa
 
 using namespace bsa;
@@ -338,30 +438,7 @@ bsa_status bsa_plan_build(const bsa_problem *prob, const bsa_mask_spec *mask,
 bsa_status bsa_attn_fwd(const bsa_problem *prob, const bsa_mask_spec *mask,
                         const bsa_options *opt, const void *q, const void *k, const void *v,
                         void *out, float *lse, void *ws, size_t ws_bytes, bsa_stream_t stream) {
-  if (q == nullptr || k == nullptr || v == nullptr || out == nullptr || lse == nullptr)
-    return BSA_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
-      (reinterpret_cast<uintptr_t>(lse) & 3u))
-    return BSA_ERR_UNSUPPORTED;
-  Prepared P;
-  bsa_status st = prepare(prob, mask, opt, ws, ws_bytes, false, &P);
-  if (st != BSA_OK) return st;
-  const bsa_problem &p = P.p;
-  CUtensorMap tq, tk, tv;
-  if (!make_map(&tq, q, p.B, p.Sq, p.H, p.D, p.q_stride) ||
-      !make_map(&tk, k, p.B, p.Skv, p.H_kv, p.D, p.k_stride) ||
-      !make_map(&tv, v, p.B, p.Skv, p.H_kv, p.D, p.v_stride))
-    return BSA_ERR_UNSUPPORTED;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  uint8_t *w = static_cast<uint8_t *>(ws);
-  if (!P.o.plan_ready) {
-    if ((st = cuda_status(launch_plan(p, P.m, P.o, P.L, w, s))) != BSA_OK) return st;
-  }
-  const MaskParams mp = mask_params(p, P.m, P.L, w);
-  if (P.o.softmax_mode == BSA_SOFTMAX_FIXED_M_GATED && !P.o.bound_ready) {
-    if ((st = cuda_status(launch_fixed_m_bound(p, mp, P.o, q, k, P.L, w, s))) != BSA_OK) return st;
-  }
-  return cuda_status(launch_fwd(p, mp, P.o, signature(p, P.m, P.o), tq, tk, tv, out, lse, P.L, w, s));
+  return bsa::attn_fwd_impl(prob, mask, opt, q, k, v, out, lse, ws, ws_bytes, stream, true);
 }
 
 bsa_status bsa_attn_bwd(const bsa_problem *prob, const bsa_mask_spec *mask,
@@ -410,6 +487,18 @@ bsa_status bsa_fixed_m_bound(const bsa_problem *prob, const bsa_mask_spec *mask,
   }
   const MaskParams mp = mask_params(P.p, P.m, P.L, w);
   return cuda_status(launch_fixed_m_bound(P.p, mp, P.o, q, k, P.L, w, s));
+}
+
+bsa_status bsa_plan_and_bound(const bsa_problem *prob, const bsa_mask_spec *mask,
+                              const bsa_options *opt, const void *q, const void *k, void *ws,
+                              size_t ws_bytes, bsa_stream_t stream) {
+  if (q == nullptr || k == nullptr) return BSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k)) return BSA_ERR_UNSUPPORTED;
+  Prepared P;
+  bsa_status st = prepare(prob, mask, opt, ws, ws_bytes, false, &P);
+  if (st != BSA_OK) return st;
+  return cuda_status(plan_and_bound(P.p, P.m, P.o, q, k, P.L, static_cast<uint8_t *>(ws),
+                                    reinterpret_cast<cudaStream_t>(stream)));
 }
 
 bsa_status bsa_bwd_preprocess(const bsa_problem *prob, const bsa_mask_spec *mask,

@@ -120,4 +120,11 @@ cudaError_t launch_bwd_convert(const bsa_problem &p, void *dq, const WsLayout &L
 
 void count_launch(int n = 1);
 
+// bsa_attn_fwd; side_stream_ok = false never forks work onto the library's side
+// stream (no stream or event is created).
+bsa_status attn_fwd_impl(const bsa_problem *prob, const bsa_mask_spec *mask,
+                         const bsa_options *opt, const void *q, const void *k, const void *v,
+                         void *out, float *lse, void *ws, size_t ws_bytes, bsa_stream_t stream,
+                         bool side_stream_ok);
+
 }  // namespace bsa

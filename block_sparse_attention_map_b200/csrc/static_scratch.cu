@@ -67,5 +67,7 @@ extern "C" bsa_status bsa_attn_fwd_static_scratch(const bsa_problem *prob,
   o.plan_ready = 0;
   o.bound_ready = 0;
   o.keep_o_residual = 0;  // no backward shares this scratch
-  return bsa_attn_fwd(prob, mask, &o, q, k, v, out, lse, ws, kStaticScratchBytes, stream);
+  // plan and bound one after the other on `stream`: no side stream, no events
+  return bsa::attn_fwd_impl(prob, mask, &o, q, k, v, out, lse, ws, kStaticScratchBytes, stream,
+                            false);
 }

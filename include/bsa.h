@@ -255,8 +255,8 @@ BSA_API bsa_status bsa_attn_bwd(const bsa_problem *prob, const bsa_mask_spec *ma
                         size_t ws_bytes, bsa_stream_t stream);
 
 /* The stages of the hot path, one call each, for callers that schedule or time
- * them separately.  bsa_attn_fwd = [bsa_plan_build] + [bsa_fixed_m_bound] +
- * forward kernel; bsa_attn_bwd = [bsa_plan_build] + bsa_bwd_preprocess +
+ * them separately.  bsa_attn_fwd = [bsa_plan_build] + [bsa_fixed_m_bound] (both
+ * at once as bsa_plan_and_bound when both are needed) + forward kernel; bsa_attn_bwd = [bsa_plan_build] + bsa_bwd_preprocess +
  * bsa_bwd_main + bsa_bwd_convert.  Each expects the workspace state the
  * previous stage leaves; arguments as for bsa_attn_fwd / bsa_attn_bwd. */
 
@@ -266,6 +266,20 @@ BSA_API bsa_status bsa_attn_bwd(const bsa_problem *prob, const bsa_mask_spec *ma
 BSA_API bsa_status bsa_fixed_m_bound(const bsa_problem *prob, const bsa_mask_spec *mask,
                                      const bsa_options *opt, const void *q, const void *k,
                                      void *ws, size_t ws_bytes, bsa_stream_t stream);
+
+/* a1 + a2 together: the block-map plan (as bsa_plan_build) and the fixed-m bound
+ * (as bsa_fixed_m_bound), the result identical to calling the two in turn.  For
+ * every mask but BSA_MASK_VARLEN (whose key validity the bound reads from the
+ * plan) the planner runs on a non-blocking stream of the library's own, created
+ * once per device, concurrently with the bound's pass over Q and K on `stream`:
+ * the side stream waits for an event recorded on `stream` and `stream` waits for
+ * the planner before the call returns, so all later work on `stream` sees both
+ * results, and a stream capture on `stream` records the same fork and join.
+ * bsa_attn_fwd takes this path when it has to build both.  Arguments and errors
+ * as for bsa_fixed_m_bound (q, k device pointers, 16-byte aligned). */
+BSA_API bsa_status bsa_plan_and_bound(const bsa_problem *prob, const bsa_mask_spec *mask,
+                                      const bsa_options *opt, const void *q, const void *k,
+                                      void *ws, size_t ws_bytes, bsa_stream_t stream);
 
 /* a4: Delta_i = sum_d dO_id O_id (fp32) into the workspace; zeroes the fp32 dQ
  * accumulator and the dQ semaphores. */
@@ -298,7 +312,9 @@ BSA_API bsa_status bsa_bwd_convert(const bsa_problem *prob, const bsa_mask_spec 
  *  - Problems whose forward workspace (bsa_workspace_size, with_backward = 0)
  *    exceeds 32 MiB are rejected with BSA_ERR_WORKSPACE_TOO_SMALL before any
  *    launch.
- *  - No cudaMalloc, cudaFree or other allocating call is made.  The first call
+ *  - No cudaMalloc, cudaFree or other allocating call is made (the plan and the
+ *    bound run one after the other on `stream`, never on the library's side
+ *    stream, so no stream or event is created either).  The first call
  *    on each device looks up the array's device address (with that device
  *    current); make that first call before any stream capture.
  *  - Every call shares the one array and rebuilds the plan in it, so calls

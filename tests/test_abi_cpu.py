@@ -150,6 +150,11 @@ def test_calls_reject_bad_arguments_before_cuda(L):
     # misaligned pointers
     assert L.bsa_attn_fwd(ctypes.byref(p), None, ctypes.byref(o), 8, 256, 512, 1024, 4096,
                           4096, 1 << 20, None) == 2
+    # the plan beside the bound: null and misaligned inputs
+    assert L.bsa_plan_and_bound(ctypes.byref(p), None, ctypes.byref(o), None, 256, 4096, 1 << 20,
+                                None) == 1
+    assert L.bsa_plan_and_bound(ctypes.byref(p), None, ctypes.byref(o), 8, 256, 4096, 1 << 20,
+                                None) == 2
     # bad order and a non-permutation
     o.bwd_order = 7
     assert L.bsa_plan_build(ctypes.byref(p), None, ctypes.byref(o), 4096, 1 << 30, None) == 1

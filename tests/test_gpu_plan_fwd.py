@@ -304,3 +304,30 @@ def test_fwd_video_full_size_sampled_rows(mode):
     assert compare_out(o[:, :, heads], O_ref, rows) <= O_TOL
     el, same = compare_lse(lse[:, heads], L_ref, rows)
     assert el <= LSE_TOL and same
+
+
+@pytest.mark.parametrize("name", ["window", "varlen", "document"])
+def test_plan_beside_bound_equals_plan_then_bound(name):
+    # bsa_plan_and_bound runs the planner on the library's side stream next to
+    # the bound (sequentially for varlen masks): the forward that follows must
+    # see exactly the state plan-then-bound leaves, on the caller's stream with
+    # no synchronisation in between
+    wl = make_workload(name, device="cuda", small=True)
+    outs = []
+    for together in (False, True):
+        st = bsa.Stages(wl.q, wl.k, wl.v, wl.mask, softmax_mode="fixed_m", order="desc")
+        for _ in range(3):  # repeated: each call forks and joins again
+            if together:
+                st.plan_and_bound()
+            else:
+                st.plan()
+                st.bound()
+            st.forward()
+        torch.cuda.synchronize()
+        assert st.ws.status() == 0
+        outs.append((st.out.clone(), st.lse.clone()))
+    assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
+    rows = sample_rows(wl.Sq, seed=4)
+    f = lambda t: t.float().cpu().numpy().astype(np.float64)
+    O_ref, L_ref = oracle.attention_forward(f(wl.q), f(wl.k), f(wl.v), mask_desc(wl), wl.scale, rows=rows)
+    assert compare_out(outs[1][0], O_ref, rows) <= O_TOL
