@@ -291,10 +291,47 @@ cudaError_t side_stream(cudaStream_t *out) {
   if (dev < 0 || dev >= kMaxSideDevices) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(g_side_mu);
   if (g_side[dev] == nullptr) {
-    e = cudaStreamCreateWithFlags(&g_side[dev], cudaStreamNonBlocking);
+    // the highest priority, so that the planner's one CTA (a whole SM's
+    // registers) is placed before the bound's CTAs fill every SM
+    int lo = 0, hi = 0;
+    e = cudaDeviceGetStreamPriorityRange(&lo, &hi);
+    if (e != cudaSuccess) return e;
+    e = cudaStreamCreateWithPriority(&g_side[dev], cudaStreamNonBlocking, hi);
     if (e != cudaSuccess) return e;
   }
   *out = g_side[dev];
+  return cudaSuccess;
+}
+
+// The fork and join events of the calling host thread on the current device,
+// created on first use and kept for the thread's lifetime: a stream wait takes
+// an event's state when it is issued, so re-recording them in the next call is
+// safe, and separate host threads never share a pair.  (Kept, not created and
+// destroyed per call, so that a call inside a stream capture creates nothing.)
+struct ThreadEvents {
+  cudaEvent_t fork[kMaxSideDevices] = {}, join[kMaxSideDevices] = {};
+  ~ThreadEvents() {
+    for (int d = 0; d < kMaxSideDevices; ++d) {
+      if (fork[d] != nullptr) cudaEventDestroy(fork[d]);
+      if (join[d] != nullptr) cudaEventDestroy(join[d]);
+    }
+  }
+};
+thread_local ThreadEvents t_events;
+
+cudaError_t thread_events(cudaEvent_t *fork, cudaEvent_t *join) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxSideDevices) return cudaErrorInvalidDevice;
+  if (t_events.fork[dev] == nullptr &&
+      (e = cudaEventCreateWithFlags(&t_events.fork[dev], cudaEventDisableTiming)) != cudaSuccess)
+    return e;
+  if (t_events.join[dev] == nullptr &&
+      (e = cudaEventCreateWithFlags(&t_events.join[dev], cudaEventDisableTiming)) != cudaSuccess)
+    return e;
+  *fork = t_events.fork[dev];
+  *join = t_events.join[dev];
   return cudaSuccess;
 }
 
@@ -317,11 +354,7 @@ cudaError_t plan_and_bound(const bsa_problem &p, const bsa_mask_spec &m, const b
   cudaError_t e = side_stream(&side);
   if (e != cudaSuccess) return e;
   cudaEvent_t fork = nullptr, join = nullptr;
-  if ((e = cudaEventCreateWithFlags(&fork, cudaEventDisableTiming)) != cudaSuccess) return e;
-  if ((e = cudaEventCreateWithFlags(&join, cudaEventDisableTiming)) != cudaSuccess) {
-    cudaEventDestroy(fork);
-    return e;
-  }
+  if ((e = thread_events(&fork, &join)) != cudaSuccess) return e;
   e = cudaEventRecord(fork, s);
   if (e == cudaSuccess) e = cudaStreamWaitEvent(side, fork, 0);
   if (e == cudaSuccess) e = launch_plan(p, m, o, L, ws, side);
@@ -330,8 +363,6 @@ cudaError_t plan_and_bound(const bsa_problem &p, const bsa_mask_spec &m, const b
   if (e == cudaSuccess) eb = launch_fixed_m_bound(p, mp, o, q, k, L, ws, s);
   // join even when the bound failed to launch, so `s` never runs ahead of the plan
   if (e == cudaSuccess) e = cudaStreamWaitEvent(s, join, 0);
-  cudaEventDestroy(fork);  // released once the recorded work completes
-  cudaEventDestroy(join);
   return e != cudaSuccess ? e : eb;
 }
 

@@ -756,41 +756,58 @@ __global__ void __launch_bounds__(256) k_bwd_delta(const __nv_bfloat16 *__restri
                                                    int64_t sb, int64_t ss, int64_t sh, int B,
                                                    int Sq, int H, int rows_pad,
                                                    const __nv_bfloat16 *__restrict__ resid,
-                                                   float *__restrict__ delta) {
+                                                   float *__restrict__ delta,
+                                                   uint32_t *__restrict__ sem, int64_t n_sem) {
   // D/8 threads per (b, h, i) row vector, 16 bytes of O, dO (and the O
-  // residual) each; rows past Sq (the last q-block's padding) get Delta = 0
+  // residual) each.  A block takes two runs of 256 / (D/8) consecutive rows of
+  // one head (the Delta layout), both runs' loads in flight before either is
+  // reduced; rows past Sq (the last q-block's padding) get Delta = 0.  The
+  // grid also zeroes the dQ semaphores.
   constexpr int TPV = D / 8;
-  const int64_t g = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) / TPV;
+  constexpr int VPB = 256 / TPV;
+  for (int64_t z = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; z < n_sem;
+       z += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    sem[z] = 0u;
   const int t = threadIdx.x % TPV;
   const int64_t total = static_cast<int64_t>(B) * H * rows_pad;
-  const bool in = g < total;  // no early return: the shuffles below need every lane
-  const int i = static_cast<int>(g % rows_pad);
-  const int bh = static_cast<int>(g / rows_pad);
-  const int b = bh / H, h = bh % H;
-  float acc = 0.f;
-  if (in && i < Sq) {
-    const int64_t off = b * sb + static_cast<int64_t>(i) * ss + h * sh + t * 8;
-    const int4 a = __ldg(reinterpret_cast<const int4 *>(o + off));
-    const int4 c = __ldg(reinterpret_cast<const int4 *>(dout + off));
-    int4 r = make_int4(0, 0, 0, 0);
-    if (resid != nullptr)
-      r = __ldg(reinterpret_cast<const int4 *>(resid + ((static_cast<int64_t>(b) * Sq + i) * H + h) * D + t * 8));
-    const uint32_t xa[4] = {static_cast<uint32_t>(a.x), static_cast<uint32_t>(a.y),
-                            static_cast<uint32_t>(a.z), static_cast<uint32_t>(a.w)};
-    const uint32_t xc[4] = {static_cast<uint32_t>(c.x), static_cast<uint32_t>(c.y),
-                            static_cast<uint32_t>(c.z), static_cast<uint32_t>(c.w)};
-    const uint32_t xr[4] = {static_cast<uint32_t>(r.x), static_cast<uint32_t>(r.y),
-                            static_cast<uint32_t>(r.z), static_cast<uint32_t>(r.w)};
+  int64_t g[2];
+  bool in[2];
+  int4 av[2], cv[2], rv[2];
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    g[j] = (static_cast<int64_t>(blockIdx.x) * 2 + j) * VPB + threadIdx.x / TPV;
+    in[j] = g[j] < total;  // no early return: the shuffles below need every lane
+    const int i = static_cast<int>(g[j] % rows_pad);
+    const int bh = static_cast<int>(g[j] / rows_pad);
+    const int b = bh / H, h = bh % H;
+    av[j] = cv[j] = rv[j] = make_int4(0, 0, 0, 0);
+    if (in[j] && i < Sq) {
+      const int64_t off = b * sb + static_cast<int64_t>(i) * ss + h * sh + t * 8;
+      av[j] = __ldg(reinterpret_cast<const int4 *>(o + off));
+      cv[j] = __ldg(reinterpret_cast<const int4 *>(dout + off));
+      if (resid != nullptr)
+        rv[j] = __ldg(reinterpret_cast<const int4 *>(resid + ((static_cast<int64_t>(b) * Sq + i) * H + h) * D + t * 8));
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    const uint32_t xa[4] = {static_cast<uint32_t>(av[j].x), static_cast<uint32_t>(av[j].y),
+                            static_cast<uint32_t>(av[j].z), static_cast<uint32_t>(av[j].w)};
+    const uint32_t xc[4] = {static_cast<uint32_t>(cv[j].x), static_cast<uint32_t>(cv[j].y),
+                            static_cast<uint32_t>(cv[j].z), static_cast<uint32_t>(cv[j].w)};
+    const uint32_t xr[4] = {static_cast<uint32_t>(rv[j].x), static_cast<uint32_t>(rv[j].y),
+                            static_cast<uint32_t>(rv[j].z), static_cast<uint32_t>(rv[j].w)};
+    float acc = 0.f;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const float2 fo = unpack_bf16x2(xa[q]), fd = unpack_bf16x2(xc[q]), fr = unpack_bf16x2(xr[q]);
       acc = fmaf(fo.x + fr.x, fd.x, acc);
       acc = fmaf(fo.y + fr.y, fd.y, acc);
     }
-  }
 #pragma unroll
-  for (int s = TPV / 2; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
-  if (t == 0 && in) delta[g] = acc;
+    for (int sft = TPV / 2; sft > 0; sft >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, sft);
+    if (t == 0 && in[j]) delta[g[j]] = acc;
+  }
 }
 
 // ---------------------------------------------------------------- a7: dQ convert
@@ -886,17 +903,21 @@ cudaError_t launch_bwd_preprocess(const bsa_problem &p, const bsa_options &o, co
   float *delta = reinterpret_cast<float *>(ws + L.delta);
   const __nv_bfloat16 *resid =
       o.keep_o_residual ? reinterpret_cast<const __nv_bfloat16 *>(ws + L.o_resid) : nullptr;
-  const unsigned blocks = static_cast<unsigned>((groups * (p.D / 8) + 255) / 256);
+  // two runs of 256 / (D / 8) vectors per block
+  const int64_t vpb = 2 * (256 / (p.D / 8));
+  const unsigned blocks = static_cast<unsigned>((groups + vpb - 1) / vpb);
+  uint32_t *sem = reinterpret_cast<uint32_t *>(ws + L.sem);
+  const int64_t n_sem = static_cast<int64_t>(p.B) * p.H * L.nM;
   if (p.D == 64)
     k_bwd_delta<64><<<blocks, 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(out),
                                            static_cast<const __nv_bfloat16 *>(dout), p.o_stride[0],
                                            p.o_stride[1], p.o_stride[2], p.B, p.Sq, p.H, rows_pad,
-                                           resid, delta);
+                                           resid, delta, sem, n_sem);
   else
     k_bwd_delta<128><<<blocks, 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(out),
                                             static_cast<const __nv_bfloat16 *>(dout), p.o_stride[0],
                                             p.o_stride[1], p.o_stride[2], p.B, p.Sq, p.H, rows_pad,
-                                            resid, delta);
+                                            resid, delta, sem, n_sem);
   count_launch();
   cudaError_t e = cudaSuccess;
   if (!o.deterministic) {
@@ -905,8 +926,6 @@ cudaError_t launch_bwd_preprocess(const bsa_problem &p, const bsa_options &o, co
     e = cudaMemsetAsync(ws + L.dq_accum, 0, sizeof(float) * static_cast<size_t>(groups) * p.D, s);
     if (e != cudaSuccess) return e;
   }
-  e = cudaMemsetAsync(ws + L.sem, 0, sizeof(uint32_t) * static_cast<size_t>(p.B) * p.H * L.nM, s);
-  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

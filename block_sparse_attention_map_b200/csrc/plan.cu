@@ -444,7 +444,8 @@ __global__ void k_col_fill(const uint8_t *__restrict__ cls, const int32_t *__res
 // Exclusive scan of n counts in shared memory into out[0..n] (out[n] = total),
 // by the whole block: each thread sums a contiguous run, the runs' sums are
 // scanned across the block, then each thread writes its run's offsets.
-__device__ void block_scan_to(const int32_t *cnt, int n, int32_t *out, int32_t *scratch) {
+__device__ void block_scan_to(const int32_t *cnt, int n, int32_t *out, int32_t *scratch,
+                              int32_t *out_s = nullptr) {
   const int per = (n + blockDim.x - 1) / blockDim.x;
   const int lo = min(n, static_cast<int>(threadIdx.x) * per), hi = min(n, lo + per);
   int32_t run = 0;
@@ -471,11 +472,32 @@ __device__ void block_scan_to(const int32_t *cnt, int n, int32_t *out, int32_t *
   int32_t acc = (wid > 0 ? scratch[wid - 1] : 0) + x - run;
   for (int i = lo; i < hi; ++i) {
     out[i] = acc;
+    if (out_s != nullptr) out_s[i] = acc;
     acc += cnt[i];
   }
-  if (threadIdx.x == blockDim.x - 1) out[n] = acc;
+  if (threadIdx.x == blockDim.x - 1) {
+    out[n] = acc;
+    if (out_s != nullptr) out_s[n] = acc;
+  }
   __syncthreads();
 }
+
+// Offsets (in int32 words) of k_plan_fused's shared-memory arrays.
+struct FusedPlanSmem {
+  int rcnt, ccnt, scratch, gw, rptr, cptr, rank, cls, keys;
+  __host__ __device__ FusedPlanSmem(int B, int nM, int nN) {
+    const int BnM = B * nM, BnN = B * nN;
+    rcnt = 0;
+    ccnt = rcnt + BnM;
+    scratch = ccnt + BnN;
+    gw = scratch + 32;
+    rptr = gw + nN;
+    cptr = rptr + BnM + 1;
+    rank = cptr + BnN + 1;
+    cls = rank + BnM * nN;
+    keys = (cls + (BnM * nN + 3) / 4 + 1) & ~1;  // 8-byte boundary for the u64 keys
+  }
+};
 
 struct FusedPlanArgs {
   ClassifyArgs ca;  // row_cnt / col_cnt unused: the counts live in shared memory
@@ -489,19 +511,26 @@ struct FusedPlanArgs {
 // ids: header reset, tile classes with row and column counts, both CSR scans,
 // pi (closed form or greedy), the row lists with rank(m, n), and the column
 // lists sorted by (rank, m) (a warp per column, ranking its entries in shared
-// memory).  Same results as the multi-kernel path.
+// memory).  Same results as the multi-kernel path.  The tile classes, ranks
+// and CSR offsets the later phases read stay in shared memory (their global
+// copies are written, never read back): the phases do not wait on global
+// round trips, which another kernel streaming through HBM beside the planner
+// would lengthen.
 __global__ void __launch_bounds__(1024, 1) k_plan_fused(FusedPlanArgs pa) {
   extern __shared__ int32_t shm[];
   const ClassifyArgs &a = pa.ca;
   const int B = a.B, nM = a.nM, nN = a.nN, BnM = B * nM, BnN = B * nN;
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  int32_t *rcnt = shm;                 // [BnM]
-  int32_t *ccnt = rcnt + BnM;          // [BnN]
-  int32_t *scratch = ccnt + BnN;       // [32]
-  int32_t *gw = scratch + 32;          // [nN] greedy presumed waits
-  // [nw][nM] column keys, on an 8-byte boundary after the int32 arrays
-  unsigned long long *keys =
-      reinterpret_cast<unsigned long long *>(shm + ((BnM + BnN + 32 + nN + 1) & ~1));
+  const FusedPlanSmem F(B, nM, nN);
+  int32_t *rcnt = shm + F.rcnt;        // [BnM]
+  int32_t *ccnt = shm + F.ccnt;        // [BnN]
+  int32_t *scratch = shm + F.scratch;  // [32]
+  int32_t *gw = shm + F.gw;            // [nN] greedy presumed waits
+  int32_t *rptr = shm + F.rptr;        // [BnM + 1]
+  int32_t *cptr = shm + F.cptr;        // [BnN + 1]
+  int32_t *rank_s = shm + F.rank;      // [BnM * nN]
+  uint8_t *cls_s = reinterpret_cast<uint8_t *>(shm + F.cls);  // [BnM * nN]
+  unsigned long long *keys = reinterpret_cast<unsigned long long *>(shm + F.keys);  // [nw][nM]
   if (threadIdx.x < kHdrWords) pa.hdr[threadIdx.x] = 0u;
   for (int i = threadIdx.x; i < BnN; i += blockDim.x) ccnt[i] = 0;
   __syncthreads();
@@ -524,6 +553,7 @@ __global__ void __launch_bounds__(1024, 1) k_plan_fused(FusedPlanArgs pa) {
       }
       if (n < nN) {
         crow[n] = c;
+        cls_s[row * nN + n] = c;
         if (c != BSA_TILE_EMPTY) atomicAdd(ccnt + b * nN + n, 1);
       }
       cnt += __popc(__ballot_sync(0xffffffffu, c != BSA_TILE_EMPTY));
@@ -531,8 +561,8 @@ __global__ void __launch_bounds__(1024, 1) k_plan_fused(FusedPlanArgs pa) {
     if (lane == 0) rcnt[row] = cnt;
   }
   __syncthreads();
-  block_scan_to(rcnt, BnM, pa.row_ptr, scratch);
-  block_scan_to(ccnt, BnN, pa.col_ptr, scratch);
+  block_scan_to(rcnt, BnM, pa.row_ptr, scratch, rptr);
+  block_scan_to(ccnt, BnN, pa.col_ptr, scratch, cptr);
   // pi
   const bool in_ws = order_in_workspace(pa.order);
   if (pa.order == BSA_ORDER_GREEDY) {
@@ -574,7 +604,7 @@ __global__ void __launch_bounds__(1024, 1) k_plan_fused(FusedPlanArgs pa) {
       __syncthreads();
       const int c = chosen;
       for (int bm = wid; bm < BnM; bm += nw) {
-        const uint8_t *crow = a.cls + static_cast<int64_t>(bm) * nN;
+        const uint8_t *crow = cls_s + bm * nN;
         if (crow[c] == BSA_TILE_EMPTY) continue;
         for (int n = lane; n < nN; n += 32)
           if (crow[n] != BSA_TILE_EMPTY && gw[n] != kPlaced) atomicAdd(gw + n, 1);
@@ -587,8 +617,8 @@ __global__ void __launch_bounds__(1024, 1) k_plan_fused(FusedPlanArgs pa) {
   __syncthreads();
   // row lists and rank(m, n), a warp per row block
   for (int row = wid; row < BnM; row += nw) {
-    const uint8_t *crow = a.cls + static_cast<int64_t>(row) * nN;
-    int pos = pa.row_ptr[row];
+    const uint8_t *crow = cls_s + row * nN;
+    int pos = rptr[row];
     for (int n0 = 0; n0 < nN; n0 += 32) {
       const int n = n0 + lane;
       const uint8_t c = n < nN ? crow[n] : BSA_TILE_EMPTY;
@@ -598,6 +628,7 @@ __global__ void __launch_bounds__(1024, 1) k_plan_fused(FusedPlanArgs pa) {
       pos += __popc(bal);
     }
     int32_t *rk = pa.rank + static_cast<int64_t>(row) * nN;
+    int32_t *rks = rank_s + row * nN;
     int r = 0;
     for (int t0 = 0; t0 < nN; t0 += 32) {
       const int t = t0 + lane;
@@ -605,7 +636,11 @@ __global__ void __launch_bounds__(1024, 1) k_plan_fused(FusedPlanArgs pa) {
       if (t < nN) n = in_ws ? pa.perm[t] : closed_form_order(pa.order, t, nN);
       const bool ne = n >= 0 && crow[n] != BSA_TILE_EMPTY;
       const uint32_t bal = __ballot_sync(0xffffffffu, ne);
-      if (n >= 0) rk[n] = ne ? r + __popc(bal & ((1u << lane) - 1u)) : -1;
+      if (n >= 0) {
+        const int32_t v = ne ? r + __popc(bal & ((1u << lane) - 1u)) : -1;
+        rk[n] = v;
+        rks[n] = v;
+      }
       r += __popc(bal);
     }
   }
@@ -620,11 +655,11 @@ __global__ void __launch_bounds__(1024, 1) k_plan_fused(FusedPlanArgs pa) {
       unsigned long long key = 0;
       bool ne = false;
       if (m < nM) {
-        const int64_t t = (static_cast<int64_t>(b) * nM + m) * nN + n;
-        const uint8_t k = a.cls[t];
+        const int t = (b * nM + m) * nN + n;
+        const uint8_t k = cls_s[t];
         ne = k != BSA_TILE_EMPTY;
         if (ne)
-          key = (static_cast<unsigned long long>(pa.rank[t]) << 32) |
+          key = (static_cast<unsigned long long>(rank_s[t]) << 32) |
                 (static_cast<unsigned long long>(m) << 1) | (k == BSA_TILE_FULL ? 1ull : 0ull);
       }
       const uint32_t bal = __ballot_sync(0xffffffffu, ne);
@@ -632,7 +667,7 @@ __global__ void __launch_bounds__(1024, 1) k_plan_fused(FusedPlanArgs pa) {
       cnt += __popc(bal);
     }
     __syncwarp();
-    const int base = pa.col_ptr[bn];
+    const int base = cptr[bn];
     for (int e = lane; e < cnt; e += 32) {
       const unsigned long long ke = mykeys[e];
       int pos = 0;
@@ -660,8 +695,8 @@ __global__ void __launch_bounds__(1024, 1) k_plan_fused(FusedPlanArgs pa) {
 
 // Shared memory of k_plan_fused, and whether the fused path applies.
 inline size_t fused_plan_smem(int B, int nM, int nN) {
-  const size_t ints = (static_cast<size_t>(B) * nM + static_cast<size_t>(B) * nN + 32 + nN + 1) & ~size_t{1};
-  return sizeof(int32_t) * ints + sizeof(unsigned long long) * 32 * static_cast<size_t>(nM);
+  const FusedPlanSmem F(B, nM, nN);
+  return sizeof(int32_t) * static_cast<size_t>(F.keys) + sizeof(unsigned long long) * 32 * static_cast<size_t>(nM);
 }
 
 inline unsigned cdiv(int64_t a, int64_t b) { return static_cast<unsigned>((a + b - 1) / b); }

@@ -271,7 +271,8 @@ BSA_API bsa_status bsa_fixed_m_bound(const bsa_problem *prob, const bsa_mask_spe
  * (as bsa_fixed_m_bound), the result identical to calling the two in turn.  For
  * every mask but BSA_MASK_VARLEN (whose key validity the bound reads from the
  * plan) the planner runs on a non-blocking stream of the library's own, created
- * once per device, concurrently with the bound's pass over Q and K on `stream`:
+ * once per device (with a fork / join event pair per host thread, created on
+ * first use), concurrently with the bound's pass over Q and K on `stream`:
  * the side stream waits for an event recorded on `stream` and `stream` waits for
  * the planner before the call returns, so all later work on `stream` sees both
  * results, and a stream capture on `stream` records the same fork and join.
