@@ -64,7 +64,7 @@ WsLayout compute_layout(const bsa_problem &p) {
   L.fwd_end = off;
   L.delta = take(4 * static_cast<size_t>(B * H * nM * kTile));
   L.dq_accum = take(4 * static_cast<size_t>(B * H * nM * kTile * p.D));
-  L.sem = take(4 * static_cast<size_t>(B * H * nM));
+  L.sem = take(4 * 4 * static_cast<size_t>(B * H * nM));  // one per 32-row quarter of a q-block
   L.o_resid = take(2 * static_cast<size_t>(B * H * p.Sq * p.D));
   L.total = off;
   return L;

@@ -9,7 +9,8 @@
 //     dQ_m part = dS K_n and adds it to the fp32 dQ accumulator.  With the
 //     deterministic protocol the add for q-block m waits until the per-m_block
 //     semaphore equals rank(m, n), then increments it, so every dQ row sums its
-//     contributions in the fixed order pi ("Add more optimal dk order optional
+//     contributions in the fixed order pi (the semaphore is kept per 32-row
+//     quarter of the block, one chain per dQ warp; "Add more optimal dk order optional
 //     arg", flash-attention PR #2512, "Sliding window perf issue" and "A simplish
 //     fix").  Columns are handed out by an atomic ticket in pi order, so a column
 //     only ever waits on columns that some running CTA already holds.
@@ -28,7 +29,8 @@
 //               ids), P^T back to TMEM as the
 //               A operand of dV, dS^T to shared memory (128-byte swizzle, K-major
 //               for dK, read MN-major as the A operand of dQ), dK/dV epilogue
-//   warps 12..15 dQ: one query row per thread, semaphore wait, vector reductions
+//   warps 12..15 dQ: one query row per thread; each warp waits on and releases
+//               its own quarter's semaphore around its vector reductions
 // TMEM columns: S^T / P^T [0,128)  dP^T / dQ [128,256)  dV [256,256+D)  dK [256+D,256+2D)
 #include <cfloat>
 
@@ -80,7 +82,7 @@ struct BwdSmem {
                        bSFull = bDOEmpty + NDO, bDPFull = bSFull + 1, bPReady = bDPFull + 1,
                        bDSReady = bPReady + 1, bDSFree = bDSReady + 1, bDQFull = bDSFree + 1,
                        bDQFree = bDQFull + 1, bDKVFull = bDQFree + 1, bDKVFree = bDKVFull + 1,
-                       bVecReady = bDKVFree + 1, bDQAdded = bVecReady + 2, bFinal = bDQAdded + 2,
+                       bVecReady = bDKVFree + 1, bFinal = bVecReady + 2,
                        kNumBars = bFinal + 1;
   static constexpr int kMisc = kBar + kNumBars * 8;
   static constexpr int kAlloc = kMisc + 16;
@@ -170,7 +172,6 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
           i == L::bVecReady + 1)
         cnt = kComputeThreads;
       if (i == L::bDQFree) cnt = 128;
-      if (i == L::bDQAdded || i == L::bDQAdded + 1) cnt = 4;
       mbar_init(&bars[i], cnt);
     }
     *abort_flag = 0;
@@ -687,7 +688,8 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
           read_dq();
         }
         ahead = false;
-        uint32_t *sem = p.sem + bh * p.nM + m;
+        // one semaphore per 32-row quarter of the q-block: this warp's rows
+        uint32_t *sem = p.sem + (bh * p.nM + m) * 4 + quarter;
         int ok = 1;
         if (p.deterministic) {
           if (lane == 0) ok = sem_wait(sem, rank, p.sem_timeout_ns, p.hdr + kHdrStatus) ? 1 : 0;
@@ -719,20 +721,14 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
           ahead = true;
         }
         if (p.deterministic) {
-          // Pass the turn on once all four warps' adds are ordered before it:
-          // each thread's adds precede its device-scope acq_rel fence, the
-          // warps meet on a CTA mbarrier (release / acquire), and the one
-          // release add on the semaphore is cumulative over what that thread
-          // has observed.  (A second, sequentially consistent fence before the
-          // release cost 10% of this kernel and is not needed for the order.)
+          // Pass this quarter's turn on once the warp's adds are ordered before
+          // it: each thread's adds precede its device-scope acq_rel fence, the
+          // warp synchronises, and lane 0's release add on the semaphore is
+          // cumulative over what it has observed.  Each warp runs its own
+          // quarter's chain: a hop carries 16 KB, and no warp waits for another.
           asm volatile("fence.acq_rel.gpu;" ::: "memory");
           __syncwarp();
-          if (lane == 0) mbar_arrive(&bars[L::bDQAdded + (ec & 1)]);
-          if (warp == 12 && lane == 0) {
-            if (wd.wait(&bars[L::bDQAdded + (ec & 1)], (ec >> 1) & 1)) {
-              red_release_gpu_add(sem, 1u);
-            }
-          }
+          if (lane == 0) red_release_gpu_add(sem, 1u);
           __syncwarp();
         }
       }
@@ -907,7 +903,7 @@ cudaError_t launch_bwd_preprocess(const bsa_problem &p, const bsa_options &o, co
   const int64_t vpb = 2 * (256 / (p.D / 8));
   const unsigned blocks = static_cast<unsigned>((groups + vpb - 1) / vpb);
   uint32_t *sem = reinterpret_cast<uint32_t *>(ws + L.sem);
-  const int64_t n_sem = static_cast<int64_t>(p.B) * p.H * L.nM;
+  const int64_t n_sem = static_cast<int64_t>(p.B) * p.H * L.nM * 4;  // a quarter each
   if (p.D == 64)
     k_bwd_delta<64><<<blocks, 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(out),
                                            static_cast<const __nv_bfloat16 *>(dout), p.o_stride[0],

@@ -210,7 +210,8 @@ typedef struct bsa_workspace_view {
   size_t off_gate;             /* int32  [B, H]       1 = fixed-m, 0 = online        */
   size_t off_delta;            /* fp32   [B, H, nM*128]  backward Delta              */
   size_t off_dq_accum;         /* fp32   backward dQ accumulator                     */
-  size_t off_sem;              /* int32  [B, H, nM]   dQ semaphores                  */
+  size_t off_sem;              /* int32  [B, H, nM, 4] dQ semaphores, one per 32-row
+                                  quarter of each q-block                          */
   size_t off_kbar;             /* fp32   [B, H_kv, D] k-smoothing center             */
   size_t off_qdot;             /* fp32   [B, H, Sq]   q_i . center                   */
   size_t off_o_resid;          /* bf16   [B, Sq, H, D] O - bf16(O) (keep_o_residual)  */
