@@ -442,27 +442,41 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       if ((mk.flags & BSA_MASK_KV_VALID_LEN) && j >= mk.kv_valid_len[k.b]) qhi = -1;
       const int seg_j = (use_seg && row_ok) ? mk.seg_kv[static_cast<int64_t>(k.b) * p.Skv + j] : INT_MIN;
       uint8_t *ds_tile = sm + L::kDS;
+      // The entry's list word and this thread's -LSE*log2e (half 0; -inf where
+      // the row has no key or lies past Sq) or -Delta (half 1) of the q-block,
+      // negated so the element loops are one packed FMA / add.  Fetched ahead
+      // (the list word two entries ahead, the value one entry ahead, its
+      // address then known) so that both global loads fall under the previous
+      // entries' work instead of delaying this entry's staging.
+      auto vec_of = [&](int xx, uint32_t ent_x) -> float {
+        const int64_t bh_x = static_cast<int64_t>(k.b) * p.H + k.head(xx);
+        const int i_x = static_cast<int>(ent_x & kIndexMask) * kTile + r;
+        if (half == 0) {
+          float v = -INFINITY;
+          if (i_x < p.Sq) {
+            const float lv = p.lse[bh_x * p.Sq + i_x];
+            if (lv != -INFINITY) v = -lv * kLog2e;
+          }
+          return v;
+        }
+        return -p.delta[bh_x * p.nM * kTile + i_x];
+      };
+      uint32_t ent_a = k.tot > 0 ? p.col_ent[k.entry(0)] : 0u;  // entry x
+      uint32_t ent_b = k.tot > 1 ? p.col_ent[k.entry(1)] : 0u;  // entry x + 1
+      float vec_a = k.tot > 0 ? vec_of(0, ent_a) : 0.f;
       for (int x = 0; x < k.tot; ++x, ++ec) {
-        const int e = k.entry(x);
-        const int64_t bh = static_cast<int64_t>(k.b) * p.H + k.head(x);
-        const uint32_t ent = p.col_ent[e];
+        const uint32_t ent = ent_a;
+        const float vecv = vec_a;
+        if (x + 1 < k.tot) vec_a = vec_of(x + 1, ent_b);
+        ent_a = ent_b;
+        if (x + 2 < k.tot) ent_b = p.col_ent[k.entry(x + 2)];
         const int m = static_cast<int>(ent & kIndexMask);
         const bool full = (ent & kFullBit) != 0;
-        // stage -LSE*log2e (half 0; -inf where the row has no key or lies past
-        // Sq) and -Delta (half 1) of this q-block, negated so the element loops
-        // are one packed FMA / add
         {
-          const int i = m * kTile + r;
-          if (half == 0) {
-            float nl2 = -INFINITY;
-            if (i < p.Sq) {
-              const float lv = p.lse[bh * p.Sq + i];
-              if (lv != -INFINITY) nl2 = -lv * kLog2e;
-            }
-            vec_nl[(ec & 1) * kTile + r] = nl2;
-          } else {
-            vec_nd[(ec & 1) * kTile + r] = -p.delta[bh * p.nM * kTile + i];
-          }
+          if (half == 0)
+            vec_nl[(ec & 1) * kTile + r] = vecv;
+          else
+            vec_nd[(ec & 1) * kTile + r] = vecv;
           mbar_arrive(&bars[L::bVecReady + (ec & 1)]);
         }
         // allowed-query bits of this half's two 32-query words for this key

@@ -394,8 +394,12 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       }
       const int seg_i = (use_seg && row_ok) ? mk.seg_q[static_cast<int64_t>(b) * p.Sq + i] : INT_MIN;
 
+      // the tile's list word is fetched one tile ahead, its latency under the
+      // previous tile's softmax
+      uint32_t ent_next = p.row_ent[rs];
       for (int j = rs; j < re; ++j, ++tcount) {
-        const uint32_t ent = p.row_ent[j];
+        const uint32_t ent = ent_next;
+        if (j + 1 < re) ent_next = p.row_ent[j + 1];
         const int n = static_cast<int>(ent & kIndexMask);
         const bool full = (ent & kFullBit) != 0;
         // allowed-key bits of this tile for this row (range AND segment ids),
