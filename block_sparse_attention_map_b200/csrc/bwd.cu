@@ -760,6 +760,8 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
 }
 
 // ---------------------------------------------------------------- a4: Delta
+constexpr int kDeltaRuns = 2;  // runs of consecutive rows per block, loads all in flight
+
 template <int D>
 __global__ void __launch_bounds__(256) k_bwd_delta(const __nv_bfloat16 *__restrict__ o,
                                                    const __nv_bfloat16 *__restrict__ dout,
@@ -769,9 +771,9 @@ __global__ void __launch_bounds__(256) k_bwd_delta(const __nv_bfloat16 *__restri
                                                    float *__restrict__ delta,
                                                    uint32_t *__restrict__ sem, int64_t n_sem) {
   // D/8 threads per (b, h, i) row vector, 16 bytes of O, dO (and the O
-  // residual) each.  A block takes two runs of 256 / (D/8) consecutive rows of
-  // one head (the Delta layout), both runs' loads in flight before either is
-  // reduced; rows past Sq (the last q-block's padding) get Delta = 0.  The
+  // residual) each.  A block takes kDeltaRuns runs of 256 / (D/8) consecutive
+  // rows of one head (the Delta layout), every run's loads in flight before any
+  // is reduced; rows past Sq (the last q-block's padding) get Delta = 0.  The
   // grid also zeroes the dQ semaphores.
   constexpr int TPV = D / 8;
   constexpr int VPB = 256 / TPV;
@@ -780,12 +782,12 @@ __global__ void __launch_bounds__(256) k_bwd_delta(const __nv_bfloat16 *__restri
     sem[z] = 0u;
   const int t = threadIdx.x % TPV;
   const int64_t total = static_cast<int64_t>(B) * H * rows_pad;
-  int64_t g[2];
-  bool in[2];
-  int4 av[2], cv[2], rv[2];
+  int64_t g[kDeltaRuns];
+  bool in[kDeltaRuns];
+  int4 av[kDeltaRuns], cv[kDeltaRuns], rv[kDeltaRuns];
 #pragma unroll
-  for (int j = 0; j < 2; ++j) {
-    g[j] = (static_cast<int64_t>(blockIdx.x) * 2 + j) * VPB + threadIdx.x / TPV;
+  for (int j = 0; j < kDeltaRuns; ++j) {
+    g[j] = (static_cast<int64_t>(blockIdx.x) * kDeltaRuns + j) * VPB + threadIdx.x / TPV;
     in[j] = g[j] < total;  // no early return: the shuffles below need every lane
     const int i = static_cast<int>(g[j] % rows_pad);
     const int bh = static_cast<int>(g[j] / rows_pad);
@@ -800,7 +802,7 @@ __global__ void __launch_bounds__(256) k_bwd_delta(const __nv_bfloat16 *__restri
     }
   }
 #pragma unroll
-  for (int j = 0; j < 2; ++j) {
+  for (int j = 0; j < kDeltaRuns; ++j) {
     const uint32_t xa[4] = {static_cast<uint32_t>(av[j].x), static_cast<uint32_t>(av[j].y),
                             static_cast<uint32_t>(av[j].z), static_cast<uint32_t>(av[j].w)};
     const uint32_t xc[4] = {static_cast<uint32_t>(cv[j].x), static_cast<uint32_t>(cv[j].y),
@@ -913,8 +915,8 @@ cudaError_t launch_bwd_preprocess(const bsa_problem &p, const bsa_options &o, co
   float *delta = reinterpret_cast<float *>(ws + L.delta);
   const __nv_bfloat16 *resid =
       o.keep_o_residual ? reinterpret_cast<const __nv_bfloat16 *>(ws + L.o_resid) : nullptr;
-  // two runs of 256 / (D / 8) vectors per block
-  const int64_t vpb = 2 * (256 / (p.D / 8));
+  // kDeltaRuns runs of 256 / (D / 8) vectors per block
+  const int64_t vpb = kDeltaRuns * (256 / (p.D / 8));
   const unsigned blocks = static_cast<unsigned>((groups + vpb - 1) / vpb);
   uint32_t *sem = reinterpret_cast<uint32_t *>(ws + L.sem);
   const int64_t n_sem = static_cast<int64_t>(p.B) * p.H * L.nM * 4;  // a quarter each

@@ -681,7 +681,9 @@ __global__ void __launch_bounds__(256) k_key_centers(const NormArgs a) {
 // flight; a block takes kVPB consecutive vectors of one batch row (rows are
 // contiguous over heads).  Per-head maxima are reduced in shared memory first,
 // then one global atomic per head and block.
-template <int D>
+// CENTER: k-smoothing on (a.center != 0), a compile-time choice so that the
+// plain norm's inner loop carries no per-element test of it
+template <int D, bool CENTER>
 __global__ void __launch_bounds__(256) k_row_norms(const NormArgs a) {
   constexpr int kT = D / 32;          // threads per vector, four 16-byte loads each
   constexpr int kVPB = 256 / kT;      // vectors per block and pass
@@ -728,8 +730,8 @@ __global__ void __launch_bounds__(256) k_row_norms(const NormArgs a) {
       const int row = in[j] ? static_cast<int>(vv[j] / Hx) : 0, hh = in[j] ? static_cast<int>(vv[j] % Hx) : 0;
       float acc = 0.f, dot = 0.f;
       if (in[j]) {
-        const float *c = a.center ? a.kbar + (static_cast<int64_t>(b) * a.Hk + (is_key ? hh : hh / grp)) * D + 32 * t
-                                  : nullptr;
+        const float *c = CENTER ? a.kbar + (static_cast<int64_t>(b) * a.Hk + (is_key ? hh : hh / grp)) * D + 32 * t
+                                : nullptr;
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           const uint32_t xw[4] = {static_cast<uint32_t>(w[j][u].x), static_cast<uint32_t>(w[j][u].y),
@@ -737,7 +739,7 @@ __global__ void __launch_bounds__(256) k_row_norms(const NormArgs a) {
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             float2 f = unpack_bf16x2(xw[q]);
-            if (c != nullptr) {
+            if (CENTER) {
               const float2 cc = *reinterpret_cast<const float2 *>(c + 8 * u + 2 * q);
               if (is_key) {
                 f.x -= cc.x;
@@ -765,7 +767,7 @@ __global__ void __launch_bounds__(256) k_row_norms(const NormArgs a) {
         } else {
           const int64_t idx = (static_cast<int64_t>(b) * H + hh) * S + row;
           a.qnorm[idx] = nrm;
-          if (a.center) a.qdot[idx] = dot;
+          if (CENTER) a.qdot[idx] = dot;
         }
         if (valid) atomicMax(&smax[hh], __float_as_uint(nrm));
       }
@@ -888,8 +890,13 @@ cudaError_t launch_fixed_m_bound(const bsa_problem &p, const MaskParams &mp,
   const int64_t want = std::max<int64_t>(1, (4 * 148) / (static_cast<int64_t>(p.B) * (na.only_q ? 1 : 2)));
   const int bpb = static_cast<int>(std::min<int64_t>(want, (vec + vpb - 1) / vpb));
   const dim3 grid(static_cast<unsigned>(p.B * bpb), na.only_q ? 1u : 2u);
-  if (p.D == 64) k_row_norms<64><<<grid, 256, smem, s>>>(na);
-  else k_row_norms<128><<<grid, 256, smem, s>>>(na);
+  if (p.D == 64) {
+    if (na.center) k_row_norms<64, true><<<grid, 256, smem, s>>>(na);
+    else k_row_norms<64, false><<<grid, 256, smem, s>>>(na);
+  } else {
+    if (na.center) k_row_norms<128, true><<<grid, 256, smem, s>>>(na);
+    else k_row_norms<128, false><<<grid, 256, smem, s>>>(na);
+  }
   count_launch();
   return cudaGetLastError();
 }
