@@ -202,6 +202,11 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
     if ((smem_u32(sm) & 1023u) != 0u) wd.trip(BSA_ERR_UNSUPPORTED);
   }
   __syncthreads();
+  // launched as a programmatic dependent of the Delta pass: the setup above
+  // touches only the plan header; Delta, the semaphores and the accumulator
+  // are read after the pass has completed.  The dQ convert may then launch.
+  pdl_wait();
+  pdl_trigger();
 
   const uint32_t T_S = tmem, T_DP = tmem + 128, T_DV = tmem + 256, T_DK = tmem + 256 + D;
   constexpr uint32_t kIdS = idesc_bf16_f32(128, 128, 0, 0);      // S^T, dP^T: both K-major
@@ -777,6 +782,8 @@ __global__ void __launch_bounds__(256) k_bwd_delta(const __nv_bfloat16 *__restri
   // grid also zeroes the dQ semaphores.
   constexpr int TPV = D / 8;
   constexpr int VPB = 256 / TPV;
+  pdl_wait();  // O comes from the forward, launched just before
+  pdl_trigger();
   for (int64_t z = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; z < n_sem;
        z += static_cast<int64_t>(gridDim.x) * blockDim.x)
     sem[z] = 0u;
@@ -836,6 +843,7 @@ __global__ void __launch_bounds__(256) k_dq_convert(const float *__restrict__ ac
   constexpr int kC = D / 4, kRows = 32, kLD = D + 4;
   constexpr int kPer = kC * kRows / 256;  // float4 loads per thread
   __shared__ __align__(16) float tile[kRows * kLD];
+  pdl_wait();  // the accumulator is final once the backward main kernel completed
   const int64_t bhm = blockIdx.x / (kTile / kRows);
   const int r0 = static_cast<int>(blockIdx.x % (kTile / kRows)) * kRows;
   const int m = static_cast<int>(bhm % nM);
@@ -900,7 +908,9 @@ cudaError_t run_bwd_main(const BwdParams &bp, const CUtensorMap &tq, const CUten
     attr = true;
   }
   const int grid = std::max(1, std::min(bp.n_tickets, sm_count_bwd()));
-  k_attn_bwd<D, NQ, NDO><<<grid, kThreads, L::kAlloc, s>>>(tq, tk, tv, tdo, bp);
+  const cudaError_t e = launch_pdl(k_attn_bwd<D, NQ, NDO>, dim3(grid), dim3(kThreads), L::kAlloc, s,
+                                   tq, tk, tv, tdo, bp);
+  if (e != cudaSuccess) return e;
   count_launch();
   return cudaGetLastError();
 }
@@ -920,18 +930,13 @@ cudaError_t launch_bwd_preprocess(const bsa_problem &p, const bsa_options &o, co
   const unsigned blocks = static_cast<unsigned>((groups + vpb - 1) / vpb);
   uint32_t *sem = reinterpret_cast<uint32_t *>(ws + L.sem);
   const int64_t n_sem = static_cast<int64_t>(p.B) * p.H * L.nM * 4;  // a quarter each
-  if (p.D == 64)
-    k_bwd_delta<64><<<blocks, 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(out),
-                                           static_cast<const __nv_bfloat16 *>(dout), p.o_stride[0],
-                                           p.o_stride[1], p.o_stride[2], p.B, p.Sq, p.H, rows_pad,
-                                           resid, delta, sem, n_sem);
-  else
-    k_bwd_delta<128><<<blocks, 256, 0, s>>>(static_cast<const __nv_bfloat16 *>(out),
-                                            static_cast<const __nv_bfloat16 *>(dout), p.o_stride[0],
-                                            p.o_stride[1], p.o_stride[2], p.B, p.Sq, p.H, rows_pad,
-                                            resid, delta, sem, n_sem);
+  // a programmatic dependent of the forward (which reads O first after it)
+  cudaError_t e = launch_pdl(p.D == 64 ? k_bwd_delta<64> : k_bwd_delta<128>, dim3(blocks), dim3(256), 0, s,
+                             static_cast<const __nv_bfloat16 *>(out), static_cast<const __nv_bfloat16 *>(dout),
+                             p.o_stride[0], p.o_stride[1], p.o_stride[2], p.B, p.Sq, p.H, rows_pad, resid,
+                             delta, sem, n_sem);
+  if (e != cudaSuccess) return e;
   count_launch();
-  cudaError_t e = cudaSuccess;
   if (!o.deterministic) {
     // atomic adds need a zeroed accumulator; the deterministic path initialises
     // it with the first contributor's stores instead
@@ -993,12 +998,11 @@ cudaError_t launch_bwd_convert(const bsa_problem &p, void *dq, const WsLayout &L
   const unsigned blocks = static_cast<unsigned>(static_cast<int64_t>(p.B) * p.H * L.nM * (kTile / 32));
   const int32_t *row_ptr = reinterpret_cast<const int32_t *>(ws + L.row_ptr);
   __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(dq);
-  if (p.D == 64)
-    k_dq_convert<64><<<blocks, 256, 0, s>>>(acc, p.B, p.H, p.Sq, L.nM, row_ptr, out, p.q_stride[0],
-                                            p.q_stride[1], p.q_stride[2]);
-  else
-    k_dq_convert<128><<<blocks, 256, 0, s>>>(acc, p.B, p.H, p.Sq, L.nM, row_ptr, out, p.q_stride[0],
-                                             p.q_stride[1], p.q_stride[2]);
+  // a programmatic dependent of the backward main kernel
+  const cudaError_t e = launch_pdl(p.D == 64 ? k_dq_convert<64> : k_dq_convert<128>, dim3(blocks), dim3(256), 0,
+                                   s, acc, p.B, p.H, p.Sq, L.nM, row_ptr, out, p.q_stride[0], p.q_stride[1],
+                                   p.q_stride[2]);
+  if (e != cudaSuccess) return e;
   count_launch();
   return cudaGetLastError();
 }

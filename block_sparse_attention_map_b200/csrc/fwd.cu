@@ -193,6 +193,7 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
     if ((smem_u32(sm) & 1023u) != 0u) wd.trip(BSA_ERR_UNSUPPORTED);
   }
   __syncthreads();
+  pdl_trigger();  // the Delta pass of a backward may launch (it waits for our completion)
 
   constexpr uint32_t kIdescS = idesc_bf16_f32(128, 128, 0, 0);
   constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, 0, 1);

@@ -5,6 +5,7 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <utility>
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -119,6 +120,25 @@ cudaError_t launch_bwd_convert(const bsa_problem &p, void *dq, const WsLayout &L
                                cudaStream_t s);
 
 void count_launch(int n = 1);
+
+// Launch with programmatic stream serialization: the kernel may start while
+// the stream's preceding kernel finishes, and must call pdl_wait() before it
+// touches anything that kernel writes or reads.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t s, Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // bsa_attn_fwd; side_stream_ok = false never forks work onto the library's side
 // stream (no stream or event is created).

@@ -315,6 +315,15 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
+// Programmatic dependent launch.  pdl_wait: block until the preceding kernel
+// of the stream has completed and its memory operations are visible (a no-op
+// when this kernel was launched without a programmatic dependency); every
+// global access to data the predecessor writes, or reads, comes after it.
+// pdl_trigger: let the next kernel of the stream launch (its CTAs start as
+// this kernel's leave the SMs; it still waits for our completion in pdl_wait).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
