@@ -27,8 +27,9 @@
 //               query mask of PARTIAL tiles (a prefix key is seen by every query;
 //               other keys by a query range thinned by the dilation, AND segment
 //               ids), P^T back to TMEM as the
-//               A operand of dV, dS^T to shared memory (128-byte swizzle, K-major
-//               for dK, read MN-major as the A operand of dQ), dK/dV epilogue
+//               A operand of dV, dS^T to TMEM over the read dP^T columns (the A
+//               operand of dK) and to shared memory (128-byte swizzle, read
+//               MN-major as the A operand of dQ), dK/dV epilogue
 //   warps 12..15 dQ: one query row per thread; each warp waits on and releases
 //               its own quarter's semaphore around its vector reductions
 // TMEM columns: S^T / P^T [0,128)  dP^T / dQ [128,256)  dV [256,256+D)  dK [256+D,256+2D)
@@ -285,7 +286,7 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
     }
     } else if (run && warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    // Per entry e: dV(e), S^T(e+1), dQ(e), dK(e), dP^T(e+1).  S^T(e+1) reuses the
+    // Per entry e: dV(e), S^T(e+1), dK(e), dQ(e), dP^T(e+1).  S^T(e+1) reuses the
     // columns dV(e) reads P^T from: tcgen05.mma ops issued by one thread run in
     // issue order, so it follows dV(e) without a wait and the next entry's
     // exponentials overlap this entry's dK and dQ.
@@ -356,8 +357,19 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
           if (!last && !issue_s(ec + 1)) { stop = true; break; }
           if (!wd.wait(&bars[L::bDSReady], ec & 1)) { stop = true; break; }
           tc_fence_after();
-          // dQ_m part = dS K_n   (dS read MN-major from the dS^T tile), first: the
-          // dQ warps' read of it gates the next dP^T, which shares its columns
+          // dK += dS^T Q_m, dS^T from TMEM (the compute warps wrote it over the
+          // dP^T columns they had read, laid out like P^T), so only Q comes
+          // from shared memory
+          const uint32_t q_addr = smem_u32(sm + L::kQ + qs * kTB);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts(T_DK, T_DP + kk * 8 + (kk >= 4 ? 32 : 0), sw128_desc(q_addr + kk * 2048, 16384, 1024),
+                   kIdKV, (!first || kk > 0) ? 1u : 0u);
+          mma_commit(&bars[L::bQEmpty + qs]);
+          // dQ_m part = dS K_n (dS read MN-major from the shared dS^T tile) into
+          // the dP^T columns: issued after dK, which reads dS^T from them
+          // (tcgen05.mma ops of one thread run in issue order).  The dQ warps'
+          // read of it gates the next dP^T, which shares those columns.
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
             mma_ss(T_DP, sw128_desc(ds_addr + kk * 2048, 16384, 1024),
@@ -365,15 +377,6 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
           mma_commit(&bars[L::bDQFull]);
           // K's last use is the column's last dQ: its buffer takes the next V
           if (last) mma_commit(&bars[L::bXFree + kb]);
-          // dK += dS^T Q_m
-          const uint32_t q_addr = smem_u32(sm + L::kQ + qs * kTB);
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-            mma_ss(T_DK, sw128_desc(ds_addr + off, 16, 1024),
-                   sw128_desc(q_addr + kk * 2048, 16384, 1024), kIdKV, (!first || kk > 0) ? 1u : 0u);
-          }
-          mma_commit(&bars[L::bQEmpty + qs]);
           mma_commit(&bars[L::bDSFree]);
           if (last) {
             mma_commit(&bars[L::bDKVFull]);
@@ -565,8 +568,10 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&bars[L::bPReady]);
-        // phase 2: dS^T = P^T o (dP^T - Delta) in fp32 from the fp16 P^T -> bf16
-        // shared tile (128-byte swizzle, K-major)
+        // phase 2: dS^T = P^T o (dP^T - Delta) in fp32 from the fp16 P^T -> bf16,
+        // into the shared tile (128-byte swizzle, K-major; the dQ MMA reads it
+        // MN-major) and into TMEM over this half's dP^T columns, already read
+        // (the A operand of dK, laid out like P^T for dV)
         if (ec >= 1 && !wwait(&bars[L::bDSFree], (ec - 1) & 1)) { stop = true; break; }
         if (!wwait(&bars[L::bDPFull], ec & 1)) { stop = true; break; }
         tc_fence_after();
@@ -602,8 +607,12 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
             *reinterpret_cast<int4 *>(dst) =
                 make_int4(dk2[4 * u], dk2[4 * u + 1], dk2[4 * u + 2], dk2[4 * u + 3]);
           }
+          // piece -> TMEM columns [8sc, 8sc+8) of this half: dP^T columns
+          // already read (the load in flight is of columns 16(sc+1) on)
+          tmem_st8(T_DP + lane_off + 64 * half + 8 * sc, dk2);
           if (sc + 1 < 4) tmem_wait_ld();
         }
+        tmem_wait_st();
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(&bars[L::bDSReady]);
