@@ -158,7 +158,7 @@ def make_problem(q, k, v, o=None, scale: Optional[float] = None) -> Problem:
     p.q_stride[:] = _strides(q)
     p.k_stride[:] = _strides(k)
     p.v_stride[:] = _strides(v)
-    p.o_stride[:] = _strides(o) if o is not None else (Sq * H * D, H * D, D)
+    p.o_stride[:] = _strides(o) if o is not None else (max(Sq, 1) * H * D, H * D, D)
     p.scale = float(scale) if scale else 1.0 / math.sqrt(D)
     return p
 

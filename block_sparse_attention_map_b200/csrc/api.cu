@@ -7,6 +7,7 @@
 #include <atomic>
 #include <cmath>
 #include <cstring>
+#include <algorithm>
 #include <mutex>
 #include <vector>
 
@@ -23,6 +24,12 @@ int64_t cdiv64(int64_t a, int64_t b) { return (a + b - 1) / b; }
 }  // namespace
 
 void count_launch(int n) { g_launches.fetch_add(static_cast<uint64_t>(n)); }
+
+// No batch entries or no query rows: every check on the shape, mask and
+// options still applies, then the call does nothing.
+bool problem_is_empty(const bsa_problem *prob) {
+  return prob != nullptr && (prob->B == 0 || prob->Sq == 0);
+}
 
 WsLayout compute_layout(const bsa_problem &p) {
   WsLayout L{};
@@ -119,7 +126,7 @@ bsa_status normalise(const bsa_problem *in, bsa_problem *out) {
   if (in == nullptr) return BSA_ERR_INVALID_ARG;
   *out = *in;
   bsa_problem &p = *out;
-  if (p.B < 1 || p.H < 1 || p.Sq < 1 || p.Skv < 1) return BSA_ERR_INVALID_ARG;
+  if (p.B < 0 || p.H < 1 || p.Sq < 0 || p.Skv < 1) return BSA_ERR_INVALID_ARG;
   if (p.H_kv == 0) p.H_kv = p.H;
   if (p.H_kv < 1 || p.H % p.H_kv != 0) return BSA_ERR_INVALID_ARG;
   if (p.D != 64 && p.D != 128) return BSA_ERR_UNSUPPORTED;
@@ -129,7 +136,7 @@ bsa_status normalise(const bsa_problem *in, bsa_problem *out) {
   if (static_cast<int64_t>(p.B) * p.H * nM >= (int64_t{1} << 31)) return BSA_ERR_UNSUPPORTED;
   auto fix = [&](int64_t *s, int64_t S, int64_t heads) -> bsa_status {
     if (s[0] == 0 && s[1] == 0 && s[2] == 0) {
-      s[0] = S * heads * p.D;
+      s[0] = std::max<int64_t>(S, 1) * heads * p.D;
       s[1] = heads * p.D;
       s[2] = p.D;
     }
@@ -157,15 +164,18 @@ bsa_status check_mask(const bsa_problem &p, const bsa_mask_spec *m, bsa_mask_spe
                          BSA_MASK_CAUSAL_WINDOW | BSA_MASK_PREFIX_LM;
   if (m->flags & ~known) return BSA_ERR_INVALID_ARG;
   const bool win = (m->flags & BSA_MASK_CAUSAL_WINDOW) != 0;
-  if ((m->flags & BSA_MASK_PREFIX_LM) && (!win || m->prefix_len == nullptr))
+  // an empty problem's predicate arrays have no element, so may be null
+  const bool need = !problem_is_empty(&p);
+  if ((m->flags & BSA_MASK_PREFIX_LM) && (!win || (need && m->prefix_len == nullptr)))
     return BSA_ERR_INVALID_ARG;
   if (m->dilation < 0 || (m->dilation > 1 && !win)) return BSA_ERR_INVALID_ARG;
   out->dilation = m->dilation > 1 ? m->dilation : 1;
   out->reserved = 0;
   if (!(m->flags & BSA_MASK_PREFIX_LM)) out->prefix_len = nullptr;
-  if ((m->flags & BSA_MASK_SEGMENT_IDS) && (m->seg_q == nullptr || m->seg_kv == nullptr))
+  if ((m->flags & BSA_MASK_SEGMENT_IDS) && need && (m->seg_q == nullptr || m->seg_kv == nullptr))
     return BSA_ERR_INVALID_ARG;
-  if ((m->flags & BSA_MASK_KV_VALID_LEN) && m->kv_valid_len == nullptr) return BSA_ERR_INVALID_ARG;
+  if ((m->flags & BSA_MASK_KV_VALID_LEN) && need && m->kv_valid_len == nullptr)
+    return BSA_ERR_INVALID_ARG;
   if (m->flags & BSA_MASK_VARLEN) {
     if (m->flags & BSA_MASK_SEGMENT_IDS) return BSA_ERR_INVALID_ARG;
     if (m->cu_seqlens == nullptr || m->n_seqs < 1 || m->n_align_tail < 0 ||
@@ -254,6 +264,7 @@ struct Prepared {
   bsa_mask_spec m;
   bsa_options o;
   WsLayout L;
+  bool empty;  // nothing to compute: no workspace, pointer or device is touched
 };
 
 bsa_status prepare(const bsa_problem *prob, const bsa_mask_spec *mask, const bsa_options *opt,
@@ -265,6 +276,8 @@ bsa_status prepare(const bsa_problem *prob, const bsa_mask_spec *mask, const bsa
   if ((st = check_options(opt, out->L.nN, &out->o)) != BSA_OK) return st;
   if (out->o.bound_mode == BSA_BOUND_SMOOTHED && out->p.H_kv * out->p.D > kMaxSmoothedHD)
     return BSA_ERR_UNSUPPORTED;
+  out->empty = problem_is_empty(&out->p);
+  if (out->empty) return BSA_OK;
   if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return BSA_ERR_INVALID_ARG;
   // the O residual lives in the backward part of the workspace
   const bool full = backward || out->o.keep_o_residual != 0;
@@ -274,6 +287,25 @@ bsa_status prepare(const bsa_problem *prob, const bsa_mask_spec *mask, const bsa
 }
 
 bsa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? BSA_OK : BSA_ERR_CUDA; }
+
+// B >= 1 batches of keys but no query row: the gradient is dK = dV = 0, the
+// one result of an empty problem that has elements.
+bool keys_without_rows(const bsa_problem *prob) {
+  return prob != nullptr && prob->B > 0 && prob->Sq == 0;
+}
+
+bsa_status check_kv_grads(const void *dk, const void *dv) {
+  if (dk == nullptr || dv == nullptr) return BSA_ERR_INVALID_ARG;
+  if (!aligned16(dk) || !aligned16(dv)) return BSA_ERR_UNSUPPORTED;
+  return BSA_OK;
+}
+
+// The result of the backward calls for an empty problem (after `prepare`).
+bsa_status empty_backward(const bsa_problem &p, void *dk, void *dv, bsa_stream_t stream) {
+  if (!keys_without_rows(&p)) return BSA_OK;
+  if (!have_device()) return BSA_ERR_NO_DEVICE;
+  return cuda_status(launch_zero_kv_grads(p, dk, dv, reinterpret_cast<cudaStream_t>(stream)));
+}
 
 
 // ---------------------------------------------------------------- plan || bound
@@ -375,14 +407,16 @@ bsa_status attn_fwd_impl(const bsa_problem *prob, const bsa_mask_spec *mask,
                          const bsa_options *opt, const void *q, const void *k, const void *v,
                          void *out, float *lse, void *ws, size_t ws_bytes, bsa_stream_t stream,
                          bool side_stream_ok) {
-  if (q == nullptr || k == nullptr || v == nullptr || out == nullptr || lse == nullptr)
-    return BSA_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
-      (reinterpret_cast<uintptr_t>(lse) & 3u))
-    return BSA_ERR_UNSUPPORTED;
+  if (!problem_is_empty(prob)) {
+    if (q == nullptr || k == nullptr || v == nullptr || out == nullptr || lse == nullptr)
+      return BSA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
+        (reinterpret_cast<uintptr_t>(lse) & 3u))
+      return BSA_ERR_UNSUPPORTED;
+  }
   Prepared P;
   bsa_status st = prepare(prob, mask, opt, ws, ws_bytes, false, &P);
-  if (st != BSA_OK) return st;
+  if (st != BSA_OK || P.empty) return st;
   const bsa_problem &p = P.p;
   CUtensorMap tq, tk, tv;
   if (!make_map(&tq, q, p.B, p.Sq, p.H, p.D, p.q_stride) ||
@@ -419,7 +453,7 @@ bsa_status bsa_workspace_size(const bsa_problem *prob, const bsa_mask_spec *mask
   bsa_mask_spec m;
   if ((st = check_mask(p, mask, &m)) != BSA_OK) return st;
   const WsLayout L = compute_layout(p);
-  *bytes = with_backward ? L.total : L.fwd_end;
+  *bytes = problem_is_empty(&p) ? 0 : with_backward ? L.total : L.fwd_end;
   return BSA_OK;
 }
 
@@ -432,6 +466,12 @@ bsa_status bsa_workspace_layout(const bsa_problem *prob, const bsa_mask_spec *ma
   bsa_mask_spec m;
   if ((st = check_mask(p, mask, &m)) != BSA_OK) return st;
   const WsLayout L = compute_layout(p);
+  if (problem_is_empty(&p)) {
+    std::memset(view, 0, sizeof(*view));
+    view->nM = L.nM;
+    view->nN = L.nN;
+    return BSA_OK;
+  }
   view->total_bytes = L.total;
   view->fwd_bytes = L.fwd_end;
   view->off_status = L.status;
@@ -461,7 +501,7 @@ bsa_status bsa_plan_build(const bsa_problem *prob, const bsa_mask_spec *mask,
                           const bsa_options *opt, void *ws, size_t ws_bytes, bsa_stream_t stream) {
   Prepared P;
   bsa_status st = prepare(prob, mask, opt, ws, ws_bytes, false, &P);
-  if (st != BSA_OK) return st;
+  if (st != BSA_OK || P.empty) return st;
   return cuda_status(launch_plan(P.p, P.m, P.o, P.L, static_cast<uint8_t *>(ws),
                                  reinterpret_cast<cudaStream_t>(stream)));
 }
@@ -476,15 +516,21 @@ bsa_status bsa_attn_bwd(const bsa_problem *prob, const bsa_mask_spec *mask,
                         const bsa_options *opt, const void *q, const void *k, const void *v,
                         const void *out, const void *dout, const float *lse, void *dq, void *dk,
                         void *dv, void *ws, size_t ws_bytes, bsa_stream_t stream) {
-  if (q == nullptr || k == nullptr || v == nullptr || out == nullptr || dout == nullptr ||
-      lse == nullptr || dq == nullptr || dk == nullptr || dv == nullptr)
-    return BSA_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(dout) ||
-      !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || (reinterpret_cast<uintptr_t>(lse) & 3u))
-    return BSA_ERR_UNSUPPORTED;
+  bsa_status st;
+  if (keys_without_rows(prob)) {
+    if ((st = check_kv_grads(dk, dv)) != BSA_OK) return st;
+  } else if (!problem_is_empty(prob)) {
+    if (q == nullptr || k == nullptr || v == nullptr || out == nullptr || dout == nullptr ||
+        lse == nullptr || dq == nullptr || dk == nullptr || dv == nullptr)
+      return BSA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(dout) ||
+        !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
+        (reinterpret_cast<uintptr_t>(lse) & 3u))
+      return BSA_ERR_UNSUPPORTED;
+  }
   Prepared P;
-  bsa_status st = prepare(prob, mask, opt, ws, ws_bytes, true, &P);
-  if (st != BSA_OK) return st;
+  if ((st = prepare(prob, mask, opt, ws, ws_bytes, true, &P)) != BSA_OK) return st;
+  if (P.empty) return empty_backward(P.p, dk, dv, stream);
   const bsa_problem &p = P.p;
   CUtensorMap tq, tk, tv, tdo;
   if (!make_map(&tq, q, p.B, p.Sq, p.H, p.D, p.q_stride) ||
@@ -505,11 +551,13 @@ bsa_status bsa_attn_bwd(const bsa_problem *prob, const bsa_mask_spec *mask,
 bsa_status bsa_fixed_m_bound(const bsa_problem *prob, const bsa_mask_spec *mask,
                              const bsa_options *opt, const void *q, const void *k, void *ws,
                              size_t ws_bytes, bsa_stream_t stream) {
-  if (q == nullptr || k == nullptr) return BSA_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k)) return BSA_ERR_UNSUPPORTED;
+  if (!problem_is_empty(prob)) {
+    if (q == nullptr || k == nullptr) return BSA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k)) return BSA_ERR_UNSUPPORTED;
+  }
   Prepared P;
   bsa_status st = prepare(prob, mask, opt, ws, ws_bytes, false, &P);
-  if (st != BSA_OK) return st;
+  if (st != BSA_OK || P.empty) return st;
   uint8_t *w = static_cast<uint8_t *>(ws);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (!P.o.plan_ready) {
@@ -523,11 +571,13 @@ bsa_status bsa_fixed_m_bound(const bsa_problem *prob, const bsa_mask_spec *mask,
 bsa_status bsa_plan_and_bound(const bsa_problem *prob, const bsa_mask_spec *mask,
                               const bsa_options *opt, const void *q, const void *k, void *ws,
                               size_t ws_bytes, bsa_stream_t stream) {
-  if (q == nullptr || k == nullptr) return BSA_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k)) return BSA_ERR_UNSUPPORTED;
+  if (!problem_is_empty(prob)) {
+    if (q == nullptr || k == nullptr) return BSA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k)) return BSA_ERR_UNSUPPORTED;
+  }
   Prepared P;
   bsa_status st = prepare(prob, mask, opt, ws, ws_bytes, false, &P);
-  if (st != BSA_OK) return st;
+  if (st != BSA_OK || P.empty) return st;
   return cuda_status(plan_and_bound(P.p, P.m, P.o, q, k, P.L, static_cast<uint8_t *>(ws),
                                     reinterpret_cast<cudaStream_t>(stream)));
 }
@@ -535,11 +585,13 @@ bsa_status bsa_plan_and_bound(const bsa_problem *prob, const bsa_mask_spec *mask
 bsa_status bsa_bwd_preprocess(const bsa_problem *prob, const bsa_mask_spec *mask,
                               const bsa_options *opt, const void *out, const void *dout, void *ws,
                               size_t ws_bytes, bsa_stream_t stream) {
-  if (out == nullptr || dout == nullptr) return BSA_ERR_INVALID_ARG;
-  if (!aligned16(out) || !aligned16(dout)) return BSA_ERR_UNSUPPORTED;
+  if (!problem_is_empty(prob)) {
+    if (out == nullptr || dout == nullptr) return BSA_ERR_INVALID_ARG;
+    if (!aligned16(out) || !aligned16(dout)) return BSA_ERR_UNSUPPORTED;
+  }
   Prepared P;
   bsa_status st = prepare(prob, mask, opt, ws, ws_bytes, true, &P);
-  if (st != BSA_OK) return st;
+  if (st != BSA_OK || P.empty) return st;
   return cuda_status(launch_bwd_preprocess(P.p, P.o, out, dout, P.L, static_cast<uint8_t *>(ws),
                                            reinterpret_cast<cudaStream_t>(stream)));
 }
@@ -548,15 +600,20 @@ bsa_status bsa_bwd_main(const bsa_problem *prob, const bsa_mask_spec *mask,
                         const bsa_options *opt, const void *q, const void *k, const void *v,
                         const void *dout, const float *lse, void *dk, void *dv, void *ws,
                         size_t ws_bytes, bsa_stream_t stream) {
-  if (q == nullptr || k == nullptr || v == nullptr || dout == nullptr || lse == nullptr ||
-      dk == nullptr || dv == nullptr)
-    return BSA_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) || !aligned16(dk) ||
-      !aligned16(dv) || (reinterpret_cast<uintptr_t>(lse) & 3u))
-    return BSA_ERR_UNSUPPORTED;
+  bsa_status st;
+  if (keys_without_rows(prob)) {
+    if ((st = check_kv_grads(dk, dv)) != BSA_OK) return st;
+  } else if (!problem_is_empty(prob)) {
+    if (q == nullptr || k == nullptr || v == nullptr || dout == nullptr || lse == nullptr ||
+        dk == nullptr || dv == nullptr)
+      return BSA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) || !aligned16(dk) ||
+        !aligned16(dv) || (reinterpret_cast<uintptr_t>(lse) & 3u))
+      return BSA_ERR_UNSUPPORTED;
+  }
   Prepared P;
-  bsa_status st = prepare(prob, mask, opt, ws, ws_bytes, true, &P);
-  if (st != BSA_OK) return st;
+  if ((st = prepare(prob, mask, opt, ws, ws_bytes, true, &P)) != BSA_OK) return st;
+  if (P.empty) return empty_backward(P.p, dk, dv, stream);
   const bsa_problem &p = P.p;
   CUtensorMap tq, tk, tv, tdo;
   if (!make_map(&tq, q, p.B, p.Sq, p.H, p.D, p.q_stride) ||
@@ -576,11 +633,13 @@ bsa_status bsa_bwd_main(const bsa_problem *prob, const bsa_mask_spec *mask,
 
 bsa_status bsa_bwd_convert(const bsa_problem *prob, const bsa_mask_spec *mask, void *dq, void *ws,
                            size_t ws_bytes, bsa_stream_t stream) {
-  if (dq == nullptr) return BSA_ERR_INVALID_ARG;
-  if (!aligned16(dq)) return BSA_ERR_UNSUPPORTED;
+  if (!problem_is_empty(prob)) {
+    if (dq == nullptr) return BSA_ERR_INVALID_ARG;
+    if (!aligned16(dq)) return BSA_ERR_UNSUPPORTED;
+  }
   Prepared P;
   bsa_status st = prepare(prob, mask, nullptr, ws, ws_bytes, true, &P);
-  if (st != BSA_OK) return st;
+  if (st != BSA_OK || P.empty) return st;
   return cuda_status(launch_bwd_convert(P.p, dq, P.L, static_cast<uint8_t *>(ws),
                                         reinterpret_cast<cudaStream_t>(stream)));
 }

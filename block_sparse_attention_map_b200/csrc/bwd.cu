@@ -886,6 +886,29 @@ __global__ void __launch_bounds__(256) k_dq_convert(const float *__restrict__ ac
   }
 }
 
+// dK = dV = 0, the whole gradient of a problem with keys but no query row:
+// the 16-byte pieces of both strided [B, Skv, H_kv, D] tensors, grid-stride.
+__global__ void __launch_bounds__(256) k_zero_kv_grads(__nv_bfloat16 *__restrict__ dk,
+                                                       __nv_bfloat16 *__restrict__ dv, int Skv,
+                                                       int Hkv, int D, int64_t pieces, int64_t ksb,
+                                                       int64_t kss, int64_t ksh, int64_t vsb,
+                                                       int64_t vss, int64_t vsh) {
+  const int cpr = D / 8;
+  const int64_t step = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < 2 * pieces;
+       idx += step) {
+    const bool is_v = idx >= pieces;
+    int64_t r = is_v ? idx - pieces : idx;
+    const int c = static_cast<int>(r % cpr);
+    r /= cpr;
+    const int h = static_cast<int>(r % Hkv);
+    r /= Hkv;
+    const int64_t j = r % Skv, b = r / Skv;
+    __nv_bfloat16 *row = is_v ? dv + b * vsb + j * vss + h * vsh : dk + b * ksb + j * kss + h * ksh;
+    *reinterpret_cast<int4 *>(row + 8 * c) = make_int4(0, 0, 0, 0);
+  }
+}
+
 int sm_count_bwd() {
   static int n = 0;
   if (n == 0) {
@@ -1012,6 +1035,18 @@ cudaError_t launch_bwd_convert(const bsa_problem &p, void *dq, const WsLayout &L
                                    s, acc, p.B, p.H, p.Sq, L.nM, row_ptr, out, p.q_stride[0], p.q_stride[1],
                                    p.q_stride[2]);
   if (e != cudaSuccess) return e;
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_zero_kv_grads(const bsa_problem &p, void *dk, void *dv, cudaStream_t s) {
+  const int64_t pieces = static_cast<int64_t>(p.B) * p.Skv * p.H_kv * (p.D / 8);
+  const int64_t want = (2 * pieces + 255) / 256;
+  const unsigned blocks = static_cast<unsigned>(std::min<int64_t>(want, 8 * sm_count_bwd()));
+  k_zero_kv_grads<<<blocks, 256, 0, s>>>(static_cast<__nv_bfloat16 *>(dk),
+                                         static_cast<__nv_bfloat16 *>(dv), p.Skv, p.H_kv, p.D,
+                                         pieces, p.k_stride[0], p.k_stride[1], p.k_stride[2],
+                                         p.v_stride[0], p.v_stride[1], p.v_stride[2]);
   count_launch();
   return cudaGetLastError();
 }

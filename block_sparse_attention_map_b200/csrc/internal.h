@@ -119,6 +119,9 @@ cudaError_t launch_bwd_main(const bsa_problem &p, const MaskParams &mp, const bs
 cudaError_t launch_bwd_convert(const bsa_problem &p, void *dq, const WsLayout &L, uint8_t *ws,
                                cudaStream_t s);
 
+// dK = dV = 0 (a problem with B >= 1 key rows but Sq == 0): one kernel.
+cudaError_t launch_zero_kv_grads(const bsa_problem &p, void *dk, void *dv, cudaStream_t s);
+
 void count_launch(int n = 1);
 
 // Launch with programmatic stream serialization: the kernel may start while
@@ -139,6 +142,9 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
+
+// B == 0 or Sq == 0: the call checks its arguments and then does nothing.
+bool problem_is_empty(const bsa_problem *prob);
 
 // bsa_attn_fwd; side_stream_ok = false never forks work onto the library's side
 // stream (no stream or event is created).

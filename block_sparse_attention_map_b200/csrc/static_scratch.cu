@@ -52,11 +52,14 @@ extern "C" bsa_status bsa_attn_fwd_static_scratch(const bsa_problem *prob,
                                                   const bsa_options *opt, const void *q,
                                                   const void *k, const void *v, void *out,
                                                   float *lse, bsa_stream_t stream) {
-  if (q == nullptr || k == nullptr || v == nullptr || out == nullptr || lse == nullptr)
+  const bool empty = bsa::problem_is_empty(prob);
+  if (!empty && (q == nullptr || k == nullptr || v == nullptr || out == nullptr || lse == nullptr))
     return BSA_ERR_INVALID_ARG;
   size_t need = 0;
   bsa_status st = bsa_workspace_size(prob, mask, 0, &need);
   if (st != BSA_OK) return st;
+  // an empty problem still has its options checked, then does nothing
+  if (empty) return bsa::attn_fwd_impl(prob, mask, opt, q, k, v, out, lse, nullptr, 0, stream, false);
   if (need > kStaticScratchBytes) return BSA_ERR_WORKSPACE_TOO_SMALL;
   void *ws = nullptr;
   if ((st = scratch_for_current_device(&ws)) != BSA_OK) return st;

@@ -127,10 +127,10 @@ typedef enum bsa_status {
 #define BSA_ORDER_GREEDY 4
 
 typedef struct bsa_problem {
-  int32_t B;       /* batch; 1 for varlen                                        */
-  int32_t H;       /* query heads (Q, O, LSE, dQ, dO)                            */
-  int32_t Sq;      /* query rows per batch (varlen: total tokens T); <= 2^21      */
-  int32_t Skv;     /* keys per batch (varlen: T); <= 2^21                         */
+  int32_t B;       /* batch, >= 0; 1 for varlen                                   */
+  int32_t H;       /* query heads (Q, O, LSE, dQ, dO), >= 1                       */
+  int32_t Sq;      /* query rows per batch (varlen: total tokens T); 0 .. 2^21    */
+  int32_t Skv;     /* keys per batch (varlen: T); 1 .. 2^21                       */
   int32_t D;       /* head dim, 64 or 128                                         */
   int32_t H_kv;    /* key/value heads (K, V, dK, dV); 0 = H.  H must be a multiple:
                       query head h reads kv head h / (H / H_kv) (grouped-query
@@ -146,6 +146,17 @@ typedef struct bsa_problem {
   float scale;     /* <= 0: 1/sqrt(D)                                             */
   int32_t reserved1;
 } bsa_problem;
+/* An EMPTY problem (B == 0 or Sq == 0: no output row) is valid.  Every call
+ * checks its shape, mask and options as usual, then returns BSA_OK without
+ * touching a tensor or mask-array pointer (null allowed), the workspace
+ * (0 bytes, null allowed), the stream or the device, and launches nothing.
+ * Its workspace size is 0 and its bsa_workspace_view is all zero except nM
+ * and nN.  The one exception: with B >= 1 and Sq == 0, dK and dV have
+ * elements and their gradient is zero, so bsa_attn_bwd and bsa_bwd_main need
+ * valid 16-byte aligned dk and dv (else INVALID_ARG / UNSUPPORTED) and a
+ * device, and zero both with one kernel on `stream`.  Skv == 0 is an argument
+ * error: a row with no allowed key is expressed by the mask (its output is 0
+ * and its LSE -inf). */
 
 typedef struct bsa_mask_spec {
   uint32_t flags;              /* OR of BSA_MASK_*                                  */

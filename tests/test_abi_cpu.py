@@ -110,7 +110,11 @@ def test_workspace_size_and_validation(L):
     # the backward adds Delta, the fp32 dQ accumulator [B,H,nM*128,D] and semaphores
     assert rc == 0 and tot >= fwd + 4 * 2 * 256 * 64 + 4 * 2 * 256
     assert _size(L, _prob(D=96))[0] == 2          # unsupported head dim
-    assert _size(L, _prob(B=0))[0] == 1           # invalid
+    assert _size(L, _prob(H=0))[0] == 1           # invalid
+    assert _size(L, _prob(Skv=0))[0] == 1         # no key at all: invalid
+    assert _size(L, _prob(Sq=1 << 21, Skv=1 << 21))[0] == 0  # the longest sequence accepted
+    assert _size(L, _prob(Sq=(1 << 21) + 1))[0] == 2
+    assert _size(L, _prob(Skv=(1 << 21) + 1))[0] == 2
     p = _prob()
     p.q_stride[:] = (256 * 2 * 64, 2 * 64 + 4, 64)  # row stride not a multiple of 16 bytes
     assert _size(L, p)[0] == 2
@@ -186,6 +190,60 @@ def test_calls_reject_bad_arguments_before_cuda(L):
     assert L.bsa_plan_build(ctypes.byref(p), None, ctypes.byref(o), 4096, 16, None) == 3
     assert L.bsa_status_string(0).decode() == "ok"
     assert L.bsa_status_string(5).decode().startswith("a bounded device wait")
+
+
+def test_empty_problem_is_a_checked_no_op(L):
+    """B == 0 or Sq == 0: arguments are still checked, then every call returns
+    ok with null tensors and workspace, no device and no launch; the one
+    exception is the backward with key rows but no query row, which zeroes dK
+    and dV."""
+    for p in (_prob(B=0), _prob(Sq=0), _prob(B=0, Sq=0, D=128)):
+        assert _size(L, p, bwd=0) == (0, 0) and _size(L, p, bwd=1) == (0, 0)
+        v = bd.WorkspaceView()
+        assert L.bsa_workspace_layout(ctypes.byref(p), None, ctypes.byref(v)) == 0
+        assert v.total_bytes == v.fwd_bytes == v.off_delta == v.off_sem == 0
+        assert (v.nM, v.nN) == ((p.Sq + 127) // 128, 2)
+    for bad in (_prob(B=-1), _prob(Sq=-1), _prob(B=0, Skv=0), _prob(Sq=0, H=0)):
+        assert _size(L, bad)[0] == 1
+    assert _size(L, _prob(B=0, D=96))[0] == 2       # still an unsupported head dim
+    seg = bd.MaskSpec()
+    seg.flags = bd.MASK_SEGMENT_IDS                 # arrays of no element may be null
+    assert _size(L, _prob(B=0), seg) == (0, 0)
+    assert _size(L, _prob(), seg)[0] == 1
+    before = L.bsa_launch_count()
+    for p in (_prob(B=0), _prob(Sq=0)):
+        P, o = ctypes.byref(p), ctypes.byref(bd.Options())
+        n = None
+        assert L.bsa_workspace_size(P, ctypes.byref(seg), 1, ctypes.byref(ctypes.c_size_t())) == 0
+        assert L.bsa_plan_build(P, None, o, n, 0, n) == 0
+        assert L.bsa_attn_fwd(P, None, o, n, n, n, n, n, n, 0, n) == 0
+        assert L.bsa_attn_fwd(P, ctypes.byref(seg), o, n, n, n, n, n, n, 0, n) == 0
+        if p.B == 0:
+            assert L.bsa_attn_bwd(P, None, o, n, n, n, n, n, n, n, n, n, n, 0, n) == 0
+            assert L.bsa_bwd_main(P, None, o, n, n, n, n, n, n, n, n, 0, n) == 0
+        else:
+            # keys but no query row: dK = dV = 0 must be written, so dk and dv
+            # are checked and a device is needed (none here)
+            assert L.bsa_attn_bwd(P, None, o, n, n, n, n, n, n, n, n, n, n, 0, n) == 1
+            assert L.bsa_attn_bwd(P, None, o, n, n, n, n, n, n, n, 8, 4096, n, 0, n) == 2
+            assert L.bsa_attn_bwd(P, None, o, n, n, n, n, n, n, n, 4096, 8192, n, 0, n) == 9
+            assert L.bsa_bwd_main(P, None, o, n, n, n, n, n, n, 4096, n, 0, n) == 1
+            assert L.bsa_bwd_main(P, None, o, n, n, n, n, n, 4096, 8192, n, 0, n) == 9
+        assert L.bsa_fixed_m_bound(P, None, o, n, n, n, 0, n) == 0
+        assert L.bsa_plan_and_bound(P, None, o, n, n, n, 0, n) == 0
+        assert L.bsa_bwd_preprocess(P, None, o, n, n, n, 0, n) == 0
+        assert L.bsa_bwd_convert(P, None, n, n, 0, n) == 0
+        f = L.bsa_attn_fwd_static_scratch
+        f.restype = ctypes.c_int32
+        f.argtypes = [ctypes.POINTER(bd.Problem), ctypes.POINTER(bd.MaskSpec), ctypes.POINTER(bd.Options)] + \
+            [ctypes.c_void_p] * 6
+        assert f(P, None, o, n, n, n, n, n, n) == 0
+        # the options are still checked
+        bad = bd.Options()
+        bad.softmax_mode = 7
+        assert L.bsa_attn_fwd(P, None, ctypes.byref(bad), n, n, n, n, n, n, 0, n) == 1
+        assert f(P, None, ctypes.byref(bad), n, n, n, n, n, n) == 1
+    assert L.bsa_launch_count() == before
 
 
 def test_layout_offsets_are_aligned(L):
