@@ -797,17 +797,22 @@ __global__ void __launch_bounds__(256) k_bwd_delta(const __nv_bfloat16 *__restri
        z += static_cast<int64_t>(gridDim.x) * blockDim.x)
     sem[z] = 0u;
   const int t = threadIdx.x % TPV;
-  const int64_t total = static_cast<int64_t>(B) * H * rows_pad;
+  // the block's rows all belong to one (b, h): its index and first row come
+  // from one division per block, not per row
+  constexpr int kRowsPerBlock = kDeltaRuns * VPB;
+  const int blocks_per_bh = rows_pad / kRowsPerBlock;
+  const int bh = static_cast<int>(blockIdx.x) / blocks_per_bh;
+  const int i0 = (static_cast<int>(blockIdx.x) - bh * blocks_per_bh) * kRowsPerBlock + threadIdx.x / TPV;
+  const int b = bh / H, h = bh % H;
+  const bool in_bh = bh < B * H;  // uniform per block; no early return before the shuffles
   int64_t g[kDeltaRuns];
   bool in[kDeltaRuns];
   int4 av[kDeltaRuns], cv[kDeltaRuns], rv[kDeltaRuns];
 #pragma unroll
   for (int j = 0; j < kDeltaRuns; ++j) {
-    g[j] = (static_cast<int64_t>(blockIdx.x) * kDeltaRuns + j) * VPB + threadIdx.x / TPV;
-    in[j] = g[j] < total;  // no early return: the shuffles below need every lane
-    const int i = static_cast<int>(g[j] % rows_pad);
-    const int bh = static_cast<int>(g[j] / rows_pad);
-    const int b = bh / H, h = bh % H;
+    const int i = i0 + j * VPB;
+    g[j] = static_cast<int64_t>(bh) * rows_pad + i;
+    in[j] = in_bh;
     av[j] = cv[j] = rv[j] = make_int4(0, 0, 0, 0);
     if (in[j] && i < Sq) {
       const int64_t off = b * sb + static_cast<int64_t>(i) * ss + h * sh + t * 8;

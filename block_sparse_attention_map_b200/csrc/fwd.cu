@@ -704,31 +704,50 @@ __global__ void __launch_bounds__(256) k_row_norms(const NormArgs a) {
   for (int h = threadIdx.x; h < H; h += blockDim.x) smax[h] = 0u;
   __syncthreads();
   // Grid-stride over the batch row's (row, head) vectors, consecutive vectors
-  // on consecutive heads of a row (the tensor's memory order).  Two vectors
-  // per thread and pass keep eight 16-byte loads in flight; the per-head
+  // on consecutive heads of a row (the tensor's memory order).  kPass vectors
+  // per thread and pass keep 4 * kPass 16-byte loads in flight; the per-head
   // maxima gather in shared memory over the block's whole range, so the
   // global atomics and the fence below happen once per block.
+  constexpr int kPass = 2;  // vectors per thread and pass, all loads in flight
   const int64_t nvec = static_cast<int64_t>(S) * Hx;
   const int64_t stride = static_cast<int64_t>(bpb) * kVPB;
   const int t = threadIdx.x % kT;
-  for (int64_t base = static_cast<int64_t>(blk) * kVPB; base < nvec; base += 2 * stride) {
-    int64_t vv[2];
-    bool in[2];
-    int4 w[2][4];
+  // The thread's vectors v0 + k * stride as (row, head) pairs, stepped by a
+  // carry instead of a division per vector (vector = row * Hx + head).
+  const int64_t v0 = static_cast<int64_t>(blk) * kVPB + threadIdx.x / kT;
+  const int d_row = static_cast<int>(stride / Hx), d_hh = static_cast<int>(stride % Hx);
+  int row_k = static_cast<int>(v0 / Hx), hh_k = static_cast<int>(v0 % Hx);
+  auto step = [&](int &rw, int &hd) {
+    hd += d_hh;
+    rw += d_row;
+    if (hd >= Hx) {
+      hd -= Hx;
+      ++rw;
+    }
+  };
+  for (int64_t base = static_cast<int64_t>(blk) * kVPB; base < nvec; base += kPass * stride) {
+    int rws[kPass], hds[kPass];
 #pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      vv[j] = base + j * stride + threadIdx.x / kT;
-      in[j] = vv[j] < nvec;  // no early exit: the shuffles below need every lane
+    for (int j = 0; j < kPass; ++j) {
+      rws[j] = row_k;
+      hds[j] = hh_k;
+      step(row_k, hh_k);
+    }
+    bool in[kPass];
+    int4 w[kPass][4];
+#pragma unroll
+    for (int j = 0; j < kPass; ++j) {
+      in[j] = rws[j] < S;  // the vector is below nvec; no early exit: the shuffles need every lane
       if (in[j]) {
-        const int row = static_cast<int>(vv[j] / Hx), hh = static_cast<int>(vv[j] % Hx);
-        const int4 *src = reinterpret_cast<const int4 *>(x + b * sb + static_cast<int64_t>(row) * ss + hh * sh) + 4 * t;
+        const int4 *src =
+            reinterpret_cast<const int4 *>(x + b * sb + static_cast<int64_t>(rws[j]) * ss + hds[j] * sh) + 4 * t;
 #pragma unroll
         for (int u = 0; u < 4; ++u) w[j][u] = __ldg(src + u);
       }
     }
 #pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      const int row = in[j] ? static_cast<int>(vv[j] / Hx) : 0, hh = in[j] ? static_cast<int>(vv[j] % Hx) : 0;
+    for (int j = 0; j < kPass; ++j) {
+      const int row = rws[j], hh = hds[j];
       float acc = 0.f, dot = 0.f;
       if (in[j]) {
         const float *c = CENTER ? a.kbar + (static_cast<int64_t>(b) * a.Hk + (is_key ? hh : hh / grp)) * D + 32 * t
