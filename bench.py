@@ -170,37 +170,50 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def dist_setup(args):
+def dist_setup(args, backend: str = "nccl"):
+    """(world, rank, local rank) from the torchrun environment; with more than
+    one rank, joins the process group (NCCL on the GPUs; the CPU tests pass
+    gloo) with a short timeout, so that a rank that never arrives ends the
+    others' next collective with an error."""
     import torch
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if torch.cuda.is_available():
+        torch.cuda.set_device(local)
     if world > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    elif torch.cuda.is_available():
-        torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
     return world, rank, local
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """The maximum of x over all ranks (every rank takes part and gets it)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
 
 def barrier(world: int):
+    """All ranks meet, and this rank's device work has finished."""
     import torch
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
-    torch.cuda.synchronize()
+    if torch.cuda.is_available():
+        torch.cuda.synchronize()
+
+
+def whole_job_tflops(world: int, steps: int, flops_per_step: float, max_total_ms: float) -> float:
+    """value: the work of all ranks (each runs `steps` steps of the same
+    workload) over the slowest rank's time for them."""
+    return world * steps * flops_per_step / (max_total_ms * 1e-3) / 1e12
 
 
 def tiles_of(ws):
@@ -396,7 +409,7 @@ def run_ours(args, world, rank, local):
         launches = bsa.launch_count() - l0
     total_ms = max_over_ranks(sum(step_ms), world)
     ms_step = total_ms / args.steps
-    value = world * args.steps * (f_fwd + f_bwd) / (total_ms * 1e-3) / 1e12
+    value = whole_job_tflops(world, args.steps, f_fwd + f_bwd, total_ms)
 
     peaks = load_peaks()
     peak = peaks["bf16_tflops"]
@@ -524,7 +537,7 @@ def e2e_leg(args, wl, dev, flops, world):
     ms = max_over_ranks(e0.elapsed_time(e1), world)
     h2d = sum(t.numel() * t.element_size() for t in host.values())
     d2h = sum(t.numel() * t.element_size() for t in slots[0]["out_h"].values())
-    return {"value": world * args.steps * flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+    return {"value": whole_job_tflops(world, args.steps, flops, ms), "unit": "TFLOP/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "ms_per_step": ms / args.steps,
             "pipeline": "two buffer sets; uploads, compute and downloads on three streams"}
