@@ -220,3 +220,31 @@ def test_plan_mismatch_is_reported():
     o, lse, _ = bsa.attn_fwd(wl.q, wl.k, wl.v, wl.mask, workspace=ws, plan_ready=True)
     torch.cuda.synchronize()
     assert ws.status(clear=True) == 6  # BSA_ERR_PLAN_MISMATCH
+
+
+@pytest.mark.parametrize("deterministic", [True, False])
+def test_stage_calls_equal_the_composite_calls(deterministic):
+    """The per-stage C-ABI calls (plan, bound, forward, Delta, backward main,
+    dQ convert) give the composite calls' results: bit for bit with the
+    deterministic backward, and within the bar of the oracle with the atomic
+    one, whose dQ comes out of the convert stage."""
+    wl = make_workload("window", device="cuda", small=True)
+    st = bsa.Stages(wl.q, wl.k, wl.v, wl.mask, softmax_mode="fixed_m", order="desc",
+                    deterministic=deterministic)
+    st.plan()
+    st.bound()
+    st.forward()
+    st.preprocess(wl.dO)
+    st.backward_main(wl.dO)
+    st.convert()
+    o, lse, _ = bsa.attn_fwd(wl.q, wl.k, wl.v, wl.mask, softmax_mode="fixed_m", order="desc")
+    dq, dk, dv, ws = bsa.attn_bwd(wl.q, wl.k, wl.v, o, wl.dO, lse, wl.mask, order="desc",
+                                  deterministic=deterministic)
+    torch.cuda.synchronize()
+    assert st.ws.status() == 0 and ws.status() == 0
+    assert torch.equal(st.out, o) and torch.equal(st.lse, lse)
+    if deterministic:
+        assert torch.equal(st.dq, dq) and torch.equal(st.dk, dk) and torch.equal(st.dv, dv)
+    else:
+        gq, gk, gv = _oracle_grads(wl)
+        assert max(_err(st.dq, gq), _err(st.dk, gk), _err(st.dv, gv)) <= O_TOL
