@@ -210,6 +210,21 @@ def barrier(world: int):
         torch.cuda.synchronize()
 
 
+def window_pairs(wl):
+    """Allowed (query, key) pairs of a plain causal-window mask (no other
+    predicate), summed over batches and query heads, in closed form: row i sees
+    keys (i + o - W, i + o] within [0, Skv) with o = Skv - Sq (all keys up to
+    i + o when W = 0).  None for any other mask."""
+    import numpy as np
+    if set(wl.mask) != {"window"}:
+        return None
+    W, o = int(wl.mask["window"]), wl.Skv - wl.Sq
+    i = np.arange(wl.Sq, dtype=np.int64)
+    hi = np.minimum(i + o, wl.Skv - 1)
+    lo = np.maximum(i + o - W + 1, 0) if W > 0 else np.zeros_like(i)
+    return int(np.maximum(hi - lo + 1, 0).sum()) * wl.B * wl.H
+
+
 def whole_job_tflops(world: int, steps: int, flops_per_step: float, max_total_ms: float) -> float:
     """value: the work of all ranks (each runs `steps` steps of the same
     workload) over the slowest rank's time for them."""
@@ -410,6 +425,11 @@ def run_ours(args, world, rank, local):
     total_ms = max_over_ranks(sum(step_ms), world)
     ms_step = total_ms / args.steps
     value = whole_job_tflops(world, args.steps, f_fwd + f_bwd, total_ms)
+    # the same time over the flops of the allowed entries alone (4 D per pair
+    # forward, 2.5x that backward), where the mask has a closed form
+    pairs = window_pairs(wl)
+    exact_value = (whole_job_tflops(world, args.steps, 3.5 * 4.0 * wl.D * pairs, total_ms)
+                   if pairs is not None else None)
 
     peaks = load_peaks()
     peak = peaks["bf16_tflops"]
@@ -430,6 +450,8 @@ def run_ours(args, world, rank, local):
                    "l2": "flushed (256 MiB write) before every step, outside the timed events",
                    "parallelism": f"replicas x{world}"},
         "pct_of_bf16_peak": 100.0 * value / peak,
+        "exact_mask_tflops": exact_value,
+        "exact_mask_pairs": pairs,
         "stages_ms": avg,
         "timing": ("CUDA-graph replay of the whole step (captured once after warm-up)" if graph is not None
                    else (graph_note or "eager library calls (--no-graph)")),

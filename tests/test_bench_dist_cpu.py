@@ -1,8 +1,9 @@
-"""bench.py's multi-rank plumbing on CPU (gloo, world size 2), the path that
+"""bench.py's host logic on CPU.  Its multi-rank plumbing (gloo, world size 2), the path that
 `bench.py --gpus N` takes under torch.distributed.run: every rank joins the
 group, the timing is the maximum over ranks, the ranks meet at the barrier,
 and the whole-job value counts every rank's work over the slowest rank's time.
-The reference arm, launched the same way, prints one line from rank 0 only."""
+The reference arm, launched the same way, prints one line from rank 0 only.
+And the closed-form pair count behind the exact-mask figure."""
 
 import json
 import os
@@ -72,3 +73,20 @@ def test_reference_arm_under_torchrun_prints_from_rank_zero_only():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_exact_mask_pair_count_matches_the_oracle_predicate():
+    """bench.window_pairs (the closed form behind exact_mask_tflops) against a
+    count of the oracle's allowed(i, j) on small windows, square and
+    bottom-right rectangular, including the plain causal W = 0."""
+    import types
+
+    import numpy as np
+
+    import bench
+    import oracle
+    for Sq, Skv, W in [(300, 300, 64), (200, 500, 128), (500, 200, 64), (257, 257, 0), (64, 640, 700)]:
+        wl = types.SimpleNamespace(mask={"window": W}, Sq=Sq, Skv=Skv, B=2, H=3)
+        allowed = oracle.allowed_rows(oracle.MaskDesc(window=W), 0, np.arange(Sq), Sq, Skv)
+        assert bench.window_pairs(wl) == int(allowed.sum()) * 2 * 3, (Sq, Skv, W)
+    assert bench.window_pairs(types.SimpleNamespace(mask={"window": 8, "dilation": 2})) is None

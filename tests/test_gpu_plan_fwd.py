@@ -331,3 +331,43 @@ def test_plan_beside_bound_equals_plan_then_bound(name):
     f = lambda t: t.float().cpu().numpy().astype(np.float64)
     O_ref, L_ref = oracle.attention_forward(f(wl.q), f(wl.k), f(wl.v), mask_desc(wl), wl.scale, rows=rows)
     assert compare_out(outs[1][0], O_ref, rows) <= O_TOL
+
+
+def _gate_edge_inputs():
+    """Every query along one direction u and every key along -u: s_ij =
+    -scale a_i c_j, so the pinned m_i = scale a_i kmax sits scale a_i (kmax +
+    c_j) above each score.  With query norms up to 16 and key norms in
+    [15, 15.8] at D = 64, 2 B_h = 63.2, just under the gate limit 64, and the
+    worst row's reference is 61.6 nats above its true maximum."""
+    B, H, S, D, W = 1, 2, 1000, 64, 256
+    rng = np.random.default_rng(31)
+    u = rng.standard_normal(D)
+    u /= np.linalg.norm(u)
+    a = rng.uniform(2.0, 16.0, size=(B, S, H))
+    a[0, 700] = 16.0
+    c = rng.uniform(15.0, 15.8, size=(B, S, H))
+    q = torch.from_numpy(a[..., None] * u).to(torch.bfloat16).cuda()
+    k = torch.from_numpy(-c[..., None] * u).to(torch.bfloat16).cuda()
+    v = torch.from_numpy(rng.standard_normal((B, S, H, D))).to(torch.bfloat16).cuda()
+    return q, k, v, {"window": W}, D ** -0.5
+
+
+def test_fixed_m_at_the_gate_edge_stays_exact():
+    """A head whose pinned reference sits as far above the true row maximum as
+    the gate allows still passes the gate, runs fixed-m without a gate warning,
+    and matches the oracle and the online forward."""
+    q, k, v, mask, scale = _gate_edge_inputs()
+    md = oracle.MaskDesc(window=mask["window"])
+    _, _, bound, gate = oracle.fixed_m_bound(np64(q), np64(k), md, scale)
+    assert gate.all() and (2 * bound > 63.0).all()
+    o, lse, ws = bsa.attn_fwd(q, k, v, mask, softmax_mode="fixed_m")
+    o_on, lse_on, _ = bsa.attn_fwd(q, k, v, mask)
+    torch.cuda.synchronize()
+    assert ws.status() == 0  # no row summed below 2^-100
+    assert ws.gate().cpu().numpy().all()
+    O_ref, L_ref = oracle.attention_forward(np64(q), np64(k), np64(v), md, scale)
+    assert compare_out(o, O_ref) <= O_TOL
+    el, same = compare_lse(lse, L_ref)
+    assert el <= LSE_TOL and same
+    assert float((o.float() - o_on.float()).abs().max()) <= O_TOL
+    assert float((lse - lse_on).abs().max()) <= LSE_TOL
