@@ -231,11 +231,15 @@ typedef struct bsa_workspace_view {
 
 /* Bytes of workspace a problem needs.  with_backward = 0 sizes the forward
  * only (plan + fixed-m bound); 1 adds Delta, the fp32 dQ accumulator and the
- * semaphores.  Pure host arithmetic; no CUDA call. */
+ * semaphores.  Pure host arithmetic; no CUDA call.
+ * Errors: INVALID_ARG (null prob or bytes, a size or stride out of range, an
+ * inconsistent mask spec), UNSUPPORTED (D not 64/128, a stride not a multiple
+ * of 8 elements, a sequence over 2^21, a map over 2^30 tiles). */
 BSA_API bsa_status bsa_workspace_size(const bsa_problem *prob, const bsa_mask_spec *mask,
                               int32_t with_backward, size_t *bytes);
 
-/* Offsets of the plan and scratch arrays inside the workspace (host only). */
+/* Offsets of the plan and scratch arrays inside the workspace (host only).
+ * Errors as for bsa_workspace_size. */
 BSA_API bsa_status bsa_workspace_layout(const bsa_problem *prob, const bsa_mask_spec *mask,
                                 bsa_workspace_view *view);
 
@@ -247,19 +251,30 @@ BSA_API bsa_status bsa_plan_build(const bsa_problem *prob, const bsa_mask_spec *
                           const bsa_options *opt, void *ws, size_t ws_bytes,
                           bsa_stream_t stream);
 
-/* Forward: out (bf16, o_stride layout) and lse (fp32 [B,H,Sq]).  With
+/* Forward (step a3; "Fixed-m softmax ...", introduction and "Notes"): out
+ * (bf16, o_stride layout) and lse (fp32 [B,H,Sq]).  With
  * BSA_SOFTMAX_FIXED_M_GATED it first computes kmax/qmax/gate per (b, h) and
  * runs the fixed-m body on heads that pass the gate, online softmax on the
- * others.  Rows in the varlen alignment tail are written as 0 / -inf. */
+ * others.  Rows in the varlen alignment tail are written as 0 / -inf.
+ * Builds the plan first unless opt->plan_ready (the workspace then holds one
+ * built for this problem, mask and order, which a signature check enforces).
+ * Errors: INVALID_ARG (a null tensor or workspace, a workspace not 256-byte
+ * aligned, an invalid option), UNSUPPORTED (a tensor not 16-byte aligned, lse
+ * not 4-byte aligned, or as for bsa_workspace_size), WORKSPACE_TOO_SMALL,
+ * NO_DEVICE (no sm_100 device current), CUDA (a launch failed). */
 BSA_API bsa_status bsa_attn_fwd(const bsa_problem *prob, const bsa_mask_spec *mask,
                         const bsa_options *opt, const void *q, const void *k,
                         const void *v, void *out, float *lse, void *ws,
                         size_t ws_bytes, bsa_stream_t stream);
 
-/* Backward: dq, dk, dv (bf16) from q, k, v, the forward's out and lse and the
- * incoming gradient dout.  deterministic = 1 orders every dQ contribution by the
- * dQ semaphores (bit-identical results run to run); 0 uses atomic adds.
- * Needs a workspace sized with with_backward = 1. */
+/* Backward (steps a4, a5, a7; "Add more optimal dk order optional arg", "What
+ * does this do" and "Sliding window perf issue"): dq, dk, dv (bf16, q_stride /
+ * k_stride / v_stride layouts) from q, k, v, the forward's out and lse and the
+ * incoming gradient dout.  deterministic = 1 orders every dQ contribution by
+ * the dQ semaphores (bit-identical results run to run); 0 uses atomic adds.
+ * Needs a workspace sized with with_backward = 1.  Errors as for bsa_attn_fwd;
+ * a semaphore wait that gives up is reported by bsa_get_device_status as
+ * BSA_ERR_SEM_TIMEOUT. */
 BSA_API bsa_status bsa_attn_bwd(const bsa_problem *prob, const bsa_mask_spec *mask,
                         const bsa_options *opt, const void *q, const void *k,
                         const void *v, const void *out, const void *dout,
@@ -350,8 +365,8 @@ BSA_API bsa_status bsa_get_device_status(void *ws, size_t ws_bytes, bsa_stream_t
 /* Static description of a status code. */
 BSA_API const char *bsa_status_string(bsa_status status);
 
-/* Number of this library's kernel launches issued by the calling thread since
- * load (for the bench's launch count). */
+/* Number of this library's kernel launches issued by the whole process since
+ * the library was loaded (all threads; for the bench's launch count). */
 BSA_API uint64_t bsa_launch_count(void);
 
 #ifdef __cplusplus
