@@ -776,7 +776,7 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
 // ---------------------------------------------------------------- a4: Delta
 constexpr int kDeltaRuns = 2;  // runs of consecutive rows per block, loads all in flight
 
-template <int D>
+template <int D, bool RESID>
 __global__ void __launch_bounds__(256) k_bwd_delta(const __nv_bfloat16 *__restrict__ o,
                                                    const __nv_bfloat16 *__restrict__ dout,
                                                    int64_t sb, int64_t ss, int64_t sh, int B,
@@ -788,7 +788,8 @@ __global__ void __launch_bounds__(256) k_bwd_delta(const __nv_bfloat16 *__restri
   // residual) each.  A block takes kDeltaRuns runs of 256 / (D/8) consecutive
   // rows of one head (the Delta layout), every run's loads in flight before any
   // is reduced; rows past Sq (the last q-block's padding) get Delta = 0.  The
-  // grid also zeroes the dQ semaphores.
+  // grid also zeroes the dQ semaphores.  RESID: the O residual is added to O
+  // (a compile-time choice, so that the plain pass carries no zero vector).
   constexpr int TPV = D / 8;
   constexpr int VPB = 256 / TPV;
   pdl_wait();  // O comes from the forward, launched just before
@@ -818,7 +819,7 @@ __global__ void __launch_bounds__(256) k_bwd_delta(const __nv_bfloat16 *__restri
       const int64_t off = b * sb + static_cast<int64_t>(i) * ss + h * sh + t * 8;
       av[j] = __ldg(reinterpret_cast<const int4 *>(o + off));
       cv[j] = __ldg(reinterpret_cast<const int4 *>(dout + off));
-      if (resid != nullptr)
+      if (RESID)
         rv[j] = __ldg(reinterpret_cast<const int4 *>(resid + ((static_cast<int64_t>(b) * Sq + i) * H + h) * D + t * 8));
     }
   }
@@ -833,9 +834,15 @@ __global__ void __launch_bounds__(256) k_bwd_delta(const __nv_bfloat16 *__restri
     float acc = 0.f;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      const float2 fo = unpack_bf16x2(xa[q]), fd = unpack_bf16x2(xc[q]), fr = unpack_bf16x2(xr[q]);
-      acc = fmaf(fo.x + fr.x, fd.x, acc);
-      acc = fmaf(fo.y + fr.y, fd.y, acc);
+      float2 fo = unpack_bf16x2(xa[q]);
+      const float2 fd = unpack_bf16x2(xc[q]);
+      if (RESID) {
+        const float2 fr = unpack_bf16x2(xr[q]);
+        fo.x += fr.x;
+        fo.y += fr.y;
+      }
+      acc = fmaf(fo.x, fd.x, acc);
+      acc = fmaf(fo.y, fd.y, acc);
     }
 #pragma unroll
     for (int sft = TPV / 2; sft > 0; sft >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, sft);
@@ -968,7 +975,9 @@ cudaError_t launch_bwd_preprocess(const bsa_problem &p, const bsa_options &o, co
   uint32_t *sem = reinterpret_cast<uint32_t *>(ws + L.sem);
   const int64_t n_sem = static_cast<int64_t>(p.B) * p.H * L.nM * 4;  // a quarter each
   // a programmatic dependent of the forward (which reads O first after it)
-  cudaError_t e = launch_pdl(p.D == 64 ? k_bwd_delta<64> : k_bwd_delta<128>, dim3(blocks), dim3(256), 0, s,
+  auto kern = p.D == 64 ? (resid != nullptr ? k_bwd_delta<64, true> : k_bwd_delta<64, false>)
+                        : (resid != nullptr ? k_bwd_delta<128, true> : k_bwd_delta<128, false>);
+  cudaError_t e = launch_pdl(kern, dim3(blocks), dim3(256), 0, s,
                              static_cast<const __nv_bfloat16 *>(out), static_cast<const __nv_bfloat16 *>(dout),
                              p.o_stride[0], p.o_stride[1], p.o_stride[2], p.B, p.Sq, p.H, rows_pad, resid,
                              delta, sem, n_sem);
