@@ -145,6 +145,45 @@ def test_workspace_size_and_validation(L):
     assert _size(L, _prob(), m)[0] == 1
 
 
+def test_every_mask_and_shape_check_rejects_its_case(L):
+    """The remaining rejection branches of the problem and mask checks, each
+    against an otherwise valid problem."""
+    def varlen(**kw):
+        m = bd.MaskSpec()
+        m.flags = bd.MASK_VARLEN
+        m.cu_seqlens, m.n_seqs, m.n_align_tail = 16, 2, 0
+        for k_, v_ in kw.items():
+            setattr(m, k_, v_)
+        return m
+    sq = dict(Sq=256, Skv=256)
+    assert _size(L, _prob(**sq), varlen())[0] == 0                   # the valid case
+    assert _size(L, _prob(**sq), varlen(n_seqs=0))[0] == 1          # no sequence
+    assert _size(L, _prob(**sq), varlen(n_align_tail=3))[0] == 1    # more alignment segments than segments
+    assert _size(L, _prob(**sq), varlen(n_align_tail=-1))[0] == 1
+    assert _size(L, _prob(**sq), varlen(cu_seqlens=None))[0] == 1
+    both = varlen(flags=bd.MASK_VARLEN | bd.MASK_SEGMENT_IDS, seg_q=16, seg_kv=16)
+    assert _size(L, _prob(**sq), both)[0] == 1                        # varlen and segment ids exclude each other
+    m = bd.MaskSpec()
+    m.flags = bd.MASK_CAUSAL_WINDOW
+    m.window = -1                                                     # a negative window
+    assert _size(L, _prob(), m)[0] == 1
+    m = bd.MaskSpec()
+    m.flags = bd.MASK_KV_VALID_LEN                                    # lengths missing
+    assert _size(L, _prob(), m)[0] == 1
+    m.kv_valid_len = 16
+    assert _size(L, _prob(), m)[0] == 0
+    p = _prob(H=6)
+    p.H_kv = 4                                                        # H not a multiple of H_kv
+    assert _size(L, p)[0] == 1
+    p.H_kv = -1
+    assert _size(L, p)[0] == 1
+    p.H_kv = 3
+    assert _size(L, p)[0] == 0
+    p = _prob()
+    p.k_stride[:] = (0, -128, 64)                                     # a non-positive stride
+    assert _size(L, p)[0] == 1
+
+
 def test_calls_reject_bad_arguments_before_cuda(L):
     p = _prob()
     o = bd.Options()
