@@ -40,9 +40,19 @@ sys.path.insert(0, ROOT)
 
 WORKLOAD_NAME = "window"
 WORKLOADS = {
+    "tiny": "tiny dense: B=1, H=2, Sq=Skv=256, D=64, bf16 N(0,1) seed 0, no mask",
+    "packed": "packed segments: B=2, H=8, S=4096, D=128, bf16 N(0,1) seed 1, segment runs of "
+              "uniform{256..2048} tokens (block-diagonal)",
+    "packed_const": "packed segments with one constant id per batch row (equal to no mask): B=2, H=8, "
+                    "S=4096, D=128, bf16 N(0,1) seed 1",
     "window": "causal sliding window 512: B=1, H=16, Sq=Skv=8192, D=128, bf16 N(0,1) seed 2",
     "window_rect": "causal sliding window 512, bottom-right: B=1, H=16, Sq=4096, Skv=8192, D=128, "
                    "bf16 N(0,1) seed 2",
+    "varlen": "varlen with alignment padding: H=24, D=128, T=33024, cu_seqlens=[0,33002,33024] "
+              "(22 alignment rows), non-causal, bf16 N(0,1) seed 3; forward only",
+    "video": "video-DiT: B=1, H=40, Sq=75600 (21x45x80), Skv=75776 (KV padded to a multiple of 2048, "
+             "padding masked), D=128, q,k ~ N(0,0.5) + 3-axis RoPE, head 0 with 8 sink keys x20, seed 4; "
+             "forward only",
     "prefix_lm": "prefix-LM (causal + bidirectional prefix of 2048): B=1, H=16, Sq=Skv=8192, "
                  "D=128, bf16 N(0,1) seed 2",
     "dilated": "dilated causal window (span 1024, dilation 2): B=1, H=16, Sq=Skv=8192, D=128, "
@@ -52,14 +62,22 @@ WORKLOADS = {
     "gqa": "grouped-query causal sliding window 512: B=1, H=16 over H_kv=4, Sq=Skv=8192, D=128, "
            "bf16 N(0,1) seed 5",
 }
+# forward-only workloads (the configs state no backward for them)
+FORWARD_ONLY = ("varlen", "video")
+# dense bf16 tcgen05 rate per SM and clock (flop), for the spec peak = SMs x max SM clock x rate
+BF16_FLOP_PER_CLK_SM = 8192
+DATASHEET_BF16_TFLOPS = 2250.0
 
 
 def workload_text(args):
-    bwd = "atomic (non-deterministic)" if args.nondet else f"deterministic ({args.order} kv-column order)"
     fwd = args.softmax + (" gated" if args.softmax == "fixed_m" else "")
     if args.softmax == "fixed_m" and args.bound == "smoothed":
         fwd += ", k-smoothed bound"
-    return f"{WORKLOADS[args.workload]}; forward {fwd} + {bwd} backward"
+    if args.workload in FORWARD_ONLY:
+        return f"{WORKLOADS[args.workload]}; forward {fwd}"
+    bwd = "atomic (non-deterministic)" if args.nondet else f"deterministic ({args.order} kv-column order)"
+    resid = "" if args.o_residual == "auto" else ", no O residual"
+    return f"{WORKLOADS[args.workload]}; forward {fwd} + {bwd} backward{resid}"
 METRIC = "attention TFLOP/s (non-empty tiles) fwd+bwd on 1 B200; % of bf16 tensor peak"
 
 
@@ -74,8 +92,11 @@ def parse():
                     help="fixed-m reference: Cauchy-Schwarz on ||k|| or on the centred keys")
     ap.add_argument("--order", default="desc", choices=["asc", "desc", "outside_in", "greedy"])
     ap.add_argument("--nondet", action="store_true", help="atomic (non-deterministic) dQ backward")
-    ap.add_argument("--residual", action="store_true",
-                    help="keep O's bf16 rounding residual for an exact-to-fp32 Delta")
+    ap.add_argument("--o-residual", default="auto", choices=["auto", "drop"],
+                    help="auto (the library default): the forward keeps O's bf16 rounding residual and "
+                         "Delta is exact to the fp32 O; drop: Delta from the bf16 O")
+    ap.add_argument("--no-orders", action="store_true",
+                    help="skip timing the backward main kernel under every kv-column order and atomically")
     ap.add_argument("--workload", default=WORKLOAD_NAME, choices=sorted(WORKLOADS))
     ap.add_argument("--small", action="store_true",
                     help="small shape of the same workload (for profiler captures)")
@@ -97,20 +118,6 @@ def load_peaks():
     except Exception:
         return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
                 "source": "fallback"}
-
-
-def profiled_traffic(kernel: str, workload: str):
-    """dram bytes per launch of `kernel` on `workload` from the committed ncu
-    summary (a line `traffic <kernel> <workload> <bytes>`), else None."""
-    path = os.path.join(ROOT, "profiles", "traffic.txt")
-    try:
-        for line in open(path):
-            parts = line.split()
-            if len(parts) == 4 and parts[0] == "traffic" and parts[1] == kernel and parts[2] == workload:
-                return float(parts[3])
-    except OSError:
-        pass
-    return None
 
 
 class ClockSampler:
@@ -236,11 +243,39 @@ def tiles_of(ws):
     return int(ptr[-1])
 
 
+def source_tag(*files) -> str:
+    """sha256 prefix of the kernel sources, so that a committed DRAM-traffic
+    figure is used only for the kernel build it was measured on."""
+    import hashlib
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "block_sparse_attention_map_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel: str, workload: str, src: str):
+    """dram bytes per launch of `kernel` on `workload` from the committed ncu
+    summary (a line `traffic <kernel> <workload> <bytes> <source tag>`), when it
+    was taken on the current kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    try:
+        for line in open(path):
+            parts = line.split()
+            if (len(parts) == 5 and parts[0] == "traffic" and parts[1] == kernel and parts[2] == workload
+                    and parts[4] == src):
+                return float(parts[3])
+    except OSError:
+        pass
+    return None
+
+
 # ------------------------------------------------------------------ CPU oracle leg
 
 def oracle_sample(wl, n_rows: int, head: int = 0):
-    """Time the fp64 oracle (forward + backward) on query rows [0, n_rows) of one
-    head against all keys; returns (seconds, useful flops credited, threads)."""
+    """Time the fp64 oracle (forward, and backward where the workload has one)
+    on query rows and keys [0, n_rows) of one head under the same mask
+    predicates; returns (seconds, useful flops credited, threads)."""
     import numpy as np
     import oracle
     try:
@@ -249,23 +284,31 @@ def oracle_sample(wl, n_rows: int, head: int = 0):
     except Exception:
         threads = os.cpu_count()
     f = lambda t: t.detach().float().cpu().numpy().astype(np.float64)
+    hk = head // (wl.H // wl.k.shape[2])
     q = f(wl.q[:, :n_rows, head:head + 1])
-    k, v = f(wl.k[:, :, head:head + 1]), f(wl.v[:, :, head:head + 1])
-    do = f(wl.dO[:, :n_rows, head:head + 1])
+    k, v = f(wl.k[:, :n_rows, hk:hk + 1]), f(wl.v[:, :n_rows, hk:hk + 1])
     # the sample treats rows and keys [0, n_rows) as a square problem with the
-    # same mask predicates (segment ids cut to the sample)
+    # same mask predicates (segment ids and cu_seqlens cut to the sample)
     desc = wl.mask_numpy()
     for key in ("seg_q", "seg_kv"):
         if key in desc:
             desc[key] = desc[key][:, :n_rows]
+    if "cu_seqlens" in desc:
+        cu = np.minimum(np.asarray(desc["cu_seqlens"]), n_rows)
+        desc["cu_seqlens"] = np.unique(cu)
+        desc["n_align_tail"] = 0 if cu[-1 - desc["n_align_tail"]] >= n_rows else desc["n_align_tail"]
+    if "kv_valid_len" in desc:
+        desc["kv_valid_len"] = np.minimum(desc["kv_valid_len"], n_rows)
     sub = oracle.MaskDesc(**desc)
     cls = oracle.tile_classes(sub, 1, n_rows, n_rows)
     t0 = time.perf_counter()
-    oracle.attention_forward(q, k[:, :n_rows], v[:, :n_rows], sub, wl.scale)
-    oracle.attention_backward(q, k[:, :n_rows], v[:, :n_rows], do, sub, wl.scale)
+    oracle.attention_forward(q, k, v, sub, wl.scale)
+    if wl.backward:
+        do = f(wl.dO[:, :n_rows, head:head + 1])
+        oracle.attention_backward(q, k, v, do, sub, wl.scale)
     dt = time.perf_counter() - t0
     nnz = int((cls != oracle.EMPTY).sum())
-    flops = oracle.useful_flops(nnz, wl.D) * 3.5
+    flops = oracle.useful_flops(nnz, wl.D) * (3.5 if wl.backward else 1.0)
     return dt, flops, threads
 
 
@@ -285,8 +328,9 @@ def run_reference(args, world, rank):
         total_t += dt
         total_f += fl
     value = total_f / total_t / 1e12
+    what = "forward + backward" if wl.backward else "forward"
     sample = (f"rows and keys 0..{n_rows - 1} of head 0 of {wl.H} under the same mask, "
-              f"forward + backward in fp64, per step")
+              f"{what} in fp64, per step")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
@@ -303,6 +347,65 @@ def run_reference(args, world, rank):
 
 # ------------------------------------------------------------------ GPU arm
 
+def _median_event_ms(fn, before, n, stream):
+    """Median CUDA-event time of fn() over n runs, before() (untimed: an L2 flush,
+    a stage the timed one depends on) ahead of each."""
+    import torch
+    times = []
+    for _ in range(n):
+        before()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        times.append(a.elapsed_time(b))
+    return statistics.median(times)
+
+
+def order_table(args, wl, flush, stream, n=10):
+    """backward_main (a5) under every kv-column order and the atomic variant,
+    measured in this run on this workload: median of n launches, L2 flushed and
+    Delta / the semaphores (or the zeroed accumulator) prepared before each."""
+    import block_sparse_attention_map_b200 as bsa
+    out = {}
+    for name in ("asc", "desc", "outside_in", "greedy", "atomic"):
+        st = bsa.Stages(wl.q, wl.k, wl.v, wl.mask, softmax_mode=args.softmax,
+                        order="desc" if name == "atomic" else name, deterministic=name != "atomic",
+                        bound_mode=args.bound, o_residual=args.o_residual)
+        st.plan_and_bound()
+        st.forward()
+
+        def before():
+            flush.zero_()
+            st.preprocess(wl.dO)
+
+        out[name] = _median_event_ms(lambda: st.backward_main(wl.dO), before, n, stream)
+        if st.ws.status() != 0:
+            raise RuntimeError(f"device status {st.ws.status()} timing the {name} backward")
+        del st
+    return out
+
+
+def softmax_table(args, wl, flush, stream, n=10):
+    """The forward (a3) under online and fixed-m softmax, measured in this run:
+    median of n launches, L2 flushed before each (plan and bound built once)."""
+    import block_sparse_attention_map_b200 as bsa
+    out, gates = {}, None
+    for mode in ("online", "fixed_m"):
+        st = bsa.Stages(wl.q, wl.k, wl.v, wl.mask, softmax_mode=mode, bound_mode=args.bound,
+                        o_residual=args.o_residual)
+        st.plan_and_bound()
+        out[mode] = _median_event_ms(st.forward, flush.zero_, n, stream)
+        if st.ws.status() != 0:
+            raise RuntimeError(f"device status {st.ws.status()} timing the {mode} forward")
+        if mode == "fixed_m":
+            g = st.ws.gate().cpu()
+            gates = {"fixed_m_heads": int(g.sum()), "online_heads": int(g.numel() - g.sum())}
+        del st
+    return out, gates
+
+
 def run_ours(args, world, rank, local):
     import torch
     import block_sparse_attention_map_b200 as bsa
@@ -310,33 +413,26 @@ def run_ours(args, world, rank, local):
 
     dev = torch.device("cuda", local)
     wl = make_workload(args.workload, device=dev, small=args.small)
+    has_bwd = wl.backward
     st = bsa.Stages(wl.q, wl.k, wl.v, wl.mask, softmax_mode=args.softmax, order=args.order,
-                    deterministic=not args.nondet, bound_mode=args.bound, keep_o_residual=args.residual)
+                    deterministic=not args.nondet, bound_mode=args.bound, o_residual=args.o_residual)
     dO = wl.dO
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
     # the planner runs beside the bound's pass over Q and K (one library call,
     # the plan on the library's side stream), then the rest in order
-    names = ["plan_and_bound", "forward", "preprocess", "backward_main", "convert"]
+    names = ["plan_and_bound", "forward"] + (["preprocess", "backward_main", "convert"] if has_bwd else [])
+    calls = {"plan_and_bound": st.plan_and_bound, "forward": st.forward,
+             "preprocess": lambda: st.preprocess(dO), "backward_main": lambda: st.backward_main(dO),
+             "convert": st.convert}
 
     def step(ev=None):
+        for i, n in enumerate(names):
+            if ev is not None:
+                ev[i].record(stream)
+            calls[n]()
         if ev is not None:
-            ev[0].record(stream)
-        st.plan_and_bound()
-        if ev is not None:
-            ev[1].record(stream)
-        st.forward()
-        if ev is not None:
-            ev[2].record(stream)
-        st.preprocess(dO)
-        if ev is not None:
-            ev[3].record(stream)
-        st.backward_main(dO)
-        if ev is not None:
-            ev[4].record(stream)
-        st.convert()
-        if ev is not None:
-            ev[5].record(stream)
+            ev[len(names)].record(stream)
 
     for _ in range(args.warmup):
         flush.zero_()
@@ -347,7 +443,7 @@ def run_ours(args, world, rank, local):
         raise RuntimeError(f"device status {status} after warm-up")
     n_tiles = tiles_of(st.ws) * wl.H  # non-empty tiles over all (b, h)
     f_fwd = 4.0 * 128 * 128 * wl.D * n_tiles
-    f_bwd = 2.5 * f_fwd
+    f_bwd = 2.5 * f_fwd if has_bwd else 0.0
 
     # eager pass: one library call per stage, an event between stages (the
     # per-stage split; every call's host work sits between the launches)
@@ -428,28 +524,49 @@ def run_ours(args, world, rank, local):
     # the same time over the flops of the allowed entries alone (4 D per pair
     # forward, 2.5x that backward), where the mask has a closed form
     pairs = window_pairs(wl)
-    exact_value = (whole_job_tflops(world, args.steps, 3.5 * 4.0 * wl.D * pairs, total_ms)
+    exact_value = (whole_job_tflops(world, args.steps, (3.5 if has_bwd else 1.0) * 4.0 * wl.D * pairs, total_ms)
                    if pairs is not None else None)
 
     peaks = load_peaks()
     peak = peaks["bf16_tflops"]
-    main_tf = f_bwd / (avg["backward_main"] * 1e-3) / 1e12
+    clocks = clk.summary()
+    n_sm = torch.cuda.get_device_properties(dev).multi_processor_count
+    max_mhz = clocks.get("sm_max_mhz") or 1965.0
+    spec_peak = n_sm * max_mhz * 1e6 * BF16_FLOP_PER_CLK_SM / 1e12
     fwd_tf = f_fwd / (avg["forward"] * 1e-3) / 1e12
+    main_tf = f_bwd / (avg["backward_main"] * 1e-3) / 1e12 if has_bwd else None
     tag = f"{args.workload}{wl.Sq}" if not args.small else None
-    traffic = profiled_traffic("k_attn_bwd", tag) if not args.nondet else None
+    src_fwd, src_bwd = source_tag("fwd.cu", "ptx.cuh"), source_tag("bwd.cu", "ptx.cuh")
+    roof_fwd = {"kernel": "k_attn_fwd (a3)", "bound": "tensor", "achieved": fwd_tf, "peak": peak,
+                "unit": "TFLOP/s", "frac": fwd_tf / peak, "traffic": profiled_traffic("k_attn_fwd", tag, src_fwd),
+                "peak_source": peaks["source"] + " bf16 burst",
+                "frac_of_spec_peak": fwd_tf / spec_peak}
+    if has_bwd:
+        roof = {"kernel": "k_attn_bwd (a5)", "bound": "tensor", "achieved": main_tf, "peak": peak,
+                "unit": "TFLOP/s", "frac": main_tf / peak,
+                "traffic": profiled_traffic("k_attn_bwd", tag, src_bwd) if not args.nondet else None,
+                "peak_source": peaks["source"] + " bf16 burst", "frac_of_spec_peak": main_tf / spec_peak}
+    else:
+        roof = roof_fwd
 
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": workload_text(args) + (" [small shape]" if args.small else ""),
-                   "global_batch": wl.B * world, "seq_len": wl.Sq, "heads": wl.H,
-                   "head_dim": wl.D, "mask": wl.mask_text(), "nonempty_tiles": n_tiles,
-                   "softmax": args.softmax, "bound": args.bound, "o_residual": args.residual,
-                   "bwd_order": "nondeterministic" if args.nondet else args.order,
+                   "global_batch": wl.B * world, "seq_len": wl.Sq, "kv_len": wl.Skv, "heads": wl.H,
+                   "kv_heads": wl.k.shape[2], "head_dim": wl.D, "mask": wl.mask_text(),
+                   "nonempty_tiles": n_tiles, "softmax": args.softmax, "bound": args.bound,
+                   "passes": "forward + backward" if has_bwd else "forward only",
+                   "o_residual": args.o_residual if has_bwd else None,
+                   "bwd_order": ("nondeterministic" if args.nondet else args.order) if has_bwd else None,
                    "l2": "flushed (256 MiB write) before every step, outside the timed events",
                    "parallelism": f"replicas x{world}"},
         "pct_of_bf16_peak": 100.0 * value / peak,
+        "pct_of_spec_peak": 100.0 * value / spec_peak,
+        "spec_peak_tflops": spec_peak,
+        "spec_peak_note": f"{n_sm} SMs x {max_mhz:.0f} MHz (max SM clock) x {BF16_FLOP_PER_CLK_SM} dense bf16 "
+                          f"flop/clk/SM; datasheet {DATASHEET_BF16_TFLOPS:.0f} TFLOP/s",
         "exact_mask_tflops": exact_value,
         "exact_mask_pairs": pairs,
         "stages_ms": avg,
@@ -459,54 +576,69 @@ def run_ours(args, world, rank, local):
         "eager_gpu_launches_per_step": eager_launches / args.steps,
         "forward_tflops": fwd_tf,
         "forward_pct_of_peak": 100.0 * fwd_tf / peak,
-        "backward_tflops": f_bwd / ((avg["preprocess"] + avg["backward_main"] + avg["convert"]) * 1e-3) / 1e12,
-        "backward_main_tflops": main_tf,
-        "roofline": {"kernel": "k_attn_bwd (a5)", "bound": "tensor", "achieved": main_tf,
-                     "peak": peak, "unit": "TFLOP/s", "frac": main_tf / peak,
-                     "traffic": traffic, "peak_source": peaks["source"] + " bf16 burst"},
-        "roofline_forward": {"kernel": "k_attn_fwd (a3)", "bound": "tensor", "achieved": fwd_tf,
-                             "peak": peak, "unit": "TFLOP/s", "frac": fwd_tf / peak,
-                             "traffic": profiled_traffic("k_attn_fwd", tag)},
-        "gpu_launches": launches,
-        "wall_s_timed_loop": t_wall,
-        "clocks": clk.summary(),
+        "forward_pct_of_spec_peak": 100.0 * fwd_tf / spec_peak,
     }
+    if has_bwd:
+        bwd_ms = avg["preprocess"] + avg["backward_main"] + avg["convert"]
+        line.update({
+            "backward_tflops": f_bwd / (bwd_ms * 1e-3) / 1e12,
+            "backward_pct_of_peak": 100.0 * f_bwd / (bwd_ms * 1e-3) / 1e12 / peak,
+            "backward_main_tflops": main_tf,
+            "backward_main_pct_of_peak": 100.0 * main_tf / peak,
+            "backward_main_pct_of_spec_peak": 100.0 * main_tf / spec_peak,
+        })
+    line["roofline"] = roof
+    if has_bwd:
+        line["roofline_forward"] = roof_fwd
+    line.update({"gpu_launches": launches, "wall_s_timed_loop": t_wall, "clocks": clocks})
 
+    if has_bwd and not args.no_orders:
+        ords = order_table(args, wl, flush, stream)
+        line["backward_main_ms_by_order"] = ords
+        line["backward_main_tflops_by_order"] = {k: f_bwd / (v * 1e-3) / 1e12 for k, v in ords.items()}
+    if not has_bwd:
+        fm, gates = softmax_table(args, wl, flush, stream)
+        line["forward_ms_by_softmax"] = fm
+        line["forward_tflops_by_softmax"] = {k: f_fwd / (v * 1e-3) / 1e12 for k, v in fm.items()}
+        line["fixed_m_gate"] = gates
     if not args.no_e2e:
         line["e2e"] = e2e_leg(args, wl, dev, f_fwd + f_bwd, world)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         n_rows = min(1024, wl.Sq)
         dt, fl, threads = oracle_sample(wl, n_rows)
+        what = "forward + backward" if has_bwd else "forward"
         line["cpu_baseline"] = {
             "value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-            "sample": f"rows and keys 0..{n_rows - 1} of head 0 under the same mask, forward + "
-                      f"backward, fp64"}
+            "sample": f"rows and keys 0..{n_rows - 1} of head 0 under the same mask, {what}, fp64"}
     if rank == 0:
         print(json.dumps(line), flush=True)
 
 
 def e2e_leg(args, wl, dev, flops, world):
     """The same step through the public API with host buffers: every step copies
-    its own q, k, v, dO from pinned host memory to the device, runs the full
-    path and copies O, LSE, dQ, dK, dV back to pinned host memory, all inside
-    the timed region.  Steps are pipelined as a training loop would run them:
-    two buffer sets, the uploads, the compute and the downloads on three
-    streams (PCIe carries both directions at once), each set reused only after
-    its previous compute and download are done."""
+    its own inputs (q, k, v and, with a backward, dO) from pinned host memory to
+    the device, runs the full path and copies its results (O, LSE and dQ, dK,
+    dV) back to pinned host memory, all inside the timed region.  Steps are
+    pipelined as a training loop would run them: two buffer sets, the uploads,
+    the compute and the downloads on three streams (PCIe carries both directions
+    at once), each set reused only after its previous compute and download are
+    done."""
     import torch
     import block_sparse_attention_map_b200 as bsa
 
-    names_in = ("q", "k", "v", "dO")
+    has_bwd = wl.backward
+    names_in = ("q", "k", "v", "dO") if has_bwd else ("q", "k", "v")
     host = {n: getattr(wl, n).cpu().pin_memory() for n in names_in}
-    out_spec = (("o", wl.q.shape, torch.bfloat16), ("lse", (wl.B, wl.H, wl.Sq), torch.float32),
-                ("dq", wl.q.shape, torch.bfloat16), ("dk", wl.k.shape, torch.bfloat16),
-                ("dv", wl.v.shape, torch.bfloat16))
+    out_spec = [("o", wl.q.shape, torch.bfloat16), ("lse", (wl.B, wl.H, wl.Sq), torch.float32)]
+    if has_bwd:
+        out_spec += [("dq", wl.q.shape, torch.bfloat16), ("dk", wl.k.shape, torch.bfloat16),
+                     ("dv", wl.v.shape, torch.bfloat16)]
     slots = []
     for _ in range(2):
         dev_in = {n: torch.empty_like(getattr(wl, n)) for n in names_in}
         st = bsa.Stages(dev_in["q"], dev_in["k"], dev_in["v"], wl.mask, softmax_mode=args.softmax,
                         order=args.order, deterministic=not args.nondet, bound_mode=args.bound,
-                        keep_o_residual=args.residual)
+                        o_residual=args.o_residual)
         out_h = {n: torch.empty(shape, dtype=dt).pin_memory() for n, shape, dt in out_spec}
         ev = {k: torch.cuda.Event() for k in ("in", "comp", "out")}
         slots.append({"in": dev_in, "st": st, "out_h": out_h, "ev": ev, "used": False})
@@ -528,14 +660,16 @@ def e2e_leg(args, wl, dev, flops, world):
                 s_comp.wait_event(ev["out"])  # its outputs were read back
             st.plan_and_bound()
             st.forward()
-            st.preprocess(dev_in["dO"])
-            st.backward_main(dev_in["dO"])
-            st.convert()
+            if has_bwd:
+                st.preprocess(dev_in["dO"])
+                st.backward_main(dev_in["dO"])
+                st.convert()
             ev["comp"].record(s_comp)
         with torch.cuda.stream(s_down):
             s_down.wait_event(ev["comp"])
-            for n, src in (("o", st.out), ("lse", st.lse), ("dq", st.dq), ("dk", st.dk), ("dv", st.dv)):
-                sl["out_h"][n].copy_(src, non_blocking=True)
+            srcs = {"o": st.out, "lse": st.lse, "dq": st.dq, "dk": st.dk, "dv": st.dv}
+            for n, _, _ in out_spec:
+                sl["out_h"][n].copy_(srcs[n], non_blocking=True)
             ev["out"].record(s_down)
         sl["used"] = True
 

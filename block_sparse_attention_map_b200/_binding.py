@@ -27,6 +27,7 @@ MASK_SEGMENT_IDS, MASK_KV_VALID_LEN, MASK_VARLEN, MASK_CAUSAL_WINDOW, MASK_PREFI
 SOFTMAX_ONLINE, SOFTMAX_FIXED_M_GATED = 0, 1
 BOUND = {"norm": 0, "smoothed": 1}
 ORDER = {"asc": 0, "desc": 1, "perm": 2, "outside_in": 3, "greedy": 4}
+O_RESIDUAL = {"auto": 0, "keep": 1, "drop": 2}
 FULL_BIT = 1 << 30
 STATUS = {
     0: "BSA_OK", 1: "BSA_ERR_INVALID_ARG", 2: "BSA_ERR_UNSUPPORTED",
@@ -54,7 +55,7 @@ class Options(ctypes.Structure):
     _fields_ = [("softmax_mode", c_i32), ("gate_limit", c_f32), ("kmax_override", c_vp),
                 ("bwd_order", c_i32), ("deterministic", c_i32), ("perm", c_vp),
                 ("sem_timeout_ns", c_i64), ("plan_ready", c_i32), ("bound_ready", c_i32),
-                ("bound_mode", c_i32), ("keep_o_residual", c_i32)]
+                ("bound_mode", c_i32), ("o_residual", c_i32)]
 
 
 class WorkspaceView(ctypes.Structure):
@@ -109,6 +110,10 @@ def lib() -> ctypes.CDLL:
             "bsa_bwd_convert": (c_i32, [P(Problem), P(MaskSpec), c_vp, c_vp, ctypes.c_size_t, c_vp]),
             "bsa_get_device_status": (c_i32, [c_vp, ctypes.c_size_t, c_vp, c_i32]),
             "bsa_status_string": (ctypes.c_char_p, [c_i32]),
+            "bsa_attn_fwd_static_scratch": (c_i32, [P(Problem), P(MaskSpec), P(Options), c_vp, c_vp, c_vp, c_vp,
+                                                    c_vp, c_vp]),
+            "bsa_static_scratch_init": (c_i32, []),
+            "bsa_static_scratch_status": (c_i32, [c_vp, c_i32]),
             "bsa_launch_count": (ctypes.c_uint64, []),
         }
         for name, (res, args) in sig.items():
@@ -208,7 +213,7 @@ class Mask:
 
 def make_options(softmax_mode="online", gate_limit=0.0, kmax_override=None, order="asc",
                  perm=None, deterministic=True, sem_timeout_ns=0, plan_ready=False,
-                 bound_ready=False, bound_mode="norm", keep_o_residual=False):
+                 bound_ready=False, bound_mode="norm", o_residual="auto"):
     o = Options()
     o.softmax_mode = SOFTMAX_FIXED_M_GATED if softmax_mode in ("fixed_m", SOFTMAX_FIXED_M_GATED) else SOFTMAX_ONLINE
     o.gate_limit = float(gate_limit)
@@ -219,7 +224,7 @@ def make_options(softmax_mode="online", gate_limit=0.0, kmax_override=None, orde
     o.plan_ready = 1 if plan_ready else 0
     o.bound_ready = 1 if bound_ready else 0
     o.bound_mode = BOUND[bound_mode] if isinstance(bound_mode, str) else int(bound_mode)
-    o.keep_o_residual = 1 if keep_o_residual else 0
+    o.o_residual = O_RESIDUAL[o_residual] if isinstance(o_residual, str) else int(o_residual)
     o._perm_buf = None
     if perm is not None:
         buf = (c_i32 * len(perm))(*[int(x) for x in perm])
@@ -317,18 +322,23 @@ def plan_build(q, k, v, mask=None, workspace: Optional[Workspace] = None, backwa
 
 def attn_fwd(q, k, v, mask=None, softmax_mode="online", gate_limit=0.0, kmax_override=None,
              workspace: Optional[Workspace] = None, out=None, lse=None, plan_ready=False,
-             scale=None, order="asc", perm=None, bound_mode="norm", keep_o_residual=False):
+             scale=None, order="asc", perm=None, bound_mode="norm", o_residual="auto",
+             for_backward=True):
     """O = softmax(scale Q K^T + mask) V and LSE [B, H, Sq] through bsa_attn_fwd.
-    With keep_o_residual the workspace is sized for the backward and keeps O's
-    bf16 rounding residual for an attn_bwd on the same workspace."""
+
+    The workspace it allocates (unless one is given) is sized for a backward
+    (``for_backward``), so that with the default ``o_residual="auto"`` it keeps
+    O's bf16 rounding residual: an ``attn_bwd(..., workspace=ws)`` on the
+    returned workspace then takes Delta exact to the fp32 O.  Returns
+    (out, lse, workspace)."""
     B, Sq, H, D = q.shape
     out = torch.empty_like(q) if out is None else out
     lse = torch.empty(B, H, Sq, dtype=torch.float32, device=q.device) if lse is None else lse
     prob = make_problem(q, k, v, out, scale)
     m = Mask(mask, q.device)
     o = make_options(softmax_mode, gate_limit, kmax_override, order, perm, True, 0, plan_ready,
-                     bound_mode=bound_mode, keep_o_residual=keep_o_residual)
-    ws = workspace or Workspace(prob, m, keep_o_residual, q.device)
+                     bound_mode=bound_mode, o_residual=o_residual)
+    ws = workspace or Workspace(prob, m, for_backward or o_residual == "keep", q.device)
     _check(lib().bsa_attn_fwd(ctypes.byref(prob), ctypes.byref(m.spec), ctypes.byref(o), q.data_ptr(),
                               k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), ws.ptr(),
                               ws.nbytes, _stream()), "bsa_attn_fwd")
@@ -338,16 +348,18 @@ def attn_fwd(q, k, v, mask=None, softmax_mode="online", gate_limit=0.0, kmax_ove
 
 def attn_bwd(q, k, v, out, dout, lse, mask=None, order="asc", perm=None, deterministic=True,
              workspace: Optional[Workspace] = None, plan_ready=False, scale=None,
-             dq=None, dk=None, dv=None, sem_timeout_ns=0, keep_o_residual=False):
-    """dQ, dK, dV of sum(O * dO) through bsa_attn_bwd.  keep_o_residual: Delta
-    uses the O residual an attn_fwd(keep_o_residual=True) left in ``workspace``."""
+             dq=None, dk=None, dv=None, sem_timeout_ns=0, o_residual="auto"):
+    """dQ, dK, dV of sum(O * dO) through bsa_attn_bwd.  Pass the forward's
+    workspace: with ``o_residual="auto"`` (or "keep") Delta then uses the O
+    residual that attn_fwd kept there for this ``out`` (checked on the device);
+    without it, or with "drop", Delta comes from the bf16 O."""
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
     prob = make_problem(q, k, v, out, scale)
     m = Mask(mask, q.device)
     o = make_options("online", 0.0, None, order, perm, deterministic, sem_timeout_ns, plan_ready,
-                     keep_o_residual=keep_o_residual)
+                     o_residual=o_residual)
     ws = workspace or Workspace(prob, m, True, q.device)
     _check(lib().bsa_attn_bwd(ctypes.byref(prob), ctypes.byref(m.spec), ctypes.byref(o), q.data_ptr(),
                               k.data_ptr(), v.data_ptr(), out.data_ptr(), dout.data_ptr(), lse.data_ptr(),
@@ -363,7 +375,7 @@ class Stages:
     workspace, for callers that time or schedule stages separately."""
 
     def __init__(self, q, k, v, mask=None, softmax_mode="online", order="asc", perm=None,
-                 deterministic=True, gate_limit=0.0, bound_mode="norm", keep_o_residual=False):
+                 deterministic=True, gate_limit=0.0, bound_mode="norm", o_residual="auto"):
         self.q, self.k, self.v = q, k, v
         B, Sq, H, D = q.shape
         self.out = torch.empty_like(q)
@@ -374,7 +386,7 @@ class Stages:
         self.fixed = softmax_mode in ("fixed_m", SOFTMAX_FIXED_M_GATED)
         self.opt = make_options(softmax_mode, gate_limit, None, order, perm, deterministic, 0,
                                 plan_ready=True, bound_ready=True, bound_mode=bound_mode,
-                                keep_o_residual=keep_o_residual)
+                                o_residual=o_residual)
         self.ws = Workspace(self.prob, self.mask, True, q.device)
         self._args = (ctypes.byref(self.prob), ctypes.byref(self.mask.spec), ctypes.byref(self.opt))
 

@@ -201,6 +201,7 @@ bsa_status check_options(const bsa_options *o, int nN, bsa_options *out) {
   if (o->bwd_order < BSA_ORDER_ASC || o->bwd_order > BSA_ORDER_GREEDY) return BSA_ERR_INVALID_ARG;
   if (o->bound_mode != BSA_BOUND_NORM && o->bound_mode != BSA_BOUND_SMOOTHED) return BSA_ERR_INVALID_ARG;
   if (o->bound_mode == BSA_BOUND_SMOOTHED && o->kmax_override != nullptr) return BSA_ERR_INVALID_ARG;
+  if (o->o_residual < BSA_O_RESIDUAL_AUTO || o->o_residual > BSA_O_RESIDUAL_DROP) return BSA_ERR_INVALID_ARG;
   if (o->bwd_order == BSA_ORDER_PERM) {
     if (o->perm == nullptr) return BSA_ERR_INVALID_ARG;
     std::vector<char> seen(static_cast<size_t>(nN), 0);
@@ -280,7 +281,7 @@ bsa_status prepare(const bsa_problem *prob, const bsa_mask_spec *mask, const bsa
   if (out->empty) return BSA_OK;
   if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return BSA_ERR_INVALID_ARG;
   // the O residual lives in the backward part of the workspace
-  const bool full = backward || out->o.keep_o_residual != 0;
+  const bool full = backward || out->o.o_residual == BSA_O_RESIDUAL_KEEP;
   if (ws_bytes < (full ? out->L.total : out->L.fwd_end)) return BSA_ERR_WORKSPACE_TOO_SMALL;
   if (!have_device()) return BSA_ERR_NO_DEVICE;
   return BSA_OK;
@@ -435,7 +436,13 @@ bsa_status attn_fwd_impl(const bsa_problem *prob, const bsa_mask_spec *mask,
       return st;
   }
   const MaskParams mp = mask_params(p, P.m, P.L, w);
-  return cuda_status(launch_fwd(p, mp, P.o, signature(p, P.m, P.o), tq, tk, tv, out, lse, P.L, w, s));
+  // the residual is kept when asked for, or by default when the workspace can
+  // serve a backward; the forward records in the header which `out` it is for
+  bsa_options fo = P.o;
+  const bool keep = P.o.o_residual == BSA_O_RESIDUAL_KEEP ||
+                    (P.o.o_residual == BSA_O_RESIDUAL_AUTO && ws_bytes >= P.L.total);
+  fo.o_residual = keep ? BSA_O_RESIDUAL_KEEP : BSA_O_RESIDUAL_DROP;
+  return cuda_status(launch_fwd(p, mp, fo, signature(p, P.m, P.o), tq, tk, tv, out, lse, P.L, w, s));
 }
 
 }  // namespace bsa

@@ -776,12 +776,20 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
 // ---------------------------------------------------------------- a4: Delta
 constexpr int kDeltaRuns = 2;  // runs of consecutive rows per block, loads all in flight
 
+// Half the spacing of bf16 numbers in the binade of the bf16 value with these
+// 16 bits, 2^(e - 135) for biased exponent e (clamped for subnormals and zero).
+__device__ __forceinline__ float half_ulp_bf16(uint32_t bits) {
+  const uint32_t e = (bits >> 7) & 0xffu;
+  return __uint_as_float((max(e, 9u) - 8u) << 23);
+}
+
 template <int D, bool RESID>
 __global__ void __launch_bounds__(256) k_bwd_delta(const __nv_bfloat16 *__restrict__ o,
                                                    const __nv_bfloat16 *__restrict__ dout,
                                                    int64_t sb, int64_t ss, int64_t sh, int B,
-                                                   int Sq, int H, int rows_pad,
+                                                   int Sq, int H, int Skv, int rows_pad,
                                                    const __nv_bfloat16 *__restrict__ resid,
+                                                   const uint32_t *__restrict__ hdr,
                                                    float *__restrict__ delta,
                                                    uint32_t *__restrict__ sem, int64_t n_sem) {
   // D/8 threads per (b, h, i) row vector, 16 bytes of O, dO (and the O
@@ -789,11 +797,24 @@ __global__ void __launch_bounds__(256) k_bwd_delta(const __nv_bfloat16 *__restri
   // rows of one head (the Delta layout), every run's loads in flight before any
   // is reduced; rows past Sq (the last q-block's padding) get Delta = 0.  The
   // grid also zeroes the dQ semaphores.  RESID: the O residual is added to O
-  // (a compile-time choice, so that the plain pass carries no zero vector).
+  // (a compile-time choice, so that the plain pass carries no zero vector),
+  // and only when the header records that the last forward on this workspace
+  // kept the residual of this very `o` for this problem (else Delta comes from
+  // the bf16 O alone).  A true residual never exceeds half a bf16 ulp of its
+  // O element; a residual element above that is dropped, so that even a stale
+  // record (a workspace reused after another forward wrote into the same
+  // output buffer) moves Delta by no more than the bf16 O alone would.
   constexpr int TPV = D / 8;
   constexpr int VPB = 256 / TPV;
   pdl_wait();  // O comes from the forward, launched just before
   pdl_trigger();
+  bool use_resid = false;
+  if (RESID) {
+    const uint64_t tag = (static_cast<uint64_t>(hdr[kHdrResidHi]) << 32) | hdr[kHdrResidLo];
+    use_resid = tag == reinterpret_cast<uint64_t>(o) && hdr[kHdrResidB] == static_cast<uint32_t>(B) &&
+                hdr[kHdrResidH] == static_cast<uint32_t>(H) && hdr[kHdrResidSq] == static_cast<uint32_t>(Sq) &&
+                hdr[kHdrResidSkv] == static_cast<uint32_t>(Skv) && hdr[kHdrResidD] == static_cast<uint32_t>(D);
+  }
   for (int64_t z = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; z < n_sem;
        z += static_cast<int64_t>(gridDim.x) * blockDim.x)
     sem[z] = 0u;
@@ -819,7 +840,7 @@ __global__ void __launch_bounds__(256) k_bwd_delta(const __nv_bfloat16 *__restri
       const int64_t off = b * sb + static_cast<int64_t>(i) * ss + h * sh + t * 8;
       av[j] = __ldg(reinterpret_cast<const int4 *>(o + off));
       cv[j] = __ldg(reinterpret_cast<const int4 *>(dout + off));
-      if (RESID)
+      if (use_resid)
         rv[j] = __ldg(reinterpret_cast<const int4 *>(resid + ((static_cast<int64_t>(b) * Sq + i) * H + h) * D + t * 8));
     }
   }
@@ -836,10 +857,10 @@ __global__ void __launch_bounds__(256) k_bwd_delta(const __nv_bfloat16 *__restri
     for (int q = 0; q < 4; ++q) {
       float2 fo = unpack_bf16x2(xa[q]);
       const float2 fd = unpack_bf16x2(xc[q]);
-      if (RESID) {
+      if (use_resid) {
         const float2 fr = unpack_bf16x2(xr[q]);
-        fo.x += fr.x;
-        fo.y += fr.y;
+        fo.x += fabsf(fr.x) <= half_ulp_bf16(xa[q] & 0xffffu) ? fr.x : 0.f;
+        fo.y += fabsf(fr.y) <= half_ulp_bf16(xa[q] >> 16) ? fr.y : 0.f;
       }
       acc = fmaf(fo.x, fd.x, acc);
       acc = fmaf(fo.y, fd.y, acc);
@@ -967,8 +988,9 @@ cudaError_t launch_bwd_preprocess(const bsa_problem &p, const bsa_options &o, co
   const int rows_pad = L.nM * kTile;
   const int64_t groups = static_cast<int64_t>(p.B) * p.H * rows_pad;
   float *delta = reinterpret_cast<float *>(ws + L.delta);
-  const __nv_bfloat16 *resid =
-      o.keep_o_residual ? reinterpret_cast<const __nv_bfloat16 *>(ws + L.o_resid) : nullptr;
+  const __nv_bfloat16 *resid = o.o_residual != BSA_O_RESIDUAL_DROP
+                                   ? reinterpret_cast<const __nv_bfloat16 *>(ws + L.o_resid)
+                                   : nullptr;
   // kDeltaRuns runs of 256 / (D / 8) vectors per block
   const int64_t vpb = kDeltaRuns * (256 / (p.D / 8));
   const unsigned blocks = static_cast<unsigned>((groups + vpb - 1) / vpb);
@@ -979,8 +1001,8 @@ cudaError_t launch_bwd_preprocess(const bsa_problem &p, const bsa_options &o, co
                         : (resid != nullptr ? k_bwd_delta<128, true> : k_bwd_delta<128, false>);
   cudaError_t e = launch_pdl(kern, dim3(blocks), dim3(256), 0, s,
                              static_cast<const __nv_bfloat16 *>(out), static_cast<const __nv_bfloat16 *>(dout),
-                             p.o_stride[0], p.o_stride[1], p.o_stride[2], p.B, p.Sq, p.H, rows_pad, resid,
-                             delta, sem, n_sem);
+                             p.o_stride[0], p.o_stride[1], p.o_stride[2], p.B, p.Sq, p.H, p.Skv, rows_pad, resid,
+                             reinterpret_cast<const uint32_t *>(ws + L.status), delta, sem, n_sem);
   if (e != cudaSuccess) return e;
   count_launch();
   if (!o.deterministic) {

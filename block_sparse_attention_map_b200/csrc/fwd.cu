@@ -191,6 +191,18 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
     if (!ok) wd.trip(BSA_ERR_PLAN_MISMATCH);
     // the swizzled tiles rely on a 1024-byte aligned dynamic shared window
     if ((smem_u32(sm) & 1023u) != 0u) wd.trip(BSA_ERR_UNSUPPORTED);
+    if (blockIdx.x == 0) {
+      // which output (none: 0) and problem the O residual belongs to, for the
+      // backward's Delta
+      const uint64_t tag = (ok && p.o_resid != nullptr) ? reinterpret_cast<uint64_t>(p.out) : 0ull;
+      p.hdr[kHdrResidLo] = static_cast<uint32_t>(tag);
+      p.hdr[kHdrResidHi] = static_cast<uint32_t>(tag >> 32);
+      p.hdr[kHdrResidB] = p.B;
+      p.hdr[kHdrResidH] = p.H;
+      p.hdr[kHdrResidSq] = p.Sq;
+      p.hdr[kHdrResidSkv] = p.Skv;
+      p.hdr[kHdrResidD] = D;
+    }
   }
   __syncthreads();
   pdl_trigger();  // the Delta pass of a backward may launch (it waits for our completion)
@@ -954,7 +966,7 @@ cudaError_t launch_fwd(const bsa_problem &p, const MaskParams &mp, const bsa_opt
   fp.kmax = reinterpret_cast<const float *>(ws + L.kmax);
   fp.qnorm = reinterpret_cast<const float *>(ws + L.qnorm);
   fp.qdot = o.bound_mode == BSA_BOUND_SMOOTHED ? reinterpret_cast<const float *>(ws + L.qdot) : nullptr;
-  fp.o_resid = o.keep_o_residual ? reinterpret_cast<__nv_bfloat16 *>(ws + L.o_resid) : nullptr;
+  fp.o_resid = o.o_residual == BSA_O_RESIDUAL_KEEP ? reinterpret_cast<__nv_bfloat16 *>(ws + L.o_resid) : nullptr;
   fp.gate = reinterpret_cast<const int32_t *>(ws + L.gate);
   fp.hdr = reinterpret_cast<uint32_t *>(ws + L.status);
   fp.timeout_ns = 2000000000ull;

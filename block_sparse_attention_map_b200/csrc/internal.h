@@ -38,6 +38,17 @@ enum HeaderWord : int {
   kHdrOrder = 10,
   kHdrNSeqs = 11,
   kHdrDilation = 12,
+  kHdrPlanWords = 56,  // words [0, 56) are reset by every plan build
+  // The O-residual record (kept across plan builds): the `out` pointer whose
+  // residual the last forward on this workspace kept (0: none) and the problem
+  // it was kept for, whose layout places the residual.
+  kHdrResidLo = 56,
+  kHdrResidHi = 57,
+  kHdrResidB = 58,
+  kHdrResidH = 59,
+  kHdrResidSq = 60,
+  kHdrResidSkv = 61,
+  kHdrResidD = 62,
   kHdrWords = 64
 };
 

@@ -531,7 +531,7 @@ __global__ void __launch_bounds__(1024, 1) k_plan_fused(FusedPlanArgs pa) {
   int32_t *rank_s = shm + F.rank;      // [BnM * nN]
   uint8_t *cls_s = reinterpret_cast<uint8_t *>(shm + F.cls);  // [BnM * nN]
   unsigned long long *keys = reinterpret_cast<unsigned long long *>(shm + F.keys);  // [nw][nM]
-  if (threadIdx.x < kHdrWords) pa.hdr[threadIdx.x] = 0u;
+  if (threadIdx.x < kHdrPlanWords) pa.hdr[threadIdx.x] = 0u;
   for (int i = threadIdx.x; i < BnN; i += blockDim.x) ccnt[i] = 0;
   __syncthreads();
   // tile classes, a warp per row block
@@ -749,7 +749,7 @@ cudaError_t launch_plan(const bsa_problem &p, const bsa_mask_spec &m, const bsa_
     count_launch();
     return cudaGetLastError();
   }
-  e = cudaMemsetAsync(hdr, 0, kHdrWords * sizeof(uint32_t), s);
+  e = cudaMemsetAsync(hdr, 0, kHdrPlanWords * sizeof(uint32_t), s);
   if (e != cudaSuccess) return e;
 
   const int4 *qblk = nullptr, *kblk = nullptr;

@@ -29,7 +29,9 @@ void *g_scratch_ptr[kMaxDevices] = {};
 
 // Device address of the array for the current device.  The host-side name
 // g_bsa_static_scratch is only a stand-in symbol, never a device address, so it
-// is resolved once per device with that device current.
+// is resolved once per device with that device current.  The first lookup on a
+// device may load this library's device code there (lazy module loading),
+// which is when the driver places the array in device memory.
 bsa_status scratch_for_current_device(void **out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return BSA_ERR_NO_DEVICE;
@@ -69,8 +71,23 @@ extern "C" bsa_status bsa_attn_fwd_static_scratch(const bsa_problem *prob,
   if (opt != nullptr) o = *opt;
   o.plan_ready = 0;
   o.bound_ready = 0;
-  o.keep_o_residual = 0;  // no backward shares this scratch
+  o.o_residual = BSA_O_RESIDUAL_DROP;  // no backward shares this scratch
   // plan and bound one after the other on `stream`: no side stream, no events
   return bsa::attn_fwd_impl(prob, mask, &o, q, k, v, out, lse, ws, kStaticScratchBytes, stream,
                             false);
+}
+
+extern "C" bsa_status bsa_static_scratch_init(void) {
+  void *ws = nullptr;
+  return scratch_for_current_device(&ws);
+}
+
+extern "C" bsa_status bsa_static_scratch_status(bsa_stream_t stream, int32_t clear) {
+  void *ws = nullptr;
+  const bsa_status st = scratch_for_current_device(&ws);
+  if (st != BSA_OK) return st;
+  // the array's first bytes are the workspace header: the sticky status word,
+  // then the fixed-m gate-warning count (read into the caller's stack: no
+  // allocation)
+  return bsa_get_device_status(ws, kStaticScratchBytes, stream, clear);
 }

@@ -193,14 +193,34 @@ typedef struct bsa_options {
                                   q and k; 0: bsa_attn_fwd computes them first      */
   int32_t bound_mode;          /* BSA_BOUND_*; SMOOTHED with kmax_override or with
                                   H_kv*D > 24576 is rejected                        */
-  int32_t keep_o_residual;     /* 1: bsa_attn_fwd also writes what the bf16 rounding
-                                  of O dropped (fp32 O - bf16 O, as bf16) into the
-                                  backward part of the workspace, which must then be
-                                  sized with_backward, and bsa_bwd_preprocess forms
-                                  Delta = rowsum(dO o (O + that residual)), exact to
-                                  fp32 O; 0: Delta from the bf16 O alone.  Both calls
-                                  must get the same value.                         */
+  int32_t o_residual;          /* BSA_O_RESIDUAL_*: the bf16 rounding residual of O
+                                  (fp32 O - bf16 O, as bf16) that makes the
+                                  backward's Delta = rowsum(dO o O) exact to the
+                                  fp32 O instead of the rounded output.  AUTO (0)
+                                  is exact whenever a backward shares the
+                                  forward's workspace; see below.              */
 } bsa_options;
+
+/* bsa_options.o_residual.
+ *   AUTO  bsa_attn_fwd writes the residual into the backward part of the
+ *         workspace when ws_bytes covers a backward (bsa_workspace_size with
+ *         with_backward = 1), and records the `out` pointer it belongs to in
+ *         the workspace header; otherwise it records none.  bsa_attn_bwd /
+ *         bsa_bwd_preprocess use the residual when the header's record names
+ *         the same `out` pointer (a check made on the device, so no
+ *         synchronisation), else Delta comes from the bf16 O.  bsa_plan_build
+ *         clears the record.  The backward assumes `out` still holds what that
+ *         forward wrote, as any attention backward does.
+ *   KEEP  as AUTO, but the forward requires a workspace sized with_backward
+ *         (else BSA_ERR_WORKSPACE_TOO_SMALL).
+ *   DROP  no residual: the forward writes none (and clears the record), the
+ *         backward takes Delta from the bf16 O.  Saves one O-sized write and
+ *         read per step; Delta then carries the output's rounding, which on
+ *         rows with very few allowed keys moves dQ / dK by up to ~1e-2. */
+#define BSA_O_RESIDUAL_AUTO 0
+#define BSA_O_RESIDUAL_KEEP 1
+#define BSA_O_RESIDUAL_DROP 2
+
 
 /* Where the plan and the scratch arrays sit inside the workspace (byte offsets),
  * for inspection and tests.  Filled by bsa_workspace_layout. */
@@ -225,7 +245,7 @@ typedef struct bsa_workspace_view {
                                   quarter of each q-block                          */
   size_t off_kbar;             /* fp32   [B, H_kv, D] k-smoothing center             */
   size_t off_qdot;             /* fp32   [B, H, Sq]   q_i . center                   */
-  size_t off_o_resid;          /* bf16   [B, Sq, H, D] O - bf16(O) (keep_o_residual)  */
+  size_t off_o_resid;          /* bf16   [B, Sq, H, D] O - bf16(O) (o_residual)       */
   int32_t nM, nN;
 } bsa_workspace_view;
 
@@ -342,20 +362,40 @@ BSA_API bsa_status bsa_bwd_convert(const bsa_problem *prob, const bsa_mask_spec 
  *    launch.
  *  - No cudaMalloc, cudaFree or other allocating call is made (the plan and the
  *    bound run one after the other on `stream`, never on the library's side
- *    stream, so no stream or event is created either).  The first call
- *    on each device looks up the array's device address (with that device
- *    current); make that first call before any stream capture.
+ *    stream, so no stream or event is created either).  The first use on each
+ *    device looks up the array's device address (with that device current),
+ *    which under lazy module loading is also when the driver loads this
+ *    library's device code and places the array: call bsa_static_scratch_init
+ *    once per device before any stream capture or allocation-free section.
+ *    The looked-up address is kept; after cudaDeviceReset on a device, this
+ *    entry point must not be used there again in the same process.
  *  - Every call shares the one array and rebuilds the plan in it, so calls
  *    whose work overlaps on the GPU (different streams, or concurrent host
  *    threads) race and must be serialised by the caller.
- *  - opt->plan_ready and opt->bound_ready are ignored.  Device-side errors land
- *    in the array's status word, which callers of this entry point cannot read;
- *    argument errors are returned as usual. */
+ *  - opt->plan_ready and opt->bound_ready are ignored, and the O residual is
+ *    never kept (no backward shares this array).  Device-side errors (a bad
+ *    cu_seqlens, a bounded wait that gave up) land in the array's sticky status
+ *    word: read it with bsa_static_scratch_status.  Argument errors are
+ *    returned as usual. */
 BSA_API bsa_status bsa_attn_fwd_static_scratch(const bsa_problem *prob,
                                                const bsa_mask_spec *mask,
                                                const bsa_options *opt, const void *q,
                                                const void *k, const void *v, void *out,
                                                float *lse, bsa_stream_t stream);
+
+/* The allocation-free forward's set-up on the current device: looks up the
+ * static array's device address (loading the library's device code there if
+ * the driver loads it lazily).  Call once per device before the first
+ * bsa_attn_fwd_static_scratch inside a stream capture or any section that must
+ * not allocate.  No counterpart in the pages.  Errors: NO_DEVICE, CUDA. */
+BSA_API bsa_status bsa_static_scratch_init(void);
+
+/* Synchronises `stream`, then returns the sticky device status of the static
+ * array bsa_attn_fwd_static_scratch uses on the current device: BSA_OK unless
+ * the most recent such call recorded a device-side error (every call rebuilds
+ * the plan in the array, which resets the word).  clear = 1 resets it.
+ * Allocates nothing.  No counterpart in the pages.  Errors: NO_DEVICE, CUDA. */
+BSA_API bsa_status bsa_static_scratch_status(bsa_stream_t stream, int32_t clear);
 
 /* Synchronises `stream`, then returns the sticky device status of `ws`
  * (BSA_OK if no device-side error was recorded); clear = 1 resets it. */

@@ -1,6 +1,19 @@
 """Helpers shared by the GPU parity tests: oracle views of a workload and the
-comparison rules (tolerances from the stated bar: max-abs 1e-2 on O/dQ/dK/dV,
-1e-3 on LSE; -inf LSE / zero O exactly where a row has no allowed key)."""
+comparison rule.
+
+The bar is the stated one, flat: max-abs <= 1e-2 on O, dQ, dK, dV and
+<= 1e-3 on LSE, element by element (-inf LSE and zero O exactly where a row has
+no allowed key).  One excuse only: outputs are bf16, and a correctly rounded
+bf16 value of an exact result of magnitude >= 4 already carries up to half a
+bf16 ulp (0.0156 in [4, 8)) of pure output rounding, so an element whose oracle
+value has |x| >= 4 passes if its error is within 1e-2 + half a bf16 ulp of that
+value.  Every excused element is recorded with its raw error.
+
+Every comparison records the raw max-abs error per output under the running
+test's id; ``tests/conftest.py`` prints the table at the end of the run (and
+writes it as JSON where ``BSA_PARITY_LOG`` names a file)."""
+
+import os
 
 import numpy as np
 import torch
@@ -9,6 +22,14 @@ import oracle
 
 O_TOL = 1e-2
 LSE_TOL = 1e-3
+EXCUSE_ABS = 4.0  # |oracle| at or above which half a bf16 ulp of output rounding is excused
+
+# {test id: {output name: {"raw": max-abs, "n": elements, "excused": [(index, oracle, error), ...]}}}
+REPORT: dict = {}
+
+
+def _test_id() -> str:
+    return os.environ.get("PYTEST_CURRENT_TEST", "?").rsplit(" (", 1)[0]
 
 
 def np64(t: torch.Tensor) -> np.ndarray:
@@ -26,53 +47,53 @@ def half_ulp_bf16(x):
     return np.ldexp(1.0, np.floor(np.log2(ax)).astype(np.int64) - 8)
 
 
-def ds_rounding_terms(wl, ds, scale):
-    """Per-element error the bf16 dS operand forces on dQ and dK.
-
-    The tensor-core backward rounds dS = P o (dP - Delta) to bf16 before the
-    contractions dQ = scale dS K and dK = scale dS^T Q, so an element of dQ
-    carries up to scale * sum_j half_ulp(dS_ij) |k_jd| from that rounding alone
-    (dK likewise with |q_id|).  Where a row has few keys, P is near 1 and |dS|
-    reaches ~10 with N(0, 1) dO, and this term is of the order of the 1e-2 bar;
-    where rows have many keys it is negligible.  Computed from the oracle's fp64
-    dS (``ds``: {(b, h): [Sq, Skv]}).  Returns (extra_dq, extra_dk)."""
-    q, k = np64(wl.q), np64(wl.k)
-    B, Sq, H, D = q.shape
-    g = H // k.shape[2]
-    eq = np.zeros_like(q)
-    ek = np.zeros_like(k)
-    for (b, h), d in ds.items():
-        u = half_ulp_bf16(d) * (d != 0)
-        eq[b, :, h, :] = scale * (u @ np.abs(k[b, :, h // g, :]))
-        ek[b, :, h // g, :] += scale * (u.T @ np.abs(q[b, :, h, :]))
-    return eq, ek
+def _record(name: str, raw: float, n: int, excused=()):
+    ent = REPORT.setdefault(_test_id(), {})
+    key, i = name, 2
+    while key in ent:  # the same output checked twice in one test
+        key, i = f"{name}#{i}", i + 1
+    ent[key] = {"raw": raw, "n": int(n), "excused": list(excused)}
 
 
-def excess(x_gpu, ref, tol=O_TOL, extra=0.0):
-    """max over elements of |x_gpu - ref| - (tol + half_ulp_bf16(ref)); <= 0 passes.
+def check(name: str, x_gpu, ref, tol: float = O_TOL) -> float:
+    """Raw max |x_gpu - ref| over all elements; asserts the flat bar.
 
-    The stated bar is max-abs <= tol; outputs are bf16, so an element whose exact
-    value is large carries up to half a bf16 ulp of pure output rounding (0.0078
-    for |x| in [2, 4)), which the bar is not meant to absorb."""
-    a = np64(x_gpu) if isinstance(x_gpu, torch.Tensor) else x_gpu
-    return float(np.max(np.abs(a - ref) - (tol + half_ulp_bf16(ref) + extra)))
+    An element fails when its error exceeds ``tol``, unless |ref| >= 4 and the
+    error is within tol + half a bf16 ulp of ref (output rounding; listed in the
+    report).  NaN anywhere fails."""
+    a = np64(x_gpu) if isinstance(x_gpu, torch.Tensor) else np.asarray(x_gpu, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert a.shape == ref.shape, (name, a.shape, ref.shape)
+    err = np.abs(a - ref)
+    assert not np.isnan(err).any(), f"{name}: NaN in the comparison"
+    raw = float(err.max()) if err.size else 0.0
+    over = err > tol
+    excusable = over & (np.abs(ref) >= EXCUSE_ABS) & (err <= tol + half_ulp_bf16(ref))
+    bad = over & ~excusable
+    idx = np.argwhere(excusable)
+    excused = [(tuple(int(v) for v in ix), float(ref[tuple(ix)]), float(err[tuple(ix)])) for ix in idx[:50]]
+    _record(name, raw, err.size, excused)
+    if bad.any():
+        first = tuple(int(v) for v in np.argwhere(bad)[0])
+        raise AssertionError(
+            f"{name}: max-abs {raw:.5f} > {tol} on {int(bad.sum())} element(s) not excused by output "
+            f"rounding; first at {first}: gpu {a[first]:.6f} oracle {ref[first]:.6f}")
+    return raw
 
 
-def compare_out(o_gpu, o_ref, rows=None, tol=O_TOL):
-    """Raw max |O_gpu - O_ref| over the given rows (all rows if None); raises if
-    any element breaks the ulp-aware bar of :func:`excess`."""
+def compare_out(o_gpu, o_ref, rows=None, tol=O_TOL, name="O"):
+    """Raw max |O_gpu - O_ref| over the given rows (all rows if None), checked
+    against the flat bar by :func:`check`."""
     a = np64(o_gpu)
     if rows is not None:
         a = a[:, rows]
         o_ref = o_ref[:, rows]
-    ex = excess(a, o_ref, tol)
-    raw = float(np.max(np.abs(a - o_ref)))
-    assert ex <= 0.0, f"max-abs {raw:.5f} exceeds {tol} + half a bf16 ulp by {ex:.5f}"
-    return min(raw, tol)
+    return check(name, a, o_ref, tol)
 
 
-def compare_lse(l_gpu, l_ref, rows=None):
-    """(max |LSE_gpu - LSE_ref| over finite entries, -inf pattern equal)."""
+def compare_lse(l_gpu, l_ref, rows=None, name="LSE"):
+    """(max |LSE_gpu - LSE_ref| over finite entries, -inf pattern equal); the
+    error is recorded, the caller asserts it against LSE_TOL."""
     a = l_gpu.detach().cpu().numpy().astype(np.float64)
     if rows is not None:
         a = a[..., rows]
@@ -80,6 +101,7 @@ def compare_lse(l_gpu, l_ref, rows=None):
     fin = np.isfinite(l_ref)
     same = bool(np.array_equal(fin, np.isfinite(a)) and np.all(np.isneginf(a[~fin])))
     err = float(np.max(np.abs(a[fin] - l_ref[fin]))) if fin.any() else 0.0
+    _record(name, err, int(fin.sum()))
     return err, same
 
 

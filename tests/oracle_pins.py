@@ -1,6 +1,6 @@
-"""Pins for the fp64 oracle: each returns an error figure, so that the pin tests
-and the planted-mistake tests (which feed these a deliberately broken oracle)
-share one definition.  Nothing here re-types the oracle's formulas: every pin
+"""Helpers of the pins for the fp64 oracle (tests/test_oracle_pins.py; the
+planted-mistake tests in tests/test_oracle_planted.py run those pins against a
+deliberately broken oracle).  Nothing here re-types the oracle's formulas: every pin
 compares it with something else fixed by the pages or by mathematics (a scalar
 brute force, a library routine, autograd, finite differences, closed forms)."""
 

@@ -48,7 +48,7 @@ int main(void) {
   P(bsa_mask_spec, seg_q) P(bsa_mask_spec, cu_seqlens) P(bsa_mask_spec, n_align_tail)
   P(bsa_mask_spec, prefix_len) P(bsa_mask_spec, dilation)
   P(bsa_options, kmax_override) P(bsa_options, perm) P(bsa_options, sem_timeout_ns) P(bsa_options, plan_ready)
-  P(bsa_options, bound_mode) P(bsa_options, keep_o_residual) P(bsa_workspace_view, off_qdot)
+  P(bsa_options, bound_mode) P(bsa_options, o_residual) P(bsa_workspace_view, off_qdot)
   P(bsa_workspace_view, off_o_resid) P(bsa_problem, H_kv)
   P(bsa_workspace_view, off_sem) P(bsa_workspace_view, nN)
   return 0;
@@ -79,7 +79,7 @@ def test_ctypes_structs_match_c_layout():
     assert c["bsa_mask_spec.dilation"] == bd.MaskSpec.dilation.offset
     assert c["bsa_options.bound_mode"] == bd.Options.bound_mode.offset
     assert c["bsa_workspace_view.off_qdot"] == bd.WorkspaceView.off_qdot.offset
-    assert c["bsa_options.keep_o_residual"] == bd.Options.keep_o_residual.offset
+    assert c["bsa_options.o_residual"] == bd.Options.o_residual.offset
     assert c["bsa_workspace_view.off_o_resid"] == bd.WorkspaceView.off_o_resid.offset
     assert c["bsa_problem.H_kv"] == bd.Problem.H_kv.offset
     assert c["bsa_options.kmax_override"] == bd.Options.kmax_override.offset
@@ -219,9 +219,14 @@ def test_calls_reject_bad_arguments_before_cuda(L):
     o.kmax_override = None
     wide = _prob(H=200, D=128)                      # centers of 200 heads exceed shared memory
     assert L.bsa_plan_build(ctypes.byref(wide), None, ctypes.byref(o), 4096, 1 << 40, None) == 2
-    # keeping the O residual needs the backward-sized workspace
+    # an unknown O-residual mode; KEEP needs the backward-sized workspace, AUTO
+    # and DROP do not
     o = bd.Options()
-    o.keep_o_residual = 1
+    o.o_residual = 3
+    assert L.bsa_plan_build(ctypes.byref(p), None, ctypes.byref(o), 4096, 1 << 30, None) == 1
+    o.o_residual = -1
+    assert L.bsa_plan_build(ctypes.byref(p), None, ctypes.byref(o), 4096, 1 << 30, None) == 1
+    o.o_residual = bd.O_RESIDUAL["keep"]
     fwd_only = _size(L, p, bwd=0)[1]
     assert L.bsa_plan_build(ctypes.byref(p), None, ctypes.byref(o), 4096, fwd_only, None) == 3
     # workspace too small

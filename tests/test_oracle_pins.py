@@ -381,3 +381,31 @@ def test_key_permutation_with_mask_leaves_output():
 def test_useful_flops_per_tile():
     assert oracle.useful_flops(1, 128) == 4 * 128 * 128 * 128
     assert oracle.useful_flops(2, 64, backward=True) == 2.5 * 2 * 4 * 128 * 128 * 64
+
+
+def test_valid_keys_of_varlen_exclude_the_alignment_tail():
+    """The fixed-m bound's kmax runs over the keys a real row can see: with
+    cu_seqlens the keys of the trailing alignment segments never enter it.
+    Alignment keys scaled x100 dominate every norm; kmax must still be the
+    largest norm among the real segments' keys, a closed form taken straight
+    from the cu_seqlens boundaries; with no alignment tail it is the largest
+    norm over all keys.  Padding (kv_valid_len) and varlen together: the
+    smaller of the two boundaries."""
+    rng = np.random.default_rng(41)
+    T, H, D = 90, 2, 8
+    cu = np.array([0, 30, 70, 78, 90])
+    q = rng.standard_normal((1, T, H, D))
+    k = rng.standard_normal((1, T, H, D))
+    k[0, 70:] *= 100.0  # the two alignment segments [70, 78) and [78, 90)
+    for tail, real_end in ((2, 70), (1, 78), (0, 90)):
+        m = MaskDesc(cu_seqlens=cu, n_align_tail=tail)
+        kmax, _, _, _ = oracle.fixed_m_bound(q, k, m, SCALE)
+        for h in range(H):
+            assert kmax[0, h] == np.linalg.norm(k[0, :real_end, h], axis=1).max()
+        vk = oracle.valid_keys(m, 0, T)
+        assert vk[:real_end].all() and not vk[real_end:].any()
+    m = MaskDesc(cu_seqlens=cu, n_align_tail=1, kv_valid_len=np.array([50]))
+    kmax, _, _, _ = oracle.fixed_m_bound(q, k, m, SCALE)
+    assert kmax[0, 0] == np.linalg.norm(k[0, :50, 0], axis=1).max()
+    kbar, radius, _, _, _ = oracle.fixed_m_bound_smoothed(q, k, MaskDesc(cu_seqlens=cu, n_align_tail=2), SCALE)
+    assert np.allclose(kbar[0, 1], k[0, :70, 1].mean(axis=0), atol=1e-13)
