@@ -33,7 +33,7 @@ STATUS = {
     0: "BSA_OK", 1: "BSA_ERR_INVALID_ARG", 2: "BSA_ERR_UNSUPPORTED",
     3: "BSA_ERR_WORKSPACE_TOO_SMALL", 4: "BSA_ERR_CUDA", 5: "BSA_ERR_SEM_TIMEOUT",
     6: "BSA_ERR_PLAN_MISMATCH", 7: "BSA_ERR_BAD_MASK_DATA", 8: "BSA_WARN_GATE_VIOLATION",
-    9: "BSA_ERR_NO_DEVICE",
+    9: "BSA_ERR_NO_DEVICE", 10: "BSA_ERR_INPUT_RANGE",
 }
 
 

@@ -679,6 +679,8 @@ const char *bsa_status_string(bsa_status status) {
     case BSA_ERR_BAD_MASK_DATA: return "cu_seqlens is not a non-decreasing [0 .. Sq] sequence";
     case BSA_WARN_GATE_VIOLATION: return "a gated fixed-m row summed below 2^-100";
     case BSA_ERR_NO_DEVICE: return "no sm_100 device is current";
+    case BSA_ERR_INPUT_RANGE:
+      return "a backward input or dS entry lies beyond the fp16 range or is not finite";
   }
   return "unknown status";
 }

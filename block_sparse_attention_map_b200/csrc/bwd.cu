@@ -83,7 +83,8 @@ struct BwdSmem {
                        bSFull = bDOEmpty + NDO, bDPFull = bSFull + 1, bPReady = bDPFull + 1,
                        bDSReady = bPReady + 1, bDSFree = bDSReady + 1, bDQFull = bDSFree + 1,
                        bDQFree = bDQFull + 1, bDKVFull = bDQFree + 1, bDKVFree = bDKVFull + 1,
-                       bVecReady = bDKVFree + 1, bFinal = bVecReady + 2,
+                       bVecReady = bDKVFree + 1, bQConv = bVecReady + 2, bDOConv = bQConv + NQ,
+                       bKConv = bDOConv + NDO, bVConv = bKConv + 1, bFinal = bVConv + 1,
                        kNumBars = bFinal + 1;
   static constexpr int kMisc = kBar + kNumBars * 8;
   static constexpr int kAlloc = kMisc + 16;
@@ -91,8 +92,9 @@ struct BwdSmem {
 
 constexpr int kThreads = 512;
 constexpr int kLaunchRegs = 65536 / kThreads;  // 128: the whole register file
-constexpr int kConsumersPerTicket = 1 + 8 + 4;  // MMA lane, compute warps, dQ warps
+constexpr int kConsumersPerTicket = 1 + 8 + 4 + 2;  // MMA lane, compute warps, dQ warps, converters
 constexpr int kComputeThreads = 256;
+constexpr int kConvThreads = 64;  // warps 2 and 3
 
 __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity) {
   const uint32_t a = smem_u32(bar);
@@ -173,6 +175,7 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
           i == L::bVecReady + 1)
         cnt = kComputeThreads;
       if (i == L::bDQFree) cnt = 128;
+      if ((i >= L::bQConv && i < L::bKConv) || i == L::bKConv || i == L::bVConv) cnt = kConvThreads;
       mbar_init(&bars[i], cnt);
     }
     *abort_flag = 0;
@@ -210,9 +213,11 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
   pdl_trigger();
 
   const uint32_t T_S = tmem, T_DP = tmem + 128, T_DV = tmem + 256, T_DK = tmem + 256 + D;
-  constexpr uint32_t kIdS = idesc_bf16_f32(128, 128, 0, 0);      // S^T, dP^T: both K-major
-  constexpr uint32_t kIdKV = idesc_bf16_f32(128, D, 0, 1);       // dV (TS), dK: B MN-major
-  constexpr uint32_t kIdQ = idesc_bf16_f32(128, D, 1, 1);        // dQ: A and B MN-major
+  // every operand is fp16: Q, K, V, dO converted in shared memory by the
+  // converter warps, P^T and dS^T written as fp16 by the compute warps
+  constexpr uint32_t kIdS = idesc_f16_f32(128, 128, 0, 0);      // S^T, dP^T: both K-major
+  constexpr uint32_t kIdKV = idesc_f16_f32(128, D, 0, 1);       // dV (TS), dK: B MN-major
+  constexpr uint32_t kIdQ = idesc_f16_f32(128, D, 1, 1);        // dQ: A and B MN-major
 
   // register budgets, set first thing in each warpgroup's branch: 96 for the
   // producer / MMA warpgroup, 128 for each compute warpgroup, 160 for the dQ
@@ -296,7 +301,7 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       const uint32_t ds_addr = smem_u32(sm + L::kDS);
       auto issue_s = [&](uint32_t e_idx) -> bool {  // S^T = K_n Q_m^T
         const uint32_t qs = e_idx % NQ;
-        if (!wd.wait(&bars[L::bQFull + qs], (e_idx / NQ) & 1)) return false;
+        if (!wd.wait(&bars[L::bQConv + qs], (e_idx / NQ) & 1)) return false;
         tc_fence_after();
         const uint32_t q_addr = smem_u32(sm + L::kQ + qs * kTB);
 #pragma unroll
@@ -310,7 +315,7 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       };
       auto issue_dp = [&](uint32_t e_idx) -> bool {  // dP^T = V_n dO_m^T
         const uint32_t ds = e_idx % NDO;
-        if (!wd.wait(&bars[L::bDOFull + ds], (e_idx / NDO) & 1)) return false;
+        if (!wd.wait(&bars[L::bDOConv + ds], (e_idx / NDO) & 1)) return false;
         // the dQ of the previous entry occupies these columns until read out
         if (e_idx >= 1 && !wd.wait(&bars[L::bDQFree], (e_idx - 1) & 1)) return false;
         tc_fence_after();
@@ -335,9 +340,9 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
         const int kb = cc & 1, vb = kb ^ 1;
         k_addr = smem_u32(sm + L::kK + kb * kTB);
         v_addr = smem_u32(sm + L::kK + vb * kTB);
-        if (!wd.wait(&bars[L::bKFull], cc & 1)) break;
+        if (!wd.wait(&bars[L::bKConv], cc & 1)) break;
         bool stop = !issue_s(ec);
-        if (!stop && !wd.wait(&bars[L::bVFull], cc & 1)) stop = true;
+        if (!stop && !wd.wait(&bars[L::bVConv], cc & 1)) stop = true;
         if (!stop && !issue_dp(ec)) stop = true;
         // V's last use is the column's last dP^T: its buffer takes the next K
         if (!stop && k.tot == 1) mma_commit(&bars[L::bXFree + vb]);
@@ -394,6 +399,76 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       mma_commit(&bars[L::bFinal]);
       drain_wait(&bars[L::bFinal], 0);
     }
+    } else if (run) {
+    // ------------------------------------------------------------ converters (warps 2, 3)
+    // Every tile the MMAs read (Q_m and dO_m per entry, K_n and V_n per column)
+    // is turned from bf16 into fp16 in place as soon as its copy lands, in the
+    // producer's order: the products then take P and dS at fp16's 11
+    // significant bits instead of bf16's 8.  Values of an input beyond the
+    // fp16 range are clamped and reported as BSA_ERR_INPUT_RANGE.
+    const int ct = threadIdx.x - 64;  // 0 .. 63
+    auto wwait = [&](uint64_t *bar, uint32_t parity) {
+      return __all_sync(0xffffffffu, wd.wait(bar, parity)) != 0;
+    };
+    uint32_t in_max = 0;  // per 16-bit half: the largest |x| bit pattern seen
+    auto convert = [&](uint8_t *tile, uint64_t *done) {
+      constexpr int kChunks = kTB / 16;            // 16-byte pieces of the tile
+      constexpr int kPer = kChunks / kConvThreads;  // per thread
+      constexpr int kBatch = 8;
+      static_assert(kPer % kBatch == 0, "converter batches");
+      int4 *t4 = reinterpret_cast<int4 *>(tile);
+#pragma unroll 1
+      for (int i0 = 0; i0 < kPer; i0 += kBatch) {
+        int4 v[kBatch];
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) v[u] = t4[(i0 + u) * kConvThreads + ct];
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+          uint32_t w[4] = {static_cast<uint32_t>(v[u].x), static_cast<uint32_t>(v[u].y),
+                           static_cast<uint32_t>(v[u].z), static_cast<uint32_t>(v[u].w)};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            in_max = __vmaxu2(in_max, w[q] & 0x7fff7fffu);
+            w[q] = bf16x2_to_f16x2(w[q]);
+          }
+          t4[(i0 + u) * kConvThreads + ct] = make_int4(w[0], w[1], w[2], w[3]);
+        }
+      }
+      fence_proxy_async_smem();  // the MMAs read the tile through the async proxy
+      mbar_arrive(done);
+    };
+    uint32_t tc = 0, cc = 0, ec = 0;
+    bool stop = false;
+    for (;; ++tc) {
+      const uint32_t slot = tc & 1;
+      if (!wwait(&bars[L::bTkFull + slot], (tc >> 1) & 1)) break;
+      const int t = tk_ring[slot];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[L::bTkEmpty + slot]);
+      const Ticket k = decode_ticket(p, t);
+      if (!k.valid) break;
+      if (k.ee == k.es) continue;
+      for (int x = 0; x < k.tot; ++x, ++ec) {
+        const uint32_t qs = ec % NQ, ds = ec % NDO;
+        if (!wwait(&bars[L::bQFull + qs], (ec / NQ) & 1)) { stop = true; break; }
+        convert(sm + L::kQ + qs * kTB, &bars[L::bQConv + qs]);
+        if (x == 0) {
+          const int kb = cc & 1, vb = kb ^ 1;
+          if (!wwait(&bars[L::bKFull], cc & 1)) { stop = true; break; }
+          convert(sm + L::kK + kb * kTB, &bars[L::bKConv]);
+          if (!wwait(&bars[L::bVFull], cc & 1)) { stop = true; break; }
+          convert(sm + L::kK + vb * kTB, &bars[L::bVConv]);
+        }
+        if (!wwait(&bars[L::bDOFull + ds], (ec / NDO) & 1)) { stop = true; break; }
+        convert(sm + L::kDO + ds * kTB, &bars[L::bDOConv + ds]);
+      }
+      if (stop) break;
+      ++cc;
+    }
+    // |x| >= 65536 (bf16 bits 0x4780; bf16 has no value in (65280, 65536)),
+    // infinities and NaNs: beyond what fp16 holds
+    if ((in_max & 0xffffu) >= 0x4780u || (in_max >> 16) >= 0x4780u)
+      record_status(p.hdr + kHdrStatus, BSA_ERR_INPUT_RANGE);
     }
   } else if (warp < 12) {
     if (run) {
@@ -413,6 +488,7 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
     // own S^T columns, which only this warp reads
     const uint32_t t_p = T_S + lane_off + 64 * half;
     uint32_t tc = 0, cc = 0, ec = 0;
+    uint32_t ds_max = 0;  // per 16-bit half: the largest |dS| fp16 bit pattern written
     bool stop = false;
     for (;; ++tc) {
       const uint32_t slot = tc & 1;
@@ -524,10 +600,9 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
         if (!wwait(&bars[L::bVecReady + (ec & 1)], (ec >> 1) & 1)) { stop = true; break; }
         const float4 *nl4p = reinterpret_cast<const float4 *>(vec_nl + (ec & 1) * kTile + 64 * half);
         const float4 *nd4p = reinterpret_cast<const float4 *>(vec_nd + (ec & 1) * kTile + 64 * half);
-        // phase 1: P^T = exp2(S^T * scale * log2e - LSE*log2e) -> bf16 in TMEM
-        // (the A operand of dV) and kept in registers as fp16 pairs for dS: P
-        // lies in [0, 1], where fp16 keeps 11 significant bits to bf16's 8, so
-        // dS carries no extra rounding of P
+        // phase 1: P^T = exp2(S^T * scale * log2e - LSE*log2e) -> fp16 in TMEM
+        // (the A operand of dV) and kept in registers for dS: P lies in [0, 1],
+        // where fp16 keeps 11 significant bits to bf16's 8
         if (!wwait(&bars[L::bSFull], ec & 1)) { stop = true; break; }
         tc_fence_after();
         uint32_t pk[32];
@@ -556,19 +631,20 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
                 p0 = ((bits >> e0) & 1u) ? p0 : 0.f;
                 p1 = ((bits >> (e0 + 1)) & 1u) ? p1 : 0.f;
               }
-              pb[e0 >> 1] = pack_bf16x2(p0, p1);
-              pk[8 * sc + (e0 >> 1)] = pack_f16x2(p0, p1);
+              pb[e0 >> 1] = pack_f16x2(p0, p1);
             }
           }
-          // P^T piece -> TMEM columns [8sc, 8sc+8) of this half's region: S^T
-          // columns this warp has already read
+#pragma unroll
+          for (int q = 0; q < 8; ++q) pk[8 * sc + q] = pb[q];
+          // P^T piece (fp16) -> TMEM columns [8sc, 8sc+8) of this half's
+          // region: S^T columns this warp has already read
           tmem_st8(t_p + 8 * sc, pb);
           if (sc + 1 < 4) tmem_wait_ld();
         }
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&bars[L::bPReady]);
-        // phase 2: dS^T = P^T o (dP^T - Delta) in fp32 from the fp16 P^T -> bf16,
+        // phase 2: dS^T = P^T o (dP^T - Delta) in fp32 from the fp16 P^T -> fp16,
         // into the shared tile (128-byte swizzle, K-major; the dQ MMA reads it
         // MN-major) and into TMEM over this half's dP^T columns, already read
         // (the A operand of dK, laid out like P^T for dV)
@@ -596,7 +672,8 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
               const float2 dd = __fadd2_rn(
                   make_float2(__uint_as_float(dp[e0]), __uint_as_float(dp[e0 + 1])), nd);
               const float2 dsv = __fmul2_rn(pv, dd);
-              dk2[e0 >> 1] = pack_bf16x2(dsv.x, dsv.y);
+              dk2[e0 >> 1] = pack_f16x2_sat(dsv.x, dsv.y);
+              ds_max = __vmaxu2(ds_max, dk2[e0 >> 1] & 0x7fff7fffu);
             }
           }
 #pragma unroll
@@ -669,6 +746,9 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       }
       ++cc;
     }
+    // a dS clamped at the fp16 limit 65504 (0x7bff): reported, not silent
+    if ((ds_max & 0xffffu) >= 0x7bffu || (ds_max >> 16) >= 0x7bffu)
+      record_status(p.hdr + kHdrStatus, BSA_ERR_INPUT_RANGE);
     }
   } else {
     regs_inc<160>();

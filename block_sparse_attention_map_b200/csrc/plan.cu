@@ -164,63 +164,78 @@ __device__ __forceinline__ bool allowed_elem(const ClassifyArgs &a, int b, int i
 }
 
 // Exact class of tile (b, m, n) by the whole warp, element by element: lane l
-// takes columns l, l+32, l+64, l+96 of the tile and walks its rows.
+// takes columns l, l+32, l+64, l+96 of the tile and the warp walks the rows
+// from both ends inwards (first, last, second, second-to-last, ...), stopping
+// as soon as it has seen one allowed and one masked element (the tile is
+// PARTIAL then, whatever the remaining rows hold): most tiles the bounds leave
+// open settle within their first rows, including those whose rows change
+// segment near one end (a varlen alignment tail, a document boundary).
 __device__ uint8_t refine_tile(const ClassifyArgs &a, int b, int m, int n, int lane) {
   const int i0 = m * kTile, i1 = min(a.Sq, i0 + kTile) - 1;
   const int P = a.prefix_len != nullptr ? a.prefix_len[b] : 0;
-  const int L = (a.flags & BSA_MASK_KV_VALID_LEN) ? a.kv_valid_len[b] : a.Skv;
+  const int L = min((a.flags & BSA_MASK_KV_VALID_LEN) ? a.kv_valid_len[b] : a.Skv, a.Skv);
   bool any = false, all = true;
+  int jj[4], sj[4];
+  bool in[4];
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    jj[c] = n * kTile + lane + 32 * c;
+    in[c] = jj[c] < a.Skv;
+    if (!in[c]) all = false;
+    sj[c] = (a.seg_kv != nullptr && in[c]) ? a.seg_kv[b * a.seg_kv_bstride + jj[c]] : 0;
+  }
+  const int rows = i1 - i0 + 1;
 #pragma unroll 1
-  for (int t = lane; t < kTile; t += 32) {
-    const int j = n * kTile + t;
-    if (j >= a.Skv) {
-      all = false;
-      continue;
-    }
-    const int seg_j = a.seg_kv != nullptr ? a.seg_kv[b * a.seg_kv_bstride + j] : 0;
-#pragma unroll 1
-    for (int i = i0; i <= i1; ++i) {
-      const int seg_i = a.seg_q != nullptr ? a.seg_q[b * a.seg_q_bstride + i] : 0;
-      const bool ok = allowed_elem(a, b, i, j, seg_i, seg_j, P, min(L, a.Skv));
+  for (int k = 0; k < rows; ++k) {
+    const int i = (k & 1) ? i1 - (k >> 1) : i0 + (k >> 1);
+    const int seg_i = a.seg_q != nullptr ? a.seg_q[b * a.seg_q_bstride + i] : 0;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      if (!in[c]) continue;
+      const bool ok = allowed_elem(a, b, i, jj[c], seg_i, sj[c], P, L);
       any |= ok;
       all &= ok;
     }
+    // k runs over the same rows in every lane: the votes are warp-uniform
+    if ((k & 3) == 3 && __any_sync(0xffffffffu, any) && !__all_sync(0xffffffffu, all))
+      return BSA_TILE_PARTIAL;
   }
   any = __any_sync(0xffffffffu, any);
   all = __all_sync(0xffffffffu, all);
   return all ? BSA_TILE_FULL : (any ? BSA_TILE_PARTIAL : BSA_TILE_EMPTY);
 }
 
-// One warp per (b, m): classify the row of tiles (tiles the bounds cannot
-// settle are classified element by element by the whole warp), count its
-// non-empty tiles and add each non-empty tile to its column's count (an
-// order-independent sum).
-__global__ void k_classify_rows(ClassifyArgs a) {
-  const int wid = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+// One warp per (b, m, 32 consecutive columns): classify those tiles (tiles the
+// bounds cannot settle are classified element by element by the whole warp),
+// and add the non-empty ones to their row's and columns' counts (zeroed
+// before; order-independent integer sums).  A row with many tiles to refine
+// (the boundary block of a varlen alignment tail meets every column) spreads
+// over as many warps as it has column chunks.
+__global__ void k_classify_chunks(ClassifyArgs a) {
+  const int64_t wid = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
-  if (wid >= a.B * a.nM) return;
-  const int b = wid / a.nM, m = wid % a.nM;
-  uint8_t *row = a.cls + static_cast<int64_t>(wid) * a.nN;
-  int cnt = 0;
-  for (int n0 = 0; n0 < a.nN; n0 += 32) {
-    const int n = n0 + lane;
-    uint8_t c = BSA_TILE_EMPTY;
-    bool exact = true;
-    if (n < a.nN) c = tile_class(a, b, m, n, &exact);
-    uint32_t todo = __ballot_sync(0xffffffffu, c == BSA_TILE_PARTIAL && !exact);
-    while (todo != 0u) {
-      const int src = __ffs(todo) - 1;
-      todo &= todo - 1u;
-      const uint8_t rc = refine_tile(a, b, m, n0 + src, lane);
-      if (lane == src) c = rc;
-    }
-    if (n < a.nN) {
-      row[n] = c;
-      if (c != BSA_TILE_EMPTY) atomicAdd(a.col_cnt + b * a.nN + n, 1);
-    }
-    cnt += __popc(__ballot_sync(0xffffffffu, c != BSA_TILE_EMPTY));
+  const int chunks = (a.nN + 31) >> 5;
+  if (wid >= static_cast<int64_t>(a.B) * a.nM * chunks) return;
+  const int row_id = static_cast<int>(wid / chunks), n0 = static_cast<int>(wid % chunks) * 32;
+  const int b = row_id / a.nM, m = row_id % a.nM;
+  uint8_t *row = a.cls + static_cast<int64_t>(row_id) * a.nN;
+  const int n = n0 + lane;
+  uint8_t c = BSA_TILE_EMPTY;
+  bool exact = true;
+  if (n < a.nN) c = tile_class(a, b, m, n, &exact);
+  uint32_t todo = __ballot_sync(0xffffffffu, c == BSA_TILE_PARTIAL && !exact);
+  while (todo != 0u) {
+    const int src = __ffs(todo) - 1;
+    todo &= todo - 1u;
+    const uint8_t rc = refine_tile(a, b, m, n0 + src, lane);
+    if (lane == src) c = rc;
   }
-  if (lane == 0) a.row_cnt[wid] = cnt;
+  if (n < a.nN) {
+    row[n] = c;
+    if (c != BSA_TILE_EMPTY) atomicAdd(a.col_cnt + b * a.nN + n, 1);
+  }
+  const int cnt = __popc(__ballot_sync(0xffffffffu, c != BSA_TILE_EMPTY));
+  if (lane == 0 && cnt != 0) atomicAdd(a.row_cnt + row_id, cnt);
 }
 
 // Exclusive scans of row and column counts into CSR offsets (block 0: rows,
@@ -792,6 +807,8 @@ cudaError_t launch_plan(const bsa_problem &p, const bsa_mask_spec &m, const bsa_
   int32_t *perm = reinterpret_cast<int32_t *>(ws + L.perm);
   e = cudaMemsetAsync(col_cnt, 0, sizeof(int32_t) * B * nN, s);
   if (e != cudaSuccess) return e;
+  e = cudaMemsetAsync(row_cnt, 0, sizeof(int32_t) * B * nM, s);
+  if (e != cudaSuccess) return e;
   if (o.bwd_order == BSA_ORDER_PERM) {
     e = cudaMemcpyAsync(perm, o.perm, sizeof(int32_t) * nN, cudaMemcpyHostToDevice, s);
     if (e != cudaSuccess) return e;
@@ -812,7 +829,7 @@ cudaError_t launch_plan(const bsa_problem &p, const bsa_mask_spec &m, const bsa_
   ca.cls = ws + L.tile_class;
   ca.row_cnt = row_cnt;
   ca.col_cnt = col_cnt;
-  k_classify_rows<<<cdiv(static_cast<int64_t>(B) * nM * 32, 256), 256, 0, s>>>(ca);
+  k_classify_chunks<<<cdiv(static_cast<int64_t>(B) * nM * ((nN + 31) / 32) * 32, 256), 256, 0, s>>>(ca);
   k_scan2<<<2, 1024, 0, s>>>(row_cnt, row_ptr, B * nM, col_cnt, col_ptr, B * nN, hdr, B, p.Sq,
                              p.Skv, m.flags, m.window, o.bwd_order, m.n_seqs,
                              static_cast<uint32_t>(m.dilation));

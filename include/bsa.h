@@ -74,7 +74,11 @@ typedef enum bsa_status {
   BSA_ERR_PLAN_MISMATCH = 6,       /* device: workspace plan built for another problem */
   BSA_ERR_BAD_MASK_DATA = 7,       /* device: cu_seqlens not [0 .. Sq] non-decreasing */
   BSA_WARN_GATE_VIOLATION = 8,     /* device: a gated fixed-m row summed below 2^-100 */
-  BSA_ERR_NO_DEVICE = 9            /* no sm_100 device current                        */
+  BSA_ERR_NO_DEVICE = 9,           /* no sm_100 device current                        */
+  BSA_ERR_INPUT_RANGE = 10         /* device: a backward input (Q, K, V, dO) or an
+                                      entry of dS lies beyond the fp16 range
+                                      (|x| >= 65504) or is not finite; the
+                                      backward takes its products in fp16 */
 } bsa_status;
 
 /* Block-map tile edge (rows and keys). */

@@ -8,6 +8,8 @@ Contents
 --------
 ``attention``  dense masked softmax attention, its analytic gradient, the fixed-m
                form and the fixed-m bound / per-head gate (plain and k-smoothed).
+``bound``      the fixed-m bound per q-block (the reading taken for the pages'
+               per-segment kmax): key norms over the kv blocks a q-block reaches.
 ``blockmap``   the tile classification (EMPTY / PARTIAL / FULL) of a dense mask,
                the kv-column orders, ``rank(m, n)``, the rank-sorted column lists
                and a discrete simulation of the dQ semaphore protocol.
@@ -28,6 +30,7 @@ from .attention import (  # noqa: F401
     fixed_m_bound_smoothed,
     useful_flops,
 )
+from .bound import fixed_m_bound_blocks, row_references_blocks  # noqa: F401
 from .blockmap import (  # noqa: F401
     EMPTY,
     PARTIAL,

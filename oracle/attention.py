@@ -245,7 +245,7 @@ def attention_backward(q, k, v, dO, mask: MaskDesc, scale: float, chunk: int = 1
 
 def attention_forward_fixed_m(q, k, v, mask: MaskDesc, scale: float, kmax=None,
                               rows=None, heads=None, batches=None, chunk: int = 1024,
-                              kbar=None):
+                              kbar=None, m_rows=None):
     """The fixed-m form ("Fixed-m softmax ...", introduction).
 
     Instead of the row max, each query's reference is pinned before streaming to
@@ -260,13 +260,17 @@ def attention_forward_fixed_m(q, k, v, mask: MaskDesc, scale: float, kmax=None,
     :func:`fixed_m_bound_smoothed`) ``kmax`` is the radius max_j ||k_j - kbar||
     and the pinned reference is m_i = scale * (q_i . kbar + ||q_i|| * kmax),
     again an upper bound of every s_ij by Cauchy-Schwarz on k_j - kbar.
+
+    ``m_rows`` [B, H, Sq], when given, is each row's pinned reference itself
+    (e.g. the per q-block bound of :mod:`oracle.bound`); ``kmax`` and ``kbar``
+    are then unused.
     """
     q, k, v = _as64(q), _as64(k), _as64(v)
     B, Sq, H, D = q.shape
     Skv = k.shape[1]
-    if kmax is None:
+    if kmax is None and m_rows is None:
         kmax = fixed_m_bound(q, k, mask, scale)[0]
-    kmax = _as64(kmax)
+    kmax = _as64(kmax) if m_rows is None else None
     kvh = kv_head_of(H, k.shape[2])
     rows = np.arange(Sq) if rows is None else np.asarray(rows)
     heads = range(H) if heads is None else heads
@@ -279,9 +283,12 @@ def attention_forward_fixed_m(q, k, v, mask: MaskDesc, scale: float, kmax=None,
             has = a.any(axis=1)
             for h in heads:
                 qr = q[b, r, h, :]
-                m = scale * np.sqrt((qr * qr).sum(axis=1)) * kmax[b, h]
-                if kbar is not None:
-                    m = m + scale * (qr @ _as64(kbar)[b, h])
+                if m_rows is not None:
+                    m = _as64(m_rows)[b, h, r]
+                else:
+                    m = scale * np.sqrt((qr * qr).sum(axis=1)) * kmax[b, h]
+                    if kbar is not None:
+                        m = m + scale * (qr @ _as64(kbar)[b, h])
                 s = scale * (qr @ k[b, :, kvh(h), :].T)
                 e = np.where(a, np.exp(s - m[:, None]), 0.0)
                 l = e.sum(axis=1)

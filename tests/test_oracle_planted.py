@@ -112,3 +112,31 @@ def test_a_wrong_key_index_in_the_segment_mask_is_caught(monkeypatch):
 
     monkeypatch.setattr(A, "allowed_rows", broken)
     _must_fail(pins.test_forward_matches_brute_force, "segments")
+
+
+def test_a_block_bound_over_the_diagonal_block_only_is_caught(monkeypatch):
+    # kmax of q-block m taken over kv block m alone instead of every block its
+    # rows reach: a window row whose allowed keys lie in earlier blocks is no
+    # longer bounded
+    import oracle.bound as Bd
+
+    def broken(q, k, mask, scale, gate_limit=64.0, tile=128):
+        q, k = A._as64(q), A._as64(k)
+        B, Sq, H, D = q.shape
+        nM = -(-Sq // tile)
+        kmax = np.zeros((B, H, nM))
+        qmax = np.zeros((B, H, nM))
+        for b in range(B):
+            for h in range(H):
+                kn = np.sqrt((k[b, :, h] ** 2).sum(axis=1))
+                qn = np.sqrt((q[b, :, h] ** 2).sum(axis=1))
+                for m in range(nM):
+                    kmax[b, h, m] = kn[m * tile:(m + 1) * tile].max() if m * tile < kn.size else 0.0
+                    qmax[b, h, m] = qn[m * tile:(m + 1) * tile].max()
+        bound = scale * qmax * kmax
+        return kmax, qmax, bound, 2 * bound <= gate_limit
+
+    from tests import test_oracle_bound_blocks as tb
+    monkeypatch.setattr(Bd, "fixed_m_bound_blocks", broken)
+    monkeypatch.setattr(oracle, "fixed_m_bound_blocks", broken)
+    _must_fail(tb.test_block_bound_dominates_allowed_scores_and_the_head_bound, "window3")
