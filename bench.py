@@ -73,6 +73,8 @@ def workload_text(args):
     fwd = args.softmax + (" gated" if args.softmax == "fixed_m" else "")
     if args.softmax == "fixed_m" and args.bound == "smoothed":
         fwd += ", k-smoothed bound"
+    if args.softmax == "fixed_m" and args.bound == "block":
+        fwd += " per row, per q-block bound"
     if args.workload in FORWARD_ONLY:
         return f"{WORKLOADS[args.workload]}; forward {fwd}"
     bwd = "atomic (non-deterministic)" if args.nondet else f"deterministic ({args.order} kv-column order)"
@@ -88,8 +90,9 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--softmax", default="fixed_m", choices=["fixed_m", "online"])
-    ap.add_argument("--bound", default="norm", choices=["norm", "smoothed"],
-                    help="fixed-m reference: Cauchy-Schwarz on ||k|| or on the centred keys")
+    ap.add_argument("--bound", default="norm", choices=["norm", "smoothed", "block"],
+                    help="fixed-m reference: Cauchy-Schwarz on ||k|| (per-head gate), on the centred keys, "
+                         "or per q-block over the key blocks it reaches (per-row gate)")
     ap.add_argument("--order", default="desc", choices=["asc", "desc", "outside_in", "greedy"])
     ap.add_argument("--nondet", action="store_true", help="atomic (non-deterministic) dQ backward")
     ap.add_argument("--o-residual", default="auto", choices=["auto", "drop"],
@@ -396,12 +399,16 @@ def softmax_table(args, wl, flush, stream, n=10):
         st = bsa.Stages(wl.q, wl.k, wl.v, wl.mask, softmax_mode=mode, bound_mode=args.bound,
                         o_residual=args.o_residual)
         st.plan_and_bound()
+        st.forward()
+        fixed_rows = st.ws.fixed_rows()  # one forward since the plan build
         out[mode] = _median_event_ms(st.forward, flush.zero_, n, stream)
         if st.ws.status() != 0:
             raise RuntimeError(f"device status {st.ws.status()} timing the {mode} forward")
         if mode == "fixed_m":
-            g = st.ws.gate().cpu()
-            gates = {"fixed_m_heads": int(g.sum()), "online_heads": int(g.numel() - g.sum())}
+            gates = {"fixed_m_rows": fixed_rows, "rows": wl.B * wl.H * wl.Sq}
+            if args.bound != "block":
+                g = st.ws.gate().cpu()
+                gates.update({"fixed_m_heads": int(g.sum()), "online_heads": int(g.numel() - g.sum())})
         del st
     return out, gates
 

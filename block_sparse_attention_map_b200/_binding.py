@@ -25,7 +25,7 @@ TILE = 128
 TILE_EMPTY, TILE_PARTIAL, TILE_FULL = 0, 1, 2
 MASK_SEGMENT_IDS, MASK_KV_VALID_LEN, MASK_VARLEN, MASK_CAUSAL_WINDOW, MASK_PREFIX_LM = 1, 2, 4, 8, 16
 SOFTMAX_ONLINE, SOFTMAX_FIXED_M_GATED = 0, 1
-BOUND = {"norm": 0, "smoothed": 1}
+BOUND = {"norm": 0, "smoothed": 1, "block": 2}
 ORDER = {"asc": 0, "desc": 1, "perm": 2, "outside_in": 3, "greedy": 4}
 O_RESIDUAL = {"auto": 0, "keep": 1, "drop": 2}
 FULL_BIT = 1 << 30
@@ -63,7 +63,7 @@ class WorkspaceView(ctypes.Structure):
         "total_bytes", "fwd_bytes", "off_status", "off_tile_class", "off_rank", "off_row_ptr",
         "off_row_ent", "off_col_ptr", "off_col_ent", "off_col_rank", "off_perm", "off_kmax",
         "off_qmax", "off_gate", "off_delta", "off_dq_accum", "off_sem", "off_kbar", "off_qdot",
-        "off_o_resid")] + \
+        "off_o_resid", "off_kblk", "off_kmax_q")] + \
         [("nM", c_i32), ("nN", c_i32)]
 
 
@@ -103,7 +103,7 @@ def lib() -> ctypes.CDLL:
                                           ctypes.c_size_t, c_vp]),
             "bsa_plan_and_bound": (c_i32, [P(Problem), P(MaskSpec), P(Options), c_vp, c_vp, c_vp,
                                            ctypes.c_size_t, c_vp]),
-            "bsa_bwd_preprocess": (c_i32, [P(Problem), P(MaskSpec), P(Options), c_vp, c_vp, c_vp,
+            "bsa_bwd_preprocess": (c_i32, [P(Problem), P(MaskSpec), P(Options), c_vp, c_vp, c_vp, c_vp,
                                            ctypes.c_size_t, c_vp]),
             "bsa_bwd_main": (c_i32, [P(Problem), P(MaskSpec), P(Options), c_vp, c_vp, c_vp, c_vp, c_vp,
                                      c_vp, c_vp, c_vp, ctypes.c_size_t, c_vp]),
@@ -115,6 +115,7 @@ def lib() -> ctypes.CDLL:
             "bsa_static_scratch_init": (c_i32, []),
             "bsa_static_scratch_status": (c_i32, [c_vp, c_i32]),
             "bsa_launch_count": (ctypes.c_uint64, []),
+            "bsa_fixed_rows": (c_i32, [c_vp, ctypes.c_size_t, c_vp, P(ctypes.c_uint64)]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -286,10 +287,26 @@ class Workspace:
     def gate(self):
         return self._arr(self.view.off_gate, self.B * self.H, torch.int32).view(self.B, self.H)
 
+    def kmax_q(self):
+        """Each q-block's kmax [B, H, nM] (the per q-block bound, as the forward used it)."""
+        return self._arr(self.view.off_kmax_q, self.B * self.H * self.nM, torch.float32).view(
+            self.B, self.H, self.nM)
+
+    def kblk(self):
+        """Per kv block and key head, the largest valid ||k_j|| [B, H_kv, nN] (block bound)."""
+        return self._arr(self.view.off_kblk, self.B * self.H_kv * self.nN, torch.float32).view(
+            self.B, self.H_kv, self.nN)
+
     def kbar(self):
         """The k-smoothing centers [B, H_kv, D] (after a smoothed bound)."""
         return self._arr(self.view.off_kbar, self.B * self.H_kv * self.D, torch.float32).view(
             self.B, self.H_kv, self.D)
+
+    def fixed_rows(self):
+        """Query rows the forwards since the last plan build ran fixed-m."""
+        n = ctypes.c_uint64(0)
+        _check(lib().bsa_fixed_rows(self.ptr(), self.nbytes, _stream(), ctypes.byref(n)), "bsa_fixed_rows")
+        return int(n.value)
 
     def status(self, clear=False):
         s = torch.cuda.current_stream().cuda_stream
@@ -413,8 +430,8 @@ class Stages:
                                   _stream()), "bsa_attn_fwd")
 
     def preprocess(self, dout):
-        _check(lib().bsa_bwd_preprocess(*self._args, self.out.data_ptr(), dout.data_ptr(), self.ws.ptr(),
-                                        self.ws.nbytes, _stream()), "bsa_bwd_preprocess")
+        _check(lib().bsa_bwd_preprocess(*self._args, self.q.data_ptr(), self.out.data_ptr(), dout.data_ptr(),
+                                        self.ws.ptr(), self.ws.nbytes, _stream()), "bsa_bwd_preprocess")
 
     def backward_main(self, dout):
         _check(lib().bsa_bwd_main(*self._args, self.q.data_ptr(), self.k.data_ptr(), self.v.data_ptr(),

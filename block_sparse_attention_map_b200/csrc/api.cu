@@ -68,11 +68,15 @@ WsLayout compute_layout(const bsa_problem &p) {
   L.ksum = take(8 * static_cast<size_t>(B * H * p.D));
   L.kcount = take(4 * static_cast<size_t>(B));
   L.qdot = take(4 * static_cast<size_t>(B * H * p.Sq));
+  L.kbmax = take(4 * static_cast<size_t>(B * p.H_kv * nN));
+  L.kmax_q = take(4 * static_cast<size_t>(B * H * nM));
   L.fwd_end = off;
   L.delta = take(4 * static_cast<size_t>(B * H * nM * kTile));
   L.dq_accum = take(4 * static_cast<size_t>(B * H * nM * kTile * p.D));
   L.sem = take(4 * 4 * static_cast<size_t>(B * H * nM));  // one per 32-row quarter of a q-block
-  L.o_resid = take(2 * static_cast<size_t>(B * H * p.Sq * p.D));
+  L.o_resid = take(static_cast<size_t>(B * H * p.Sq * p.D));  // one byte per element
+  L.q16 = take(2 * static_cast<size_t>(B * H * p.Sq * p.D));
+  L.do16 = take(2 * static_cast<size_t>(B * H * p.Sq * p.D));
   L.total = off;
   return L;
 }
@@ -99,10 +103,11 @@ EncodeTiledFn get_encode() {
   return fn;
 }
 
-// 4-D map over a bf16 [B, S, H, D] tensor: dims (D, S, H, B), 64 x 128 boxes,
-// 128-byte swizzle.  Out-of-range rows read as zero.
+// 4-D map over a 16-bit [B, S, H, D] tensor (bf16, or fp16 for the backward's
+// converted copies): dims (D, S, H, B), 64 x 128 boxes, 128-byte swizzle.
+// Out-of-range rows read as zero.
 bool make_map(CUtensorMap *map, const void *ptr, int B, int S, int H, int D,
-              const int64_t *stride) {
+              const int64_t *stride, bool fp16 = false) {
   auto enc = get_encode();
   if (enc == nullptr) return false;
   const cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(S),
@@ -112,7 +117,8 @@ bool make_map(CUtensorMap *map, const void *ptr, int B, int S, int H, int D,
                                  static_cast<cuuint64_t>(stride[0]) * 2};
   const cuuint32_t box[4] = {64, static_cast<cuuint32_t>(kTile), 1, 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
-  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(ptr), dims,
+  const CUresult r = enc(map, fp16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
+                         const_cast<void *>(ptr), dims,
                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -120,6 +126,19 @@ bool make_map(CUtensorMap *map, const void *ptr, int B, int S, int H, int D,
 }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// The backward's tensor maps: Q and dO from the fp16 copies the Delta pass
+// writes into the workspace (contiguous [B, Sq, H, D]), K and V from the
+// caller's bf16 tensors (converted per kv column inside the kernel).
+bool bwd_maps(const bsa_problem &p, const WsLayout &L, uint8_t *ws, const void *k, const void *v,
+              CUtensorMap *tq, CUtensorMap *tk, CUtensorMap *tv, CUtensorMap *tdo) {
+  const int64_t cs[3] = {static_cast<int64_t>(std::max(p.Sq, 1)) * p.H * p.D,
+                         static_cast<int64_t>(p.H) * p.D, p.D};
+  return make_map(tq, ws + L.q16, p.B, p.Sq, p.H, p.D, cs, true) &&
+         make_map(tk, k, p.B, p.Skv, p.H_kv, p.D, p.k_stride) &&
+         make_map(tv, v, p.B, p.Skv, p.H_kv, p.D, p.v_stride) &&
+         make_map(tdo, ws + L.do16, p.B, p.Sq, p.H, p.D, cs, true);
+}
 
 // Resolve defaults (contiguous strides, scale) into a private copy.
 bsa_status normalise(const bsa_problem *in, bsa_problem *out) {
@@ -199,8 +218,9 @@ bsa_status check_options(const bsa_options *o, int nN, bsa_options *out) {
   if (o->softmax_mode != BSA_SOFTMAX_ONLINE && o->softmax_mode != BSA_SOFTMAX_FIXED_M_GATED)
     return BSA_ERR_INVALID_ARG;
   if (o->bwd_order < BSA_ORDER_ASC || o->bwd_order > BSA_ORDER_GREEDY) return BSA_ERR_INVALID_ARG;
-  if (o->bound_mode != BSA_BOUND_NORM && o->bound_mode != BSA_BOUND_SMOOTHED) return BSA_ERR_INVALID_ARG;
-  if (o->bound_mode == BSA_BOUND_SMOOTHED && o->kmax_override != nullptr) return BSA_ERR_INVALID_ARG;
+  if (o->bound_mode != BSA_BOUND_NORM && o->bound_mode != BSA_BOUND_SMOOTHED && o->bound_mode != BSA_BOUND_BLOCK)
+    return BSA_ERR_INVALID_ARG;
+  if (o->bound_mode != BSA_BOUND_NORM && o->kmax_override != nullptr) return BSA_ERR_INVALID_ARG;
   if (o->o_residual < BSA_O_RESIDUAL_AUTO || o->o_residual > BSA_O_RESIDUAL_DROP) return BSA_ERR_INVALID_ARG;
   if (o->bwd_order == BSA_ORDER_PERM) {
     if (o->perm == nullptr) return BSA_ERR_INVALID_ARG;
@@ -499,6 +519,8 @@ bsa_status bsa_workspace_layout(const bsa_problem *prob, const bsa_mask_spec *ma
   view->off_kbar = L.kbar;
   view->off_qdot = L.qdot;
   view->off_o_resid = L.o_resid;
+  view->off_kblk = L.kbmax;
+  view->off_kmax_q = L.kmax_q;
   view->nM = L.nM;
   view->nN = L.nN;
   return BSA_OK;
@@ -540,18 +562,14 @@ bsa_status bsa_attn_bwd(const bsa_problem *prob, const bsa_mask_spec *mask,
   if (P.empty) return empty_backward(P.p, dk, dv, stream);
   const bsa_problem &p = P.p;
   CUtensorMap tq, tk, tv, tdo;
-  if (!make_map(&tq, q, p.B, p.Sq, p.H, p.D, p.q_stride) ||
-      !make_map(&tk, k, p.B, p.Skv, p.H_kv, p.D, p.k_stride) ||
-      !make_map(&tv, v, p.B, p.Skv, p.H_kv, p.D, p.v_stride) ||
-      !make_map(&tdo, dout, p.B, p.Sq, p.H, p.D, p.o_stride))
-    return BSA_ERR_UNSUPPORTED;
+  if (!bwd_maps(p, P.L, static_cast<uint8_t *>(ws), k, v, &tq, &tk, &tv, &tdo)) return BSA_ERR_UNSUPPORTED;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   uint8_t *w = static_cast<uint8_t *>(ws);
   if (!P.o.plan_ready) {
     if ((st = cuda_status(launch_plan(p, P.m, P.o, P.L, w, s))) != BSA_OK) return st;
   }
   const MaskParams mp = mask_params(p, P.m, P.L, w);
-  return cuda_status(launch_bwd(p, mp, P.o, signature(p, P.m, P.o), tq, tk, tv, tdo, out, dout,
+  return cuda_status(launch_bwd(p, mp, P.o, signature(p, P.m, P.o), tq, tk, tv, tdo, q, out, dout,
                                 lse, dq, dk, dv, P.L, w, s));
 }
 
@@ -590,16 +608,16 @@ bsa_status bsa_plan_and_bound(const bsa_problem *prob, const bsa_mask_spec *mask
 }
 
 bsa_status bsa_bwd_preprocess(const bsa_problem *prob, const bsa_mask_spec *mask,
-                              const bsa_options *opt, const void *out, const void *dout, void *ws,
-                              size_t ws_bytes, bsa_stream_t stream) {
+                              const bsa_options *opt, const void *q, const void *out,
+                              const void *dout, void *ws, size_t ws_bytes, bsa_stream_t stream) {
   if (!problem_is_empty(prob)) {
-    if (out == nullptr || dout == nullptr) return BSA_ERR_INVALID_ARG;
-    if (!aligned16(out) || !aligned16(dout)) return BSA_ERR_UNSUPPORTED;
+    if (q == nullptr || out == nullptr || dout == nullptr) return BSA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(out) || !aligned16(dout)) return BSA_ERR_UNSUPPORTED;
   }
   Prepared P;
   bsa_status st = prepare(prob, mask, opt, ws, ws_bytes, true, &P);
   if (st != BSA_OK || P.empty) return st;
-  return cuda_status(launch_bwd_preprocess(P.p, P.o, out, dout, P.L, static_cast<uint8_t *>(ws),
+  return cuda_status(launch_bwd_preprocess(P.p, P.o, q, out, dout, P.L, static_cast<uint8_t *>(ws),
                                            reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -623,11 +641,7 @@ bsa_status bsa_bwd_main(const bsa_problem *prob, const bsa_mask_spec *mask,
   if (P.empty) return empty_backward(P.p, dk, dv, stream);
   const bsa_problem &p = P.p;
   CUtensorMap tq, tk, tv, tdo;
-  if (!make_map(&tq, q, p.B, p.Sq, p.H, p.D, p.q_stride) ||
-      !make_map(&tk, k, p.B, p.Skv, p.H_kv, p.D, p.k_stride) ||
-      !make_map(&tv, v, p.B, p.Skv, p.H_kv, p.D, p.v_stride) ||
-      !make_map(&tdo, dout, p.B, p.Sq, p.H, p.D, p.o_stride))
-    return BSA_ERR_UNSUPPORTED;
+  if (!bwd_maps(p, P.L, static_cast<uint8_t *>(ws), k, v, &tq, &tk, &tv, &tdo)) return BSA_ERR_UNSUPPORTED;
   uint8_t *w = static_cast<uint8_t *>(ws);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (!P.o.plan_ready) {
@@ -664,6 +678,18 @@ bsa_status bsa_get_device_status(void *ws, size_t ws_bytes, bsa_stream_t stream,
   }
   if (h[kHdrStatus] != 0) return static_cast<bsa_status>(h[kHdrStatus]);
   if (h[kHdrGateWarn] != 0) return BSA_WARN_GATE_VIOLATION;
+  return BSA_OK;
+}
+
+bsa_status bsa_fixed_rows(void *ws, size_t ws_bytes, bsa_stream_t stream, uint64_t *rows) {
+  if (ws == nullptr || rows == nullptr || ws_bytes < kHdrWords * 4) return BSA_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint32_t n = 0;
+  if (cudaMemcpyAsync(&n, static_cast<uint32_t *>(ws) + kHdrFixedRows, sizeof(n), cudaMemcpyDeviceToHost, s) !=
+      cudaSuccess)
+    return BSA_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return BSA_ERR_CUDA;
+  *rows = n;
   return BSA_OK;
 }
 

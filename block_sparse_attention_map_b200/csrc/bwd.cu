@@ -83,9 +83,8 @@ struct BwdSmem {
                        bSFull = bDOEmpty + NDO, bDPFull = bSFull + 1, bPReady = bDPFull + 1,
                        bDSReady = bPReady + 1, bDSFree = bDSReady + 1, bDQFull = bDSFree + 1,
                        bDQFree = bDQFull + 1, bDKVFull = bDQFree + 1, bDKVFree = bDKVFull + 1,
-                       bVecReady = bDKVFree + 1, bQConv = bVecReady + 2, bDOConv = bQConv + NQ,
-                       bKConv = bDOConv + NDO, bVConv = bKConv + 1, bFinal = bVConv + 1,
-                       kNumBars = bFinal + 1;
+                       bVecReady = bDKVFree + 1, bKConv = bVecReady + 2, bVConv = bKConv + 1,
+                       bFinal = bVConv + 1, kNumBars = bFinal + 1;
   static constexpr int kMisc = kBar + kNumBars * 8;
   static constexpr int kAlloc = kMisc + 16;
 };
@@ -175,7 +174,7 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
           i == L::bVecReady + 1)
         cnt = kComputeThreads;
       if (i == L::bDQFree) cnt = 128;
-      if ((i >= L::bQConv && i < L::bKConv) || i == L::bKConv || i == L::bVConv) cnt = kConvThreads;
+      if (i == L::bKConv || i == L::bVConv) cnt = kConvThreads;
       mbar_init(&bars[i], cnt);
     }
     *abort_flag = 0;
@@ -301,7 +300,7 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       const uint32_t ds_addr = smem_u32(sm + L::kDS);
       auto issue_s = [&](uint32_t e_idx) -> bool {  // S^T = K_n Q_m^T
         const uint32_t qs = e_idx % NQ;
-        if (!wd.wait(&bars[L::bQConv + qs], (e_idx / NQ) & 1)) return false;
+        if (!wd.wait(&bars[L::bQFull + qs], (e_idx / NQ) & 1)) return false;
         tc_fence_after();
         const uint32_t q_addr = smem_u32(sm + L::kQ + qs * kTB);
 #pragma unroll
@@ -315,7 +314,7 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       };
       auto issue_dp = [&](uint32_t e_idx) -> bool {  // dP^T = V_n dO_m^T
         const uint32_t ds = e_idx % NDO;
-        if (!wd.wait(&bars[L::bDOConv + ds], (e_idx / NDO) & 1)) return false;
+        if (!wd.wait(&bars[L::bDOFull + ds], (e_idx / NDO) & 1)) return false;
         // the dQ of the previous entry occupies these columns until read out
         if (e_idx >= 1 && !wd.wait(&bars[L::bDQFree], (e_idx - 1) & 1)) return false;
         tc_fence_after();
@@ -401,11 +400,12 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
     }
     } else if (run) {
     // ------------------------------------------------------------ converters (warps 2, 3)
-    // Every tile the MMAs read (Q_m and dO_m per entry, K_n and V_n per column)
-    // is turned from bf16 into fp16 in place as soon as its copy lands, in the
-    // producer's order: the products then take P and dS at fp16's 11
-    // significant bits instead of bf16's 8.  Values of an input beyond the
-    // fp16 range are clamped and reported as BSA_ERR_INPUT_RANGE.
+    // Every product runs on fp16 operands, so that P and dS enter them with
+    // fp16's 11 significant bits instead of bf16's 8.  Q_m and dO_m arrive as
+    // fp16 already (the Delta pass wrote fp16 copies); K_n and V_n, loaded once
+    // per kv column from the caller's bf16 tensors, are turned into fp16 in
+    // place here as soon as their copies land.  Values beyond the fp16 range
+    // are clamped and reported as BSA_ERR_INPUT_RANGE.
     const int ct = threadIdx.x - 64;  // 0 .. 63
     auto wwait = [&](uint64_t *bar, uint32_t parity) {
       return __all_sync(0xffffffffu, wd.wait(bar, parity)) != 0;
@@ -437,8 +437,7 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       fence_proxy_async_smem();  // the MMAs read the tile through the async proxy
       mbar_arrive(done);
     };
-    uint32_t tc = 0, cc = 0, ec = 0;
-    bool stop = false;
+    uint32_t tc = 0, cc = 0;
     for (;; ++tc) {
       const uint32_t slot = tc & 1;
       if (!wwait(&bars[L::bTkFull + slot], (tc >> 1) & 1)) break;
@@ -448,21 +447,11 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       const Ticket k = decode_ticket(p, t);
       if (!k.valid) break;
       if (k.ee == k.es) continue;
-      for (int x = 0; x < k.tot; ++x, ++ec) {
-        const uint32_t qs = ec % NQ, ds = ec % NDO;
-        if (!wwait(&bars[L::bQFull + qs], (ec / NQ) & 1)) { stop = true; break; }
-        convert(sm + L::kQ + qs * kTB, &bars[L::bQConv + qs]);
-        if (x == 0) {
-          const int kb = cc & 1, vb = kb ^ 1;
-          if (!wwait(&bars[L::bKFull], cc & 1)) { stop = true; break; }
-          convert(sm + L::kK + kb * kTB, &bars[L::bKConv]);
-          if (!wwait(&bars[L::bVFull], cc & 1)) { stop = true; break; }
-          convert(sm + L::kK + vb * kTB, &bars[L::bVConv]);
-        }
-        if (!wwait(&bars[L::bDOFull + ds], (ec / NDO) & 1)) { stop = true; break; }
-        convert(sm + L::kDO + ds * kTB, &bars[L::bDOConv + ds]);
-      }
-      if (stop) break;
+      const int kb = cc & 1, vb = kb ^ 1;
+      if (!wwait(&bars[L::bKFull], cc & 1)) break;
+      convert(sm + L::kK + kb * kTB, &bars[L::bKConv]);
+      if (!wwait(&bars[L::bVFull], cc & 1)) break;
+      convert(sm + L::kK + vb * kTB, &bars[L::bVConv]);
       ++cc;
     }
     // |x| >= 65536 (bf16 bits 0x4780; bf16 has no value in (65280, 65536)),
@@ -863,20 +852,29 @@ __device__ __forceinline__ float half_ulp_bf16(uint32_t bits) {
   return __uint_as_float((max(e, 9u) - 8u) << 23);
 }
 
+struct DeltaArgs {
+  const __nv_bfloat16 *o, *dout, *q;
+  int64_t sb, ss, sh;     // O and dO strides
+  int64_t qb, qs, qh;     // Q strides
+  int B, Sq, H, Skv, rows_pad;
+  const uint8_t *resid;   // [B, Sq, H, D] scaled e5m2 residual bytes
+  uint32_t *hdr;
+  float *delta;
+  uint32_t *sem;
+  int64_t n_sem;
+  uint32_t *q16, *do16;   // [B, Sq, H, D] fp16 copies for the backward's products
+};
+
 template <int D, bool RESID>
-__global__ void __launch_bounds__(256) k_bwd_delta(const __nv_bfloat16 *__restrict__ o,
-                                                   const __nv_bfloat16 *__restrict__ dout,
-                                                   int64_t sb, int64_t ss, int64_t sh, int B,
-                                                   int Sq, int H, int Skv, int rows_pad,
-                                                   const __nv_bfloat16 *__restrict__ resid,
-                                                   const uint32_t *__restrict__ hdr,
-                                                   float *__restrict__ delta,
-                                                   uint32_t *__restrict__ sem, int64_t n_sem) {
-  // D/8 threads per (b, h, i) row vector, 16 bytes of O, dO (and the O
+__global__ void __launch_bounds__(256) k_bwd_delta(const DeltaArgs a) {
+  // D/8 threads per (b, h, i) row vector, 16 bytes of O, dO, Q (and the O
   // residual) each.  A block takes kDeltaRuns runs of 256 / (D/8) consecutive
   // rows of one head (the Delta layout), every run's loads in flight before any
   // is reduced; rows past Sq (the last q-block's padding) get Delta = 0.  The
-  // grid also zeroes the dQ semaphores.  RESID: the O residual is added to O
+  // same pass writes fp16 copies of Q and dO (the backward main kernel takes
+  // every product on fp16 operands) and reports values beyond the fp16 range
+  // as BSA_ERR_INPUT_RANGE.  The grid also zeroes the dQ semaphores.  RESID:
+  // the O residual is added to O
   // (a compile-time choice, so that the plain pass carries no zero vector),
   // and only when the header records that the last forward on this workspace
   // kept the residual of this very `o` for this problem (else Delta comes from
@@ -888,16 +886,18 @@ __global__ void __launch_bounds__(256) k_bwd_delta(const __nv_bfloat16 *__restri
   constexpr int VPB = 256 / TPV;
   pdl_wait();  // O comes from the forward, launched just before
   pdl_trigger();
+  const int B = a.B, Sq = a.Sq, H = a.H, rows_pad = a.rows_pad;
+  const uint32_t *hdr = a.hdr;
   bool use_resid = false;
   if (RESID) {
     const uint64_t tag = (static_cast<uint64_t>(hdr[kHdrResidHi]) << 32) | hdr[kHdrResidLo];
-    use_resid = tag == reinterpret_cast<uint64_t>(o) && hdr[kHdrResidB] == static_cast<uint32_t>(B) &&
+    use_resid = tag == reinterpret_cast<uint64_t>(a.o) && hdr[kHdrResidB] == static_cast<uint32_t>(B) &&
                 hdr[kHdrResidH] == static_cast<uint32_t>(H) && hdr[kHdrResidSq] == static_cast<uint32_t>(Sq) &&
-                hdr[kHdrResidSkv] == static_cast<uint32_t>(Skv) && hdr[kHdrResidD] == static_cast<uint32_t>(D);
+                hdr[kHdrResidSkv] == static_cast<uint32_t>(a.Skv) && hdr[kHdrResidD] == static_cast<uint32_t>(D);
   }
-  for (int64_t z = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; z < n_sem;
+  for (int64_t z = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; z < a.n_sem;
        z += static_cast<int64_t>(gridDim.x) * blockDim.x)
-    sem[z] = 0u;
+    a.sem[z] = 0u;
   const int t = threadIdx.x % TPV;
   // the block's rows all belong to one (b, h): its index and first row come
   // from one division per block, not per row
@@ -909,36 +909,64 @@ __global__ void __launch_bounds__(256) k_bwd_delta(const __nv_bfloat16 *__restri
   const bool in_bh = bh < B * H;  // uniform per block; no early return before the shuffles
   int64_t g[kDeltaRuns];
   bool in[kDeltaRuns];
-  int4 av[kDeltaRuns], cv[kDeltaRuns], rv[kDeltaRuns];
+  int4 av[kDeltaRuns], cv[kDeltaRuns], qv[kDeltaRuns];
+  uint2 rv[kDeltaRuns];
 #pragma unroll
   for (int j = 0; j < kDeltaRuns; ++j) {
     const int i = i0 + j * VPB;
     g[j] = static_cast<int64_t>(bh) * rows_pad + i;
     in[j] = in_bh;
-    av[j] = cv[j] = rv[j] = make_int4(0, 0, 0, 0);
+    av[j] = cv[j] = qv[j] = make_int4(0, 0, 0, 0);
+    rv[j] = make_uint2(0u, 0u);
     if (in[j] && i < Sq) {
-      const int64_t off = b * sb + static_cast<int64_t>(i) * ss + h * sh + t * 8;
-      av[j] = __ldg(reinterpret_cast<const int4 *>(o + off));
-      cv[j] = __ldg(reinterpret_cast<const int4 *>(dout + off));
+      const int64_t off = b * a.sb + static_cast<int64_t>(i) * a.ss + h * a.sh + t * 8;
+      av[j] = __ldg(reinterpret_cast<const int4 *>(a.o + off));
+      cv[j] = __ldg(reinterpret_cast<const int4 *>(a.dout + off));
+      qv[j] = __ldcs(reinterpret_cast<const int4 *>(a.q + b * a.qb + static_cast<int64_t>(i) * a.qs + h * a.qh + t * 8));
       if (use_resid)
-        rv[j] = __ldg(reinterpret_cast<const int4 *>(resid + ((static_cast<int64_t>(b) * Sq + i) * H + h) * D + t * 8));
+        rv[j] = __ldg(reinterpret_cast<const uint2 *>(a.resid + ((static_cast<int64_t>(b) * Sq + i) * H + h) * D + t * 8));
     }
   }
+  // fp16 copies of Q and dO, contiguous [B, Sq, H, D]
+  uint32_t in_max = 0;
+#pragma unroll
+  for (int j = 0; j < kDeltaRuns; ++j) {
+    const int i = i0 + j * VPB;
+    if (in[j] && i < Sq) {
+      const int64_t off = ((static_cast<int64_t>(b) * Sq + i) * H + h) * (D / 2) + t * 4;
+      const uint32_t xq[4] = {static_cast<uint32_t>(qv[j].x), static_cast<uint32_t>(qv[j].y),
+                              static_cast<uint32_t>(qv[j].z), static_cast<uint32_t>(qv[j].w)};
+      const uint32_t xd[4] = {static_cast<uint32_t>(cv[j].x), static_cast<uint32_t>(cv[j].y),
+                              static_cast<uint32_t>(cv[j].z), static_cast<uint32_t>(cv[j].w)};
+      uint32_t hq[4], hd[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        in_max = __vmaxu2(in_max, __vmaxu2(xq[q] & 0x7fff7fffu, xd[q] & 0x7fff7fffu));
+        hq[q] = bf16x2_to_f16x2(xq[q]);
+        hd[q] = bf16x2_to_f16x2(xd[q]);
+      }
+      *reinterpret_cast<int4 *>(a.q16 + off) = make_int4(hq[0], hq[1], hq[2], hq[3]);
+      *reinterpret_cast<int4 *>(a.do16 + off) = make_int4(hd[0], hd[1], hd[2], hd[3]);
+    }
+  }
+  // |x| >= 65536 (bf16 bits 0x4780), infinities and NaNs: beyond what fp16 holds
+  if ((in_max & 0xffffu) >= 0x4780u || (in_max >> 16) >= 0x4780u)
+    record_status(a.hdr + kHdrStatus, BSA_ERR_INPUT_RANGE);
 #pragma unroll
   for (int j = 0; j < kDeltaRuns; ++j) {
     const uint32_t xa[4] = {static_cast<uint32_t>(av[j].x), static_cast<uint32_t>(av[j].y),
                             static_cast<uint32_t>(av[j].z), static_cast<uint32_t>(av[j].w)};
     const uint32_t xc[4] = {static_cast<uint32_t>(cv[j].x), static_cast<uint32_t>(cv[j].y),
                             static_cast<uint32_t>(cv[j].z), static_cast<uint32_t>(cv[j].w)};
-    const uint32_t xr[4] = {static_cast<uint32_t>(rv[j].x), static_cast<uint32_t>(rv[j].y),
-                            static_cast<uint32_t>(rv[j].z), static_cast<uint32_t>(rv[j].w)};
+    // residual bytes of elements 2q, 2q+1: 16 bits of rv
+    const uint32_t xr[4] = {rv[j].x & 0xffffu, rv[j].x >> 16, rv[j].y & 0xffffu, rv[j].y >> 16};
     float acc = 0.f;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       float2 fo = unpack_bf16x2(xa[q]);
       const float2 fd = unpack_bf16x2(xc[q]);
       if (use_resid) {
-        const float2 fr = unpack_bf16x2(xr[q]);
+        const float2 fr = unpack_resid_e5m2x2(xr[q]);
         fo.x += fabsf(fr.x) <= half_ulp_bf16(xa[q] & 0xffffu) ? fr.x : 0.f;
         fo.y += fabsf(fr.y) <= half_ulp_bf16(xa[q] >> 16) ? fr.y : 0.f;
       }
@@ -947,7 +975,7 @@ __global__ void __launch_bounds__(256) k_bwd_delta(const __nv_bfloat16 *__restri
     }
 #pragma unroll
     for (int sft = TPV / 2; sft > 0; sft >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, sft);
-    if (t == 0 && in[j]) delta[g[j]] = acc;
+    if (t == 0 && in[j]) a.delta[g[j]] = acc;
   }
 }
 
@@ -1062,15 +1090,13 @@ cudaError_t run_bwd_main(const BwdParams &bp, const CUtensorMap &tq, const CUten
 
 }  // namespace
 
-cudaError_t launch_bwd_preprocess(const bsa_problem &p, const bsa_options &o, const void *out,
-                                  const void *dout, const WsLayout &L, uint8_t *ws,
-                                  cudaStream_t s) {
+cudaError_t launch_bwd_preprocess(const bsa_problem &p, const bsa_options &o, const void *q,
+                                  const void *out, const void *dout, const WsLayout &L,
+                                  uint8_t *ws, cudaStream_t s) {
   const int rows_pad = L.nM * kTile;
   const int64_t groups = static_cast<int64_t>(p.B) * p.H * rows_pad;
   float *delta = reinterpret_cast<float *>(ws + L.delta);
-  const __nv_bfloat16 *resid = o.o_residual != BSA_O_RESIDUAL_DROP
-                                   ? reinterpret_cast<const __nv_bfloat16 *>(ws + L.o_resid)
-                                   : nullptr;
+  const uint8_t *resid = o.o_residual != BSA_O_RESIDUAL_DROP ? ws + L.o_resid : nullptr;
   // kDeltaRuns runs of 256 / (D / 8) vectors per block
   const int64_t vpb = kDeltaRuns * (256 / (p.D / 8));
   const unsigned blocks = static_cast<unsigned>((groups + vpb - 1) / vpb);
@@ -1079,10 +1105,29 @@ cudaError_t launch_bwd_preprocess(const bsa_problem &p, const bsa_options &o, co
   // a programmatic dependent of the forward (which reads O first after it)
   auto kern = p.D == 64 ? (resid != nullptr ? k_bwd_delta<64, true> : k_bwd_delta<64, false>)
                         : (resid != nullptr ? k_bwd_delta<128, true> : k_bwd_delta<128, false>);
-  cudaError_t e = launch_pdl(kern, dim3(blocks), dim3(256), 0, s,
-                             static_cast<const __nv_bfloat16 *>(out), static_cast<const __nv_bfloat16 *>(dout),
-                             p.o_stride[0], p.o_stride[1], p.o_stride[2], p.B, p.Sq, p.H, p.Skv, rows_pad, resid,
-                             reinterpret_cast<const uint32_t *>(ws + L.status), delta, sem, n_sem);
+  DeltaArgs da{};
+  da.o = static_cast<const __nv_bfloat16 *>(out);
+  da.dout = static_cast<const __nv_bfloat16 *>(dout);
+  da.q = static_cast<const __nv_bfloat16 *>(q);
+  da.sb = p.o_stride[0];
+  da.ss = p.o_stride[1];
+  da.sh = p.o_stride[2];
+  da.qb = p.q_stride[0];
+  da.qs = p.q_stride[1];
+  da.qh = p.q_stride[2];
+  da.B = p.B;
+  da.Sq = p.Sq;
+  da.H = p.H;
+  da.Skv = p.Skv;
+  da.rows_pad = rows_pad;
+  da.resid = resid;
+  da.hdr = reinterpret_cast<uint32_t *>(ws + L.status);
+  da.delta = delta;
+  da.sem = sem;
+  da.n_sem = n_sem;
+  da.q16 = reinterpret_cast<uint32_t *>(ws + L.q16);
+  da.do16 = reinterpret_cast<uint32_t *>(ws + L.do16);
+  cudaError_t e = launch_pdl(kern, dim3(blocks), dim3(256), 0, s, da);
   if (e != cudaSuccess) return e;
   count_launch();
   if (!o.deterministic) {
@@ -1169,10 +1214,10 @@ cudaError_t launch_zero_kv_grads(const bsa_problem &p, void *dk, void *dv, cudaS
 
 cudaError_t launch_bwd(const bsa_problem &p, const MaskParams &mp, const bsa_options &o,
                        const PlanSignature &sig, const CUtensorMap &tq, const CUtensorMap &tk,
-                       const CUtensorMap &tv, const CUtensorMap &tdo, const void *out,
+                       const CUtensorMap &tv, const CUtensorMap &tdo, const void *q, const void *out,
                        const void *dout, const float *lse, void *dq, void *dk, void *dv,
                        const WsLayout &L, uint8_t *ws, cudaStream_t s) {
-  cudaError_t e = launch_bwd_preprocess(p, o, out, dout, L, ws, s);
+  cudaError_t e = launch_bwd_preprocess(p, o, q, out, dout, L, ws, s);
   if (e != cudaSuccess) return e;
   e = launch_bwd_main(p, mp, o, sig, tq, tk, tv, tdo, lse, dk, dv, L, ws, s);
   if (e != cudaSuccess) return e;

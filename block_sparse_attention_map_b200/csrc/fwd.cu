@@ -59,10 +59,15 @@ struct FwdParams {
   int64_t o_sb, o_ss, o_sh;
   float *lse;
   int fixed_mode;
+  int block_bound;     // per q-block bound: kmax_m from kblk, ||q_i|| from the Q tile, per-row gate
+  float gate_limit;
+  int Hk, nN;
+  const float *kblk;   // [B, H_kv, nN] per kv block max ||k_j|| (block bound)
+  float *kmax_q;       // [B, H, nM] each q-block's kmax, written for inspection (block bound)
   const float *kmax;   // [B, H] (the radius R with k-smoothing)
   const float *qnorm;  // [B, H, Sq]
   const float *qdot;   // [B, H, Sq] q_i . center with k-smoothing, else null
-  __nv_bfloat16 *o_resid;  // [B, Sq, H, D] O - bf16(O), or null
+  uint8_t *o_resid;  // [B, Sq, H, D] O - bf16(O) as scaled e5m2 bytes, or null
   const int32_t *gate; // [B, H]
   uint32_t *hdr;
   uint64_t timeout_ns;
@@ -370,10 +375,15 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
     auto wwait = [&](uint64_t *bar, uint32_t parity) {
       return __all_sync(0xffffffffu, wd.wait(bar, parity)) != 0;
     };
-    uint32_t tcount = 0, ps = 0;
+    uint32_t tcount = 0, ps = 0, qm = 0;
     bool stop = false;
     for (int u = blockIdx.x; u < p.n_units && !stop; u += gridDim.x) {
       const FwdUnit w = decode_unit(p, u);
+      // the unit's Q tiles sit in the Q ring in load order (A, then B), as the
+      // producer and the MMA warp count them
+      const bool has0 = w.re[0] > w.rs[0], has1 = w.re[1] > w.rs[1];
+      const uint32_t q_i = qm + (x == 1 && has0 ? 1u : 0u);
+      qm += (has0 ? 1u : 0u) + (has1 ? 1u : 0u);
       if (w.m[x] >= p.nM) continue;
       const int rs = w.rs[x], re = w.re[x], nt = re - rs;
       const int b = w.b, h = w.h, bh = w.bh;
@@ -390,12 +400,48 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
         }
         continue;
       }
-      const bool fixed = p.fixed_mode && p.gate[bh] != 0;
+      bool fixed = p.fixed_mode && !p.block_bound && p.gate[bh] != 0;
       float m_ref = -INFINITY, l = 0.f, l_r = 0.f;
       if (fixed)
         m_ref = row_ok ? p.scale_log2 * fmaf(p.qnorm[static_cast<int64_t>(bh) * p.Sq + i], p.kmax[bh],
                                              p.qdot != nullptr ? p.qdot[static_cast<int64_t>(bh) * p.Sq + i] : 0.f)
                        : 0.f;
+      if (p.fixed_mode && p.block_bound) {
+        // per q-block bound: kmax_m over the key blocks of this q-block's row
+        // list (each warp reduces it), ||q_i|| from this row of the Q tile,
+        // and the gate per row
+        const int hk = h / p.kv_group;
+        const float *kb = p.kblk + (static_cast<int64_t>(b) * p.Hk + hk) * p.nN;
+        float km = 0.f;
+        for (int jj = rs + lane; jj < re; jj += 32) km = fmaxf(km, kb[p.row_ent[jj] & kIndexMask]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) km = fmaxf(km, __shfl_xor_sync(0xffffffffu, km, o));
+        if (!wwait(&bars[L::bQFull + q_i % NQ], (q_i / NQ) & 1)) { stop = true; break; }
+        const uint8_t *qt = sm + L::kQ + (q_i % NQ) * kTB + r * 128;
+        float ss = 0.f;
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c) {
+#pragma unroll
+          for (int k8 = 0; k8 < 8; ++k8) {
+            const int4 v = *reinterpret_cast<const int4 *>(qt + c * 16384 + ((k8 ^ (r & 7)) << 4));
+            const uint32_t xw[4] = {static_cast<uint32_t>(v.x), static_cast<uint32_t>(v.y),
+                                    static_cast<uint32_t>(v.z), static_cast<uint32_t>(v.w)};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 f2 = unpack_bf16x2(xw[e]);
+              ss = fmaf(f2.x, f2.x, fmaf(f2.y, f2.y, ss));
+            }
+          }
+        }
+        const float qn = sqrtf(ss);
+        fixed = 2.f * p.scale * qn * km <= p.gate_limit;
+        if (fixed) m_ref = p.scale_log2 * qn * km;
+        if (r == 0) p.kmax_q[static_cast<int64_t>(bh) * p.nM + w.m[x]] = km;
+      }
+      if (p.fixed_mode) {
+        const uint32_t nf = __popc(__ballot_sync(0xffffffffu, fixed && row_ok));
+        if (lane == 0 && nf != 0u) atomicAdd(p.hdr + kHdrFixedRows, nf);
+      }
       // row-constant part of the mask: allowed keys lie in [lo, hi] (the
       // window, thinned by the dilation) or in the prefix [0, pre_hi]
       int lo = 0, hi = p.Skv - 1, pre_hi = -1;
@@ -462,8 +508,9 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
         }
         if (!wwait(&bars[L::bSFull + x], tcount & 1)) { stop = true; break; }
         tc_fence_after();
-        if (!fixed) {
-          // pass 1: the tile's row max (masked)
+        if (__any_sync(0xffffffffu, !fixed)) {
+          // pass 1: the tile's row max (masked); rows whose reference is
+          // pinned never rise above it, so they take no rescale
           float mx = -INFINITY;
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
@@ -569,17 +616,20 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
           dst[0] = make_int4(wv[0], wv[1], wv[2], wv[3]);
           dst[1] = make_int4(wv[4], wv[5], wv[6], wv[7]);
           if (p.o_resid != nullptr) {
-            // what the bf16 rounding of O dropped, for an exact-to-fp32 Delta
+            // what the bf16 rounding of O dropped (exact in fp32), for the
+            // backward's Delta; 16 one-byte residuals per piece
+            uint32_t rb[4];
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-              const float2 r = unpack_bf16x2(wv[q]);
-              wv[q] = pack_bf16x2(__uint_as_float(o[2 * q]) * inv - r.x,
-                                  __uint_as_float(o[2 * q + 1]) * inv - r.y);
+            for (int q = 0; q < 4; ++q) {
+              const float2 r0 = unpack_bf16x2(wv[2 * q]), r1 = unpack_bf16x2(wv[2 * q + 1]);
+              rb[q] = pack_resid_e5m2x2(__uint_as_float(o[4 * q]) * inv - r0.x,
+                                        __uint_as_float(o[4 * q + 1]) * inv - r0.y) |
+                      (pack_resid_e5m2x2(__uint_as_float(o[4 * q + 2]) * inv - r1.x,
+                                         __uint_as_float(o[4 * q + 3]) * inv - r1.y)
+                       << 16);
             }
-            int4 *rd = reinterpret_cast<int4 *>(p.o_resid + ((static_cast<int64_t>(b) * p.Sq + i) * p.H + h) * D +
-                                                c * 16);
-            rd[0] = make_int4(wv[0], wv[1], wv[2], wv[3]);
-            rd[1] = make_int4(wv[4], wv[5], wv[6], wv[7]);
+            *reinterpret_cast<int4 *>(p.o_resid + ((static_cast<int64_t>(b) * p.Sq + i) * p.H + h) * D + c * 16) =
+                make_int4(rb[0], rb[1], rb[2], rb[3]);
           }
         }
         if (c + 1 < D / 16) tmem_wait_ld();
@@ -676,6 +726,48 @@ __global__ void __launch_bounds__(256) k_key_sums(const NormArgs a) {
     for (int e = 0; e < 8; ++e)
       if (acc[e] != 0) atomicAdd(dst + e, static_cast<unsigned long long>(acc[e]));
   }
+}
+
+// Per q-block bound, its only pass over the inputs: for each kv block n and key
+// head, the largest ||k_j|| over the block's valid keys (padding and varlen
+// alignment keys excluded; 0 when none is valid).  One warp per (b, hk, n):
+// lane l takes keys l, l+32, l+64, l+96 of the block, each row's 16-byte
+// pieces all in flight.
+template <int D>
+__global__ void __launch_bounds__(256) k_key_block_max(const NormArgs a, float *__restrict__ kblk, int nN) {
+  const int64_t wid = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (wid >= static_cast<int64_t>(a.B) * a.Hk * nN) return;
+  const int n = static_cast<int>(wid % nN);
+  const int hk = static_cast<int>((wid / nN) % a.Hk);
+  const int b = static_cast<int>(wid / (static_cast<int64_t>(nN) * a.Hk));
+  float mx = 0.f;
+#pragma unroll 1
+  for (int c = 0; c < 4; ++c) {
+    const int j = n * kTile + lane + 32 * c;
+    if (j >= a.Skv || !key_is_valid(a.mk, b, j)) continue;
+    const int4 *src = reinterpret_cast<const int4 *>(a.k + b * a.ks[0] + static_cast<int64_t>(j) * a.ks[1] +
+                                                     hk * a.ks[2]);
+    int4 v[D / 8];
+#pragma unroll
+    for (int u = 0; u < D / 8; ++u) v[u] = __ldg(src + u);
+    float acc = 0.f;
+#pragma unroll
+    for (int u = 0; u < D / 8; ++u) {
+      const uint32_t xw[4] = {static_cast<uint32_t>(v[u].x), static_cast<uint32_t>(v[u].y),
+                              static_cast<uint32_t>(v[u].z), static_cast<uint32_t>(v[u].w)};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f2 = unpack_bf16x2(xw[e]);
+        acc = fmaf(f2.x, f2.x, acc);
+        acc = fmaf(f2.y, f2.y, acc);
+      }
+    }
+    mx = fmaxf(mx, sqrtf(acc));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  if (lane == 0) kblk[wid] = mx;
 }
 
 // k-smoothing, second pass: the centers c = sum * 2^-20 / (valid keys).
@@ -896,6 +988,16 @@ cudaError_t launch_fixed_m_bound(const bsa_problem &p, const MaskParams &mp,
   na.scale = p.scale;
   na.limit = o.gate_limit > 0.f ? o.gate_limit : 64.f;
   na.gate = reinterpret_cast<int32_t *>(ws + L.gate);
+  if (o.bound_mode == BSA_BOUND_BLOCK) {
+    // the per q-block bound reads K only; the forward takes the rest
+    const int64_t warps = static_cast<int64_t>(p.B) * p.H_kv * L.nN;
+    const unsigned blocks = static_cast<unsigned>((warps * 32 + 255) / 256);
+    float *kblk = reinterpret_cast<float *>(ws + L.kbmax);
+    if (p.D == 64) k_key_block_max<64><<<blocks, 256, 0, s>>>(na, kblk, L.nN);
+    else k_key_block_max<128><<<blocks, 256, 0, s>>>(na, kblk, L.nN);
+    count_launch();
+    return cudaGetLastError();
+  }
   // kmax, qmax and the finished-block counter are adjacent: one memset
   cudaError_t e = cudaMemsetAsync(na.kmax, 0, sizeof(float) * p.B * p.H * 2 + sizeof(uint32_t), s);
   if (e != cudaSuccess) return e;
@@ -963,10 +1065,16 @@ cudaError_t launch_fwd(const bsa_problem &p, const MaskParams &mp, const bsa_opt
   fp.o_sh = p.o_stride[2];
   fp.lse = lse;
   fp.fixed_mode = o.softmax_mode == BSA_SOFTMAX_FIXED_M_GATED;
+  fp.block_bound = o.bound_mode == BSA_BOUND_BLOCK;
+  fp.gate_limit = o.gate_limit > 0.f ? o.gate_limit : 64.f;
+  fp.Hk = p.H_kv;
+  fp.nN = L.nN;
+  fp.kblk = reinterpret_cast<const float *>(ws + L.kbmax);
+  fp.kmax_q = reinterpret_cast<float *>(ws + L.kmax_q);
   fp.kmax = reinterpret_cast<const float *>(ws + L.kmax);
   fp.qnorm = reinterpret_cast<const float *>(ws + L.qnorm);
   fp.qdot = o.bound_mode == BSA_BOUND_SMOOTHED ? reinterpret_cast<const float *>(ws + L.qdot) : nullptr;
-  fp.o_resid = o.o_residual == BSA_O_RESIDUAL_KEEP ? reinterpret_cast<__nv_bfloat16 *>(ws + L.o_resid) : nullptr;
+  fp.o_resid = o.o_residual == BSA_O_RESIDUAL_KEEP ? ws + L.o_resid : nullptr;
   fp.gate = reinterpret_cast<const int32_t *>(ws + L.gate);
   fp.hdr = reinterpret_cast<uint32_t *>(ws + L.status);
   fp.timeout_ns = 2000000000ull;

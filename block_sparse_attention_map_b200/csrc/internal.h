@@ -38,6 +38,7 @@ enum HeaderWord : int {
   kHdrOrder = 10,
   kHdrNSeqs = 11,
   kHdrDilation = 12,
+  kHdrFixedRows = 13,  // query rows the forwards since the plan build ran with a pinned reference
   kHdrPlanWords = 56,  // words [0, 56) are reset by every plan build
   // The O-residual record (kept across plan builds): the `out` pointer whose
   // residual the last forward on this workspace kept (0: none) and the problem
@@ -64,9 +65,12 @@ struct WsLayout {
   size_t qnorm;                       // [B, H, Sq]
   size_t kbar, ksum, kcount, qdot;    // k-smoothing: center [B,H,D] fp32, its fixed-point
                                       // sums [B,H,D] int64, valid keys [B], q.c [B,H,Sq]
+  size_t kbmax, kmax_q;               // per q-block bound: [B,H_kv,nN] key-block maxima,
+                                      // [B,H,nM] each q-block's kmax (written by the forward)
   size_t fwd_end;
   size_t delta, dq_accum, sem;        // backward scratch
-  size_t o_resid;                     // [B, Sq, H, D] bf16 O rounding residual
+  size_t o_resid;                     // [B, Sq, H, D] O rounding residual, scaled e5m2 bytes
+  size_t q16, do16;                   // [B, Sq, H, D] fp16 copies of Q and dO (backward)
   size_t total;
   int nM, nN;
   int64_t nnz_cap;
@@ -114,13 +118,13 @@ cudaError_t launch_fwd(const bsa_problem &p, const MaskParams &mp, const bsa_opt
 
 cudaError_t launch_bwd(const bsa_problem &p, const MaskParams &mp, const bsa_options &o,
                        const PlanSignature &sig, const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
-                       const CUtensorMap &tdo, const void *out, const void *dout,
+                       const CUtensorMap &tdo, const void *q, const void *out, const void *dout,
                        const float *lse, void *dq, void *dk, void *dv, const WsLayout &L,
                        uint8_t *ws, cudaStream_t s);
 
-cudaError_t launch_bwd_preprocess(const bsa_problem &p, const bsa_options &o, const void *out,
-                                  const void *dout, const WsLayout &L, uint8_t *ws,
-                                  cudaStream_t s);
+cudaError_t launch_bwd_preprocess(const bsa_problem &p, const bsa_options &o, const void *q,
+                                  const void *out, const void *dout, const WsLayout &L,
+                                  uint8_t *ws, cudaStream_t s);
 
 cudaError_t launch_bwd_main(const bsa_problem &p, const MaskParams &mp, const bsa_options &o,
                             const PlanSignature &sig, const CUtensorMap &tq, const CUtensorMap &tk,

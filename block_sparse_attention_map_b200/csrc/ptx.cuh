@@ -318,6 +318,24 @@ __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
   return pack_f16x2_sat(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
 }
 
+// The O rounding residual's 8-bit storage: r * 2^12 as e5m2 (5 exponent bits,
+// 2 mantissa bits; clamped at +-57344), two values per 16 bits, lo first.  A
+// residual is at most half a bf16 ulp of its O element, so for |O| in
+// [2^-18, ~3500] it lands in e5m2's normal range and keeps 3 significant bits:
+// O + r then carries about 11 significant bits instead of bf16's 8.
+constexpr float kResidScale = 4096.f, kResidScaleInv = 1.f / 4096.f;
+__device__ __forceinline__ uint32_t pack_resid_e5m2x2(float lo, float hi) {
+  unsigned short r;
+  asm("cvt.rn.satfinite.e5m2x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi * kResidScale), "f"(lo * kResidScale));
+  return r;
+}
+__device__ __forceinline__ float2 unpack_resid_e5m2x2(uint32_t bits16) {
+  uint32_t h;
+  asm("cvt.rn.f16x2.e5m2x2 %0, %1;" : "=r"(h) : "h"(static_cast<unsigned short>(bits16)));
+  const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&h));
+  return make_float2(f.x * kResidScaleInv, f.y * kResidScaleInv);
+}
+
 __device__ __forceinline__ float2 unpack_f16x2(uint32_t x) {
   return __half22float2(*reinterpret_cast<const __half2 *>(&x));
 }

@@ -114,6 +114,16 @@ typedef enum bsa_status {
  *             depend on the order of the additions; any c keeps m_i a bound. */
 #define BSA_BOUND_NORM 0
 #define BSA_BOUND_SMOOTHED 1
+/*   BLOCK     the pages' per-segment kmax, read as: per q-block m, kmax_m = the
+ *             largest ||k_j|| over the valid keys of the kv blocks the block map
+ *             lets q-block m reach (its non-empty tiles), so segments, windows
+ *             and documents each get the bound of the keys their rows can see;
+ *             m_i = scale*||q_i||*kmax_m, and the gate is taken per row:
+ *             2*scale*||q_i||*kmax_m <= G (else that row runs online).  The
+ *             bound pass reads K only (one maximum per kv block and key head);
+ *             the forward takes ||q_i|| from its Q tile.  kmax_override is
+ *             rejected with it. */
+#define BSA_BOUND_BLOCK 2
 
 /* bsa_options.bwd_order: order pi of the kv columns for the dQ semaphores */
 #define BSA_ORDER_ASC 0
@@ -198,11 +208,13 @@ typedef struct bsa_options {
   int32_t bound_mode;          /* BSA_BOUND_*; SMOOTHED with kmax_override or with
                                   H_kv*D > 24576 is rejected                        */
   int32_t o_residual;          /* BSA_O_RESIDUAL_*: the bf16 rounding residual of O
-                                  (fp32 O - bf16 O, as bf16) that makes the
-                                  backward's Delta = rowsum(dO o O) exact to the
-                                  fp32 O instead of the rounded output.  AUTO (0)
-                                  is exact whenever a backward shares the
-                                  forward's workspace; see below.              */
+                                  (fp32 O - bf16 O, one byte per element: an
+                                  e5m2 of the residual times 2^12), with which
+                                  the backward's Delta = rowsum(dO o O) uses O
+                                  at ~11 significant bits instead of the bf16
+                                  output's 8.  AUTO (0) applies it whenever a
+                                  backward shares the forward's workspace; see
+                                  below.                                       */
 } bsa_options;
 
 /* bsa_options.o_residual.
@@ -249,7 +261,9 @@ typedef struct bsa_workspace_view {
                                   quarter of each q-block                          */
   size_t off_kbar;             /* fp32   [B, H_kv, D] k-smoothing center             */
   size_t off_qdot;             /* fp32   [B, H, Sq]   q_i . center                   */
-  size_t off_o_resid;          /* bf16   [B, Sq, H, D] O - bf16(O) (o_residual)       */
+  size_t off_o_resid;          /* u8     [B, Sq, H, D] O - bf16(O) (o_residual)       */
+  size_t off_kblk;             /* fp32   [B, H_kv, nN] per kv block max ||k_j|| (BLOCK) */
+  size_t off_kmax_q;           /* fp32   [B, H, nM]   per q-block kmax (BLOCK)         */
   int32_t nM, nN;
 } bsa_workspace_view;
 
@@ -333,16 +347,21 @@ BSA_API bsa_status bsa_plan_and_bound(const bsa_problem *prob, const bsa_mask_sp
                                       const bsa_options *opt, const void *q, const void *k,
                                       void *ws, size_t ws_bytes, bsa_stream_t stream);
 
-/* a4: Delta_i = sum_d dO_id O_id (fp32) into the workspace; zeroes the fp32 dQ
- * accumulator and the dQ semaphores. */
+/* a4: Delta_i = sum_d dO_id O_id (fp32) into the workspace (with the O
+ * residual per opt->o_residual); zeroes the dQ semaphores (and, for the atomic
+ * backward, the fp32 dQ accumulator); writes fp16 copies of q and dout into the
+ * workspace, on which bsa_bwd_main takes its products (values beyond the fp16
+ * range are reported as BSA_ERR_INPUT_RANGE). */
 BSA_API bsa_status bsa_bwd_preprocess(const bsa_problem *prob, const bsa_mask_spec *mask,
-                                      const bsa_options *opt, const void *out,
+                                      const bsa_options *opt, const void *q, const void *out,
                                       const void *dout, void *ws, size_t ws_bytes,
                                       bsa_stream_t stream);
 
 /* a5 ("Add more optimal dk order optional arg", "Sliding window perf issue"):
  * dK, dV written (bf16); dQ contributions accumulated into the workspace in
- * the order pi when opt->deterministic. */
+ * the order pi when opt->deterministic.  Reads Q and dO from the fp16 copies
+ * bsa_bwd_preprocess left in the workspace (q and dout are checked as usual),
+ * K and V from k and v. */
 BSA_API bsa_status bsa_bwd_main(const bsa_problem *prob, const bsa_mask_spec *mask,
                                 const bsa_options *opt, const void *q, const void *k,
                                 const void *v, const void *dout, const float *lse, void *dk,
@@ -405,6 +424,13 @@ BSA_API bsa_status bsa_static_scratch_status(bsa_stream_t stream, int32_t clear)
  * (BSA_OK if no device-side error was recorded); clear = 1 resets it. */
 BSA_API bsa_status bsa_get_device_status(void *ws, size_t ws_bytes, bsa_stream_t stream,
                                  int32_t clear);
+
+/* Number of query rows that the forwards on `ws` since its last plan build
+ * ran with the pinned fixed-m reference (rows of heads, q-blocks or, with
+ * BSA_BOUND_BLOCK, single rows that passed the gate); the rest ran online
+ * softmax.  Synchronises `stream`, like bsa_get_device_status.  Errors:
+ * INVALID_ARG (null or too small a workspace), CUDA. */
+BSA_API bsa_status bsa_fixed_rows(void *ws, size_t ws_bytes, bsa_stream_t stream, uint64_t *rows);
 
 /* Static description of a status code. */
 BSA_API const char *bsa_status_string(bsa_status status);

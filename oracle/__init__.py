@@ -30,7 +30,7 @@ from .attention import (  # noqa: F401
     fixed_m_bound_smoothed,
     useful_flops,
 )
-from .bound import fixed_m_bound_blocks, row_references_blocks  # noqa: F401
+from .bound import fixed_m_bound_blocks, gate_rows_blocks, row_references_blocks  # noqa: F401
 from .blockmap import (  # noqa: F401
     EMPTY,
     PARTIAL,

@@ -65,3 +65,11 @@ def row_references_blocks(q, kmax_blocks, scale: float, tile: int = 128):
     qn = np.sqrt((q ** 2).sum(axis=3)).transpose(0, 2, 1)  # [B, H, Sq]
     blk = np.arange(Sq) // tile
     return scale * qn * np.asarray(kmax_blocks)[:, :, blk]
+
+
+def gate_rows_blocks(q, kmax_blocks, scale: float, gate_limit: float = 64.0, tile: int = 128):
+    """The per-row gate of the per q-block bound, [B, H, Sq] bool: row i runs
+    fixed-m iff 2 * scale * ||q_i|| * kmax[b, h, m(i)] <= gate_limit (every
+    score of the row lies within +-scale ||q_i|| kmax, so the pinned reference
+    sits at most that far above the row's true maximum)."""
+    return 2.0 * row_references_blocks(q, kmax_blocks, scale, tile) <= gate_limit

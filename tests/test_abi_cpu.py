@@ -49,7 +49,7 @@ int main(void) {
   P(bsa_mask_spec, prefix_len) P(bsa_mask_spec, dilation)
   P(bsa_options, kmax_override) P(bsa_options, perm) P(bsa_options, sem_timeout_ns) P(bsa_options, plan_ready)
   P(bsa_options, bound_mode) P(bsa_options, o_residual) P(bsa_workspace_view, off_qdot)
-  P(bsa_workspace_view, off_o_resid) P(bsa_problem, H_kv)
+  P(bsa_workspace_view, off_o_resid) P(bsa_problem, H_kv) P(bsa_workspace_view, off_kmax_q)
   P(bsa_workspace_view, off_sem) P(bsa_workspace_view, nN)
   return 0;
 }
@@ -81,6 +81,7 @@ def test_ctypes_structs_match_c_layout():
     assert c["bsa_workspace_view.off_qdot"] == bd.WorkspaceView.off_qdot.offset
     assert c["bsa_options.o_residual"] == bd.Options.o_residual.offset
     assert c["bsa_workspace_view.off_o_resid"] == bd.WorkspaceView.off_o_resid.offset
+    assert c["bsa_workspace_view.off_kmax_q"] == bd.WorkspaceView.off_kmax_q.offset
     assert c["bsa_problem.H_kv"] == bd.Problem.H_kv.offset
     assert c["bsa_options.kmax_override"] == bd.Options.kmax_override.offset
     assert c["bsa_options.perm"] == bd.Options.perm.offset
@@ -209,13 +210,15 @@ def test_calls_reject_bad_arguments_before_cuda(L):
     o = bd.Options()
     o.bwd_order = 5
     assert L.bsa_plan_build(ctypes.byref(p), None, ctypes.byref(o), 4096, 16, None) == 1
-    # unknown bound mode; the smoothed bound with a caller-supplied kmax
+    # unknown bound mode; the smoothed and per q-block bounds with a caller-supplied kmax
     o = bd.Options()
-    o.bound_mode = 2
+    o.bound_mode = 3
     assert L.bsa_plan_build(ctypes.byref(p), None, ctypes.byref(o), 4096, 1 << 30, None) == 1
+    for mode in (1, 2):
+        o.bound_mode = mode
+        o.kmax_override = 4096
+        assert L.bsa_plan_build(ctypes.byref(p), None, ctypes.byref(o), 4096, 1 << 30, None) == 1
     o.bound_mode = 1
-    o.kmax_override = 4096
-    assert L.bsa_plan_build(ctypes.byref(p), None, ctypes.byref(o), 4096, 1 << 30, None) == 1
     o.kmax_override = None
     wide = _prob(H=200, D=128)                      # centers of 200 heads exceed shared memory
     assert L.bsa_plan_build(ctypes.byref(wide), None, ctypes.byref(o), 4096, 1 << 40, None) == 2
@@ -275,7 +278,7 @@ def test_empty_problem_is_a_checked_no_op(L):
             assert L.bsa_bwd_main(P, None, o, n, n, n, n, n, 4096, 8192, n, 0, n) == 9
         assert L.bsa_fixed_m_bound(P, None, o, n, n, n, 0, n) == 0
         assert L.bsa_plan_and_bound(P, None, o, n, n, n, 0, n) == 0
-        assert L.bsa_bwd_preprocess(P, None, o, n, n, n, 0, n) == 0
+        assert L.bsa_bwd_preprocess(P, None, o, n, n, n, n, 0, n) == 0
         assert L.bsa_bwd_convert(P, None, n, n, 0, n) == 0
         f = L.bsa_attn_fwd_static_scratch
         f.restype = ctypes.c_int32

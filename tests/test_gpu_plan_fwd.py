@@ -371,3 +371,57 @@ def test_fixed_m_at_the_gate_edge_stays_exact():
     assert el <= LSE_TOL and same
     assert float((o.float() - o_on.float()).abs().max()) <= O_TOL
     assert float((lse - lse_on).abs().max()) <= LSE_TOL
+
+
+def _gate_rows_count(wl, kmax, G=64.0):
+    """(rows the oracle's per-row gate pins, rows within 1e-3 of the limit) over
+    the q-blocks the forward visits (those with a non-empty tile)."""
+    cls = oracle.tile_classes(mask_desc(wl), wl.B, wl.Sq, wl.Skv)
+    vis = (cls != oracle.EMPTY).any(axis=2)  # [B, nM]
+    ref2 = 2.0 * oracle.row_references_blocks(np64(wl.q), kmax, wl.scale)  # [B, H, Sq]
+    blk = np.arange(wl.Sq) // 128
+    live = vis[:, None, blk]  # [B, 1, Sq]
+    live = np.broadcast_to(live, ref2.shape)
+    sure = live & (ref2 <= G * (1 - 1e-3))
+    near = live & (np.abs(ref2 - G) < G * 1e-3)
+    return int(sure.sum()), int(near.sum())
+
+
+@pytest.mark.parametrize("name", ["window", "packed", "document", "varlen", "video", "dilated", "gqa"])
+def test_block_bound_matches_oracle(name):
+    """The per q-block bound (BSA_BOUND_BLOCK): each q-block's kmax equals the
+    oracle's (the largest valid key norm over the kv blocks its row list
+    reaches), the rows the device ran fixed-m are the rows the oracle's per-row
+    gate passes, and O / LSE match the oracle."""
+    wl = make_workload(name, device="cuda", small=True)
+    eo, el, same, o, lse, ws = _fwd_vs_oracle(wl, "fixed_m", bound_mode="block")
+    assert el <= LSE_TOL and same, (eo, el, same)
+    kmax, qmax, bound, gate = oracle.fixed_m_bound_blocks(np64(wl.q), np64(wl.k), mask_desc(wl), wl.scale)
+    cls = oracle.tile_classes(mask_desc(wl), wl.B, wl.Sq, wl.Skv)
+    vis = np.broadcast_to((cls != oracle.EMPTY).any(axis=2)[:, None, :], kmax.shape)
+    got = ws.kmax_q().cpu().numpy()
+    assert np.allclose(got[vis], kmax[vis], rtol=1e-5, atol=0)
+    sure, near = _gate_rows_count(wl, kmax)
+    assert sure <= ws.fixed_rows() <= sure + near
+
+
+def test_block_bound_gates_rows_the_head_gate_sends_online():
+    """Packed segments with one hot segment (batch 0, segment 1, keys x20): the
+    per-head gate sends both heads of batch 0 to online softmax, the per
+    q-block bound pins every row of batch 0 whose q-block does not reach the
+    hot keys; the results match the oracle either way."""
+    wl = make_workload("packed", device="cuda", small=True)
+    seg0 = wl.mask["seg_kv"][0].cpu().numpy()
+    hot = torch.from_numpy(seg0 == 1).to(wl.k.device)
+    k = wl.k.float()
+    k[0, hot] *= 20.0
+    wl.k = k.to(torch.bfloat16)
+    _, _, _, _, _, ws_head = _fwd_vs_oracle(wl, "fixed_m")
+    g = ws_head.gate().cpu().numpy()
+    assert not g[0].any() and g[1].all()
+    assert ws_head.fixed_rows() == wl.H * wl.Sq  # batch 1 only
+    _, _, _, _, _, ws_blk = _fwd_vs_oracle(wl, "fixed_m", bound_mode="block")
+    kmax = oracle.fixed_m_bound_blocks(np64(wl.q), np64(wl.k), mask_desc(wl), wl.scale)[0]
+    sure, near = _gate_rows_count(wl, kmax)
+    assert sure <= ws_blk.fixed_rows() <= sure + near
+    assert ws_blk.fixed_rows() > wl.H * wl.Sq + wl.H * 128  # pinned rows in batch 0 too

@@ -71,6 +71,16 @@ def test_block_bound_closed_form_with_one_hot_segment():
     gate = oracle.fixed_m_bound_blocks(q, k, mask, scale, gate_limit=G, tile=tile)[3]
     assert gate[0][:, [0, 1, 4, 5, 6, 7]].all() and not gate[0][:, [2, 3]].any()
     assert not oracle.fixed_m_bound(q, k, mask, scale, gate_limit=G)[3].any()
+    # per row: a q-block that passes passes every one of its rows (qmax bounds
+    # each row's norm); in a failing block at least the row of largest norm fails
+    rows = oracle.gate_rows_blocks(q, kmax, scale, gate_limit=G, tile=tile)
+    for h in range(H):
+        for mb in range(S // tile):
+            r = rows[0, h, mb * tile:(mb + 1) * tile]
+            if gate[0, h, mb]:
+                assert r.all()
+            else:
+                assert not r[np.argmax(np.linalg.norm(q[0, mb * tile:(mb + 1) * tile, h], axis=1))]
 
 
 def test_fixed_m_with_block_references_equals_online():
