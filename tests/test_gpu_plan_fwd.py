@@ -406,13 +406,15 @@ def test_block_bound_matches_oracle(name):
 
 
 def test_block_bound_gates_rows_the_head_gate_sends_online():
-    """Packed segments with one hot segment (batch 0, segment 1, keys x20): the
-    per-head gate sends both heads of batch 0 to online softmax, the per
-    q-block bound pins every row of batch 0 whose q-block does not reach the
-    hot keys; the results match the oracle either way."""
+    """Packed segments with one hot segment (batch 0, its last segment, keys
+    x20): the per-head gate sends both heads of batch 0 to online softmax, the
+    per q-block bound pins every row of batch 0 whose q-block does not reach
+    the hot keys; the results match the oracle either way."""
     wl = make_workload("packed", device="cuda", small=True)
     seg0 = wl.mask["seg_kv"][0].cpu().numpy()
-    hot = torch.from_numpy(seg0 == 1).to(wl.k.device)
+    hot_np = seg0 == seg0[-1]
+    assert np.argmax(hot_np) >= 256  # the first two q-blocks see only cold keys
+    hot = torch.from_numpy(hot_np).to(wl.k.device)
     k = wl.k.float()
     k[0, hot] *= 20.0
     wl.k = k.to(torch.bfloat16)
