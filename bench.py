@@ -599,6 +599,13 @@ def run_ours(args, world, rank, local):
         line["roofline_forward"] = roof_fwd
     line.update({"gpu_launches": launches, "wall_s_timed_loop": t_wall, "clocks": clocks})
 
+    # the plan and the bound each alone, beside their overlapped call (eager,
+    # median of 10, L2 flushed before each): how much the two overlap
+    if args.softmax == "fixed_m":
+        iso = {"plan": _median_event_ms(st.plan, flush.zero_, 10, stream),
+               "bound": _median_event_ms(st.bound, flush.zero_, 10, stream),
+               "plan_and_bound": _median_event_ms(st.plan_and_bound, flush.zero_, 10, stream)}
+        line["plan_bound_isolated_ms"] = iso
     if has_bwd and not args.no_orders:
         ords = order_table(args, wl, flush, stream)
         line["backward_main_ms_by_order"] = ords
