@@ -1,23 +1,23 @@
 #!/usr/bin/env python
 """Throughput of the block-sparse attention hot path on B200.
 
-One step = the whole hot path over the causal sliding-window workload
-(B=1, H=16, Sq=Skv=8192, D=128, window 512, bf16 N(0,1), seed 2):
+One step = the whole hot path over one workload (default: the causal
+sliding-window workload, B=1, H=16, Sq=Skv=8192, D=128, window 512, bf16
+N(0,1), seed 2):
   a1+a6  block map + rank-sorted column lists      (bsa_plan_build)
-  a2     fixed-m bound and per-head gate            (bsa_fixed_m_bound)
-  a3     forward, fixed-m gated                     (bsa_attn_fwd)
-  a4     Delta, zeroed dQ accumulator / semaphores  (bsa_bwd_preprocess)
+  a2     fixed-m bound and per-head gate            (bsa_fixed_m_bound; beside a1)
+  a3     forward, fixed-m gated, O residual kept    (bsa_attn_fwd)
+  a4     Delta, fp16 copies of Q and dO, semaphores (bsa_bwd_preprocess)
   a5     deterministic backward, descending order   (bsa_bwd_main)
   a7     dQ convert                                 (bsa_bwd_convert)
+(the forward-only workloads, varlen and video: a1, a2, a3).
 Metric: useful TFLOP/s = (non-empty 128x128 tiles x per-tile flops) / time, with
 per-tile flops 4*128*128*D forward and 2.5x that backward.  L2 is flushed
-(a 256 MiB write) before every step, outside the step's events.
+before every step, outside the step's events (class L2Flush).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-
-The other mask families and kv-column orders are measured the same way with
---workload prefix_lm|dilated|document|window_rect, --order desc|outside_in|greedy
-and --nondet (the atomic dQ backward).
+                    [--workload NAME] [--softmax fixed_m|online] [--bound norm|smoothed|block]
+                    [--order desc|asc|outside_in|greedy] [--nondet] [--o-residual auto|drop]
 
 With N > 1 it runs under torch.distributed.run, one rank per GPU, every rank
 running the same workload (replicas: the (b, h) units are independent and
@@ -350,6 +350,23 @@ def run_reference(args, world, rank):
 
 # ------------------------------------------------------------------ GPU arm
 
+class L2Flush:
+    """Empties L2 between timed steps: a 256 MiB write (more than the 126 MB
+    L2), then a 256 MiB read of a second buffer.  The write alone leaves L2
+    full of dirty lines whose write-back the next step's first kernel would pay
+    for; after the read, L2 holds clean lines of the flush buffer only."""
+
+    def __init__(self, dev):
+        import torch
+        self.w = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+        self.r = torch.zeros(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+        self.acc = torch.zeros((), dtype=torch.float32, device=dev)
+
+    def __call__(self):
+        self.w.zero_()
+        self.acc.copy_(self.r.sum())
+
+
 def _median_event_ms(fn, before, n, stream):
     """Median CUDA-event time of fn() over n runs, before() (untimed: an L2 flush,
     a stage the timed one depends on) ahead of each."""
@@ -380,7 +397,7 @@ def order_table(args, wl, flush, stream, n=10):
         st.forward()
 
         def before():
-            flush.zero_()
+            flush()
             st.preprocess(wl.dO)
 
         out[name] = _median_event_ms(lambda: st.backward_main(wl.dO), before, n, stream)
@@ -401,7 +418,7 @@ def softmax_table(args, wl, flush, stream, n=10):
         st.plan_and_bound()
         st.forward()
         fixed_rows = st.ws.fixed_rows()  # one forward since the plan build
-        out[mode] = _median_event_ms(st.forward, flush.zero_, n, stream)
+        out[mode] = _median_event_ms(st.forward, flush, n, stream)
         if st.ws.status() != 0:
             raise RuntimeError(f"device status {st.ws.status()} timing the {mode} forward")
         if mode == "fixed_m":
@@ -424,7 +441,7 @@ def run_ours(args, world, rank, local):
     st = bsa.Stages(wl.q, wl.k, wl.v, wl.mask, softmax_mode=args.softmax, order=args.order,
                     deterministic=not args.nondet, bound_mode=args.bound, o_residual=args.o_residual)
     dO = wl.dO
-    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    flush = L2Flush(dev)
     stream = torch.cuda.current_stream()
     # the planner runs beside the bound's pass over Q and K (one library call,
     # the plan on the library's side stream), then the rest in order
@@ -442,7 +459,7 @@ def run_ours(args, world, rank, local):
             ev[len(names)].record(stream)
 
     for _ in range(args.warmup):
-        flush.zero_()
+        flush()
         step()
     torch.cuda.synchronize()
     status = st.ws.status()
@@ -458,7 +475,7 @@ def run_ours(args, world, rank, local):
     launches0 = bsa.launch_count()
     barrier(world)
     for s in range(args.steps):
-        flush.zero_()
+        flush()
         step(events[s])
     torch.cuda.synchronize()
     barrier(world)
@@ -487,7 +504,7 @@ def run_ours(args, world, rank, local):
                 step()
             launches_per_step = bsa.launch_count() - l0
             for _ in range(args.warmup):
-                flush.zero_()
+                flush()
                 g.replay()
             torch.cuda.synchronize()
             if st.ws.status() != 0:
@@ -503,7 +520,7 @@ def run_ours(args, world, rank, local):
             ev_g = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                     for _ in range(args.steps)]
             for s in range(args.steps):
-                flush.zero_()
+                flush()
                 ev_g[s][0].record(stream)
                 graph.replay()
                 ev_g[s][1].record(stream)
@@ -511,7 +528,7 @@ def run_ours(args, world, rank, local):
             ev_e = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)] for _ in range(args.steps)]
             l0 = bsa.launch_count()
             for s in range(args.steps):
-                flush.zero_()
+                flush()
                 step(ev_e[s])
         torch.cuda.synchronize()
         t_wall = time.perf_counter() - t_wall
@@ -567,7 +584,8 @@ def run_ours(args, world, rank, local):
                    "passes": "forward + backward" if has_bwd else "forward only",
                    "o_residual": args.o_residual if has_bwd else None,
                    "bwd_order": ("nondeterministic" if args.nondet else args.order) if has_bwd else None,
-                   "l2": "flushed (256 MiB write) before every step, outside the timed events",
+                   "l2": "flushed before every step, outside the timed events: a 256 MiB write, then a 256 MiB "
+                         "read that writes the dirty lines back, so the step starts on a clean L2",
                    "parallelism": f"replicas x{world}"},
         "pct_of_bf16_peak": 100.0 * value / peak,
         "pct_of_spec_peak": 100.0 * value / spec_peak,
@@ -599,12 +617,19 @@ def run_ours(args, world, rank, local):
         line["roofline_forward"] = roof_fwd
     line.update({"gpu_launches": launches, "wall_s_timed_loop": t_wall, "clocks": clocks})
 
-    # the plan and the bound each alone, beside their overlapped call (eager,
-    # median of 10, L2 flushed before each): how much the two overlap
-    if args.softmax == "fixed_m":
-        iso = {"plan": _median_event_ms(st.plan, flush.zero_, 10, stream),
-               "bound": _median_event_ms(st.bound, flush.zero_, 10, stream),
-               "plan_and_bound": _median_event_ms(st.plan_and_bound, flush.zero_, 10, stream)}
+    # the plan and the bound each alone, beside their overlapped call, each
+    # captured into its own CUDA graph (no host gaps) and replayed: median of
+    # 10, L2 flushed before each, outside the events
+    if args.softmax == "fixed_m" and graph is not None:
+        iso = {}
+        for nm, fn in (("plan", st.plan), ("bound", st.bound), ("plan_and_bound", st.plan_and_bound)):
+            gi = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gi, capture_error_mode="thread_local"):
+                fn()
+            iso[nm] = _median_event_ms(gi.replay, flush, 10, stream)
+            del gi
+        if st.ws.status() != 0:
+            raise RuntimeError(f"device status {st.ws.status()} timing the plan and the bound")
         line["plan_bound_isolated_ms"] = iso
     if has_bwd and not args.no_orders:
         ords = order_table(args, wl, flush, stream)

@@ -462,7 +462,7 @@ bsa_status attn_fwd_impl(const bsa_problem *prob, const bsa_mask_spec *mask,
   const bool keep = P.o.o_residual == BSA_O_RESIDUAL_KEEP ||
                     (P.o.o_residual == BSA_O_RESIDUAL_AUTO && ws_bytes >= P.L.total);
   fo.o_residual = keep ? BSA_O_RESIDUAL_KEEP : BSA_O_RESIDUAL_DROP;
-  return cuda_status(launch_fwd(p, mp, fo, signature(p, P.m, P.o), tq, tk, tv, out, lse, P.L, w, s));
+  return cuda_status(launch_fwd(p, mp, fo, signature(p, P.m, P.o), tq, tk, tv, q, out, lse, P.L, w, s));
 }
 
 }  // namespace bsa

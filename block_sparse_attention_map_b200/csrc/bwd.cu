@@ -895,6 +895,14 @@ __global__ void __launch_bounds__(256) k_bwd_delta(const DeltaArgs a) {
                 hdr[kHdrResidH] == static_cast<uint32_t>(H) && hdr[kHdrResidSq] == static_cast<uint32_t>(Sq) &&
                 hdr[kHdrResidSkv] == static_cast<uint32_t>(a.Skv) && hdr[kHdrResidD] == static_cast<uint32_t>(D);
   }
+  // the forward that kept this residual also wrote the fp16 copy of Q, if its
+  // record names this very q (pointer and strides): Q need not be read again
+  bool have_q16 = false;
+  if (RESID && use_resid) {
+    const uint64_t qtag = (static_cast<uint64_t>(hdr[kHdrQ16Hi]) << 32) | hdr[kHdrQ16Lo];
+    have_q16 = qtag == reinterpret_cast<uint64_t>(a.q) && hdr[kHdrQ16Sb] == static_cast<uint32_t>(a.qb) &&
+               hdr[kHdrQ16Ss] == static_cast<uint32_t>(a.qs) && hdr[kHdrQ16Sh] == static_cast<uint32_t>(a.qh);
+  }
   for (int64_t z = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; z < a.n_sem;
        z += static_cast<int64_t>(gridDim.x) * blockDim.x)
     a.sem[z] = 0u;
@@ -922,7 +930,8 @@ __global__ void __launch_bounds__(256) k_bwd_delta(const DeltaArgs a) {
       const int64_t off = b * a.sb + static_cast<int64_t>(i) * a.ss + h * a.sh + t * 8;
       av[j] = __ldg(reinterpret_cast<const int4 *>(a.o + off));
       cv[j] = __ldg(reinterpret_cast<const int4 *>(a.dout + off));
-      qv[j] = __ldcs(reinterpret_cast<const int4 *>(a.q + b * a.qb + static_cast<int64_t>(i) * a.qs + h * a.qh + t * 8));
+      if (!have_q16)
+        qv[j] = __ldcs(reinterpret_cast<const int4 *>(a.q + b * a.qb + static_cast<int64_t>(i) * a.qs + h * a.qh + t * 8));
       if (use_resid)
         rv[j] = __ldg(reinterpret_cast<const uint2 *>(a.resid + ((static_cast<int64_t>(b) * Sq + i) * H + h) * D + t * 8));
     }
@@ -945,7 +954,7 @@ __global__ void __launch_bounds__(256) k_bwd_delta(const DeltaArgs a) {
         hq[q] = bf16x2_to_f16x2(xq[q]);
         hd[q] = bf16x2_to_f16x2(xd[q]);
       }
-      *reinterpret_cast<int4 *>(a.q16 + off) = make_int4(hq[0], hq[1], hq[2], hq[3]);
+      if (!have_q16) *reinterpret_cast<int4 *>(a.q16 + off) = make_int4(hq[0], hq[1], hq[2], hq[3]);
       *reinterpret_cast<int4 *>(a.do16 + off) = make_int4(hd[0], hd[1], hd[2], hd[3]);
     }
   }

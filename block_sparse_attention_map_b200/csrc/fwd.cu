@@ -68,6 +68,9 @@ struct FwdParams {
   const float *qnorm;  // [B, H, Sq]
   const float *qdot;   // [B, H, Sq] q_i . center with k-smoothing, else null
   uint8_t *o_resid;  // [B, Sq, H, D] O - bf16(O) as scaled e5m2 bytes, or null
+  const __nv_bfloat16 *q;  // the caller's Q (recorded with its fp16 copy)
+  int64_t q_sb, q_ss, q_sh;
+  __half *q16;       // [B, Sq, H, D] fp16 copy of Q for the backward (with the residual), or null
   const int32_t *gate; // [B, H]
   uint32_t *hdr;
   uint64_t timeout_ns;
@@ -169,6 +172,9 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       uint32_t cnt = 1;
       if ((i >= L::bPFull && i < L::bPFull + 2) || (i >= L::bSegReady && i < L::bSegReady + 4))
         cnt = 128;
+      // a Q slot is free once the unit's MMAs are done and, when the fp16
+      // copy is written, warps 2-3 have read it
+      if (i >= L::bQEmpty && i < L::bQEmpty + NQ && p.q16 != nullptr) cnt = 1 + 64;
       mbar_init(&bars[i], cnt);
     }
     *abort_flag = 0;
@@ -207,6 +213,12 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       p.hdr[kHdrResidSq] = p.Sq;
       p.hdr[kHdrResidSkv] = p.Skv;
       p.hdr[kHdrResidD] = D;
+      const uint64_t qtag = (ok && p.q16 != nullptr) ? reinterpret_cast<uint64_t>(p.q) : 0ull;
+      p.hdr[kHdrQ16Lo] = static_cast<uint32_t>(qtag);
+      p.hdr[kHdrQ16Hi] = static_cast<uint32_t>(qtag >> 32);
+      p.hdr[kHdrQ16Sb] = static_cast<uint32_t>(p.q_sb);
+      p.hdr[kHdrQ16Ss] = static_cast<uint32_t>(p.q_ss);
+      p.hdr[kHdrQ16Sh] = static_cast<uint32_t>(p.q_sh);
     }
   }
   __syncthreads();
@@ -359,6 +371,56 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       // every tcgen05 op this thread issued is complete before TMEM is freed
       mma_commit(&bars[L::bFinal]);
       drain_wait(&bars[L::bFinal], 0);
+    }
+  } else if (warp == 2 || warp == 3) {
+    // ------------------------------------------------------------ fp16 Q (warps 2, 3)
+    // When the forward keeps the O residual (a backward is expected on this
+    // workspace), each Q tile it loads is also written out as fp16 for the
+    // backward's products, while it sits in shared memory: the backward's
+    // Delta pass then need not read Q again.  16-byte pieces, a row's pieces
+    // on consecutive threads; the slot is released to the producer only after
+    // these reads (its empty barrier counts them).
+    if (p.q16 != nullptr) {
+      const int ct = threadIdx.x - 64;
+      auto wwait = [&](uint64_t *bar, uint32_t parity) {
+        return __all_sync(0xffffffffu, wd.wait(bar, parity)) != 0;
+      };
+      constexpr int kCpr = D / 8;  // 16-byte pieces per row
+      uint32_t qm = 0, in_max = 0;
+      bool stop = false;
+      for (int u = blockIdx.x; u < p.n_units && !stop; u += gridDim.x) {
+        const FwdUnit w = decode_unit(p, u);
+#pragma unroll 1
+        for (int x = 0; x < 2; ++x) {
+          if (w.re[x] <= w.rs[x]) continue;
+          const uint32_t qs = qm % NQ, par = (qm / NQ) & 1;
+          ++qm;
+          if (!wwait(&bars[L::bQFull + qs], par)) { stop = true; break; }
+          const uint8_t *tile = sm + L::kQ + qs * kTB;
+#pragma unroll 4
+          for (int idx = ct; idx < kTile * kCpr; idx += 64) {
+            const int r = idx / kCpr, piece = idx % kCpr, c = piece >> 3, k8 = piece & 7;
+            const int i = w.m[x] * kTile + r;
+            const int4 v = *reinterpret_cast<const int4 *>(tile + c * 16384 + r * 128 + ((k8 ^ (r & 7)) << 4));
+            if (i < p.Sq) {
+              const uint32_t xw[4] = {static_cast<uint32_t>(v.x), static_cast<uint32_t>(v.y),
+                                      static_cast<uint32_t>(v.z), static_cast<uint32_t>(v.w)};
+              uint32_t hw[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                in_max = __vmaxu2(in_max, xw[e] & 0x7fff7fffu);
+                hw[e] = bf16x2_to_f16x2(xw[e]);
+              }
+              *reinterpret_cast<int4 *>(p.q16 + ((static_cast<int64_t>(w.b) * p.Sq + i) * p.H + w.h) * D +
+                                        piece * 8) = make_int4(hw[0], hw[1], hw[2], hw[3]);
+            }
+          }
+          mbar_arrive(&bars[L::bQEmpty + qs]);
+        }
+      }
+      // |x| >= 65536 (bf16 bits 0x4780), infinities and NaNs: beyond what fp16 holds
+      if ((in_max & 0xffffu) >= 0x4780u || (in_max >> 16) >= 0x4780u)
+        record_status(p.hdr + kHdrStatus, BSA_ERR_INPUT_RANGE);
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------ softmax, group x
@@ -730,22 +792,24 @@ __global__ void __launch_bounds__(256) k_key_sums(const NormArgs a) {
 
 // Per q-block bound, its only pass over the inputs: for each kv block n and key
 // head, the largest ||k_j|| over the block's valid keys (padding and varlen
-// alignment keys excluded; 0 when none is valid).  One warp per (b, hk, n):
-// lane l takes keys l, l+32, l+64, l+96 of the block, each row's 16-byte
-// pieces all in flight.
+// alignment keys excluded; 0 when none is valid).  One warp per (b, hk, n,
+// 32-key quarter): lane l takes key 32 c + l of the block, the row's 16-byte
+// pieces all in flight; the warp's maximum goes into the block's slot with an
+// integer atomic max (non-negative floats order like their bit patterns; the
+// slots are zeroed before the launch).
 template <int D>
 __global__ void __launch_bounds__(256) k_key_block_max(const NormArgs a, float *__restrict__ kblk, int nN) {
   const int64_t wid = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
-  if (wid >= static_cast<int64_t>(a.B) * a.Hk * nN) return;
-  const int n = static_cast<int>(wid % nN);
-  const int hk = static_cast<int>((wid / nN) % a.Hk);
-  const int b = static_cast<int>(wid / (static_cast<int64_t>(nN) * a.Hk));
+  if (wid >= static_cast<int64_t>(a.B) * a.Hk * nN * 4) return;
+  const int64_t blk = wid >> 2;
+  const int c = static_cast<int>(wid & 3);
+  const int n = static_cast<int>(blk % nN);
+  const int hk = static_cast<int>((blk / nN) % a.Hk);
+  const int b = static_cast<int>(blk / (static_cast<int64_t>(nN) * a.Hk));
   float mx = 0.f;
-#pragma unroll 1
-  for (int c = 0; c < 4; ++c) {
-    const int j = n * kTile + lane + 32 * c;
-    if (j >= a.Skv || !key_is_valid(a.mk, b, j)) continue;
+  const int j = n * kTile + lane + 32 * c;
+  if (j < a.Skv && key_is_valid(a.mk, b, j)) {
     const int4 *src = reinterpret_cast<const int4 *>(a.k + b * a.ks[0] + static_cast<int64_t>(j) * a.ks[1] +
                                                      hk * a.ks[2]);
     int4 v[D / 8];
@@ -763,11 +827,11 @@ __global__ void __launch_bounds__(256) k_key_block_max(const NormArgs a, float *
         acc = fmaf(f2.y, f2.y, acc);
       }
     }
-    mx = fmaxf(mx, sqrtf(acc));
+    mx = sqrtf(acc);
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-  if (lane == 0) kblk[wid] = mx;
+  if (lane == 0 && mx > 0.f) atomicMax(reinterpret_cast<unsigned int *>(kblk) + blk, __float_as_uint(mx));
 }
 
 // k-smoothing, second pass: the centers c = sum * 2^-20 / (valid keys).
@@ -990,9 +1054,11 @@ cudaError_t launch_fixed_m_bound(const bsa_problem &p, const MaskParams &mp,
   na.gate = reinterpret_cast<int32_t *>(ws + L.gate);
   if (o.bound_mode == BSA_BOUND_BLOCK) {
     // the per q-block bound reads K only; the forward takes the rest
-    const int64_t warps = static_cast<int64_t>(p.B) * p.H_kv * L.nN;
+    const int64_t warps = static_cast<int64_t>(p.B) * p.H_kv * L.nN * 4;
     const unsigned blocks = static_cast<unsigned>((warps * 32 + 255) / 256);
     float *kblk = reinterpret_cast<float *>(ws + L.kbmax);
+    cudaError_t e0 = cudaMemsetAsync(kblk, 0, sizeof(float) * static_cast<size_t>(p.B) * p.H_kv * L.nN, s);
+    if (e0 != cudaSuccess) return e0;
     if (p.D == 64) k_key_block_max<64><<<blocks, 256, 0, s>>>(na, kblk, L.nN);
     else k_key_block_max<128><<<blocks, 256, 0, s>>>(na, kblk, L.nN);
     count_launch();
@@ -1017,11 +1083,15 @@ cudaError_t launch_fixed_m_bound(const bsa_problem &p, const MaskParams &mp,
     }
     count_launch(2);
   }
-  // blocks per batch row: about four per SM over the whole grid, and no more
-  // than the larger tensor's vectors fill at 256 / (D / 32) per block
+  // blocks per batch row: about two per SM over the whole grid (each thread
+  // keeps eight 16-byte loads in flight, which covers the memory latency), and
+  // no more than the larger tensor's vectors fill at 256 / (D / 32) per block.
+  // Two leave an SM's other half of threads and registers to the planner,
+  // which runs beside this pass on the library's side stream; four measured
+  // the same pass time but kept the planner waiting for a free SM.
   const int64_t vec = static_cast<int64_t>(std::max(p.Sq * p.H, p.Skv * p.H_kv));
   const int64_t vpb = 256 / (p.D / 32);
-  const int64_t want = std::max<int64_t>(1, (4 * 148) / (static_cast<int64_t>(p.B) * (na.only_q ? 1 : 2)));
+  const int64_t want = std::max<int64_t>(1, (2 * 148) / (static_cast<int64_t>(p.B) * (na.only_q ? 1 : 2)));
   const int bpb = static_cast<int>(std::min<int64_t>(want, (vec + vpb - 1) / vpb));
   const dim3 grid(static_cast<unsigned>(p.B * bpb), na.only_q ? 1u : 2u);
   if (p.D == 64) {
@@ -1037,9 +1107,10 @@ cudaError_t launch_fixed_m_bound(const bsa_problem &p, const MaskParams &mp,
 
 cudaError_t launch_fwd(const bsa_problem &p, const MaskParams &mp, const bsa_options &o,
                        const PlanSignature &sig, const CUtensorMap &tq, const CUtensorMap &tk,
-                       const CUtensorMap &tv, void *out, float *lse, const WsLayout &L,
-                       uint8_t *ws, cudaStream_t s) {
+                       const CUtensorMap &tv, const void *q, void *out, float *lse,
+                       const WsLayout &L, uint8_t *ws, cudaStream_t s) {
   FwdParams fp{};
+  fp.q = static_cast<const __nv_bfloat16 *>(q);
   fp.mask = mp;
   fp.B = p.B;
   fp.H = p.H;
@@ -1075,6 +1146,11 @@ cudaError_t launch_fwd(const bsa_problem &p, const MaskParams &mp, const bsa_opt
   fp.qnorm = reinterpret_cast<const float *>(ws + L.qnorm);
   fp.qdot = o.bound_mode == BSA_BOUND_SMOOTHED ? reinterpret_cast<const float *>(ws + L.qdot) : nullptr;
   fp.o_resid = o.o_residual == BSA_O_RESIDUAL_KEEP ? ws + L.o_resid : nullptr;
+  // the fp16 copy of Q for the backward goes with the residual
+  fp.q16 = fp.o_resid != nullptr ? reinterpret_cast<__half *>(ws + L.q16) : nullptr;
+  fp.q_sb = p.q_stride[0];
+  fp.q_ss = p.q_stride[1];
+  fp.q_sh = p.q_stride[2];
   fp.gate = reinterpret_cast<const int32_t *>(ws + L.gate);
   fp.hdr = reinterpret_cast<uint32_t *>(ws + L.status);
   fp.timeout_ns = 2000000000ull;

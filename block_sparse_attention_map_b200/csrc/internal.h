@@ -39,7 +39,16 @@ enum HeaderWord : int {
   kHdrNSeqs = 11,
   kHdrDilation = 12,
   kHdrFixedRows = 13,  // query rows the forwards since the plan build ran with a pinned reference
-  kHdrPlanWords = 56,  // words [0, 56) are reset by every plan build
+  kHdrPlanWords = 48,  // words [0, 48) are reset by every plan build
+  // The fp16-Q record (kept across plan builds): the `q` pointer and strides
+  // whose fp16 copy the last forward on this workspace wrote (pointer 0: none);
+  // it is written only together with the O residual, whose record below holds
+  // the problem.
+  kHdrQ16Lo = 48,
+  kHdrQ16Hi = 49,
+  kHdrQ16Sb = 50,
+  kHdrQ16Ss = 51,
+  kHdrQ16Sh = 52,
   // The O-residual record (kept across plan builds): the `out` pointer whose
   // residual the last forward on this workspace kept (0: none) and the problem
   // it was kept for, whose layout places the residual.
@@ -113,8 +122,8 @@ cudaError_t launch_fixed_m_bound(const bsa_problem &p, const MaskParams &mp,
 
 cudaError_t launch_fwd(const bsa_problem &p, const MaskParams &mp, const bsa_options &o,
                        const PlanSignature &sig, const CUtensorMap &tq, const CUtensorMap &tk,
-                       const CUtensorMap &tv, void *out, float *lse, const WsLayout &L,
-                       uint8_t *ws, cudaStream_t s);
+                       const CUtensorMap &tv, const void *q, void *out, float *lse,
+                       const WsLayout &L, uint8_t *ws, cudaStream_t s);
 
 cudaError_t launch_bwd(const bsa_problem &p, const MaskParams &mp, const bsa_options &o,
                        const PlanSignature &sig, const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,

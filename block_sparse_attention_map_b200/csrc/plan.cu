@@ -86,12 +86,12 @@ struct ClassifyArgs {
 
 // Tile class of (b, m, n): the AND-combination of one class per enabled
 // predicate (EMPTY if any predicate is empty, FULL if all are full).  The
-// window (with its prefix), padding and out-of-range columns are classified
-// analytically and exactly over the tile's in-range rows and columns; a
-// dilated window and segment ids only through bounds (the undilated band,
-// per-block [min, max] id intervals).  *exact is cleared when the PARTIAL
-// answer may be wrong: a bound-only predicate, or two predicates that are
-// each partial (their allowed parts may not meet).
+// window (with its prefix and its dilation), padding and out-of-range columns
+// are classified exactly over the tile's in-range rows and columns, in closed
+// form; segment ids only through bounds (per-block [min, max] id intervals).
+// *exact is cleared when the PARTIAL answer may be wrong: a bound-only
+// predicate, or two predicates that are each partial (their allowed parts may
+// not meet).
 __device__ __forceinline__ uint8_t tile_class(const ClassifyArgs &a, int b, int m, int n,
                                               bool *exact) {
   const int i0 = m * kTile, i1 = min(a.Sq, i0 + kTile) - 1;
@@ -116,10 +116,22 @@ __device__ __forceinline__ uint8_t tile_class(const ClassifyArgs &a, int b, int 
     bool all = pre_all || band_all(ja);
     if (!any) return BSA_TILE_EMPTY;
     if (a.dilation > 1 && !pre_all) {
+      // the dilated band over the columns the prefix does not cover: every
+      // distance t = i + o - j in [i0 + o - jv1, i1 + o - ja] occurs in the
+      // tile (i and j each run over a range), so the tile holds a kept key iff
+      // that range cut to the band [0, W) holds a multiple of d; it is never
+      // full unless that part is a single element, which is checked element
+      // by element
+      bool dil_any = false;
+      if (ja <= jv1) {
+        const int d = a.dilation;
+        const int lo = max(i0 + o - jv1, 0);
+        const int hi = W > 0 ? min(i1 + o - ja, W - 1) : i1 + o - ja;
+        dil_any = lo <= hi && (hi / d) * d >= lo;
+      }
+      if (!pre_any && !dil_any) return BSA_TILE_EMPTY;
       all = false;
-      // the band is exact without a dilation; with one its kept keys may miss
-      // the tile, unless the prefix alone already makes it non-empty
-      if (!pre_any) bound_only = true;
+      if (i0 == i1 && ja == jv1) bound_only = true;
     }
     if (!all) {
       c = BSA_TILE_PARTIAL;
@@ -530,8 +542,10 @@ struct FusedPlanArgs {
 // and CSR offsets the later phases read stay in shared memory (their global
 // copies are written, never read back): the phases do not wait on global
 // round trips, which another kernel streaming through HBM beside the planner
-// would lengthen.
-__global__ void __launch_bounds__(1024, 1) k_plan_fused(FusedPlanArgs pa) {
+// would lengthen.  Held to 32 registers per thread (1024 x 32 = half an SM's
+// registers) so that it fits on an SM beside the fixed-m bound's blocks, which
+// run concurrently on the caller's stream.
+__global__ void __launch_bounds__(1024, 2) k_plan_fused(FusedPlanArgs pa) {
   extern __shared__ int32_t shm[];
   const ClassifyArgs &a = pa.ca;
   const int B = a.B, nM = a.nM, nN = a.nN, BnM = B * nM, BnN = B * nN;

@@ -302,6 +302,20 @@ def test_residual_is_used_only_for_the_output_it_was_kept_for():
     assert all(torch.equal(x, y) for x, y in zip(cleared[:3], drop[:3]))
 
 
+def test_fp16_q_from_the_forward_equals_the_delta_pass_conversion():
+    """With the O residual kept, the forward also writes the fp16 copy of Q the
+    backward's products read, and the Delta pass skips Q when the workspace's
+    record names this very q.  A backward given a copy of q (another pointer,
+    the same values) converts Q itself: the gradients are the same bits."""
+    wl = make_workload("window", device="cuda", small=True)
+    o, lse, ws = bsa.attn_fwd(wl.q, wl.k, wl.v, wl.mask)
+    a = bsa.attn_bwd(wl.q, wl.k, wl.v, o, wl.dO, lse, wl.mask, workspace=ws)
+    b = bsa.attn_bwd(wl.q.clone(), wl.k, wl.v, o, wl.dO, lse, wl.mask, workspace=ws)
+    torch.cuda.synchronize()
+    assert ws.status() == 0
+    assert all(torch.equal(x, y) for x, y in zip(a[:3], b[:3]))
+
+
 @pytest.mark.parametrize("deterministic", [True, False])
 def test_stage_calls_equal_the_composite_calls(deterministic):
     """The per-stage C-ABI calls (plan, bound, forward, Delta, backward main,
