@@ -840,6 +840,7 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+  if (threadIdx.x == 0) release_ticket(p.hdr + kHdrBwdTicket, p.hdr + kHdrBwdDone);
 }
 
 // ---------------------------------------------------------------- a4: Delta
@@ -884,8 +885,11 @@ __global__ void __launch_bounds__(256) k_bwd_delta(const DeltaArgs a) {
   // output buffer) moves Delta by no more than the bf16 O alone would.
   constexpr int TPV = D / 8;
   constexpr int VPB = 256 / TPV;
-  pdl_wait();  // O comes from the forward, launched just before
-  pdl_trigger();
+  // O comes from the forward, launched just before.  No early trigger: the
+  // backward main kernel, one persistent CTA per SM, launches as this pass's
+  // blocks leave (measured 368 -> 330 us per step on the 8192 window against
+  // a trigger here, which let its CTAs take SMs during the pass)
+  pdl_wait();
   const int B = a.B, Sq = a.Sq, H = a.H, rows_pad = a.rows_pad;
   const uint32_t *hdr = a.hdr;
   bool use_resid = false;
@@ -1188,8 +1192,8 @@ cudaError_t launch_bwd_main(const bsa_problem &p, const MaskParams &mp, const bs
       o.sem_timeout_ns > 0 ? static_cast<uint64_t>(o.sem_timeout_ns) : 1000000000ull;
   for (int i = 0; i < kSigWords; ++i) bp.sig[i] = sig.w[i];
   bp.sig_mask = (1u << kSigWords) - 1u;
-  cudaError_t e = cudaMemsetAsync(bp.hdr + kHdrBwdTicket, 0, sizeof(uint32_t), s);
-  if (e != cudaSuccess) return e;
+  // the column ticket is zero: the plan build clears it and every launch's
+  // last CTA puts it back
   return (p.D == 64) ? run_bwd_main<64, 2, 2>(bp, tq, tk, tv, tdo, s)
                      : run_bwd_main<128, 2, 2>(bp, tq, tk, tv, tdo, s);
 }

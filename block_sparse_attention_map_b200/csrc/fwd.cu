@@ -16,8 +16,12 @@
 // q-blocks (A = 2g, B = 2g+1) of one (b, h).  The CTA walks the union of the
 // two row lists, so each K/V tile is loaded once for both q-blocks.  With
 // grouped-query attention head h reads the K/V of kv head h / (H / H_kv).
-//   warp 0      TMA producer: Q_A, Q_B once per unit; K and V tiles through
-//               separate stage rings, 128-byte swizzled 64 x 128 boxes.
+// Units are handed out by an atomic ticket, so an SM whose loads wait longer
+// takes fewer of them.
+//   warp 0      ticket + TMA producer: draws a unit, decodes it into a
+//               two-slot shared ring the other roles read, then loads Q_A, Q_B
+//               once per unit and K and V tiles through separate stage rings,
+//               128-byte swizzled 64 x 128 boxes.
 //   warp 1      owns TMEM (512 columns) and issues tcgen05.mma from one lane,
 //               ping-ponging the two groups: PV_A(u), S_A(u+1), PV_B(u),
 //               S_B(u+1), so one group's softmax overlaps the other's MMAs.
@@ -28,7 +32,8 @@
 //               128-bit allowed-key mask (the window's key range thinned by
 //               its dilation, OR the prefix, AND segment ids); online
 //               mode takes the tile max in a first pass over TMEM and rescales
-//               O lazily; the epilogue writes O / l_r (bf16) and LSE.
+//               O lazily; the epilogue writes O / l_r (bf16), the O residual
+//               and LSE, 32 bytes per store.
 // TMEM columns: S_A [0,128) S_B [128,256) O_A [256,256+D) O_B [256+D,256+2D).
 #include <cfloat>
 
@@ -41,11 +46,7 @@ namespace {
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: tolerate p up to 2^8
-// a group's Q slot goes back with its last S of the unit (true) or with the
-// unit's last MMAs (false).  With three slots the next unit's Q_A loads during
-// this unit either way; the late release measured faster (78.8 vs 80.9 us on
-// the 8192 window), as it did with two slots.
-constexpr bool kEarlyQRelease = false;
+constexpr int kUnitWords = 10;  // a decoded unit in the shared ring: valid, b, h, bh, m[2], rs[2], re[2]
 
 struct FwdParams {
   MaskParams mask;
@@ -70,6 +71,7 @@ struct FwdParams {
   uint8_t *o_resid;  // [B, Sq, H, D] O - bf16(O) as scaled e5m2 bytes, or null
   const __nv_bfloat16 *q;  // the caller's Q (recorded with its fp16 copy)
   int64_t q_sb, q_ss, q_sh;
+  int o_v8;          // O rows and row strides are 32-byte aligned: one store per 16 columns
   __half *q16;       // [B, Sq, H, D] fp16 copy of Q for the backward (with the residual), or null
   const int32_t *gate; // [B, H]
   uint32_t *hdr;
@@ -86,11 +88,14 @@ struct FwdSmem {
   static constexpr int kV = kK + NK * kTB;             // V ring
   static constexpr int kSeg = kV + NV * kTB;           // int32 [group][buffer][128]
   static constexpr int kBar = kSeg + 4 * kTile * 4;
+  // bTkFull / bTkEmpty: the unit ring
   static constexpr int bQFull = 0, bQEmpty = NQ, bKFull = 2 * NQ, bKEmpty = bKFull + NK,
                        bVFull = bKEmpty + NK, bVEmpty = bVFull + NV, bSFull = bVEmpty + NV,
                        bPFull = bSFull + 2, bPVDone = bPFull + 2, bSegReady = bPVDone + 2,
-                       bFinal = bSegReady + 4, kNumBars = bFinal + 1;
-  static constexpr int kMisc = kBar + kNumBars * 8;  // tmem slot, abort flag
+                       bTkFull = bSegReady + 4, bTkEmpty = bTkFull + 2, bFinal = bTkEmpty + 2,
+                       kNumBars = bFinal + 1;
+  static constexpr int kUnit = kBar + kNumBars * 8;         // int32 [2][kUnitWords]
+  static constexpr int kMisc = kUnit + 2 * kUnitWords * 4;  // tmem slot, abort flag
   static constexpr int kAlloc = kMisc + 16;
 };
 
@@ -137,6 +142,33 @@ __device__ __forceinline__ FwdUnit decode_unit(const FwdParams &p, int u) {
   return w;
 }
 
+__device__ __forceinline__ void write_unit(int32_t *e, bool valid, const FwdUnit &w) {
+  e[0] = valid ? 1 : 0;
+  e[1] = w.b;
+  e[2] = w.h;
+  e[3] = w.bh;
+  e[4] = w.m[0];
+  e[5] = w.m[1];
+  e[6] = w.rs[0];
+  e[7] = w.rs[1];
+  e[8] = w.re[0];
+  e[9] = w.re[1];
+}
+
+// Read after the slot's full barrier (acquire); false once the tickets are spent.
+__device__ __forceinline__ bool read_unit(const int32_t *e, FwdUnit &w) {
+  w.b = e[1];
+  w.h = e[2];
+  w.bh = e[3];
+  w.m[0] = e[4];
+  w.m[1] = e[5];
+  w.rs[0] = e[6];
+  w.rs[1] = e[7];
+  w.re[0] = e[8];
+  w.re[1] = e[9];
+  return e[0] != 0;
+}
+
 // Walks the union of the two row lists in ascending kv-block order.
 struct UnionWalk {
   const uint32_t *ent;
@@ -164,6 +196,7 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::kMisc);
   int *abort_flag = reinterpret_cast<int *>(sm + L::kMisc + 4);
   int32_t *seg_sm = reinterpret_cast<int32_t *>(sm + L::kSeg);
+  int32_t *unit_ring = reinterpret_cast<int32_t *>(sm + L::kUnit);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -175,6 +208,9 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       // a Q slot is free once the unit's MMAs are done and, when the fp16
       // copy is written, warps 2-3 have read it
       if (i >= L::bQEmpty && i < L::bQEmpty + NQ && p.q16 != nullptr) cnt = 1 + 64;
+      // the unit ring's readers: the MMA lane, the eight softmax warps and,
+      // when the fp16 copy of Q is written, warps 2-3
+      if (i >= L::bTkEmpty && i < L::bTkEmpty + 2) cnt = 1 + 8 + (p.q16 != nullptr ? 2 : 0);
       mbar_init(&bars[i], cnt);
     }
     *abort_flag = 0;
@@ -222,7 +258,9 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
     }
   }
   __syncthreads();
-  pdl_trigger();  // the Delta pass of a backward may launch (it waits for our completion)
+  // no early trigger for a backward's Delta pass: it launches as our CTAs
+  // leave (an early trigger measured 2-8 us per step slower on the 8192
+  // window, gqa and document workloads)
 
   constexpr uint32_t kIdescS = idesc_bf16_f32(128, 128, 0, 0);
   constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, 0, 1);
@@ -235,8 +273,16 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
     if (lane == 0) {
       uint32_t kv = 0, qi = 0, k_issued = 0, v_issued = 0;
       bool stop = false;
-      for (int u = blockIdx.x; u < p.n_units && !stop; u += gridDim.x) {
-        const FwdUnit w = decode_unit(p, u);
+      for (uint32_t tc = 0; !stop; ++tc) {
+        const uint32_t slot = tc & 1;
+        if (tc >= 2 && !wd.wait(&bars[L::bTkEmpty + slot], ((tc >> 1) - 1) & 1)) break;
+        const int u = static_cast<int>(atomicAdd(p.hdr + kHdrFwdTicket, 1u));
+        const bool valid = u < p.n_units;
+        FwdUnit w{};
+        if (valid) w = decode_unit(p, u);
+        write_unit(unit_ring + slot * kUnitWords, valid, w);
+        mbar_arrive(&bars[L::bTkFull + slot]);
+        if (!valid) break;
         const bool has[2] = {w.re[0] > w.rs[0], w.re[1] > w.rs[1]};
         if (!has[0] && !has[1]) continue;
 #pragma unroll
@@ -290,7 +336,6 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       uint32_t kv = 0, qm = 0, tcount[2] = {0, 0};
       bool stop = false;
       uint32_t q_addr[2] = {0, 0}, q_slot[2] = {0, 0};
-      int s_left[2] = {0, 0};  // S ops of the group still to issue in this unit
       // S_x = Q_x K^T into the S columns of group x.  The previous PV_x still
       // reads P_x from those columns; tcgen05.mma ops issued by one thread
       // execute in issue order, so no completion wait is needed in between.
@@ -305,19 +350,21 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
                  sw128_desc(k_addr + off, 16, 1024), kIdescS, kk > 0);
         }
         mma_commit(&bars[L::bSFull + x]);
-        // the group's last S of the unit: its Q slot can take the next Q tile
-        if (kEarlyQRelease && --s_left[x] == 0) mma_commit(&bars[L::bQEmpty + q_slot[x]]);
         return true;
       };
-      for (int u = blockIdx.x; u < p.n_units && !stop; u += gridDim.x) {
-        const FwdUnit w = decode_unit(p, u);
+      for (uint32_t tc = 0; !stop; ++tc) {
+        const uint32_t slot = tc & 1;
+        if (!wd.wait(&bars[L::bTkFull + slot], (tc >> 1) & 1)) break;
+        FwdUnit w;
+        const bool valid = read_unit(unit_ring + slot * kUnitWords, w);
+        mbar_arrive(&bars[L::bTkEmpty + slot]);
+        if (!valid) break;
         const bool has[2] = {w.re[0] > w.rs[0], w.re[1] > w.rs[1]};
         if (!has[0] && !has[1]) continue;
         for (int x = 0; x < 2; ++x) {
           if (!has[x]) continue;
           q_slot[x] = qm % NQ;
           q_addr[x] = smem_u32(sm + L::kQ + q_slot[x] * kTB);
-          s_left[x] = w.re[x] - w.rs[x];
           if (!wd.wait(&bars[L::bQFull + q_slot[x]], (qm / NQ) & 1)) stop = true;
           ++qm;
         }
@@ -364,9 +411,8 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
         }
         if (stop) break;
         kv = kv_cur + 1;
-        if (!kEarlyQRelease)
-          for (int x = 0; x < 2; ++x)
-            if (has[x]) mma_commit(&bars[L::bQEmpty + q_slot[x]]);
+        for (int x = 0; x < 2; ++x)
+          if (has[x]) mma_commit(&bars[L::bQEmpty + q_slot[x]]);
       }
       // every tcgen05 op this thread issued is complete before TMEM is freed
       mma_commit(&bars[L::bFinal]);
@@ -388,8 +434,14 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
       constexpr int kCpr = D / 8;  // 16-byte pieces per row
       uint32_t qm = 0, in_max = 0;
       bool stop = false;
-      for (int u = blockIdx.x; u < p.n_units && !stop; u += gridDim.x) {
-        const FwdUnit w = decode_unit(p, u);
+      for (uint32_t tc = 0; !stop; ++tc) {
+        const uint32_t slot = tc & 1;
+        if (!wwait(&bars[L::bTkFull + slot], (tc >> 1) & 1)) break;
+        FwdUnit w;
+        const bool valid = read_unit(unit_ring + slot * kUnitWords, w);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[L::bTkEmpty + slot]);
+        if (!valid) break;
 #pragma unroll 1
         for (int x = 0; x < 2; ++x) {
           if (w.re[x] <= w.rs[x]) continue;
@@ -439,8 +491,14 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
     };
     uint32_t tcount = 0, ps = 0, qm = 0;
     bool stop = false;
-    for (int u = blockIdx.x; u < p.n_units && !stop; u += gridDim.x) {
-      const FwdUnit w = decode_unit(p, u);
+    for (uint32_t tc = 0; !stop; ++tc) {
+      const uint32_t slot = tc & 1;
+      if (!wwait(&bars[L::bTkFull + slot], (tc >> 1) & 1)) break;
+      FwdUnit w;
+      const bool valid = read_unit(unit_ring + slot * kUnitWords, w);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[L::bTkEmpty + slot]);
+      if (!valid) break;
       // the unit's Q tiles sit in the Q ring in load order (A, then B), as the
       // producer and the MMA warp count them
       const bool has0 = w.re[0] > w.rs[0], has1 = w.re[1] > w.rs[1];
@@ -654,15 +712,18 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
         mbar_arrive(&bars[L::bPFull + x]);
       }
       if (stop) break;
-      // epilogue: O / l_r -> bf16, LSE
+      // epilogue: O / l_r -> bf16, the O residual, LSE
       if (!wwait(&bars[L::bPVDone + x], (tcount - 1) & 1)) break;
       tc_fence_after();
       const float inv = l_r > 0.f ? 1.f / l_r : 0.f;
       __nv_bfloat16 *orow = p.out + b * p.o_sb + static_cast<int64_t>(i) * p.o_ss + h * p.o_sh;
-      float *lse_p = p.lse + static_cast<int64_t>(bh) * p.Sq + i;
+      uint8_t *rrow = p.o_resid != nullptr
+                          ? p.o_resid + ((static_cast<int64_t>(b) * p.Sq + i) * p.H + h) * D : nullptr;
       // 16-column pieces of O, the next piece's TMEM load in flight while this
-      // one is converted and stored (a wait covers every load issued before it)
-      uint32_t ob[2][16];
+      // one is converted and stored (a wait covers every load issued before
+      // it); a piece of O is one 32-byte store, two pieces' residual bytes
+      // another
+      uint32_t ob[2][16], rb[8];
       tmem_ld16(t_o, ob[0]);
       tmem_wait_ld();
 #pragma unroll
@@ -674,29 +735,33 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
 #pragma unroll
           for (int q = 0; q < 8; ++q)
             wv[q] = pack_bf16x2(__uint_as_float(o[2 * q]) * inv, __uint_as_float(o[2 * q + 1]) * inv);
-          int4 *dst = reinterpret_cast<int4 *>(orow + c * 16);
-          dst[0] = make_int4(wv[0], wv[1], wv[2], wv[3]);
-          dst[1] = make_int4(wv[4], wv[5], wv[6], wv[7]);
-          if (p.o_resid != nullptr) {
+          if (p.o_v8) {
+            st_global_v8(orow + c * 16, wv);
+          } else {
+            int4 *dst = reinterpret_cast<int4 *>(orow + c * 16);
+            dst[0] = make_int4(wv[0], wv[1], wv[2], wv[3]);
+            dst[1] = make_int4(wv[4], wv[5], wv[6], wv[7]);
+          }
+          if (rrow != nullptr) {
             // what the bf16 rounding of O dropped (exact in fp32), for the
             // backward's Delta; 16 one-byte residuals per piece
-            uint32_t rb[4];
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
               const float2 r0 = unpack_bf16x2(wv[2 * q]), r1 = unpack_bf16x2(wv[2 * q + 1]);
-              rb[q] = pack_resid_e5m2x2(__uint_as_float(o[4 * q]) * inv - r0.x,
-                                        __uint_as_float(o[4 * q + 1]) * inv - r0.y) |
-                      (pack_resid_e5m2x2(__uint_as_float(o[4 * q + 2]) * inv - r1.x,
-                                         __uint_as_float(o[4 * q + 3]) * inv - r1.y)
-                       << 16);
+              rb[(c & 1) * 4 + q] =
+                  pack_resid_e5m2x2(__uint_as_float(o[4 * q]) * inv - r0.x,
+                                    __uint_as_float(o[4 * q + 1]) * inv - r0.y) |
+                  (pack_resid_e5m2x2(__uint_as_float(o[4 * q + 2]) * inv - r1.x,
+                                     __uint_as_float(o[4 * q + 3]) * inv - r1.y)
+                   << 16);
             }
-            *reinterpret_cast<int4 *>(p.o_resid + ((static_cast<int64_t>(b) * p.Sq + i) * p.H + h) * D + c * 16) =
-                make_int4(rb[0], rb[1], rb[2], rb[3]);
+            if (c & 1) st_global_v8(rrow + (c - 1) * 16, rb);
           }
         }
         if (c + 1 < D / 16) tmem_wait_ld();
       }
       tc_fence_before();
+      float *lse_p = p.lse + static_cast<int64_t>(bh) * p.Sq + i;
       if (row_ok) *lse_p = l > 0.f ? (m_ref + __log2f(l)) * kLn2 : -INFINITY;
       if (fixed && l > 0.f && l < 7.888609052210118e-31f /* 2^-100 */)
         atomicAdd(p.hdr + kHdrGateWarn, 1u);
@@ -709,6 +774,7 @@ k_attn_fwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+  if (threadIdx.x == 0) release_ticket(p.hdr + kHdrFwdTicket, p.hdr + kHdrFwdDone);
 }
 
 // ---------------------------------------------------------------- fixed-m bound
@@ -1014,6 +1080,8 @@ cudaError_t run_fwd(const FwdParams &fp, const CUtensorMap &tq, const CUtensorMa
     if (e != cudaSuccess) return e;
     attr = true;
   }
+  // the unit ticket is zero: the plan build clears it and every launch's
+  // last CTA puts it back
   const int grid = std::min(fp.n_units, sm_count());
   k_attn_fwd<D, NQ, NK, NV><<<grid, 384, L::kAlloc, s>>>(tq, tk, tv, fp);
   count_launch();
@@ -1134,6 +1202,8 @@ cudaError_t launch_fwd(const bsa_problem &p, const MaskParams &mp, const bsa_opt
   fp.o_sb = p.o_stride[0];
   fp.o_ss = p.o_stride[1];
   fp.o_sh = p.o_stride[2];
+  fp.o_v8 = (reinterpret_cast<uintptr_t>(out) & 31u) == 0 && p.o_stride[0] % 16 == 0 &&
+            p.o_stride[1] % 16 == 0 && p.o_stride[2] % 16 == 0;
   fp.lse = lse;
   fp.fixed_mode = o.softmax_mode == BSA_SOFTMAX_FIXED_M_GATED;
   fp.block_bound = o.bound_mode == BSA_BOUND_BLOCK;

@@ -39,6 +39,8 @@ enum HeaderWord : int {
   kHdrNSeqs = 11,
   kHdrDilation = 12,
   kHdrFixedRows = 13,  // query rows the forwards since the plan build ran with a pinned reference
+  kHdrFwdDone = 14,    // forward CTAs finished; the last one puts both forward words back to 0
+  kHdrBwdDone = 15,    // the same for the backward's column ticket
   kHdrPlanWords = 48,  // words [0, 48) are reset by every plan build
   // The fp16-Q record (kept across plan builds): the `q` pointer and strides
   // whose fp16 copy the last forward on this workspace wrote (pointer 0: none);

@@ -207,7 +207,7 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       : "memory");
 }
 
-// 32 lanes x 16 columns store (used for half-width P chunks).
+// 32 lanes x 8 columns store (half-width P chunks are 8 packed columns).
 __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
@@ -225,7 +225,27 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       : "memory");
 }
 
+// One 32-byte global store (the address is 32-byte aligned).
+__device__ __forceinline__ void st_global_v8(void *ptr, const uint32_t (&v)[8]) {
+  asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(ptr), "r"(v[0]), "r"(v[1]),
+               "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+               : "memory");
+}
+
 // ------------------------------------------------------------------ global sync
+// Called by one thread of every CTA as it leaves a persistent kernel whose
+// work is drawn from the ticket word: the last CTA out puts the ticket and
+// the exit count back to zero, so the next launch on this workspace starts
+// from ticket 0 without a memset between the kernels.  Every CTA reaches
+// its end, the aborted paths too (all waits are bounded).
+__device__ __forceinline__ void release_ticket(uint32_t *ticket, uint32_t *done) {
+  __threadfence();
+  if (atomicAdd(done, 1u) == gridDim.x - 1) {
+    atomicExch(ticket, 0u);
+    atomicExch(done, 0u);
+  }
+}
+
 __device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t *p) {
   uint32_t v;
   asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
