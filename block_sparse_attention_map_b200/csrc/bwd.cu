@@ -846,13 +846,6 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
 // ---------------------------------------------------------------- a4: Delta
 constexpr int kDeltaRuns = 2;  // runs of consecutive rows per block, loads all in flight
 
-// Half the spacing of bf16 numbers in the binade of the bf16 value with these
-// 16 bits, 2^(e - 135) for biased exponent e (clamped for subnormals and zero).
-__device__ __forceinline__ float half_ulp_bf16(uint32_t bits) {
-  const uint32_t e = (bits >> 7) & 0xffu;
-  return __uint_as_float((max(e, 9u) - 8u) << 23);
-}
-
 struct DeltaArgs {
   const __nv_bfloat16 *o, *dout, *q;
   int64_t sb, ss, sh;     // O and dO strides
@@ -940,52 +933,62 @@ __global__ void __launch_bounds__(256) k_bwd_delta(const DeltaArgs a) {
         rv[j] = __ldg(reinterpret_cast<const uint2 *>(a.resid + ((static_cast<int64_t>(b) * Sq + i) * H + h) * D + t * 8));
     }
   }
-  // fp16 copies of Q and dO, contiguous [B, Sq, H, D]
+  // fp16 copies of Q and dO, contiguous [B, Sq, H, D], and the dot products;
+  // dO is unpacked once for both
   uint32_t in_max = 0;
+  float accs[kDeltaRuns];
 #pragma unroll
   for (int j = 0; j < kDeltaRuns; ++j) {
     const int i = i0 + j * VPB;
-    if (in[j] && i < Sq) {
-      const int64_t off = ((static_cast<int64_t>(b) * Sq + i) * H + h) * (D / 2) + t * 4;
+    const bool row = in[j] && i < Sq;
+    const int64_t off = ((static_cast<int64_t>(b) * Sq + i) * H + h) * (D / 2) + t * 4;
+    if (row && !have_q16) {
       const uint32_t xq[4] = {static_cast<uint32_t>(qv[j].x), static_cast<uint32_t>(qv[j].y),
                               static_cast<uint32_t>(qv[j].z), static_cast<uint32_t>(qv[j].w)};
-      const uint32_t xd[4] = {static_cast<uint32_t>(cv[j].x), static_cast<uint32_t>(cv[j].y),
-                              static_cast<uint32_t>(cv[j].z), static_cast<uint32_t>(cv[j].w)};
-      uint32_t hq[4], hd[4];
+      uint32_t hq[4];
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        in_max = __vmaxu2(in_max, __vmaxu2(xq[q] & 0x7fff7fffu, xd[q] & 0x7fff7fffu));
+        in_max = __vmaxu2(in_max, xq[q] & 0x7fff7fffu);
         hq[q] = bf16x2_to_f16x2(xq[q]);
-        hd[q] = bf16x2_to_f16x2(xd[q]);
       }
-      if (!have_q16) *reinterpret_cast<int4 *>(a.q16 + off) = make_int4(hq[0], hq[1], hq[2], hq[3]);
-      *reinterpret_cast<int4 *>(a.do16 + off) = make_int4(hd[0], hd[1], hd[2], hd[3]);
+      *reinterpret_cast<int4 *>(a.q16 + off) = make_int4(hq[0], hq[1], hq[2], hq[3]);
     }
-  }
-  // |x| >= 65536 (bf16 bits 0x4780), infinities and NaNs: beyond what fp16 holds
-  if ((in_max & 0xffffu) >= 0x4780u || (in_max >> 16) >= 0x4780u)
-    record_status(a.hdr + kHdrStatus, BSA_ERR_INPUT_RANGE);
-#pragma unroll
-  for (int j = 0; j < kDeltaRuns; ++j) {
     const uint32_t xa[4] = {static_cast<uint32_t>(av[j].x), static_cast<uint32_t>(av[j].y),
                             static_cast<uint32_t>(av[j].z), static_cast<uint32_t>(av[j].w)};
     const uint32_t xc[4] = {static_cast<uint32_t>(cv[j].x), static_cast<uint32_t>(cv[j].y),
                             static_cast<uint32_t>(cv[j].z), static_cast<uint32_t>(cv[j].w)};
     // residual bytes of elements 2q, 2q+1: 16 bits of rv
     const uint32_t xr[4] = {rv[j].x & 0xffffu, rv[j].x >> 16, rv[j].y & 0xffffu, rv[j].y >> 16};
-    float acc = 0.f;
+    float acc = 0.f, accr = 0.f;
+    uint32_t hd[4];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      float2 fo = unpack_bf16x2(xa[q]);
+      const float2 fo = unpack_bf16x2(xa[q]);
       const float2 fd = unpack_bf16x2(xc[q]);
+      in_max = __vmaxu2(in_max, xc[q] & 0x7fff7fffu);
+      hd[q] = pack_f16x2_sat(fd.x, fd.y);
       if (use_resid) {
-        const float2 fr = unpack_resid_e5m2x2(xr[q]);
-        fo.x += fabsf(fr.x) <= half_ulp_bf16(xa[q] & 0xffffu) ? fr.x : 0.f;
-        fo.y += fabsf(fr.y) <= half_ulp_bf16(xa[q] >> 16) ? fr.y : 0.f;
+        // the residual scaled by 2^12 (its stored form), kept when |r| is at
+        // most half a bf16 ulp of its O element, 2^(e - 135) for O's exponent
+        // field e: |r 2^12| <= 2^(e - 123), the float with exponent field e + 4
+        const float2 fr = unpack_f16x2(e5m2x2_to_f16x2(xr[q]));
+        const float hu0 = __uint_as_float(((xa[q] << 16) & 0x7f800000u) + (4u << 23));
+        const float hu1 = __uint_as_float((xa[q] & 0x7f800000u) + (4u << 23));
+        accr = fmaf(fabsf(fr.x) <= hu0 ? fr.x : 0.f, fd.x, accr);
+        accr = fmaf(fabsf(fr.y) <= hu1 ? fr.y : 0.f, fd.y, accr);
       }
       acc = fmaf(fo.x, fd.x, acc);
       acc = fmaf(fo.y, fd.y, acc);
     }
+    if (row) *reinterpret_cast<int4 *>(a.do16 + off) = make_int4(hd[0], hd[1], hd[2], hd[3]);
+    accs[j] = use_resid ? fmaf(accr, kResidScaleInv, acc) : acc;
+  }
+  // |x| >= 65536 (bf16 bits 0x4780), infinities and NaNs: beyond what fp16 holds
+  if ((in_max & 0xffffu) >= 0x4780u || (in_max >> 16) >= 0x4780u)
+    record_status(a.hdr + kHdrStatus, BSA_ERR_INPUT_RANGE);
+#pragma unroll
+  for (int j = 0; j < kDeltaRuns; ++j) {
+    float acc = accs[j];
 #pragma unroll
     for (int sft = TPV / 2; sft > 0; sft >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, sft);
     if (t == 0 && in[j]) a.delta[g[j]] = acc;

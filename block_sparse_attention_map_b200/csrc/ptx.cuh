@@ -349,11 +349,11 @@ __device__ __forceinline__ uint32_t pack_resid_e5m2x2(float lo, float hi) {
   asm("cvt.rn.satfinite.e5m2x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi * kResidScale), "f"(lo * kResidScale));
   return r;
 }
-__device__ __forceinline__ float2 unpack_resid_e5m2x2(uint32_t bits16) {
+// Two stored residuals (16 bits, lo first) back to fp16x2, still scaled by 2^12.
+__device__ __forceinline__ uint32_t e5m2x2_to_f16x2(uint32_t bits16) {
   uint32_t h;
   asm("cvt.rn.f16x2.e5m2x2 %0, %1;" : "=r"(h) : "h"(static_cast<unsigned short>(bits16)));
-  const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&h));
-  return make_float2(f.x * kResidScaleInv, f.y * kResidScaleInv);
+  return h;
 }
 
 __device__ __forceinline__ float2 unpack_f16x2(uint32_t x) {
