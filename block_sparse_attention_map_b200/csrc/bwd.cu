@@ -844,7 +844,8 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
 }
 
 // ---------------------------------------------------------------- a4: Delta
-constexpr int kDeltaRuns = 2;  // runs of consecutive rows per block, loads all in flight
+constexpr int kDeltaRuns = 2;         // runs of consecutive rows per tile, loads all in flight
+constexpr int kDeltaBlocksPerSm = 3;  // the persistent grid (2 and 4 measured slower)
 
 struct DeltaArgs {
   const __nv_bfloat16 *o, *dout, *q;
@@ -860,11 +861,11 @@ struct DeltaArgs {
 };
 
 template <int D, bool RESID>
-__global__ void __launch_bounds__(256) k_bwd_delta(const DeltaArgs a) {
+__global__ void __launch_bounds__(256, 3) k_bwd_delta(const DeltaArgs a) {
   // D/8 threads per (b, h, i) row vector, 16 bytes of O, dO, Q (and the O
-  // residual) each.  A block takes kDeltaRuns runs of 256 / (D/8) consecutive
-  // rows of one head (the Delta layout), every run's loads in flight before any
-  // is reduced; rows past Sq (the last q-block's padding) get Delta = 0.  The
+  // residual) each.  A tile is kDeltaRuns runs of 256 / (D/8) consecutive rows
+  // of one head (the Delta layout), every run's loads in flight before any is
+  // reduced; rows past Sq (the last q-block's padding) get Delta = 0.  The
   // same pass writes fp16 copies of Q and dO (the backward main kernel takes
   // every product on fp16 operands) and reports values beyond the fp16 range
   // as BSA_ERR_INPUT_RANGE.  The grid also zeroes the dQ semaphores.  RESID:
@@ -904,95 +905,112 @@ __global__ void __launch_bounds__(256) k_bwd_delta(const DeltaArgs a) {
        z += static_cast<int64_t>(gridDim.x) * blockDim.x)
     a.sem[z] = 0u;
   const int t = threadIdx.x % TPV;
-  // the block's rows all belong to one (b, h): its index and first row come
-  // from one division per block, not per row
-  constexpr int kRowsPerBlock = kDeltaRuns * VPB;
-  const int blocks_per_bh = rows_pad / kRowsPerBlock;
-  const int bh = static_cast<int>(blockIdx.x) / blocks_per_bh;
-  const int i0 = (static_cast<int>(blockIdx.x) - bh * blocks_per_bh) * kRowsPerBlock + threadIdx.x / TPV;
-  const int b = bh / H, h = bh % H;
-  const bool in_bh = bh < B * H;  // uniform per block; no early return before the shuffles
-  int64_t g[kDeltaRuns];
-  bool in[kDeltaRuns];
-  int4 av[kDeltaRuns], cv[kDeltaRuns], qv[kDeltaRuns];
-  uint2 rv[kDeltaRuns];
+  // Persistent over tiles of kDeltaRuns runs of VPB consecutive rows of one
+  // (b, h) (the Delta layout), two tiles in flight: the next tile's loads are
+  // issued before this tile's conversions and dot products, so the memory
+  // system always has a tile's loads outstanding.
+  constexpr int kRowsPerTile = kDeltaRuns * VPB;
+  const int tiles_per_bh = rows_pad / kRowsPerTile;
+  const int n_tiles = B * H * tiles_per_bh;
+  struct Loaded {
+    int4 av[kDeltaRuns], cv[kDeltaRuns], qv[kDeltaRuns];
+    uint2 rv[kDeltaRuns];
+  };
+  auto load = [&](int tile, Loaded &x) {
+    const int bh = tile / tiles_per_bh;
+    const int i0 = (tile - bh * tiles_per_bh) * kRowsPerTile + threadIdx.x / TPV;
+    const int b = bh / H, h = bh % H;
 #pragma unroll
-  for (int j = 0; j < kDeltaRuns; ++j) {
-    const int i = i0 + j * VPB;
-    g[j] = static_cast<int64_t>(bh) * rows_pad + i;
-    in[j] = in_bh;
-    av[j] = cv[j] = qv[j] = make_int4(0, 0, 0, 0);
-    rv[j] = make_uint2(0u, 0u);
-    if (in[j] && i < Sq) {
-      const int64_t off = b * a.sb + static_cast<int64_t>(i) * a.ss + h * a.sh + t * 8;
-      av[j] = __ldg(reinterpret_cast<const int4 *>(a.o + off));
-      cv[j] = __ldg(reinterpret_cast<const int4 *>(a.dout + off));
-      if (!have_q16)
-        qv[j] = __ldcs(reinterpret_cast<const int4 *>(a.q + b * a.qb + static_cast<int64_t>(i) * a.qs + h * a.qh + t * 8));
-      if (use_resid)
-        rv[j] = __ldg(reinterpret_cast<const uint2 *>(a.resid + ((static_cast<int64_t>(b) * Sq + i) * H + h) * D + t * 8));
+    for (int j = 0; j < kDeltaRuns; ++j) {
+      const int i = i0 + j * VPB;
+      x.av[j] = x.cv[j] = x.qv[j] = make_int4(0, 0, 0, 0);
+      x.rv[j] = make_uint2(0u, 0u);
+      if (tile < n_tiles && i < Sq) {
+        const int64_t off = b * a.sb + static_cast<int64_t>(i) * a.ss + h * a.sh + t * 8;
+        x.av[j] = __ldg(reinterpret_cast<const int4 *>(a.o + off));
+        x.cv[j] = __ldg(reinterpret_cast<const int4 *>(a.dout + off));
+        if (!have_q16)
+          x.qv[j] = __ldcs(reinterpret_cast<const int4 *>(a.q + b * a.qb + static_cast<int64_t>(i) * a.qs + h * a.qh + t * 8));
+        if (use_resid)
+          x.rv[j] = __ldg(reinterpret_cast<const uint2 *>(a.resid + ((static_cast<int64_t>(b) * Sq + i) * H + h) * D + t * 8));
+      }
     }
-  }
-  // fp16 copies of Q and dO, contiguous [B, Sq, H, D], and the dot products;
-  // dO is unpacked once for both
+  };
   uint32_t in_max = 0;
-  float accs[kDeltaRuns];
+  auto process = [&](int tile, const Loaded &x) {
+    const int bh = tile / tiles_per_bh;
+    const int i0 = (tile - bh * tiles_per_bh) * kRowsPerTile + threadIdx.x / TPV;
+    const int b = bh / H, h = bh % H;
 #pragma unroll
-  for (int j = 0; j < kDeltaRuns; ++j) {
-    const int i = i0 + j * VPB;
-    const bool row = in[j] && i < Sq;
-    const int64_t off = ((static_cast<int64_t>(b) * Sq + i) * H + h) * (D / 2) + t * 4;
-    if (row && !have_q16) {
-      const uint32_t xq[4] = {static_cast<uint32_t>(qv[j].x), static_cast<uint32_t>(qv[j].y),
-                              static_cast<uint32_t>(qv[j].z), static_cast<uint32_t>(qv[j].w)};
-      uint32_t hq[4];
+    for (int j = 0; j < kDeltaRuns; ++j) {
+      const int i = i0 + j * VPB;
+      const bool row = i < Sq;
+      // fp16 copies of Q and dO, contiguous [B, Sq, H, D], and the dot
+      // product; dO is unpacked once for both
+      const int64_t off = ((static_cast<int64_t>(b) * Sq + i) * H + h) * (D / 2) + t * 4;
+      if (row && !have_q16) {
+        const uint32_t xq[4] = {static_cast<uint32_t>(x.qv[j].x), static_cast<uint32_t>(x.qv[j].y),
+                                static_cast<uint32_t>(x.qv[j].z), static_cast<uint32_t>(x.qv[j].w)};
+        uint32_t hq[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          in_max = __vmaxu2(in_max, xq[q] & 0x7fff7fffu);
+          hq[q] = bf16x2_to_f16x2(xq[q]);
+        }
+        *reinterpret_cast<int4 *>(a.q16 + off) = make_int4(hq[0], hq[1], hq[2], hq[3]);
+      }
+      const uint32_t xa[4] = {static_cast<uint32_t>(x.av[j].x), static_cast<uint32_t>(x.av[j].y),
+                              static_cast<uint32_t>(x.av[j].z), static_cast<uint32_t>(x.av[j].w)};
+      const uint32_t xc[4] = {static_cast<uint32_t>(x.cv[j].x), static_cast<uint32_t>(x.cv[j].y),
+                              static_cast<uint32_t>(x.cv[j].z), static_cast<uint32_t>(x.cv[j].w)};
+      // residual bytes of elements 2q, 2q+1: 16 bits of rv
+      const uint32_t xr[4] = {x.rv[j].x & 0xffffu, x.rv[j].x >> 16, x.rv[j].y & 0xffffu, x.rv[j].y >> 16};
+      float acc = 0.f, accr = 0.f;
+      uint32_t hd[4];
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        in_max = __vmaxu2(in_max, xq[q] & 0x7fff7fffu);
-        hq[q] = bf16x2_to_f16x2(xq[q]);
+        const float2 fo = unpack_bf16x2(xa[q]);
+        const float2 fd = unpack_bf16x2(xc[q]);
+        in_max = __vmaxu2(in_max, xc[q] & 0x7fff7fffu);
+        hd[q] = pack_f16x2_sat(fd.x, fd.y);
+        if (use_resid) {
+          // the residual scaled by 2^12 (its stored form), kept when |r| is at
+          // most half a bf16 ulp of its O element, 2^(e - 135) for O's exponent
+          // field e: |r 2^12| <= 2^(e - 123), the float with exponent field e + 4
+          const float2 fr = unpack_f16x2(e5m2x2_to_f16x2(xr[q]));
+          const float hu0 = __uint_as_float(((xa[q] << 16) & 0x7f800000u) + (4u << 23));
+          const float hu1 = __uint_as_float((xa[q] & 0x7f800000u) + (4u << 23));
+          accr = fmaf(fabsf(fr.x) <= hu0 ? fr.x : 0.f, fd.x, accr);
+          accr = fmaf(fabsf(fr.y) <= hu1 ? fr.y : 0.f, fd.y, accr);
+        }
+        acc = fmaf(fo.x, fd.x, acc);
+        acc = fmaf(fo.y, fd.y, acc);
       }
-      *reinterpret_cast<int4 *>(a.q16 + off) = make_int4(hq[0], hq[1], hq[2], hq[3]);
-    }
-    const uint32_t xa[4] = {static_cast<uint32_t>(av[j].x), static_cast<uint32_t>(av[j].y),
-                            static_cast<uint32_t>(av[j].z), static_cast<uint32_t>(av[j].w)};
-    const uint32_t xc[4] = {static_cast<uint32_t>(cv[j].x), static_cast<uint32_t>(cv[j].y),
-                            static_cast<uint32_t>(cv[j].z), static_cast<uint32_t>(cv[j].w)};
-    // residual bytes of elements 2q, 2q+1: 16 bits of rv
-    const uint32_t xr[4] = {rv[j].x & 0xffffu, rv[j].x >> 16, rv[j].y & 0xffffu, rv[j].y >> 16};
-    float acc = 0.f, accr = 0.f;
-    uint32_t hd[4];
+      if (row) *reinterpret_cast<int4 *>(a.do16 + off) = make_int4(hd[0], hd[1], hd[2], hd[3]);
+      if (use_resid) acc = fmaf(accr, kResidScaleInv, acc);
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const float2 fo = unpack_bf16x2(xa[q]);
-      const float2 fd = unpack_bf16x2(xc[q]);
-      in_max = __vmaxu2(in_max, xc[q] & 0x7fff7fffu);
-      hd[q] = pack_f16x2_sat(fd.x, fd.y);
-      if (use_resid) {
-        // the residual scaled by 2^12 (its stored form), kept when |r| is at
-        // most half a bf16 ulp of its O element, 2^(e - 135) for O's exponent
-        // field e: |r 2^12| <= 2^(e - 123), the float with exponent field e + 4
-        const float2 fr = unpack_f16x2(e5m2x2_to_f16x2(xr[q]));
-        const float hu0 = __uint_as_float(((xa[q] << 16) & 0x7f800000u) + (4u << 23));
-        const float hu1 = __uint_as_float((xa[q] & 0x7f800000u) + (4u << 23));
-        accr = fmaf(fabsf(fr.x) <= hu0 ? fr.x : 0.f, fd.x, accr);
-        accr = fmaf(fabsf(fr.y) <= hu1 ? fr.y : 0.f, fd.y, accr);
-      }
-      acc = fmaf(fo.x, fd.x, acc);
-      acc = fmaf(fo.y, fd.y, acc);
+      for (int sft = TPV / 2; sft > 0; sft >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, sft);
+      // rows past Sq get Delta = 0
+      if (t == 0) a.delta[static_cast<int64_t>(bh) * rows_pad + i] = acc;
     }
-    if (row) *reinterpret_cast<int4 *>(a.do16 + off) = make_int4(hd[0], hd[1], hd[2], hd[3]);
-    accs[j] = use_resid ? fmaf(accr, kResidScaleInv, acc) : acc;
+  };
+  Loaded x0, x1;
+  int tile = blockIdx.x;
+  load(tile, x0);
+  // two stages unrolled, so the buffers swap roles without copies; the loop
+  // bounds are uniform per block (every lane reaches the shuffles)
+  while (tile < n_tiles) {
+    load(tile + gridDim.x, x1);
+    process(tile, x0);
+    tile += gridDim.x;
+    if (tile >= n_tiles) break;
+    load(tile + gridDim.x, x0);
+    process(tile, x1);
+    tile += gridDim.x;
   }
   // |x| >= 65536 (bf16 bits 0x4780), infinities and NaNs: beyond what fp16 holds
   if ((in_max & 0xffffu) >= 0x4780u || (in_max >> 16) >= 0x4780u)
     record_status(a.hdr + kHdrStatus, BSA_ERR_INPUT_RANGE);
-#pragma unroll
-  for (int j = 0; j < kDeltaRuns; ++j) {
-    float acc = accs[j];
-#pragma unroll
-    for (int sft = TPV / 2; sft > 0; sft >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, sft);
-    if (t == 0 && in[j]) a.delta[g[j]] = acc;
-  }
 }
 
 // ---------------------------------------------------------------- a7: dQ convert
@@ -1113,9 +1131,11 @@ cudaError_t launch_bwd_preprocess(const bsa_problem &p, const bsa_options &o, co
   const int64_t groups = static_cast<int64_t>(p.B) * p.H * rows_pad;
   float *delta = reinterpret_cast<float *>(ws + L.delta);
   const uint8_t *resid = o.o_residual != BSA_O_RESIDUAL_DROP ? ws + L.o_resid : nullptr;
-  // kDeltaRuns runs of 256 / (D / 8) vectors per block
+  // kDeltaRuns runs of 256 / (D / 8) rows per tile; a persistent grid of
+  // kDeltaBlocksPerSm blocks per SM walks the tiles
   const int64_t vpb = kDeltaRuns * (256 / (p.D / 8));
-  const unsigned blocks = static_cast<unsigned>((groups + vpb - 1) / vpb);
+  const int64_t n_tiles = (groups + vpb - 1) / vpb;
+  const unsigned blocks = static_cast<unsigned>(std::min<int64_t>(n_tiles, kDeltaBlocksPerSm * sm_count_bwd()));
   uint32_t *sem = reinterpret_cast<uint32_t *>(ws + L.sem);
   const int64_t n_sem = static_cast<int64_t>(p.B) * p.H * L.nM * 4;  // a quarter each
   // a programmatic dependent of the forward (which reads O first after it)
