@@ -255,6 +255,10 @@ class Workspace:
         return self.buf[off:off + n].view(dtype)
 
     # inspection helpers (tests)
+    def header(self):
+        """The workspace header's 64 uint32 words (status, tickets, plan signature, records)."""
+        return self._arr(self.view.off_status, 64, torch.int32)
+
     def tile_classes(self):
         return self._arr(self.view.off_tile_class, self.B * self.nM * self.nN, torch.uint8).view(
             self.B, self.nM, self.nN)
