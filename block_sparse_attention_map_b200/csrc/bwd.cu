@@ -858,6 +858,7 @@ struct DeltaArgs {
   uint32_t *sem;
   int64_t n_sem;
   uint32_t *q16, *do16;   // [B, Sq, H, D] fp16 copies for the backward's products
+  uint32_t dq_mode;       // recorded for the dQ convert: 1 semaphore-ordered, 2 atomic
 };
 
 template <int D, bool RESID>
@@ -884,6 +885,9 @@ __global__ void __launch_bounds__(256, 3) k_bwd_delta(const DeltaArgs a) {
   // blocks leave (measured 368 -> 330 us per step on the 8192 window against
   // a trigger here, which let its CTAs take SMs during the pass)
   pdl_wait();
+  // which dQ protocol the backward main kernel will follow: the convert polls
+  // the semaphores only when they count every contribution
+  if (blockIdx.x == 0 && threadIdx.x == 0) a.hdr[kHdrDqMode] = a.dq_mode;
   const int B = a.B, Sq = a.Sq, H = a.H, rows_pad = a.rows_pad;
   const uint32_t *hdr = a.hdr;
   bool use_resid = false;
@@ -1014,51 +1018,137 @@ __global__ void __launch_bounds__(256, 3) k_bwd_delta(const DeltaArgs a) {
 }
 
 // ---------------------------------------------------------------- a7: dQ convert
-// A block per 32 rows of one q-block: the rows' slice of the interleaved
-// accumulator [B, H, nM, D/4, 128, 4] (32 consecutive float4 per column group:
-// contiguous) is read with every thread keeping its loads in flight, staged in
-// shared memory, and written as whole bf16 rows.  Q-blocks that no kv column
-// reaches get zeros.
+struct ConvertArgs {
+  const float *acc;        // the interleaved accumulator [B, H, nM, D/4, 128, 4]
+  const uint32_t *sem;     // [B, H, nM, 4] dQ semaphores
+  uint32_t *hdr;
+  const int32_t *row_ptr;
+  __nv_bfloat16 *dq;
+  int64_t sb, ss, sh;
+  int B, H, Sq, nM;
+};
+
+constexpr uint64_t kConvertPollNs = 50000000ull;  // then wait for the whole backward grid
+
+__device__ __forceinline__ uint32_t ld_relaxed_gpu(const uint32_t *p) {
+  uint32_t v;
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p));
+  return v;
+}
+
+// Polls a dQ semaphore (acquire, as the backward's contributors do) until it
+// reaches target: 1 when it did; 0 after limit_ns or once a device error has
+// been recorded, when the caller waits for the backward grid instead.
+__device__ int sem_poll(const uint32_t *sem, uint32_t target, uint64_t limit_ns,
+                        const uint32_t *status) {
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 0;; ++it) {
+    if (ld_acquire_gpu(sem) == target) return 1;
+    if ((it & 15u) == 15u) {
+      if (*reinterpret_cast<const volatile uint32_t *>(status) != 0u) return 0;
+      if (globaltimer_ns() - t0 > limit_ns) return 0;
+    }
+    __nanosleep(128);
+  }
+}
+
+// A block per 32-row quarter of one q-block: the rows' slice of the
+// interleaved accumulator (32 consecutive float4 per column group: contiguous)
+// is read with every thread keeping its loads in flight, staged in shared
+// memory, and written as whole bf16 rows.  Q-blocks that no kv column reaches
+// get zeros.
+//
+// After a semaphore-ordered backward a block does not wait for the whole
+// backward grid: the quarter's semaphore counts the contributions released so
+// far, and once it equals the length of the q-block's row list the rows are
+// final.  Blocks placed on SMs the backward's CTAs have left thus convert the
+// q-blocks already complete while its last columns still run.  Blocks take
+// the q-blocks in the order they complete (the highest first under the
+// descending column order, else the lowest first), heads interleaved.  The
+// last block to finish waits for the backward grid, so that the convert's
+// completion still implies the backward's.
 template <int D>
-__global__ void __launch_bounds__(256) k_dq_convert(const float *__restrict__ acc, int B, int H,
-                                                    int Sq, int nM, const int32_t *__restrict__ row_ptr,
-                                                    __nv_bfloat16 *__restrict__ dq,
-                                                    int64_t sb, int64_t ss, int64_t sh) {
+__global__ void __launch_bounds__(256) k_dq_convert(const ConvertArgs a) {
   constexpr int kC = D / 4, kRows = 32, kLD = D + 4;
   constexpr int kPer = kC * kRows / 256;  // float4 loads per thread
   __shared__ __align__(16) float tile[kRows * kLD];
-  pdl_wait();  // the accumulator is final once the backward main kernel completed
-  const int64_t bhm = blockIdx.x / (kTile / kRows);
-  const int r0 = static_cast<int>(blockIdx.x % (kTile / kRows)) * kRows;
-  const int m = static_cast<int>(bhm % nM);
-  const int64_t bh = bhm / nM;
-  const int b = static_cast<int>(bh / H), h = static_cast<int>(bh % H);
-  const bool empty = row_ptr[b * nM + m + 1] == row_ptr[b * nM + m];
-  const float4 *src = reinterpret_cast<const float4 *>(acc) + bhm * kC * kTile;
+  __shared__ int ready_s;
+  // launched once every backward CTA has passed its own wait for the Delta
+  // pass (and so for everything before it): the plan and the header words that
+  // pass wrote are visible here.  One round trip for all the block decides on:
+  // the header words, both candidate q-blocks' row lengths and (thread 0) their
+  // semaphores, read relaxed; thread 0 then reads the one it uses again with
+  // acquire, and the block barrier orders every thread's reads after that
+  const int64_t BH = static_cast<int64_t>(a.B) * a.H;
+  const int quarter = static_cast<int>(blockIdx.x & 3u);
+  const int64_t u = blockIdx.x >> 2;
+  const int64_t bh = u % BH;
+  const int mr = static_cast<int>(u / BH);
+  const int b = static_cast<int>(bh / a.H), h = static_cast<int>(bh % a.H);
+  const int m_asc = mr, m_desc = a.nM - 1 - mr;
+  const uint32_t mode = a.hdr[kHdrDqMode], order = a.hdr[kHdrOrder];
+  const int32_t *rp = a.row_ptr + b * a.nM;
+  const int ra0 = rp[m_asc], ra1 = rp[m_asc + 1], rd0 = rp[m_desc], rd1 = rp[m_desc + 1];
+  const uint32_t *sem_a = a.sem + (bh * a.nM + m_asc) * 4 + quarter;
+  const uint32_t *sem_d = a.sem + (bh * a.nM + m_desc) * 4 + quarter;
+  uint32_t sv_a = 0, sv_d = 0;
+  if (threadIdx.x == 0) {
+    sv_a = ld_relaxed_gpu(sem_a);
+    sv_d = ld_relaxed_gpu(sem_d);
+  }
+  const bool desc = order == static_cast<uint32_t>(BSA_ORDER_DESC);
+  const int m = desc ? m_desc : m_asc;
+  const int rl = desc ? rd1 - rd0 : ra1 - ra0;
+  const bool empty = rl == 0;
+  const int r0 = quarter * kRows;
+  if (!empty) {
+    if (threadIdx.x == 0) {
+      int ready = 0;
+      if (mode == 1u) {
+        // the relaxed read saw the last release: one acquire read of the same
+        // word then orders the block's reads after the contributions (measured
+        // faster than a fence after the relaxed read)
+        if ((desc ? sv_d : sv_a) == static_cast<uint32_t>(rl))
+          ready = ld_acquire_gpu(desc ? sem_d : sem_a) == static_cast<uint32_t>(rl) ? 1 : 0;
+        if (!ready) {
+          ready = sem_poll(desc ? sem_d : sem_a, static_cast<uint32_t>(rl), kConvertPollNs, a.hdr + kHdrStatus);
+        }
+      }
+      ready_s = ready;
+    }
+    __syncthreads();
+    // atomic adds (final once the backward main kernel completed), or a poll
+    // that gave up
+    if (!ready_s) pdl_wait();
+  }
+  const float4 *src = reinterpret_cast<const float4 *>(a.acc) + (bh * a.nM + m) * kC * kTile;
   float4 v[kPer];
 #pragma unroll
-  for (int u = 0; u < kPer; ++u) {
-    const int idx = threadIdx.x + u * 256;  // (column group, row) with rows fastest
+  for (int w = 0; w < kPer; ++w) {
+    const int idx = threadIdx.x + w * 256;  // (column group, row) with rows fastest
     const int c = idx / kRows, rr = idx % kRows;
-    v[u] = empty ? make_float4(0.f, 0.f, 0.f, 0.f) : __ldcs(src + c * kTile + r0 + rr);
+    // from L2: the contributions were reductions there
+    v[w] = empty ? make_float4(0.f, 0.f, 0.f, 0.f) : __ldcg(src + c * kTile + r0 + rr);
   }
 #pragma unroll
-  for (int u = 0; u < kPer; ++u) {
-    const int idx = threadIdx.x + u * 256;
+  for (int w = 0; w < kPer; ++w) {
+    const int idx = threadIdx.x + w * 256;
     const int c = idx / kRows, rr = idx % kRows;
-    *reinterpret_cast<float4 *>(tile + rr * kLD + 4 * c) = v[u];
+    *reinterpret_cast<float4 *>(tile + rr * kLD + 4 * c) = v[w];
   }
   __syncthreads();
   constexpr int kCPR = D / 8;  // 16-byte output pieces per row
   for (int idx = threadIdx.x; idx < kRows * kCPR; idx += 256) {
     const int rr = idx / kCPR, j = idx % kCPR;
     const int i = m * kTile + r0 + rr;
-    if (i >= Sq) continue;
+    if (i >= a.Sq) continue;
     const float *t = tile + rr * kLD + 8 * j;
     const int4 w = make_int4(pack_bf16x2(t[0], t[1]), pack_bf16x2(t[2], t[3]),
                              pack_bf16x2(t[4], t[5]), pack_bf16x2(t[6], t[7]));
-    *reinterpret_cast<int4 *>(dq + b * sb + static_cast<int64_t>(i) * ss + h * sh + 8 * j) = w;
+    *reinterpret_cast<int4 *>(a.dq + b * a.sb + static_cast<int64_t>(i) * a.ss + h * a.sh + 8 * j) = w;
   }
+  // the grid completes only after the backward main kernel
+  if (blockIdx.x == gridDim.x - 1 && threadIdx.x == 0) pdl_wait();
 }
 
 // dK = dV = 0, the whole gradient of a problem with keys but no query row:
@@ -1163,6 +1253,7 @@ cudaError_t launch_bwd_preprocess(const bsa_problem &p, const bsa_options &o, co
   da.n_sem = n_sem;
   da.q16 = reinterpret_cast<uint32_t *>(ws + L.q16);
   da.do16 = reinterpret_cast<uint32_t *>(ws + L.do16);
+  da.dq_mode = o.deterministic ? 1u : 2u;
   cudaError_t e = launch_pdl(kern, dim3(blocks), dim3(256), 0, s, da);
   if (e != cudaSuccess) return e;
   count_launch();
@@ -1223,14 +1314,23 @@ cudaError_t launch_bwd_main(const bsa_problem &p, const MaskParams &mp, const bs
 
 cudaError_t launch_bwd_convert(const bsa_problem &p, void *dq, const WsLayout &L, uint8_t *ws,
                                cudaStream_t s) {
-  const float *acc = reinterpret_cast<const float *>(ws + L.dq_accum);
+  ConvertArgs a{};
+  a.acc = reinterpret_cast<const float *>(ws + L.dq_accum);
+  a.sem = reinterpret_cast<const uint32_t *>(ws + L.sem);
+  a.hdr = reinterpret_cast<uint32_t *>(ws + L.status);
+  a.row_ptr = reinterpret_cast<const int32_t *>(ws + L.row_ptr);
+  a.dq = static_cast<__nv_bfloat16 *>(dq);
+  a.sb = p.q_stride[0];
+  a.ss = p.q_stride[1];
+  a.sh = p.q_stride[2];
+  a.B = p.B;
+  a.H = p.H;
+  a.Sq = p.Sq;
+  a.nM = L.nM;
   const unsigned blocks = static_cast<unsigned>(static_cast<int64_t>(p.B) * p.H * L.nM * (kTile / 32));
-  const int32_t *row_ptr = reinterpret_cast<const int32_t *>(ws + L.row_ptr);
-  __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(dq);
   // a programmatic dependent of the backward main kernel
   const cudaError_t e = launch_pdl(p.D == 64 ? k_dq_convert<64> : k_dq_convert<128>, dim3(blocks), dim3(256), 0,
-                                   s, acc, p.B, p.H, p.Sq, L.nM, row_ptr, out, p.q_stride[0], p.q_stride[1],
-                                   p.q_stride[2]);
+                                   s, a);
   if (e != cudaSuccess) return e;
   count_launch();
   return cudaGetLastError();

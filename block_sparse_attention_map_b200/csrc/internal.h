@@ -41,6 +41,7 @@ enum HeaderWord : int {
   kHdrFixedRows = 13,  // query rows the forwards since the plan build ran with a pinned reference
   kHdrFwdDone = 14,    // forward CTAs finished; the last one puts both forward words back to 0
   kHdrBwdDone = 15,    // the same for the backward's column ticket
+  kHdrDqMode = 16,     // the last Delta pass's dQ protocol: 1 semaphore-ordered, 2 atomic (0: none)
   kHdrPlanWords = 48,  // words [0, 48) are reset by every plan build
   // The fp16-Q record (kept across plan builds): the `q` pointer and strides
   // whose fp16 copy the last forward on this workspace wrote (pointer 0: none);

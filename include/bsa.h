@@ -367,7 +367,11 @@ BSA_API bsa_status bsa_bwd_main(const bsa_problem *prob, const bsa_mask_spec *ma
                                 const void *v, const void *dout, const float *lse, void *dk,
                                 void *dv, void *ws, size_t ws_bytes, bsa_stream_t stream);
 
-/* a7: dQ = bf16(dQ accumulator); zero rows for q-blocks no kv column reaches. */
+/* a7: dQ = bf16(dQ accumulator); zero rows for q-blocks no kv column reaches.
+ * After a semaphore-ordered bsa_bwd_main on the same stream, the blocks may
+ * start while that kernel's last columns still run: each converts its 32 rows
+ * once their dQ semaphore counts every contribution of the row list.  The
+ * call's work still completes only after bsa_bwd_main's. */
 BSA_API bsa_status bsa_bwd_convert(const bsa_problem *prob, const bsa_mask_spec *mask,
                                    void *dq, void *ws, size_t ws_bytes, bsa_stream_t stream);
 
