@@ -341,3 +341,37 @@ def test_stage_calls_equal_the_composite_calls(deterministic):
         assert torch.equal(st.dq, dq) and torch.equal(st.dk, dk) and torch.equal(st.dv, dv)
     else:
         _check_grads(st.dq, st.dk, st.dv, _oracle_grads(wl))
+
+
+def test_dq_convert_polls_then_falls_back_and_repeats_bitwise():
+    """After a semaphore-ordered Delta pass the dQ convert polls each quarter's
+    semaphore rather than waiting for the backward grid.  With no backward main
+    kernel in between the counts never complete: each poll gives up after its
+    bound, the call still finishes (no error is recorded: it falls back to the
+    grid wait), and a backward run afterwards gives the composite call's dQ.  A
+    second convert on complete semaphores gives the same dQ bit for bit."""
+    import time
+    wl = make_workload("window", device="cuda", small=True)
+    st = bsa.Stages(wl.q, wl.k, wl.v, wl.mask, softmax_mode="fixed_m", order="desc")
+    st.plan_and_bound()
+    st.forward()
+    st.preprocess(wl.dO)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    st.convert()
+    torch.cuda.synchronize()
+    assert time.perf_counter() - t0 < 5.0
+    assert st.ws.status() == 0
+    st.preprocess(wl.dO)
+    st.backward_main(wl.dO)
+    st.convert()
+    torch.cuda.synchronize()
+    first = st.dq.clone()
+    st.convert()
+    torch.cuda.synchronize()
+    assert st.ws.status() == 0
+    assert torch.equal(st.dq, first)
+    o, lse, wsf = bsa.attn_fwd(wl.q, wl.k, wl.v, wl.mask, softmax_mode="fixed_m", order="desc")
+    dq, _, _, ws = bsa.attn_bwd(wl.q, wl.k, wl.v, o, wl.dO, lse, wl.mask, order="desc", workspace=wsf)
+    torch.cuda.synchronize()
+    assert ws.status() == 0 and torch.equal(st.dq, dq)
