@@ -112,6 +112,10 @@ def test_semaphore_protocol_deadlock_free_and_ordered(order, workers):
     for (b, m), seq in acc.items():
         expect = [int(n) for n in pi if cls[b, m, n] != EMPTY]
         assert seq == expect
+        # the final count is the row's number of non-empty tiles: the dQ
+        # convert takes a q-block as complete exactly when its semaphore
+        # reaches the row list's length
+        assert len(seq) == int((cls[b, m] != EMPTY).sum())
 
 
 def test_unified_list_never_slower_than_partial_then_full():
