@@ -109,9 +109,14 @@ __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity) {
   }
 }
 
-// One work unit: a pair of q-blocks (A = 2g, B = 2g+1) of one (b, h).  The
-// pairs that would make a last, partly filled wave are split into two single
-// q-block units each (slot A only), so that wave takes about half as long.
+// One work unit: a pair of q-blocks (A = 2g, B = 2g+1) of one (b, h).  Units
+// are handed out with the pair index descending and every (b, h) of a pair
+// index in turn: under causal, prefix and document masks a q-block's row list
+// grows with m, so the longest units go first and the short ones fill the last
+// wave (the document forward measured 151 -> 118 us against (b, h)-major
+// ascending order, packed 120 -> 105 us, the window unchanged).  The pairs
+// that would make a last, partly filled wave are split into two single q-block
+// units each (slot A only), so that wave takes about half as long.
 struct FwdUnit {
   int b, h, bh, m[2], rs[2], re[2];
 };
@@ -125,8 +130,9 @@ __device__ __forceinline__ FwdUnit decode_unit(const FwdParams &p, int u) {
     pu = p.n_pairs + (s >> 1);
     only = s & 1;
   }
-  w.bh = pu / nP;
-  const int g = pu % nP;
+  const int BH = p.B * p.H;
+  w.bh = pu % BH;
+  const int g = nP - 1 - pu / BH;
   w.b = w.bh / p.H;
   w.h = w.bh % p.H;
 #pragma unroll
