@@ -46,17 +46,34 @@ __global__ void k_varlen_expand(const int32_t *__restrict__ cu, int n_seqs, int 
 // #alignment positions] over the in-range positions of the block.  With
 // neg_is_align (varlen) negative ids mark alignment positions; caller-supplied
 // segment ids may take any int32 value.
-__global__ void k_block_summary(const int32_t *__restrict__ seg, int S, int nblk, int B,
-                                int64_t bstride, int neg_is_align, int4 *__restrict__ out) {
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+// The planner's first launch with segment or varlen ids: the block summaries
+// of both id arrays (a warp per block, q blocks first), and the row and column
+// counts (and, unless hdr is null, the plan's header words) zeroed, in one
+// grid rather than two summary launches and three memsets.
+__global__ void k_plan_prep(const int32_t *__restrict__ seg_q, const int32_t *__restrict__ seg_kv,
+                            int Sq, int Skv, int nM, int nN, int B, int64_t bq, int64_t bk,
+                            int neg_is_align, int4 *__restrict__ qb, int4 *__restrict__ kb,
+                            uint32_t *__restrict__ hdr, int32_t *__restrict__ row_cnt,
+                            int32_t *__restrict__ col_cnt) {
+  const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t nthr = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  if (hdr != nullptr && tid < kHdrPlanWords) hdr[tid] = 0u;  // null: reset by the caller already
+  for (int64_t i = tid; i < static_cast<int64_t>(B) * nM; i += nthr) row_cnt[i] = 0;
+  for (int64_t i = tid; i < static_cast<int64_t>(B) * nN; i += nthr) col_cnt[i] = 0;
+  const int warp = static_cast<int>(tid >> 5);
   const int lane = threadIdx.x & 31;
-  if (warp >= B * nblk) return;
-  const int b = warp / nblk, blk = warp % nblk;
+  const int nq = B * nM;
+  if (warp >= nq + B * nN) return;
+  const bool is_q = warp < nq;
+  const int blk = is_q ? warp : warp - nq, nb = is_q ? nM : nN, S = is_q ? Sq : Skv;
+  const int b = blk / nb, j = blk % nb;
+  const int32_t *seg = is_q ? seg_q : seg_kv;
+  const int64_t bs = is_q ? bq : bk;
   int mn = 0x7fffffff, mx = -0x7fffffff - 1, nreal = 0, nbad = 0;
   for (int t = lane; t < kTile; t += 32) {
-    const int i = blk * kTile + t;
+    const int i = j * kTile + t;
     if (i >= S) break;
-    const int v = seg[b * bstride + i];
+    const int v = seg[b * bs + i];
     if (neg_is_align && v < 0) { ++nbad; continue; }
     mn = min(mn, v);
     mx = max(mx, v);
@@ -68,7 +85,7 @@ __global__ void k_block_summary(const int32_t *__restrict__ seg, int S, int nblk
     nreal += __shfl_xor_sync(0xffffffffu, nreal, o);
     nbad += __shfl_xor_sync(0xffffffffu, nbad, o);
   }
-  if (lane == 0) out[warp] = make_int4(mn, mx, nreal, nbad);
+  if (lane == 0) (is_q ? qb : kb)[blk] = make_int4(mn, mx, nreal, nbad);
 }
 
 struct ClassifyArgs {
@@ -778,17 +795,24 @@ cudaError_t launch_plan(const bsa_problem &p, const bsa_mask_spec &m, const bsa_
     count_launch();
     return cudaGetLastError();
   }
-  e = cudaMemsetAsync(hdr, 0, kHdrPlanWords * sizeof(uint32_t), s);
-  if (e != cudaSuccess) return e;
-
   const int4 *qblk = nullptr, *kblk = nullptr;
   const int32_t *seg_q_ids = nullptr, *seg_kv_ids = nullptr;
   int64_t seg_q_bs = 0, seg_kv_bs = 0;
   const bool varlen = m.flags & BSA_MASK_VARLEN;
+  int32_t *rank = reinterpret_cast<int32_t *>(ws + L.rank);
+  int32_t *row_cnt = reinterpret_cast<int32_t *>(ws + L.row_cnt);
+  int32_t *row_ptr = reinterpret_cast<int32_t *>(ws + L.row_ptr);
+  int32_t *col_cnt = reinterpret_cast<int32_t *>(ws + L.col_cnt);
+  int32_t *col_ptr = reinterpret_cast<int32_t *>(ws + L.col_ptr);
+  int32_t *perm = reinterpret_cast<int32_t *>(ws + L.perm);
   if (varlen || (m.flags & BSA_MASK_SEGMENT_IDS)) {
     const int32_t *sq = m.seg_q, *sk = m.seg_kv;
     int64_t bq = p.Sq, bk = p.Skv;
     if (varlen) {
+      // the expansion records bad cu_seqlens in the status word: the header
+      // is reset before it
+      e = cudaMemsetAsync(hdr, 0, kHdrPlanWords * sizeof(uint32_t), s);
+      if (e != cudaSuccess) return e;
       int32_t *dq = reinterpret_cast<int32_t *>(ws + L.seg_q);
       int32_t *dk = reinterpret_cast<int32_t *>(ws + L.seg_kv);
       k_varlen_expand<<<cdiv(p.Sq, 256), 256, 0, s>>>(m.cu_seqlens, m.n_seqs, m.n_align_tail,
@@ -800,29 +824,23 @@ cudaError_t launch_plan(const bsa_problem &p, const bsa_mask_spec &m, const bsa_
     }
     int4 *qb = reinterpret_cast<int4 *>(ws + L.qblk);
     int4 *kb = reinterpret_cast<int4 *>(ws + L.kblk);
-    k_block_summary<<<cdiv(static_cast<int64_t>(B) * nM * 32, 256), 256, 0, s>>>(sq, p.Sq, nM, B,
-                                                                                bq, varlen, qb);
-    k_block_summary<<<cdiv(static_cast<int64_t>(B) * nN * 32, 256), 256, 0, s>>>(sk, p.Skv, nN,
-                                                                                B, bk, varlen, kb);
-    count_launch(2);
+    k_plan_prep<<<cdiv(static_cast<int64_t>(B) * (nM + nN) * 32, 256), 256, 0, s>>>(
+        sq, sk, p.Sq, p.Skv, nM, nN, B, bq, bk, varlen, qb, kb, varlen ? nullptr : hdr, row_cnt, col_cnt);
+    count_launch();
     qblk = qb;
     kblk = kb;
     seg_q_ids = sq;
     seg_kv_ids = sk;
     seg_q_bs = bq;
     seg_kv_bs = bk;
+  } else {
+    e = cudaMemsetAsync(hdr, 0, kHdrPlanWords * sizeof(uint32_t), s);
+    if (e != cudaSuccess) return e;
+    e = cudaMemsetAsync(col_cnt, 0, sizeof(int32_t) * B * nN, s);
+    if (e != cudaSuccess) return e;
+    e = cudaMemsetAsync(row_cnt, 0, sizeof(int32_t) * B * nM, s);
+    if (e != cudaSuccess) return e;
   }
-
-  int32_t *rank = reinterpret_cast<int32_t *>(ws + L.rank);
-  int32_t *row_cnt = reinterpret_cast<int32_t *>(ws + L.row_cnt);
-  int32_t *row_ptr = reinterpret_cast<int32_t *>(ws + L.row_ptr);
-  int32_t *col_cnt = reinterpret_cast<int32_t *>(ws + L.col_cnt);
-  int32_t *col_ptr = reinterpret_cast<int32_t *>(ws + L.col_ptr);
-  int32_t *perm = reinterpret_cast<int32_t *>(ws + L.perm);
-  e = cudaMemsetAsync(col_cnt, 0, sizeof(int32_t) * B * nN, s);
-  if (e != cudaSuccess) return e;
-  e = cudaMemsetAsync(row_cnt, 0, sizeof(int32_t) * B * nM, s);
-  if (e != cudaSuccess) return e;
   if (o.bwd_order == BSA_ORDER_PERM) {
     e = cudaMemcpyAsync(perm, o.perm, sizeof(int32_t) * nN, cudaMemcpyHostToDevice, s);
     if (e != cudaSuccess) return e;
