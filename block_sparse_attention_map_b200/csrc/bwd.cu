@@ -1065,8 +1065,8 @@ __device__ int sem_poll(const uint32_t *sem, uint32_t target, uint64_t limit_ns,
 // q-blocks already complete while its last columns still run.  Blocks take
 // the q-blocks in the order they complete (the highest first under the
 // descending column order, else the lowest first), heads interleaved.  The
-// last block to finish waits for the backward grid, so that the convert's
-// completion still implies the backward's.
+// block with the last index waits for the backward grid, so that the
+// convert's completion still implies the backward's.
 template <int D>
 __global__ void __launch_bounds__(256) k_dq_convert(const ConvertArgs a) {
   constexpr int kC = D / 4, kRows = 32, kLD = D + 4;

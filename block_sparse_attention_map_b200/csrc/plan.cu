@@ -42,14 +42,14 @@ __global__ void k_varlen_expand(const int32_t *__restrict__ cu, int n_seqs, int 
   seg_kv[i] = align ? -2 : lo;
 }
 
-// Per-block summary of segment ids: [min, max, #positions with a real id,
-// #alignment positions] over the in-range positions of the block.  With
-// neg_is_align (varlen) negative ids mark alignment positions; caller-supplied
-// segment ids may take any int32 value.
-// The planner's first launch with segment or varlen ids: the block summaries
-// of both id arrays (a warp per block, q blocks first), and the row and column
-// counts (and, unless hdr is null, the plan's header words) zeroed, in one
-// grid rather than two summary launches and three memsets.
+// The planner's first launch with segment or varlen ids: the per-block
+// summaries of both id arrays (a warp per block, q blocks first), and the row
+// and column counts (and, unless hdr is null, the plan's header words) zeroed,
+// in one grid rather than two summary launches and three memsets.  A summary
+// is [min, max, #positions with a real id, #alignment positions] over the
+// in-range positions of the block; with neg_is_align (varlen) negative ids
+// mark alignment positions, while caller-supplied segment ids may take any
+// int32 value.
 __global__ void k_plan_prep(const int32_t *__restrict__ seg_q, const int32_t *__restrict__ seg_kv,
                             int Sq, int Skv, int nM, int nN, int B, int64_t bq, int64_t bk,
                             int neg_is_align, int4 *__restrict__ qb, int4 *__restrict__ kb,
