@@ -52,6 +52,7 @@ struct FwdParams {
   MaskParams mask;
   int B, H, Sq, Skv, nM, n_units;
   int n_pairs;   // units [0, n_pairs) are q-block pairs; the rest are single q-blocks
+  int head_group;  // (b, h) interleaved in groups of this many (a divisor of B * H)
   int kv_group;  // query heads per key/value head (grouped-query attention)
   float scale, scale_log2;
   const int32_t *row_ptr;
@@ -109,12 +110,16 @@ __device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity) {
   }
 }
 
-// One work unit: a pair of q-blocks (A = 2g, B = 2g+1) of one (b, h).  Units
-// are handed out with the pair index descending and every (b, h) of a pair
-// index in turn: under causal, prefix and document masks a q-block's row list
-// grows with m, so the longest units go first and the short ones fill the last
-// wave (the document forward measured 151 -> 118 us against (b, h)-major
-// ascending order, packed 120 -> 105 us, the window unchanged).  The pairs
+// One work unit: a pair of q-blocks (A = 2g, B = 2g+1) of one (b, h).  The
+// (b, h) are taken in groups of head_group; within a group the units go with
+// the pair index descending and every (b, h) of the group in turn.  Under
+// causal, prefix and document masks a q-block's row list grows with m, so the
+// long units go first and the short ones fill the last wave, and the group's
+// heads share the work of each pair index (document forward 151 -> 116 us,
+// prefix-LM 385 -> 310 us against (b, h)-major ascending order).  The group is
+// as large as keeps its heads' K and V within half the L2 (every head at the
+// window and document shapes; one at the video shape, whose heads' K and V
+// would otherwise stream through the L2 together: 113 -> 137 ms).  The pairs
 // that would make a last, partly filled wave are split into two single q-block
 // units each (slot A only), so that wave takes about half as long.
 struct FwdUnit {
@@ -130,9 +135,10 @@ __device__ __forceinline__ FwdUnit decode_unit(const FwdParams &p, int u) {
     pu = p.n_pairs + (s >> 1);
     only = s & 1;
   }
-  const int BH = p.B * p.H;
-  w.bh = pu % BH;
-  const int g = nP - 1 - pu / BH;
+  const int G = p.head_group, per_group = G * nP;
+  const int r = pu % per_group;
+  w.bh = (pu / per_group) * G + r % G;
+  const int g = nP - 1 - r / G;
   w.b = w.bh / p.H;
   w.h = w.bh % p.H;
 #pragma unroll
@@ -1199,6 +1205,14 @@ cudaError_t launch_fwd(const bsa_problem &p, const MaskParams &mp, const bsa_opt
     const int r = pairs % grid0;
     fp.n_pairs = (r != 0 && 2 * r <= grid0) ? pairs - r : pairs;
     fp.n_units = pairs + (pairs - fp.n_pairs);
+    // the largest divisor of B * H whose heads' K and V (4 D Skv bytes each)
+    // fit in 64 MB, half the L2
+    const int BH = p.B * p.H;
+    const int64_t per_head = 4ll * p.D * p.Skv;
+    const int64_t fit = std::max<int64_t>(1, (int64_t{64} << 20) / per_head);
+    fp.head_group = 1;
+    for (int d = 1; d <= BH; ++d)
+      if (BH % d == 0 && d <= fit) fp.head_group = d;
   }
   fp.scale = p.scale;
   fp.scale_log2 = p.scale * kLog2e;
