@@ -194,8 +194,8 @@ def test_bench_step_full_size_matches_oracle_and_repeats_bitwise():
     8192 x 8192, D=128): plan and bound in one call, fixed-m gated forward,
     Delta, the deterministic backward in the descending kv-column order and the
     dQ convert, through the per-stage C-ABI calls on one workspace.  O and LSE
-    of heads 0 and 15 on sampled rows and the gradients of head 0 against the
-    oracle; ten steps bit-identical."""
+    of heads 0 and 15 on sampled rows and the gradients of heads 0 and 15
+    against the oracle; ten steps bit-identical."""
     wl = make_workload("window", device="cuda")
     st = bsa.Stages(wl.q, wl.k, wl.v, wl.mask, softmax_mode="fixed_m", order="desc")
     outs = None
@@ -221,10 +221,13 @@ def test_bench_step_full_size_matches_oracle_and_repeats_bitwise():
     compare_out(o[:, :, heads], O_ref, rows)
     el, same = compare_lse(lse[:, heads], L_ref, rows)
     assert el <= LSE_TOL and same
-    gq, gk, gv = _oracle_grads(wl, heads=[0])
-    check("dQ", np64(dq[:, :, [0]]), gq)
-    check("dK", np64(dk[:, :, [0]]), gk)
-    check("dV", np64(dv[:, :, [0]]), gv)
+    # the first and the last head: the forward hands units out and the dQ
+    # convert takes q-blocks with the heads interleaved
+    for h in (0, wl.H - 1):
+        gq, gk, gv = _oracle_grads(wl, heads=[h])
+        check("dQ", np64(dq[:, :, [h]]), gq)
+        check("dK", np64(dk[:, :, [h]]), gk)
+        check("dV", np64(dv[:, :, [h]]), gv)
 
 
 def test_packed_full_size_forward_and_backward_per_batch():
