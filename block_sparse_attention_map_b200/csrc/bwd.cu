@@ -791,6 +791,9 @@ k_attn_bwd(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUten
         if (p.deterministic) {
           if (lane == 0) ok = sem_wait(sem, rank, p.sem_timeout_ns, p.hdr + kHdrStatus) ? 1 : 0;
           ok = __shfl_sync(0xffffffffu, ok, 0);
+          // the warp barrier orders every lane's adds below after lane 0's
+          // acquire (a shuffle alone carries no memory ordering)
+          __syncwarp();
         }
         if (ok) {
           float *base = p.dq_accum + (bh * p.nM + m) * (D / 4) * (kTile * 4);
